@@ -1,0 +1,326 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself.
+
+Every function of ``oracle.hstu_oracle`` is checked here by at least one of: hand-worked values
+(``tests/golden``), exact arithmetic, a scalar brute-force evaluator written independently,
+closed forms, invariants (causality, jagged independence), a library routine (torch's
+LayerNorm and dense ops for the page's dense formulation) and central finite differences.
+"""
+import decimal
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import hstu_oracle as O
+from oracle.bruteforce import layer_fwd_scalar
+from hstu_sequential_transduction_causal_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+THR = O.time_bucket_thresholds(128)
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        rows = [ln for ln in f if ln.strip() and not ln.startswith("#")]
+    return [float(v) for v in rows[0].split()]
+
+
+# ---------------------------------------------------------------------------------------------
+# time buckets and position indices
+# ---------------------------------------------------------------------------------------------
+
+def test_threshold_head_matches_hand_values():
+    assert list(THR[:12]) == [int(v) for v in _golden("time_bucket_thresholds_head.txt")]
+
+
+def test_bucket_matches_decimal_logarithm():
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([np.arange(-3, 5000), rng.integers(5000, 2 ** 62, 3000),
+                           (2 ** rng.uniform(0, 62, 3000)).astype(np.int64)])
+    got = O.time_bucket(vals, THR)
+    ctx = decimal.Context(prec=60)
+    for v, g in zip(vals[::7], got[::7]):
+        ln = ctx.ln(decimal.Decimal(max(int(v), 1)))
+        ref = int((ln / decimal.Decimal("0.301")).to_integral_value(decimal.ROUND_FLOOR))
+        assert g == min(127, ref), (v, g, ref)
+    # the bulk against float64 logs, where the float value is far from an integer
+    f = np.log(np.maximum(vals, 1).astype(np.float64)) / 0.301
+    safe = np.abs(f - np.round(f)) > 1e-9
+    assert np.array_equal(got[safe], np.minimum(127, np.floor(f[safe])).astype(np.int64))
+
+
+def test_bucket_threshold_edges():
+    for k in range(1, 128):
+        t = int(THR[k - 1])
+        assert O.time_bucket(t, THR) >= k
+        assert O.time_bucket(t - 1, THR) <= k - 1
+    assert O.time_bucket(-10 ** 12, THR) == 0
+    assert O.time_bucket(0, THR) == 0 and O.time_bucket(1, THR) == 0
+    assert O.time_bucket(2 ** 63 - 1, THR) == 127
+    # bucket 1 is empty: tau_1 == tau_2 == 2
+    assert O.time_bucket(2, THR) == 2
+
+
+def test_rel_pos_index():
+    L = 8
+    assert O.rel_pos_index(5, 5, L) == L - 1
+    assert O.rel_pos_index(7, 0, L) == 2 * L - 2
+    assert O.rel_pos_index(100, 0, L) == 2 * L - 2      # clamped
+    assert O.rel_pos_index(0, 3, L) == L - 1 - 3
+    assert O.rel_pos_index(0, 100, L) == 0
+
+
+# ---------------------------------------------------------------------------------------------
+# activation
+# ---------------------------------------------------------------------------------------------
+
+def test_silu_values_and_gradient():
+    assert O.silu(0.0) == 0.0
+    assert abs(O.silu(1.0) - 0.7310585786300049) < 1e-15          # sigma(1)
+    assert abs(O.silu(50.0) - 50.0) < 1e-12 and abs(O.silu(-50.0)) < 1e-18
+    z = np.linspace(-8, 8, 101)
+    h = 1e-6
+    fd = (O.silu(z + h) - O.silu(z - h)) / (2 * h)
+    assert np.allclose(O.silu_grad(z), fd, atol=1e-8)
+
+
+# ---------------------------------------------------------------------------------------------
+# layer forward: brute force, closed forms, invariants, page's dense formulation
+# ---------------------------------------------------------------------------------------------
+
+def _tiny(lengths, D=8, H=2, seed=3, L=16, spread=False):
+    rng = np.random.default_rng(seed)
+    wl = W.make_workload("c1", seed=seed, lengths=lengths, D=D, H=H, pos_max_len=L, N=L)
+    p = wl.layers[0]
+    # non-zero biases / affine so that every term is exercised
+    p.b1 = rng.standard_normal(4 * D).astype(np.float32) * 0.3
+    p.b2 = rng.standard_normal(D).astype(np.float32) * 0.3
+    p.gamma = (1 + 0.3 * rng.standard_normal(D)).astype(np.float32)
+    p.beta = (0.3 * rng.standard_normal(D)).astype(np.float32)
+    p.rab_pos = rng.standard_normal(2 * L - 1).astype(np.float32)
+    p.rab_time = rng.standard_normal(128).astype(np.float32)
+    if spread:   # time gaps spanning many buckets, some equal and some out of order
+        wl.timestamps = (wl.timestamps + rng.integers(-5, 10 ** 9, wl.T)).astype(np.int64)
+    return wl, p
+
+
+@pytest.mark.parametrize("spread", [False, True])
+def test_layer_matches_scalar_bruteforce(spread):
+    wl, p = _tiny([1, 3, 0, 5, 2], spread=spread)
+    inv_N = 1.0 / 7.0
+    y, _ = O.layer_fwd(wl.x, p, wl.offsets, wl.timestamps, wl.H, inv_N, wl.pos_max_len, THR)
+    yb = layer_fwd_scalar(wl.x.astype(float).tolist(), p.W1.astype(float).tolist(),
+                          p.b1.tolist(), p.W2.astype(float).tolist(), p.b2.tolist(),
+                          p.gamma.tolist(), p.beta.tolist(), p.rab_pos.tolist(),
+                          p.rab_time.tolist(), wl.offsets.tolist(), wl.timestamps.tolist(),
+                          wl.H, inv_N, wl.pos_max_len)
+    assert np.allclose(y, np.array(yb), rtol=1e-10, atol=1e-10)
+
+
+def test_causality_later_tokens_do_not_leak():
+    wl, p = _tiny([9, 6])
+    y0, _ = O.layer_fwd(wl.x, p, wl.offsets, wl.timestamps, wl.H, 0.1, wl.pos_max_len, THR)
+    x2 = wl.x.copy()
+    ts2 = wl.timestamps.copy()
+    i = 4                                         # perturb tokens 5..8 of sequence 0
+    x2[i + 1:9] += 3.0
+    ts2[i + 1:9] += 123456
+    y1, _ = O.layer_fwd(x2, p, wl.offsets, ts2, wl.H, 0.1, wl.pos_max_len, THR)
+    assert np.array_equal(y0[:i + 1], y1[:i + 1])
+    assert np.array_equal(y0[9:], y1[9:])
+    assert not np.allclose(y0[i + 1:9], y1[i + 1:9])
+
+
+def test_jagged_independence():
+    wl, p = _tiny([5, 0, 7, 3])
+    y, _ = O.layer_fwd(wl.x, p, wl.offsets, wl.timestamps, wl.H, 0.2, wl.pos_max_len, THR)
+    for b in range(wl.B):
+        s, e = wl.offsets[b], wl.offsets[b + 1]
+        if e == s:
+            continue
+        yb, _ = O.layer_fwd(wl.x[s:e], p, np.array([0, e - s]), wl.timestamps[s:e], wl.H, 0.2,
+                            wl.pos_max_len, THR)
+        # identical up to the BLAS's rounding order of the row-block GEMMs
+        assert np.allclose(y[s:e], yb, rtol=1e-13, atol=1e-13)
+
+
+def test_closed_form_zero_query_key():
+    """Q = K = 0 and zero tables: A = SiLU(0)/N = 0, O = 0, LN(O) = beta, so
+    Y = (beta (.) U) W2^T + b2 + X; with beta = b2 = 0 it is X exactly."""
+    wl, p = _tiny([4, 6])
+    D = wl.D
+    p.W1 = p.W1.copy()
+    p.W1[2 * D:] = 0
+    p.b1 = p.b1.copy()
+    p.b1[2 * D:] = 0
+    p.rab_pos = np.zeros_like(p.rab_pos)
+    p.rab_time = np.zeros_like(p.rab_time)
+    y, sv = O.layer_fwd(wl.x, p, wl.offsets, wl.timestamps, wl.H, 0.3, wl.pos_max_len, THR)
+    u = sv["s"][:, :D]
+    assert np.array_equal(sv["o"], np.zeros_like(sv["o"]))
+    ref = (p.beta.astype(float) * u) @ p.W2.astype(float).T + p.b2 + wl.x
+    assert np.allclose(y, ref, rtol=1e-14, atol=1e-14)
+    p.beta = np.zeros_like(p.beta)
+    p.b2 = np.zeros_like(p.b2)
+    y, _ = O.layer_fwd(wl.x, p, wl.offsets, wl.timestamps, wl.H, 0.3, wl.pos_max_len, THR)
+    assert np.array_equal(y, wl.x.astype(np.float64))
+
+
+def test_closed_form_single_token():
+    rng = np.random.default_rng(5)
+    H, d, L = 2, 4, 8
+    q, k, v = (rng.standard_normal((1, H, d)) for _ in range(3))
+    rp = rng.standard_normal(2 * L - 1)
+    rt = rng.standard_normal(128)
+    o = O.pointwise_attention_fwd(q, k, v, [0, 1], np.array([77]), rp, rt, 0.25, L, THR)
+    for h in range(H):
+        p_ = float(q[0, h] @ k[0, h]) + rp[L - 1] + rt[0]
+        assert np.allclose(o[0, h], p_ / (1 + math.exp(-p_)) * 0.25 * v[0, h], rtol=1e-14)
+
+
+def test_constant_v_hand_values():
+    L = 4
+    rp = np.zeros(2 * L - 1)
+    rp[L - 1 + 0], rp[L - 1 + 1], rp[L - 1 + 2] = 0.5, 1.0, -1.0
+    q = np.zeros((3, 1, 2))
+    v = np.ones((3, 1, 2))
+    o = O.pointwise_attention_fwd(q, q, v, [0, 3], np.array([0, 0, 0]), rp, np.zeros(128), 1.0,
+                                  L, THR)
+    exp = _golden("constant_v_n3.txt")
+    for i in range(3):
+        assert np.allclose(o[i, 0], exp[i], rtol=0, atol=1e-15)
+
+
+def test_dense_formulation_of_the_first_page():
+    """The first page's sketch formulates one padded sequence densely: a per-head [n, n]
+    position bias, causal lower triangle, division by n, LayerNorm over d_model, gate with U,
+    f2 and the residual (its extra input LayerNorm left out, reading R1; no time bias).
+    Restated here with torch CPU ops and torch's LayerNorm; the oracle must agree."""
+    n, D, H, L = 12, 16, 2, 16
+    rng = np.random.default_rng(11)
+    wl = W.make_workload("c1", seed=2, lengths=[n], D=D, H=H, pos_max_len=L, N=n)
+    p = wl.layers[0]
+    p.rab_time = np.zeros(128, np.float32)
+    p.rab_pos = rng.standard_normal(2 * L - 1).astype(np.float32)
+    y, _ = O.layer_fwd(wl.x, p, wl.offsets, wl.timestamps, H, 1.0 / n, L, THR)
+
+    x = torch.tensor(wl.x, dtype=torch.float64)[None]              # [1, n, D]
+    f1 = torch.nn.Linear(D, 4 * D).double()
+    f2 = torch.nn.Linear(D, D).double()
+    with torch.no_grad():
+        f1.weight.copy_(torch.tensor(p.W1))
+        f1.bias.copy_(torch.tensor(p.b1))
+        f2.weight.copy_(torch.tensor(p.W2))
+        f2.bias.copy_(torch.tensor(p.b2))
+    ii = torch.arange(n)[:, None]
+    jj = torch.arange(n)[None, :]
+    dense = torch.tensor(p.rab_pos, dtype=torch.float64)[(ii - jj).clamp(-(L - 1), L - 1) + L - 1]
+    dense = dense[None].expand(H, n, n)                             # same bias for every head
+    u, v, q, k = torch.nn.functional.silu(f1(x)).chunk(4, dim=-1)
+    heads = lambda t: t.view(1, n, H, D // H).transpose(1, 2)
+    sc = heads(q) @ heads(k).transpose(-1, -2) + dense
+    a = torch.nn.functional.silu(sc).masked_fill(~torch.ones(n, n, dtype=torch.bool).tril(), 0) / n
+    av = (a @ heads(v)).transpose(1, 2).reshape(1, n, D)
+    ln = torch.nn.functional.layer_norm(av, (D,), torch.tensor(p.gamma, dtype=torch.float64),
+                                        torch.tensor(p.beta, dtype=torch.float64), eps=1e-5)
+    yt = (x + f2(ln * u))[0].detach().numpy()
+    assert np.allclose(y, yt, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# backward: central finite differences of the oracle's own forward
+# ---------------------------------------------------------------------------------------------
+
+def test_backward_matches_finite_differences():
+    wl, p = _tiny([3, 5, 1], D=8, H=2, seed=7, L=8, spread=True)
+    inv_N = 0.5
+    rng = np.random.default_rng(8)
+    dy = rng.standard_normal((wl.T, wl.D))
+    for name in ("W1", "b1", "W2", "b2", "gamma", "beta", "rab_pos", "rab_time"):
+        setattr(p, name, getattr(p, name).astype(np.float64))
+    x = wl.x.astype(np.float64)
+
+    def loss(xx, pp):
+        yy, _ = O.layer_fwd(xx, pp, wl.offsets, wl.timestamps, wl.H, inv_N, wl.pos_max_len, THR)
+        return float((yy * dy).sum())
+
+    y, sv = O.layer_fwd(x, p, wl.offsets, wl.timestamps, wl.H, inv_N, wl.pos_max_len, THR)
+    g = O.layer_bwd(dy, p, sv, wl.offsets, wl.timestamps, wl.H, inv_N, wl.pos_max_len, THR)
+    h = 1e-6
+    checks = [("dx", None, x)] + [("d" + n, n, getattr(p, n)) for n in
+                                  ("W1", "b1", "W2", "b2", "gamma", "beta", "rab_pos",
+                                   "rab_time")]
+    for gname, pname, arr in checks:
+        flat = arr.reshape(-1)
+        idx = rng.choice(flat.size, size=min(flat.size, 25), replace=False)
+        if pname == "rab_time":
+            used = np.unique(O.time_bucket(
+                wl.timestamps[:, None] - wl.timestamps[None, :], THR))
+            idx = np.union1d(idx[:5], used)
+        for t in idx:
+            old = flat[t]
+            flat[t] = old + h
+            lp = loss(x, p)
+            flat[t] = old - h
+            lm = loss(x, p)
+            flat[t] = old
+            fd = (lp - lm) / (2 * h)
+            an = g[gname].reshape(-1)[t]
+            assert abs(fd - an) <= 1e-6 + 1e-5 * abs(fd), (gname, t, fd, an)
+
+
+# ---------------------------------------------------------------------------------------------
+# M-FALCON, Stochastic Length, work list
+# ---------------------------------------------------------------------------------------------
+
+def test_falcon_equals_naive_last_row():
+    fw = W.make_falcon_workload(seed=4, users=2, prefix=6, m=3, b_m=2, D=8, H=2, layers=2,
+                                N=7, pos_max_len=8)
+    yc, yp = O.falcon_fwd(fw.layers, fw.prefix_offsets, fw.prefix_ts, fw.prefix_x, fw.cand_x,
+                          fw.request_ts, fw.m, fw.H, 1 / fw.N, fw.pos_max_len, THR)
+    for u in range(fw.users):
+        s, e = fw.prefix_offsets[u], fw.prefix_offsets[u + 1]
+        for c in range(fw.m):
+            xs = np.concatenate([fw.prefix_x[s:e], fw.cand_x[u * fw.m + c][None]])
+            ts = np.concatenate([fw.prefix_ts[s:e], [fw.request_ts[u]]])
+            off = np.array([0, xs.shape[0]])
+            for p in fw.layers:
+                xs, _ = O.layer_fwd(xs, p, off, ts, fw.H, 1 / fw.N, fw.pos_max_len, THR)
+            assert np.allclose(yc[u * fw.m + c], xs[-1], rtol=1e-12, atol=1e-12)
+            assert np.allclose(yp[s:e], xs[:-1], rtol=1e-12, atol=1e-12)
+
+
+def test_stochastic_length_counts_and_selection():
+    assert O.stochastic_length_keep(512, 1.6) == 147       # 512**0.8 = 146.9
+    assert O.stochastic_length_keep(4096, 1.6) == 776      # 2**9.6 = 776.05
+    assert O.stochastic_length_keep(3, 1.6) == 2           # 3**0.8 = 2.41
+    assert O.stochastic_length_keep(1, 1.6) == 1 and O.stochastic_length_keep(0, 1.6) == 0
+    # n**0.8 is never within 1e-9 of a rounding boundary for the lengths the workloads draw
+    n = np.arange(1, 10001, dtype=np.float64)
+    f = n ** 0.8
+    assert np.all(np.abs(f - np.floor(f) - 0.5) > 1e-9)
+    rng = np.random.default_rng(0)
+    lens = [0, 1, 5, 40, 17]
+    off = W.offsets_from_lengths(lens)
+    keys = rng.integers(0, 50, off[-1])                  # many ties on purpose
+    new_off, kept = O.stochastic_length(off, keys, 1.6)
+    for b, n_ in enumerate(lens):
+        L = O.stochastic_length_keep(n_, 1.6)
+        assert new_off[b + 1] - new_off[b] == L
+        sel = kept[new_off[b]:new_off[b + 1]] - off[b]
+        assert np.all(np.diff(sel) > 0)
+        # brute force: a token is kept iff fewer than L tokens precede it in (key, position)
+        for j in range(n_):
+            rank = sum(1 for i in range(n_) if (keys[off[b] + i], i) < (keys[off[b] + j], j))
+            assert (j in sel) == (rank < L)
+
+
+def test_work_list_invariants():
+    off = W.offsets_from_lengths([0, 1, 128, 129, 700, 256])
+    wlst = O.tile_work_list(off, 128)
+    expect = {(b, t) for b, n in enumerate(np.diff(off)) for t in range(-(-int(n) // 128))}
+    assert {tuple(r) for r in wlst} == expect and len(wlst) == len(expect)
+    for a, b in zip(wlst[:-1], wlst[1:]):
+        assert a[1] > b[1] or (a[1] == b[1] and a[0] < b[0])
