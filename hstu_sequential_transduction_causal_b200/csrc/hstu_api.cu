@@ -1,0 +1,343 @@
+// hstu_api.cu - the extern "C" entry points of libhstu.so: argument validation, workspace
+// layout, tensor-map encoding and kernel dispatch on the caller's stream. No allocation, no
+// synchronisation (except hstu_sync_status, whose job it is).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/hstu.h"
+#include "hstu_internal.h"
+
+namespace hstu {
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+unsigned long long g_wait_limit = 1ull << 31;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hstu_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return HSTU_OK;
+  g_last_cuda_error = static_cast<int32_t>(e);
+  return e == cudaErrorInvalidValue ? HSTU_ERR_UNSUPPORTED : HSTU_ERR_CUDA;
+}
+
+int* ws_status(void* ws) { return static_cast<int*>(ws); }
+
+// attention workspace: [0,256) status | [256,512) count | [512, ...) items (int32 x 2 x capacity)
+size_t attn_ws_bytes(int64_t capacity) { return kWsHeader + 256 + align_up(static_cast<size_t>(capacity) * 8, 256); }
+
+int64_t capacity_of(const hstu_jagged_t* j) { return static_cast<int64_t>(j->B) + (j->T + kQTile - 1) / kQTile; }
+
+hstu_status_t check_jagged(const hstu_jagged_t* j) {
+  if (!j || j->B < 0 || j->T < 0 || j->max_len < 0) return HSTU_ERR_INVALID_ARG;
+  if (!j->offsets) return HSTU_ERR_INVALID_ARG;
+  if (j->T > 0 && !j->timestamps) return HSTU_ERR_INVALID_ARG;
+  if (j->T >= (1ll << 31)) return HSTU_ERR_UNSUPPORTED;   // row coordinates of the tensor maps are int32
+  return HSTU_OK;
+}
+
+hstu_status_t check_attn(const hstu_attn_desc_t* d, const hstu_jagged_t* j) {
+  hstu_status_t s = check_jagged(j);
+  if (s != HSTU_OK) return s;
+  if (!d || d->H <= 0 || d->d_qk <= 0 || d->d_v <= 0 || d->pos_max_len <= 0) return HSTU_ERR_INVALID_ARG;
+  if (d->n_time_buckets < 1 || d->n_time_buckets > 128) return HSTU_ERR_UNSUPPORTED;
+  if (!isfinite(d->inv_N)) return HSTU_ERR_INVALID_ARG;
+  if (d->dtype == HSTU_BF16) {
+    if (d->d_qk != 64 || d->d_v != 64) return HSTU_ERR_UNSUPPORTED;
+    if (d->ld_q % 8 || d->ld_k % 8 || d->ld_v % 8 || d->ld_o % 8) return HSTU_ERR_UNSUPPORTED;
+  } else if (d->dtype == HSTU_F32) {
+    if (d->d_qk > 64 || d->d_v > 64) return HSTU_ERR_UNSUPPORTED;
+  } else {
+    return HSTU_ERR_UNSUPPORTED;
+  }
+  if (d->ld_q < static_cast<int64_t>(d->H) * d->d_qk || d->ld_k < static_cast<int64_t>(d->H) * d->d_qk ||
+      d->ld_v < static_cast<int64_t>(d->H) * d->d_v || d->ld_o < static_cast<int64_t>(d->H) * d->d_v)
+    return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, const void* q, const void* k,
+                           const void* v, const float* rab_pos, const float* rab_time, void* out, void* ws,
+                           cudaStream_t st) {
+  const int64_t cap = capacity_of(j);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int32_t* count = reinterpret_cast<int32_t*>(w + kWsHeader);
+  int32_t* items = reinterpret_cast<int32_t*>(w + kWsHeader + 256);
+  AttnArgs a{};
+  a.B = j->B; a.T = j->T; a.max_len = j->max_len; a.offsets = j->offsets; a.ts = j->timestamps;
+  a.H = d->H; a.dqk = d->d_qk; a.dv = d->d_v; a.inv_N = d->inv_N; a.pos_max_len = d->pos_max_len;
+  a.n_buckets = d->n_time_buckets;
+  a.q = q; a.ld_q = d->ld_q; a.k = k; a.ld_k = d->ld_k; a.v = v; a.ld_v = d->ld_v; a.o = out; a.ld_o = d->ld_o;
+  a.rab_pos = rab_pos; a.rab_time = rab_time; a.items = items; a.count = count; a.capacity = cap;
+  a.status = ws_status(ws);
+  cudaError_t e = launch_worklist(j->offsets, j->B, j->T, j->max_len, items, count, a.status, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (j->T == 0) return HSTU_OK;
+  e = d->dtype == HSTU_BF16 ? attn_fwd_bf16_tc(a, st) : attn_fwd_f32_simt(a, st);
+  return cuda_status(e);
+}
+
+hstu_status_t run_uvqk(int64_t T, int32_t D, hstu_dtype_t dtype, const void* x, int64_t ld_x, const void* W1,
+                       const float* b1, void* uvqk, void* z, int* status, cudaStream_t st) {
+  GemmArgs g{};
+  g.A = x; g.lda = ld_x; g.a_mn = false;
+  g.B = W1; g.ldb = D; g.b_mn = false;
+  g.M = T; g.N = 4ll * D; g.K = D; g.splits = 1;
+  g.epi.kind = kEpiSilu; g.epi.bias = b1;
+  g.epi.out0 = uvqk; g.epi.out0_f32 = dtype == HSTU_F32; g.epi.ld_out0 = 4ll * D;
+  g.epi.out1 = z; g.epi.out1_f32 = dtype == HSTU_F32; g.epi.ld_out1 = 4ll * D;
+  g.status = status;
+  return cuda_status(dtype == HSTU_BF16 ? gemm_bf16(g, st) : gemm_f32(g, st));
+}
+
+hstu_status_t run_out_proj(int64_t T, int32_t D, hstu_dtype_t dtype, const void* g_in, const void* W2,
+                           const float* b2, const void* x, hstu_dtype_t x_dtype, void* y, hstu_dtype_t y_dtype,
+                           void* y_bf16, int* status, cudaStream_t st) {
+  GemmArgs g{};
+  g.A = g_in; g.lda = D; g.a_mn = false;
+  g.B = W2; g.ldb = D; g.b_mn = false;
+  g.M = T; g.N = D; g.K = D; g.splits = 1;
+  g.epi.kind = kEpiLinear; g.epi.bias = b2;
+  g.epi.resid = x; g.epi.resid_f32 = x_dtype == HSTU_F32; g.epi.ld_resid = D;
+  g.epi.out0 = y; g.epi.out0_f32 = y_dtype == HSTU_F32; g.epi.ld_out0 = D;
+  g.epi.out1 = y_bf16; g.epi.out1_f32 = 0; g.epi.ld_out1 = D;
+  g.status = status;
+  return cuda_status(dtype == HSTU_BF16 ? gemm_bf16(g, st) : gemm_f32(g, st));
+}
+
+hstu_status_t check_dense(int64_t T, int32_t D, hstu_dtype_t dtype) {
+  if (T < 0 || D <= 0) return HSTU_ERR_INVALID_ARG;
+  if (dtype != HSTU_BF16 && dtype != HSTU_F32) return HSTU_ERR_UNSUPPORTED;
+  if (dtype == HSTU_BF16 && D % 64) return HSTU_ERR_UNSUPPORTED;
+  if (T >= (1ll << 31)) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+}  // namespace
+
+WaitCtl wait_ctl(int* status) { return WaitCtl{status, g_wait_limit}; }
+
+bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld_elems,
+                         int box_inner, int box_outer) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn || !aligned16(base) || inner <= 0 || outer <= 0 || (ld_elems * 2) % 16) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_elems) * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace hstu
+
+using namespace hstu;
+
+extern "C" {
+
+int32_t hstu_abi_version(void) { return HSTU_ABI_VERSION; }
+
+const char* hstu_status_string(hstu_status_t s) {
+  switch (s) {
+    case HSTU_OK: return "HSTU_OK";
+    case HSTU_ERR_INVALID_ARG: return "HSTU_ERR_INVALID_ARG";
+    case HSTU_ERR_UNSUPPORTED: return "HSTU_ERR_UNSUPPORTED";
+    case HSTU_ERR_WORKSPACE: return "HSTU_ERR_WORKSPACE";
+    case HSTU_ERR_CUDA: return "HSTU_ERR_CUDA";
+    case HSTU_ERR_TIMEOUT: return "HSTU_ERR_TIMEOUT";
+    case HSTU_ERR_DEVICE: return "HSTU_ERR_DEVICE";
+  }
+  return "HSTU_ERR_UNKNOWN";
+}
+
+int32_t hstu_last_cuda_error(void) { return g_last_cuda_error; }
+
+void hstu_set_wait_limit(uint64_t cycles) { g_wait_limit = cycles ? cycles : (1ull << 31); }
+
+hstu_status_t hstu_sync_status(void* ws, hstu_stream_t stream, int32_t* device_status) {
+  if (!ws || !device_status) return HSTU_ERR_INVALID_ARG;
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(int32_t), stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  *device_status = v;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_debug_timeout_probe(void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  if (!ws) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < kWsHeader) return HSTU_ERR_WORKSPACE;
+  return cuda_status(launch_timeout_probe(ws_status(ws), stream));
+}
+
+int64_t hstu_worklist_capacity(const hstu_jagged_t* jag) {
+  if (check_jagged(jag) != HSTU_OK) return -1;
+  return capacity_of(jag);
+}
+
+hstu_status_t hstu_jagged_worklist(const hstu_jagged_t* jag, int32_t* items, int32_t* count, hstu_stream_t stream) {
+  hstu_status_t s = check_jagged(jag);
+  if (s != HSTU_OK) return s;
+  if (!items || !count) return HSTU_ERR_INVALID_ARG;
+  return cuda_status(launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, nullptr, stream));
+}
+
+hstu_status_t hstu_time_buckets(const hstu_jagged_t* jag, int32_t n_buckets, const int64_t* sq_offsets, uint8_t* out,
+                                hstu_stream_t stream) {
+  hstu_status_t s = check_jagged(jag);
+  if (s != HSTU_OK) return s;
+  if (n_buckets < 1 || n_buckets > 128) return HSTU_ERR_UNSUPPORTED;
+  if (jag->T > 0 && (!sq_offsets || !out)) return HSTU_ERR_INVALID_ARG;
+  return cuda_status(launch_time_buckets(jag->offsets, jag->timestamps, jag->B, jag->T, n_buckets, sq_offsets, out,
+                                         stream));
+}
+
+hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* x, int64_t ld_x, const void* W1,
+                            const float* b1, void* uvqk, void* z, void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  hstu_status_t s = check_dense(T, D, dtype);
+  if (s != HSTU_OK) return s;
+  if (!ws) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < kWsHeader) return HSTU_ERR_WORKSPACE;
+  if (T == 0) return HSTU_OK;
+  if (!x || !W1 || !uvqk || ld_x < D) return HSTU_ERR_INVALID_ARG;
+  if (dtype == HSTU_BF16 && (ld_x % 8 || !aligned16(x) || !aligned16(W1) || !aligned16(uvqk) || (z && !aligned16(z))))
+    return HSTU_ERR_UNSUPPORTED;
+  return run_uvqk(T, D, dtype, x, ld_x, W1, b1, uvqk, z, ws_status(ws), stream);
+}
+
+size_t hstu_attn_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag) {
+  (void)desc;
+  if (check_jagged(jag) != HSTU_OK) return 0;
+  return attn_ws_bytes(capacity_of(jag));
+}
+
+hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const void* q, const void* k,
+                            const void* v, const float* rab_pos, const float* rab_time, void* out, void* ws,
+                            size_t ws_bytes, hstu_stream_t stream) {
+  hstu_status_t s = check_attn(desc, jag);
+  if (s != HSTU_OK) return s;
+  if (!ws) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < attn_ws_bytes(capacity_of(jag))) return HSTU_ERR_WORKSPACE;
+  if (jag->T > 0 && (!q || !k || !v || !rab_pos || !rab_time || !out)) return HSTU_ERR_INVALID_ARG;
+  if (desc->dtype == HSTU_BF16 && jag->T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)))
+    return HSTU_ERR_UNSUPPORTED;
+  return run_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, ws, stream);
+}
+
+hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* o, int64_t ld_o, const void* u,
+                                 int64_t ld_u, const float* gamma, const float* beta, float eps, void* g, float* mu,
+                                 float* rstd, hstu_stream_t stream) {
+  if (T < 0) return HSTU_ERR_INVALID_ARG;
+  if (dtype != HSTU_BF16 && dtype != HSTU_F32) return HSTU_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128 && D != 256 && D != 512 && D != 1024) return HSTU_ERR_UNSUPPORTED;
+  if (T == 0) return HSTU_OK;
+  if (!o || !u || !gamma || !beta || !g || ld_o < D || ld_u < D) return HSTU_ERR_INVALID_ARG;
+  const int vec = dtype == HSTU_BF16 ? 8 : 4;
+  if (!aligned16(o) || !aligned16(u) || !aligned16(g) || !aligned16(gamma) || !aligned16(beta) || ld_o % vec ||
+      ld_u % vec)
+    return HSTU_ERR_UNSUPPORTED;
+  return cuda_status(norm_gate_fwd(T, D, dtype == HSTU_BF16, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, stream));
+}
+
+hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* g, const void* W2,
+                                const float* b2, const void* x, hstu_dtype_t x_dtype, void* y, hstu_dtype_t y_dtype,
+                                void* y_bf16, void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  hstu_status_t s = check_dense(T, D, dtype);
+  if (s != HSTU_OK) return s;
+  if (!ws) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < kWsHeader) return HSTU_ERR_WORKSPACE;
+  if ((x_dtype != HSTU_F32 && x_dtype != HSTU_BF16) || (y_dtype != HSTU_F32 && y_dtype != HSTU_BF16))
+    return HSTU_ERR_UNSUPPORTED;
+  if (dtype == HSTU_F32 && (x_dtype != HSTU_F32 || y_dtype != HSTU_F32 || y_bf16)) return HSTU_ERR_UNSUPPORTED;
+  if (T == 0) return HSTU_OK;
+  if (!g || !W2 || !x || !y) return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(g) || !aligned16(W2) || !aligned16(x) || !aligned16(y) || (y_bf16 && !aligned16(y_bf16)))
+    return HSTU_ERR_UNSUPPORTED;
+  return run_out_proj(T, D, dtype, g, W2, b2, x, x_dtype, y, y_dtype, y_bf16, ws_status(ws), stream);
+}
+
+size_t hstu_layer_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag) {
+  if (!desc || check_jagged(jag) != HSTU_OK) return 0;
+  size_t bytes = attn_ws_bytes(capacity_of(jag));
+  if (desc->dtype == HSTU_BF16 && desc->x_dtype == HSTU_F32)
+    bytes += align_up(static_cast<size_t>(jag->T) * desc->D * 2, 256);
+  return bytes;
+}
+
+hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag, const hstu_layer_weights_t* w,
+                             const void* x, const void* x_bf16, void* y, void* y_bf16, const hstu_layer_saved_t* saved,
+                             void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  if (!desc || !w || !saved) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t s = check_jagged(jag);
+  if (s != HSTU_OK) return s;
+  const int32_t D = desc->D, H = desc->H;
+  if (H <= 0 || D <= 0 || D % H) return HSTU_ERR_INVALID_ARG;
+  s = check_dense(jag->T, D, desc->dtype);
+  if (s != HSTU_OK) return s;
+  hstu_attn_desc_t ad{};
+  ad.H = H; ad.d_qk = D / H; ad.d_v = D / H; ad.inv_N = desc->inv_N; ad.pos_max_len = desc->pos_max_len;
+  ad.n_time_buckets = desc->n_time_buckets; ad.dtype = desc->dtype;
+  ad.ld_q = ad.ld_k = ad.ld_v = 4ll * D; ad.ld_o = D;
+  s = check_attn(&ad, jag);
+  if (s != HSTU_OK) return s;
+  if (desc->dtype == HSTU_F32 && (desc->x_dtype != HSTU_F32 || desc->y_dtype != HSTU_F32 || y_bf16))
+    return HSTU_ERR_UNSUPPORTED;
+  if (!ws) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < hstu_layer_workspace_size(desc, jag)) return HSTU_ERR_WORKSPACE;
+  const int64_t T = jag->T;
+  if (T == 0) return HSTU_OK;
+  if (!x || !y || !w->W1 || !w->b1 || !w->W2 || !w->b2 || !w->gamma || !w->beta || !w->rab_pos || !w->rab_time ||
+      !saved->uvqk || !saved->o || !saved->g || !saved->mu || !saved->rstd)
+    return HSTU_ERR_INVALID_ARG;
+  cudaStream_t st = stream;
+  int* status = ws_status(ws);
+  const void* x_op = x;
+  if (desc->dtype == HSTU_BF16 && desc->x_dtype == HSTU_F32) {
+    if (x_bf16) {
+      x_op = x_bf16;
+    } else {
+      void* conv = static_cast<uint8_t*>(ws) + attn_ws_bytes(capacity_of(jag));
+      cudaError_t e = convert_f32_to_bf16(static_cast<const float*>(x), conv, T * D, st);
+      if (e != cudaSuccess) return cuda_status(e);
+      x_op = conv;
+    }
+  }
+  s = run_uvqk(T, D, desc->dtype, x_op, D, w->W1, w->b1, saved->uvqk, saved->z, status, st);
+  if (s != HSTU_OK) return s;
+  const size_t es = desc->dtype == HSTU_BF16 ? 2 : 4;
+  const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
+  s = run_attn_fwd(&ad, jag, uvqk + 2 * D * es, uvqk + 3 * D * es, uvqk + 1 * D * es, w->rab_pos, w->rab_time,
+                   saved->o, ws, st);
+  if (s != HSTU_OK) return s;
+  cudaError_t e = norm_gate_fwd(T, D, desc->dtype == HSTU_BF16, saved->o, D, uvqk, 4ll * D, w->gamma, w->beta,
+                                desc->ln_eps, saved->g, saved->mu, saved->rstd, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  return run_out_proj(T, D, desc->dtype, saved->g, w->W2, w->b2, x, desc->x_dtype, y, desc->y_dtype, y_bf16, status,
+                      st);
+}
+
+}  // extern "C"

@@ -1,0 +1,108 @@
+// hstu_internal.h - declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sm100_ptx.cuh"
+
+namespace hstu {
+
+// ---------------------------------------------------------------------------------------------
+// workspace layout: [0, 256) status word + padding, then per-call regions
+// ---------------------------------------------------------------------------------------------
+constexpr size_t kWsHeader = 256;
+constexpr int kQTile = 128;       // rows of a query / key tile
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+WaitCtl wait_ctl(int* status);
+
+// ---------------------------------------------------------------------------------------------
+// GEMM
+// ---------------------------------------------------------------------------------------------
+enum : int { kEpiSilu = 0, kEpiLinear = 1, kEpiAtomic = 2 };
+
+struct GemmEpilogue {
+  int kind;
+  const float* bias;      // [N] or null
+  const void* resid;      // [M, N] or null (LINEAR)
+  int resid_f32;
+  int64_t ld_resid;
+  void* out0;             // SILU: SiLU(Z); LINEAR: Y; ATOMIC: fp32 accumulation target
+  int out0_f32;
+  int64_t ld_out0;
+  void* out1;             // SILU: Z; LINEAR: second copy of Y; or null
+  int out1_f32;
+  int64_t ld_out1;
+};
+
+struct GemmArgs {
+  const void* A;   // K-major: [M, K] (lda); MN-major: [K, M] (lda)
+  int64_t lda;
+  bool a_mn;
+  const void* B;   // K-major: [N, K] (ldb); MN-major: [K, N] (ldb)
+  int64_t ldb;
+  bool b_mn;
+  int64_t M, N, K;
+  int splits;      // split-K factor (ATOMIC epilogue only)
+  GemmEpilogue epi;
+  int* status;     // device status word
+};
+
+bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t outer,
+                         int64_t ld_elems, int box_inner, int box_outer);
+
+cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st);
+cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
+
+// ---------------------------------------------------------------------------------------------
+// jagged metadata / time buckets
+// ---------------------------------------------------------------------------------------------
+cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
+                            int32_t* count, int* status, cudaStream_t st);
+cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T,
+                                int n_buckets, const int64_t* sq_offsets, uint8_t* out,
+                                cudaStream_t st);
+
+// ---------------------------------------------------------------------------------------------
+// attention
+// ---------------------------------------------------------------------------------------------
+struct AttnArgs {
+  int B;
+  int64_t T;
+  int max_len;
+  const int64_t* offsets;
+  const int64_t* ts;
+  int H, dqk, dv;
+  float inv_N;
+  int pos_max_len;
+  int n_buckets;
+  const void* q; int64_t ld_q;
+  const void* k; int64_t ld_k;
+  const void* v; int64_t ld_v;
+  void* o; int64_t ld_o;
+  const float* rab_pos;
+  const float* rab_time;
+  const int32_t* items;    // work list (b, tile)
+  const int32_t* count;
+  int64_t capacity;
+  int* status;
+};
+
+cudaError_t attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t st);
+cudaError_t attn_fwd_f32_simt(const AttnArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------------------------------------
+// LayerNorm (.) U
+// ---------------------------------------------------------------------------------------------
+cudaError_t norm_gate_fwd(int64_t T, int D, bool bf16, const void* o, int64_t ld_o, const void* u,
+                          int64_t ld_u, const float* gamma, const float* beta, float eps, void* g,
+                          float* mu, float* rstd, cudaStream_t st);
+
+cudaError_t convert_f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t st);
+
+cudaError_t launch_timeout_probe(int* status, cudaStream_t st);
+
+}  // namespace hstu

@@ -1,0 +1,286 @@
+// jagged_norm.cu - HBM-bound kernels: jagged work list, time-bucket debug output, LayerNorm (.) U
+// gating, dtype conversion, and the timeout probe of the failure path.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hstu_internal.h"
+#include "sm100_ptx.cuh"
+#include "time_bucket_dev.cuh"
+
+namespace hstu {
+
+namespace {
+
+// ----------------------------------------------------------------------------------------------
+// Jagged tile work list ("4.4 Scaling Recommendation Models", Efficiency tricks: kernels over
+// variable-length sequences). One block: emits (b, t) for every query tile t of every sequence,
+// tiles with more causal key tiles first, ties by increasing b. Also validates the offsets:
+// offsets[0] == 0, non-decreasing, every length <= max_len, offsets[B] == T; a violation records
+// kDevBadInput and empties the list so no later kernel reads out of bounds.
+// ----------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024)
+worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items,
+                int32_t* count, int* status) {
+  __shared__ int s_warp[32];
+  __shared__ int s_max_tiles;
+  __shared__ int s_bad;
+  __shared__ int s_base;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    s_max_tiles = 0;
+    s_bad = (B < 0 || off[0] != 0 || off[B] != T) ? 1 : 0;
+    s_base = 0;
+  }
+  __syncthreads();
+  for (int b = tid; b < B; b += blockDim.x) {
+    const int64_t n = off[b + 1] - off[b];
+    if (n < 0 || n > max_len) atomicOr(&s_bad, 1);
+    else atomicMax(&s_max_tiles, static_cast<int>((n + kQTile - 1) / kQTile));
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) {
+      *count = 0;
+      report_error(status, kDevBadInput);
+    }
+    return;
+  }
+  const int max_tiles = s_max_tiles;
+  for (int t = max_tiles - 1; t >= 0; --t) {
+    for (int c0 = 0; c0 < B; c0 += blockDim.x) {
+      const int b = c0 + tid;
+      bool flag = false;
+      if (b < B) flag = (off[b + 1] - off[b] + kQTile - 1) / kQTile > t;
+      const unsigned m = __ballot_sync(0xffffffffu, flag);
+      if (lane == 0) s_warp[warp] = __popc(m);
+      __syncthreads();
+      if (warp == 0) {
+        const int v = s_warp[lane];
+        int inc = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, inc, d);
+          if (lane >= d) inc += y;
+        }
+        s_warp[lane] = inc - v;   // exclusive prefix over warps
+      }
+      __syncthreads();
+      const int pos = s_base + s_warp[warp] + __popc(m & ((1u << lane) - 1u));
+      if (flag) {
+        items[2 * pos] = b;
+        items[2 * pos + 1] = t;
+      }
+      __syncthreads();
+      if (tid == blockDim.x - 1) s_base = pos + (flag ? 1 : 0);
+      __syncthreads();
+    }
+  }
+  if (tid == 0) *count = s_base;
+}
+
+// One warp per query row: writes bucket(t_i - t_j) for every key j of the row's sequence.
+__global__ void __launch_bounds__(256)
+time_bucket_kernel(const int64_t* __restrict__ off, const int64_t* __restrict__ ts, int B, int64_t T,
+                   int nb, const int64_t* __restrict__ sq_off, uint8_t* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= T) return;
+  int lo = 0, hi = B;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (off[mid] <= row) lo = mid; else hi = mid;
+  }
+  const long long s0 = off[lo];
+  const long long n = off[lo + 1] - s0;
+  const long long ti = ts[row];
+  uint8_t* dst = out + sq_off[lo] + (row - s0) * n;
+  for (long long j = lane; j < n; j += 32) dst[j] = static_cast<uint8_t>(time_bucket_dev(ti - ts[s0 + j], c_time_octaves, nb));
+}
+
+// ----------------------------------------------------------------------------------------------
+// LayerNorm (.) U ("4.4 Scaling Recommendation Models", Generative Recommenders and HSTU, third
+// equation Norm(AV) (.) U; "HSTU: The First Exploration of the Scaling Law", 7.1.4 Innovation 3):
+// one warp per token, lane l holds features [l*VPT, (l+1)*VPT); mean and variance by warp
+// shuffles (two passes over registers), fp32 statistics stored for the backward.
+// ----------------------------------------------------------------------------------------------
+template <int VPT, bool BF16>
+__device__ __forceinline__ void load_vec(const void* base, int64_t idx, float* v) {
+  if constexpr (BF16) {
+    const uint16_t* p = reinterpret_cast<const uint16_t*>(base) + idx;
+    if constexpr (VPT % 8 == 0) {
+#pragma unroll
+      for (int q = 0; q < VPT / 8; ++q) {
+        const uint4 t = reinterpret_cast<const uint4*>(p)[q];
+        const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[8 * q + 2 * e] = __uint_as_float(w[e] << 16);
+          v[8 * q + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < VPT; ++e) v[e] = bf16_bits_to_float(p[e]);
+    }
+  } else {
+    const float* p = reinterpret_cast<const float*>(base) + idx;
+    if constexpr (VPT % 4 == 0) {
+#pragma unroll
+      for (int q = 0; q < VPT / 4; ++q) {
+        const float4 t = reinterpret_cast<const float4*>(p)[q];
+        v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < VPT; ++e) v[e] = p[e];
+    }
+  }
+}
+
+template <int VPT, bool BF16>
+__device__ __forceinline__ void store_vec(void* base, int64_t idx, const float* v) {
+  if constexpr (BF16) {
+    uint16_t* p = reinterpret_cast<uint16_t*>(base) + idx;
+    if constexpr (VPT % 8 == 0) {
+#pragma unroll
+      for (int q = 0; q < VPT / 8; ++q)
+        reinterpret_cast<uint4*>(p)[q] =
+            make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+    } else {
+#pragma unroll
+      for (int e = 0; e < VPT; e += 2) reinterpret_cast<uint32_t*>(p)[e / 2] = pack_bf16x2(v[e], v[e + 1]);
+    }
+  } else {
+    float* p = reinterpret_cast<float*>(base) + idx;
+#pragma unroll
+    for (int e = 0; e < VPT; ++e) p[e] = v[e];
+  }
+}
+
+template <int VPT, bool BF16>
+__global__ void __launch_bounds__(256)
+norm_gate_kernel(int64_t T, const void* __restrict__ o, int64_t ld_o, const void* __restrict__ u,
+                 int64_t ld_u, const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
+                 void* __restrict__ g, float* __restrict__ mu_out, float* __restrict__ rstd_out) {
+  constexpr int D = VPT * 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= T) return;
+  float x[VPT], uu[VPT];
+  load_vec<VPT, BF16>(o, row * ld_o + lane * VPT, x);
+  load_vec<VPT, BF16>(u, row * ld_u + lane * VPT, uu);
+  float s = 0.0f;
+#pragma unroll
+  for (int e = 0; e < VPT; ++e) s += x[e];
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+  const float mean = s * (1.0f / D);
+  float q = 0.0f;
+#pragma unroll
+  for (int e = 0; e < VPT; ++e) {
+    const float d = x[e] - mean;
+    q = fmaf(d, d, q);
+  }
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) q += __shfl_xor_sync(0xffffffffu, q, m);
+  const float rstd = rsqrtf(q * (1.0f / D) + eps);
+  float gm[VPT], bt[VPT];
+  load_vec<VPT, false>(gamma, lane * VPT, gm);
+  load_vec<VPT, false>(beta, lane * VPT, bt);
+#pragma unroll
+  for (int e = 0; e < VPT; ++e) x[e] = fmaf((x[e] - mean) * rstd, gm[e], bt[e]) * uu[e];
+  store_vec<VPT, BF16>(g, row * D + lane * VPT, x);
+  if (lane == 0) {
+    if (mu_out) mu_out[row] = mean;
+    if (rstd_out) rstd_out[row] = rstd;
+  }
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ in, uint16_t* __restrict__ out, int64_t n) {
+  const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i + 3 < n) {
+    const float4 v = *reinterpret_cast<const float4*>(in + i);
+    *reinterpret_cast<uint2*>(out + i) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  } else {
+    for (int64_t k = i; k < n; ++k) {
+      __nv_bfloat16 b = __float2bfloat16_rn(in[k]);
+      out[k] = *reinterpret_cast<uint16_t*>(&b);
+    }
+  }
+}
+
+// Waits on an mbarrier that nothing arrives at; the bounded wait records kDevTimeout.
+__global__ void timeout_probe_kernel(WaitCtl ctl) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, ctl);
+  __syncthreads();
+}
+
+template <int VPT, bool BF16>
+cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int64_t ld_u, const float* gamma,
+                      const float* beta, float eps, void* g, float* mu, float* rstd, cudaStream_t st) {
+  const int64_t blocks = (T + 7) / 8;
+  norm_gate_kernel<VPT, BF16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(T, o, ld_o, u, ld_u, gamma, beta, eps,
+                                                                             g, mu, rstd);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
+                            int32_t* count, int* status, cudaStream_t st) {
+  worklist_kernel<<<1, 1024, 0, st>>>(offsets, B, T, max_len, items, count, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int n_buckets,
+                                const int64_t* sq_offsets, uint8_t* out, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  cudaError_t e = upload_time_octaves();
+  if (e != cudaSuccess) return e;
+  time_bucket_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, st>>>(offsets, ts, B, T, n_buckets,
+                                                                          sq_offsets, out);
+  return cudaGetLastError();
+}
+
+cudaError_t norm_gate_fwd(int64_t T, int D, bool bf16, const void* o, int64_t ld_o, const void* u, int64_t ld_u,
+                          const float* gamma, const float* beta, float eps, void* g, float* mu, float* rstd,
+                          cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+#define HSTU_NG(VPT)                                                                                   \
+  return bf16 ? launch_ng<VPT, true>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st)           \
+              : launch_ng<VPT, false>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st)
+  switch (D) {
+    case 64: HSTU_NG(2);
+    case 128: HSTU_NG(4);
+    case 256: HSTU_NG(8);
+    case 512: HSTU_NG(16);
+    case 1024: HSTU_NG(32);
+    default: return cudaErrorInvalidValue;
+  }
+#undef HSTU_NG
+}
+
+cudaError_t convert_f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int64_t threads = (n + 3) / 4;
+  f32_to_bf16_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0, st>>>(in, static_cast<uint16_t*>(out), n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_timeout_probe(int* status, cudaStream_t st) {
+  timeout_probe_kernel<<<1, 32, 0, st>>>(wait_ctl(status));
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

@@ -1,0 +1,250 @@
+"""ctypes binding of libhstu.so: the C ABI's entry points under the same names.
+
+Argument marshalling only: descriptors become ctypes structures, torch tensors become device
+pointers, the current torch CUDA stream becomes the cudaStream_t. Every step of the computation
+runs in the library's CUDA kernels; nothing here computes. If the library is missing, every
+call raises -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+from .build import LIB as _LIB_PATH
+
+c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+HSTU_F32, HSTU_BF16 = 0, 1
+STATUS = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED", 3: "HSTU_ERR_WORKSPACE",
+          4: "HSTU_ERR_CUDA", 5: "HSTU_ERR_TIMEOUT", 6: "HSTU_ERR_DEVICE"}
+
+
+class HstuError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        extra = ""
+        if code == 4 and _lib is not None:
+            extra = f" (cudaError {_lib.hstu_last_cuda_error()})"
+        super().__init__(f"{fn} returned {STATUS.get(code, code)}{extra}")
+
+
+class hstu_jagged_t(ctypes.Structure):
+    _fields_ = [("B", c_i32), ("max_len", c_i32), ("T", c_i64), ("offsets", c_vp), ("timestamps", c_vp)]
+
+
+class hstu_attn_desc_t(ctypes.Structure):
+    _fields_ = [("H", c_i32), ("d_qk", c_i32), ("d_v", c_i32), ("inv_N", c_f32), ("pos_max_len", c_i32),
+                ("n_time_buckets", c_i32), ("dtype", c_i32), ("ld_q", c_i64), ("ld_k", c_i64),
+                ("ld_v", c_i64), ("ld_o", c_i64)]
+
+
+class hstu_layer_desc_t(ctypes.Structure):
+    _fields_ = [("D", c_i32), ("H", c_i32), ("inv_N", c_f32), ("pos_max_len", c_i32),
+                ("n_time_buckets", c_i32), ("ln_eps", c_f32), ("dtype", c_i32), ("x_dtype", c_i32),
+                ("y_dtype", c_i32)]
+
+
+class hstu_layer_weights_t(ctypes.Structure):
+    _fields_ = [(n, c_vp) for n in ("W1", "b1", "W2", "b2", "gamma", "beta", "rab_pos", "rab_time")]
+
+
+class hstu_layer_saved_t(ctypes.Structure):
+    _fields_ = [(n, c_vp) for n in ("uvqk", "z", "o", "g", "mu", "rstd")]
+
+
+class hstu_layer_grads_t(ctypes.Structure):
+    _fields_ = [(n, c_vp) for n in ("dW1", "db1", "dW2", "db2", "dgamma", "dbeta", "drab_pos", "drab_time")]
+
+
+P = ctypes.POINTER
+# name -> (restype, argtypes); the list every test checks against include/hstu.h
+SIGNATURES = {
+    "hstu_abi_version": (c_i32, []),
+    "hstu_status_string": (ctypes.c_char_p, [c_i32]),
+    "hstu_last_cuda_error": (c_i32, []),
+    "hstu_sync_status": (c_i32, [c_vp, c_vp, P(c_i32)]),
+    "hstu_set_wait_limit": (None, [ctypes.c_uint64]),
+    "hstu_debug_timeout_probe": (c_i32, [c_vp, c_sz, c_vp]),
+    "hstu_worklist_capacity": (c_i64, [P(hstu_jagged_t)]),
+    "hstu_jagged_worklist": (c_i32, [P(hstu_jagged_t), c_vp, c_vp, c_vp]),
+    "hstu_time_buckets": (c_i32, [P(hstu_jagged_t), c_i32, c_vp, c_vp, c_vp]),
+    "hstu_uvqk_fwd": (c_i32, [c_i64, c_i32, c_i32, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "hstu_attn_workspace_size": (c_sz, [P(hstu_attn_desc_t), P(hstu_jagged_t)]),
+    "hstu_attn_fwd": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                              c_vp, c_sz, c_vp]),
+    "hstu_norm_gate_fwd": (c_i32, [c_i64, c_i32, c_i32, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_f32, c_vp,
+                                   c_vp, c_vp, c_vp]),
+    "hstu_out_proj_fwd": (c_i32, [c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_i32, c_vp,
+                                  c_vp, c_sz, c_vp]),
+    "hstu_layer_workspace_size": (c_sz, [P(hstu_layer_desc_t), P(hstu_jagged_t)]),
+    "hstu_layer_fwd": (c_i32, [P(hstu_layer_desc_t), P(hstu_jagged_t), P(hstu_layer_weights_t), c_vp, c_vp,
+                               c_vp, c_vp, P(hstu_layer_saved_t), c_vp, c_sz, c_vp]),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libhstu.so (built in-tree by ``build.py``); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libhstu.so not built ({_LIB_PATH}); run "
+                               "`python -m hstu_sequential_transduction_causal_b200.build`")
+        l = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+# ----------------------------------------------------------------------------------------------
+# marshalling helpers
+# ----------------------------------------------------------------------------------------------
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    return t.data_ptr()
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return HSTU_BF16
+    if t.dtype == torch.float32:
+        return HSTU_F32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _check(fn: str, code: int):
+    if code != 0:
+        raise HstuError(fn, code)
+
+
+def make_jagged(offsets: torch.Tensor, timestamps: torch.Tensor, max_len: int) -> hstu_jagged_t:
+    """offsets: int64 [B+1] on the GPU; timestamps: int64 [T] on the GPU; T is read from the
+    caller's host knowledge of the batch (``timestamps.shape[0]``), never from the device."""
+    assert offsets.dtype == torch.int64 and timestamps.dtype == torch.int64
+    return hstu_jagged_t(B=offsets.shape[0] - 1, max_len=int(max_len), T=timestamps.shape[0],
+                         offsets=_ptr(offsets), timestamps=_ptr(timestamps) if timestamps.numel() else None)
+
+
+def make_attn_desc(H, d_qk, d_v, inv_N, pos_max_len, dtype_code, ld_q, ld_k, ld_v, ld_o,
+                   n_time_buckets=128) -> hstu_attn_desc_t:
+    return hstu_attn_desc_t(H=H, d_qk=d_qk, d_v=d_v, inv_N=inv_N, pos_max_len=pos_max_len,
+                            n_time_buckets=n_time_buckets, dtype=dtype_code, ld_q=ld_q, ld_k=ld_k,
+                            ld_v=ld_v, ld_o=ld_o)
+
+
+def make_layer_desc(D, H, inv_N, pos_max_len, dtype_code, x_dtype_code, y_dtype_code,
+                    n_time_buckets=128, ln_eps=1e-5) -> hstu_layer_desc_t:
+    return hstu_layer_desc_t(D=D, H=H, inv_N=inv_N, pos_max_len=pos_max_len, n_time_buckets=n_time_buckets,
+                             ln_eps=ln_eps, dtype=dtype_code, x_dtype=x_dtype_code, y_dtype=y_dtype_code)
+
+
+# ----------------------------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ----------------------------------------------------------------------------------------------
+
+def hstu_abi_version() -> int:
+    return lib().hstu_abi_version()
+
+
+def hstu_status_string(code: int) -> str:
+    return lib().hstu_status_string(code).decode()
+
+
+def hstu_sync_status(ws: torch.Tensor, stream=None) -> int:
+    out = c_i32(0)
+    _check("hstu_sync_status", lib().hstu_sync_status(_ptr(ws), _stream(stream), ctypes.byref(out)))
+    return out.value
+
+
+def hstu_set_wait_limit(cycles: int) -> None:
+    lib().hstu_set_wait_limit(int(cycles))
+
+
+def hstu_debug_timeout_probe(ws: torch.Tensor, stream=None) -> None:
+    _check("hstu_debug_timeout_probe", lib().hstu_debug_timeout_probe(_ptr(ws), ws.numel() * ws.element_size(),
+                                                                      _stream(stream)))
+
+
+def hstu_worklist_capacity(jag: hstu_jagged_t) -> int:
+    return lib().hstu_worklist_capacity(ctypes.byref(jag))
+
+
+def hstu_jagged_worklist(jag: hstu_jagged_t, items: torch.Tensor, count: torch.Tensor, stream=None) -> None:
+    _check("hstu_jagged_worklist", lib().hstu_jagged_worklist(ctypes.byref(jag), _ptr(items), _ptr(count),
+                                                              _stream(stream)))
+
+
+def hstu_time_buckets(jag: hstu_jagged_t, n_buckets: int, sq_offsets: torch.Tensor, out: torch.Tensor,
+                      stream=None) -> None:
+    _check("hstu_time_buckets", lib().hstu_time_buckets(ctypes.byref(jag), n_buckets, _ptr(sq_offsets),
+                                                        _ptr(out), _stream(stream)))
+
+
+def hstu_uvqk_fwd(T, D, dtype_code, x, ld_x, W1, b1, uvqk, z, ws, stream=None) -> None:
+    _check("hstu_uvqk_fwd", lib().hstu_uvqk_fwd(T, D, dtype_code, _ptr(x), ld_x, _ptr(W1), _ptr(b1), _ptr(uvqk),
+                                                _ptr(z), _ptr(ws), ws.numel() * ws.element_size(),
+                                                _stream(stream)))
+
+
+def hstu_attn_workspace_size(desc: hstu_attn_desc_t, jag: hstu_jagged_t) -> int:
+    return lib().hstu_attn_workspace_size(ctypes.byref(desc), ctypes.byref(jag))
+
+
+def hstu_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, ws, stream=None) -> None:
+    _check("hstu_attn_fwd", lib().hstu_attn_fwd(ctypes.byref(desc), ctypes.byref(jag), _ptr(q), _ptr(k), _ptr(v),
+                                                _ptr(rab_pos), _ptr(rab_time), _ptr(out), _ptr(ws),
+                                                ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def hstu_norm_gate_fwd(T, D, dtype_code, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, stream=None) -> None:
+    _check("hstu_norm_gate_fwd", lib().hstu_norm_gate_fwd(T, D, dtype_code, _ptr(o), ld_o, _ptr(u), ld_u,
+                                                          _ptr(gamma), _ptr(beta), eps, _ptr(g), _ptr(mu),
+                                                          _ptr(rstd), _stream(stream)))
+
+
+def hstu_out_proj_fwd(T, D, dtype_code, g, W2, b2, x, x_dtype_code, y, y_dtype_code, y_bf16, ws,
+                      stream=None) -> None:
+    _check("hstu_out_proj_fwd", lib().hstu_out_proj_fwd(T, D, dtype_code, _ptr(g), _ptr(W2), _ptr(b2), _ptr(x),
+                                                        x_dtype_code, _ptr(y), y_dtype_code, _ptr(y_bf16),
+                                                        _ptr(ws), ws.numel() * ws.element_size(),
+                                                        _stream(stream)))
+
+
+def hstu_layer_workspace_size(desc: hstu_layer_desc_t, jag: hstu_jagged_t) -> int:
+    return lib().hstu_layer_workspace_size(ctypes.byref(desc), ctypes.byref(jag))
+
+
+def hstu_layer_fwd(desc, jag, weights: hstu_layer_weights_t, x, x_bf16, y, y_bf16, saved: hstu_layer_saved_t,
+                   ws, stream=None) -> None:
+    _check("hstu_layer_fwd", lib().hstu_layer_fwd(ctypes.byref(desc), ctypes.byref(jag), ctypes.byref(weights),
+                                                  _ptr(x), _ptr(x_bf16), _ptr(y), _ptr(y_bf16),
+                                                  ctypes.byref(saved), _ptr(ws), ws.numel() * ws.element_size(),
+                                                  _stream(stream)))
+
+
+def layer_weights(W1, b1, W2, b2, gamma, beta, rab_pos, rab_time) -> hstu_layer_weights_t:
+    return hstu_layer_weights_t(*[_ptr(t) for t in (W1, b1, W2, b2, gamma, beta, rab_pos, rab_time)])
+
+
+def layer_saved(uvqk, z, o, g, mu, rstd) -> hstu_layer_saved_t:
+    return hstu_layer_saved_t(*[_ptr(t) for t in (uvqk, z, o, g, mu, rstd)])

@@ -1,0 +1,116 @@
+"""Host-side orchestration around the C ABI: device buffers, workspaces, descriptors.
+
+Nothing here computes: it uploads seeded inputs, allocates the caller-owned buffers the library
+writes into (via torch, which owns device memory and streams), fills the descriptors and calls
+the binding. Every arithmetic step runs inside libhstu.so.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import hstu as H
+
+
+def to_dev(a: np.ndarray, dtype: torch.dtype, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device=device, dtype=dtype)
+
+
+@dataclass
+class DeviceLayer:
+    """One layer's parameters on the GPU in the layout the library expects."""
+    D: int
+    H: int
+    dtype_code: int
+    W1: torch.Tensor
+    b1: torch.Tensor
+    W2: torch.Tensor
+    b2: torch.Tensor
+    gamma: torch.Tensor
+    beta: torch.Tensor
+    rab_pos: torch.Tensor
+    rab_time: torch.Tensor
+
+    @classmethod
+    def upload(cls, p, D: int, H_: int, bf16: bool, device="cuda") -> "DeviceLayer":
+        wdt = torch.bfloat16 if bf16 else torch.float32
+        f32 = torch.float32
+        return cls(D=D, H=H_, dtype_code=H.HSTU_BF16 if bf16 else H.HSTU_F32,
+                   W1=to_dev(p.W1, wdt, device), b1=to_dev(p.b1, f32, device), W2=to_dev(p.W2, wdt, device),
+                   b2=to_dev(p.b2, f32, device), gamma=to_dev(p.gamma, f32, device),
+                   beta=to_dev(p.beta, f32, device), rab_pos=to_dev(p.rab_pos, f32, device),
+                   rab_time=to_dev(p.rab_time, f32, device))
+
+    def weights(self) -> H.hstu_layer_weights_t:
+        return H.layer_weights(self.W1, self.b1, self.W2, self.b2, self.gamma, self.beta, self.rab_pos,
+                               self.rab_time)
+
+
+@dataclass
+class SavedActs:
+    uvqk: torch.Tensor
+    z: Optional[torch.Tensor]
+    o: torch.Tensor
+    g: torch.Tensor
+    mu: torch.Tensor
+    rstd: torch.Tensor
+
+    @classmethod
+    def empty(cls, T: int, D: int, dtype: torch.dtype, keep_z: bool, device="cuda") -> "SavedActs":
+        return cls(uvqk=torch.empty(T, 4 * D, dtype=dtype, device=device),
+                   z=torch.empty(T, 4 * D, dtype=dtype, device=device) if keep_z else None,
+                   o=torch.empty(T, D, dtype=dtype, device=device), g=torch.empty(T, D, dtype=dtype, device=device),
+                   mu=torch.empty(T, dtype=torch.float32, device=device),
+                   rstd=torch.empty(T, dtype=torch.float32, device=device))
+
+    def struct(self) -> H.hstu_layer_saved_t:
+        return H.layer_saved(self.uvqk, self.z, self.o, self.g, self.mu, self.rstd)
+
+
+class JaggedBatch:
+    """Offsets and timestamps on the GPU plus the host-side sizes the descriptors need."""
+
+    def __init__(self, offsets: np.ndarray, timestamps: np.ndarray, max_len: Optional[int] = None,
+                 device="cuda"):
+        self.offsets_np = np.asarray(offsets, np.int64)
+        self.B = int(self.offsets_np.shape[0] - 1)
+        self.T = int(self.offsets_np[-1])
+        lens = np.diff(self.offsets_np)
+        self.max_len = int(max_len if max_len is not None else (lens.max() if self.B else 0))
+        self.offsets = to_dev(self.offsets_np, torch.int64, device)
+        self.timestamps = to_dev(np.asarray(timestamps, np.int64), torch.int64, device)
+        self.struct = H.make_jagged(self.offsets, self.timestamps, self.max_len)
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace (its first word is the device status word)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+class LayerRunner:
+    """Runs ``hstu_layer_fwd`` for one layer on a fixed jagged batch with reusable buffers."""
+
+    def __init__(self, layer: DeviceLayer, jag: JaggedBatch, inv_N: float, pos_max_len: int,
+                 x_dtype: torch.dtype, y_dtype: torch.dtype, keep_z: bool = False, device="cuda"):
+        self.layer, self.jag = layer, jag
+        cdt = torch.bfloat16 if layer.dtype_code == H.HSTU_BF16 else torch.float32
+        code = {torch.bfloat16: H.HSTU_BF16, torch.float32: H.HSTU_F32}
+        self.desc = H.make_layer_desc(layer.D, layer.H, inv_N, pos_max_len, layer.dtype_code, code[x_dtype],
+                                      code[y_dtype])
+        self.saved = SavedActs.empty(jag.T, layer.D, cdt, keep_z, device)
+        self.saved_struct = self.saved.struct()
+        self.ws = workspace(H.hstu_layer_workspace_size(self.desc, jag.struct), device)
+        self.y = torch.empty(jag.T, layer.D, dtype=y_dtype, device=device)
+        self.weights = layer.weights()
+
+    def forward(self, x: torch.Tensor, x_bf16: Optional[torch.Tensor] = None,
+                y_bf16: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        H.hstu_layer_fwd(self.desc, self.jag.struct, self.weights, x, x_bf16, self.y, y_bf16,
+                         self.saved_struct, self.ws, stream)
+        return self.y
+
+    def device_status(self) -> int:
+        return H.hstu_sync_status(self.ws)

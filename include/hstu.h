@@ -1,0 +1,247 @@
+/*
+ * hstu.h - C ABI of the B200 (sm_100a) HSTU layer library (libhstu.so).
+ *
+ * The library computes the HSTU layer of Generative Recommenders over jagged (variable-length,
+ * offset-indexed) user action sequences:
+ *
+ *   U, V, Q, K = Split(SiLU(X W1^T + b1))                                   (f1, phi1)
+ *   O_i        = sum_{j <= i, same sequence} SiLU(q_i.k_j + rab_pos[i-j] + rab_time[b_ij]) / N * v_j
+ *   Y          = (LayerNorm(O) (.) U) W2^T + b2 + X                          (f2 + residual)
+ *
+ * as stated in "4.4 Scaling Recommendation Models" (LLM learning path), section "Generative
+ * Recommenders and HSTU" (the three layer equations and the pointwise-aggregation bullet) and
+ * its section "Code" (chunk order U|V|Q|K, causal lower triangle including the diagonal, division
+ * by a constant, LayerNorm over d_model, residual after f2); and in "HSTU: The First Exploration
+ * of the Scaling Law" (fun-rec 7.1), 7.1.4 Innovations 1-3 and 7.1.5 (Stochastic Length,
+ * M-FALCON).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor argument is a DEVICE pointer owned by the caller unless stated otherwise;
+ *    descriptor structs are host memory read during the call only. The library never allocates,
+ *    frees or synchronises: scratch space comes from a caller workspace whose size the matching
+ *    *_workspace_size() returns. A workspace must be zero-filled once before its first use
+ *    (it holds the device status word) and must not be shared by calls that overlap on the GPU.
+ *  - Work is enqueued on `stream` (a cudaStream_t); calls return once it is enqueued.
+ *  - Matrices are row-major; ld_* arguments are row strides in ELEMENTS. bf16 tensors use the
+ *    bfloat16 bit layout (uint16). Pointers handed to the tensor-core kernels must be 16-byte
+ *    aligned and their row strides multiples of 8 elements (16 bytes).
+ *  - Host-side argument errors return HSTU_ERR_INVALID_ARG / HSTU_ERR_UNSUPPORTED /
+ *    HSTU_ERR_WORKSPACE before anything is enqueued. A CUDA launch error returns HSTU_ERR_CUDA
+ *    (hstu_last_cuda_error() gives the cudaError_t). Errors found on the device (a bounded wait
+ *    that ran out, a violated jagged contract) are recorded in the workspace status word and
+ *    reported by hstu_sync_status(); the kernels then return early, never trap.
+ *  - Jagged layout: sequence b owns rows [offsets[b], offsets[b+1]) of every [T, ...] tensor.
+ *    offsets must be non-decreasing with offsets[0] = 0 and offsets[B] = T; max_len must bound
+ *    every length. Timestamps are int64 (any unit, any order); the time bucket of a pair is
+ *    min(n_buckets-1, floor(ln(max(t_i - t_j, 1)) / 0.301)), evaluated exactly in integers.
+ *  - rab_pos has 2*pos_max_len-1 fp32 entries indexed by clip(i-j, -(L-1), L-1) + L-1 with i, j
+ *    positions inside the sequence; rab_time has n_time_buckets (<= 128) fp32 entries. Both are
+ *    shared by all heads.
+ */
+#ifndef HSTU_H_
+#define HSTU_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HSTU_ABI_VERSION 1
+
+typedef struct CUstream_st* hstu_stream_t; /* same type as cudaStream_t; NULL = legacy stream */
+
+typedef enum hstu_status_t {
+  HSTU_OK = 0,
+  HSTU_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent descriptor */
+  HSTU_ERR_UNSUPPORTED = 2,  /* shape / dtype / alignment the kernels do not implement */
+  HSTU_ERR_WORKSPACE = 3,    /* workspace missing or smaller than *_workspace_size() */
+  HSTU_ERR_CUDA = 4,         /* a CUDA runtime call failed; see hstu_last_cuda_error() */
+  HSTU_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out (reported on the device) */
+  HSTU_ERR_DEVICE = 6        /* a device-side check failed (reported on the device) */
+} hstu_status_t;
+
+typedef enum hstu_dtype_t { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype_t;
+
+/* Jagged batch of B sequences, T tokens in total. */
+typedef struct hstu_jagged_t {
+  int32_t B;                  /* number of sequences (>= 0) */
+  int32_t max_len;            /* host upper bound on every sequence length */
+  int64_t T;                  /* total tokens = offsets[B] */
+  const int64_t* offsets;     /* device, [B+1] */
+  const int64_t* timestamps;  /* device, [T] */
+} hstu_jagged_t;
+
+/* Pointwise attention of one layer. */
+typedef struct hstu_attn_desc_t {
+  int32_t H;               /* heads */
+  int32_t d_qk;            /* per-head query/key width (bf16: 64; f32: 1..64) */
+  int32_t d_v;             /* per-head value width (bf16: 64; f32: 1..64) */
+  float inv_N;             /* 1/N, the constant normaliser */
+  int32_t pos_max_len;     /* L: rab_pos has 2L-1 entries */
+  int32_t n_time_buckets;  /* 1..128 */
+  hstu_dtype_t dtype;      /* dtype of q, k, v, out */
+  int64_t ld_q, ld_k, ld_v, ld_o; /* row strides (elements); head h occupies columns [h*d, (h+1)*d) */
+} hstu_attn_desc_t;
+
+/* One HSTU layer, d_qk = d_v = D/H. */
+typedef struct hstu_layer_desc_t {
+  int32_t D;               /* d_model */
+  int32_t H;               /* heads */
+  float inv_N;
+  int32_t pos_max_len;
+  int32_t n_time_buckets;
+  float ln_eps;            /* LayerNorm epsilon (1e-5) */
+  hstu_dtype_t dtype;      /* compute dtype: BF16 (tensor cores, fp32 accumulate) or F32 */
+  hstu_dtype_t x_dtype;    /* dtype of X; F32 with BF16 compute = fp32 residual stream */
+  hstu_dtype_t y_dtype;    /* dtype of Y */
+} hstu_layer_desc_t;
+
+/* Layer parameters. W1 [4D, D] rows ordered U|V|Q|K, W2 [D, D], both of the compute dtype;
+ * the vectors are fp32: b1 [4D], b2 [D], gamma [D], beta [D], rab_pos [2L-1], rab_time [nb]. */
+typedef struct hstu_layer_weights_t {
+  const void* W1;
+  const float* b1;
+  const void* W2;
+  const float* b2;
+  const float* gamma;
+  const float* beta;
+  const float* rab_pos;
+  const float* rab_time;
+} hstu_layer_weights_t;
+
+/* Activations a layer forward writes and its backward reads (compute dtype unless noted).
+ * uvqk [T, 4D] = SiLU(Z); z [T, 4D] pre-activation (may be NULL when no backward follows);
+ * o [T, D] attention output; g [T, D] = LN(O) (.) U; mu, rstd [T] fp32 LayerNorm statistics. */
+typedef struct hstu_layer_saved_t {
+  void* uvqk;
+  void* z;
+  void* o;
+  void* g;
+  float* mu;
+  float* rstd;
+} hstu_layer_saved_t;
+
+/* Weight gradients of one layer (fp32, overwritten): dW1 [4D, D], db1 [4D], dW2 [D, D], db2 [D],
+ * dgamma [D], dbeta [D], drab_pos [2L-1], drab_time [nb]. */
+typedef struct hstu_layer_grads_t {
+  float* dW1;
+  float* db1;
+  float* dW2;
+  float* db2;
+  float* dgamma;
+  float* dbeta;
+  float* drab_pos;
+  float* drab_time;
+} hstu_layer_grads_t;
+
+/* ---------------------------------------------------------------------------------------------
+ * Library information and device status
+ * ------------------------------------------------------------------------------------------- */
+
+/* ABI version of the loaded library (HSTU_ABI_VERSION). */
+int32_t hstu_abi_version(void);
+
+/* Static string naming a status; never NULL. */
+const char* hstu_status_string(hstu_status_t s);
+
+/* The cudaError_t of the last failed CUDA call made by the library on this host thread. */
+int32_t hstu_last_cuda_error(void);
+
+/* Reads the device status word of `ws` (after synchronising `stream`), resets it to 0 and
+ * stores it in *device_status (HSTU_OK when no kernel reported an error). The return value is
+ * HSTU_OK unless reading itself failed. */
+hstu_status_t hstu_sync_status(void* ws, hstu_stream_t stream, int32_t* device_status);
+
+/* Upper bound, in SM clock cycles, of every device-side wait; 0 restores the default
+ * (2^31 cycles, about a second). Process-wide; affects launches made after the call. */
+void hstu_set_wait_limit(uint64_t cycles);
+
+/* Test surface for the failure path: launches one CTA that waits on an mbarrier nothing ever
+ * arrives at, bounded by the wait limit; it records HSTU_ERR_TIMEOUT in the status word of `ws`
+ * and returns. Lets a test check the timeout path without a hang. */
+hstu_status_t hstu_debug_timeout_probe(void* ws, size_t ws_bytes, hstu_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Jagged metadata  ("4.4 Scaling Recommendation Models", Efficiency tricks: kernels over
+ * variable-length sequences; padding is never computed)
+ * ------------------------------------------------------------------------------------------- */
+
+/* Number of (sequence, 128-row query tile) items a batch can produce: B + ceil(T / 128). */
+int64_t hstu_worklist_capacity(const hstu_jagged_t* jag);
+
+/* Builds the causal tile work list: every (sequence b, query tile t) pair with t <
+ * ceil(n_b/128), ordered by decreasing cost (tile t visits t+1 key tiles), ties by increasing b.
+ * items: device int32 [capacity, 2] receiving (b, t); count: device int32 [1]. */
+hstu_status_t hstu_jagged_worklist(const hstu_jagged_t* jag, int32_t* items, int32_t* count,
+                                   hstu_stream_t stream);
+
+/* Debug surface of the relative-time bias index ("HSTU: The First Exploration of the Scaling
+ * Law", 7.1.4 Innovation 2): for every sequence b writes the n_b x n_b matrix of bucket(t_i -
+ * t_j) (row i query, column j key, u8) at out + sq_offsets[b]; sq_offsets: device int64 [B+1],
+ * the prefix sums of n_b^2. n_buckets in 1..128. */
+hstu_status_t hstu_time_buckets(const hstu_jagged_t* jag, int32_t n_buckets,
+                                const int64_t* sq_offsets, uint8_t* out, hstu_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Layer steps
+ * ------------------------------------------------------------------------------------------- */
+
+/* f1 + SiLU + split ("Generative Recommenders and HSTU", first equation):
+ * uvqk[t, :] = SiLU(x[t, :] W1^T + b1), [T, 4D] with row stride 4D; z (nullable) receives the
+ * pre-activation. x, W1, uvqk, z have the compute dtype; ld_x is x's row stride. ws: any
+ * workspace of at least 256 bytes (its status word receives device-side errors). */
+hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* x,
+                            int64_t ld_x, const void* W1, const float* b1, void* uvqk, void* z,
+                            void* ws, size_t ws_bytes, hstu_stream_t stream);
+
+/* Workspace bytes hstu_attn_fwd / hstu_attn_bwd need for this batch. */
+size_t hstu_attn_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag);
+
+/* Pointwise causal attention forward ("Generative Recommenders and HSTU", second equation and
+ * the pointwise-aggregation bullet; "HSTU: The First Exploration of the Scaling Law", 7.1.4
+ * Innovations 1-2): out[i, h] = sum_{j<=i} SiLU(q_i.k_j + rab_pos + rab_time) * inv_N * v_j.
+ * q, k, v, out: [T, ...] of desc->dtype with strides ld_q.. ld_o. Rows of empty work are not
+ * written; every valid row is. */
+hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag,
+                            const void* q, const void* k, const void* v, const float* rab_pos,
+                            const float* rab_time, void* out, void* ws, size_t ws_bytes,
+                            hstu_stream_t stream);
+
+/* LayerNorm (.) U gating ("Generative Recommenders and HSTU", third equation; "HSTU: The First
+ * Exploration of the Scaling Law", 7.1.4 Innovation 3): g = (gamma (o - mu) rstd + beta) (.) u
+ * over all D features of a token; mu, rstd (fp32 [T]) are stored for the backward. */
+hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* o,
+                                 int64_t ld_o, const void* u, int64_t ld_u, const float* gamma,
+                                 const float* beta, float eps, void* g, float* mu, float* rstd,
+                                 hstu_stream_t stream);
+
+/* f2 + residual ("Generative Recommenders and HSTU", third equation; residual of the "Code"
+ * sketch): y = g W2^T + b2 + x. g, W2 have the compute dtype; x has x_dtype; y has y_dtype;
+ * y_bf16 (nullable) receives a second, bf16 copy of y (the next layer's GEMM operand).
+ * ws: any workspace of at least 256 bytes (status word). F32 compute needs F32 x and y. */
+hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* g,
+                                const void* W2, const float* b2, const void* x,
+                                hstu_dtype_t x_dtype, void* y, hstu_dtype_t y_dtype,
+                                void* y_bf16, void* ws, size_t ws_bytes, hstu_stream_t stream);
+
+/* Workspace bytes hstu_layer_fwd / hstu_layer_bwd need. */
+size_t hstu_layer_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
+
+/* Whole layer forward: uvqk -> attention -> norm-gate -> out-projection, on `stream`.
+ * x: [T, D] of desc->x_dtype; x_bf16 (nullable) a bf16 copy of x used as the f1 operand when
+ * x_dtype is F32 with BF16 compute (converted into the workspace when NULL). y: [T, D] of
+ * desc->y_dtype; y_bf16 nullable second output. saved: buffers for the intermediates (all
+ * required except z). */
+hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag,
+                             const hstu_layer_weights_t* w, const void* x, const void* x_bf16,
+                             void* y, void* y_bf16, const hstu_layer_saved_t* saved, void* ws,
+                             size_t ws_bytes, hstu_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_H_ */

@@ -1,0 +1,290 @@
+"""GPU parity of the forward path: each step and the whole layer, through the C ABI, against the
+CPU oracle on the same seeded inputs. Integer work (work list, time buckets) is bit-exact;
+floating outputs meet |d| <= 1e-2 + 1e-2|ref| (bf16) or 1e-4 + 1e-4|ref| (fp32)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import hstu_oracle as O
+from hstu_sequential_transduction_causal_b200 import hstu as H
+from hstu_sequential_transduction_causal_b200 import workloads as W
+from hstu_sequential_transduction_causal_b200.runtime import (DeviceLayer, JaggedBatch, LayerRunner, to_dev,
+                                                              workspace)
+from tests._util import BF16_TOL, F32_TOL, THR, assert_close, layer_oracle, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from hstu_sequential_transduction_causal_b200 import build
+    build.build()
+    H.lib()
+    torch.cuda.init()
+
+
+def _bf16(a):
+    return W.round_bf16(np.asarray(a, np.float64))
+
+
+def _silu_like(rng, shape):
+    z = rng.standard_normal(shape)
+    return _bf16(z / (1 + np.exp(-z)))
+
+
+# ---------------------------------------------------------------------------------------------
+# integer steps: bit-exact
+# ---------------------------------------------------------------------------------------------
+
+def test_worklist_bit_exact():
+    lengths = [0, 1, 127, 128, 129, 300, 1024, 5, 0, 700, 256, 257]
+    off = W.offsets_from_lengths(lengths)
+    jag = JaggedBatch(off, np.zeros(off[-1], np.int64), max_len=1024)
+    cap = H.hstu_worklist_capacity(jag.struct)
+    items = torch.full((cap, 2), -1, dtype=torch.int32, device="cuda")
+    count = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    H.hstu_jagged_worklist(jag.struct, items, count)
+    exp = O.tile_work_list(off, 128)
+    n = int(count.item())
+    assert n == len(exp)
+    assert np.array_equal(items[:n].cpu().numpy().astype(np.int64), exp)
+
+
+def test_time_buckets_bit_exact():
+    rng = np.random.default_rng(3)
+    lengths = [3, 70, 0, 200, 1]
+    off = W.offsets_from_lengths(lengths)
+    T = int(off[-1])
+    ts = W.draw_timestamps(rng, lengths)
+    # sequence 1: out of order, negative and threshold-adjacent differences, huge gaps
+    s1 = slice(int(off[1]), int(off[2]))
+    taus = THR[rng.integers(0, 127, size=70)]
+    ts[s1] = 10 ** 15 + np.where(rng.random(70) < 0.5, taus, taus - 1) * rng.choice([-1, 1], 70)
+    ts[int(off[3]):int(off[3]) + 5] = [0, 2 ** 62, -(2 ** 61), 7, 7]
+    jag = JaggedBatch(off, ts)
+    lens = np.diff(off)
+    sq = W.offsets_from_lengths(lens ** 2)
+    out = torch.full((int(sq[-1]),), 255, dtype=torch.uint8, device="cuda")
+    H.hstu_time_buckets(jag.struct, 128, to_dev(sq, torch.int64), out)
+    got = out.cpu().numpy()
+    for b in range(len(lengths)):
+        s, e = off[b], off[b + 1]
+        exp = O.time_bucket(ts[s:e][:, None] - ts[s:e][None, :], THR).reshape(-1)
+        assert np.array_equal(got[sq[b]:sq[b + 1]].astype(np.int64), exp), b
+
+
+# ---------------------------------------------------------------------------------------------
+# single steps
+# ---------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_uvqk_fwd(dtype):
+    rng = np.random.default_rng(1)
+    T, D = (333, 256) if dtype == "bf16" else (437, 64)
+    bf = dtype == "bf16"
+    tdt = torch.bfloat16 if bf else torch.float32
+    cast = _bf16 if bf else (lambda a: np.asarray(a, np.float32))
+    x = cast(rng.standard_normal((T, D)))
+    W1 = cast(rng.standard_normal((4 * D, D)) / np.sqrt(D))
+    b1 = (0.1 * rng.standard_normal(4 * D)).astype(np.float32)
+    uvqk = torch.empty(T, 4 * D, dtype=tdt, device="cuda")
+    z = torch.empty(T, 4 * D, dtype=tdt, device="cuda")
+    ws = workspace(256)
+    H.hstu_uvqk_fwd(T, D, H.HSTU_BF16 if bf else H.HSTU_F32, to_dev(x, tdt), D, to_dev(W1, tdt),
+                    to_dev(b1, torch.float32), uvqk, z, ws)
+    ze, se = O.uvqk_fwd(x, W1, b1)
+    tol = BF16_TOL if bf else F32_TOL
+    assert_close(z.float().cpu().numpy(), ze, *tol, what="Z")
+    assert_close(uvqk.float().cpu().numpy(), se, *tol, what="SiLU(Z)")
+    assert H.hstu_sync_status(ws) == 0
+
+
+def _attn_case(lengths, Hh, d, L, inv_N, bf, seed=0, table_std=1.0, spread_ts=False):
+    rng = np.random.default_rng(seed)
+    off = W.offsets_from_lengths(lengths)
+    T = int(off[-1])
+    ts = W.draw_timestamps(rng, lengths)
+    if spread_ts:
+        ts = ts + rng.integers(-10 ** 6, 10 ** 9, size=T)
+    cast = _bf16 if bf else (lambda a: np.asarray(a, np.float32))
+    q = _silu_like(rng, (T, Hh * d)) if bf else rng.standard_normal((T, Hh * d)).astype(np.float32)
+    k = _silu_like(rng, (T, Hh * d)) if bf else rng.standard_normal((T, Hh * d)).astype(np.float32)
+    v = _silu_like(rng, (T, Hh * d)) if bf else rng.standard_normal((T, Hh * d)).astype(np.float32)
+    q, k, v = cast(q), cast(k), cast(v)
+    rp = (table_std * rng.standard_normal(2 * L - 1)).astype(np.float32)
+    rt = (table_std * rng.standard_normal(128)).astype(np.float32)
+    return off, ts, q, k, v, rp, rt
+
+
+def _run_attn(off, ts, q, k, v, rp, rt, Hh, d, L, inv_N, bf, max_len=None):
+    tdt = torch.bfloat16 if bf else torch.float32
+    jag = JaggedBatch(off, ts, max_len=max_len)
+    T = jag.T
+    desc = H.make_attn_desc(Hh, d, d, inv_N, L, H.HSTU_BF16 if bf else H.HSTU_F32, Hh * d, Hh * d, Hh * d, Hh * d)
+    ws = workspace(H.hstu_attn_workspace_size(desc, jag.struct))
+    out = torch.full((T, Hh * d), float("nan"), dtype=tdt, device="cuda")
+    H.hstu_attn_fwd(desc, jag.struct, to_dev(q, tdt), to_dev(k, tdt), to_dev(v, tdt), to_dev(rp, torch.float32),
+                    to_dev(rt, torch.float32), out, ws)
+    st = H.hstu_sync_status(ws)
+    return out.float().cpu().numpy(), st
+
+
+@pytest.mark.parametrize("spread", [False, True])
+def test_attn_fwd_bf16_ragged(spread):
+    lengths = [1, 127, 128, 129, 300, 0, 513, 64, 2]
+    Hh, d, L = 2, 64, 600
+    inv_N = 1.0 / 512
+    off, ts, q, k, v, rp, rt = _attn_case(lengths, Hh, d, L, inv_N, True, seed=2, spread_ts=spread)
+    got, st = _run_attn(off, ts, q, k, v, rp, rt, Hh, d, L, inv_N, True)
+    assert st == 0
+    T = int(off[-1])
+    exp = O.pointwise_attention_fwd(q.reshape(T, Hh, d), k.reshape(T, Hh, d), v.reshape(T, Hh, d), off, ts, rp, rt,
+                                    inv_N, L, THR).reshape(T, Hh * d)
+    scale = float(np.sqrt(np.mean(exp ** 2)))
+    assert_close(got, exp, 1e-2 * scale, 1e-2, what="O bf16")
+
+
+def test_attn_fwd_f32_single_layer_workload():
+    wl = W.make_workload("c1", seed=0)
+    Hh, d, L = wl.H, wl.D // wl.H, wl.pos_max_len
+    off, ts, q, k, v, rp, rt = _attn_case([17, 64, 100, 256], Hh, d, L, 1 / 256, False, seed=5)
+    got, st = _run_attn(off, ts, q, k, v, rp, rt, Hh, d, L, 1 / 256, False)
+    assert st == 0
+    T = int(off[-1])
+    exp = O.pointwise_attention_fwd(q.reshape(T, Hh, d), k.reshape(T, Hh, d), v.reshape(T, Hh, d), off, ts, rp, rt,
+                                    1 / 256, L, THR).reshape(T, Hh * d)
+    assert_close(got, exp, *F32_TOL, what="O f32")
+
+
+def test_norm_gate_bf16():
+    rng = np.random.default_rng(4)
+    T, D = 257, 512
+    o = _bf16(0.05 * rng.standard_normal((T, D)) + 0.02)
+    uvqk = _silu_like(rng, (T, 4 * D))
+    gamma = (1 + 0.2 * rng.standard_normal(D)).astype(np.float32)
+    beta = (0.2 * rng.standard_normal(D)).astype(np.float32)
+    g = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+    mu = torch.empty(T, dtype=torch.float32, device="cuda")
+    rstd = torch.empty(T, dtype=torch.float32, device="cuda")
+    H.hstu_norm_gate_fwd(T, D, H.HSTU_BF16, to_dev(o, torch.bfloat16), D, to_dev(uvqk, torch.bfloat16), 4 * D,
+                         to_dev(gamma, torch.float32), to_dev(beta, torch.float32), 1e-5, g, mu, rstd)
+    ge, mue, rse = O.norm_gate_fwd(o, uvqk[:, :D], gamma, beta)
+    assert_close(g.float().cpu().numpy(), ge, *BF16_TOL, what="G")
+    assert_close(mu.cpu().numpy(), mue, 1e-6, 1e-5, what="mu")
+    assert_close(rstd.cpu().numpy(), rse, 1e-6, 1e-4, what="rstd")
+
+
+@pytest.mark.parametrize("xdt,ydt", [("bf16", "bf16"), ("f32", "f32")])
+def test_out_proj_bf16(xdt, ydt):
+    rng = np.random.default_rng(6)
+    T, D = 300, 512
+    g = _bf16(rng.standard_normal((T, D)))
+    W2 = _bf16(rng.standard_normal((D, D)) / np.sqrt(D))
+    b2 = (0.1 * rng.standard_normal(D)).astype(np.float32)
+    x = _bf16(rng.standard_normal((T, D))) if xdt == "bf16" else rng.standard_normal((T, D)).astype(np.float32)
+    tx = torch.bfloat16 if xdt == "bf16" else torch.float32
+    ty = torch.bfloat16 if ydt == "bf16" else torch.float32
+    y = torch.empty(T, D, dtype=ty, device="cuda")
+    y2 = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
+    ws = workspace(256)
+    H.hstu_out_proj_fwd(T, D, H.HSTU_BF16, to_dev(g, torch.bfloat16), to_dev(W2, torch.bfloat16),
+                        to_dev(b2, torch.float32), to_dev(x, tx), H._dtype_code(y.new_empty(0, dtype=tx)), y,
+                        H._dtype_code(y), y2, ws)
+    ye = O.out_proj_fwd(g, W2, b2, x)
+    assert_close(y.float().cpu().numpy(), ye, *BF16_TOL, what="Y")
+    assert_close(y2.float().cpu().numpy(), ye, *BF16_TOL, what="Y bf16 copy")
+
+
+# ---------------------------------------------------------------------------------------------
+# whole layer
+# ---------------------------------------------------------------------------------------------
+
+def _run_layer(wl, x_dtype=None, y_dtype=None, x_override=None):
+    bf = wl.dtype == "bf16"
+    cdt = torch.bfloat16 if bf else torch.float32
+    x_dtype = x_dtype or cdt
+    y_dtype = y_dtype or cdt
+    jag = JaggedBatch(wl.offsets, wl.timestamps, max_len=max(wl.max_len, 1))
+    layer = DeviceLayer.upload(wl.layers[0], wl.D, wl.H, bf)
+    run = LayerRunner(layer, jag, 1.0 / wl.N, wl.pos_max_len, x_dtype, y_dtype, keep_z=True)
+    x = wl.x if x_override is None else x_override
+    y = run.forward(to_dev(x, x_dtype))
+    torch.cuda.synchronize()
+    return y.float().cpu().numpy(), run
+
+
+def test_layer_fwd_single_layer_fp32_workload():
+    wl = W.make_workload("c1", seed=0)
+    y, run = _run_layer(wl)
+    assert run.device_status() == 0
+    ye, _ = layer_oracle(wl)
+    assert_close(y, ye, *F32_TOL, what="Y c1 fp32")
+
+
+def test_layer_fwd_bf16_32_sequences_full():
+    wl = W.make_workload("c2", seed=0)
+    y, run = _run_layer(wl)
+    assert run.device_status() == 0
+    ye, inter = layer_oracle(wl)
+    assert_close(y, ye, *BF16_TOL, what="Y c2 bf16")
+
+
+def test_layer_fwd_long_sequences_sampled_rows():
+    wl = W.make_workload("c3", seed=0)
+    y, run = _run_layer(wl)
+    assert run.device_status() == 0
+    rows = sample_rows(wl.offsets, per_seq=6)
+    ye, _ = layer_oracle(wl, rows=rows)
+    assert_close(y[rows], ye, *BF16_TOL, what="Y c3 bf16 (sampled rows)")
+
+
+def test_layer_fwd_fp32_residual_stream():
+    wl = W.make_workload("c4", seed=1, lengths=[200, 1, 0, 385, 128], layers=1)
+    x32 = np.random.default_rng(9).standard_normal((wl.T, wl.D)).astype(np.float32)
+    y, run = _run_layer(wl, torch.float32, torch.float32, x_override=x32)
+    assert run.device_status() == 0
+    # the f1 operand is the bf16 rounding of the fp32 residual; the residual itself stays fp32
+    p = wl.layers[0]
+    xr = W.round_bf16(x32)
+    D = wl.D
+    z, s = O.uvqk_fwd(xr, p.W1, p.b1)
+    u, v, q, k = O.split_uvqk(s, D)
+    T, d = wl.T, D // wl.H
+    o = O.pointwise_attention_fwd(q.reshape(T, wl.H, d), k.reshape(T, wl.H, d), v.reshape(T, wl.H, d), wl.offsets,
+                                  wl.timestamps, p.rab_pos, p.rab_time, 1 / wl.N, wl.pos_max_len, THR).reshape(T, D)
+    g, _, _ = O.norm_gate_fwd(o, u, p.gamma, p.beta)
+    ye = O.out_proj_fwd(g, p.W2, p.b2, x32)
+    assert_close(y, ye, *BF16_TOL, what="Y fp32 residual")
+
+
+# ---------------------------------------------------------------------------------------------
+# failure paths (host-injected; no GPU fault)
+# ---------------------------------------------------------------------------------------------
+
+def test_timeout_probe_reports_timeout_status():
+    ws = workspace(256)
+    H.hstu_set_wait_limit(1 << 20)
+    try:
+        H.hstu_debug_timeout_probe(ws)
+        assert H.hstu_sync_status(ws) == 5
+        assert H.hstu_sync_status(ws) == 0     # read resets it
+    finally:
+        H.hstu_set_wait_limit(0)
+
+
+def test_offsets_violating_max_len_are_reported_not_read():
+    off = W.offsets_from_lengths([10, 300])
+    ts = np.zeros(310, np.int64)
+    Hh, d = 1, 64
+    q = np.zeros((310, 64), np.float32)
+    got, st = _run_attn(off, ts, q, q, q, np.zeros(15, np.float32), np.zeros(128, np.float32), Hh, d, 8, 1.0, True,
+                        max_len=100)
+    assert st == 6
+    assert np.all(np.isnan(got))           # nothing written
+
+
+def test_empty_sequences_only():
+    off = W.offsets_from_lengths([0, 0, 0])
+    got, st = _run_attn(off, np.zeros(0, np.int64), np.zeros((0, 64)), np.zeros((0, 64)), np.zeros((0, 64)),
+                        np.zeros(15, np.float32), np.zeros(128, np.float32), 1, 64, 8, 1.0, True, max_len=1)
+    assert st == 0 and got.shape == (0, 64)
