@@ -206,7 +206,7 @@ def main():
     x = to_dev(wl.x, torch.bfloat16, dev)
     y = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
     sv = SavedActs.empty(T, D, torch.bfloat16, keep_z=False, device=dev)
-    adesc = H.make_attn_desc(Hh, D // Hh, D // Hh, 1.0 / wl.N, wl.pos_max_len, H.HSTU_BF16, 4 * D, 4 * D, 4 * D, D)
+    adesc = H.make_attn_desc(Hh, D // Hh, D // Hh, 1.0 / wl.N, wl.pos_max_len, H.HSTU_F16, 4 * D, 4 * D, 4 * D, D)
     ws = workspace(H.hstu_attn_workspace_size(adesc, jag.struct), dev)
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     n_kernels = {"uvqk": 1, "attn": 2, "norm_gate": 1, "out_proj": 1}
@@ -214,14 +214,14 @@ def main():
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        H.hstu_uvqk_fwd(T, D, H.HSTU_BF16, x, D, layer.W1, layer.b1, sv.uvqk, None, ws)
+        H.hstu_uvqk_fwd(T, D, H.HSTU_BF16, H.HSTU_F16, x, D, layer.W1, layer.b1, sv.uvqk, None, ws)
         if ev:
             ev[1].record(stream)
         H.hstu_attn_fwd(adesc, jag.struct, sv.uvqk[:, 2 * D:], sv.uvqk[:, 3 * D:], sv.uvqk[:, D:], layer.rab_pos,
                         layer.rab_time, sv.o, ws)
         if ev:
             ev[2].record(stream)
-        H.hstu_norm_gate_fwd(T, D, H.HSTU_BF16, sv.o, D, sv.uvqk, 4 * D, layer.gamma, layer.beta, 1e-5, sv.g, sv.mu,
+        H.hstu_norm_gate_fwd(T, D, H.HSTU_F32, H.HSTU_F16, H.HSTU_BF16, sv.o, D, sv.uvqk, 4 * D, layer.gamma, layer.beta, 1e-5, sv.g, sv.mu,
                              sv.rstd)
         if ev:
             ev[3].record(stream)

@@ -6,7 +6,7 @@
 // pointwise-aggregation bullet; "HSTU: The First Exploration of the Scaling Law", 7.1.4
 // Innovation 1 (SiLU, no softmax, no 1/sqrt(d) scale) and Innovation 2 (position and time bias).)
 //
-// bf16 tensor-core kernel, one CTA per (sequence, 128-row query tile, head) from the jagged work
+// Tensor-core kernel (bf16 or fp16 operands, fp32 accumulation), one CTA per (sequence, 128-row query tile, head) from the jagged work
 // list (longest causal rows first). Only key tiles 0..t of the query tile's own sequence are
 // visited (causal tile skipping; padding never exists in the jagged layout).
 //   warp 4  : TMA producer (Q once, K/V double-buffered, 128-byte swizzle)
@@ -49,6 +49,7 @@ __device__ __forceinline__ int pos_index(long long r, int L) {
   return static_cast<int>(r) + L - 1;
 }
 
+template <bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, AttnArgs a, WaitCtl ctl) {
@@ -142,8 +143,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   } else if (warp == 5) {
     // ---------------- tcgen05 issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, 0, 0);
-      constexpr uint32_t idesc_pv = make_idesc_bf16(128, 64, 0, 1);
+      constexpr uint32_t idesc_qk = make_idesc_f16kind(128, 128, 0, 0, F16);
+      constexpr uint32_t idesc_pv = make_idesc_f16kind(128, 64, 0, 1, F16);
       bool ok = mbar_wait(bar_q, 0, abort_flag, ctl);
       auto issue_pv = [&](int t) -> bool {
         const int s = t & 1;
@@ -225,7 +226,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const float x = __uint_as_float(sv[j + e]) + pw[-col] + s_rab_time[bkt];
             y[e] = (!diag || col <= r) ? silu_fast(x) : 0.0f;
           }
-          pk[j / 2] = pack_bf16x2(y[0], y[1]);
+          pk[j / 2] = F16 ? pack_f16x2(y[0], y[1]) : pack_bf16x2(y[0], y[1]);
         }
         uint8_t* chunk = prow + (c >> 1) * 16384;
 #pragma unroll
@@ -248,20 +249,31 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tmem_ld_wait();
       if (qi < n) {
         const float sc = a.inv_N;
-        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) +
-                                              (seq0 + qi) * a.ld_o + h * kD);
+        if (a.o_f32) {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + (seq0 + qi) * a.ld_o + h * kD);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          dst[q] = make_uint4(pack_bf16x2(__uint_as_float(o0[8 * q]) * sc, __uint_as_float(o0[8 * q + 1]) * sc),
-                              pack_bf16x2(__uint_as_float(o0[8 * q + 2]) * sc, __uint_as_float(o0[8 * q + 3]) * sc),
-                              pack_bf16x2(__uint_as_float(o0[8 * q + 4]) * sc, __uint_as_float(o0[8 * q + 5]) * sc),
-                              pack_bf16x2(__uint_as_float(o0[8 * q + 6]) * sc, __uint_as_float(o0[8 * q + 7]) * sc));
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(o0[4 * q]) * sc, __uint_as_float(o0[4 * q + 1]) * sc,
+                                 __uint_as_float(o0[4 * q + 2]) * sc, __uint_as_float(o0[4 * q + 3]) * sc);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          dst[4 + q] = make_uint4(pack_bf16x2(__uint_as_float(o1[8 * q]) * sc, __uint_as_float(o1[8 * q + 1]) * sc),
-                                  pack_bf16x2(__uint_as_float(o1[8 * q + 2]) * sc, __uint_as_float(o1[8 * q + 3]) * sc),
-                                  pack_bf16x2(__uint_as_float(o1[8 * q + 4]) * sc, __uint_as_float(o1[8 * q + 5]) * sc),
-                                  pack_bf16x2(__uint_as_float(o1[8 * q + 6]) * sc, __uint_as_float(o1[8 * q + 7]) * sc));
+          for (int q = 0; q < 8; ++q)
+            dst[8 + q] = make_float4(__uint_as_float(o1[4 * q]) * sc, __uint_as_float(o1[4 * q + 1]) * sc,
+                                     __uint_as_float(o1[4 * q + 2]) * sc, __uint_as_float(o1[4 * q + 3]) * sc);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + (seq0 + qi) * a.ld_o + h * kD);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16x2(__uint_as_float(o0[8 * q]) * sc, __uint_as_float(o0[8 * q + 1]) * sc),
+                                pack_bf16x2(__uint_as_float(o0[8 * q + 2]) * sc, __uint_as_float(o0[8 * q + 3]) * sc),
+                                pack_bf16x2(__uint_as_float(o0[8 * q + 4]) * sc, __uint_as_float(o0[8 * q + 5]) * sc),
+                                pack_bf16x2(__uint_as_float(o0[8 * q + 6]) * sc, __uint_as_float(o0[8 * q + 7]) * sc));
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[4 + q] = make_uint4(pack_bf16x2(__uint_as_float(o1[8 * q]) * sc, __uint_as_float(o1[8 * q + 1]) * sc),
+                                    pack_bf16x2(__uint_as_float(o1[8 * q + 2]) * sc, __uint_as_float(o1[8 * q + 3]) * sc),
+                                    pack_bf16x2(__uint_as_float(o1[8 * q + 4]) * sc, __uint_as_float(o1[8 * q + 5]) * sc),
+                                    pack_bf16x2(__uint_as_float(o1[8 * q + 6]) * sc, __uint_as_float(o1[8 * q + 7]) * sc));
+        }
       }
     }
   }
@@ -321,14 +333,16 @@ cudaError_t attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   CUtensorMap tq, tk, tv;
-  if (!encode_tmap_2d_bf16(&tq, a.q, static_cast<int64_t>(a.H) * kD, a.T, a.ld_q, 64, 128) ||
-      !encode_tmap_2d_bf16(&tk, a.k, static_cast<int64_t>(a.H) * kD, a.T, a.ld_k, 64, 128) ||
-      !encode_tmap_2d_bf16(&tv, a.v, static_cast<int64_t>(a.H) * kD, a.T, a.ld_v, 64, 128))
+  const bool f16 = a.in_f16 != 0;
+  if (!encode_tmap_2d_bf16(&tq, a.q, static_cast<int64_t>(a.H) * kD, a.T, a.ld_q, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tk, a.k, static_cast<int64_t>(a.H) * kD, a.T, a.ld_k, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tv, a.v, static_cast<int64_t>(a.H) * kD, a.T, a.ld_v, 64, 128, f16))
     return cudaErrorInvalidValue;
-  e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::kTotal);
+  auto kern = f16 ? attn_fwd_tc_kernel<true> : attn_fwd_tc_kernel<false>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::kTotal);
   if (e != cudaSuccess) return e;
   const long long blocks = a.capacity * a.H;
-  attn_fwd_tc_kernel<<<static_cast<unsigned>(blocks), kThreads, AttnSmem::kTotal, st>>>(tq, tk, tv, a, wait_ctl(a.status));
+  kern<<<static_cast<unsigned>(blocks), kThreads, AttnSmem::kTotal, st>>>(tq, tk, tv, a, wait_ctl(a.status));
   return cudaGetLastError();
 }
 

@@ -12,6 +12,7 @@
 // and the split into U, V, Q, K; f2 followed by the residual of the "Code" sketch.)
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -36,22 +37,30 @@ struct GemmSmem {
   static constexpr int kTotal = kTileBytes + 256 + 1024;   // barriers + alignment slack
 };
 
-__device__ __forceinline__ void store_row32(void* out, int is_f32, const float* v) {
-  if (is_f32) {
+__host__ __device__ __forceinline__ int dt_size(int dt) { return dt == kDtF32 ? 4 : 2; }
+
+// 32 consecutive values of one row, stored as fp32, bf16 or fp16 (16-byte vector stores).
+__device__ __forceinline__ void store_row32(void* out, int dt, const float* v) {
+  if (dt == kDtF32) {
     float4* o = reinterpret_cast<float4*>(out);
 #pragma unroll
     for (int q = 0; q < 8; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
   } else {
     uint4* o = reinterpret_cast<uint4*>(out);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      o[q] = make_uint4(pack_bf16x2(v[8 * q + 0], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                        pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+    for (int q = 0; q < 4; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        w[e] = dt == kDtBF16 ? pack_bf16x2(v[8 * q + 2 * e], v[8 * q + 2 * e + 1])
+                             : pack_f16x2(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]);
+      o[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
 }
 
-__device__ __forceinline__ void load_row32(const void* in, int is_f32, float* v) {
-  if (is_f32) {
+__device__ __forceinline__ void load_row32(const void* in, int dt, float* v) {
+  if (dt == kDtF32) {
     const float4* p = reinterpret_cast<const float4*>(in);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -66,17 +75,30 @@ __device__ __forceinline__ void load_row32(const void* in, int is_f32, float* v)
       const uint32_t w[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        v[8 * q + 2 * e] = __uint_as_float(w[e] << 16);
-        v[8 * q + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+        const float2 f = dt == kDtBF16 ? unpack_bf16x2(w[e]) : unpack_f16x2(w[e]);
+        v[8 * q + 2 * e] = f.x;
+        v[8 * q + 2 * e + 1] = f.y;
       }
     }
   }
 }
 
+__device__ __forceinline__ void store_one(void* base, int dt, int64_t idx, float v) {
+  if (dt == kDtF32) reinterpret_cast<float*>(base)[idx] = v;
+  else if (dt == kDtBF16) reinterpret_cast<__nv_bfloat16*>(base)[idx] = __float2bfloat16_rn(v);
+  else reinterpret_cast<__half*>(base)[idx] = __float2half_rn(v);
+}
+
+__device__ __forceinline__ float load_one(const void* base, int dt, int64_t idx) {
+  if (dt == kDtF32) return reinterpret_cast<const float*>(base)[idx];
+  if (dt == kDtBF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx]);
+  return __half2float(reinterpret_cast<const __half*>(base)[idx]);
+}
+
 template <int BN, int STAGES, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    int M, int N, int num_kb, int kb_per_split, GemmEpilogue epi, WaitCtl ctl) {
+                    int M, int N, int num_kb, int kb_per_split, uint32_t idesc, GemmEpilogue epi, WaitCtl ctl) {
   using L = GemmSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -137,7 +159,6 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
   } else if (warp == 5) {
     if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc_bf16(kBM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
       bool ok = true;
       for (int i = 0; i < nkb; ++i) {
         const int s = i % STAGES;
@@ -193,26 +214,26 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (epi.kind == kEpiSilu) {
           if (epi.out1) {
             uint8_t* o1 = reinterpret_cast<uint8_t*>(epi.out1) +
-                          (static_cast<int64_t>(row) * epi.ld_out1 + n) * (epi.out1_f32 ? 4 : 2);
-            store_row32(o1, epi.out1_f32, v);
+                          (static_cast<int64_t>(row) * epi.ld_out1 + n) * dt_size(epi.out1_dt);
+            store_row32(o1, epi.out1_dt, v);
           }
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = silu_fast(v[j]);
         } else if (epi.resid) {
           float rv[32];
           const uint8_t* rp = reinterpret_cast<const uint8_t*>(epi.resid) +
-                              (static_cast<int64_t>(row) * epi.ld_resid + n) * (epi.resid_f32 ? 4 : 2);
-          load_row32(rp, epi.resid_f32, rv);
+                              (static_cast<int64_t>(row) * epi.ld_resid + n) * dt_size(epi.resid_dt);
+          load_row32(rp, epi.resid_dt, rv);
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] += rv[j];
         }
         uint8_t* o0 = reinterpret_cast<uint8_t*>(epi.out0) +
-                      (static_cast<int64_t>(row) * epi.ld_out0 + n) * (epi.out0_f32 ? 4 : 2);
-        store_row32(o0, epi.out0_f32, v);
+                      (static_cast<int64_t>(row) * epi.ld_out0 + n) * dt_size(epi.out0_dt);
+        store_row32(o0, epi.out0_dt, v);
         if (epi.kind == kEpiLinear && epi.out1) {
           uint8_t* o1 = reinterpret_cast<uint8_t*>(epi.out1) +
-                        (static_cast<int64_t>(row) * epi.ld_out1 + n) * (epi.out1_f32 ? 4 : 2);
-          store_row32(o1, epi.out1_f32, v);
+                        (static_cast<int64_t>(row) * epi.ld_out1 + n) * dt_size(epi.out1_dt);
+          store_row32(o1, epi.out1_dt, v);
         }
       }
     }
@@ -276,18 +297,14 @@ gemm_f32_simt_kernel(const float* __restrict__ A, int64_t sam, int64_t sak, cons
       }
       if (epi.bias) v += epi.bias[n];
       if (epi.kind == kEpiSilu) {
-        if (epi.out1) reinterpret_cast<float*>(epi.out1)[m * epi.ld_out1 + n] = v;
+        if (epi.out1) store_one(epi.out1, epi.out1_dt, static_cast<int64_t>(m) * epi.ld_out1 + n, v);
         v = v / (1.0f + expf(-v));
       } else if (epi.resid) {
-        v += epi.resid_f32 ? reinterpret_cast<const float*>(epi.resid)[m * epi.ld_resid + n]
-                           : bf16_bits_to_float(reinterpret_cast<const uint16_t*>(epi.resid)[m * epi.ld_resid + n]);
+        v += load_one(epi.resid, epi.resid_dt, static_cast<int64_t>(m) * epi.ld_resid + n);
       }
-      if (epi.out0_f32) reinterpret_cast<float*>(epi.out0)[m * epi.ld_out0 + n] = v;
-      else reinterpret_cast<__nv_bfloat16*>(epi.out0)[m * epi.ld_out0 + n] = __float2bfloat16_rn(v);
-      if (epi.kind == kEpiLinear && epi.out1) {
-        if (epi.out1_f32) reinterpret_cast<float*>(epi.out1)[m * epi.ld_out1 + n] = v;
-        else reinterpret_cast<__nv_bfloat16*>(epi.out1)[m * epi.ld_out1 + n] = __float2bfloat16_rn(v);
-      }
+      store_one(epi.out0, epi.out0_dt, static_cast<int64_t>(m) * epi.ld_out0 + n, v);
+      if (epi.kind == kEpiLinear && epi.out1)
+        store_one(epi.out1, epi.out1_dt, static_cast<int64_t>(m) * epi.ld_out1 + n, v);
     }
   }
 }
@@ -298,14 +315,14 @@ cudaError_t launch_tc(const GemmArgs& g, cudaStream_t st) {
   CUtensorMap tmA, tmB;
   // A: K-major -> [M rows, K] box {64, 128}; MN-major -> [K rows, M] box {64, 64}
   if (!A_MN) {
-    if (!encode_tmap_2d_bf16(&tmA, g.A, g.K, g.M, g.lda, 64, kBM)) return cudaErrorInvalidValue;
+    if (!encode_tmap_2d_bf16(&tmA, g.A, g.K, g.M, g.lda, 64, kBM, g.f16)) return cudaErrorInvalidValue;
   } else {
-    if (!encode_tmap_2d_bf16(&tmA, g.A, g.M, g.K, g.lda, 64, 64)) return cudaErrorInvalidValue;
+    if (!encode_tmap_2d_bf16(&tmA, g.A, g.M, g.K, g.lda, 64, 64, g.f16)) return cudaErrorInvalidValue;
   }
   if (!B_MN) {
-    if (!encode_tmap_2d_bf16(&tmB, g.B, g.K, g.N, g.ldb, 64, BN)) return cudaErrorInvalidValue;
+    if (!encode_tmap_2d_bf16(&tmB, g.B, g.K, g.N, g.ldb, 64, BN, g.f16)) return cudaErrorInvalidValue;
   } else {
-    if (!encode_tmap_2d_bf16(&tmB, g.B, g.N, g.K, g.ldb, 64, 64)) return cudaErrorInvalidValue;
+    if (!encode_tmap_2d_bf16(&tmB, g.B, g.N, g.K, g.ldb, 64, 64, g.f16)) return cudaErrorInvalidValue;
   }
   auto kern = gemm_bf16_tc_kernel<BN, STAGES, A_MN, B_MN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
@@ -316,8 +333,9 @@ cudaError_t launch_tc(const GemmArgs& g, cudaStream_t st) {
   const int zdim = (num_kb + kb_per - 1) / kb_per;
   dim3 grid(static_cast<unsigned>((g.N + BN - 1) / BN), static_cast<unsigned>((g.M + kBM - 1) / kBM),
             static_cast<unsigned>(zdim < 1 ? 1 : zdim));
+  const uint32_t idesc = make_idesc_f16kind(kBM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0, g.f16);
   kern<<<grid, kThreads, L::kTotal, st>>>(tmA, tmB, static_cast<int>(g.M), static_cast<int>(g.N), num_kb,
-                                          kb_per, g.epi, wait_ctl(g.status));
+                                          kb_per, idesc, g.epi, wait_ctl(g.status));
   return cudaGetLastError();
 }
 

@@ -56,17 +56,20 @@ hstu_status_t check_jagged(const hstu_jagged_t* j) {
   return HSTU_OK;
 }
 
+bool is_tc_dtype(int dt) { return dt == HSTU_BF16 || dt == HSTU_F16; }
+
 hstu_status_t check_attn(const hstu_attn_desc_t* d, const hstu_jagged_t* j) {
   hstu_status_t s = check_jagged(j);
   if (s != HSTU_OK) return s;
   if (!d || d->H <= 0 || d->d_qk <= 0 || d->d_v <= 0 || d->pos_max_len <= 0) return HSTU_ERR_INVALID_ARG;
   if (d->n_time_buckets < 1 || d->n_time_buckets > 128) return HSTU_ERR_UNSUPPORTED;
   if (!isfinite(d->inv_N)) return HSTU_ERR_INVALID_ARG;
-  if (d->dtype == HSTU_BF16) {
+  if (d->o_dtype != HSTU_F32 && d->o_dtype != HSTU_BF16) return HSTU_ERR_UNSUPPORTED;
+  if (is_tc_dtype(d->dtype)) {
     if (d->d_qk != 64 || d->d_v != 64) return HSTU_ERR_UNSUPPORTED;
     if (d->ld_q % 8 || d->ld_k % 8 || d->ld_v % 8 || d->ld_o % 8) return HSTU_ERR_UNSUPPORTED;
   } else if (d->dtype == HSTU_F32) {
-    if (d->d_qk > 64 || d->d_v > 64) return HSTU_ERR_UNSUPPORTED;
+    if (d->d_qk > 64 || d->d_v > 64 || d->o_dtype != HSTU_F32) return HSTU_ERR_UNSUPPORTED;
   } else {
     return HSTU_ERR_UNSUPPORTED;
   }
@@ -87,25 +90,28 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
   a.B = j->B; a.T = j->T; a.max_len = j->max_len; a.offsets = j->offsets; a.ts = j->timestamps;
   a.H = d->H; a.dqk = d->d_qk; a.dv = d->d_v; a.inv_N = d->inv_N; a.pos_max_len = d->pos_max_len;
   a.n_buckets = d->n_time_buckets;
-  a.q = q; a.ld_q = d->ld_q; a.k = k; a.ld_k = d->ld_k; a.v = v; a.ld_v = d->ld_v; a.o = out; a.ld_o = d->ld_o;
+  a.q = q; a.ld_q = d->ld_q; a.k = k; a.ld_k = d->ld_k; a.v = v; a.ld_v = d->ld_v;
+  a.o = out; a.ld_o = d->ld_o; a.o_f32 = d->o_dtype == HSTU_F32;
+  a.in_f16 = d->dtype == HSTU_F16;
   a.rab_pos = rab_pos; a.rab_time = rab_time; a.items = items; a.count = count; a.capacity = cap;
   a.status = ws_status(ws);
   cudaError_t e = launch_worklist(j->offsets, j->B, j->T, j->max_len, items, count, a.status, st);
   if (e != cudaSuccess) return cuda_status(e);
   if (j->T == 0) return HSTU_OK;
-  e = d->dtype == HSTU_BF16 ? attn_fwd_bf16_tc(a, st) : attn_fwd_f32_simt(a, st);
+  e = is_tc_dtype(d->dtype) ? attn_fwd_bf16_tc(a, st) : attn_fwd_f32_simt(a, st);
   return cuda_status(e);
 }
 
-hstu_status_t run_uvqk(int64_t T, int32_t D, hstu_dtype_t dtype, const void* x, int64_t ld_x, const void* W1,
-                       const float* b1, void* uvqk, void* z, int* status, cudaStream_t st) {
+// f1: operands x, W1 of `dtype` (BF16 tensor cores or F32 CUDA cores); uvqk / z of act_dtype.
+hstu_status_t run_uvqk(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t act_dtype, const void* x, int64_t ld_x,
+                       const void* W1, const float* b1, void* uvqk, void* z, int* status, cudaStream_t st) {
   GemmArgs g{};
   g.A = x; g.lda = ld_x; g.a_mn = false;
-  g.B = W1; g.ldb = D; g.b_mn = false;
+  g.B = W1; g.ldb = D; g.b_mn = false; g.f16 = false;
   g.M = T; g.N = 4ll * D; g.K = D; g.splits = 1;
   g.epi.kind = kEpiSilu; g.epi.bias = b1;
-  g.epi.out0 = uvqk; g.epi.out0_f32 = dtype == HSTU_F32; g.epi.ld_out0 = 4ll * D;
-  g.epi.out1 = z; g.epi.out1_f32 = dtype == HSTU_F32; g.epi.ld_out1 = 4ll * D;
+  g.epi.out0 = uvqk; g.epi.out0_dt = act_dtype; g.epi.ld_out0 = 4ll * D;
+  g.epi.out1 = z; g.epi.out1_dt = act_dtype; g.epi.ld_out1 = 4ll * D;
   g.status = status;
   return cuda_status(dtype == HSTU_BF16 ? gemm_bf16(g, st) : gemm_f32(g, st));
 }
@@ -115,12 +121,12 @@ hstu_status_t run_out_proj(int64_t T, int32_t D, hstu_dtype_t dtype, const void*
                            void* y_bf16, int* status, cudaStream_t st) {
   GemmArgs g{};
   g.A = g_in; g.lda = D; g.a_mn = false;
-  g.B = W2; g.ldb = D; g.b_mn = false;
+  g.B = W2; g.ldb = D; g.b_mn = false; g.f16 = false;
   g.M = T; g.N = D; g.K = D; g.splits = 1;
   g.epi.kind = kEpiLinear; g.epi.bias = b2;
-  g.epi.resid = x; g.epi.resid_f32 = x_dtype == HSTU_F32; g.epi.ld_resid = D;
-  g.epi.out0 = y; g.epi.out0_f32 = y_dtype == HSTU_F32; g.epi.ld_out0 = D;
-  g.epi.out1 = y_bf16; g.epi.out1_f32 = 0; g.epi.ld_out1 = D;
+  g.epi.resid = x; g.epi.resid_dt = x_dtype; g.epi.ld_resid = D;
+  g.epi.out0 = y; g.epi.out0_dt = y_dtype; g.epi.ld_out0 = D;
+  g.epi.out1 = y_bf16; g.epi.out1_dt = kDtBF16; g.epi.ld_out1 = D;
   g.status = status;
   return cuda_status(dtype == HSTU_BF16 ? gemm_bf16(g, st) : gemm_f32(g, st));
 }
@@ -138,14 +144,14 @@ hstu_status_t check_dense(int64_t T, int32_t D, hstu_dtype_t dtype) {
 WaitCtl wait_ctl(int* status) { return WaitCtl{status, g_wait_limit}; }
 
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld_elems,
-                         int box_inner, int box_outer) {
+                         int box_inner, int box_outer, bool f16) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn || !aligned16(base) || inner <= 0 || outer <= 0 || (ld_elems * 2) % 16) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_elems) * 2};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -216,17 +222,19 @@ hstu_status_t hstu_time_buckets(const hstu_jagged_t* jag, int32_t n_buckets, con
                                          stream));
 }
 
-hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* x, int64_t ld_x, const void* W1,
-                            const float* b1, void* uvqk, void* z, void* ws, size_t ws_bytes, hstu_stream_t stream) {
+hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t act_dtype, const void* x,
+                            int64_t ld_x, const void* W1, const float* b1, void* uvqk, void* z, void* ws,
+                            size_t ws_bytes, hstu_stream_t stream) {
   hstu_status_t s = check_dense(T, D, dtype);
   if (s != HSTU_OK) return s;
+  if (dtype == HSTU_F32 ? act_dtype != HSTU_F32 : !is_tc_dtype(act_dtype)) return HSTU_ERR_UNSUPPORTED;
   if (!ws) return HSTU_ERR_INVALID_ARG;
   if (ws_bytes < kWsHeader) return HSTU_ERR_WORKSPACE;
   if (T == 0) return HSTU_OK;
   if (!x || !W1 || !uvqk || ld_x < D) return HSTU_ERR_INVALID_ARG;
   if (dtype == HSTU_BF16 && (ld_x % 8 || !aligned16(x) || !aligned16(W1) || !aligned16(uvqk) || (z && !aligned16(z))))
     return HSTU_ERR_UNSUPPORTED;
-  return run_uvqk(T, D, dtype, x, ld_x, W1, b1, uvqk, z, ws_status(ws), stream);
+  return run_uvqk(T, D, dtype, act_dtype, x, ld_x, W1, b1, uvqk, z, ws_status(ws), stream);
 }
 
 size_t hstu_attn_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag) {
@@ -243,24 +251,28 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
   if (!ws) return HSTU_ERR_INVALID_ARG;
   if (ws_bytes < attn_ws_bytes(capacity_of(jag))) return HSTU_ERR_WORKSPACE;
   if (jag->T > 0 && (!q || !k || !v || !rab_pos || !rab_time || !out)) return HSTU_ERR_INVALID_ARG;
-  if (desc->dtype == HSTU_BF16 && jag->T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)))
+  if (is_tc_dtype(desc->dtype) && jag->T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)))
     return HSTU_ERR_UNSUPPORTED;
   return run_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, ws, stream);
 }
 
-hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* o, int64_t ld_o, const void* u,
-                                 int64_t ld_u, const float* gamma, const float* beta, float eps, void* g, float* mu,
-                                 float* rstd, hstu_stream_t stream) {
+hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t o_dtype, hstu_dtype_t u_dtype,
+                                 hstu_dtype_t g_dtype, const void* o, int64_t ld_o, const void* u, int64_t ld_u,
+                                 const float* gamma, const float* beta, float eps, void* g, float* mu, float* rstd,
+                                 hstu_stream_t stream) {
   if (T < 0) return HSTU_ERR_INVALID_ARG;
-  if (dtype != HSTU_BF16 && dtype != HSTU_F32) return HSTU_ERR_UNSUPPORTED;
+  const bool combo = (o_dtype == HSTU_F32 && u_dtype == HSTU_F32 && g_dtype == HSTU_F32) ||
+                     (o_dtype == HSTU_F32 && is_tc_dtype(u_dtype) && g_dtype == HSTU_BF16) ||
+                     (o_dtype == HSTU_BF16 && u_dtype == HSTU_BF16 && g_dtype == HSTU_BF16);
+  if (!combo) return HSTU_ERR_UNSUPPORTED;
   if (D != 64 && D != 128 && D != 256 && D != 512 && D != 1024) return HSTU_ERR_UNSUPPORTED;
   if (T == 0) return HSTU_OK;
   if (!o || !u || !gamma || !beta || !g || ld_o < D || ld_u < D) return HSTU_ERR_INVALID_ARG;
-  const int vec = dtype == HSTU_BF16 ? 8 : 4;
-  if (!aligned16(o) || !aligned16(u) || !aligned16(g) || !aligned16(gamma) || !aligned16(beta) || ld_o % vec ||
-      ld_u % vec)
+  if (!aligned16(o) || !aligned16(u) || !aligned16(g) || !aligned16(gamma) || !aligned16(beta) || ld_o % 8 ||
+      ld_u % 8)
     return HSTU_ERR_UNSUPPORTED;
-  return cuda_status(norm_gate_fwd(T, D, dtype == HSTU_BF16, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, stream));
+  return cuda_status(norm_gate_fwd(T, D, o_dtype, u_dtype, g_dtype, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd,
+                                   stream));
 }
 
 hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* g, const void* W2,
@@ -300,7 +312,7 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   if (s != HSTU_OK) return s;
   hstu_attn_desc_t ad{};
   ad.H = H; ad.d_qk = D / H; ad.d_v = D / H; ad.inv_N = desc->inv_N; ad.pos_max_len = desc->pos_max_len;
-  ad.n_time_buckets = desc->n_time_buckets; ad.dtype = desc->dtype;
+  ad.n_time_buckets = desc->n_time_buckets; ad.dtype = desc->dtype; ad.o_dtype = HSTU_F32;
   ad.ld_q = ad.ld_k = ad.ld_v = 4ll * D; ad.ld_o = D;
   s = check_attn(&ad, jag);
   if (s != HSTU_OK) return s;
@@ -326,14 +338,18 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
       x_op = conv;
     }
   }
-  s = run_uvqk(T, D, desc->dtype, x_op, D, w->W1, w->b1, saved->uvqk, saved->z, status, st);
+  // tensor-core mode keeps U|V|Q|K (and Z) in fp16: same MMA rate as bf16, 8x finer rounding of
+  // the attention operands, whose errors LayerNorm(O) would otherwise amplify
+  const hstu_dtype_t act = desc->dtype == HSTU_BF16 ? HSTU_F16 : HSTU_F32;
+  s = run_uvqk(T, D, desc->dtype, act, x_op, D, w->W1, w->b1, saved->uvqk, saved->z, status, st);
   if (s != HSTU_OK) return s;
-  const size_t es = desc->dtype == HSTU_BF16 ? 2 : 4;
+  ad.dtype = act;
+  const size_t es = act == HSTU_F32 ? 4 : 2;
   const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
   s = run_attn_fwd(&ad, jag, uvqk + 2 * D * es, uvqk + 3 * D * es, uvqk + 1 * D * es, w->rab_pos, w->rab_time,
                    saved->o, ws, st);
   if (s != HSTU_OK) return s;
-  cudaError_t e = norm_gate_fwd(T, D, desc->dtype == HSTU_BF16, saved->o, D, uvqk, 4ll * D, w->gamma, w->beta,
+  cudaError_t e = norm_gate_fwd(T, D, kDtF32, act, desc->dtype, saved->o, D, uvqk, 4ll * D, w->gamma, w->beta,
                                 desc->ln_eps, saved->g, saved->mu, saved->rstd, st);
   if (e != cudaSuccess) return cuda_status(e);
   return run_out_proj(T, D, desc->dtype, saved->g, w->W2, w->b2, x, desc->x_dtype, y, desc->y_dtype, y_bf16, status,

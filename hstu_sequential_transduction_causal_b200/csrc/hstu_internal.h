@@ -28,13 +28,13 @@ struct GemmEpilogue {
   int kind;
   const float* bias;      // [N] or null
   const void* resid;      // [M, N] or null (LINEAR)
-  int resid_f32;
+  int resid_dt;
   int64_t ld_resid;
   void* out0;             // SILU: SiLU(Z); LINEAR: Y; ATOMIC: fp32 accumulation target
-  int out0_f32;
+  int out0_dt;
   int64_t ld_out0;
   void* out1;             // SILU: Z; LINEAR: second copy of Y; or null
-  int out1_f32;
+  int out1_dt;
   int64_t ld_out1;
 };
 
@@ -45,14 +45,16 @@ struct GemmArgs {
   const void* B;   // K-major: [N, K] (ldb); MN-major: [K, N] (ldb)
   int64_t ldb;
   bool b_mn;
+  bool f16;        // A and B are fp16 (else bf16)
   int64_t M, N, K;
   int splits;      // split-K factor (ATOMIC epilogue only)
   GemmEpilogue epi;
   int* status;     // device status word
 };
 
+// 2D tensor map of a 2-byte element matrix (bf16, or fp16 when f16), 128-byte swizzle.
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t outer,
-                         int64_t ld_elems, int box_inner, int box_outer);
+                         int64_t ld_elems, int box_inner, int box_outer, bool f16 = false);
 
 cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st);
 cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
@@ -82,7 +84,8 @@ struct AttnArgs {
   const void* q; int64_t ld_q;
   const void* k; int64_t ld_k;
   const void* v; int64_t ld_v;
-  void* o; int64_t ld_o;
+  void* o; int64_t ld_o; int o_f32;
+  int in_f16;              // q, k, v are fp16 (else bf16) on the tensor-core path
   const float* rab_pos;
   const float* rab_time;
   const int32_t* items;    // work list (b, tile)
@@ -97,9 +100,10 @@ cudaError_t attn_fwd_f32_simt(const AttnArgs& a, cudaStream_t st);
 // ---------------------------------------------------------------------------------------------
 // LayerNorm (.) U
 // ---------------------------------------------------------------------------------------------
-cudaError_t norm_gate_fwd(int64_t T, int D, bool bf16, const void* o, int64_t ld_o, const void* u,
-                          int64_t ld_u, const float* gamma, const float* beta, float eps, void* g,
-                          float* mu, float* rstd, cudaStream_t st);
+// o_dt: f32 or bf16; u_dt: any; g_dt: any (kDt* codes). g has row stride D.
+cudaError_t norm_gate_fwd(int64_t T, int D, int o_dt, int u_dt, int g_dt, const void* o, int64_t ld_o,
+                          const void* u, int64_t ld_u, const float* gamma, const float* beta,
+                          float eps, void* g, float* mu, float* rstd, cudaStream_t st);
 
 cudaError_t convert_f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t st);
 

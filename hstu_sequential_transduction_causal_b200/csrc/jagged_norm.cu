@@ -8,6 +8,7 @@
 #include "hstu_internal.h"
 #include "sm100_ptx.cuh"
 #include "time_bucket_dev.cuh"
+#include "vec_io.cuh"
 
 namespace hstu {
 
@@ -105,62 +106,7 @@ time_bucket_kernel(const int64_t* __restrict__ off, const int64_t* __restrict__ 
 // one warp per token, lane l holds features [l*VPT, (l+1)*VPT); mean and variance by warp
 // shuffles (two passes over registers), fp32 statistics stored for the backward.
 // ----------------------------------------------------------------------------------------------
-template <int VPT, bool BF16>
-__device__ __forceinline__ void load_vec(const void* base, int64_t idx, float* v) {
-  if constexpr (BF16) {
-    const uint16_t* p = reinterpret_cast<const uint16_t*>(base) + idx;
-    if constexpr (VPT % 8 == 0) {
-#pragma unroll
-      for (int q = 0; q < VPT / 8; ++q) {
-        const uint4 t = reinterpret_cast<const uint4*>(p)[q];
-        const uint32_t w[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[8 * q + 2 * e] = __uint_as_float(w[e] << 16);
-          v[8 * q + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < VPT; ++e) v[e] = bf16_bits_to_float(p[e]);
-    }
-  } else {
-    const float* p = reinterpret_cast<const float*>(base) + idx;
-    if constexpr (VPT % 4 == 0) {
-#pragma unroll
-      for (int q = 0; q < VPT / 4; ++q) {
-        const float4 t = reinterpret_cast<const float4*>(p)[q];
-        v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < VPT; ++e) v[e] = p[e];
-    }
-  }
-}
-
-template <int VPT, bool BF16>
-__device__ __forceinline__ void store_vec(void* base, int64_t idx, const float* v) {
-  if constexpr (BF16) {
-    uint16_t* p = reinterpret_cast<uint16_t*>(base) + idx;
-    if constexpr (VPT % 8 == 0) {
-#pragma unroll
-      for (int q = 0; q < VPT / 8; ++q)
-        reinterpret_cast<uint4*>(p)[q] =
-            make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-    } else {
-#pragma unroll
-      for (int e = 0; e < VPT; e += 2) reinterpret_cast<uint32_t*>(p)[e / 2] = pack_bf16x2(v[e], v[e + 1]);
-    }
-  } else {
-    float* p = reinterpret_cast<float*>(base) + idx;
-#pragma unroll
-    for (int e = 0; e < VPT; ++e) p[e] = v[e];
-  }
-}
-
-template <int VPT, bool BF16>
+template <int VPT, int OT, int UT, int GT>
 __global__ void __launch_bounds__(256)
 norm_gate_kernel(int64_t T, const void* __restrict__ o, int64_t ld_o, const void* __restrict__ u,
                  int64_t ld_u, const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
@@ -170,8 +116,8 @@ norm_gate_kernel(int64_t T, const void* __restrict__ o, int64_t ld_o, const void
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= T) return;
   float x[VPT], uu[VPT];
-  load_vec<VPT, BF16>(o, row * ld_o + lane * VPT, x);
-  load_vec<VPT, BF16>(u, row * ld_u + lane * VPT, uu);
+  load_vec<VPT, OT>(o, row * ld_o + lane * VPT, x);
+  load_vec<VPT, UT>(u, row * ld_u + lane * VPT, uu);
   float s = 0.0f;
 #pragma unroll
   for (int e = 0; e < VPT; ++e) s += x[e];
@@ -188,11 +134,11 @@ norm_gate_kernel(int64_t T, const void* __restrict__ o, int64_t ld_o, const void
   for (int m = 16; m > 0; m >>= 1) q += __shfl_xor_sync(0xffffffffu, q, m);
   const float rstd = rsqrtf(q * (1.0f / D) + eps);
   float gm[VPT], bt[VPT];
-  load_vec<VPT, false>(gamma, lane * VPT, gm);
-  load_vec<VPT, false>(beta, lane * VPT, bt);
+  load_vec<VPT, kDtF32>(gamma, lane * VPT, gm);
+  load_vec<VPT, kDtF32>(beta, lane * VPT, bt);
 #pragma unroll
   for (int e = 0; e < VPT; ++e) x[e] = fmaf((x[e] - mean) * rstd, gm[e], bt[e]) * uu[e];
-  store_vec<VPT, BF16>(g, row * D + lane * VPT, x);
+  store_vec<VPT, GT>(g, row * D + lane * VPT, x);
   if (lane == 0) {
     if (mu_out) mu_out[row] = mean;
     if (rstd_out) rstd_out[row] = rstd;
@@ -226,11 +172,11 @@ __global__ void timeout_probe_kernel(WaitCtl ctl) {
   __syncthreads();
 }
 
-template <int VPT, bool BF16>
+template <int VPT, int OT, int UT, int GT>
 cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int64_t ld_u, const float* gamma,
                       const float* beta, float eps, void* g, float* mu, float* rstd, cudaStream_t st) {
   const int64_t blocks = (T + 7) / 8;
-  norm_gate_kernel<VPT, BF16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(T, o, ld_o, u, ld_u, gamma, beta, eps,
+  norm_gate_kernel<VPT, OT, UT, GT><<<static_cast<unsigned>(blocks), 256, 0, st>>>(T, o, ld_o, u, ld_u, gamma, beta, eps,
                                                                              g, mu, rstd);
   return cudaGetLastError();
 }
@@ -253,13 +199,22 @@ cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B
   return cudaGetLastError();
 }
 
-cudaError_t norm_gate_fwd(int64_t T, int D, bool bf16, const void* o, int64_t ld_o, const void* u, int64_t ld_u,
-                          const float* gamma, const float* beta, float eps, void* g, float* mu, float* rstd,
-                          cudaStream_t st) {
+cudaError_t norm_gate_fwd(int64_t T, int D, int o_dt, int u_dt, int g_dt, const void* o, int64_t ld_o, const void* u,
+                          int64_t ld_u, const float* gamma, const float* beta, float eps, void* g, float* mu,
+                          float* rstd, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-#define HSTU_NG(VPT)                                                                                   \
-  return bf16 ? launch_ng<VPT, true>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st)           \
-              : launch_ng<VPT, false>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st)
+  // supported (o, u, g) combinations: exact fp32; fp32 O with fp16 or bf16 U and bf16 G (tensor-core
+  // layer); all bf16.
+#define HSTU_NG(VPT)                                                                                     \
+  if (o_dt == kDtF32 && u_dt == kDtF32 && g_dt == kDtF32)                                               \
+    return launch_ng<VPT, kDtF32, kDtF32, kDtF32>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+  if (o_dt == kDtF32 && u_dt == kDtF16 && g_dt == kDtBF16)                                              \
+    return launch_ng<VPT, kDtF32, kDtF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+  if (o_dt == kDtF32 && u_dt == kDtBF16 && g_dt == kDtBF16)                                             \
+    return launch_ng<VPT, kDtF32, kDtBF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+  if (o_dt == kDtBF16 && u_dt == kDtBF16 && g_dt == kDtBF16)                                            \
+    return launch_ng<VPT, kDtBF16, kDtBF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+  return cudaErrorInvalidValue
   switch (D) {
     case 64: HSTU_NG(2);
     case 128: HSTU_NG(4);

@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace hstu {
@@ -153,8 +154,18 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
       : "memory");
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
-// a_mn / b_mn: operand is MN-major (1) or K-major (0).
+// Instruction descriptor for kind::f16 with fp32 D; A and B are both bf16 (f16 = false) or both
+// fp16 (f16 = true). a_mn / b_mn: operand is MN-major (1) or K-major (0).
+__host__ __device__ constexpr uint32_t make_idesc_f16kind(int M, int N, int a_mn, int b_mn, bool f16) {
+  return (1u << 4)                                  // D format: f32
+         | ((f16 ? 0u : 1u) << 7)                   // A format: f16 (0) / bf16 (1)
+         | ((f16 ? 0u : 1u) << 10)                  // B format: same as A
+         | (static_cast<uint32_t>(a_mn) << 15)      // A major
+         | (static_cast<uint32_t>(b_mn) << 16)      // B major
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
+}
+
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn, int b_mn) {
   return (1u << 4)                                  // D format: f32
          | (1u << 7)                                // A format: bf16
@@ -202,9 +213,26 @@ __device__ __forceinline__ void tmem_ld_wait() {
 // small numeric helpers
 // ------------------------------------------------------------------------------------------------
 
+// element types of activations and operands (same codes as hstu_dtype_t)
+enum : int { kDtF32 = 0, kDtBF16 = 1, kDtF16 = 2 };
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ float2 unpack_f16x2(uint32_t w) {
+  __half2 h = *reinterpret_cast<__half2*>(&w);
+  return __half22float2(h);
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {

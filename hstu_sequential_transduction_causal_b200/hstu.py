@@ -17,7 +17,7 @@ from .build import LIB as _LIB_PATH
 
 c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
-HSTU_F32, HSTU_BF16 = 0, 1
+HSTU_F32, HSTU_BF16, HSTU_F16 = 0, 1, 2
 STATUS = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED", 3: "HSTU_ERR_WORKSPACE",
           4: "HSTU_ERR_CUDA", 5: "HSTU_ERR_TIMEOUT", 6: "HSTU_ERR_DEVICE"}
 
@@ -37,7 +37,7 @@ class hstu_jagged_t(ctypes.Structure):
 
 class hstu_attn_desc_t(ctypes.Structure):
     _fields_ = [("H", c_i32), ("d_qk", c_i32), ("d_v", c_i32), ("inv_N", c_f32), ("pos_max_len", c_i32),
-                ("n_time_buckets", c_i32), ("dtype", c_i32), ("ld_q", c_i64), ("ld_k", c_i64),
+                ("n_time_buckets", c_i32), ("dtype", c_i32), ("o_dtype", c_i32), ("ld_q", c_i64), ("ld_k", c_i64),
                 ("ld_v", c_i64), ("ld_o", c_i64)]
 
 
@@ -71,12 +71,12 @@ SIGNATURES = {
     "hstu_worklist_capacity": (c_i64, [P(hstu_jagged_t)]),
     "hstu_jagged_worklist": (c_i32, [P(hstu_jagged_t), c_vp, c_vp, c_vp]),
     "hstu_time_buckets": (c_i32, [P(hstu_jagged_t), c_i32, c_vp, c_vp, c_vp]),
-    "hstu_uvqk_fwd": (c_i32, [c_i64, c_i32, c_i32, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "hstu_uvqk_fwd": (c_i32, [c_i64, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "hstu_attn_workspace_size": (c_sz, [P(hstu_attn_desc_t), P(hstu_jagged_t)]),
     "hstu_attn_fwd": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                               c_vp, c_sz, c_vp]),
-    "hstu_norm_gate_fwd": (c_i32, [c_i64, c_i32, c_i32, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_f32, c_vp,
-                                   c_vp, c_vp, c_vp]),
+    "hstu_norm_gate_fwd": (c_i32, [c_i64, c_i32, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp,
+                                   c_f32, c_vp, c_vp, c_vp, c_vp]),
     "hstu_out_proj_fwd": (c_i32, [c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_i32, c_vp,
                                   c_vp, c_sz, c_vp]),
     "hstu_layer_workspace_size": (c_sz, [P(hstu_layer_desc_t), P(hstu_jagged_t)]),
@@ -129,6 +129,8 @@ def _dtype_code(t: torch.Tensor) -> int:
         return HSTU_BF16
     if t.dtype == torch.float32:
         return HSTU_F32
+    if t.dtype == torch.float16:
+        return HSTU_F16
     raise ValueError(f"unsupported dtype {t.dtype}")
 
 
@@ -146,10 +148,10 @@ def make_jagged(offsets: torch.Tensor, timestamps: torch.Tensor, max_len: int) -
 
 
 def make_attn_desc(H, d_qk, d_v, inv_N, pos_max_len, dtype_code, ld_q, ld_k, ld_v, ld_o,
-                   n_time_buckets=128) -> hstu_attn_desc_t:
+                   n_time_buckets=128, o_dtype_code=HSTU_F32) -> hstu_attn_desc_t:
     return hstu_attn_desc_t(H=H, d_qk=d_qk, d_v=d_v, inv_N=inv_N, pos_max_len=pos_max_len,
-                            n_time_buckets=n_time_buckets, dtype=dtype_code, ld_q=ld_q, ld_k=ld_k,
-                            ld_v=ld_v, ld_o=ld_o)
+                            n_time_buckets=n_time_buckets, dtype=dtype_code, o_dtype=o_dtype_code, ld_q=ld_q,
+                            ld_k=ld_k, ld_v=ld_v, ld_o=ld_o)
 
 
 def make_layer_desc(D, H, inv_N, pos_max_len, dtype_code, x_dtype_code, y_dtype_code,
@@ -200,8 +202,9 @@ def hstu_time_buckets(jag: hstu_jagged_t, n_buckets: int, sq_offsets: torch.Tens
                                                         _ptr(out), _stream(stream)))
 
 
-def hstu_uvqk_fwd(T, D, dtype_code, x, ld_x, W1, b1, uvqk, z, ws, stream=None) -> None:
-    _check("hstu_uvqk_fwd", lib().hstu_uvqk_fwd(T, D, dtype_code, _ptr(x), ld_x, _ptr(W1), _ptr(b1), _ptr(uvqk),
+def hstu_uvqk_fwd(T, D, dtype_code, act_dtype_code, x, ld_x, W1, b1, uvqk, z, ws, stream=None) -> None:
+    _check("hstu_uvqk_fwd", lib().hstu_uvqk_fwd(T, D, dtype_code, act_dtype_code, _ptr(x), ld_x, _ptr(W1), _ptr(b1),
+                                                _ptr(uvqk),
                                                 _ptr(z), _ptr(ws), ws.numel() * ws.element_size(),
                                                 _stream(stream)))
 
@@ -216,8 +219,10 @@ def hstu_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, ws, stream=None) -
                                                 ws.numel() * ws.element_size(), _stream(stream)))
 
 
-def hstu_norm_gate_fwd(T, D, dtype_code, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, stream=None) -> None:
-    _check("hstu_norm_gate_fwd", lib().hstu_norm_gate_fwd(T, D, dtype_code, _ptr(o), ld_o, _ptr(u), ld_u,
+def hstu_norm_gate_fwd(T, D, o_dtype_code, u_dtype_code, g_dtype_code, o, ld_o, u, ld_u, gamma, beta, eps, g, mu,
+                       rstd, stream=None) -> None:
+    _check("hstu_norm_gate_fwd", lib().hstu_norm_gate_fwd(T, D, o_dtype_code, u_dtype_code, g_dtype_code, _ptr(o),
+                                                          ld_o, _ptr(u), ld_u,
                                                           _ptr(gamma), _ptr(beta), eps, _ptr(g), _ptr(mu),
                                                           _ptr(rstd), _stream(stream)))
 

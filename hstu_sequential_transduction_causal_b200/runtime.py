@@ -60,9 +60,11 @@ class SavedActs:
 
     @classmethod
     def empty(cls, T: int, D: int, dtype: torch.dtype, keep_z: bool, device="cuda") -> "SavedActs":
-        return cls(uvqk=torch.empty(T, 4 * D, dtype=dtype, device=device),
-                   z=torch.empty(T, 4 * D, dtype=dtype, device=device) if keep_z else None,
-                   o=torch.empty(T, D, dtype=dtype, device=device), g=torch.empty(T, D, dtype=dtype, device=device),
+        act = torch.float16 if dtype == torch.bfloat16 else dtype     # U|V|Q|K and Z in fp16
+        return cls(uvqk=torch.empty(T, 4 * D, dtype=act, device=device),
+                   z=torch.empty(T, 4 * D, dtype=act, device=device) if keep_z else None,
+                   o=torch.empty(T, D, dtype=torch.float32, device=device),
+                   g=torch.empty(T, D, dtype=dtype, device=device),
                    mu=torch.empty(T, dtype=torch.float32, device=device),
                    rstd=torch.empty(T, dtype=torch.float32, device=device))
 

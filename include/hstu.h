@@ -63,7 +63,7 @@ typedef enum hstu_status_t {
   HSTU_ERR_DEVICE = 6        /* a device-side check failed (reported on the device) */
 } hstu_status_t;
 
-typedef enum hstu_dtype_t { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype_t;
+typedef enum hstu_dtype_t { HSTU_F32 = 0, HSTU_BF16 = 1, HSTU_F16 = 2 } hstu_dtype_t;
 
 /* Jagged batch of B sequences, T tokens in total. */
 typedef struct hstu_jagged_t {
@@ -77,12 +77,13 @@ typedef struct hstu_jagged_t {
 /* Pointwise attention of one layer. */
 typedef struct hstu_attn_desc_t {
   int32_t H;               /* heads */
-  int32_t d_qk;            /* per-head query/key width (bf16: 64; f32: 1..64) */
-  int32_t d_v;             /* per-head value width (bf16: 64; f32: 1..64) */
+  int32_t d_qk;            /* per-head query/key width (bf16/f16: 64; f32: 1..64) */
+  int32_t d_v;             /* per-head value width (bf16/f16: 64; f32: 1..64) */
   float inv_N;             /* 1/N, the constant normaliser */
   int32_t pos_max_len;     /* L: rab_pos has 2L-1 entries */
   int32_t n_time_buckets;  /* 1..128 */
-  hstu_dtype_t dtype;      /* dtype of q, k, v, out */
+  hstu_dtype_t dtype;      /* dtype of q, k, v: BF16 or F16 (tensor cores) or F32 (CUDA cores) */
+  hstu_dtype_t o_dtype;    /* dtype of out: F32 (any dtype) or BF16 (BF16 inputs only) */
   int64_t ld_q, ld_k, ld_v, ld_o; /* row strides (elements); head h occupies columns [h*d, (h+1)*d) */
 } hstu_attn_desc_t;
 
@@ -94,7 +95,9 @@ typedef struct hstu_layer_desc_t {
   int32_t pos_max_len;
   int32_t n_time_buckets;
   float ln_eps;            /* LayerNorm epsilon (1e-5) */
-  hstu_dtype_t dtype;      /* compute dtype: BF16 (tensor cores, fp32 accumulate) or F32 */
+  hstu_dtype_t dtype;      /* BF16: bf16 X / W1 / W2 / G on the tensor cores with fp32 accumulation,
+                              U|V|Q|K, Z and the attention weights P in fp16, O in fp32;
+                              F32: every step in fp32 on the CUDA cores */
   hstu_dtype_t x_dtype;    /* dtype of X; F32 with BF16 compute = fp32 residual stream */
   hstu_dtype_t y_dtype;    /* dtype of Y */
 } hstu_layer_desc_t;
@@ -112,9 +115,12 @@ typedef struct hstu_layer_weights_t {
   const float* rab_time;
 } hstu_layer_weights_t;
 
-/* Activations a layer forward writes and its backward reads (compute dtype unless noted).
- * uvqk [T, 4D] = SiLU(Z); z [T, 4D] pre-activation (may be NULL when no backward follows);
- * o [T, D] attention output; g [T, D] = LN(O) (.) U; mu, rstd [T] fp32 LayerNorm statistics. */
+/* Activations a layer forward writes and its backward reads. In BF16 mode uvqk [T, 4D] = SiLU(Z)
+ * and z [T, 4D] (the pre-activation; may be NULL when no backward follows) are fp16 and g is
+ * bf16; in F32 mode all are fp32.
+ * o [T, D] attention output, always fp32 (LayerNorm divides by its spread across features,
+ * which is far smaller than its mean, so bf16 storage would be amplified); g [T, D] =
+ * LN(O) (.) U; mu, rstd [T] fp32 LayerNorm statistics. */
 typedef struct hstu_layer_saved_t {
   void* uvqk;
   void* z;
@@ -191,9 +197,10 @@ hstu_status_t hstu_time_buckets(const hstu_jagged_t* jag, int32_t n_buckets,
 
 /* f1 + SiLU + split ("Generative Recommenders and HSTU", first equation):
  * uvqk[t, :] = SiLU(x[t, :] W1^T + b1), [T, 4D] with row stride 4D; z (nullable) receives the
- * pre-activation. x, W1, uvqk, z have the compute dtype; ld_x is x's row stride. ws: any
- * workspace of at least 256 bytes (its status word receives device-side errors). */
-hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* x,
+ * pre-activation. x and W1 have `dtype` (BF16 or F32); uvqk and z have act_dtype (F16 or BF16
+ * for BF16 operands, F32 for F32); ld_x is x's row stride. ws: any workspace of at least 256
+ * bytes (its status word receives device-side errors). */
+hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t act_dtype, const void* x,
                             int64_t ld_x, const void* W1, const float* b1, void* uvqk, void* z,
                             void* ws, size_t ws_bytes, hstu_stream_t stream);
 
@@ -212,9 +219,12 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
 
 /* LayerNorm (.) U gating ("Generative Recommenders and HSTU", third equation; "HSTU: The First
  * Exploration of the Scaling Law", 7.1.4 Innovation 3): g = (gamma (o - mu) rstd + beta) (.) u
- * over all D features of a token; mu, rstd (fp32 [T]) are stored for the backward. */
-hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* o,
-                                 int64_t ld_o, const void* u, int64_t ld_u, const float* gamma,
+ * over all D features of a token; mu, rstd (fp32 [T]) are stored for the backward. g is [T, D]
+ * with row stride D. Supported (o, u, g) dtypes: (F32, F32, F32), (F32, F16 or BF16, BF16),
+ * (BF16, BF16, BF16). D in {64, 128, 256, 512, 1024}. */
+hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t o_dtype, hstu_dtype_t u_dtype,
+                                 hstu_dtype_t g_dtype, const void* o, int64_t ld_o, const void* u,
+                                 int64_t ld_u, const float* gamma,
                                  const float* beta, float eps, void* g, float* mu, float* rstd,
                                  hstu_stream_t stream);
 

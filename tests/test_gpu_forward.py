@@ -77,21 +77,22 @@ def test_time_buckets_bit_exact():
 # single steps
 # ---------------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_uvqk_fwd(dtype):
+@pytest.mark.parametrize("dtype,act", [("bf16", "f16"), ("bf16", "bf16"), ("f32", "f32")])
+def test_uvqk_fwd(dtype, act):
     rng = np.random.default_rng(1)
     T, D = (333, 256) if dtype == "bf16" else (437, 64)
     bf = dtype == "bf16"
     tdt = torch.bfloat16 if bf else torch.float32
+    adt = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}[act]
     cast = _bf16 if bf else (lambda a: np.asarray(a, np.float32))
     x = cast(rng.standard_normal((T, D)))
     W1 = cast(rng.standard_normal((4 * D, D)) / np.sqrt(D))
     b1 = (0.1 * rng.standard_normal(4 * D)).astype(np.float32)
-    uvqk = torch.empty(T, 4 * D, dtype=tdt, device="cuda")
-    z = torch.empty(T, 4 * D, dtype=tdt, device="cuda")
+    uvqk = torch.empty(T, 4 * D, dtype=adt, device="cuda")
+    z = torch.empty(T, 4 * D, dtype=adt, device="cuda")
     ws = workspace(256)
-    H.hstu_uvqk_fwd(T, D, H.HSTU_BF16 if bf else H.HSTU_F32, to_dev(x, tdt), D, to_dev(W1, tdt),
-                    to_dev(b1, torch.float32), uvqk, z, ws)
+    H.hstu_uvqk_fwd(T, D, H.HSTU_BF16 if bf else H.HSTU_F32, H._dtype_code(uvqk), to_dev(x, tdt), D,
+                    to_dev(W1, tdt), to_dev(b1, torch.float32), uvqk, z, ws)
     ze, se = O.uvqk_fwd(x, W1, b1)
     tol = BF16_TOL if bf else F32_TOL
     assert_close(z.float().cpu().numpy(), ze, *tol, what="Z")
@@ -99,14 +100,18 @@ def test_uvqk_fwd(dtype):
     assert H.hstu_sync_status(ws) == 0
 
 
-def _attn_case(lengths, Hh, d, L, inv_N, bf, seed=0, table_std=1.0, spread_ts=False):
+def _f16(a):
+    return np.asarray(a, np.float64).astype(np.float16).astype(np.float32)
+
+
+def _attn_case(lengths, Hh, d, L, inv_N, bf, seed=0, table_std=1.0, spread_ts=False, f16=False):
     rng = np.random.default_rng(seed)
     off = W.offsets_from_lengths(lengths)
     T = int(off[-1])
     ts = W.draw_timestamps(rng, lengths)
     if spread_ts:
         ts = ts + rng.integers(-10 ** 6, 10 ** 9, size=T)
-    cast = _bf16 if bf else (lambda a: np.asarray(a, np.float32))
+    cast = (_f16 if f16 else _bf16) if bf else (lambda a: np.asarray(a, np.float32))
     q = _silu_like(rng, (T, Hh * d)) if bf else rng.standard_normal((T, Hh * d)).astype(np.float32)
     k = _silu_like(rng, (T, Hh * d)) if bf else rng.standard_normal((T, Hh * d)).astype(np.float32)
     v = _silu_like(rng, (T, Hh * d)) if bf else rng.standard_normal((T, Hh * d)).astype(np.float32)
@@ -116,32 +121,36 @@ def _attn_case(lengths, Hh, d, L, inv_N, bf, seed=0, table_std=1.0, spread_ts=Fa
     return off, ts, q, k, v, rp, rt
 
 
-def _run_attn(off, ts, q, k, v, rp, rt, Hh, d, L, inv_N, bf, max_len=None):
-    tdt = torch.bfloat16 if bf else torch.float32
+def _run_attn(off, ts, q, k, v, rp, rt, Hh, d, L, inv_N, bf, max_len=None, out_bf16=False, f16=False):
+    tdt = (torch.float16 if f16 else torch.bfloat16) if bf else torch.float32
     jag = JaggedBatch(off, ts, max_len=max_len)
     T = jag.T
-    desc = H.make_attn_desc(Hh, d, d, inv_N, L, H.HSTU_BF16 if bf else H.HSTU_F32, Hh * d, Hh * d, Hh * d, Hh * d)
+    desc = H.make_attn_desc(Hh, d, d, inv_N, L, H._dtype_code(torch.empty(0, dtype=tdt)), Hh * d, Hh * d, Hh * d, Hh * d,
+                            o_dtype_code=H.HSTU_BF16 if out_bf16 else H.HSTU_F32)
     ws = workspace(H.hstu_attn_workspace_size(desc, jag.struct))
-    out = torch.full((T, Hh * d), float("nan"), dtype=tdt, device="cuda")
+    out = torch.full((T, Hh * d), float("nan"), dtype=torch.bfloat16 if out_bf16 else torch.float32,
+                     device="cuda")
     H.hstu_attn_fwd(desc, jag.struct, to_dev(q, tdt), to_dev(k, tdt), to_dev(v, tdt), to_dev(rp, torch.float32),
                     to_dev(rt, torch.float32), out, ws)
     st = H.hstu_sync_status(ws)
     return out.float().cpu().numpy(), st
 
 
-@pytest.mark.parametrize("spread", [False, True])
-def test_attn_fwd_bf16_ragged(spread):
+@pytest.mark.parametrize("spread,out_bf16,f16", [(False, False, True), (True, False, True), (False, True, False),
+                                                  (True, False, False)])
+def test_attn_fwd_tensor_core_ragged(spread, out_bf16, f16):
     lengths = [1, 127, 128, 129, 300, 0, 513, 64, 2]
     Hh, d, L = 2, 64, 600
     inv_N = 1.0 / 512
-    off, ts, q, k, v, rp, rt = _attn_case(lengths, Hh, d, L, inv_N, True, seed=2, spread_ts=spread)
-    got, st = _run_attn(off, ts, q, k, v, rp, rt, Hh, d, L, inv_N, True)
+    off, ts, q, k, v, rp, rt = _attn_case(lengths, Hh, d, L, inv_N, True, seed=2, spread_ts=spread, f16=f16)
+    got, st = _run_attn(off, ts, q, k, v, rp, rt, Hh, d, L, inv_N, True, out_bf16=out_bf16, f16=f16)
     assert st == 0
     T = int(off[-1])
     exp = O.pointwise_attention_fwd(q.reshape(T, Hh, d), k.reshape(T, Hh, d), v.reshape(T, Hh, d), off, ts, rp, rt,
                                     inv_N, L, THR).reshape(T, Hh * d)
     scale = float(np.sqrt(np.mean(exp ** 2)))
-    assert_close(got, exp, 1e-2 * scale, 1e-2, what="O bf16")
+    # the attention output alone: |d| <= 1e-2 rms(ref) + 1e-2 |ref| (16-bit operands, fp32 accumulate)
+    assert_close(got, exp, 1e-2 * scale, 1e-2, what="O")
 
 
 def test_attn_fwd_f32_single_layer_workload():
@@ -156,17 +165,22 @@ def test_attn_fwd_f32_single_layer_workload():
     assert_close(got, exp, *F32_TOL, what="O f32")
 
 
-def test_norm_gate_bf16():
+@pytest.mark.parametrize("o_bf16", [False, True])
+def test_norm_gate_bf16(o_bf16):
     rng = np.random.default_rng(4)
     T, D = 257, 512
-    o = _bf16(0.05 * rng.standard_normal((T, D)) + 0.02)
-    uvqk = _silu_like(rng, (T, 4 * D))
+    o = 0.05 * rng.standard_normal((T, D)) + 0.02
+    o = _bf16(o) if o_bf16 else o.astype(np.float32)
+    udt = torch.bfloat16 if o_bf16 else torch.float16
+    uvqk = _silu_like(rng, (T, 4 * D)) if o_bf16 else _f16(_silu_like(rng, (T, 4 * D)))
     gamma = (1 + 0.2 * rng.standard_normal(D)).astype(np.float32)
     beta = (0.2 * rng.standard_normal(D)).astype(np.float32)
     g = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
     mu = torch.empty(T, dtype=torch.float32, device="cuda")
     rstd = torch.empty(T, dtype=torch.float32, device="cuda")
-    H.hstu_norm_gate_fwd(T, D, H.HSTU_BF16, to_dev(o, torch.bfloat16), D, to_dev(uvqk, torch.bfloat16), 4 * D,
+    H.hstu_norm_gate_fwd(T, D, H.HSTU_BF16 if o_bf16 else H.HSTU_F32, H._dtype_code(torch.empty(0, dtype=udt)),
+                         H.HSTU_BF16, to_dev(o, torch.bfloat16 if o_bf16 else torch.float32), D, to_dev(uvqk, udt),
+                         4 * D,
                          to_dev(gamma, torch.float32), to_dev(beta, torch.float32), 1e-5, g, mu, rstd)
     ge, mue, rse = O.norm_gate_fwd(o, uvqk[:, :D], gamma, beta)
     assert_close(g.float().cpu().numpy(), ge, *BF16_TOL, what="G")
