@@ -7,6 +7,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/hstu.h"
 #include "hstu_internal.h"
 
@@ -357,3 +359,67 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Attention forward without a caller workspace.
+//
+// Some callers cannot hand the library any device memory of their own: a serving process that
+// reserved its whole memory budget at start-up and forbids allocation on the request path, or a
+// plain C host program that has no device allocator to carve a workspace from. For them the
+// attention forward's scratch (status word, work-list count and the (sequence, tile) items) lives
+// in a fixed array compiled into the library. Every GPU that loads the library holds this array
+// until the process exits.
+// ---------------------------------------------------------------------------------------------
+namespace hstu {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = kWsHeader + 256 + 8ull * HSTU_NOALLOC_MAX_ITEMS;   // 524,800 bytes
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch per device. In host code the array's name is only a
+// host-side stand-in, so the address must be asked for once per device, with that device current.
+struct NoAllocSlot {
+  bool ready;
+  void* ptr;
+};
+NoAllocSlot g_noalloc_slots[64];
+std::mutex g_noalloc_mutex;
+
+hstu_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= 64) return HSTU_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_slots[dev].ready) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    g_noalloc_slots[dev].ptr = p;
+    g_noalloc_slots[dev].ready = true;
+  }
+  *out = g_noalloc_slots[dev].ptr;
+  return HSTU_OK;
+}
+
+}  // namespace
+}  // namespace hstu
+
+extern "C" hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const void* q,
+                                               const void* k, const void* v, const float* rab_pos,
+                                               const float* rab_time, void* out, hstu_stream_t stream) {
+  hstu_status_t s = check_attn(desc, jag);
+  if (s != HSTU_OK) return s;
+  if (capacity_of(jag) > HSTU_NOALLOC_MAX_ITEMS) return HSTU_ERR_WORKSPACE;
+  if (jag->T > 0 && (!q || !k || !v || !rab_pos || !rab_time || !out)) return HSTU_ERR_INVALID_ARG;
+  if (is_tc_dtype(desc->dtype) && jag->T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)))
+    return HSTU_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != HSTU_OK) return s;
+  // the status word must start at zero for this call (kernels record only the first error);
+  // the work list is rewritten completely by every call
+  cudaError_t e = cudaMemsetAsync(scratch, 0, kWsHeader, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  return run_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, scratch, stream);
+}

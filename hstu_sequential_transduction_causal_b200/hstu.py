@@ -75,6 +75,8 @@ SIGNATURES = {
     "hstu_attn_workspace_size": (c_sz, [P(hstu_attn_desc_t), P(hstu_jagged_t)]),
     "hstu_attn_fwd": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                               c_vp, c_sz, c_vp]),
+    "hstu_attn_fwd_noalloc": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                      c_vp]),
     "hstu_norm_gate_fwd": (c_i32, [c_i64, c_i32, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp,
                                    c_f32, c_vp, c_vp, c_vp, c_vp]),
     "hstu_out_proj_fwd": (c_i32, [c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_i32, c_vp,
@@ -217,6 +219,14 @@ def hstu_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, ws, stream=None) -
     _check("hstu_attn_fwd", lib().hstu_attn_fwd(ctypes.byref(desc), ctypes.byref(jag), _ptr(q), _ptr(k), _ptr(v),
                                                 _ptr(rab_pos), _ptr(rab_time), _ptr(out), _ptr(ws),
                                                 ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def hstu_attn_fwd_noalloc(desc, jag, q, k, v, rab_pos, rab_time, out, stream=None) -> None:
+    """hstu_attn_fwd without a workspace: the scratch is a fixed array inside the library (for
+    callers that cannot allocate device memory); calls that overlap on the GPU race."""
+    _check("hstu_attn_fwd_noalloc", lib().hstu_attn_fwd_noalloc(ctypes.byref(desc), ctypes.byref(jag), _ptr(q), _ptr(k),
+                                                                _ptr(v), _ptr(rab_pos), _ptr(rab_time), _ptr(out),
+                                                                _stream(stream)))
 
 
 def hstu_norm_gate_fwd(T, D, o_dtype_code, u_dtype_code, g_dtype_code, o, ld_o, u, ld_u, gamma, beta, eps, g, mu,

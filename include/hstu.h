@@ -217,6 +217,30 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
                             const float* rab_time, void* out, void* ws, size_t ws_bytes,
                             hstu_stream_t stream);
 
+/* Largest number of (sequence, 128-row tile) work items, B + ceil(T / 128), that
+ * hstu_attn_fwd_noalloc accepts. */
+#define HSTU_NOALLOC_MAX_ITEMS 65536
+
+/* hstu_attn_fwd for callers that cannot allocate device memory and so cannot pass a workspace:
+ * for example a serving process that reserves its whole memory budget at start-up and forbids
+ * allocation on the request path, or a plain C host with no device allocator of its own. The
+ * pages have no counterpart; it exists for integration only. Same arguments and result as
+ * hstu_attn_fwd without ws / ws_bytes. Its scratch (status word, work list) is a fixed array of
+ * 524,800 bytes compiled into the library: every GPU that loads the library holds it until the
+ * process exits, and the call itself allocates and frees nothing.
+ *  - Batches needing more than HSTU_NOALLOC_MAX_ITEMS work items return HSTU_ERR_WORKSPACE
+ *    before anything is enqueued.
+ *  - The first call on each device looks up that device's address of the array (with the device
+ *    current); make that first call before any stream capture.
+ *  - All calls share the one array and each call clears its status word: calls that overlap on
+ *    the GPU (other streams, other host threads) race and must be serialised by the caller.
+ *    Device-side errors of this variant are not reported; use hstu_attn_fwd with a workspace and
+ *    hstu_sync_status to diagnose. */
+hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag,
+                                    const void* q, const void* k, const void* v,
+                                    const float* rab_pos, const float* rab_time, void* out,
+                                    hstu_stream_t stream);
+
 /* LayerNorm (.) U gating ("Generative Recommenders and HSTU", third equation; "HSTU: The First
  * Exploration of the Scaling Law", 7.1.4 Innovation 3): g = (gamma (o - mu) rstd + beta) (.) u
  * over all D features of a token; mu, rstd (fp32 [T]) are stored for the backward. g is [T, D]
