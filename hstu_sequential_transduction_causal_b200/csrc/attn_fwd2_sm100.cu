@@ -1,0 +1,401 @@
+// attn_fwd2_sm100.cu - jagged causal pointwise attention forward, tensor-core kernel.
+//
+//   O_i = sum_{j <= i, same sequence} SiLU(q_i . k_j + rab_pos[i-j] + rab_time[bucket(t_i - t_j)])
+//         * inv_N * v_j                                                   (per head)
+// ("4.4 Scaling Recommendation Models", Generative Recommenders and HSTU: second equation and the
+// pointwise-aggregation bullet; "HSTU: The First Exploration of the Scaling Law", 7.1.4
+// Innovation 1 (SiLU instead of softmax, no 1/sqrt(d)) and Innovation 2 (position and time bias).)
+//
+// Two kernels:
+//  1. attn_bias_kernel: for every causal (query tile, key tile) pair of every sequence, the
+//     relative bias 0.5 * (rab_pos[i-j] + rab_time[bucket(t_i - t_j)]) as an fp16 128x128 tile in
+//     the workspace. The bias does not depend on the head, so it is computed once per pair
+//     instead of once per pair and head; buckets are exact integer evaluations.
+//  2. attn_fwd_tc2_kernel<F16, G>: one CTA per (sequence, 128-row query tile, group of G heads),
+//     longest causal rows first; only key tiles 0..t of the tile's own sequence are visited.
+//       warp 8   : TMA producer: Q of the G heads once; per key tile the bias tile (2 stages);
+//                  per (key tile, head) K and V (3 stages); all 128-byte swizzled.
+//       warp 9   : tcgen05 issuer: S = Q K^T into one of two TMEM tiles; then O_h += P V with the
+//                  A operand P read from TMEM (P overwrites the S tile it came from).
+//       warps 0-7: TMEM lane quadrant (warp & 3), key half (warp >> 2). Per element, in packed
+//                  fp16: h = 0.5 s + 0.5 bias, P = h + h tanh(h) = SiLU(s + bias); causal mask on
+//                  the diagonal tile only; P back into TMEM.
+//     1/N is applied to the fp32 accumulator in the epilogue; O is written in fp32 (or bf16).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hstu_internal.h"
+#include "sm100_ptx.cuh"
+#include "time_bucket_dev.cuh"
+
+namespace hstu {
+
+namespace {
+
+constexpr int kD = 64;
+constexpr int kNS = 3;                 // K/V stages
+constexpr int kSiluWarps = 8;
+constexpr int kThreads2 = 32 * (kSiluWarps + 2);
+constexpr uint32_t kHalf2Half = 0x38003800u;   // (0.5, 0.5) in fp16
+
+__device__ __forceinline__ int pos_index2(long long r, int L) {
+  r = r > L - 1 ? L - 1 : r;
+  r = r < -(L - 1) ? -(L - 1) : r;
+  return static_cast<int>(r) + L - 1;
+}
+
+// ----------------------------------------------------------------------------------------------
+// 1. bias tiles
+// ----------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+attn_bias_kernel(AttnArgs a) {
+  const int item = blockIdx.x;
+  const int kt = blockIdx.y;
+  if (item >= *a.count) return;
+  const int b = a.items[2 * item];
+  const int qt = a.items[2 * item + 1];
+  if (kt > qt) return;
+  const long long seq0 = a.offsets[b];
+  const int n = static_cast<int>(a.offsets[b + 1] - seq0);
+  const long long pair = a.pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2 + kt;
+
+  __shared__ long long s_kts[128];
+  __shared__ float s_win[256];
+  __shared__ float s_rt[128];
+  __shared__ long long s_oct[63][4];
+  const int tid = threadIdx.x;
+  const int L = a.pos_max_len;
+  const int nb = a.n_buckets;
+  if (tid < 128) {
+    const int kj = kt * kQTile + tid;
+    s_kts[tid] = kj < n ? a.ts[seq0 + kj] : 0;
+    if (tid < nb) s_rt[tid] = a.rab_time[tid];
+  }
+  {
+    const long long rel0 = static_cast<long long>(qt - kt) * kQTile - 127;
+    if (tid < 255) s_win[tid] = a.rab_pos[pos_index2(rel0 + tid, L)];
+  }
+  for (int e = tid; e < 63 * 4; e += 256) s_oct[e / 4][e % 4] = c_time_octaves[e / 4][e % 4];
+  __syncthreads();
+
+  const int r = tid >> 1;        // query row within the tile
+  const int c = tid & 1;         // key half
+  const int qi = qt * kQTile + r;
+  const long long t_i = a.ts[seq0 + (qi < n ? qi : n - 1)];
+  uint16_t* dst = reinterpret_cast<uint16_t*>(a.bias) + (pair * kQTile + r) * kQTile + 64 * c;
+#pragma unroll 1
+  for (int u = 0; u < 8; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float v2[2];
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const int col = 64 * c + 8 * u + 2 * e + x;
+        const int bkt = time_bucket_dev(t_i - s_kts[col], s_oct, nb);
+        v2[x] = 0.5f * (s_win[r - col + 127] + s_rt[bkt]);
+      }
+      w[e] = pack_f16x2(v2[0], v2[1]);
+    }
+    reinterpret_cast<uint4*>(dst)[u] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// ----------------------------------------------------------------------------------------------
+// 2. attention
+// ----------------------------------------------------------------------------------------------
+template <int G>
+struct Smem2 {
+  static constexpr int kQ = 0;
+  static constexpr int kKV = G * 16384;
+  static constexpr int kBias = kKV + kNS * 32768;
+  static constexpr int kBar = kBias + 2 * 32768;
+  static constexpr int kTotal = kBar + 256 + 1024;
+};
+
+template <bool F16, int G>
+__global__ void __launch_bounds__(kThreads2, 1)
+attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB, AttnArgs a,
+                    WaitCtl ctl) {
+  using L = Smem2<G>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int HG = a.H / G;
+  const int item = blockIdx.x / HG;
+  const int hg = blockIdx.x - item * HG;
+  if (item >= *a.count) return;
+  const int b = a.items[2 * item];
+  const int qt = a.items[2 * item + 1];
+  const long long seq0 = a.offsets[b];
+  const int n = static_cast<int>(a.offsets[b + 1] - seq0);
+  const int nkt = qt + 1;
+  const int nsteps = nkt * G;
+  const long long pair0 = a.pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  // 0 q_full | 1..3 kv_full | 4..6 kv_empty | 7,8 b_full | 9,10 b_empty | 11,12 s_full |
+  // 13,14 p_full | 15 o_full
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t bar0 = smem_u32(bars);
+  auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  const uint32_t bar_q = BAR(0), bar_o = BAR(15);
+  auto bar_kv_full = [&](int s) { return BAR(1 + s); };
+  auto bar_kv_empty = [&](int s) { return BAR(4 + s); };
+  auto bar_b_full = [&](int s) { return BAR(7 + s); };
+  auto bar_b_empty = [&](int s) { return BAR(9 + s); };
+  auto bar_s_full = [&](int s) { return BAR(11 + s); };
+  auto bar_p_full = [&](int s) { return BAR(13 + s); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr int kSiluThreads = 32 * kSiluWarps;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(bar_kv_full(s), 1);
+      mbar_init(bar_kv_empty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_b_full(s), 1);
+      mbar_init(bar_b_empty(s), kSiluThreads);
+      mbar_init(bar_s_full(s), 1);
+      mbar_init(bar_p_full(s), kSiluThreads);
+    }
+    mbar_init(bar_o, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kSiluWarps && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;    // S0 cols [0,128), S1 [128,256), O_h [256 + 64h, +64)
+
+  const uint32_t sQ = smem_u32(smem + L::kQ);
+  const uint32_t sKV = smem_u32(smem + L::kKV);
+  const uint32_t sB = smem_u32(smem + L::kBias);
+  const int qrow0 = static_cast<int>(seq0) + qt * kQTile;
+
+  if (warp == kSiluWarps) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, G * 16384);
+      for (int h = 0; h < G; ++h) tma_load_2d(sQ + h * 16384, &tmQ, bar_q, (hg * G + h) * kD, qrow0);
+      bool ok = true;
+      int s = 0;
+      for (int kt = 0; ok && kt < nkt; ++kt) {
+        const int bs = kt & 1;
+        if (kt >= 2 && !mbar_wait(bar_b_empty(bs), ((kt >> 1) & 1) ^ 1, abort_flag, ctl)) break;
+        const int brow = static_cast<int>((pair0 + kt) * kQTile);
+        mbar_arrive_expect_tx(bar_b_full(bs), 32768);
+        tma_load_2d(sB + bs * 32768, &tmB, bar_b_full(bs), 0, brow);
+        tma_load_2d(sB + bs * 32768 + 16384, &tmB, bar_b_full(bs), 64, brow);
+        const int krow = static_cast<int>(seq0) + kt * kQTile;
+        for (int h = 0; h < G; ++h, ++s) {
+          const int st = s % kNS;
+          if (s >= kNS && !mbar_wait(bar_kv_empty(st), ((s / kNS) - 1) & 1, abort_flag, ctl)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_kv_full(st), 32768);
+          tma_load_2d(sKV + st * 32768, &tmK, bar_kv_full(st), (hg * G + h) * kD, krow);
+          tma_load_2d(sKV + st * 32768 + 16384, &tmV, bar_kv_full(st), (hg * G + h) * kD, krow);
+        }
+      }
+    }
+  } else if (warp == kSiluWarps + 1) {
+    // ---------------- tcgen05 issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = make_idesc_f16kind(128, 128, 0, 0, F16);
+      constexpr uint32_t idesc_pv = make_idesc_f16kind(128, 64, 0, 1, F16);
+      bool ok = mbar_wait(bar_q, 0, abort_flag, ctl);
+      auto issue_pv = [&](int t) -> bool {
+        const int buf = t & 1, st = t % kNS, h = t % G;
+        if (!mbar_wait(bar_p_full(buf), (t >> 1) & 1, abort_flag, ctl)) return false;
+        tc_fence_after();
+        const uint32_t v = sKV + st * 32768 + 16384;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t a_tmem = tmem + buf * 128 + 64 * (kk >> 2) + 8 * (kk & 3);
+          umma_f16_ts(tmem + 256 + 64 * h, a_tmem, make_sdesc_sw128(v + kk * 2048, 16384, 1024), idesc_pv,
+                      (t >= G || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar_kv_empty(st));
+        return true;
+      };
+      for (int s = 0; ok && s < nsteps; ++s) {
+        const int buf = s & 1, st = s % kNS, h = s % G;
+        if (!mbar_wait(bar_kv_full(st), (s / kNS) & 1, abort_flag, ctl)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kb = sKV + st * 32768;
+        const uint32_t qb = sQ + h * 16384;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_f16_ss(tmem + buf * 128, make_sdesc_sw128(qb + kk * 32, 16, 1024),
+                      make_sdesc_sw128(kb + kk * 32, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        umma_commit(bar_s_full(buf));
+        if (s >= 1 && !issue_pv(s - 1)) { ok = false; break; }
+      }
+      if (ok && issue_pv(nsteps - 1)) umma_commit(bar_o);
+    }
+  } else {
+    // ---------------- SiLU warps ----------------
+    const int quad = warp & 3;
+    const int half = warp >> 2;          // keys [64 half, 64 half + 64)
+    const int r = quad * 32 + lane;      // query row within the tile == TMEM lane
+    const int qi = qt * kQTile + r;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    bool ok = true;
+    for (int kt = 0; ok && kt < nkt; ++kt) {
+      const int bs = kt & 1;
+      if (!mbar_wait(bar_b_full(bs), (kt >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
+      uint32_t hb[32];
+      {
+        const uint8_t* brow = smem + L::kBias + bs * 32768 + half * 16384 + r * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = *reinterpret_cast<const uint4*>(brow + ((u ^ (r & 7)) << 4));
+          hb[4 * u] = v.x; hb[4 * u + 1] = v.y; hb[4 * u + 2] = v.z; hb[4 * u + 3] = v.w;
+        }
+      }
+      mbar_arrive(bar_b_empty(bs));
+      const bool diag = (kt == qt);
+      for (int h = 0; h < G; ++h) {
+        const int s = kt * G + h;
+        const int buf = s & 1;
+        if (!mbar_wait(bar_s_full(buf), (s >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t p[32];
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+          uint32_t sv[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + buf * 128 + 64 * half + 32 * hc, sv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const uint32_t s2 = pack_f16x2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1]));
+            const uint32_t h2 = hfma2_u32(s2, kHalf2Half, hb[16 * hc + j]);
+            const uint32_t t2 = tanh_f16x2(h2);
+            uint32_t y2 = hfma2_u32(h2, t2, h2);
+            if (!F16) {   // the P V MMA takes A and B of one type: P as bf16 next to bf16 V
+              const float2 f = unpack_f16x2(y2);
+              y2 = pack_bf16x2(f.x, f.y);
+            }
+            if (diag) {
+              const int col = 64 * half + 32 * hc + 2 * j;
+              const uint32_t m = (col + 1 <= r) ? 0xFFFFFFFFu : ((col <= r) ? 0x0000FFFFu : 0u);
+              y2 &= m;
+            }
+            p[16 * hc + j] = y2;
+          }
+        }
+        tmem_st_32x32b_x32(tmem + lane_base + buf * 128 + 64 * half, p);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p_full(buf));
+      }
+    }
+    if (ok && mbar_wait(bar_o, 0, abort_flag, ctl)) {
+      tc_fence_after();
+      // G == 1: both key halves split head 0's 64 columns; G >= 2: half c handles heads c, c+2, ...
+      constexpr int kHeadsPerWarp = G == 1 ? 1 : G / 2;
+      constexpr int kCols = G == 1 ? 32 : 64;
+      const float sc = a.inv_N;
+#pragma unroll 1
+      for (int e = 0; e < kHeadsPerWarp; ++e) {
+        const int h = G == 1 ? 0 : half + 2 * e;
+        const int col0 = G == 1 ? 32 * half : 0;
+#pragma unroll 1
+        for (int cc = 0; cc < kCols; cc += 32) {
+          uint32_t ov[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h + col0 + cc, ov);
+          tmem_ld_wait();
+          if (qi < n) {
+            const long long orow = seq0 + qi;
+            const int ocol = (hg * G + h) * kD + col0 + cc;
+            if (a.o_f32) {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + orow * a.ld_o + ocol);
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(__uint_as_float(ov[4 * q]) * sc, __uint_as_float(ov[4 * q + 1]) * sc,
+                                     __uint_as_float(ov[4 * q + 2]) * sc, __uint_as_float(ov[4 * q + 3]) * sc);
+            } else {
+              uint4* dst =
+                  reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + orow * a.ld_o + ocol);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                dst[q] = make_uint4(
+                    pack_bf16x2(__uint_as_float(ov[8 * q]) * sc, __uint_as_float(ov[8 * q + 1]) * sc),
+                    pack_bf16x2(__uint_as_float(ov[8 * q + 2]) * sc, __uint_as_float(ov[8 * q + 3]) * sc),
+                    pack_bf16x2(__uint_as_float(ov[8 * q + 4]) * sc, __uint_as_float(ov[8 * q + 5]) * sc),
+                    pack_bf16x2(__uint_as_float(ov[8 * q + 6]) * sc, __uint_as_float(ov[8 * q + 7]) * sc));
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <bool F16, int G>
+cudaError_t launch_attn2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tb,
+                         const AttnArgs& a, cudaStream_t st) {
+  auto kern = attn_fwd_tc2_kernel<F16, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem2<G>::kTotal);
+  if (e != cudaSuccess) return e;
+  const long long blocks = a.capacity * (a.H / G);
+  kern<<<static_cast<unsigned>(blocks), kThreads2, Smem2<G>::kTotal, st>>>(tq, tk, tv, tb, a, wait_ctl(a.status));
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int64_t attn_max_pairs(int64_t capacity, int max_len) {
+  const int64_t mt = (static_cast<int64_t>(max_len) + kQTile - 1) / kQTile;
+  return capacity * (mt + 1) / 2;
+}
+
+cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
+  cudaError_t e = upload_time_octaves();
+  if (e != cudaSuccess) return e;
+  if (a.T == 0 || a.capacity == 0) return cudaSuccess;
+  const int mt = (a.max_len + kQTile - 1) / kQTile;
+  if (mt == 0) return cudaSuccess;
+  attn_bias_kernel<<<dim3(static_cast<unsigned>(a.capacity), static_cast<unsigned>(mt)), 256, 0, st>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap tq, tk, tv, tb;
+  const bool f16 = a.in_f16 != 0;
+  if (!encode_tmap_2d_bf16(&tq, a.q, static_cast<int64_t>(a.H) * kD, a.T, a.ld_q, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tk, a.k, static_cast<int64_t>(a.H) * kD, a.T, a.ld_k, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tv, a.v, static_cast<int64_t>(a.H) * kD, a.T, a.ld_v, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tb, a.bias, kQTile, a.max_pairs * kQTile, kQTile, 64, 128, true))
+    return cudaErrorInvalidValue;
+  const int G = (a.H % 2 == 0) ? 2 : 1;
+  if (f16) return G == 2 ? launch_attn2<true, 2>(tq, tk, tv, tb, a, st) : launch_attn2<true, 1>(tq, tk, tv, tb, a, st);
+  return G == 2 ? launch_attn2<false, 2>(tq, tk, tv, tb, a, st) : launch_attn2<false, 1>(tq, tk, tv, tb, a, st);
+}
+
+}  // namespace hstu

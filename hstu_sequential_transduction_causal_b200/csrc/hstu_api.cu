@@ -46,9 +46,28 @@ hstu_status_t cuda_status(cudaError_t e) {
 int* ws_status(void* ws) { return static_cast<int*>(ws); }
 
 // attention workspace: [0,256) status | [256,512) count | [512, ...) items (int32 x 2 x capacity)
-size_t attn_ws_bytes(int64_t capacity) { return kWsHeader + 256 + align_up(static_cast<size_t>(capacity) * 8, 256); }
-
 int64_t capacity_of(const hstu_jagged_t* j) { return static_cast<int64_t>(j->B) + (j->T + kQTile - 1) / kQTile; }
+
+// attention workspace: [0,256) status | [256,512) work-list count | items (int32 x 2 x capacity) |
+// pair_base (int64 x (B+1)) | fp16 bias tiles (32 KB per causal tile pair, 1024-aligned)
+struct AttnWs {
+  size_t items, pairs, bias, items_end, total;
+  int64_t max_pairs;
+};
+
+AttnWs attn_ws_layout(const hstu_jagged_t* j) {
+  AttnWs w{};
+  const int64_t cap = capacity_of(j);
+  w.items = kWsHeader + 256;
+  w.items_end = w.items + align_up(static_cast<size_t>(cap) * 8, 256);
+  w.pairs = w.items_end;
+  w.bias = align_up(w.pairs + align_up(static_cast<size_t>(j->B + 1) * 8, 256), 1024);
+  w.max_pairs = attn_max_pairs(cap, j->max_len);
+  w.total = w.bias + static_cast<size_t>(w.max_pairs) * kQTile * kQTile * 2;
+  return w;
+}
+
+size_t attn_ws_bytes(const hstu_jagged_t* j) { return attn_ws_layout(j).total; }
 
 hstu_status_t check_jagged(const hstu_jagged_t* j) {
   if (!j || j->B < 0 || j->T < 0 || j->max_len < 0) return HSTU_ERR_INVALID_ARG;
@@ -81,13 +100,16 @@ hstu_status_t check_attn(const hstu_attn_desc_t* d, const hstu_jagged_t* j) {
   return HSTU_OK;
 }
 
+// tile_pairs: the workspace has the full attn_ws_layout (bias tiles); otherwise only the work list
+// fits and the tensor-core path runs the kernel that evaluates the bias per element and head.
 hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, const void* q, const void* k,
                            const void* v, const float* rab_pos, const float* rab_time, void* out, void* ws,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool tile_pairs = true) {
   const int64_t cap = capacity_of(j);
+  const AttnWs lay = attn_ws_layout(j);
   uint8_t* w = static_cast<uint8_t*>(ws);
   int32_t* count = reinterpret_cast<int32_t*>(w + kWsHeader);
-  int32_t* items = reinterpret_cast<int32_t*>(w + kWsHeader + 256);
+  int32_t* items = reinterpret_cast<int32_t*>(w + lay.items);
   AttnArgs a{};
   a.B = j->B; a.T = j->T; a.max_len = j->max_len; a.offsets = j->offsets; a.ts = j->timestamps;
   a.H = d->H; a.dqk = d->d_qk; a.dv = d->d_v; a.inv_N = d->inv_N; a.pos_max_len = d->pos_max_len;
@@ -97,10 +119,18 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
   a.in_f16 = d->dtype == HSTU_F16;
   a.rab_pos = rab_pos; a.rab_time = rab_time; a.items = items; a.count = count; a.capacity = cap;
   a.status = ws_status(ws);
-  cudaError_t e = launch_worklist(j->offsets, j->B, j->T, j->max_len, items, count, a.status, st);
+  const bool pairs = tile_pairs && is_tc_dtype(d->dtype);
+  if (pairs) {
+    a.pair_base = reinterpret_cast<const long long*>(w + lay.pairs);
+    a.bias = w + lay.bias;
+    a.max_pairs = lay.max_pairs;
+  }
+  cudaError_t e = launch_worklist(j->offsets, j->B, j->T, j->max_len, items, count, a.status, st,
+                                  pairs ? reinterpret_cast<long long*>(w + lay.pairs) : nullptr);
   if (e != cudaSuccess) return cuda_status(e);
   if (j->T == 0) return HSTU_OK;
-  e = is_tc_dtype(d->dtype) ? attn_fwd_bf16_tc(a, st) : attn_fwd_f32_simt(a, st);
+  if (!is_tc_dtype(d->dtype)) e = attn_fwd_f32_simt(a, st);
+  else e = pairs ? attn_fwd_tc2(a, st) : attn_fwd_bf16_tc(a, st);
   return cuda_status(e);
 }
 
@@ -242,7 +272,7 @@ hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype
 size_t hstu_attn_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag) {
   (void)desc;
   if (check_jagged(jag) != HSTU_OK) return 0;
-  return attn_ws_bytes(capacity_of(jag));
+  return attn_ws_bytes(jag);
 }
 
 hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const void* q, const void* k,
@@ -251,7 +281,7 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
   hstu_status_t s = check_attn(desc, jag);
   if (s != HSTU_OK) return s;
   if (!ws) return HSTU_ERR_INVALID_ARG;
-  if (ws_bytes < attn_ws_bytes(capacity_of(jag))) return HSTU_ERR_WORKSPACE;
+  if (ws_bytes < attn_ws_bytes(jag)) return HSTU_ERR_WORKSPACE;
   if (jag->T > 0 && (!q || !k || !v || !rab_pos || !rab_time || !out)) return HSTU_ERR_INVALID_ARG;
   if (is_tc_dtype(desc->dtype) && jag->T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)))
     return HSTU_ERR_UNSUPPORTED;
@@ -296,7 +326,7 @@ hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const 
 
 size_t hstu_layer_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag) {
   if (!desc || check_jagged(jag) != HSTU_OK) return 0;
-  size_t bytes = attn_ws_bytes(capacity_of(jag));
+  size_t bytes = attn_ws_bytes(jag);
   if (desc->dtype == HSTU_BF16 && desc->x_dtype == HSTU_F32)
     bytes += align_up(static_cast<size_t>(jag->T) * desc->D * 2, 256);
   return bytes;
@@ -334,7 +364,7 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
     if (x_bf16) {
       x_op = x_bf16;
     } else {
-      void* conv = static_cast<uint8_t*>(ws) + attn_ws_bytes(capacity_of(jag));
+      void* conv = static_cast<uint8_t*>(ws) + attn_ws_bytes(jag);
       cudaError_t e = convert_f32_to_bf16(static_cast<const float*>(x), conv, T * D, st);
       if (e != cudaSuccess) return cuda_status(e);
       x_op = conv;
@@ -421,5 +451,5 @@ extern "C" hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_desc_t* desc, con
   // the work list is rewritten completely by every call
   cudaError_t e = cudaMemsetAsync(scratch, 0, kWsHeader, stream);
   if (e != cudaSuccess) return cuda_status(e);
-  return run_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, scratch, stream);
+  return run_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, scratch, stream, false);
 }

@@ -62,8 +62,10 @@ cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
 // ---------------------------------------------------------------------------------------------
 // jagged metadata / time buckets
 // ---------------------------------------------------------------------------------------------
+// Builds the (sequence, query tile) work list; with pair_base (device, [B+1]) also the index of
+// each sequence's first causal (query tile, key tile) pair and, in pair_base[B], their total.
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
-                            int32_t* count, int* status, cudaStream_t st);
+                            int32_t* count, int* status, cudaStream_t st, long long* pair_base = nullptr);
 cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T,
                                 int n_buckets, const int64_t* sq_offsets, uint8_t* out,
                                 cudaStream_t st);
@@ -92,9 +94,16 @@ struct AttnArgs {
   const int32_t* count;
   int64_t capacity;
   int* status;
+  const long long* pair_base;   // [B+1] first causal tile pair of each sequence (tile-pair kernel)
+  void* bias;                   // fp16 [max_pairs, 128, 128] bias tiles (tile-pair kernel)
+  int64_t max_pairs;
 };
 
-cudaError_t attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t st);
+// Bound on the number of causal (query tile, key tile) pairs of a batch.
+int64_t attn_max_pairs(int64_t capacity, int max_len);
+
+cudaError_t attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t st);     // work list only
+cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st);         // bias tiles + work list
 cudaError_t attn_fwd_f32_simt(const AttnArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------------

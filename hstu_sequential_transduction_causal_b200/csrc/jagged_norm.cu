@@ -23,7 +23,7 @@ namespace {
 // ----------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
 worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items,
-                int32_t* count, int* status) {
+                int32_t* count, int* status, long long* pair_base) {
   __shared__ int s_warp[32];
   __shared__ int s_max_tiles;
   __shared__ int s_bad;
@@ -45,6 +45,7 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
     if (tid == 0) {
       *count = 0;
       report_error(status, kDevBadInput);
+      if (pair_base) pair_base[B > 0 ? B : 0] = 0;
     }
     return;
   }
@@ -79,6 +80,46 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
     }
   }
   if (tid == 0) *count = s_base;
+  if (!pair_base) return;
+  // pair_base[b] = sum_{b' < b} nt_b' (nt_b' + 1) / 2: index of sequence b's first causal
+  // (query tile, key tile) pair; pair_base[B] is the total.
+  __shared__ long long s_wsum[32];
+  __shared__ long long s_run;
+  if (tid == 0) s_run = 0;
+  __syncthreads();
+  for (int c0 = 0; c0 < B; c0 += blockDim.x) {
+    const int b = c0 + tid;
+    long long v = 0;
+    if (b < B) {
+      const long long nt = (off[b + 1] - off[b] + kQTile - 1) / kQTile;
+      v = nt * (nt + 1) / 2;
+    }
+    long long inc = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const long long y = __shfl_up_sync(0xffffffffu, inc, d);
+      if (lane >= d) inc += y;
+    }
+    if (lane == 31) s_wsum[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+      const long long w = s_wsum[lane];
+      long long winc = w;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, winc, d);
+        if (lane >= d) winc += y;
+      }
+      s_wsum[lane] = winc - w;
+    }
+    __syncthreads();
+    const long long excl = s_run + s_wsum[warp] + inc - v;
+    if (b < B) pair_base[b] = excl;
+    __syncthreads();
+    if (tid == blockDim.x - 1) s_run = excl + v;
+    __syncthreads();
+  }
+  if (tid == 0) pair_base[B] = s_run;
 }
 
 // One warp per query row: writes bucket(t_i - t_j) for every key j of the row's sequence.
@@ -184,8 +225,8 @@ cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int
 }  // namespace
 
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
-                            int32_t* count, int* status, cudaStream_t st) {
-  worklist_kernel<<<1, 1024, 0, st>>>(offsets, B, T, max_len, items, count, status);
+                            int32_t* count, int* status, cudaStream_t st, long long* pair_base) {
+  worklist_kernel<<<1, 1024, 0, st>>>(offsets, B, T, max_len, items, count, status, pair_base);
   return cudaGetLastError();
 }
 

@@ -153,6 +153,20 @@ def test_attn_fwd_tensor_core_ragged(spread, out_bf16, f16):
     assert_close(got, exp, 1e-2 * scale, 1e-2, what="O")
 
 
+def test_attn_fwd_tensor_core_odd_head_count():
+    lengths = [130, 1, 385]
+    Hh, d, L = 3, 64, 400
+    inv_N = 1.0 / 300
+    off, ts, q, k, v, rp, rt = _attn_case(lengths, Hh, d, L, inv_N, True, seed=7, f16=True)
+    got, st = _run_attn(off, ts, q, k, v, rp, rt, Hh, d, L, inv_N, True, f16=True)
+    assert st == 0
+    T = int(off[-1])
+    exp = O.pointwise_attention_fwd(q.reshape(T, Hh, d), k.reshape(T, Hh, d), v.reshape(T, Hh, d), off, ts, rp, rt,
+                                    inv_N, L, THR).reshape(T, Hh * d)
+    scale = float(np.sqrt(np.mean(exp ** 2)))
+    assert_close(got, exp, 1e-2 * scale, 1e-2, what="O (3 heads)")
+
+
 def test_attn_fwd_f32_single_layer_workload():
     wl = W.make_workload("c1", seed=0)
     Hh, d, L = wl.H, wl.D // wl.H, wl.pos_max_len
