@@ -1,0 +1,447 @@
+// attn_bwd_sm100.cu - jagged causal pointwise attention, backward.
+//
+// With x_ij = q_i.k_j + rab(i, j), A_ij = SiLU(x_ij) inv_N on causal pairs (j <= i) and 0 elsewhere,
+// O = A V (per head). Given dO:
+//   dV = A^T dO,  dA = dO V^T,  dX = dA (.) SiLU'(x) inv_N (causal pairs),
+//   dQ = dX K,  dK = dX^T Q,  d rab_pos[idx(i-j)] += sum_h dX_ij,  d rab_time[bucket(t_i - t_j)] += sum_h dX_ij
+// (derived from the forward of "4.4 Scaling Recommendation Models", Generative Recommenders and HSTU,
+// second equation, and the bias of "HSTU: The First Exploration of the Scaling Law", 7.1.4
+// Innovation 2).
+//
+// attn_bias_t_kernel: per causal (query tile, key tile) pair, the transposed fp16 half-bias tile
+// [key][query] and the u8 time-bucket tile [key][query] (head independent, computed once).
+// attn_bwd_tc_kernel<F16>: one CTA per (sequence, 128-key tile, head), key tiles that visit the
+// most query tiles first; it walks the query tiles t >= its key tile:
+//   warp 8   : TMA: K, V once; Q and dO of each query tile (2 stages); bias and bucket tiles.
+//   warp 9   : tcgen05: S^T = K Q^T and dA^T = V dO^T into TMEM; after the elementwise step
+//              dV += P^T dO (P^T from TMEM), dK += dX^T Q and dQ_tile = dX K (dX^T from shared
+//              memory, read K-major for dK and MN-major for dQ).
+//   warps 0-7: key row = TMEM lane (warp & 3), query half (warp >> 2): x = s + bias,
+//              P^T = SiLU(x), dX^T = dA SiLU'(x) inv_N in fp32, causal and length masks; the
+//              position-bias gradient by shared atomics (one window per query tile), the time-bias
+//              gradient by runs of equal bucket; dQ_tile added to the fp32 dQ by vector atomics.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hstu_internal.h"
+#include "sm100_ptx.cuh"
+#include "time_bucket_dev.cuh"
+
+namespace hstu {
+
+namespace {
+
+constexpr int kD = 64;
+constexpr int kSiluWarpsB = 8;
+constexpr int kThreadsB = 32 * (kSiluWarpsB + 2);
+constexpr int kSiluThreadsB = 32 * kSiluWarpsB;
+
+__device__ __forceinline__ int pos_index_b(long long r, int L) {
+  r = r > L - 1 ? L - 1 : r;
+  r = r < -(L - 1) ? -(L - 1) : r;
+  return static_cast<int>(r) + L - 1;
+}
+
+// ----------------------------------------------------------------------------------------------
+// transposed bias and bucket tiles
+// ----------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+attn_bias_t_kernel(AttnBwdArgs A) {
+  const AttnArgs& a = A.f;
+  const int item = blockIdx.x;
+  const int kt = blockIdx.y;
+  if (item >= *a.count) return;
+  const int b = a.items[2 * item];
+  const int qt = a.items[2 * item + 1];
+  if (kt > qt) return;
+  const long long seq0 = a.offsets[b];
+  const int n = static_cast<int>(a.offsets[b + 1] - seq0);
+  const long long pair = a.pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2 + kt;
+
+  __shared__ long long s_qts[128];
+  __shared__ float s_win[256];
+  __shared__ float s_rt[128];
+  __shared__ long long s_oct[63][4];
+  const int tid = threadIdx.x;
+  const int L = a.pos_max_len;
+  const int nb = a.n_buckets;
+  if (tid < 128) {
+    const int qi = qt * kQTile + tid;
+    s_qts[tid] = a.ts[seq0 + (qi < n ? qi : n - 1)];
+    if (tid < nb) s_rt[tid] = a.rab_time[tid];
+  }
+  {
+    const long long rel0 = static_cast<long long>(qt - kt) * kQTile - 127;
+    if (tid < 255) s_win[tid] = a.rab_pos[pos_index_b(rel0 + tid, L)];
+  }
+  for (int e = tid; e < 63 * 4; e += 256) s_oct[e / 4][e % 4] = c_time_octaves[e / 4][e % 4];
+  __syncthreads();
+
+  const int j = blockIdx.z * 32 + (tid >> 3);   // key row within the tile
+  const int cg = tid & 7;                        // queries [16 cg, 16 cg + 16)
+  const int kj = kt * kQTile + j;
+  const long long t_j = a.ts[seq0 + (kj < n ? kj : n - 1)];
+  uint16_t* dst = reinterpret_cast<uint16_t*>(A.bias_t) + (pair * kQTile + j) * kQTile + 16 * cg;
+  uint8_t* dstb = reinterpret_cast<uint8_t*>(A.bucket_t) + (pair * kQTile + j) * kQTile + 16 * cg;
+  uint32_t bw[4];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float v2[2];
+      int k2[2];
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const int col = 16 * cg + 8 * u + 2 * e + x;
+        k2[x] = time_bucket_dev(s_qts[col] - t_j, s_oct, nb);
+        v2[x] = 0.5f * (s_win[col - j + 127] + s_rt[k2[x]]);
+      }
+      w[e] = pack_f16x2(v2[0], v2[1]);
+      const int byte = 8 * u + 2 * e;       // position of k2[0] among the 16 buckets
+      if ((byte & 3) == 0) bw[byte >> 2] = 0;
+      bw[byte >> 2] |= (static_cast<uint32_t>(k2[0]) << (8 * (byte & 3))) |
+                       (static_cast<uint32_t>(k2[1]) << (8 * ((byte & 3) + 1)));
+    }
+    reinterpret_cast<uint4*>(dst)[u] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  *reinterpret_cast<uint4*>(dstb) = make_uint4(bw[0], bw[1], bw[2], bw[3]);
+}
+
+// ----------------------------------------------------------------------------------------------
+// backward kernel
+// ----------------------------------------------------------------------------------------------
+struct BwdSmem {
+  static constexpr int kK = 0;
+  static constexpr int kV = 16384;
+  static constexpr int kQ0 = 32768;          // stage st: Q at kQ0 + st * 32768, dO at +16384
+  static constexpr int kBT = kQ0 + 2 * 32768;   // bias^T: 2 chunks of 64 queries
+  static constexpr int kBK = kBT + 32768;       // bucket^T: 128 x 128 bytes
+  static constexpr int kDX = kBK + 16384;       // dX^T: 2 chunks of 64 queries
+  static constexpr int kHist = kDX + 32768;     // dtime[128] | dpos[2][256]
+  static constexpr int kBar = kHist + 512 + 2048;
+  static constexpr int kTotal = kBar + 256 + 1024;
+};
+
+template <bool F16>
+__global__ void __launch_bounds__(kThreadsB, 1)
+attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                   const __grid_constant__ CUtensorMap tmBT, const __grid_constant__ CUtensorMap tmBK, AttnBwdArgs A,
+                   WaitCtl ctl) {
+  using Lb = BwdSmem;
+  const AttnArgs& a = A.f;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int item = blockIdx.x / a.H;
+  const int h = blockIdx.x - item * a.H;
+  if (item >= *A.kcount) return;
+  const int b = A.kitems[2 * item];
+  const int kt = A.kitems[2 * item + 1];
+  const long long seq0 = a.offsets[b];
+  const int n = static_cast<int>(a.offsets[b + 1] - seq0);
+  const int nt = (n + kQTile - 1) / kQTile;
+  const int nsteps = nt - kt;              // query tiles kt .. nt-1
+  const long long pbase = a.pair_base[b];
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lb::kBar);
+  // 0 kv_full | 1,2 qdo_full | 3,4 qdo_empty | 5 bb_full | 6 bb_empty | 7 s_full | 8 p_ready |
+  // 9 dq_full | 10 fin | 11 group barrier of the elementwise warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t bar0 = smem_u32(bars);
+  auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  float* s_dtime = reinterpret_cast<float*>(smem + Lb::kHist);
+  float* s_dpos = s_dtime + 128;   // [2][256]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
+
+  if (tid == 0) {
+    mbar_init(BAR(0), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(BAR(1 + s), 1);
+      mbar_init(BAR(3 + s), 1);
+    }
+    mbar_init(BAR(5), 1);
+    mbar_init(BAR(6), kSiluThreadsB);
+    mbar_init(BAR(7), 1);
+    mbar_init(BAR(8), kSiluThreadsB);
+    mbar_init(BAR(9), 1);
+    mbar_init(BAR(10), 1);
+    mbar_init(BAR(11), kSiluThreadsB);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  for (int e = tid; e < 128 + 512; e += kThreadsB) s_dtime[e] = 0.0f;
+  if (warp == kSiluWarpsB && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmBT);
+    tma_prefetch_desc(&tmBK);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tDA = tmem + 128, tDV = tmem + 256, tDK = tmem + 320, tDQ = tmem + 384;
+
+  const uint32_t sK = smem_u32(smem + Lb::kK), sV = smem_u32(smem + Lb::kV);
+  const uint32_t sQ0 = smem_u32(smem + Lb::kQ0);
+  const uint32_t sBT = smem_u32(smem + Lb::kBT), sBK = smem_u32(smem + Lb::kBK);
+  const uint32_t sDX = smem_u32(smem + Lb::kDX);
+  const int krow = static_cast<int>(seq0) + kt * kQTile;
+
+  if (warp == kSiluWarpsB) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(BAR(0), 32768);
+      tma_load_2d(sK, &tmK, BAR(0), h * kD, krow);
+      tma_load_2d(sV, &tmV, BAR(0), h * kD, krow);
+      for (int s = 0; s < nsteps; ++s) {
+        const int qt = kt + s, st = s & 1;
+        if (s >= 2 && !mbar_wait(BAR(3 + st), ((s >> 1) & 1) ^ 1, abort_flag, ctl)) break;
+        const int qrow = static_cast<int>(seq0) + qt * kQTile;
+        mbar_arrive_expect_tx(BAR(1 + st), 32768);
+        tma_load_2d(sQ0 + st * 32768, &tmQ, BAR(1 + st), h * kD, qrow);
+        tma_load_2d(sQ0 + st * 32768 + 16384, &tmDO, BAR(1 + st), h * kD, qrow);
+        if (s >= 1 && !mbar_wait(BAR(6), (s - 1) & 1, abort_flag, ctl)) break;
+        const int prow = static_cast<int>((pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt) * kQTile);
+        mbar_arrive_expect_tx(BAR(5), 32768 + 16384);
+        tma_load_2d(sBT, &tmBT, BAR(5), 0, prow);
+        tma_load_2d(sBT + 16384, &tmBT, BAR(5), 64, prow);
+        tma_load_2d(sBK, &tmBK, BAR(5), 0, prow);
+      }
+    }
+  } else if (warp == kSiluWarpsB + 1) {
+    // ---------------- tcgen05 issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t id_ss = make_idesc_f16kind(128, 128, 0, 0, F16);
+      constexpr uint32_t id_kmn = make_idesc_f16kind(128, 64, 0, 1, F16);
+      constexpr uint32_t id_mnmn = make_idesc_f16kind(128, 64, 1, 1, F16);
+      bool ok = mbar_wait(BAR(0), 0, abort_flag, ctl);
+      for (int s = 0; ok && s < nsteps; ++s) {
+        const int st = s & 1;
+        if (!mbar_wait(BAR(1 + st), (s >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sQ = sQ0 + st * 32768, sDO = sQ + 16384;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_f16_ss(tS, make_sdesc_sw128(sK + kk * 32, 16, 1024), make_sdesc_sw128(sQ + kk * 32, 16, 1024), id_ss,
+                      kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_f16_ss(tDA, make_sdesc_sw128(sV + kk * 32, 16, 1024), make_sdesc_sw128(sDO + kk * 32, 16, 1024),
+                      id_ss, kk > 0 ? 1u : 0u);
+        umma_commit(BAR(7));
+        if (!mbar_wait(BAR(8), s & 1, abort_flag, ctl)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)   // dV += P^T dO
+          umma_f16_ts(tDV, tS + 64 * (kk >> 2) + 8 * (kk & 3), make_sdesc_sw128(sDO + kk * 2048, 16384, 1024),
+                      id_kmn, (s > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)   // dK += dX^T Q
+          umma_f16_ss(tDK, make_sdesc_sw128(sDX + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                      make_sdesc_sw128(sQ + kk * 2048, 16384, 1024), id_kmn, (s > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)   // dQ_tile = dX K
+          umma_f16_ss(tDQ, make_sdesc_sw128(sDX + kk * 2048, 16384, 1024),
+                      make_sdesc_sw128(sK + kk * 2048, 16384, 1024), id_mnmn, kk > 0 ? 1u : 0u);
+        umma_commit(BAR(9));
+        umma_commit(BAR(3 + st));
+      }
+      if (ok) umma_commit(BAR(10));
+    }
+  } else {
+    // ---------------- elementwise warps ----------------
+    const int quad = warp & 3;
+    const int hq = warp >> 2;             // queries [64 hq, 64 hq + 64)
+    const int rj = quad * 32 + lane;      // key row == TMEM lane of S^T, dA^T, dV, dK
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const bool key_ok = kt * kQTile + rj < n;
+    const float inv_N = a.inv_N;
+    int cur_b = -1;
+    float acc_t = 0.0f;
+    bool ok = true;
+    auto flush_dq = [&](int s_prev) {
+      // dQ tile of query tile kt + s_prev: TMEM lane = query row, columns [32 hq, 32 hq + 32)
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tDQ + lane_base + 32 * hq, v);
+      tmem_ld_wait();
+      const int qi = (kt + s_prev) * kQTile + quad * 32 + lane;
+      if (qi < n) {
+        float4* dst = reinterpret_cast<float4*>(A.dq + (seq0 + qi) * A.ld_g + h * kD + 32 * hq);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          atomicAdd(dst + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                         __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+      }
+    };
+    for (int s = 0; ok && s < nsteps; ++s) {
+      const int qt = kt + s;
+      const bool diag = (s == 0);
+      if (!mbar_wait(BAR(5), s & 1, abort_flag, ctl) || !mbar_wait(BAR(7), s & 1, abort_flag, ctl)) {
+        ok = false;
+        break;
+      }
+      if (s >= 1) {
+        if (!mbar_wait(BAR(9), (s - 1) & 1, abort_flag, ctl)) { ok = false; break; }
+        tc_fence_after();
+        flush_dq(s - 1);
+      }
+      tc_fence_after();
+      float* dpos = s_dpos + 256 * (s & 1);
+#pragma unroll 1
+      for (int hc = 0; hc < 2; ++hc) {
+        uint32_t sv[32], dav[32];
+        tmem_ld_32x32b_x32(tS + lane_base + 64 * hq + 32 * hc, sv);
+        tmem_ld_32x32b_x32(tDA + lane_base + 64 * hq + 32 * hc, dav);
+        // bias^T (chunk hq, row rj, units 4 hc .. 4 hc + 3) and buckets (row rj, units 4 hq + 2 hc + {0,1})
+        uint32_t hb[16], bk[8];
+        {
+          const uint8_t* brow = smem + Lb::kBT + hq * 16384 + rj * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 w = *reinterpret_cast<const uint4*>(brow + (((4 * hc + q) ^ (rj & 7)) << 4));
+            hb[4 * q] = w.x; hb[4 * q + 1] = w.y; hb[4 * q + 2] = w.z; hb[4 * q + 3] = w.w;
+          }
+          const uint8_t* krow_b = smem + Lb::kBK + rj * 128;
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint4 w = *reinterpret_cast<const uint4*>(krow_b + (((4 * hq + 2 * hc + q) ^ (rj & 7)) << 4));
+            bk[4 * q] = w.x; bk[4 * q + 1] = w.y; bk[4 * q + 2] = w.z; bk[4 * q + 3] = w.w;
+          }
+        }
+        tmem_ld_wait();
+        uint32_t pp[16], dxp[16];
+#pragma unroll
+        for (int e2 = 0; e2 < 16; ++e2) {
+          const float2 hbf = unpack_f16x2(hb[e2]);
+          float pv[2], dv2[2];
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            const int e = 2 * e2 + x;
+            const int ci = 64 * hq + 32 * hc + e;   // query column in the tile
+            const bool valid = (qt * kQTile + ci < n) && (!diag || ci >= rj);
+            const float xs = __uint_as_float(sv[e]) + 2.0f * (x ? hbf.y : hbf.x);
+            const float sg = fmaf(0.5f, tanh_f32_approx(0.5f * xs), 0.5f);
+            const float av = xs * sg;
+            const float gp = fmaf(av, 1.0f - sg, sg);
+            const float dx = valid ? __uint_as_float(dav[e]) * gp * inv_N : 0.0f;
+            pv[x] = valid ? av : 0.0f;
+            dv2[x] = dx;
+            atomicAdd(dpos + (ci - rj + 127), dx);
+            const int bkt = static_cast<int>((bk[e >> 2] >> (8 * (e & 3))) & 0xFFu);
+            if (bkt != cur_b) {
+              if (acc_t != 0.0f) atomicAdd(s_dtime + cur_b, acc_t);
+              acc_t = 0.0f;
+              cur_b = bkt;
+            }
+            acc_t += dx;
+          }
+          pp[e2] = F16 ? pack_f16x2(pv[0], pv[1]) : pack_bf16x2(pv[0], pv[1]);
+          dxp[e2] = F16 ? pack_f16x2(dv2[0], dv2[1]) : pack_bf16x2(dv2[0], dv2[1]);
+        }
+        tmem_st_32x32b_x16(tS + lane_base + 64 * hq + 16 * hc, pp);
+        uint8_t* drow = smem + Lb::kDX + hq * 16384 + rj * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(drow + (((4 * hc + q) ^ (rj & 7)) << 4)) =
+              make_uint4(dxp[4 * q], dxp[4 * q + 1], dxp[4 * q + 2], dxp[4 * q + 3]);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(6));    // bias / bucket stage read
+      mbar_arrive(BAR(8));    // P^T in TMEM, dX^T in shared memory
+      // flush this query tile's position-gradient window
+      mbar_arrive(BAR(11));
+      if (!mbar_wait(BAR(11), s & 1, abort_flag, ctl)) { ok = false; break; }
+      const int t = tid;     // elementwise threads are 0..255
+      if (t < 255) {
+        const float v = dpos[t];
+        if (v != 0.0f) {
+          const long long rel = static_cast<long long>(s) * kQTile + t - 127;
+          atomicAdd(A.drab_pos + pos_index_b(rel, a.pos_max_len), v);
+        }
+        dpos[t] = 0.0f;
+      }
+    }
+    if (ok && nsteps > 0 && mbar_wait(BAR(9), (nsteps - 1) & 1, abort_flag, ctl)) {
+      tc_fence_after();
+      flush_dq(nsteps - 1);
+    }
+    if (ok && mbar_wait(BAR(10), 0, abort_flag, ctl)) {
+      tc_fence_after();
+      uint32_t vk[32], vv[32];
+      tmem_ld_32x32b_x32(tDK + lane_base + 32 * hq, vk);
+      tmem_ld_32x32b_x32(tDV + lane_base + 32 * hq, vv);
+      tmem_ld_wait();
+      if (key_ok) {
+        const long long row = seq0 + kt * kQTile + rj;
+        float4* dk = reinterpret_cast<float4*>(A.dk + row * A.ld_g + h * kD + 32 * hq);
+        float4* dvp = reinterpret_cast<float4*>(A.dv + row * A.ld_g + h * kD + 32 * hq);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          dk[q] = make_float4(__uint_as_float(vk[4 * q]), __uint_as_float(vk[4 * q + 1]),
+                              __uint_as_float(vk[4 * q + 2]), __uint_as_float(vk[4 * q + 3]));
+          dvp[q] = make_float4(__uint_as_float(vv[4 * q]) * inv_N, __uint_as_float(vv[4 * q + 1]) * inv_N,
+                               __uint_as_float(vv[4 * q + 2]) * inv_N, __uint_as_float(vv[4 * q + 3]) * inv_N);
+        }
+      }
+    }
+    if (acc_t != 0.0f) atomicAdd(s_dtime + cur_b, acc_t);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  for (int t = tid; t < a.n_buckets; t += kThreadsB)
+    if (s_dtime[t] != 0.0f) atomicAdd(A.drab_time + t, s_dtime[t]);
+}
+
+}  // namespace
+
+cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
+  const AttnArgs& a = A.f;
+  cudaError_t e = upload_time_octaves();
+  if (e != cudaSuccess) return e;
+  if (a.T == 0 || a.capacity == 0) return cudaSuccess;
+  const int mt = (a.max_len + kQTile - 1) / kQTile;
+  if (mt == 0) return cudaSuccess;
+  attn_bias_t_kernel<<<dim3(static_cast<unsigned>(a.capacity), static_cast<unsigned>(mt), 4), 256, 0, st>>>(A);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap tq, tk, tv, tdo, tbt, tbk;
+  const bool f16 = a.in_f16 != 0;
+  const int64_t W = static_cast<int64_t>(a.H) * kD;
+  if (!encode_tmap_2d_bf16(&tq, a.q, W, a.T, a.ld_q, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tk, a.k, W, a.T, a.ld_k, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tv, a.v, W, a.T, a.ld_v, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tdo, A.dout, W, a.T, A.ld_do, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tbt, A.bias_t, kQTile, a.max_pairs * kQTile, kQTile, 64, 128, true) ||
+      !encode_tmap_2d_u8(&tbk, A.bucket_t, kQTile, a.max_pairs * kQTile, kQTile, 128, 128))
+    return cudaErrorInvalidValue;
+  auto kern = f16 ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
+  e = ensure_smem_attr(reinterpret_cast<const void*>(kern), BwdSmem::kTotal);
+  if (e != cudaSuccess) return e;
+  const long long blocks = a.capacity * a.H;
+  kern<<<static_cast<unsigned>(blocks), kThreadsB, BwdSmem::kTotal, st>>>(tq, tk, tv, tdo, tbt, tbk, A,
+                                                                          wait_ctl(a.status));
+  return cudaGetLastError();
+}
+
+}  // namespace hstu

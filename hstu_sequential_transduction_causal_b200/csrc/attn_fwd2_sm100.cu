@@ -81,20 +81,20 @@ attn_bias_kernel(AttnArgs a) {
   for (int e = tid; e < 63 * 4; e += 256) s_oct[e / 4][e % 4] = c_time_octaves[e / 4][e % 4];
   __syncthreads();
 
-  const int r = tid >> 1;        // query row within the tile
-  const int c = tid & 1;         // key half
+  const int r = blockIdx.z * 32 + (tid >> 3);   // query row within the tile (32 rows per block)
+  const int cg = tid & 7;                        // 16 keys [16 cg, 16 cg + 16)
   const int qi = qt * kQTile + r;
   const long long t_i = a.ts[seq0 + (qi < n ? qi : n - 1)];
-  uint16_t* dst = reinterpret_cast<uint16_t*>(a.bias) + (pair * kQTile + r) * kQTile + 64 * c;
-#pragma unroll 1
-  for (int u = 0; u < 8; ++u) {
+  uint16_t* dst = reinterpret_cast<uint16_t*>(a.bias) + (pair * kQTile + r) * kQTile + 16 * cg;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
     uint32_t w[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       float v2[2];
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        const int col = 64 * c + 8 * u + 2 * e + x;
+        const int col = 16 * cg + 8 * u + 2 * e + x;
         const int bkt = time_bucket_dev(t_i - s_kts[col], s_oct, nb);
         v2[x] = 0.5f * (s_win[r - col + 127] + s_rt[bkt]);
       }
@@ -363,7 +363,7 @@ template <bool F16, int G>
 cudaError_t launch_attn2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tb,
                          const AttnArgs& a, cudaStream_t st) {
   auto kern = attn_fwd_tc2_kernel<F16, G>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem2<G>::kTotal);
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), Smem2<G>::kTotal);
   if (e != cudaSuccess) return e;
   const long long blocks = a.capacity * (a.H / G);
   kern<<<static_cast<unsigned>(blocks), kThreads2, Smem2<G>::kTotal, st>>>(tq, tk, tv, tb, a, wait_ctl(a.status));
@@ -383,7 +383,7 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  attn_bias_kernel<<<dim3(static_cast<unsigned>(a.capacity), static_cast<unsigned>(mt)), 256, 0, st>>>(a);
+  attn_bias_kernel<<<dim3(static_cast<unsigned>(a.capacity), static_cast<unsigned>(mt), 4), 256, 0, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv, tb;

@@ -339,7 +339,7 @@ cudaError_t attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t st) {
       !encode_tmap_2d_bf16(&tv, a.v, static_cast<int64_t>(a.H) * kD, a.T, a.ld_v, 64, 128, f16))
     return cudaErrorInvalidValue;
   auto kern = f16 ? attn_fwd_tc_kernel<true> : attn_fwd_tc_kernel<false>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnSmem::kTotal);
+  e = ensure_smem_attr(reinterpret_cast<const void*>(kern), AttnSmem::kTotal);
   if (e != cudaSuccess) return e;
   const long long blocks = a.capacity * a.H;
   kern<<<static_cast<unsigned>(blocks), kThreads, AttnSmem::kTotal, st>>>(tq, tk, tv, a, wait_ctl(a.status));

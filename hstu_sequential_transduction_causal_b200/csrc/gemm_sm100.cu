@@ -325,7 +325,7 @@ cudaError_t launch_tc(const GemmArgs& g, cudaStream_t st) {
     if (!encode_tmap_2d_bf16(&tmB, g.B, g.N, g.K, g.ldb, 64, 64, g.f16)) return cudaErrorInvalidValue;
   }
   auto kern = gemm_bf16_tc_kernel<BN, STAGES, A_MN, B_MN>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kTotal);
   if (e != cudaSuccess) return e;
   const int num_kb = static_cast<int>((g.K + kBK - 1) / kBK);
   const int splits = g.splits < 1 ? 1 : g.splits;

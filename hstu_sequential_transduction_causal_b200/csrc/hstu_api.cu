@@ -69,6 +69,24 @@ AttnWs attn_ws_layout(const hstu_jagged_t* j) {
 
 size_t attn_ws_bytes(const hstu_jagged_t* j) { return attn_ws_layout(j).total; }
 
+// attention-backward workspace: the forward layout up to pair_base, then the key-tile work list,
+// the transposed fp16 bias tiles (32 KB per pair) and the u8 bucket tiles (16 KB per pair).
+struct AttnBwdWs {
+  AttnWs f;
+  size_t kitems, bias_t, bucket_t, total;
+};
+
+AttnBwdWs attn_bwd_ws_layout(const hstu_jagged_t* j) {
+  AttnBwdWs w{};
+  w.f = attn_ws_layout(j);
+  const int64_t cap = capacity_of(j);
+  w.kitems = w.f.bias;   // the forward bias region is not used by the backward
+  w.bias_t = align_up(w.kitems + align_up(static_cast<size_t>(cap) * 8, 256), 1024);
+  w.bucket_t = w.bias_t + static_cast<size_t>(w.f.max_pairs) * kQTile * kQTile * 2;
+  w.total = w.bucket_t + static_cast<size_t>(w.f.max_pairs) * kQTile * kQTile;
+  return w;
+}
+
 hstu_status_t check_jagged(const hstu_jagged_t* j) {
   if (!j || j->B < 0 || j->T < 0 || j->max_len < 0) return HSTU_ERR_INVALID_ARG;
   if (!j->offsets) return HSTU_ERR_INVALID_ARG;
@@ -189,6 +207,40 @@ bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int6
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld_bytes,
+                       int box_inner, int box_outer) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn || !aligned16(base) || inner <= 0 || outer <= 0 || ld_bytes % 16) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t ensure_smem_attr(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static const void* done[256];
+  static int done_dev[256];
+  static int n_done = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i] == kernel && done_dev[i] == dev) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && n_done < 256) {
+    done[n_done] = kernel;
+    done_dev[n_done] = dev;
+    ++n_done;
+  }
+  return e;
+}
+
 }  // namespace hstu
 
 using namespace hstu;
@@ -286,6 +338,63 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
   if (is_tc_dtype(desc->dtype) && jag->T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)))
     return HSTU_ERR_UNSUPPORTED;
   return run_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, ws, stream);
+}
+
+size_t hstu_attn_bwd_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag) {
+  (void)desc;
+  if (check_jagged(jag) != HSTU_OK) return 0;
+  return attn_bwd_ws_layout(jag).total;
+}
+
+hstu_status_t hstu_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const void* q, const void* k,
+                            const void* v, const void* d_out, const float* rab_pos, const float* rab_time, float* dq,
+                            float* dk, float* dv, float* d_rab_pos, float* d_rab_time, void* ws, size_t ws_bytes,
+                            hstu_stream_t stream) {
+  hstu_status_t s = check_attn(desc, jag);
+  if (s != HSTU_OK) return s;
+  if (!is_tc_dtype(desc->dtype)) return HSTU_ERR_UNSUPPORTED;
+  if (!ws) return HSTU_ERR_INVALID_ARG;
+  const AttnBwdWs lay = attn_bwd_ws_layout(jag);
+  if (ws_bytes < lay.total) return HSTU_ERR_WORKSPACE;
+  if (!d_rab_pos || !d_rab_time) return HSTU_ERR_INVALID_ARG;
+  cudaStream_t st = stream;
+  const int64_t W = static_cast<int64_t>(desc->H) * desc->d_qk;
+  cudaError_t e = cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (2 * static_cast<size_t>(desc->pos_max_len) - 1), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, sizeof(float) * desc->n_time_buckets, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (jag->T == 0) return HSTU_OK;
+  if (!q || !k || !v || !d_out || !rab_pos || !rab_time || !dq || !dk || !dv) return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_out) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return HSTU_ERR_UNSUPPORTED;
+  e = cudaMemsetAsync(dq, 0, sizeof(float) * static_cast<size_t>(jag->T) * W, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  AttnBwdArgs A{};
+  AttnArgs& a = A.f;
+  int32_t* count = reinterpret_cast<int32_t*>(w + kWsHeader);
+  int32_t* kcount = count + 1;
+  int32_t* items = reinterpret_cast<int32_t*>(w + lay.f.items);
+  a.B = jag->B; a.T = jag->T; a.max_len = jag->max_len; a.offsets = jag->offsets; a.ts = jag->timestamps;
+  a.H = desc->H; a.dqk = desc->d_qk; a.dv = desc->d_v; a.inv_N = desc->inv_N; a.pos_max_len = desc->pos_max_len;
+  a.n_buckets = desc->n_time_buckets;
+  a.q = q; a.ld_q = desc->ld_q; a.k = k; a.ld_k = desc->ld_k; a.v = v; a.ld_v = desc->ld_v;
+  a.in_f16 = desc->dtype == HSTU_F16;
+  a.rab_pos = rab_pos; a.rab_time = rab_time; a.items = items; a.count = count; a.capacity = capacity_of(jag);
+  a.status = ws_status(ws);
+  a.pair_base = reinterpret_cast<const long long*>(w + lay.f.pairs);
+  a.max_pairs = lay.f.max_pairs;
+  A.dout = d_out; A.ld_do = desc->ld_o;
+  A.dq = dq; A.dk = dk; A.dv = dv; A.ld_g = W;
+  A.drab_pos = d_rab_pos; A.drab_time = d_rab_time;
+  A.bias_t = w + lay.bias_t; A.bucket_t = w + lay.bucket_t;
+  A.kitems = reinterpret_cast<int32_t*>(w + lay.kitems); A.kcount = kcount;
+  e = launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, a.status, st,
+                      reinterpret_cast<long long*>(w + lay.f.pairs));
+  if (e == cudaSuccess)
+    e = launch_bwd_worklist(jag->offsets, jag->B, count, reinterpret_cast<int32_t*>(w + lay.kitems), kcount, st);
+  if (e == cudaSuccess) e = attn_bwd_tc(A, st);
+  return cuda_status(e);
 }
 
 hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t o_dtype, hstu_dtype_t u_dtype,

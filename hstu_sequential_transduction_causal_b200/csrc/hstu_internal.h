@@ -55,6 +55,12 @@ struct GemmArgs {
 // 2D tensor map of a 2-byte element matrix (bf16, or fp16 when f16), 128-byte swizzle.
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t outer,
                          int64_t ld_elems, int box_inner, int box_outer, bool f16 = false);
+// 2D tensor map of a u8 matrix, 128-byte swizzle (box_inner * 1 byte <= 128).
+bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld_bytes,
+                       int box_inner, int box_outer);
+
+// Sets a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t ensure_smem_attr(const void* kernel, int bytes);
 
 cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st);
 cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
@@ -98,6 +104,22 @@ struct AttnArgs {
   void* bias;                   // fp16 [max_pairs, 128, 128] bias tiles (tile-pair kernel)
   int64_t max_pairs;
 };
+
+struct AttnBwdArgs {
+  AttnArgs f;                  // forward arguments (q, k, v, tables, work list with pair_base)
+  const void* dout; int64_t ld_do;   // upstream gradient of O, same dtype as q
+  float* dq; float* dk; float* dv;   // fp32 [T, H*64], dq accumulated (must be zero on entry)
+  int64_t ld_g;                      // row stride of dq, dk, dv
+  float* drab_pos; float* drab_time; // accumulated (must be zero on entry)
+  void* bias_t;                // fp16 [max_pairs, 128 keys, 128 queries] half-bias, transposed
+  void* bucket_t;              // u8   [max_pairs, 128 keys, 128 queries] time bucket, transposed
+  const int32_t* kitems;       // backward work list (b, key tile)
+  const int32_t* kcount;
+};
+
+cudaError_t launch_bwd_worklist(const int64_t* offsets, int B, const int32_t* fwd_count, int32_t* items,
+                                int32_t* count, cudaStream_t st);
+cudaError_t attn_bwd_tc(const AttnBwdArgs& a, cudaStream_t st);
 
 // Bound on the number of causal (query tile, key tile) pairs of a batch.
 int64_t attn_max_pairs(int64_t capacity, int max_len);

@@ -75,6 +75,9 @@ SIGNATURES = {
     "hstu_attn_workspace_size": (c_sz, [P(hstu_attn_desc_t), P(hstu_jagged_t)]),
     "hstu_attn_fwd": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                               c_vp, c_sz, c_vp]),
+    "hstu_attn_bwd_workspace_size": (c_sz, [P(hstu_attn_desc_t), P(hstu_jagged_t)]),
+    "hstu_attn_bwd": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                              c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "hstu_attn_fwd_noalloc": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                       c_vp]),
     "hstu_norm_gate_fwd": (c_i32, [c_i64, c_i32, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp,
@@ -218,6 +221,18 @@ def hstu_attn_workspace_size(desc: hstu_attn_desc_t, jag: hstu_jagged_t) -> int:
 def hstu_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, ws, stream=None) -> None:
     _check("hstu_attn_fwd", lib().hstu_attn_fwd(ctypes.byref(desc), ctypes.byref(jag), _ptr(q), _ptr(k), _ptr(v),
                                                 _ptr(rab_pos), _ptr(rab_time), _ptr(out), _ptr(ws),
+                                                ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def hstu_attn_bwd_workspace_size(desc: hstu_attn_desc_t, jag: hstu_jagged_t) -> int:
+    return lib().hstu_attn_bwd_workspace_size(ctypes.byref(desc), ctypes.byref(jag))
+
+
+def hstu_attn_bwd(desc, jag, q, k, v, d_out, rab_pos, rab_time, dq, dk, dv, d_rab_pos, d_rab_time, ws,
+                  stream=None) -> None:
+    _check("hstu_attn_bwd", lib().hstu_attn_bwd(ctypes.byref(desc), ctypes.byref(jag), _ptr(q), _ptr(k), _ptr(v),
+                                                _ptr(d_out), _ptr(rab_pos), _ptr(rab_time), _ptr(dq), _ptr(dk),
+                                                _ptr(dv), _ptr(d_rab_pos), _ptr(d_rab_time), _ptr(ws),
                                                 ws.numel() * ws.element_size(), _stream(stream)))
 
 

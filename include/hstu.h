@@ -217,6 +217,22 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
                             const float* rab_time, void* out, void* ws, size_t ws_bytes,
                             hstu_stream_t stream);
 
+/* Workspace bytes hstu_attn_bwd needs for this batch. */
+size_t hstu_attn_bwd_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag);
+
+/* Pointwise causal attention backward (derived from the forward's definition; tensor-core dtypes
+ * F16 / BF16 only). With x_ij = q_i.k_j + rab(i, j) and A_ij = SiLU(x_ij) inv_N on causal pairs:
+ * dv = A^T dout, dq = dX k, dk = dX^T q with dX_ij = (dout_i . v_j) SiLU'(x_ij) inv_N, and
+ * d_rab_pos / d_rab_time receive the sum over heads of dX_ij at the entry each pair reads.
+ * q, k, v, d_out: desc->dtype with strides ld_q, ld_k, ld_v, ld_o. dq, dk, dv: fp32 [T, H*64],
+ * row stride H*64, overwritten. d_rab_pos [2L-1], d_rab_time [nb]: fp32, overwritten. Gradients
+ * are accumulated with atomics, so their summation order (and last bits) may differ run to run. */
+hstu_status_t hstu_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag,
+                            const void* q, const void* k, const void* v, const void* d_out,
+                            const float* rab_pos, const float* rab_time, float* dq, float* dk,
+                            float* dv, float* d_rab_pos, float* d_rab_time, void* ws,
+                            size_t ws_bytes, hstu_stream_t stream);
+
 /* Largest number of (sequence, 128-row tile) work items, B + ceil(T / 128), that
  * hstu_attn_fwd_noalloc accepts. */
 #define HSTU_NOALLOC_MAX_ITEMS 65536
