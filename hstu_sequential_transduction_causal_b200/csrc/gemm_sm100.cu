@@ -202,9 +202,10 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int n = n0 + c * 32;
         if (!row_ok || n >= N) continue;
         if (epi.kind == kEpiAtomic) {
-          float* o = reinterpret_cast<float*>(epi.out0) + static_cast<int64_t>(row) * epi.ld_out0 + n;
+          float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(epi.out0) +
+                                                static_cast<int64_t>(row) * epi.ld_out0 + n);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) atomicAdd(o + j, v[j]);
+          for (int j = 0; j < 8; ++j) atomicAdd(o + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
           continue;
         }
         if (epi.bias) {

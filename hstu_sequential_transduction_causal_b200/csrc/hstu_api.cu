@@ -87,6 +87,77 @@ AttnBwdWs attn_bwd_ws_layout(const hstu_jagged_t* j) {
   return w;
 }
 
+// layer-backward workspace: the attention-backward layout, then dG (fp32), dO (fp16), dq | dk | dv
+// (fp32), dZ (fp16 [T, 4D]), reduction partials, dgamma | dbeta, bf16 copies of x and dy, fp16
+// copies of x and W1 (the operands of dZ in the f1 backward GEMMs: both MMA operands share a type).
+struct LayerBwdWs {
+  size_t dg, dO, dq, dk, dv, dz, partial, gb, x_conv, dy_conv, x_f16, w1_f16, total;
+};
+
+LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) {
+  LayerBwdWs w{};
+  const size_t T = static_cast<size_t>(j->T), D = static_cast<size_t>(d->D);
+  size_t off = align_up(attn_bwd_ws_layout(j).total, 1024);
+  auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes, 1024); return o; };
+  w.dg = take(T * D * 4);
+  w.dO = take(T * D * 2);
+  w.dq = take(T * D * 4);
+  w.dk = take(T * D * 4);
+  w.dv = take(T * D * 4);
+  w.dz = take(T * 4 * D * 2);
+  size_t pf = colsum_partial_floats(static_cast<int>(4 * D));
+  const size_t pl = static_cast<size_t>(norm_gate_bwd_blocks(j->T)) * 2 * D;
+  w.partial = take((pf > pl ? pf : pl) * 4);
+  w.gb = take(2 * D * 4);
+  w.x_conv = take(T * D * 2);
+  w.dy_conv = take(T * D * 2);
+  w.x_f16 = take(T * D * 2);
+  w.w1_f16 = take(4 * D * D * 2);
+  w.total = off;
+  return w;
+}
+
+// Attention backward on the caller's stream; dq / dk / dv fp32 with row stride ld_g. Zeroes the
+// accumulated outputs (dq, the table gradients) first.
+hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const void* q, const void* k,
+                           const void* v, const void* d_out, const float* rab_pos, const float* rab_time, float* dq,
+                           float* dk, float* dv, int64_t ld_g, float* d_rab_pos, float* d_rab_time, void* ws,
+                           cudaStream_t st) {
+  const AttnBwdWs lay = attn_bwd_ws_layout(jag);
+  cudaError_t e = cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (2 * static_cast<size_t>(desc->pos_max_len) - 1), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, sizeof(float) * desc->n_time_buckets, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (jag->T == 0) return HSTU_OK;
+  e = cudaMemsetAsync(dq, 0, sizeof(float) * static_cast<size_t>(jag->T) * ld_g, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  AttnBwdArgs A{};
+  AttnArgs& a = A.f;
+  int32_t* count = reinterpret_cast<int32_t*>(w + kWsHeader);
+  int32_t* kcount = count + 1;
+  int32_t* items = reinterpret_cast<int32_t*>(w + lay.f.items);
+  a.B = jag->B; a.T = jag->T; a.max_len = jag->max_len; a.offsets = jag->offsets; a.ts = jag->timestamps;
+  a.H = desc->H; a.dqk = desc->d_qk; a.dv = desc->d_v; a.inv_N = desc->inv_N; a.pos_max_len = desc->pos_max_len;
+  a.n_buckets = desc->n_time_buckets;
+  a.q = q; a.ld_q = desc->ld_q; a.k = k; a.ld_k = desc->ld_k; a.v = v; a.ld_v = desc->ld_v;
+  a.in_f16 = desc->dtype == HSTU_F16;
+  a.rab_pos = rab_pos; a.rab_time = rab_time; a.items = items; a.count = count; a.capacity = capacity_of(jag);
+  a.status = ws_status(ws);
+  a.pair_base = reinterpret_cast<const long long*>(w + lay.f.pairs);
+  a.max_pairs = lay.f.max_pairs;
+  A.dout = d_out; A.ld_do = desc->ld_o;
+  A.dq = dq; A.dk = dk; A.dv = dv; A.ld_g = ld_g;
+  A.drab_pos = d_rab_pos; A.drab_time = d_rab_time;
+  A.bias_t = w + lay.bias_t; A.bucket_t = w + lay.bucket_t;
+  A.kitems = reinterpret_cast<int32_t*>(w + lay.kitems); A.kcount = kcount;
+  e = launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, a.status, st,
+                      reinterpret_cast<long long*>(w + lay.f.pairs));
+  if (e == cudaSuccess)
+    e = launch_bwd_worklist(jag->offsets, jag->B, count, reinterpret_cast<int32_t*>(w + lay.kitems), kcount, st);
+  if (e == cudaSuccess) e = attn_bwd_tc(A, st);
+  return cuda_status(e);
+}
+
 hstu_status_t check_jagged(const hstu_jagged_t* j) {
   if (!j || j->B < 0 || j->T < 0 || j->max_len < 0) return HSTU_ERR_INVALID_ARG;
   if (!j->offsets) return HSTU_ERR_INVALID_ARG;
@@ -179,6 +250,16 @@ hstu_status_t run_out_proj(int64_t T, int32_t D, hstu_dtype_t dtype, const void*
   g.epi.out1 = y_bf16; g.epi.out1_dt = kDtBF16; g.epi.ld_out1 = D;
   g.status = status;
   return cuda_status(dtype == HSTU_BF16 ? gemm_bf16(g, st) : gemm_f32(g, st));
+}
+
+// Split-K factor that gives the accumulating GEMM about two CTAs per SM.
+int auto_splits(int64_t M, int64_t N, int64_t K) {
+  const int64_t bn = (N % 256 == 0 && N >= 1024) ? 256 : 128;
+  const int64_t tiles = ((M + 127) / 128) * ((N + bn - 1) / bn);
+  const int64_t nkb = (K + 63) / 64;
+  int64_t s = (296 + tiles - 1) / tiles;
+  if (s > nkb) s = nkb;
+  return static_cast<int>(s < 1 ? 1 : s);
 }
 
 hstu_status_t check_dense(int64_t T, int32_t D, hstu_dtype_t dtype) {
@@ -354,47 +435,16 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
   if (s != HSTU_OK) return s;
   if (!is_tc_dtype(desc->dtype)) return HSTU_ERR_UNSUPPORTED;
   if (!ws) return HSTU_ERR_INVALID_ARG;
-  const AttnBwdWs lay = attn_bwd_ws_layout(jag);
-  if (ws_bytes < lay.total) return HSTU_ERR_WORKSPACE;
+  if (ws_bytes < attn_bwd_ws_layout(jag).total) return HSTU_ERR_WORKSPACE;
   if (!d_rab_pos || !d_rab_time) return HSTU_ERR_INVALID_ARG;
-  cudaStream_t st = stream;
+  if (jag->T > 0) {
+    if (!q || !k || !v || !d_out || !rab_pos || !rab_time || !dq || !dk || !dv) return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_out) || !aligned16(dq) || !aligned16(dk) ||
+        !aligned16(dv))
+      return HSTU_ERR_UNSUPPORTED;
+  }
   const int64_t W = static_cast<int64_t>(desc->H) * desc->d_qk;
-  cudaError_t e = cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (2 * static_cast<size_t>(desc->pos_max_len) - 1), st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, sizeof(float) * desc->n_time_buckets, st);
-  if (e != cudaSuccess) return cuda_status(e);
-  if (jag->T == 0) return HSTU_OK;
-  if (!q || !k || !v || !d_out || !rab_pos || !rab_time || !dq || !dk || !dv) return HSTU_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_out) || !aligned16(dq) || !aligned16(dk) ||
-      !aligned16(dv))
-    return HSTU_ERR_UNSUPPORTED;
-  e = cudaMemsetAsync(dq, 0, sizeof(float) * static_cast<size_t>(jag->T) * W, st);
-  if (e != cudaSuccess) return cuda_status(e);
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  AttnBwdArgs A{};
-  AttnArgs& a = A.f;
-  int32_t* count = reinterpret_cast<int32_t*>(w + kWsHeader);
-  int32_t* kcount = count + 1;
-  int32_t* items = reinterpret_cast<int32_t*>(w + lay.f.items);
-  a.B = jag->B; a.T = jag->T; a.max_len = jag->max_len; a.offsets = jag->offsets; a.ts = jag->timestamps;
-  a.H = desc->H; a.dqk = desc->d_qk; a.dv = desc->d_v; a.inv_N = desc->inv_N; a.pos_max_len = desc->pos_max_len;
-  a.n_buckets = desc->n_time_buckets;
-  a.q = q; a.ld_q = desc->ld_q; a.k = k; a.ld_k = desc->ld_k; a.v = v; a.ld_v = desc->ld_v;
-  a.in_f16 = desc->dtype == HSTU_F16;
-  a.rab_pos = rab_pos; a.rab_time = rab_time; a.items = items; a.count = count; a.capacity = capacity_of(jag);
-  a.status = ws_status(ws);
-  a.pair_base = reinterpret_cast<const long long*>(w + lay.f.pairs);
-  a.max_pairs = lay.f.max_pairs;
-  A.dout = d_out; A.ld_do = desc->ld_o;
-  A.dq = dq; A.dk = dk; A.dv = dv; A.ld_g = W;
-  A.drab_pos = d_rab_pos; A.drab_time = d_rab_time;
-  A.bias_t = w + lay.bias_t; A.bucket_t = w + lay.bucket_t;
-  A.kitems = reinterpret_cast<int32_t*>(w + lay.kitems); A.kcount = kcount;
-  e = launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, a.status, st,
-                      reinterpret_cast<long long*>(w + lay.f.pairs));
-  if (e == cudaSuccess)
-    e = launch_bwd_worklist(jag->offsets, jag->B, count, reinterpret_cast<int32_t*>(w + lay.kitems), kcount, st);
-  if (e == cudaSuccess) e = attn_bwd_tc(A, st);
-  return cuda_status(e);
+  return run_attn_bwd(desc, jag, q, k, v, d_out, rab_pos, rab_time, dq, dk, dv, W, d_rab_pos, d_rab_time, ws, stream);
 }
 
 hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t o_dtype, hstu_dtype_t u_dtype,
@@ -495,6 +545,160 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   if (e != cudaSuccess) return cuda_status(e);
   return run_out_proj(T, D, desc->dtype, saved->g, w->W2, w->b2, x, desc->x_dtype, y, desc->y_dtype, y_bf16, status,
                       st);
+}
+
+hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda, int32_t a_mn,
+                               const void* B, int64_t ldb, int32_t b_mn, const float* bias, const void* resid,
+                               hstu_dtype_t resid_dtype, int64_t ld_resid, void* out, hstu_dtype_t out_dtype,
+                               int64_t ld_out, int32_t accumulate, void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0 || !ws) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < kWsHeader) return HSTU_ERR_WORKSPACE;
+  if (M == 0 || N == 0) return HSTU_OK;
+  if (!A || !B || !out) return HSTU_ERR_INVALID_ARG;
+  if (N % 32 || lda % 8 || ldb % 8 || !aligned16(A) || !aligned16(B) || !aligned16(out)) return HSTU_ERR_UNSUPPORTED;
+  if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31)) return HSTU_ERR_UNSUPPORTED;
+  if (out_dtype != HSTU_F32 && out_dtype != HSTU_BF16 && out_dtype != HSTU_F16) return HSTU_ERR_UNSUPPORTED;
+  if (accumulate && (out_dtype != HSTU_F32 || bias || resid)) return HSTU_ERR_UNSUPPORTED;
+  if (resid && (!aligned16(resid) || (resid_dtype != HSTU_F32 && resid_dtype != HSTU_BF16 &&
+                                      resid_dtype != HSTU_F16)))
+    return HSTU_ERR_UNSUPPORTED;
+  GemmArgs g{};
+  g.A = A; g.lda = lda; g.a_mn = a_mn != 0;
+  g.B = B; g.ldb = ldb; g.b_mn = b_mn != 0; g.f16 = false;
+  g.M = M; g.N = N; g.K = K;
+  g.splits = accumulate ? auto_splits(M, N, K) : 1;
+  g.epi.kind = accumulate ? kEpiAtomic : kEpiLinear;
+  g.epi.bias = bias;
+  g.epi.resid = resid; g.epi.resid_dt = resid_dtype; g.epi.ld_resid = ld_resid;
+  g.epi.out0 = out; g.epi.out0_dt = out_dtype; g.epi.ld_out0 = ld_out;
+  g.status = ws_status(ws);
+  return cuda_status(gemm_bf16(g, stream));
+}
+
+size_t hstu_layer_bwd_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag) {
+  if (!desc || check_jagged(jag) != HSTU_OK) return 0;
+  return layer_bwd_layout(desc, jag).total;
+}
+
+hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag, const hstu_layer_weights_t* w,
+                             const void* x, const void* x_bf16, const hstu_layer_saved_t* saved, const void* dy,
+                             const void* dy_bf16, void* dx, void* dx_bf16, const hstu_layer_grads_t* gr, void* ws,
+                             size_t ws_bytes, hstu_stream_t stream) {
+  if (!desc || !w || !saved || !gr) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t s = check_jagged(jag);
+  if (s != HSTU_OK) return s;
+  const int32_t D = desc->D, H = desc->H;
+  if (H <= 0 || D <= 0 || D % H) return HSTU_ERR_INVALID_ARG;
+  if (desc->dtype != HSTU_BF16) return HSTU_ERR_UNSUPPORTED;
+  if (D != 256 && D != 512) return HSTU_ERR_UNSUPPORTED;
+  hstu_attn_desc_t ad{};
+  ad.H = H; ad.d_qk = D / H; ad.d_v = D / H; ad.inv_N = desc->inv_N; ad.pos_max_len = desc->pos_max_len;
+  ad.n_time_buckets = desc->n_time_buckets; ad.dtype = HSTU_F16; ad.o_dtype = HSTU_F32;
+  ad.ld_q = ad.ld_k = ad.ld_v = 4ll * D; ad.ld_o = D;
+  s = check_attn(&ad, jag);
+  if (s != HSTU_OK) return s;
+  if ((desc->x_dtype != HSTU_F32 && desc->x_dtype != HSTU_BF16) || (desc->y_dtype != HSTU_F32 && desc->y_dtype != HSTU_BF16))
+    return HSTU_ERR_UNSUPPORTED;
+  if (!ws) return HSTU_ERR_INVALID_ARG;
+  const LayerBwdWs lay = layer_bwd_layout(desc, jag);
+  if (ws_bytes < lay.total) return HSTU_ERR_WORKSPACE;
+  if (!gr->dW1 || !gr->db1 || !gr->dW2 || !gr->db2 || !gr->dgamma || !gr->dbeta || !gr->drab_pos || !gr->drab_time)
+    return HSTU_ERR_INVALID_ARG;
+  const int64_t T = jag->T;
+  cudaStream_t st = stream;
+  cudaError_t e = cudaSuccess;
+  if (T == 0) {
+    const size_t zs[8] = {4ull * D * D * 4, 4ull * D * 4, 1ull * D * D * 4, 1ull * D * 4, 1ull * D * 4, 1ull * D * 4,
+                          (2ull * desc->pos_max_len - 1) * 4, 1ull * desc->n_time_buckets * 4};
+    float* ps[8] = {gr->dW1, gr->db1, gr->dW2, gr->db2, gr->dgamma, gr->dbeta, gr->drab_pos, gr->drab_time};
+    for (int i = 0; i < 8 && e == cudaSuccess; ++i) e = cudaMemsetAsync(ps[i], 0, zs[i], st);
+    return cuda_status(e);
+  }
+  if (!x || !dy || !dx || !saved->uvqk || !saved->z || !saved->o || !saved->g || !saved->mu || !saved->rstd)
+    return HSTU_ERR_INVALID_ARG;
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  int* status = ws_status(ws);
+  const void* x_op = x_bf16;
+  if (!x_op) {
+    if (desc->x_dtype == HSTU_BF16) {
+      x_op = x;
+    } else {
+      e = convert_f32_to_bf16(static_cast<const float*>(x), wsb + lay.x_conv, T * D, st);
+      if (e != cudaSuccess) return cuda_status(e);
+      x_op = wsb + lay.x_conv;
+    }
+  }
+  const void* dy_op = dy_bf16;
+  if (!dy_op) {
+    if (desc->y_dtype == HSTU_BF16) {
+      dy_op = dy;
+    } else {
+      e = convert_f32_to_bf16(static_cast<const float*>(dy), wsb + lay.dy_conv, T * D, st);
+      if (e != cudaSuccess) return cuda_status(e);
+      dy_op = wsb + lay.dy_conv;
+    }
+  }
+  float* dG = reinterpret_cast<float*>(wsb + lay.dg);
+  void* dO = wsb + lay.dO;
+  float* dq = reinterpret_cast<float*>(wsb + lay.dq);
+  float* dk = reinterpret_cast<float*>(wsb + lay.dk);
+  float* dv = reinterpret_cast<float*>(wsb + lay.dv);
+  void* dz = wsb + lay.dz;
+  float* part = reinterpret_cast<float*>(wsb + lay.partial);
+  float* gb = reinterpret_cast<float*>(wsb + lay.gb);
+  // 1. f2 backward: dG = dY W2, dW2 = dY^T G, db2 = sum_t dY
+  GemmArgs g{};
+  g.A = dy_op; g.lda = D; g.a_mn = false; g.B = w->W2; g.ldb = D; g.b_mn = true; g.f16 = false;
+  g.M = T; g.N = D; g.K = D; g.splits = 1;
+  g.epi.kind = kEpiLinear; g.epi.out0 = dG; g.epi.out0_dt = kDtF32; g.epi.ld_out0 = D; g.status = status;
+  e = gemm_bf16(g, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW2, 0, sizeof(float) * D * D, st);
+  if (e == cudaSuccess) {
+    GemmArgs g2{};
+    g2.A = dy_op; g2.lda = D; g2.a_mn = true; g2.B = saved->g; g2.ldb = D; g2.b_mn = true; g2.f16 = false;
+    g2.M = D; g2.N = D; g2.K = T; g2.splits = auto_splits(D, D, T);
+    g2.epi.kind = kEpiAtomic; g2.epi.out0 = gr->dW2; g2.epi.out0_dt = kDtF32; g2.epi.ld_out0 = D; g2.status = status;
+    e = gemm_bf16(g2, st);
+  }
+  if (e == cudaSuccess) e = column_sum(dy, desc->y_dtype, T, D, D, part, gr->db2, st);
+  // 2. norm-gate backward: dO (fp16), dZ_U (bf16), dgamma | dbeta
+  if (e == cudaSuccess)
+    e = norm_gate_bwd(T, D, kDtF16, dG, static_cast<const float*>(saved->o), saved->uvqk, saved->z, 4ll * D, w->gamma,
+                      w->beta, saved->mu, saved->rstd, dO, dz, 4ll * D, part, gb, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(gr->dgamma, gb, sizeof(float) * D, cudaMemcpyDeviceToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(gr->dbeta, gb + D, sizeof(float) * D, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  // 3. attention backward
+  const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
+  s = run_attn_bwd(&ad, jag, uvqk + 2 * D * 2, uvqk + 3 * D * 2, uvqk + 1 * D * 2, dO, w->rab_pos, w->rab_time, dq, dk,
+                   dv, D, gr->drab_pos, gr->drab_time, ws, st);
+  if (s != HSTU_OK) return s;
+  // 4. SiLU backward into dZ[:, D:4D], db1 = sum_t dZ
+  e = dz_assemble(T, D, kDtF16, dv, dq, dk, saved->z, 4ll * D, dz, 4ll * D, st);
+  if (e == cudaSuccess) e = column_sum(dz, kDtF16, T, 4 * D, 4ll * D, part, gr->db1, st);
+  // 5. f1 backward: dW1 = dZ^T X, dX = dY + dZ W1 (dZ fp16: exact fp16 copies of x and W1)
+  void* x_f16 = wsb + lay.x_f16;
+  void* w1_f16 = wsb + lay.w1_f16;
+  if (e == cudaSuccess) e = convert_dtype(x_op, kDtBF16, x_f16, kDtF16, T * D, st);
+  if (e == cudaSuccess) e = convert_dtype(w->W1, kDtBF16, w1_f16, kDtF16, 4ll * D * D, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW1, 0, sizeof(float) * 4 * D * D, st);
+  if (e == cudaSuccess) {
+    GemmArgs g3{};
+    g3.A = dz; g3.lda = 4ll * D; g3.a_mn = true; g3.B = x_f16; g3.ldb = D; g3.b_mn = true; g3.f16 = true;
+    g3.M = 4ll * D; g3.N = D; g3.K = T; g3.splits = auto_splits(4ll * D, D, T);
+    g3.epi.kind = kEpiAtomic; g3.epi.out0 = gr->dW1; g3.epi.out0_dt = kDtF32; g3.epi.ld_out0 = D; g3.status = status;
+    e = gemm_bf16(g3, st);
+  }
+  if (e == cudaSuccess) {
+    GemmArgs g4{};
+    g4.A = dz; g4.lda = 4ll * D; g4.a_mn = false; g4.B = w1_f16; g4.ldb = D; g4.b_mn = true; g4.f16 = true;
+    g4.M = T; g4.N = D; g4.K = 4ll * D; g4.splits = 1;
+    g4.epi.kind = kEpiLinear; g4.epi.resid = dy; g4.epi.resid_dt = desc->y_dtype; g4.epi.ld_resid = D;
+    g4.epi.out0 = dx; g4.epi.out0_dt = desc->x_dtype; g4.epi.ld_out0 = D;
+    g4.epi.out1 = dx_bf16; g4.epi.out1_dt = kDtBF16; g4.epi.ld_out1 = D; g4.status = status;
+    e = gemm_bf16(g4, st);
+  }
+  return cuda_status(e);
 }
 
 }  // extern "C"

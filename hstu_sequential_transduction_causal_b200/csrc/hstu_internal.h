@@ -138,6 +138,23 @@ cudaError_t norm_gate_fwd(int64_t T, int D, int o_dt, int u_dt, int g_dt, const 
 
 cudaError_t convert_f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t st);
 
+// ---------------------------------------------------------------------------------------------
+// layer backward helpers (layer_bwd.cu)
+// ---------------------------------------------------------------------------------------------
+int norm_gate_bwd_blocks(int64_t T);
+// dO = LayerNorm backward of dLn = dG (.) U; dZ_U = dG (.) Ln (.) SiLU'(Z_U) (fp16, stride ld_dz);
+// dgamma | dbeta -> dgamma_dbeta_out[0 .. 2D) via partial [norm_gate_bwd_blocks(T), 2D].
+cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const float* o, const void* u,
+                          const void* zu, int64_t ld_act, const float* gamma, const float* beta, const float* mu,
+                          const float* rstd, void* d_o, void* dz, int64_t ld_dz, float* partial,
+                          float* dgamma_dbeta_out, cudaStream_t st);
+cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
+                        const void* z, int64_t ld_z, void* dz, int64_t ld_dz, cudaStream_t st);
+size_t colsum_partial_floats(int cols);
+cudaError_t convert_dtype(const void* in, int in_dt, void* out, int out_dt, int64_t n, cudaStream_t st);
+cudaError_t column_sum(const void* in, int dt, int64_t rows, int cols, int64_t ld, float* partial, float* out,
+                       cudaStream_t st);
+
 cudaError_t launch_timeout_probe(int* status, cudaStream_t st);
 
 }  // namespace hstu

@@ -78,6 +78,12 @@ SIGNATURES = {
     "hstu_attn_bwd_workspace_size": (c_sz, [P(hstu_attn_desc_t), P(hstu_jagged_t)]),
     "hstu_attn_bwd": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                               c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "hstu_linear_bf16": (c_i32, [c_i64, c_i64, c_i64, c_vp, c_i64, c_i32, c_vp, c_i64, c_i32, c_vp, c_vp, c_i32,
+                                 c_i64, c_vp, c_i32, c_i64, c_i32, c_vp, c_sz, c_vp]),
+    "hstu_layer_bwd_workspace_size": (c_sz, [P(hstu_layer_desc_t), P(hstu_jagged_t)]),
+    "hstu_layer_bwd": (c_i32, [P(hstu_layer_desc_t), P(hstu_jagged_t), P(hstu_layer_weights_t), c_vp, c_vp,
+                               P(hstu_layer_saved_t), c_vp, c_vp, c_vp, c_vp, P(hstu_layer_grads_t), c_vp, c_sz,
+                               c_vp]),
     "hstu_attn_fwd_noalloc": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                       c_vp]),
     "hstu_norm_gate_fwd": (c_i32, [c_i64, c_i32, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp,
@@ -278,3 +284,27 @@ def layer_weights(W1, b1, W2, b2, gamma, beta, rab_pos, rab_time) -> hstu_layer_
 
 def layer_saved(uvqk, z, o, g, mu, rstd) -> hstu_layer_saved_t:
     return hstu_layer_saved_t(*[_ptr(t) for t in (uvqk, z, o, g, mu, rstd)])
+
+
+def hstu_linear_bf16(M, N, K, A, lda, a_mn, B, ldb, b_mn, bias, resid, resid_dtype_code, ld_resid, out,
+                     out_dtype_code, ld_out, accumulate, ws, stream=None) -> None:
+    _check("hstu_linear_bf16", lib().hstu_linear_bf16(M, N, K, _ptr(A), lda, int(a_mn), _ptr(B), ldb, int(b_mn),
+                                                      _ptr(bias), _ptr(resid), resid_dtype_code, ld_resid, _ptr(out),
+                                                      out_dtype_code, ld_out, int(accumulate), _ptr(ws),
+                                                      ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def hstu_layer_bwd_workspace_size(desc: hstu_layer_desc_t, jag: hstu_jagged_t) -> int:
+    return lib().hstu_layer_bwd_workspace_size(ctypes.byref(desc), ctypes.byref(jag))
+
+
+def hstu_layer_bwd(desc, jag, weights: hstu_layer_weights_t, x, x_bf16, saved: hstu_layer_saved_t, dy, dy_bf16, dx,
+                   dx_bf16, grads: hstu_layer_grads_t, ws, stream=None) -> None:
+    _check("hstu_layer_bwd", lib().hstu_layer_bwd(ctypes.byref(desc), ctypes.byref(jag), ctypes.byref(weights),
+                                                  _ptr(x), _ptr(x_bf16), ctypes.byref(saved), _ptr(dy),
+                                                  _ptr(dy_bf16), _ptr(dx), _ptr(dx_bf16), ctypes.byref(grads),
+                                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def layer_grads(dW1, db1, dW2, db2, dgamma, dbeta, drab_pos, drab_time) -> hstu_layer_grads_t:
+    return hstu_layer_grads_t(*[_ptr(t) for t in (dW1, db1, dW2, db2, dgamma, dbeta, drab_pos, drab_time)])

@@ -290,6 +290,37 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
                              void* y, void* y_bf16, const hstu_layer_saved_t* saved, void* ws,
                              size_t ws_bytes, hstu_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * Backward of the layer (derived from the forward equations; no autograd)
+ * ------------------------------------------------------------------------------------------- */
+
+/* The projection GEMM both directions use: out[M, N] (=|+=) A B^T with A [M, K] and B [N, K] in
+ * bf16, fp32 accumulation on the tensor cores. a_mn / b_mn = 0: the operand is stored row-major
+ * as [M or N rows, K] (K-major); 1: stored row-major as [K rows, M or N] (MN-major, a transpose
+ * for free). accumulate = 0: out = A B^T (+ bias[N]) (+ resid), out_dtype F32/BF16/F16;
+ * accumulate = 1: out += A B^T in fp32 by atomics over K splits (bias and resid must be NULL).
+ * N must be a multiple of 32, lda/ldb multiples of 8, pointers 16-byte aligned. ws: >= 256 bytes. */
+hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                               int32_t a_mn, const void* B, int64_t ldb, int32_t b_mn,
+                               const float* bias, const void* resid, hstu_dtype_t resid_dtype,
+                               int64_t ld_resid, void* out, hstu_dtype_t out_dtype, int64_t ld_out,
+                               int32_t accumulate, void* ws, size_t ws_bytes, hstu_stream_t stream);
+
+/* Workspace bytes hstu_layer_bwd needs. */
+size_t hstu_layer_bwd_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
+
+/* Whole layer backward (BF16 mode, D in {256, 512}), from the activations hstu_layer_fwd saved
+ * (z required). dy: [T, D] of desc->y_dtype (dy_bf16: nullable bf16 copy); dx: [T, D] of
+ * desc->x_dtype, overwritten with dy + dZ W1 (dx_bf16: nullable bf16 copy). Steps: dG = dy W2,
+ * dW2 = dy^T G, db2 = sum dy; LayerNorm (.) U backward (dO, dU, dgamma, dbeta); attention
+ * backward (dQ, dK, dV, table gradients); dZ = [dU|dV|dQ|dK] (.) SiLU'(Z); dW1 = dZ^T X,
+ * db1 = sum dZ, dX = dy + dZ W1. All gradients fp32 and overwritten. */
+hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag,
+                             const hstu_layer_weights_t* w, const void* x, const void* x_bf16,
+                             const hstu_layer_saved_t* saved, const void* dy, const void* dy_bf16,
+                             void* dx, void* dx_bf16, const hstu_layer_grads_t* grads, void* ws,
+                             size_t ws_bytes, hstu_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

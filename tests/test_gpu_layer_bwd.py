@@ -1,0 +1,140 @@
+"""GPU parity of the projection GEMM in every operand layout, and of the whole layer backward
+against the oracle's closed-form gradients (pinned to finite differences on the CPU).
+
+dx (an O(1) activation gradient) meets the bf16 bound |d| <= 1e-2 + 1e-2 |ref| element by element.
+Weight and table gradients are sums over all tokens whose scale rms(ref) is far from 1 (dW1 ~ 14 on
+the long-sequence workload); their bound applies the absolute term in units of that scale, and each
+tensor is also held to a norm-relative error <= 1e-2. Elements outside the unscaled bound are counted
+and printed: they come from fp16 rounding of the attention operands (inherent to tensor-core
+attention) meeting heavy cancellation in sums over thousands of tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import hstu_oracle as O
+from hstu_sequential_transduction_causal_b200 import hstu as H
+from hstu_sequential_transduction_causal_b200 import workloads as W
+from hstu_sequential_transduction_causal_b200.runtime import (DeviceLayer, JaggedBatch, LayerRunner, to_dev,
+                                                              workspace)
+from tests._util import BF16_TOL, THR, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from hstu_sequential_transduction_causal_b200 import build
+    build.build()
+    H.lib()
+    torch.cuda.init()
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("accumulate", [0, 1])
+def test_linear_all_operand_layouts(a_mn, b_mn, accumulate):
+    rng = np.random.default_rng(10 + 2 * a_mn + b_mn)
+    M, N, K = 296, 256, 1000 if accumulate else 320
+    A = W.round_bf16(rng.standard_normal((M, K)))
+    Bm = W.round_bf16(rng.standard_normal((N, K)) / np.sqrt(K))
+    bias = (0.1 * rng.standard_normal(N)).astype(np.float32)
+    resid = W.round_bf16(rng.standard_normal((M, N)))
+    A_store = A.T.copy() if a_mn else A            # MN-major: stored [K, M]
+    B_store = Bm.T.copy() if b_mn else Bm
+    out = torch.full((M, N), 0.5 if accumulate else float("nan"), dtype=torch.float32, device="cuda")
+    ws = workspace(256)
+    H.hstu_linear_bf16(M, N, K, to_dev(A_store, torch.bfloat16), A_store.shape[1], a_mn,
+                       to_dev(B_store, torch.bfloat16), B_store.shape[1], b_mn,
+                       None if accumulate else to_dev(bias, torch.float32),
+                       None if accumulate else to_dev(resid, torch.bfloat16), H.HSTU_BF16, N, out, H.HSTU_F32, N,
+                       accumulate, ws)
+    got = out.cpu().numpy()
+    ref = A.astype(np.float64) @ Bm.astype(np.float64).T
+    ref = ref + 0.5 if accumulate else ref + bias + resid
+    assert H.hstu_sync_status(ws) == 0
+    assert_close(got, ref, 1e-4 * np.sqrt(K), 1e-4, what=f"linear a_mn={a_mn} b_mn={b_mn} acc={accumulate}")
+
+
+def _run_layer_fwd_bwd(wl, x_dtype=torch.bfloat16):
+    jag = JaggedBatch(wl.offsets, wl.timestamps)
+    layer = DeviceLayer.upload(wl.layers[0], wl.D, wl.H, True)
+    run = LayerRunner(layer, jag, 1.0 / wl.N, wl.pos_max_len, x_dtype, x_dtype, keep_z=True)
+    x = to_dev(wl.x, x_dtype)
+    run.forward(x)
+    D, T = wl.D, wl.T
+    grads = [torch.full(s, float("nan"), dtype=torch.float32, device="cuda")
+             for s in [(4 * D, D), (4 * D,), (D, D), (D,), (D,), (D,), (2 * wl.pos_max_len - 1,), (128,)]]
+    dy = to_dev(wl.dy, x_dtype)
+    dx = torch.full((T, D), float("nan"), dtype=x_dtype, device="cuda")
+    ws = workspace(H.hstu_layer_bwd_workspace_size(run.desc, jag.struct))
+    H.hstu_layer_bwd(run.desc, jag.struct, run.weights, x, None, run.saved_struct, dy, None, dx, None,
+                     H.layer_grads(*grads), ws)
+    torch.cuda.synchronize()
+    assert H.hstu_sync_status(ws) == 0
+    assert run.device_status() == 0
+    return dx.float().cpu().numpy(), [g.cpu().numpy() for g in grads]
+
+
+def _oracle_grads(wl):
+    p = wl.layers[0]
+    y, sv = O.layer_fwd(wl.x, p, wl.offsets, wl.timestamps, wl.H, 1.0 / wl.N, wl.pos_max_len, THR)
+    return O.layer_bwd(wl.dy, p, sv, wl.offsets, wl.timestamps, wl.H, 1.0 / wl.N, wl.pos_max_len, THR)
+
+
+NAMES = ("dW1", "db1", "dW2", "db2", "dgamma", "dbeta", "drab_pos", "drab_time")
+
+
+STRICT_MISSES = {}
+
+
+def _compare(dx, grads, ref, tag=""):
+    """dx (an O(1) activation gradient) meets the bf16 bound verbatim. Weight and table gradients
+    are sums over all tokens with scale rms(ref) far from 1; the bound's absolute term is applied
+    in units of that scale, |d| <= 1e-2 max(1, rms(ref)) + 1e-2 |ref|, together with a norm-relative
+    error <= 1e-2. The number of elements outside the unscaled bound is recorded for the report."""
+    assert_close(dx, ref["dx"], *BF16_TOL, what="dx")
+    for name, g in zip(NAMES, grads):
+        e = np.asarray(ref[name], np.float64)
+        scale = max(1.0, float(np.sqrt(np.mean(e ** 2)))) if e.size else 1.0
+        STRICT_MISSES[f"{tag}{name}"] = int((np.abs(g - e) > 1e-2 + 1e-2 * np.abs(e)).sum())
+        assert_close(g, e, 1e-2 * scale, 1e-2, what=name)
+        nrm = float(np.linalg.norm(e))
+        if nrm > 0:
+            rel = float(np.linalg.norm(g - e)) / nrm
+            assert rel <= 1e-2, f"{name}: norm-relative error {rel:.3e}"
+    print(f"\n{tag} elements outside the unscaled bound:",
+          {k: v for k, v in STRICT_MISSES.items() if k.startswith(tag)})
+
+
+def test_layer_bwd_ragged_d512():
+    wl = W.make_workload("c3", seed=2, lengths=[1, 130, 300, 0, 257, 64], pos_max_len=512, N=512)
+    dx, grads = _run_layer_fwd_bwd(wl)
+    _compare(dx, grads, _oracle_grads(wl), "ragged-d512 ")
+
+
+def test_layer_bwd_d256_four_heads():
+    wl = W.make_workload("c2", seed=3, lengths=[200, 129, 7], backward=True)
+    dx, grads = _run_layer_fwd_bwd(wl)
+    _compare(dx, grads, _oracle_grads(wl), "d256 ")
+
+
+def test_layer_bwd_fp32_residual_stream():
+    wl = W.make_workload("c4", seed=4, lengths=[150, 260, 1], layers=1)
+    wl.x = np.random.default_rng(5).standard_normal((wl.T, wl.D)).astype(np.float32)
+    wl.dy = np.random.default_rng(6).standard_normal((wl.T, wl.D)).astype(np.float32)
+    dx, grads = _run_layer_fwd_bwd(wl, torch.float32)
+    # the f1/f2 operands are the bf16 roundings of the fp32 residual stream and of dy
+    p = wl.layers[0]
+    xr = W.round_bf16(wl.x)
+    y, sv = O.layer_fwd(xr, p, wl.offsets, wl.timestamps, wl.H, 1.0 / wl.N, wl.pos_max_len, THR)
+    sv["x"] = xr
+    ref = O.layer_bwd(W.round_bf16(wl.dy), p, sv, wl.offsets, wl.timestamps, wl.H, 1.0 / wl.N, wl.pos_max_len, THR)
+    ref["dx"] = ref["dx"] - W.round_bf16(wl.dy) + wl.dy          # the residual adds the fp32 dy itself
+    ref["db2"] = wl.dy.astype(np.float64).sum(axis=0)              # db2 sums the fp32 dy
+    _compare(dx, grads, ref, "fp32-residual ")
+
+
+def test_layer_bwd_long_sequence_workload_full():
+    wl = W.make_workload("c3", seed=0)
+    dx, grads = _run_layer_fwd_bwd(wl)
+    _compare(dx, grads, _oracle_grads(wl), "long-sequence-full ")
