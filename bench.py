@@ -259,10 +259,11 @@ def main():
         H.hstu_attn_fwd(adesc, jag.struct, sv.uvqk[:, 2 * D:], sv.uvqk[:, 3 * D:], sv.uvqk[:, D:], layer.rab_pos,
                         layer.rab_time, sv.o, ws)
         rec(2)
-        H.hstu_norm_gate_fwd(T, D, H.HSTU_F32, H.HSTU_F16, H.HSTU_BF16, sv.o, D, sv.uvqk, 4 * D, layer.gamma,
+        H.hstu_norm_gate_fwd(T, D, H.HSTU_F32, H.HSTU_F16, H.HSTU_F16, sv.o, D, sv.uvqk, 4 * D, layer.gamma,
                              layer.beta, 1e-5, sv.g, sv.mu, sv.rstd)
         rec(3)
-        H.hstu_out_proj_fwd(T, D, H.HSTU_BF16, sv.g, layer.W2, layer.b2, x, H.HSTU_BF16, y, H.HSTU_BF16, None, ws)
+        H.hstu_out_proj_fwd(T, D, H.HSTU_BF16, H.HSTU_F16, sv.g, layer.W2, layer.b2, x, H.HSTU_BF16, y, H.HSTU_BF16,
+                            None, ws)
         rec(4)
         if backward:
             H.hstu_layer_bwd(ldesc, jag.struct, weights, x, None, svs, dy, None, dx, None, grads, ws)
@@ -373,7 +374,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": WORKLOADS[args.workload]["desc"], "global_batch": wl.B * world,
                        "tokens_per_rank": T, "seq_len": "jagged", "parallelism": f"dp{world}",
-                       "attention_operands": "fp16 U|V|Q|K and P, fp32 accumulation and O",
+                       "attention_operands": "fp16 U|V|Q|K, P and G, fp32 accumulation and O",
                        "l2": "flushed (512 MB write) before every timed step"},
             "roofline": {"bound": "tensor", "kernel": "jagged attention forward (bias tiles + attn_fwd_tc2_kernel)",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,

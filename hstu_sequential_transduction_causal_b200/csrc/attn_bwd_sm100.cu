@@ -37,6 +37,8 @@ constexpr int kD = 64;
 constexpr int kSiluWarpsB = 8;
 constexpr int kThreadsB = 32 * (kSiluWarpsB + 2);
 constexpr int kSiluThreadsB = 32 * kSiluWarpsB;
+constexpr uint32_t kHalf2HalfB = 0x38003800u;       // (0.5, 0.5) in fp16
+constexpr uint32_t kHalf2MinusHalfB = 0xB800B800u;  // (-0.5, -0.5)
 
 __device__ __forceinline__ int pos_index_b(long long r, int L) {
   r = r > L - 1 ? L - 1 : r;
@@ -63,7 +65,7 @@ attn_bias_t_kernel(AttnBwdArgs A) {
   __shared__ long long s_qts[128];
   __shared__ float s_win[256];
   __shared__ float s_rt[128];
-  __shared__ long long s_oct[63][4];
+  __shared__ long long s_tau[kTauEntries];
   const int tid = threadIdx.x;
   const int L = a.pos_max_len;
   const int nb = a.n_buckets;
@@ -76,7 +78,7 @@ attn_bias_t_kernel(AttnBwdArgs A) {
     const long long rel0 = static_cast<long long>(qt - kt) * kQTile - 127;
     if (tid < 255) s_win[tid] = a.rab_pos[pos_index_b(rel0 + tid, L)];
   }
-  for (int e = tid; e < 63 * 4; e += 256) s_oct[e / 4][e % 4] = c_time_octaves[e / 4][e % 4];
+  for (int e = tid; e < kTauEntries; e += 256) s_tau[e] = c_time_taus[e];
   __syncthreads();
 
   const int j = blockIdx.z * 32 + (tid >> 3);   // key row within the tile
@@ -96,7 +98,7 @@ attn_bias_t_kernel(AttnBwdArgs A) {
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
         const int col = 16 * cg + 8 * u + 2 * e + x;
-        k2[x] = time_bucket_dev(s_qts[col] - t_j, s_oct, nb);
+        k2[x] = time_bucket_dev(s_qts[col] - t_j, s_tau, nb);
         v2[x] = 0.5f * (s_win[col - j + 127] + s_rt[k2[x]]);
       }
       w[e] = pack_f16x2(v2[0], v2[1]);
@@ -114,16 +116,18 @@ attn_bias_t_kernel(AttnBwdArgs A) {
 // backward kernel
 // ----------------------------------------------------------------------------------------------
 struct BwdSmem {
-  static constexpr int kK = 0;
-  static constexpr int kV = 16384;
-  static constexpr int kQ0 = 32768;          // stage st: Q at kQ0 + st * 32768, dO at +16384
-  static constexpr int kBT = kQ0 + 2 * 32768;   // bias^T: 2 chunks of 64 queries
-  static constexpr int kBK = kBT + 32768;       // bucket^T: 128 x 128 bytes
-  static constexpr int kDX = kBK + 16384;       // dX^T: 2 chunks of 64 queries
-  static constexpr int kHist = kDX + 32768;     // dtime[128] | dpos[2][256]
-  static constexpr int kBar = kHist + 512 + 2048;
+  static constexpr int kK = 0;                  // K tile of the CTA (16 KB)
+  static constexpr int kV = 16384;              // V tile (16 KB)
+  static constexpr int kQ0 = 32768;             // stage st: Q at kQ0 + st * 32768, dO at +16384
+  static constexpr int kBT0 = kQ0 + 2 * 32768;  // stage st: half-bias^T, overwritten in place by dX^T
+  static constexpr int kBK0 = kBT0 + 2 * 32768; // stage st: bucket^T (16 KB)
+  static constexpr int kTime = kBK0 + 2 * 16384;   // d rab_time partial sums, one copy per lane [128][32]
+  static constexpr int kPos = kTime + 128 * 32 * 4;  // d rab_pos partial sums of the CTA's diagonals
+  static constexpr int kPosWin = 4352;          // diagonals 128 s + d, -127 <= d <= 127, s <= 32
+  static constexpr int kBar = kPos + kPosWin * 4;
   static constexpr int kTotal = kBar + 256 + 1024;
 };
+static_assert(BwdSmem::kTotal <= 232448, "shared memory of the backward kernel");
 
 template <bool F16>
 __global__ void __launch_bounds__(kThreadsB, 1)
@@ -147,14 +151,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const long long pbase = a.pair_base[b];
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lb::kBar);
-  // 0 kv_full | 1,2 qdo_full | 3,4 qdo_empty | 5 bb_full | 6 bb_empty | 7 s_full | 8 p_ready |
-  // 9 dq_full | 10 fin | 11 group barrier of the elementwise warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  // 0 kv_full | 1,2 qdo_full | 3,4 qdo_empty | 5,6 bb_full | 7,8 bb_empty | 9 s_full | 10 p_ready |
+  // 11 dq_full | 12 fin
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  float* s_dtime = reinterpret_cast<float*>(smem + Lb::kHist);
-  float* s_dpos = s_dtime + 128;   // [2][256]
+  float* s_dtime = reinterpret_cast<float*>(smem + Lb::kTime);
+  float* s_dpos = reinterpret_cast<float*>(smem + Lb::kPos);
+  const int pos_used = min(Lb::kPosWin, 128 * nsteps + 255);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -165,18 +170,18 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(1 + s), 1);
       mbar_init(BAR(3 + s), 1);
+      mbar_init(BAR(5 + s), 1);
+      mbar_init(BAR(7 + s), 1);
     }
-    mbar_init(BAR(5), 1);
-    mbar_init(BAR(6), kSiluThreadsB);
-    mbar_init(BAR(7), 1);
-    mbar_init(BAR(8), kSiluThreadsB);
     mbar_init(BAR(9), 1);
-    mbar_init(BAR(10), 1);
-    mbar_init(BAR(11), kSiluThreadsB);
+    mbar_init(BAR(10), kSiluThreadsB);
+    mbar_init(BAR(11), 1);
+    mbar_init(BAR(12), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  for (int e = tid; e < 128 + 512; e += kThreadsB) s_dtime[e] = 0.0f;
+  for (int e = tid; e < 128 * 32; e += kThreadsB) s_dtime[e] = 0.0f;
+  for (int e = tid; e < pos_used; e += kThreadsB) s_dpos[e] = 0.0f;
   if (warp == kSiluWarpsB && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -197,8 +202,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   const uint32_t sK = smem_u32(smem + Lb::kK), sV = smem_u32(smem + Lb::kV);
   const uint32_t sQ0 = smem_u32(smem + Lb::kQ0);
-  const uint32_t sBT = smem_u32(smem + Lb::kBT), sBK = smem_u32(smem + Lb::kBK);
-  const uint32_t sDX = smem_u32(smem + Lb::kDX);
+  const uint32_t sBT0 = smem_u32(smem + Lb::kBT0), sBK0 = smem_u32(smem + Lb::kBK0);
   const int krow = static_cast<int>(seq0) + kt * kQTile;
 
   if (warp == kSiluWarpsB) {
@@ -209,17 +213,18 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tma_load_2d(sV, &tmV, BAR(0), h * kD, krow);
       for (int s = 0; s < nsteps; ++s) {
         const int qt = kt + s, st = s & 1;
-        if (s >= 2 && !mbar_wait(BAR(3 + st), ((s >> 1) & 1) ^ 1, abort_flag, ctl)) break;
+        const uint32_t ph_free = ((s >> 1) & 1) ^ 1;
+        if (s >= 2 && !mbar_wait(BAR(3 + st), ph_free, abort_flag, ctl)) break;
         const int qrow = static_cast<int>(seq0) + qt * kQTile;
         mbar_arrive_expect_tx(BAR(1 + st), 32768);
         tma_load_2d(sQ0 + st * 32768, &tmQ, BAR(1 + st), h * kD, qrow);
         tma_load_2d(sQ0 + st * 32768 + 16384, &tmDO, BAR(1 + st), h * kD, qrow);
-        if (s >= 1 && !mbar_wait(BAR(6), (s - 1) & 1, abort_flag, ctl)) break;
+        if (s >= 2 && !mbar_wait(BAR(7 + st), ph_free, abort_flag, ctl)) break;
         const int prow = static_cast<int>((pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt) * kQTile);
-        mbar_arrive_expect_tx(BAR(5), 32768 + 16384);
-        tma_load_2d(sBT, &tmBT, BAR(5), 0, prow);
-        tma_load_2d(sBT + 16384, &tmBT, BAR(5), 64, prow);
-        tma_load_2d(sBK, &tmBK, BAR(5), 0, prow);
+        mbar_arrive_expect_tx(BAR(5 + st), 32768 + 16384);
+        tma_load_2d(sBT0 + st * 32768, &tmBT, BAR(5 + st), 0, prow);
+        tma_load_2d(sBT0 + st * 32768 + 16384, &tmBT, BAR(5 + st), 64, prow);
+        tma_load_2d(sBK0 + st * 16384, &tmBK, BAR(5 + st), 0, prow);
       }
     }
   } else if (warp == kSiluWarpsB + 1) {
@@ -234,6 +239,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!mbar_wait(BAR(1 + st), (s >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
         tc_fence_after();
         const uint32_t sQ = sQ0 + st * 32768, sDO = sQ + 16384;
+        const uint32_t sDX = sBT0 + st * 32768;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           umma_f16_ss(tS, make_sdesc_sw128(sK + kk * 32, 16, 1024), make_sdesc_sw128(sQ + kk * 32, 16, 1024), id_ss,
@@ -242,8 +248,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int kk = 0; kk < 4; ++kk)
           umma_f16_ss(tDA, make_sdesc_sw128(sV + kk * 32, 16, 1024), make_sdesc_sw128(sDO + kk * 32, 16, 1024),
                       id_ss, kk > 0 ? 1u : 0u);
-        umma_commit(BAR(7));
-        if (!mbar_wait(BAR(8), s & 1, abort_flag, ctl)) { ok = false; break; }
+        umma_commit(BAR(9));
+        if (!mbar_wait(BAR(10), s & 1, abort_flag, ctl)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)   // dV += P^T dO
@@ -257,10 +263,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int kk = 0; kk < 8; ++kk)   // dQ_tile = dX K
           umma_f16_ss(tDQ, make_sdesc_sw128(sDX + kk * 2048, 16384, 1024),
                       make_sdesc_sw128(sK + kk * 2048, 16384, 1024), id_mnmn, kk > 0 ? 1u : 0u);
-        umma_commit(BAR(9));
+        umma_commit(BAR(11));
         umma_commit(BAR(3 + st));
+        umma_commit(BAR(7 + st));
       }
-      if (ok) umma_commit(BAR(10));
+      if (ok) umma_commit(BAR(12));
     }
   } else {
     // ---------------- elementwise warps ----------------
@@ -271,6 +278,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const bool key_ok = kt * kQTile + rj < n;
     const float inv_N = a.inv_N;
     int cur_b = -1;
+    uint32_t cur_rep = 0xFFFFFFFFu;
     float acc_t = 0.0f;
     bool ok = true;
     auto flush_dq = [&](int s_prev) {
@@ -288,100 +296,147 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
     };
     for (int s = 0; ok && s < nsteps; ++s) {
-      const int qt = kt + s;
-      const bool diag = (s == 0);
-      if (!mbar_wait(BAR(5), s & 1, abort_flag, ctl) || !mbar_wait(BAR(7), s & 1, abort_flag, ctl)) {
+      const int qt = kt + s, st = s & 1;
+      if (!mbar_wait(BAR(5 + st), (s >> 1) & 1, abort_flag, ctl) || !mbar_wait(BAR(9), s & 1, abort_flag, ctl)) {
         ok = false;
         break;
       }
       if (s >= 1) {
-        if (!mbar_wait(BAR(9), (s - 1) & 1, abort_flag, ctl)) { ok = false; break; }
+        if (!mbar_wait(BAR(11), (s - 1) & 1, abort_flag, ctl)) { ok = false; break; }
         tc_fence_after();
         flush_dq(s - 1);
       }
       tc_fence_after();
-      float* dpos = s_dpos + 256 * (s & 1);
+      // masks: the diagonal tile keeps queries >= key; the last query tile keeps queries < n; a key
+      // row past n keeps nothing (it only occurs in the diagonal tile of the last key tile)
+      const bool need_mask = (s == 0) || (qt == nt - 1);
+      const int lo_col = (s == 0) ? rj : 0;
+      const int hi_col = key_ok ? min(kQTile, n - qt * kQTile) : 0;
+      uint8_t* bt_row = smem + Lb::kBT0 + st * 32768 + hq * 16384 + rj * 128;
+      const uint8_t* bk_row = smem + Lb::kBK0 + st * 16384 + rj * 128;
 #pragma unroll 1
       for (int hc = 0; hc < 2; ++hc) {
+        const int c0 = 64 * hq + 32 * hc;   // first query column of the chunk
         uint32_t sv[32], dav[32];
-        tmem_ld_32x32b_x32(tS + lane_base + 64 * hq + 32 * hc, sv);
-        tmem_ld_32x32b_x32(tDA + lane_base + 64 * hq + 32 * hc, dav);
-        // bias^T (chunk hq, row rj, units 4 hc .. 4 hc + 3) and buckets (row rj, units 4 hq + 2 hc + {0,1})
+        tmem_ld_32x32b_x32(tS + lane_base + c0, sv);
+        tmem_ld_32x32b_x32(tDA + lane_base + c0, dav);
         uint32_t hb[16], bk[8];
-        {
-          const uint8_t* brow = smem + Lb::kBT + hq * 16384 + rj * 128;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 w = *reinterpret_cast<const uint4*>(brow + (((4 * hc + q) ^ (rj & 7)) << 4));
-            hb[4 * q] = w.x; hb[4 * q + 1] = w.y; hb[4 * q + 2] = w.z; hb[4 * q + 3] = w.w;
-          }
-          const uint8_t* krow_b = smem + Lb::kBK + rj * 128;
+        for (int q = 0; q < 4; ++q) {
+          const uint4 w = *reinterpret_cast<const uint4*>(bt_row + (((4 * hc + q) ^ (rj & 7)) << 4));
+          hb[4 * q] = w.x; hb[4 * q + 1] = w.y; hb[4 * q + 2] = w.z; hb[4 * q + 3] = w.w;
+        }
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const uint4 w = *reinterpret_cast<const uint4*>(krow_b + (((4 * hq + 2 * hc + q) ^ (rj & 7)) << 4));
-            bk[4 * q] = w.x; bk[4 * q + 1] = w.y; bk[4 * q + 2] = w.z; bk[4 * q + 3] = w.w;
-          }
+        for (int q = 0; q < 2; ++q) {
+          const uint4 w = *reinterpret_cast<const uint4*>(bk_row + (((4 * hq + 2 * hc + q) ^ (rj & 7)) << 4));
+          bk[4 * q] = w.x; bk[4 * q + 1] = w.y; bk[4 * q + 2] = w.z; bk[4 * q + 3] = w.w;
         }
         tmem_ld_wait();
+        // F16: packed fp16 per pair of queries: h = x/2, t = tanh(h), sigma(x) = (1 + t)/2,
+        // P = SiLU(x) = h (1 + t), SiLU'(x) = sigma + P (1 - sigma), dX = dA inv_N SiLU'(x).
+        // BF16 operands (8x coarser P and dX for the MMAs): the same in fp32, rounded once.
         uint32_t pp[16], dxp[16];
+        float xf[32];
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
-          const float2 hbf = unpack_f16x2(hb[e2]);
-          float pv[2], dv2[2];
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            const int e = 2 * e2 + x;
-            const int ci = 64 * hq + 32 * hc + e;   // query column in the tile
-            const bool valid = (qt * kQTile + ci < n) && (!diag || ci >= rj);
-            const float xs = __uint_as_float(sv[e]) + 2.0f * (x ? hbf.y : hbf.x);
-            const float sg = fmaf(0.5f, tanh_f32_approx(0.5f * xs), 0.5f);
-            const float av = xs * sg;
-            const float gp = fmaf(av, 1.0f - sg, sg);
-            const float dx = valid ? __uint_as_float(dav[e]) * gp * inv_N : 0.0f;
-            pv[x] = valid ? av : 0.0f;
-            dv2[x] = dx;
-            atomicAdd(dpos + (ci - rj + 127), dx);
-            const int bkt = static_cast<int>((bk[e >> 2] >> (8 * (e & 3))) & 0xFFu);
-            if (bkt != cur_b) {
-              if (acc_t != 0.0f) atomicAdd(s_dtime + cur_b, acc_t);
-              acc_t = 0.0f;
-              cur_b = bkt;
-            }
-            acc_t += dx;
+          uint32_t m = 0xFFFFFFFFu;
+          if (need_mask) {
+            const int col = c0 + 2 * e2;
+            m = ((col >= lo_col && col < hi_col) ? 0x0000FFFFu : 0u) |
+                ((col + 1 >= lo_col && col + 1 < hi_col) ? 0xFFFF0000u : 0u);
           }
-          pp[e2] = F16 ? pack_f16x2(pv[0], pv[1]) : pack_bf16x2(pv[0], pv[1]);
-          dxp[e2] = F16 ? pack_f16x2(dv2[0], dv2[1]) : pack_bf16x2(dv2[0], dv2[1]);
+          if constexpr (F16) {
+            const uint32_t s2 = pack_f16x2(__uint_as_float(sv[2 * e2]), __uint_as_float(sv[2 * e2 + 1]));
+            const uint32_t h2 = hfma2_u32(s2, kHalf2HalfB, hb[e2]);
+            const uint32_t t2 = tanh_f16x2(h2);
+            const uint32_t p2 = hfma2_u32(h2, t2, h2);
+            const uint32_t sg = hfma2_u32(t2, kHalf2HalfB, kHalf2HalfB);        // sigma
+            const uint32_t osg = hfma2_u32(t2, kHalf2MinusHalfB, kHalf2HalfB);  // 1 - sigma
+            const uint32_t g2 = hfma2_u32(p2, osg, sg);                          // SiLU'(x)
+            const uint32_t da2 =
+                pack_f16x2(__uint_as_float(dav[2 * e2]) * inv_N, __uint_as_float(dav[2 * e2 + 1]) * inv_N);
+            const uint32_t x2 = hmul2_u32(da2, g2) & m;
+            const float2 xv = unpack_f16x2(x2);
+            xf[2 * e2] = xv.x;
+            xf[2 * e2 + 1] = xv.y;
+            pp[e2] = p2 & m;
+            dxp[e2] = x2;
+          } else {
+            const float2 hbf = unpack_f16x2(hb[e2]);
+            float pv[2], dv2[2];
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const float xs = __uint_as_float(sv[2 * e2 + x]) + 2.0f * (x ? hbf.y : hbf.x);
+              const float sg = fmaf(0.5f, tanh_f32_approx(0.5f * xs), 0.5f);
+              const float av = xs * sg;
+              const bool keep = (m >> (16 * x)) & 1u;
+              pv[x] = keep ? av : 0.0f;
+              dv2[x] = keep ? __uint_as_float(dav[2 * e2 + x]) * inv_N * fmaf(av, 1.0f - sg, sg) : 0.0f;
+            }
+            pp[e2] = pack_bf16x2(pv[0], pv[1]);
+            dxp[e2] = pack_bf16x2(dv2[0], dv2[1]);
+            xf[2 * e2] = dv2[0];
+            xf[2 * e2 + 1] = dv2[1];
+          }
         }
         tmem_st_32x32b_x16(tS + lane_base + 64 * hq + 16 * hc, pp);
-        uint8_t* drow = smem + Lb::kDX + hq * 16384 + rj * 128;
+        // dX^T replaces the half-bias just read: same row, same swizzled 16-byte units
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(drow + (((4 * hc + q) ^ (rj & 7)) << 4)) =
+          *reinterpret_cast<uint4*>(bt_row + (((4 * hc + q) ^ (rj & 7)) << 4)) =
               make_uint4(dxp[4 * q], dxp[4 * q + 1], dxp[4 * q + 2], dxp[4 * q + 3]);
+        // d rab_pos: the chunk is a 32x32 block (key rows 32 quad + l, query columns c0 + e); lane L
+        // gathers diagonal e - l = L from lane e - L and diagonal L - 32 from lane e - L + 32
+        {
+          float up = 0.0f, lo = 0.0f;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float v = __shfl_sync(0xffffffffu, xf[e], (e - lane) & 31);
+            if (e >= lane) up += v;
+            else lo += v;
+          }
+          // window index of relative position r = 128 s + (c0 + d) - 32 quad, stored at r + 127
+          const int w_up = 128 * s + c0 - 32 * quad + 127 + lane;
+          const int w_lo = w_up - 32;
+          if (w_up < Lb::kPosWin) atomicAdd(s_dpos + w_up, up);
+          else atomicAdd(A.drab_pos + pos_index_b(w_up - 127, a.pos_max_len), up);
+          if (lane > 0) {
+            if (w_lo < Lb::kPosWin) atomicAdd(s_dpos + w_lo, lo);
+            else atomicAdd(A.drab_pos + pos_index_b(w_lo - 127, a.pos_max_len), lo);
+          }
+        }
+        // d rab_time: runs of equal bucket along the row (4 buckets per word)
+#pragma unroll
+        for (int wq = 0; wq < 8; ++wq) {
+          const uint32_t wd = bk[wq];
+          if (wd == cur_rep) {
+            acc_t += (xf[4 * wq] + xf[4 * wq + 1]) + (xf[4 * wq + 2] + xf[4 * wq + 3]);
+          } else {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const int bkt = static_cast<int>((wd >> (8 * x)) & 0xFFu);
+              if (bkt != cur_b) {
+                // each lane owns a copy of the histogram: lanes of a warp never collide
+                if (acc_t != 0.0f) atomicAdd(s_dtime + cur_b * 32 + lane, acc_t);
+                acc_t = 0.0f;
+                cur_b = bkt;
+                cur_rep = 0x01010101u * static_cast<uint32_t>(bkt);
+              }
+              acc_t += xf[4 * wq + x];
+            }
+          }
+        }
       }
       tmem_st_wait();
       tc_fence_before();
       fence_proxy_async_smem();
-      mbar_arrive(BAR(6));    // bias / bucket stage read
-      mbar_arrive(BAR(8));    // P^T in TMEM, dX^T in shared memory
-      // flush this query tile's position-gradient window
-      mbar_arrive(BAR(11));
-      if (!mbar_wait(BAR(11), s & 1, abort_flag, ctl)) { ok = false; break; }
-      const int t = tid;     // elementwise threads are 0..255
-      if (t < 255) {
-        const float v = dpos[t];
-        if (v != 0.0f) {
-          const long long rel = static_cast<long long>(s) * kQTile + t - 127;
-          atomicAdd(A.drab_pos + pos_index_b(rel, a.pos_max_len), v);
-        }
-        dpos[t] = 0.0f;
-      }
+      mbar_arrive(BAR(10));    // P^T in TMEM, dX^T in shared memory
     }
-    if (ok && nsteps > 0 && mbar_wait(BAR(9), (nsteps - 1) & 1, abort_flag, ctl)) {
+    if (ok && nsteps > 0 && mbar_wait(BAR(11), (nsteps - 1) & 1, abort_flag, ctl)) {
       tc_fence_after();
       flush_dq(nsteps - 1);
     }
-    if (ok && mbar_wait(BAR(10), 0, abort_flag, ctl)) {
+    if (ok && mbar_wait(BAR(12), 0, abort_flag, ctl)) {
       tc_fence_after();
       uint32_t vk[32], vv[32];
       tmem_ld_32x32b_x32(tDK + lane_base + 32 * hq, vk);
@@ -400,7 +455,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
     }
-    if (acc_t != 0.0f) atomicAdd(s_dtime + cur_b, acc_t);
+    if (acc_t != 0.0f) atomicAdd(s_dtime + cur_b * 32 + lane, acc_t);
   }
 
   tc_fence_before();
@@ -409,15 +464,21 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  for (int t = tid; t < a.n_buckets; t += kThreadsB)
-    if (s_dtime[t] != 0.0f) atomicAdd(A.drab_time + t, s_dtime[t]);
+  for (int t = tid; t < a.n_buckets; t += kThreadsB) {
+    float v = 0.0f;
+#pragma unroll 8
+    for (int l = 0; l < 32; ++l) v += s_dtime[t * 32 + ((l + t) & 31)];
+    if (v != 0.0f) atomicAdd(A.drab_time + t, v);
+  }
+  for (int w = tid; w < pos_used; w += kThreadsB)
+    if (s_dpos[w] != 0.0f) atomicAdd(A.drab_pos + pos_index_b(w - 127, a.pos_max_len), s_dpos[w]);
 }
 
 }  // namespace
 
 cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   const AttnArgs& a = A.f;
-  cudaError_t e = upload_time_octaves();
+  cudaError_t e = upload_time_taus();
   if (e != cudaSuccess) return e;
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;

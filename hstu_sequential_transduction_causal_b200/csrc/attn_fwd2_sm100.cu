@@ -65,7 +65,7 @@ attn_bias_kernel(AttnArgs a) {
   __shared__ long long s_kts[128];
   __shared__ float s_win[256];
   __shared__ float s_rt[128];
-  __shared__ long long s_oct[63][4];
+  __shared__ long long s_tau[kTauEntries];
   const int tid = threadIdx.x;
   const int L = a.pos_max_len;
   const int nb = a.n_buckets;
@@ -78,7 +78,7 @@ attn_bias_kernel(AttnArgs a) {
     const long long rel0 = static_cast<long long>(qt - kt) * kQTile - 127;
     if (tid < 255) s_win[tid] = a.rab_pos[pos_index2(rel0 + tid, L)];
   }
-  for (int e = tid; e < 63 * 4; e += 256) s_oct[e / 4][e % 4] = c_time_octaves[e / 4][e % 4];
+  for (int e = tid; e < kTauEntries; e += 256) s_tau[e] = c_time_taus[e];
   __syncthreads();
 
   const int r = blockIdx.z * 32 + (tid >> 3);   // query row within the tile (32 rows per block)
@@ -95,7 +95,7 @@ attn_bias_kernel(AttnArgs a) {
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
         const int col = 16 * cg + 8 * u + 2 * e + x;
-        const int bkt = time_bucket_dev(t_i - s_kts[col], s_oct, nb);
+        const int bkt = time_bucket_dev(t_i - s_kts[col], s_tau, nb);
         v2[x] = 0.5f * (s_win[r - col + 127] + s_rt[bkt]);
       }
       w[e] = pack_f16x2(v2[0], v2[1]);
@@ -116,7 +116,7 @@ struct Smem2 {
   static constexpr int kTotal = kBar + 256 + 1024;
 };
 
-template <bool F16, int G>
+template <bool F16, int G, bool FALCON>
 __global__ void __launch_bounds__(kThreads2, 1)
 attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB, AttnArgs a,
@@ -127,14 +127,24 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const int HG = a.H / G;
   const int item = blockIdx.x / HG;
   const int hg = blockIdx.x - item * HG;
-  if (item >= *a.count) return;
-  const int b = a.items[2 * item];
-  const int qt = a.items[2 * item + 1];
+  int b, qt;
+  if constexpr (FALCON) {
+    // (user, candidate tile): every tile of a user visits all of the user's prefix key tiles
+    const int qpu = (a.cand_rows + kQTile - 1) / kQTile;
+    if (qpu == 0 || item >= a.B * qpu) return;
+    b = item / qpu;
+    qt = item - b * qpu;
+  } else {
+    if (item >= *a.count) return;
+    b = a.items[2 * item];
+    qt = a.items[2 * item + 1];
+  }
   const long long seq0 = a.offsets[b];
   const int n = static_cast<int>(a.offsets[b + 1] - seq0);
-  const int nkt = qt + 1;
+  // FALCON: keys past the bias row (a prefix longer than its contract allows) are not visited
+  const int nkt = FALCON ? max(0, min((n + kQTile - 1) / kQTile, static_cast<int>(a.kbias_ld / kQTile))) : qt + 1;
   const int nsteps = nkt * G;
-  const long long pair0 = a.pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2;
+  const long long pair0 = FALCON ? 0 : a.pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   // 0 q_full | 1..3 kv_full | 4..6 kv_empty | 7,8 b_full | 9,10 b_empty | 11,12 s_full |
@@ -175,7 +185,7 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    tma_prefetch_desc(&tmB);
+    if (!FALCON) tma_prefetch_desc(&tmB);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -189,7 +199,7 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const uint32_t sQ = smem_u32(smem + L::kQ);
   const uint32_t sKV = smem_u32(smem + L::kKV);
   const uint32_t sB = smem_u32(smem + L::kBias);
-  const int qrow0 = static_cast<int>(seq0) + qt * kQTile;
+  const int qrow0 = FALCON ? b * a.cand_rows + qt * kQTile : static_cast<int>(seq0) + qt * kQTile;
 
   if (warp == kSiluWarps) {
     // ---------------- TMA producer ----------------
@@ -199,12 +209,14 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       bool ok = true;
       int s = 0;
       for (int kt = 0; ok && kt < nkt; ++kt) {
-        const int bs = kt & 1;
-        if (kt >= 2 && !mbar_wait(bar_b_empty(bs), ((kt >> 1) & 1) ^ 1, abort_flag, ctl)) break;
-        const int brow = static_cast<int>((pair0 + kt) * kQTile);
-        mbar_arrive_expect_tx(bar_b_full(bs), 32768);
-        tma_load_2d(sB + bs * 32768, &tmB, bar_b_full(bs), 0, brow);
-        tma_load_2d(sB + bs * 32768 + 16384, &tmB, bar_b_full(bs), 64, brow);
+        if constexpr (!FALCON) {
+          const int bs = kt & 1;
+          if (kt >= 2 && !mbar_wait(bar_b_empty(bs), ((kt >> 1) & 1) ^ 1, abort_flag, ctl)) break;
+          const int brow = static_cast<int>((pair0 + kt) * kQTile);
+          mbar_arrive_expect_tx(bar_b_full(bs), 32768);
+          tma_load_2d(sB + bs * 32768, &tmB, bar_b_full(bs), 0, brow);
+          tma_load_2d(sB + bs * 32768 + 16384, &tmB, bar_b_full(bs), 64, brow);
+        }
         const int krow = static_cast<int>(seq0) + kt * kQTile;
         for (int h = 0; h < G; ++h, ++s) {
           const int st = s % kNS;
@@ -251,7 +263,7 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         umma_commit(bar_s_full(buf));
         if (s >= 1 && !issue_pv(s - 1)) { ok = false; break; }
       }
-      if (ok && issue_pv(nsteps - 1)) umma_commit(bar_o);
+      if (ok && nsteps > 0 && issue_pv(nsteps - 1)) umma_commit(bar_o);
     }
   } else {
     // ---------------- SiLU warps ----------------
@@ -262,19 +274,29 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     bool ok = true;
     for (int kt = 0; ok && kt < nkt; ++kt) {
-      const int bs = kt & 1;
-      if (!mbar_wait(bar_b_full(bs), (kt >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
       uint32_t hb[32];
-      {
+      if constexpr (FALCON) {
+        // the bias depends on the key only: one 64-key row shared by every query row
+        const uint4* src = reinterpret_cast<const uint4*>(a.kbias + b * a.kbias_ld + kt * kQTile + 64 * half);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 v = __ldg(src + u);
+          hb[4 * u] = v.x; hb[4 * u + 1] = v.y; hb[4 * u + 2] = v.z; hb[4 * u + 3] = v.w;
+        }
+      } else {
+        const int bs = kt & 1;
+        if (!mbar_wait(bar_b_full(bs), (kt >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
         const uint8_t* brow = smem + L::kBias + bs * 32768 + half * 16384 + r * 128;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const uint4 v = *reinterpret_cast<const uint4*>(brow + ((u ^ (r & 7)) << 4));
           hb[4 * u] = v.x; hb[4 * u + 1] = v.y; hb[4 * u + 2] = v.z; hb[4 * u + 3] = v.w;
         }
+        mbar_arrive(bar_b_empty(bs));
       }
-      mbar_arrive(bar_b_empty(bs));
-      const bool diag = (kt == qt);
+      // FALCON: keys past the user's prefix (last tile) are masked; causal: the diagonal tile
+      const int key_lim = FALCON ? n - kt * kQTile : 0;
+      const bool diag = FALCON ? key_lim < kQTile : (kt == qt);
       for (int h = 0; h < G; ++h) {
         const int s = kt * G + h;
         const int buf = s & 1;
@@ -298,7 +320,8 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             if (diag) {
               const int col = 64 * half + 32 * hc + 2 * j;
-              const uint32_t m = (col + 1 <= r) ? 0xFFFFFFFFu : ((col <= r) ? 0x0000FFFFu : 0u);
+              const int lim = FALCON ? key_lim - 1 : r;    // last key column kept
+              const uint32_t m = (col + 1 <= lim) ? 0xFFFFFFFFu : ((col <= lim) ? 0x0000FFFFu : 0u);
               y2 &= m;
             }
             p[16 * hc + j] = y2;
@@ -310,24 +333,69 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         mbar_arrive(bar_p_full(buf));
       }
     }
-    if (ok && mbar_wait(bar_o, 0, abort_flag, ctl)) {
+    if (ok && (nkt == 0 || mbar_wait(bar_o, 0, abort_flag, ctl))) {
       tc_fence_after();
       // G == 1: both key halves split head 0's 64 columns; G >= 2: half c handles heads c, c+2, ...
       constexpr int kHeadsPerWarp = G == 1 ? 1 : G / 2;
       constexpr int kCols = G == 1 ? 32 : 64;
       const float sc = a.inv_N;
+      const bool row_ok = FALCON ? qi < a.cand_rows : qi < n;
+      const long long orow = FALCON ? static_cast<long long>(b) * a.cand_rows + qi : seq0 + qi;
 #pragma unroll 1
       for (int e = 0; e < kHeadsPerWarp; ++e) {
         const int h = G == 1 ? 0 : half + 2 * e;
         const int col0 = G == 1 ? 32 * half : 0;
+        float self_a = 0.0f;    // FALCON: SiLU(q_c.k_c + self bias), the candidate's own weight
+        if (FALCON && row_ok) {
+          const int hc0 = (hg * G + h) * kD;
+          const uint4* qp = reinterpret_cast<const uint4*>(
+              static_cast<const uint16_t*>(a.q) + orow * a.ld_q + hc0);
+          const uint4* kp = reinterpret_cast<const uint4*>(
+              static_cast<const uint16_t*>(a.kc) + orow * a.ld_c + hc0);
+          float dot = 0.0f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint4 qv = qp[u], kv = kp[u];
+            const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w}, kw[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int w2 = 0; w2 < 4; ++w2) {
+              const float2 qf = F16 ? unpack_f16x2(qw[w2]) : unpack_bf16x2(qw[w2]);
+              const float2 kf = F16 ? unpack_f16x2(kw[w2]) : unpack_bf16x2(kw[w2]);
+              dot = fmaf(qf.x, kf.x, dot);
+              dot = fmaf(qf.y, kf.y, dot);
+            }
+          }
+          const float xs = dot + *a.self_bias;
+          self_a = xs / (1.0f + __expf(-xs));
+        }
 #pragma unroll 1
         for (int cc = 0; cc < kCols; cc += 32) {
           uint32_t ov[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h + col0 + cc, ov);
-          tmem_ld_wait();
-          if (qi < n) {
-            const long long orow = seq0 + qi;
+          if (nkt > 0) {
+            tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h + col0 + cc, ov);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) ov[q] = 0u;
+          }
+          if (row_ok) {
             const int ocol = (hg * G + h) * kD + col0 + cc;
+            if (FALCON) {   // + SiLU(self) v_c
+              const uint4* vp = reinterpret_cast<const uint4*>(
+                  static_cast<const uint16_t*>(a.vc) + orow * a.ld_c + ocol);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const uint4 vv = vp[u];
+                const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+                for (int w2 = 0; w2 < 4; ++w2) {
+                  const float2 vf = F16 ? unpack_f16x2(vw[w2]) : unpack_bf16x2(vw[w2]);
+                  ov[8 * u + 2 * w2] = __float_as_uint(fmaf(self_a, vf.x, __uint_as_float(ov[8 * u + 2 * w2])));
+                  ov[8 * u + 2 * w2 + 1] =
+                      __float_as_uint(fmaf(self_a, vf.y, __uint_as_float(ov[8 * u + 2 * w2 + 1])));
+                }
+              }
+            }
             if (a.o_f32) {
               float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + orow * a.ld_o + ocol);
 #pragma unroll
@@ -359,13 +427,44 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   }
 }
 
-template <bool F16, int G>
+// M-FALCON per-key half-bias: kbias[u * ld + j] = 0.5 (rab_pos[idx(n_u - j)] +
+// rab_time[bucket(request_ts[u] - t_j)]) for j < n_u, 0 up to ld. A prefix longer than ld is a
+// contract violation: recorded in the status word (the attention then stops at ld keys).
+__global__ void __launch_bounds__(256)
+falcon_key_bias_kernel(const int64_t* __restrict__ off, const int64_t* __restrict__ ts, const int64_t* __restrict__ req,
+                       const float* __restrict__ rab_pos, const float* __restrict__ rab_time, int L, int nb,
+                       uint16_t* kbias, int64_t ld, float* self_bias, int* status) {
+  __shared__ long long s_tau[kTauEntries];
+  for (int e = threadIdx.x; e < kTauEntries; e += blockDim.x) s_tau[e] = c_time_taus[e];
+  __syncthreads();
+  const int u = blockIdx.y;
+  if (u == 0 && blockIdx.x == 0 && threadIdx.x == 0) *self_bias = rab_pos[L - 1] + rab_time[0];
+  const long long s0 = off[u];
+  const long long n = off[u + 1] - s0;
+  if (n > ld || n < 0) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) report_error(status, kDevBadInput);
+  }
+  const long long treq = req[u];
+  for (long long j = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; j < ld;
+       j += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float v = 0.0f;
+    if (j < n) {
+      const int bkt = time_bucket_dev(treq - ts[s0 + j], s_tau, nb);
+      v = 0.5f * (rab_pos[pos_index2(n - j, L)] + rab_time[bkt]);
+    }
+    kbias[u * ld + j] = __half_as_ushort(__float2half_rn(v));
+  }
+}
+
+template <bool F16, int G, bool FALCON>
 cudaError_t launch_attn2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tb,
                          const AttnArgs& a, cudaStream_t st) {
-  auto kern = attn_fwd_tc2_kernel<F16, G>;
+  auto kern = attn_fwd_tc2_kernel<F16, G, FALCON>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), Smem2<G>::kTotal);
   if (e != cudaSuccess) return e;
-  const long long blocks = a.capacity * (a.H / G);
+  const long long blocks =
+      (FALCON ? static_cast<long long>(a.B) * ((a.cand_rows + kQTile - 1) / kQTile) : a.capacity) * (a.H / G);
+  if (blocks == 0) return cudaSuccess;
   kern<<<static_cast<unsigned>(blocks), kThreads2, Smem2<G>::kTotal, st>>>(tq, tk, tv, tb, a, wait_ctl(a.status));
   return cudaGetLastError();
 }
@@ -378,7 +477,7 @@ int64_t attn_max_pairs(int64_t capacity, int max_len) {
 }
 
 cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
-  cudaError_t e = upload_time_octaves();
+  cudaError_t e = upload_time_taus();
   if (e != cudaSuccess) return e;
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
@@ -394,8 +493,46 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
       !encode_tmap_2d_bf16(&tb, a.bias, kQTile, a.max_pairs * kQTile, kQTile, 64, 128, true))
     return cudaErrorInvalidValue;
   const int G = (a.H % 2 == 0) ? 2 : 1;
-  if (f16) return G == 2 ? launch_attn2<true, 2>(tq, tk, tv, tb, a, st) : launch_attn2<true, 1>(tq, tk, tv, tb, a, st);
-  return G == 2 ? launch_attn2<false, 2>(tq, tk, tv, tb, a, st) : launch_attn2<false, 1>(tq, tk, tv, tb, a, st);
+  if (f16)
+    return G == 2 ? launch_attn2<true, 2, false>(tq, tk, tv, tb, a, st)
+                  : launch_attn2<true, 1, false>(tq, tk, tv, tb, a, st);
+  return G == 2 ? launch_attn2<false, 2, false>(tq, tk, tv, tb, a, st)
+                : launch_attn2<false, 1, false>(tq, tk, tv, tb, a, st);
+}
+
+cudaError_t falcon_key_bias(const int64_t* offsets, const int64_t* ts, int users, int max_len,
+                            const int64_t* request_ts, const float* rab_pos, const float* rab_time, int pos_max_len,
+                            int n_buckets, uint16_t* kbias, int64_t kbias_ld, float* self_bias, int* status,
+                            cudaStream_t st) {
+  cudaError_t e = upload_time_taus();
+  if (e != cudaSuccess || users == 0) return e;
+  int64_t blocks = (kbias_ld + 255) / 256;
+  blocks = blocks < 1 ? 1 : (blocks > 64 ? 64 : blocks);
+  const unsigned gx = static_cast<unsigned>(blocks);
+  falcon_key_bias_kernel<<<dim3(gx, static_cast<unsigned>(users)), 256, 0, st>>>(
+      offsets, ts, request_ts, rab_pos, rab_time, pos_max_len, n_buckets, kbias, kbias_ld, self_bias, status);
+  (void)max_len;
+  return cudaGetLastError();
+}
+
+cudaError_t attn_falcon_tc(const AttnArgs& a, cudaStream_t st) {
+  if (a.B == 0 || a.cand_rows == 0 || a.q_rows == 0) return cudaSuccess;
+  CUtensorMap tq, tk, tv;
+  const bool f16 = a.in_f16 != 0;
+  const int64_t W = static_cast<int64_t>(a.H) * kD;
+  // an empty prefix batch still needs valid K/V maps: they are never loaded from (no key tiles)
+  const int64_t kv_rows = a.T > 0 ? a.T : 1;
+  if (!encode_tmap_2d_bf16(&tq, a.q, W, a.q_rows, a.ld_q, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tk, a.k, W, kv_rows, a.ld_k, 64, 128, f16) ||
+      !encode_tmap_2d_bf16(&tv, a.v, W, kv_rows, a.ld_v, 64, 128, f16))
+    return cudaErrorInvalidValue;
+  // two heads per CTA only when that still leaves about two CTAs per SM
+  const long long tiles = static_cast<long long>(a.B) * ((a.cand_rows + kQTile - 1) / kQTile);
+  const int G = (a.H % 2 == 0 && tiles * (a.H / 2) >= 2 * 148) ? 2 : 1;
+  if (f16)
+    return G == 2 ? launch_attn2<true, 2, true>(tq, tk, tv, tq, a, st) : launch_attn2<true, 1, true>(tq, tk, tv, tq, a, st);
+  return G == 2 ? launch_attn2<false, 2, true>(tq, tk, tv, tq, a, st)
+                : launch_attn2<false, 1, true>(tq, tk, tv, tq, a, st);
 }
 
 }  // namespace hstu

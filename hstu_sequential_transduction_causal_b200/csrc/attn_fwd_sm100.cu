@@ -66,7 +66,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const int nkt = qt + 1;
 
   float* s_rab_time = reinterpret_cast<float*>(smem + AttnSmem::kRabTime);
-  long long (*s_oct)[4] = reinterpret_cast<long long (*)[4]>(smem + AttnSmem::kOct);
+  long long* s_tau = reinterpret_cast<long long*>(smem + AttnSmem::kOct);
   long long* s_kts = reinterpret_cast<long long*>(smem + AttnSmem::kKts);
   float* s_pos = reinterpret_cast<float*>(smem + AttnSmem::kPos);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + AttnSmem::kBar);
@@ -104,7 +104,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     fence_barrier_init();
   }
   for (int e = tid; e < a.n_buckets && e < 128; e += kThreads) s_rab_time[e] = a.rab_time[e];
-  for (int e = tid; e < 63 * 4; e += kThreads) s_oct[e / 4][e % 4] = c_time_octaves[e / 4][e % 4];
+  for (int e = tid; e < kTauEntries; e += kThreads) s_tau[e] = c_time_taus[e];
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
@@ -222,7 +222,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int col = c * 32 + j + e;
-            const int bkt = time_bucket_dev(t_i - kts[col], s_oct, nb);
+            const int bkt = time_bucket_dev(t_i - kts[col], s_tau, nb);
             const float x = __uint_as_float(sv[j + e]) + pw[-col] + s_rab_time[bkt];
             y[e] = (!diag || col <= r) ? silu_fast(x) : 0.0f;
           }
@@ -314,7 +314,7 @@ attn_fwd_f32_kernel(AttnArgs a) {
     float part = (lane < a.dqk ? q0 * kr[lane] : 0.0f) + (lane + 32 < a.dqk ? q1 * kr[lane + 32] : 0.0f);
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
-    const int bkt = time_bucket_dev(t_i - a.ts[j], c_time_octaves, a.n_buckets);
+    const int bkt = time_bucket_dev(t_i - a.ts[j], c_time_taus, a.n_buckets);
     const float x = part + a.rab_pos[pos_index(i - j, L)] + a.rab_time[bkt];
     const float w = x / (1.0f + expf(-x)) * a.inv_N;
     const float* vr = reinterpret_cast<const float*>(a.v) + j * a.ld_v + h * a.dv;
@@ -329,7 +329,7 @@ attn_fwd_f32_kernel(AttnArgs a) {
 }  // namespace
 
 cudaError_t attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t st) {
-  cudaError_t e = upload_time_octaves();
+  cudaError_t e = upload_time_taus();
   if (e != cudaSuccess) return e;
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   CUtensorMap tq, tk, tv;
@@ -347,7 +347,7 @@ cudaError_t attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t st) {
 }
 
 cudaError_t attn_fwd_f32_simt(const AttnArgs& a, cudaStream_t st) {
-  cudaError_t e = upload_time_octaves();
+  cudaError_t e = upload_time_taus();
   if (e != cudaSuccess) return e;
   const long long warps = a.T * a.H;
   if (warps == 0) return cudaSuccess;

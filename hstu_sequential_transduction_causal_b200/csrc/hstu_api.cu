@@ -88,10 +88,10 @@ AttnBwdWs attn_bwd_ws_layout(const hstu_jagged_t* j) {
 }
 
 // layer-backward workspace: the attention-backward layout, then dG (fp32), dO (fp16), dq | dk | dv
-// (fp32), dZ (fp16 [T, 4D]), reduction partials, dgamma | dbeta, bf16 copies of x and dy, fp16
-// copies of x and W1 (the operands of dZ in the f1 backward GEMMs: both MMA operands share a type).
+// (fp32), dZ (fp16 [T, 4D]), reduction partials, dgamma | dbeta, and the fp16 GEMM operands: copies
+// of dy, x, W1 and W2 (both MMA operands share a type; G and dZ are fp16).
 struct LayerBwdWs {
-  size_t dg, dO, dq, dk, dv, dz, partial, gb, x_conv, dy_conv, x_f16, w1_f16, total;
+  size_t dg, dO, dq, dk, dv, dz, partial, gb, dy_f16, x_f16, w1_f16, w2_f16, total;
 };
 
 LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) {
@@ -109,10 +109,10 @@ LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) 
   const size_t pl = static_cast<size_t>(norm_gate_bwd_blocks(j->T)) * 2 * D;
   w.partial = take((pf > pl ? pf : pl) * 4);
   w.gb = take(2 * D * 4);
-  w.x_conv = take(T * D * 2);
-  w.dy_conv = take(T * D * 2);
+  w.dy_f16 = take(T * D * 2);
   w.x_f16 = take(T * D * 2);
   w.w1_f16 = take(4 * D * D * 2);
+  w.w2_f16 = take(D * D * 2);
   w.total = off;
   return w;
 }
@@ -224,11 +224,13 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
 }
 
 // f1: operands x, W1 of `dtype` (BF16 tensor cores or F32 CUDA cores); uvqk / z of act_dtype.
+// f16_ops: x and W1 are fp16 copies (the fp32-residual path) instead of bf16.
 hstu_status_t run_uvqk(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t act_dtype, const void* x, int64_t ld_x,
-                       const void* W1, const float* b1, void* uvqk, void* z, int* status, cudaStream_t st) {
+                       const void* W1, const float* b1, void* uvqk, void* z, int* status, cudaStream_t st,
+                       bool f16_ops = false) {
   GemmArgs g{};
   g.A = x; g.lda = ld_x; g.a_mn = false;
-  g.B = W1; g.ldb = D; g.b_mn = false; g.f16 = false;
+  g.B = W1; g.ldb = D; g.b_mn = false; g.f16 = f16_ops;
   g.M = T; g.N = 4ll * D; g.K = D; g.splits = 1;
   g.epi.kind = kEpiSilu; g.epi.bias = b1;
   g.epi.out0 = uvqk; g.epi.out0_dt = act_dtype; g.epi.ld_out0 = 4ll * D;
@@ -237,17 +239,23 @@ hstu_status_t run_uvqk(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t ac
   return cuda_status(dtype == HSTU_BF16 ? gemm_bf16(g, st) : gemm_f32(g, st));
 }
 
-hstu_status_t run_out_proj(int64_t T, int32_t D, hstu_dtype_t dtype, const void* g_in, const void* W2,
-                           const float* b2, const void* x, hstu_dtype_t x_dtype, void* y, hstu_dtype_t y_dtype,
-                           void* y_bf16, int* status, cudaStream_t st) {
+// g_dtype F16: W2 is read through an fp16 copy written to w2_f16 ([D, D]) first.
+hstu_status_t run_out_proj(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t g_dtype, const void* g_in,
+                           const void* W2, const float* b2, const void* x, hstu_dtype_t x_dtype, void* y,
+                           hstu_dtype_t y_dtype, void* y_f16, int* status, cudaStream_t st, void* w2_f16) {
+  const bool f16 = g_dtype == HSTU_F16;
+  if (f16) {
+    cudaError_t e = convert_dtype(W2, kDtBF16, w2_f16, kDtF16, static_cast<int64_t>(D) * D, st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
   GemmArgs g{};
   g.A = g_in; g.lda = D; g.a_mn = false;
-  g.B = W2; g.ldb = D; g.b_mn = false; g.f16 = false;
+  g.B = f16 ? w2_f16 : W2; g.ldb = D; g.b_mn = false; g.f16 = f16;
   g.M = T; g.N = D; g.K = D; g.splits = 1;
   g.epi.kind = kEpiLinear; g.epi.bias = b2;
   g.epi.resid = x; g.epi.resid_dt = x_dtype; g.epi.ld_resid = D;
   g.epi.out0 = y; g.epi.out0_dt = y_dtype; g.epi.ld_out0 = D;
-  g.epi.out1 = y_bf16; g.epi.out1_dt = kDtBF16; g.epi.ld_out1 = D;
+  g.epi.out1 = y_f16; g.epi.out1_dt = kDtF16; g.epi.ld_out1 = D;
   g.status = status;
   return cuda_status(dtype == HSTU_BF16 ? gemm_bf16(g, st) : gemm_f32(g, st));
 }
@@ -454,6 +462,7 @@ hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t o_dtype, hst
   if (T < 0) return HSTU_ERR_INVALID_ARG;
   const bool combo = (o_dtype == HSTU_F32 && u_dtype == HSTU_F32 && g_dtype == HSTU_F32) ||
                      (o_dtype == HSTU_F32 && is_tc_dtype(u_dtype) && g_dtype == HSTU_BF16) ||
+                     (o_dtype == HSTU_F32 && u_dtype == HSTU_F16 && g_dtype == HSTU_F16) ||
                      (o_dtype == HSTU_BF16 && u_dtype == HSTU_BF16 && g_dtype == HSTU_BF16);
   if (!combo) return HSTU_ERR_UNSUPPORTED;
   if (D != 64 && D != 128 && D != 256 && D != 512 && D != 1024) return HSTU_ERR_UNSUPPORTED;
@@ -466,33 +475,60 @@ hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t o_dtype, hst
                                    stream));
 }
 
-hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* g, const void* W2,
-                                const float* b2, const void* x, hstu_dtype_t x_dtype, void* y, hstu_dtype_t y_dtype,
-                                void* y_bf16, void* ws, size_t ws_bytes, hstu_stream_t stream) {
+size_t hstu_out_proj_workspace_size(int32_t D, hstu_dtype_t g_dtype) {
+  if (D <= 0) return 0;
+  return kWsHeader + (g_dtype == HSTU_F16 ? align_up(static_cast<size_t>(D) * D * 2, 256) : 0);
+}
+
+hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t g_dtype, const void* g,
+                                const void* W2, const float* b2, const void* x, hstu_dtype_t x_dtype, void* y,
+                                hstu_dtype_t y_dtype, void* y_f16, void* ws, size_t ws_bytes, hstu_stream_t stream) {
   hstu_status_t s = check_dense(T, D, dtype);
   if (s != HSTU_OK) return s;
   if (!ws) return HSTU_ERR_INVALID_ARG;
-  if (ws_bytes < kWsHeader) return HSTU_ERR_WORKSPACE;
+  const bool g_ok = dtype == HSTU_F32 ? g_dtype == HSTU_F32 : (g_dtype == HSTU_BF16 || g_dtype == HSTU_F16);
+  if (!g_ok) return HSTU_ERR_UNSUPPORTED;
+  if (ws_bytes < hstu_out_proj_workspace_size(D, g_dtype)) return HSTU_ERR_WORKSPACE;
   if ((x_dtype != HSTU_F32 && x_dtype != HSTU_BF16) || (y_dtype != HSTU_F32 && y_dtype != HSTU_BF16))
     return HSTU_ERR_UNSUPPORTED;
-  if (dtype == HSTU_F32 && (x_dtype != HSTU_F32 || y_dtype != HSTU_F32 || y_bf16)) return HSTU_ERR_UNSUPPORTED;
+  if (dtype == HSTU_F32 && (x_dtype != HSTU_F32 || y_dtype != HSTU_F32 || y_f16)) return HSTU_ERR_UNSUPPORTED;
   if (T == 0) return HSTU_OK;
   if (!g || !W2 || !x || !y) return HSTU_ERR_INVALID_ARG;
-  if (!aligned16(g) || !aligned16(W2) || !aligned16(x) || !aligned16(y) || (y_bf16 && !aligned16(y_bf16)))
+  if (!aligned16(g) || !aligned16(W2) || !aligned16(x) || !aligned16(y) || (y_f16 && !aligned16(y_f16)))
     return HSTU_ERR_UNSUPPORTED;
-  return run_out_proj(T, D, dtype, g, W2, b2, x, x_dtype, y, y_dtype, y_bf16, ws_status(ws), stream);
+  return run_out_proj(T, D, dtype, g_dtype, g, W2, b2, x, x_dtype, y, y_dtype, y_f16, ws_status(ws), stream,
+                      static_cast<uint8_t*>(ws) + kWsHeader);
+}
+
+// layer-forward workspace: the attention workspace, then (BF16 compute) the fp16 copy of W2 and,
+// for an fp32 X, fp16 copies of X and W1 (the f1 operands).
+struct LayerFwdWs {
+  size_t w2_f16, x_f16, w1_f16, total;
+};
+
+LayerFwdWs layer_fwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) {
+  LayerFwdWs w{};
+  const size_t T = static_cast<size_t>(j->T), D = static_cast<size_t>(d->D);
+  size_t off = align_up(attn_ws_bytes(j), 1024);
+  auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes, 1024); return o; };
+  if (d->dtype == HSTU_BF16) {
+    w.w2_f16 = take(D * D * 2);
+    if (d->x_dtype == HSTU_F32) {
+      w.x_f16 = take(T * D * 2);
+      w.w1_f16 = take(4 * D * D * 2);
+    }
+  }
+  w.total = off;
+  return w;
 }
 
 size_t hstu_layer_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag) {
-  if (!desc || check_jagged(jag) != HSTU_OK) return 0;
-  size_t bytes = attn_ws_bytes(jag);
-  if (desc->dtype == HSTU_BF16 && desc->x_dtype == HSTU_F32)
-    bytes += align_up(static_cast<size_t>(jag->T) * desc->D * 2, 256);
-  return bytes;
+  if (!desc || check_jagged(jag) != HSTU_OK || desc->D <= 0) return 0;
+  return layer_fwd_layout(desc, jag).total;
 }
 
 hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag, const hstu_layer_weights_t* w,
-                             const void* x, const void* x_bf16, void* y, void* y_bf16, const hstu_layer_saved_t* saved,
+                             const void* x, const void* x_f16, void* y, void* y_f16, const hstu_layer_saved_t* saved,
                              void* ws, size_t ws_bytes, hstu_stream_t stream) {
   if (!desc || !w || !saved) return HSTU_ERR_INVALID_ARG;
   hstu_status_t s = check_jagged(jag);
@@ -507,7 +543,7 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   ad.ld_q = ad.ld_k = ad.ld_v = 4ll * D; ad.ld_o = D;
   s = check_attn(&ad, jag);
   if (s != HSTU_OK) return s;
-  if (desc->dtype == HSTU_F32 && (desc->x_dtype != HSTU_F32 || desc->y_dtype != HSTU_F32 || y_bf16))
+  if (desc->dtype == HSTU_F32 && (desc->x_dtype != HSTU_F32 || desc->y_dtype != HSTU_F32 || y_f16))
     return HSTU_ERR_UNSUPPORTED;
   if (!ws) return HSTU_ERR_INVALID_ARG;
   if (ws_bytes < hstu_layer_workspace_size(desc, jag)) return HSTU_ERR_WORKSPACE;
@@ -518,21 +554,25 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
     return HSTU_ERR_INVALID_ARG;
   cudaStream_t st = stream;
   int* status = ws_status(ws);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  const LayerFwdWs lay = layer_fwd_layout(desc, jag);
+  // f1 operands: bf16 X with bf16 W1 as given; an fp32 X (residual stream) through fp16 copies of
+  // X and W1, 8x finer than bf16 at the same MMA rate
+  const bool x32 = desc->dtype == HSTU_BF16 && desc->x_dtype == HSTU_F32;
   const void* x_op = x;
-  if (desc->dtype == HSTU_BF16 && desc->x_dtype == HSTU_F32) {
-    if (x_bf16) {
-      x_op = x_bf16;
-    } else {
-      void* conv = static_cast<uint8_t*>(ws) + attn_ws_bytes(jag);
-      cudaError_t e = convert_f32_to_bf16(static_cast<const float*>(x), conv, T * D, st);
-      if (e != cudaSuccess) return cuda_status(e);
-      x_op = conv;
-    }
+  const void* w1_op = w->W1;
+  if (x32) {
+    cudaError_t e = cudaSuccess;
+    if (!x_f16) e = convert_dtype(x, kDtF32, wsb + lay.x_f16, kDtF16, T * D, st);
+    if (e == cudaSuccess) e = convert_dtype(w->W1, kDtBF16, wsb + lay.w1_f16, kDtF16, 4ll * D * D, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    x_op = x_f16 ? x_f16 : wsb + lay.x_f16;
+    w1_op = wsb + lay.w1_f16;
   }
   // tensor-core mode keeps U|V|Q|K (and Z) in fp16: same MMA rate as bf16, 8x finer rounding of
   // the attention operands, whose errors LayerNorm(O) would otherwise amplify
   const hstu_dtype_t act = desc->dtype == HSTU_BF16 ? HSTU_F16 : HSTU_F32;
-  s = run_uvqk(T, D, desc->dtype, act, x_op, D, w->W1, w->b1, saved->uvqk, saved->z, status, st);
+  s = run_uvqk(T, D, desc->dtype, act, x_op, D, w1_op, w->b1, saved->uvqk, saved->z, status, st, x32);
   if (s != HSTU_OK) return s;
   ad.dtype = act;
   const size_t es = act == HSTU_F32 ? 4 : 2;
@@ -540,11 +580,13 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   s = run_attn_fwd(&ad, jag, uvqk + 2 * D * es, uvqk + 3 * D * es, uvqk + 1 * D * es, w->rab_pos, w->rab_time,
                    saved->o, ws, st);
   if (s != HSTU_OK) return s;
-  cudaError_t e = norm_gate_fwd(T, D, kDtF32, act, desc->dtype, saved->o, D, uvqk, 4ll * D, w->gamma, w->beta,
+  // G in fp16 (BF16 mode): f2 then reads an fp16 copy of W2
+  const hstu_dtype_t g_dt = desc->dtype == HSTU_BF16 ? HSTU_F16 : HSTU_F32;
+  cudaError_t e = norm_gate_fwd(T, D, kDtF32, act, g_dt, saved->o, D, uvqk, 4ll * D, w->gamma, w->beta,
                                 desc->ln_eps, saved->g, saved->mu, saved->rstd, st);
   if (e != cudaSuccess) return cuda_status(e);
-  return run_out_proj(T, D, desc->dtype, saved->g, w->W2, w->b2, x, desc->x_dtype, y, desc->y_dtype, y_bf16, status,
-                      st);
+  return run_out_proj(T, D, desc->dtype, g_dt, saved->g, w->W2, w->b2, x, desc->x_dtype, y, desc->y_dtype, y_f16,
+                      status, st, wsb + lay.w2_f16);
 }
 
 hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda, int32_t a_mn,
@@ -581,8 +623,8 @@ size_t hstu_layer_bwd_workspace_size(const hstu_layer_desc_t* desc, const hstu_j
 }
 
 hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag, const hstu_layer_weights_t* w,
-                             const void* x, const void* x_bf16, const hstu_layer_saved_t* saved, const void* dy,
-                             const void* dy_bf16, void* dx, void* dx_bf16, const hstu_layer_grads_t* gr, void* ws,
+                             const void* x, const void* x_f16, const hstu_layer_saved_t* saved, const void* dy,
+                             const void* dy_f16, void* dx, void* dx_f16, const hstu_layer_grads_t* gr, void* ws,
                              size_t ws_bytes, hstu_stream_t stream) {
   if (!desc || !w || !saved || !gr) return HSTU_ERR_INVALID_ARG;
   hstu_status_t s = check_jagged(jag);
@@ -618,26 +660,18 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
     return HSTU_ERR_INVALID_ARG;
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   int* status = ws_status(ws);
-  const void* x_op = x_bf16;
-  if (!x_op) {
-    if (desc->x_dtype == HSTU_BF16) {
-      x_op = x;
-    } else {
-      e = convert_f32_to_bf16(static_cast<const float*>(x), wsb + lay.x_conv, T * D, st);
-      if (e != cudaSuccess) return cuda_status(e);
-      x_op = wsb + lay.x_conv;
-    }
-  }
-  const void* dy_op = dy_bf16;
-  if (!dy_op) {
-    if (desc->y_dtype == HSTU_BF16) {
-      dy_op = dy;
-    } else {
-      e = convert_f32_to_bf16(static_cast<const float*>(dy), wsb + lay.dy_conv, T * D, st);
-      if (e != cudaSuccess) return cuda_status(e);
-      dy_op = wsb + lay.dy_conv;
-    }
-  }
+  // fp16 operands: dy (of dG and dW2, next to fp16 G and W2), x (of dW1, next to fp16 dZ), W1, W2
+  const int x_dt = desc->x_dtype == HSTU_F32 ? kDtF32 : kDtBF16;
+  const int y_dt = desc->y_dtype == HSTU_F32 ? kDtF32 : kDtBF16;
+  const void* dy_op = dy_f16 ? dy_f16 : wsb + lay.dy_f16;
+  const void* x_op = x_f16 ? x_f16 : wsb + lay.x_f16;
+  void* w1_f16 = wsb + lay.w1_f16;
+  void* w2_f16 = wsb + lay.w2_f16;
+  if (!dy_f16) e = convert_dtype(dy, y_dt, wsb + lay.dy_f16, kDtF16, T * D, st);
+  if (e == cudaSuccess && !x_f16) e = convert_dtype(x, x_dt, wsb + lay.x_f16, kDtF16, T * D, st);
+  if (e == cudaSuccess) e = convert_dtype(w->W1, kDtBF16, w1_f16, kDtF16, 4ll * D * D, st);
+  if (e == cudaSuccess) e = convert_dtype(w->W2, kDtBF16, w2_f16, kDtF16, 1ll * D * D, st);
+  if (e != cudaSuccess) return cuda_status(e);
   float* dG = reinterpret_cast<float*>(wsb + lay.dg);
   void* dO = wsb + lay.dO;
   float* dq = reinterpret_cast<float*>(wsb + lay.dq);
@@ -648,14 +682,14 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   float* gb = reinterpret_cast<float*>(wsb + lay.gb);
   // 1. f2 backward: dG = dY W2, dW2 = dY^T G, db2 = sum_t dY
   GemmArgs g{};
-  g.A = dy_op; g.lda = D; g.a_mn = false; g.B = w->W2; g.ldb = D; g.b_mn = true; g.f16 = false;
+  g.A = dy_op; g.lda = D; g.a_mn = false; g.B = w2_f16; g.ldb = D; g.b_mn = true; g.f16 = true;
   g.M = T; g.N = D; g.K = D; g.splits = 1;
   g.epi.kind = kEpiLinear; g.epi.out0 = dG; g.epi.out0_dt = kDtF32; g.epi.ld_out0 = D; g.status = status;
   e = gemm_bf16(g, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW2, 0, sizeof(float) * D * D, st);
   if (e == cudaSuccess) {
     GemmArgs g2{};
-    g2.A = dy_op; g2.lda = D; g2.a_mn = true; g2.B = saved->g; g2.ldb = D; g2.b_mn = true; g2.f16 = false;
+    g2.A = dy_op; g2.lda = D; g2.a_mn = true; g2.B = saved->g; g2.ldb = D; g2.b_mn = true; g2.f16 = true;
     g2.M = D; g2.N = D; g2.K = T; g2.splits = auto_splits(D, D, T);
     g2.epi.kind = kEpiAtomic; g2.epi.out0 = gr->dW2; g2.epi.out0_dt = kDtF32; g2.epi.ld_out0 = D; g2.status = status;
     e = gemm_bf16(g2, st);
@@ -676,15 +710,11 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   // 4. SiLU backward into dZ[:, D:4D], db1 = sum_t dZ
   e = dz_assemble(T, D, kDtF16, dv, dq, dk, saved->z, 4ll * D, dz, 4ll * D, st);
   if (e == cudaSuccess) e = column_sum(dz, kDtF16, T, 4 * D, 4ll * D, part, gr->db1, st);
-  // 5. f1 backward: dW1 = dZ^T X, dX = dY + dZ W1 (dZ fp16: exact fp16 copies of x and W1)
-  void* x_f16 = wsb + lay.x_f16;
-  void* w1_f16 = wsb + lay.w1_f16;
-  if (e == cudaSuccess) e = convert_dtype(x_op, kDtBF16, x_f16, kDtF16, T * D, st);
-  if (e == cudaSuccess) e = convert_dtype(w->W1, kDtBF16, w1_f16, kDtF16, 4ll * D * D, st);
+  // 5. f1 backward: dW1 = dZ^T X, dX = dY + dZ W1 (fp16 dZ, x and W1)
   if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW1, 0, sizeof(float) * 4 * D * D, st);
   if (e == cudaSuccess) {
     GemmArgs g3{};
-    g3.A = dz; g3.lda = 4ll * D; g3.a_mn = true; g3.B = x_f16; g3.ldb = D; g3.b_mn = true; g3.f16 = true;
+    g3.A = dz; g3.lda = 4ll * D; g3.a_mn = true; g3.B = x_op; g3.ldb = D; g3.b_mn = true; g3.f16 = true;
     g3.M = 4ll * D; g3.N = D; g3.K = T; g3.splits = auto_splits(4ll * D, D, T);
     g3.epi.kind = kEpiAtomic; g3.epi.out0 = gr->dW1; g3.epi.out0_dt = kDtF32; g3.epi.ld_out0 = D; g3.status = status;
     e = gemm_bf16(g3, st);
@@ -695,7 +725,7 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
     g4.M = T; g4.N = D; g4.K = 4ll * D; g4.splits = 1;
     g4.epi.kind = kEpiLinear; g4.epi.resid = dy; g4.epi.resid_dt = desc->y_dtype; g4.epi.ld_resid = D;
     g4.epi.out0 = dx; g4.epi.out0_dt = desc->x_dtype; g4.epi.ld_out0 = D;
-    g4.epi.out1 = dx_bf16; g4.epi.out1_dt = kDtBF16; g4.epi.ld_out1 = D; g4.status = status;
+    g4.epi.out1 = dx_f16; g4.epi.out1_dt = kDtF16; g4.epi.ld_out1 = D; g4.status = status;
     e = gemm_bf16(g4, st);
   }
   return cuda_status(e);
@@ -765,4 +795,224 @@ extern "C" hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_desc_t* desc, con
   cudaError_t e = cudaMemsetAsync(scratch, 0, kWsHeader, stream);
   if (e != cudaSuccess) return cuda_status(e);
   return run_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, scratch, stream, false);
+}
+
+// ---------------------------------------------------------------------------------------------
+// M-FALCON ("HSTU: The First Exploration of the Scaling Law", 7.1.5 M-FALCON)
+// ---------------------------------------------------------------------------------------------
+namespace hstu {
+namespace {
+
+// Layer 0 reads the bf16 inputs; every later layer reads the fp32 residual stream.
+hstu_layer_desc_t falcon_layer_desc(const hstu_falcon_desc_t* d, bool first) {
+  hstu_layer_desc_t l{};
+  l.D = d->D; l.H = d->H; l.inv_N = d->inv_N; l.pos_max_len = d->pos_max_len;
+  l.n_time_buckets = d->n_time_buckets; l.ln_eps = d->ln_eps;
+  l.dtype = HSTU_BF16; l.x_dtype = first ? HSTU_BF16 : HSTU_F32; l.y_dtype = HSTU_F32;
+  return l;
+}
+
+// Workspace: the prefix layer's workspace first (its status word is the call's status word), then
+// the prefix activations of one layer, the fp32 prefix stream (two buffers) and its fp16 copy, the
+// per-layer key bias rows (+ the self bias), and one candidate micro-batch of
+// R = users * min(b_m, m) rows: its bf16 input rows, fp32 stream (two buffers) and fp16 copy,
+// U|V|Q|K, O, G, mu, rstd, and the fp16 copies of W1 and W2 of the candidate pass.
+struct FalconWs {
+  size_t p_uvqk, p_o, p_g, p_mu, p_rstd, p_x0, p_x1, p_x16, kbias, self_bias, c_in, c_x0, c_x1, c_x16, c_uvqk, c_o,
+      c_g, c_mu, c_rstd, w1_f16, w2_f16, total;
+  int64_t kbias_ld, R;
+};
+
+FalconWs falcon_layout(const hstu_falcon_desc_t* d, const hstu_jagged_t* p) {
+  FalconWs w{};
+  const hstu_layer_desc_t ld = falcon_layer_desc(d, false);   // the larger of the two layer workspaces
+  const size_t Tp = static_cast<size_t>(p->T), D = static_cast<size_t>(d->D);
+  w.kbias_ld = static_cast<int64_t>(align_up(static_cast<size_t>(p->max_len), kQTile));
+  const int64_t per = d->b_m < d->m ? d->b_m : d->m;
+  w.R = static_cast<int64_t>(d->users) * (per > 0 ? per : 0);
+  const size_t R = static_cast<size_t>(w.R);
+  size_t off = align_up(hstu_layer_workspace_size(&ld, p), 1024);
+  auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes, 1024); return o; };
+  w.p_uvqk = take(Tp * 4 * D * 2);
+  w.p_o = take(Tp * D * 4);
+  w.p_g = take(Tp * D * 2);
+  w.p_mu = take(Tp * 4);
+  w.p_rstd = take(Tp * 4);
+  w.p_x0 = take(Tp * D * 4);
+  w.p_x1 = take(Tp * D * 4);
+  w.p_x16 = take(Tp * D * 2);
+  w.kbias = take(static_cast<size_t>(d->L) * d->users * w.kbias_ld * 2);
+  w.self_bias = take(static_cast<size_t>(d->L) * 4);
+  w.c_in = take(R * D * 2);
+  w.c_x0 = take(R * D * 4);
+  w.c_x1 = take(R * D * 4);
+  w.c_x16 = take(R * D * 2);
+  w.c_uvqk = take(R * 4 * D * 2);
+  w.c_o = take(R * D * 4);
+  w.c_g = take(R * D * 2);
+  w.c_mu = take(R * 4);
+  w.c_rstd = take(R * 4);
+  w.w1_f16 = take(4 * D * D * 2);
+  w.w2_f16 = take(D * D * 2);
+  w.total = off;
+  return w;
+}
+
+hstu_status_t check_falcon(const hstu_falcon_desc_t* d, const hstu_jagged_t* p) {
+  if (!d) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t s = check_jagged(p);
+  if (s != HSTU_OK) return s;
+  if (d->L < 1 || d->users < 0 || d->m < 0 || d->b_m < 1 || d->users != p->B) return HSTU_ERR_INVALID_ARG;
+  if (d->H <= 0 || d->D <= 0 || d->D % d->H) return HSTU_ERR_INVALID_ARG;
+  if (d->D / d->H != 64 || d->D % 64) return HSTU_ERR_UNSUPPORTED;
+  if (d->pos_max_len <= 0 || !isfinite(d->inv_N)) return HSTU_ERR_INVALID_ARG;
+  if (d->n_time_buckets < 1 || d->n_time_buckets > 128) return HSTU_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(d->users) * d->m >= (1ll << 31)) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+}  // namespace
+}  // namespace hstu
+
+extern "C" size_t hstu_falcon_cache_size(const hstu_falcon_desc_t* desc, const hstu_jagged_t* prefix) {
+  if (check_falcon(desc, prefix) != HSTU_OK) return 0;
+  return static_cast<size_t>(desc->L) * static_cast<size_t>(prefix->T) * 2 * desc->D * 2;
+}
+
+extern "C" size_t hstu_falcon_workspace_size(const hstu_falcon_desc_t* desc, const hstu_jagged_t* prefix) {
+  if (check_falcon(desc, prefix) != HSTU_OK) return 0;
+  return falcon_layout(desc, prefix).total;
+}
+
+extern "C" hstu_status_t hstu_falcon_fwd(const hstu_falcon_desc_t* desc, const hstu_layer_weights_t* layers,
+                                         const hstu_jagged_t* prefix, const void* prefix_x, void* kv_cache,
+                                         int32_t cache_valid, void* prefix_out, const void* cand_x,
+                                         const int64_t* request_ts, void* out, void* ws, size_t ws_bytes,
+                                         hstu_stream_t stream) {
+  hstu_status_t s = check_falcon(desc, prefix);
+  if (s != HSTU_OK) return s;
+  if (!layers || !ws) return HSTU_ERR_INVALID_ARG;
+  const FalconWs lay = falcon_layout(desc, prefix);
+  if (ws_bytes < lay.total) return HSTU_ERR_WORKSPACE;
+  const int32_t D = desc->D, L = desc->L, users = desc->users, m = desc->m;
+  const int64_t Tp = prefix->T;
+  if (users == 0 || m == 0) return HSTU_OK;
+  if (!cand_x || !request_ts || !out || (Tp > 0 && !kv_cache) || (!cache_valid && Tp > 0 && !prefix_x))
+    return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(cand_x) || !aligned16(out) || (kv_cache && !aligned16(kv_cache)) ||
+      (prefix_x && !aligned16(prefix_x)) || (prefix_out && !aligned16(prefix_out)))
+    return HSTU_ERR_UNSUPPORTED;
+  for (int l = 0; l < L; ++l) {
+    const hstu_layer_weights_t& w = layers[l];
+    if (!w.W1 || !w.b1 || !w.W2 || !w.b2 || !w.gamma || !w.beta || !w.rab_pos || !w.rab_time)
+      return HSTU_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = stream;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = ws_status(ws);
+  const hstu_layer_desc_t ldesc0 = falcon_layer_desc(desc, true), ldesc = falcon_layer_desc(desc, false);
+  const size_t layer_ws = hstu_layer_workspace_size(&ldesc, prefix);
+  const size_t kv_layer = static_cast<size_t>(Tp) * 2 * D;   // fp16 elements per layer of the cache
+  uint16_t* cache = static_cast<uint16_t*>(kv_cache);
+  void* x16 = nullptr;
+
+  // 1. prefix: L causal layers on an fp32 residual stream; layer l's K and V go to the cache
+  if (!cache_valid && Tp > 0) {
+    hstu_layer_saved_t sv{};
+    sv.uvqk = base + lay.p_uvqk; sv.z = nullptr; sv.o = base + lay.p_o; sv.g = base + lay.p_g;
+    sv.mu = reinterpret_cast<float*>(base + lay.p_mu); sv.rstd = reinterpret_cast<float*>(base + lay.p_rstd);
+    const void* xin = prefix_x;
+    x16 = base + lay.p_x16;
+    for (int l = 0; l < L; ++l) {
+      void* y = (l == L - 1 && prefix_out) ? prefix_out : static_cast<void*>(base + ((l & 1) ? lay.p_x1 : lay.p_x0));
+      // layer l reads the fp16 copy of its input that layer l - 1 wrote, and writes the next one
+      s = hstu_layer_fwd(l == 0 ? &ldesc0 : &ldesc, prefix, &layers[l], xin, l == 0 ? nullptr : x16, y,
+                         l + 1 < L ? x16 : nullptr, &sv, ws, layer_ws, st);
+      if (s != HSTU_OK) return s;
+      const uint16_t* uvqk = static_cast<const uint16_t*>(sv.uvqk);
+      uint16_t* kv = cache + l * kv_layer;
+      cudaError_t e = cudaMemcpy2DAsync(kv, 2 * D * 2, uvqk + 3 * D, 4 * D * 2, D * 2, Tp, cudaMemcpyDeviceToDevice, st);
+      if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(kv + D, 2 * D * 2, uvqk + D, 4 * D * 2, D * 2, Tp, cudaMemcpyDeviceToDevice, st);
+      if (e != cudaSuccess) return cuda_status(e);
+      xin = y;
+    }
+  }
+
+  // 2. per layer: the half-bias of every prefix key as seen from the request time
+  uint16_t* kbias = reinterpret_cast<uint16_t*>(base + lay.kbias);
+  float* self_bias = reinterpret_cast<float*>(base + lay.self_bias);
+  for (int l = 0; l < L; ++l) {
+    cudaError_t e = falcon_key_bias(prefix->offsets, prefix->timestamps, users, prefix->max_len, request_ts,
+                                    layers[l].rab_pos, layers[l].rab_time, desc->pos_max_len, desc->n_time_buckets,
+                                    kbias + static_cast<size_t>(l) * users * lay.kbias_ld, lay.kbias_ld,
+                                    self_bias + l, status, st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+
+  // 3. candidates, b_m per user at a time, on an fp32 residual stream; every layer reads its cached
+  //    prefix K, V
+  const bool one_pass = desc->b_m >= m;
+  void* c_x[2] = {base + lay.c_x0, base + lay.c_x1};
+  void* c_x16 = base + lay.c_x16;
+  void* c_uvqk = base + lay.c_uvqk;
+  void* w1_f16 = base + lay.w1_f16;
+  void* w2_f16 = base + lay.w2_f16;
+  const uint16_t* cu = static_cast<const uint16_t*>(c_uvqk);
+  for (int32_t c0 = 0; c0 < m; c0 += desc->b_m) {
+    const int32_t rows = (m - c0) < desc->b_m ? (m - c0) : desc->b_m;
+    const int64_t R = static_cast<int64_t>(users) * rows;
+    const void* xin = cand_x;
+    if (!one_pass) {   // gather rows [u m + c0, u m + c0 + rows) of every user
+      cudaError_t e = cudaMemcpy2DAsync(base + lay.c_in, static_cast<size_t>(rows) * D * 2,
+                                        static_cast<const uint16_t*>(cand_x) + static_cast<size_t>(c0) * D,
+                                        static_cast<size_t>(m) * D * 2, static_cast<size_t>(rows) * D * 2, users,
+                                        cudaMemcpyDeviceToDevice, st);
+      if (e != cudaSuccess) return cuda_status(e);
+      xin = base + lay.c_in;
+    }
+    for (int l = 0; l < L; ++l) {
+      const hstu_layer_weights_t& w = layers[l];
+      const bool last = l == L - 1;
+      void* y = (one_pass && last) ? out : c_x[l & 1];
+      if (l == 0) {
+        s = run_uvqk(R, D, HSTU_BF16, HSTU_F16, xin, D, w.W1, w.b1, c_uvqk, nullptr, status, st);
+      } else {
+        cudaError_t e = convert_dtype(w.W1, kDtBF16, w1_f16, kDtF16, 4ll * D * D, st);
+        if (e != cudaSuccess) return cuda_status(e);
+        s = run_uvqk(R, D, HSTU_BF16, HSTU_F16, c_x16, D, w1_f16, w.b1, c_uvqk, nullptr, status, st, true);
+      }
+      if (s != HSTU_OK) return s;
+      AttnArgs a{};
+      a.B = users; a.T = Tp; a.max_len = prefix->max_len; a.offsets = prefix->offsets; a.ts = prefix->timestamps;
+      a.H = desc->H; a.dqk = 64; a.dv = 64; a.inv_N = desc->inv_N; a.pos_max_len = desc->pos_max_len;
+      a.n_buckets = desc->n_time_buckets;
+      a.q = cu + 2 * D; a.ld_q = 4 * D;
+      a.k = cache + l * kv_layer; a.ld_k = 2 * D;
+      a.v = cache + l * kv_layer + D; a.ld_v = 2 * D;
+      a.o = base + lay.c_o; a.ld_o = D; a.o_f32 = 1; a.in_f16 = 1;
+      a.rab_pos = w.rab_pos; a.rab_time = w.rab_time; a.status = status;
+      a.cand_rows = rows; a.q_rows = R;
+      a.kc = cu + 3 * D; a.vc = cu + D; a.ld_c = 4 * D;
+      a.kbias = kbias + static_cast<size_t>(l) * users * lay.kbias_ld; a.kbias_ld = lay.kbias_ld;
+      a.self_bias = self_bias + l;
+      cudaError_t e = attn_falcon_tc(a, st);
+      if (e == cudaSuccess)
+        e = norm_gate_fwd(R, D, kDtF32, kDtF16, kDtF16, base + lay.c_o, D, c_uvqk, 4ll * D, w.gamma, w.beta,
+                          desc->ln_eps, base + lay.c_g, reinterpret_cast<float*>(base + lay.c_mu),
+                          reinterpret_cast<float*>(base + lay.c_rstd), st);
+      if (e != cudaSuccess) return cuda_status(e);
+      s = run_out_proj(R, D, HSTU_BF16, HSTU_F16, base + lay.c_g, w.W2, w.b2, xin, l == 0 ? HSTU_BF16 : HSTU_F32, y,
+                       HSTU_F32, last ? nullptr : c_x16, status, st, w2_f16);
+      if (s != HSTU_OK) return s;
+      xin = y;
+    }
+    if (!one_pass) {   // scatter back
+      cudaError_t e = cudaMemcpy2DAsync(static_cast<float*>(out) + static_cast<size_t>(c0) * D,
+                                        static_cast<size_t>(m) * D * 4, xin, static_cast<size_t>(rows) * D * 4,
+                                        static_cast<size_t>(rows) * D * 4, users, cudaMemcpyDeviceToDevice, st);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
+  }
+  return HSTU_OK;
 }

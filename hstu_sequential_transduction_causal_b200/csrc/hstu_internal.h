@@ -103,6 +103,16 @@ struct AttnArgs {
   const long long* pair_base;   // [B+1] first causal tile pair of each sequence (tile-pair kernel)
   void* bias;                   // fp16 [max_pairs, 128, 128] bias tiles (tile-pair kernel)
   int64_t max_pairs;
+  // M-FALCON candidate attention (attn_falcon_tc): B users, offsets / ts / k / v describe the
+  // prefixes (T prefix rows); q holds q_rows = B * cand_rows candidate rows, user-major.
+  int cand_rows;                // candidate rows per user
+  int64_t q_rows;
+  const void* kc;               // candidates' own K and V (same dtype as q), row stride ld_c
+  const void* vc;
+  int64_t ld_c;
+  const uint16_t* kbias;        // fp16 half-bias per prefix key: [B, kbias_ld], user u at u * kbias_ld
+  int64_t kbias_ld;             // multiple of 128 >= every prefix length
+  const float* self_bias;       // device: rab_pos[idx(0)] + rab_time[bucket(0)]
 };
 
 struct AttnBwdArgs {
@@ -127,6 +137,13 @@ int64_t attn_max_pairs(int64_t capacity, int max_len);
 cudaError_t attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t st);     // work list only
 cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st);         // bias tiles + work list
 cudaError_t attn_fwd_f32_simt(const AttnArgs& a, cudaStream_t st);
+// M-FALCON: the per-key half-bias of every prefix token (one launch per layer), then the candidate
+// attention; tc dtypes only, d = 64, O fp32.
+cudaError_t falcon_key_bias(const int64_t* offsets, const int64_t* ts, int users, int max_len,
+                            const int64_t* request_ts, const float* rab_pos, const float* rab_time,
+                            int pos_max_len, int n_buckets, uint16_t* kbias, int64_t kbias_ld, float* self_bias,
+                            int* status, cudaStream_t st);
+cudaError_t attn_falcon_tc(const AttnArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------------
 // LayerNorm (.) U

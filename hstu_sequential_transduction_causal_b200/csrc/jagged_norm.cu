@@ -237,7 +237,7 @@ time_bucket_kernel(const int64_t* __restrict__ off, const int64_t* __restrict__ 
   const long long n = off[lo + 1] - s0;
   const long long ti = ts[row];
   uint8_t* dst = out + sq_off[lo] + (row - s0) * n;
-  for (long long j = lane; j < n; j += 32) dst[j] = static_cast<uint8_t>(time_bucket_dev(ti - ts[s0 + j], c_time_octaves, nb));
+  for (long long j = lane; j < n; j += 32) dst[j] = static_cast<uint8_t>(time_bucket_dev(ti - ts[s0 + j], c_time_taus, nb));
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -338,7 +338,7 @@ cudaError_t launch_bwd_worklist(const int64_t* offsets, int B, const int32_t* fw
 cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int n_buckets,
                                 const int64_t* sq_offsets, uint8_t* out, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  cudaError_t e = upload_time_octaves();
+  cudaError_t e = upload_time_taus();
   if (e != cudaSuccess) return e;
   time_bucket_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, st>>>(offsets, ts, B, T, n_buckets,
                                                                           sq_offsets, out);
@@ -349,11 +349,13 @@ cudaError_t norm_gate_fwd(int64_t T, int D, int o_dt, int u_dt, int g_dt, const 
                           int64_t ld_u, const float* gamma, const float* beta, float eps, void* g, float* mu,
                           float* rstd, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  // supported (o, u, g) combinations: exact fp32; fp32 O with fp16 or bf16 U and bf16 G (tensor-core
-  // layer); all bf16.
+  // supported (o, u, g) combinations: exact fp32; fp32 O with fp16 U and fp16 G (tensor-core
+  // layer); fp32 O with fp16 or bf16 U and bf16 G; all bf16.
 #define HSTU_NG(VPT)                                                                                     \
   if (o_dt == kDtF32 && u_dt == kDtF32 && g_dt == kDtF32)                                               \
     return launch_ng<VPT, kDtF32, kDtF32, kDtF32>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+  if (o_dt == kDtF32 && u_dt == kDtF16 && g_dt == kDtF16)                                               \
+    return launch_ng<VPT, kDtF32, kDtF16, kDtF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
   if (o_dt == kDtF32 && u_dt == kDtF16 && g_dt == kDtBF16)                                              \
     return launch_ng<VPT, kDtF32, kDtF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
   if (o_dt == kDtF32 && u_dt == kDtBF16 && g_dt == kDtBF16)                                             \

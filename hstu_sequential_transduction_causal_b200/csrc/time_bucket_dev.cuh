@@ -1,8 +1,10 @@
 // time_bucket_dev.cuh - device evaluation of the relative-time bucket
-//   bucket(dt) = min(nb - 1, floor(ln(max(dt, 1)) / 0.301))
-// from the exact integer thresholds of time_bucket_table.h: o = floor(log2 dt) selects an octave,
-// whose base count plus up to three comparisons give the bucket. No floating point is involved,
-// so the result is exact for every int64 dt. Each translation unit holds its own constant copy.
+//   bucket(dt) = min(nb - 1, floor(ln(max(dt, 1)) / 0.301)) = min(nb - 1, #{k >= 1 : tau_k <= dt})
+// from the exact integer thresholds tau_k = ceil(exp(0.301 k)) of time_bucket_table.h. A float
+// estimate of ln(dt) / 0.301 (error about 1e-5, so its integer part is at most one away from the
+// exact count) is corrected by one integer comparison on each side: the result is exact for every
+// int64 dt. The table is staged as tau[0..128] with tau_0 = INT64_MIN and tau_128 = INT64_MAX
+// sentinels. Each translation unit holds its own constant copy.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -12,25 +14,30 @@
 namespace hstu {
 namespace {
 
-__constant__ long long c_time_octaves[63][4];
+constexpr int kTauEntries = 129;
+__constant__ long long c_time_taus[kTauEntries];
 
-__device__ __forceinline__ int time_bucket_dev(long long dt, const long long (*oct)[4], int nb) {
-  int b = 0;
-  if (dt > 1) {
-    const int o = 63 - __clzll(dt);
-    b = static_cast<int>(oct[o][3]) + (dt >= oct[o][0]) + (dt >= oct[o][1]) + (dt >= oct[o][2]);
-  }
-  return min(b, nb - 1);
+__device__ __forceinline__ int time_bucket_dev(long long dt, const long long* tau, int nb) {
+  if (dt <= 1) return 0;
+  constexpr float kLn2Over0301 = 0.693147180559945f / 0.301f;
+  const float lf = __log2f(__ll2float_rn(dt)) * kLn2Over0301;   // >= 2.3 for dt >= 2
+  int k = min(static_cast<int>(lf), 126);
+  k += (dt >= tau[k + 1] ? 1 : 0) - (dt < tau[k] ? 1 : 0);
+  return min(k, nb - 1);
 }
 
-// Copies the octave table to this translation unit's constant bank, once per device.
-inline cudaError_t upload_time_octaves() {
+// Copies tau_0..tau_128 to this translation unit's constant bank, once per device.
+inline cudaError_t upload_time_taus() {
   static bool done[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-  e = cudaMemcpyToSymbol(c_time_octaves, kHstuTimeOctaves, sizeof(kHstuTimeOctaves));
+  long long taus[kTauEntries];
+  taus[0] = -0x7fffffffffffffffLL - 1;
+  for (int k = 1; k <= HSTU_TB_NUM_THRESHOLDS; ++k) taus[k] = kHstuTimeThresholds[k - 1];
+  for (int k = HSTU_TB_NUM_THRESHOLDS + 1; k < kTauEntries; ++k) taus[k] = 0x7fffffffffffffffLL;
+  e = cudaMemcpyToSymbol(c_time_taus, taus, sizeof(taus));
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
   return e;
 }

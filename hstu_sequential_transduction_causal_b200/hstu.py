@@ -59,6 +59,11 @@ class hstu_layer_grads_t(ctypes.Structure):
     _fields_ = [(n, c_vp) for n in ("dW1", "db1", "dW2", "db2", "dgamma", "dbeta", "drab_pos", "drab_time")]
 
 
+class hstu_falcon_desc_t(ctypes.Structure):
+    _fields_ = [("L", c_i32), ("users", c_i32), ("m", c_i32), ("b_m", c_i32), ("D", c_i32), ("H", c_i32),
+                ("inv_N", c_f32), ("pos_max_len", c_i32), ("n_time_buckets", c_i32), ("ln_eps", c_f32)]
+
+
 P = ctypes.POINTER
 # name -> (restype, argtypes); the list every test checks against include/hstu.h
 SIGNATURES = {
@@ -88,11 +93,16 @@ SIGNATURES = {
                                       c_vp]),
     "hstu_norm_gate_fwd": (c_i32, [c_i64, c_i32, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp,
                                    c_f32, c_vp, c_vp, c_vp, c_vp]),
-    "hstu_out_proj_fwd": (c_i32, [c_i64, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_i32, c_vp,
+    "hstu_out_proj_workspace_size": (c_sz, [c_i32, c_i32]),
+    "hstu_out_proj_fwd": (c_i32, [c_i64, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_i32, c_vp,
                                   c_vp, c_sz, c_vp]),
     "hstu_layer_workspace_size": (c_sz, [P(hstu_layer_desc_t), P(hstu_jagged_t)]),
     "hstu_layer_fwd": (c_i32, [P(hstu_layer_desc_t), P(hstu_jagged_t), P(hstu_layer_weights_t), c_vp, c_vp,
                                c_vp, c_vp, P(hstu_layer_saved_t), c_vp, c_sz, c_vp]),
+    "hstu_falcon_cache_size": (c_sz, [P(hstu_falcon_desc_t), P(hstu_jagged_t)]),
+    "hstu_falcon_workspace_size": (c_sz, [P(hstu_falcon_desc_t), P(hstu_jagged_t)]),
+    "hstu_falcon_fwd": (c_i32, [P(hstu_falcon_desc_t), P(hstu_layer_weights_t), P(hstu_jagged_t), c_vp, c_vp, c_i32,
+                                c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -258,22 +268,25 @@ def hstu_norm_gate_fwd(T, D, o_dtype_code, u_dtype_code, g_dtype_code, o, ld_o, 
                                                           _ptr(rstd), _stream(stream)))
 
 
-def hstu_out_proj_fwd(T, D, dtype_code, g, W2, b2, x, x_dtype_code, y, y_dtype_code, y_bf16, ws,
+def hstu_out_proj_workspace_size(D: int, g_dtype_code: int) -> int:
+    return lib().hstu_out_proj_workspace_size(D, g_dtype_code)
+
+
+def hstu_out_proj_fwd(T, D, dtype_code, g_dtype_code, g, W2, b2, x, x_dtype_code, y, y_dtype_code, y_f16, ws,
                       stream=None) -> None:
-    _check("hstu_out_proj_fwd", lib().hstu_out_proj_fwd(T, D, dtype_code, _ptr(g), _ptr(W2), _ptr(b2), _ptr(x),
-                                                        x_dtype_code, _ptr(y), y_dtype_code, _ptr(y_bf16),
-                                                        _ptr(ws), ws.numel() * ws.element_size(),
-                                                        _stream(stream)))
+    _check("hstu_out_proj_fwd", lib().hstu_out_proj_fwd(T, D, dtype_code, g_dtype_code, _ptr(g), _ptr(W2), _ptr(b2),
+                                                        _ptr(x), x_dtype_code, _ptr(y), y_dtype_code, _ptr(y_f16),
+                                                        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def hstu_layer_workspace_size(desc: hstu_layer_desc_t, jag: hstu_jagged_t) -> int:
     return lib().hstu_layer_workspace_size(ctypes.byref(desc), ctypes.byref(jag))
 
 
-def hstu_layer_fwd(desc, jag, weights: hstu_layer_weights_t, x, x_bf16, y, y_bf16, saved: hstu_layer_saved_t,
+def hstu_layer_fwd(desc, jag, weights: hstu_layer_weights_t, x, x_f16, y, y_f16, saved: hstu_layer_saved_t,
                    ws, stream=None) -> None:
     _check("hstu_layer_fwd", lib().hstu_layer_fwd(ctypes.byref(desc), ctypes.byref(jag), ctypes.byref(weights),
-                                                  _ptr(x), _ptr(x_bf16), _ptr(y), _ptr(y_bf16),
+                                                  _ptr(x), _ptr(x_f16), _ptr(y), _ptr(y_f16),
                                                   ctypes.byref(saved), _ptr(ws), ws.numel() * ws.element_size(),
                                                   _stream(stream)))
 
@@ -298,13 +311,36 @@ def hstu_layer_bwd_workspace_size(desc: hstu_layer_desc_t, jag: hstu_jagged_t) -
     return lib().hstu_layer_bwd_workspace_size(ctypes.byref(desc), ctypes.byref(jag))
 
 
-def hstu_layer_bwd(desc, jag, weights: hstu_layer_weights_t, x, x_bf16, saved: hstu_layer_saved_t, dy, dy_bf16, dx,
-                   dx_bf16, grads: hstu_layer_grads_t, ws, stream=None) -> None:
+def hstu_layer_bwd(desc, jag, weights: hstu_layer_weights_t, x, x_f16, saved: hstu_layer_saved_t, dy, dy_f16, dx,
+                   dx_f16, grads: hstu_layer_grads_t, ws, stream=None) -> None:
     _check("hstu_layer_bwd", lib().hstu_layer_bwd(ctypes.byref(desc), ctypes.byref(jag), ctypes.byref(weights),
-                                                  _ptr(x), _ptr(x_bf16), ctypes.byref(saved), _ptr(dy),
-                                                  _ptr(dy_bf16), _ptr(dx), _ptr(dx_bf16), ctypes.byref(grads),
+                                                  _ptr(x), _ptr(x_f16), ctypes.byref(saved), _ptr(dy),
+                                                  _ptr(dy_f16), _ptr(dx), _ptr(dx_f16), ctypes.byref(grads),
                                                   _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def layer_grads(dW1, db1, dW2, db2, dgamma, dbeta, drab_pos, drab_time) -> hstu_layer_grads_t:
     return hstu_layer_grads_t(*[_ptr(t) for t in (dW1, db1, dW2, db2, dgamma, dbeta, drab_pos, drab_time)])
+
+
+def make_falcon_desc(L, users, m, b_m, D, H, inv_N, pos_max_len, n_time_buckets=128,
+                     ln_eps=1e-5) -> hstu_falcon_desc_t:
+    return hstu_falcon_desc_t(L, users, m, b_m, D, H, inv_N, pos_max_len, n_time_buckets, ln_eps)
+
+
+def hstu_falcon_cache_size(desc: hstu_falcon_desc_t, prefix: hstu_jagged_t) -> int:
+    return lib().hstu_falcon_cache_size(ctypes.byref(desc), ctypes.byref(prefix))
+
+
+def hstu_falcon_workspace_size(desc: hstu_falcon_desc_t, prefix: hstu_jagged_t) -> int:
+    return lib().hstu_falcon_workspace_size(ctypes.byref(desc), ctypes.byref(prefix))
+
+
+def hstu_falcon_fwd(desc: hstu_falcon_desc_t, layers, prefix: hstu_jagged_t, prefix_x, kv_cache, cache_valid,
+                    prefix_out, cand_x, request_ts, out, ws, stream=None) -> None:
+    """layers: a sequence of hstu_layer_weights_t (marshalled into the host array the call reads)."""
+    arr = (hstu_layer_weights_t * len(layers))(*layers)
+    _check("hstu_falcon_fwd", lib().hstu_falcon_fwd(ctypes.byref(desc), arr, ctypes.byref(prefix), _ptr(prefix_x),
+                                                    _ptr(kv_cache), int(cache_valid), _ptr(prefix_out),
+                                                    _ptr(cand_x), _ptr(request_ts), _ptr(out), _ptr(ws),
+                                                    ws.numel() * ws.element_size(), _stream(stream)))

@@ -60,11 +60,11 @@ class SavedActs:
 
     @classmethod
     def empty(cls, T: int, D: int, dtype: torch.dtype, keep_z: bool, device="cuda") -> "SavedActs":
-        act = torch.float16 if dtype == torch.bfloat16 else dtype     # U|V|Q|K and Z in fp16
+        act = torch.float16 if dtype == torch.bfloat16 else dtype     # U|V|Q|K, Z and G in fp16
         return cls(uvqk=torch.empty(T, 4 * D, dtype=act, device=device),
                    z=torch.empty(T, 4 * D, dtype=act, device=device) if keep_z else None,
                    o=torch.empty(T, D, dtype=torch.float32, device=device),
-                   g=torch.empty(T, D, dtype=dtype, device=device),
+                   g=torch.empty(T, D, dtype=act, device=device),
                    mu=torch.empty(T, dtype=torch.float32, device=device),
                    rstd=torch.empty(T, dtype=torch.float32, device=device))
 
@@ -108,9 +108,9 @@ class LayerRunner:
         self.y = torch.empty(jag.T, layer.D, dtype=y_dtype, device=device)
         self.weights = layer.weights()
 
-    def forward(self, x: torch.Tensor, x_bf16: Optional[torch.Tensor] = None,
-                y_bf16: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-        H.hstu_layer_fwd(self.desc, self.jag.struct, self.weights, x, x_bf16, self.y, y_bf16,
+    def forward(self, x: torch.Tensor, x_f16: Optional[torch.Tensor] = None,
+                y_f16: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        H.hstu_layer_fwd(self.desc, self.jag.struct, self.weights, x, x_f16, self.y, y_f16,
                          self.saved_struct, self.ws, stream)
         return self.y
 

@@ -204,7 +204,8 @@ class FalconWorkload:
 
 
 def make_falcon_workload(seed: int = 0, *, users=None, prefix=None, m=None, b_m=None,
-                         D=None, H=None, layers=None, N=None, pos_max_len=None) -> FalconWorkload:
+                         D=None, H=None, layers=None, N=None, pos_max_len=None,
+                         prefix_lengths=None) -> FalconWorkload:
     cfg = dict(CONFIGS["c5"])
     for k, v in dict(users=users, prefix=prefix, m=m, b_m=b_m, D=D, H=H, layers=layers, N=N,
                      pos_max_len=pos_max_len).items():
@@ -212,12 +213,16 @@ def make_falcon_workload(seed: int = 0, *, users=None, prefix=None, m=None, b_m=
             cfg[k] = v
     rng = np.random.default_rng(seed)
     U, n, D = cfg["users"], cfg["prefix"], cfg["D"]
-    lens = np.full(U, n, dtype=np.int64)
+    if prefix_lengths is not None:      # ragged prefixes (tests); users follows the list
+        lens = np.asarray(prefix_lengths, dtype=np.int64)
+        U = cfg["users"] = len(lens)
+    else:
+        lens = np.full(U, n, dtype=np.int64)
     off = offsets_from_lengths(lens)
     ts = draw_timestamps(rng, lens)
-    last = ts[off[1:] - 1] if n > 0 else np.full(U, T0, dtype=np.int64)
+    last = np.array([ts[off[u + 1] - 1] if lens[u] > 0 else T0 for u in range(U)], dtype=np.int64)
     req = last + np.floor(rng.exponential(GAP_MEAN_S, size=U)).astype(np.int64)
-    px = round_bf16(rng.standard_normal((U * n, D)))
+    px = round_bf16(rng.standard_normal((int(off[-1]), D)))
     cx = round_bf16(rng.standard_normal((U * cfg["m"], D)))
     layer_list = [draw_layer(rng, D, cfg["pos_max_len"], True) for _ in range(cfg["layers"])]
     return FalconWorkload(D=D, H=cfg["H"], N=float(cfg["N"]), pos_max_len=cfg["pos_max_len"],

@@ -95,10 +95,13 @@ typedef struct hstu_layer_desc_t {
   int32_t pos_max_len;
   int32_t n_time_buckets;
   float ln_eps;            /* LayerNorm epsilon (1e-5) */
-  hstu_dtype_t dtype;      /* BF16: bf16 X / W1 / W2 / G on the tensor cores with fp32 accumulation,
-                              U|V|Q|K, Z and the attention weights P in fp16, O in fp32;
+  hstu_dtype_t dtype;      /* BF16: bf16 weights and activations on the tensor cores with fp32
+                              accumulation: U|V|Q|K, Z, the attention weights P and G in fp16
+                              (8x finer than bf16 at the same MMA rate), O in fp32; f2 reads an
+                              fp16 copy of W2 (exact for bf16 values in the fp16 range);
                               F32: every step in fp32 on the CUDA cores */
-  hstu_dtype_t x_dtype;    /* dtype of X; F32 with BF16 compute = fp32 residual stream */
+  hstu_dtype_t x_dtype;    /* dtype of X; F32 with BF16 compute = fp32 residual stream (f1 then
+                              reads an fp16 copy of X and of W1) */
   hstu_dtype_t y_dtype;    /* dtype of Y */
 } hstu_layer_desc_t;
 
@@ -115,9 +118,9 @@ typedef struct hstu_layer_weights_t {
   const float* rab_time;
 } hstu_layer_weights_t;
 
-/* Activations a layer forward writes and its backward reads. In BF16 mode uvqk [T, 4D] = SiLU(Z)
- * and z [T, 4D] (the pre-activation; may be NULL when no backward follows) are fp16 and g is
- * bf16; in F32 mode all are fp32.
+/* Activations a layer forward writes and its backward reads. In BF16 mode uvqk [T, 4D] = SiLU(Z),
+ * z [T, 4D] (the pre-activation; may be NULL when no backward follows) and g are fp16; in F32
+ * mode all are fp32.
  * o [T, D] attention output, always fp32 (LayerNorm divides by its spread across features,
  * which is far smaller than its mean, so bf16 storage would be amplified); g [T, D] =
  * LN(O) (.) U; mu, rstd [T] fp32 LayerNorm statistics. */
@@ -260,8 +263,8 @@ hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_desc_t* desc, const hstu_jag
 /* LayerNorm (.) U gating ("Generative Recommenders and HSTU", third equation; "HSTU: The First
  * Exploration of the Scaling Law", 7.1.4 Innovation 3): g = (gamma (o - mu) rstd + beta) (.) u
  * over all D features of a token; mu, rstd (fp32 [T]) are stored for the backward. g is [T, D]
- * with row stride D. Supported (o, u, g) dtypes: (F32, F32, F32), (F32, F16 or BF16, BF16),
- * (BF16, BF16, BF16). D in {64, 128, 256, 512, 1024}. */
+ * with row stride D. Supported (o, u, g) dtypes: (F32, F32, F32), (F32, F16, F16),
+ * (F32, F16 or BF16, BF16), (BF16, BF16, BF16). D in {64, 128, 256, 512, 1024}. */
 hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t o_dtype, hstu_dtype_t u_dtype,
                                  hstu_dtype_t g_dtype, const void* o, int64_t ld_o, const void* u,
                                  int64_t ld_u, const float* gamma,
@@ -269,25 +272,28 @@ hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t o_dtype, hst
                                  hstu_stream_t stream);
 
 /* f2 + residual ("Generative Recommenders and HSTU", third equation; residual of the "Code"
- * sketch): y = g W2^T + b2 + x. g, W2 have the compute dtype; x has x_dtype; y has y_dtype;
- * y_bf16 (nullable) receives a second, bf16 copy of y (the next layer's GEMM operand).
- * ws: any workspace of at least 256 bytes (status word). F32 compute needs F32 x and y. */
-hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, const void* g,
-                                const void* W2, const float* b2, const void* x,
+ * sketch): y = g W2^T + b2 + x. W2 has the compute dtype `dtype`; g has g_dtype (F32 compute: F32;
+ * BF16 compute: BF16, or F16 with W2 read through an fp16 copy made in the workspace); x has
+ * x_dtype; y has y_dtype; y_f16 (nullable) receives a second, fp16 copy of y (the next layer's
+ * f1 operand when the residual stream is fp32). ws: at least hstu_out_proj_workspace_size(D, g_dtype)
+ * bytes (status word, fp16 W2). F32 compute needs F32 x and y. */
+size_t hstu_out_proj_workspace_size(int32_t D, hstu_dtype_t g_dtype);
+hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t g_dtype,
+                                const void* g, const void* W2, const float* b2, const void* x,
                                 hstu_dtype_t x_dtype, void* y, hstu_dtype_t y_dtype,
-                                void* y_bf16, void* ws, size_t ws_bytes, hstu_stream_t stream);
+                                void* y_f16, void* ws, size_t ws_bytes, hstu_stream_t stream);
 
 /* Workspace bytes hstu_layer_fwd / hstu_layer_bwd need. */
 size_t hstu_layer_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
 
 /* Whole layer forward: uvqk -> attention -> norm-gate -> out-projection, on `stream`.
- * x: [T, D] of desc->x_dtype; x_bf16 (nullable) a bf16 copy of x used as the f1 operand when
- * x_dtype is F32 with BF16 compute (converted into the workspace when NULL). y: [T, D] of
- * desc->y_dtype; y_bf16 nullable second output. saved: buffers for the intermediates (all
- * required except z). */
+ * x: [T, D] of desc->x_dtype; x_f16 (nullable) an fp16 copy of x, the f1 operand when x_dtype is
+ * F32 with BF16 compute (converted into the workspace when NULL; ignored otherwise). y: [T, D] of
+ * desc->y_dtype; y_f16 (nullable) a second, fp16 copy of y (the next stacked layer's x_f16).
+ * saved: buffers for the intermediates (all required except z). */
 hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag,
-                             const hstu_layer_weights_t* w, const void* x, const void* x_bf16,
-                             void* y, void* y_bf16, const hstu_layer_saved_t* saved, void* ws,
+                             const hstu_layer_weights_t* w, const void* x, const void* x_f16,
+                             void* y, void* y_f16, const hstu_layer_saved_t* saved, void* ws,
                              size_t ws_bytes, hstu_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
@@ -310,16 +316,72 @@ hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
 size_t hstu_layer_bwd_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
 
 /* Whole layer backward (BF16 mode, D in {256, 512}), from the activations hstu_layer_fwd saved
- * (z required). dy: [T, D] of desc->y_dtype (dy_bf16: nullable bf16 copy); dx: [T, D] of
- * desc->x_dtype, overwritten with dy + dZ W1 (dx_bf16: nullable bf16 copy). Steps: dG = dy W2,
+ * (z required). x_f16: nullable fp16 copy of x (the dW1 operand; converted when NULL). dy: [T, D]
+ * of desc->y_dtype (dy_f16: nullable fp16 copy, the operand of dG and dW2; converted when NULL);
+ * dx: [T, D] of desc->x_dtype, overwritten with dy + dZ W1 (dx_f16: nullable fp16 copy, the
+ * previous stacked layer's dy_f16). Every GEMM reads fp16 operands (exact copies of bf16 data).
+ * Steps: dG = dy W2,
  * dW2 = dy^T G, db2 = sum dy; LayerNorm (.) U backward (dO, dU, dgamma, dbeta); attention
  * backward (dQ, dK, dV, table gradients); dZ = [dU|dV|dQ|dK] (.) SiLU'(Z); dW1 = dZ^T X,
  * db1 = sum dZ, dX = dy + dZ W1. All gradients fp32 and overwritten. */
 hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag,
-                             const hstu_layer_weights_t* w, const void* x, const void* x_bf16,
-                             const hstu_layer_saved_t* saved, const void* dy, const void* dy_bf16,
-                             void* dx, void* dx_bf16, const hstu_layer_grads_t* grads, void* ws,
+                             const hstu_layer_weights_t* w, const void* x, const void* x_f16,
+                             const hstu_layer_saved_t* saved, const void* dy, const void* dy_f16,
+                             void* dx, void* dx_f16, const hstu_layer_grads_t* grads, void* ws,
                              size_t ws_bytes, hstu_stream_t stream);
+
+/* --------------------------------------------------------------------------------------------
+ * M-FALCON candidate scoring ("HSTU: The First Exploration of the Scaling Law", 7.1.5 M-FALCON).
+ *
+ * A stack of L layers (all BF16 mode, one hstu_layer_weights_t each) scores m candidates per
+ * user against that user's history (the prefix). Layer l of candidate c of user u sees, as keys,
+ * every prefix token j of u through layer l (relative position n_u - j, time difference
+ * request_ts[u] - t_j) and itself (relative position 0, time difference 0); candidates never see
+ * one another. Its attention output is
+ *   O_c = inv_N * ( sum_j SiLU(q_c.k_j + rab_pos[idx(n_u - j)] + rab_time[bucket(request_ts[u] - t_j)]) v_j
+ *                   + SiLU(q_c.k_c + rab_pos[idx(0)] + rab_time[0]) v_c ),
+ * which equals the last row of a causal layer over [prefix, c]; LayerNorm (.) U, f2 and the
+ * residual follow as in hstu_layer_fwd, and the layer's output is the next layer's input. The
+ * residual stream between layers is fp32 (BF16 compute with an fp32 X, as in a stacked encoder).
+ *
+ * The prefix's K and V of every layer are computed once (cache_valid = 0: the prefix runs through
+ * the L causal layers and kv_cache is filled) and reused by every candidate micro-batch of b_m
+ * candidates per user (the result does not depend on b_m). With cache_valid = 1, kv_cache must
+ * hold the K|V of the same prefix and weights from an earlier call, and prefix_x is not read.
+ * -------------------------------------------------------------------------------------------- */
+typedef struct hstu_falcon_desc_t {
+  int32_t L;               /* layers (>= 1) */
+  int32_t users;           /* number of users == prefix->B */
+  int32_t m;               /* candidates per user (>= 0) */
+  int32_t b_m;             /* candidates per user in one pass (micro-batch), >= 1 */
+  int32_t D, H;            /* d_model, heads (D/H = 64) */
+  float inv_N;
+  int32_t pos_max_len;     /* every n_u < pos_max_len keeps the positions unclipped */
+  int32_t n_time_buckets;
+  float ln_eps;
+} hstu_falcon_desc_t;
+
+/* Bytes of the K|V cache: L x T_prefix x 2D fp16 (layer l, token t: K in columns [0, D), V in
+ * [D, 2D)). The caller owns it; it outlives a call when cache_valid = 1 is used later. */
+size_t hstu_falcon_cache_size(const hstu_falcon_desc_t* desc, const hstu_jagged_t* prefix);
+size_t hstu_falcon_workspace_size(const hstu_falcon_desc_t* desc, const hstu_jagged_t* prefix);
+
+/* layers: HOST array of L weight structs (device pointers inside, W1/W2 bf16).
+ * prefix: B = users jagged prefixes (offsets, int64 timestamps), max_len >= every n_u.
+ * prefix_x: bf16 [T_prefix, D] (read only when cache_valid = 0).
+ * kv_cache: fp16, hstu_falcon_cache_size() bytes; written when cache_valid = 0, read always.
+ * prefix_out: fp32 [T_prefix, D], the prefix's output of the last layer, or NULL (only written
+ *   when cache_valid = 0).
+ * cand_x: bf16 [users * m, D], user u's candidates in rows [u m, (u+1) m).
+ * request_ts: device int64 [users], the request time of each user.
+ * out: fp32 [users * m, D], the candidates' output of the last layer.
+ * Errors: the host checks of hstu_layer_fwd (D % 64 == 0, D/H == 64) plus
+ * HSTU_ERR_INVALID_ARG for users != prefix->B, L < 1 or b_m < 1. */
+hstu_status_t hstu_falcon_fwd(const hstu_falcon_desc_t* desc, const hstu_layer_weights_t* layers,
+                              const hstu_jagged_t* prefix, const void* prefix_x, void* kv_cache,
+                              int32_t cache_valid, void* prefix_out, const void* cand_x,
+                              const int64_t* request_ts, void* out, void* ws, size_t ws_bytes,
+                              hstu_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -73,6 +73,26 @@ def test_time_buckets_bit_exact():
         assert np.array_equal(got[sq[b]:sq[b + 1]].astype(np.int64), exp), b
 
 
+def test_time_buckets_every_threshold_edge():
+    """Differences tau_k - 1, tau_k, tau_k + 1 for every threshold (and 0, 1, 2, int64-sized gaps)
+    against the first token: each bucket edge is hit from both sides."""
+    vals = [0, 1, 2]
+    for t in THR:
+        vals += [int(t) - 1, int(t), int(t) + 1]
+    vals += [2 ** 40, 2 ** 55 + 3, 2 ** 62 - 1]
+    ts = np.array(vals, dtype=np.int64)
+    n = len(ts)
+    off = np.array([0, n], np.int64)
+    jag = JaggedBatch(off, ts)
+    sq = np.array([0, n * n], np.int64)
+    out = torch.full((n * n,), 255, dtype=torch.uint8, device="cuda")
+    H.hstu_time_buckets(jag.struct, 128, to_dev(sq, torch.int64), out)
+    got = out.cpu().numpy().astype(np.int64).reshape(n, n)
+    exp = O.time_bucket(ts[:, None] - ts[None, :], THR)
+    assert np.array_equal(got, exp)
+    assert np.array_equal(got[:, 0], O.time_bucket(ts, THR))
+
+
 # ---------------------------------------------------------------------------------------------
 # single steps
 # ---------------------------------------------------------------------------------------------
@@ -202,25 +222,30 @@ def test_norm_gate_bf16(o_bf16):
     assert_close(rstd.cpu().numpy(), rse, 1e-6, 1e-4, what="rstd")
 
 
-@pytest.mark.parametrize("xdt,ydt", [("bf16", "bf16"), ("f32", "f32")])
-def test_out_proj_bf16(xdt, ydt):
+@pytest.mark.parametrize("xdt,ydt,gdt", [("bf16", "bf16", "bf16"), ("f32", "f32", "bf16"), ("bf16", "f32", "f16"),
+                                         ("f32", "f32", "f16")])
+def test_out_proj_bf16(xdt, ydt, gdt):
     rng = np.random.default_rng(6)
     T, D = 300, 512
-    g = _bf16(rng.standard_normal((T, D)))
+    tg = torch.bfloat16 if gdt == "bf16" else torch.float16
+    g = _bf16(rng.standard_normal((T, D))) if gdt == "bf16" else \
+        rng.standard_normal((T, D)).astype(np.float16).astype(np.float32)
     W2 = _bf16(rng.standard_normal((D, D)) / np.sqrt(D))
     b2 = (0.1 * rng.standard_normal(D)).astype(np.float32)
     x = _bf16(rng.standard_normal((T, D))) if xdt == "bf16" else rng.standard_normal((T, D)).astype(np.float32)
     tx = torch.bfloat16 if xdt == "bf16" else torch.float32
     ty = torch.bfloat16 if ydt == "bf16" else torch.float32
     y = torch.empty(T, D, dtype=ty, device="cuda")
-    y2 = torch.empty(T, D, dtype=torch.bfloat16, device="cuda")
-    ws = workspace(256)
-    H.hstu_out_proj_fwd(T, D, H.HSTU_BF16, to_dev(g, torch.bfloat16), to_dev(W2, torch.bfloat16),
+    y2 = torch.empty(T, D, dtype=torch.float16, device="cuda")
+    gcode = H._dtype_code(y.new_empty(0, dtype=tg))
+    ws = workspace(H.hstu_out_proj_workspace_size(D, gcode))
+    H.hstu_out_proj_fwd(T, D, H.HSTU_BF16, gcode, to_dev(g, tg), to_dev(W2, torch.bfloat16),
                         to_dev(b2, torch.float32), to_dev(x, tx), H._dtype_code(y.new_empty(0, dtype=tx)), y,
                         H._dtype_code(y), y2, ws)
     ye = O.out_proj_fwd(g, W2, b2, x)
-    assert_close(y.float().cpu().numpy(), ye, *BF16_TOL, what="Y")
-    assert_close(y2.float().cpu().numpy(), ye, *BF16_TOL, what="Y bf16 copy")
+    tol = BF16_TOL if ydt == "bf16" else (1e-3, 1e-3)     # fp32 output: only accumulation-order error
+    assert_close(y.float().cpu().numpy(), ye, *tol, what="Y")
+    assert_close(y2.float().cpu().numpy(), ye, *BF16_TOL, what="Y fp16 copy")
 
 
 # ---------------------------------------------------------------------------------------------
@@ -267,22 +292,32 @@ def test_layer_fwd_long_sequences_sampled_rows():
 
 
 def test_layer_fwd_fp32_residual_stream():
+    """An fp32 residual stream: the oracle takes the fp32 X as it is (the kernels' fp16 f1 operand
+    is their own rounding), the residual is added in fp32."""
     wl = W.make_workload("c4", seed=1, lengths=[200, 1, 0, 385, 128], layers=1)
     x32 = np.random.default_rng(9).standard_normal((wl.T, wl.D)).astype(np.float32)
     y, run = _run_layer(wl, torch.float32, torch.float32, x_override=x32)
     assert run.device_status() == 0
-    # the f1 operand is the bf16 rounding of the fp32 residual; the residual itself stays fp32
-    p = wl.layers[0]
-    xr = W.round_bf16(x32)
-    D = wl.D
-    z, s = O.uvqk_fwd(xr, p.W1, p.b1)
-    u, v, q, k = O.split_uvqk(s, D)
-    T, d = wl.T, D // wl.H
-    o = O.pointwise_attention_fwd(q.reshape(T, wl.H, d), k.reshape(T, wl.H, d), v.reshape(T, wl.H, d), wl.offsets,
-                                  wl.timestamps, p.rab_pos, p.rab_time, 1 / wl.N, wl.pos_max_len, THR).reshape(T, D)
-    g, _, _ = O.norm_gate_fwd(o, u, p.gamma, p.beta)
-    ye = O.out_proj_fwd(g, p.W2, p.b2, x32)
+    ye, _ = layer_oracle(wl, x=x32)
     assert_close(y, ye, *BF16_TOL, what="Y fp32 residual")
+
+
+def test_layer_fwd_fp16_copies_match_the_fp32_path():
+    """x_f16 / y_f16: a layer fed the fp16 copy of its input gives the same bits as one that converts
+    it itself, and its y_f16 output is the fp16 rounding of y."""
+    wl = W.make_workload("c4", seed=3, lengths=[130, 77], layers=1)
+    x32 = np.random.default_rng(4).standard_normal((wl.T, wl.D)).astype(np.float32)
+    jag = JaggedBatch(wl.offsets, wl.timestamps)
+    layer = DeviceLayer.upload(wl.layers[0], wl.D, wl.H, True)
+    run = LayerRunner(layer, jag, 1.0 / wl.N, wl.pos_max_len, torch.float32, torch.float32, keep_z=True)
+    x = to_dev(x32, torch.float32)
+    y_a = run.forward(x).clone()
+    y16 = torch.empty(wl.T, wl.D, dtype=torch.float16, device="cuda")
+    y_b = run.forward(x, x.half(), y16).clone()
+    torch.cuda.synchronize()
+    assert run.device_status() == 0
+    assert torch.equal(y_a, y_b)
+    assert torch.equal(y16, y_b.half())
 
 
 # ---------------------------------------------------------------------------------------------

@@ -119,19 +119,12 @@ def test_layer_bwd_d256_four_heads():
 
 
 def test_layer_bwd_fp32_residual_stream():
+    """fp32 X and dY: the oracle takes them as they are (the kernels read fp16 copies)."""
     wl = W.make_workload("c4", seed=4, lengths=[150, 260, 1], layers=1)
     wl.x = np.random.default_rng(5).standard_normal((wl.T, wl.D)).astype(np.float32)
     wl.dy = np.random.default_rng(6).standard_normal((wl.T, wl.D)).astype(np.float32)
     dx, grads = _run_layer_fwd_bwd(wl, torch.float32)
-    # the f1/f2 operands are the bf16 roundings of the fp32 residual stream and of dy
-    p = wl.layers[0]
-    xr = W.round_bf16(wl.x)
-    y, sv = O.layer_fwd(xr, p, wl.offsets, wl.timestamps, wl.H, 1.0 / wl.N, wl.pos_max_len, THR)
-    sv["x"] = xr
-    ref = O.layer_bwd(W.round_bf16(wl.dy), p, sv, wl.offsets, wl.timestamps, wl.H, 1.0 / wl.N, wl.pos_max_len, THR)
-    ref["dx"] = ref["dx"] - W.round_bf16(wl.dy) + wl.dy          # the residual adds the fp32 dy itself
-    ref["db2"] = wl.dy.astype(np.float64).sum(axis=0)              # db2 sums the fp32 dy
-    _compare(dx, grads, ref, "fp32-residual ")
+    _compare(dx, grads, _oracle_grads(wl), "fp32-residual ")
 
 
 def test_layer_bwd_long_sequence_workload_full():
