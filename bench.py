@@ -238,11 +238,12 @@ def main():
     ws = workspace(max(H.hstu_attn_workspace_size(adesc, jag.struct),
                        H.hstu_layer_bwd_workspace_size(ldesc, jag.struct) if backward else 0), dev)
     sizes = [4 * D * D, 4 * D, D * D, D, D, D, 2 * wl.pos_max_len - 1, 128]
-    flat = torch.zeros(sum(sizes), dtype=torch.float32, device=dev)
+    padded = [(n_ + 3) // 4 * 4 for n_ in sizes]      # every gradient view 16-byte aligned
+    flat = torch.zeros(sum(padded), dtype=torch.float32, device=dev)
     views, o = [], 0
-    for n_ in sizes:
+    for n_, pn in zip(sizes, padded):
         views.append(flat[o:o + n_])
-        o += n_
+        o += pn
     grads = H.layer_grads(*views)
     weights = layer.weights()
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)

@@ -552,6 +552,11 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   if (!x || !y || !w->W1 || !w->b1 || !w->W2 || !w->b2 || !w->gamma || !w->beta || !w->rab_pos || !w->rab_time ||
       !saved->uvqk || !saved->o || !saved->g || !saved->mu || !saved->rstd)
     return HSTU_ERR_INVALID_ARG;
+  if (desc->dtype == HSTU_BF16) {   // 16-byte vector and TMA access
+    const void* v16[] = {x, x_f16, y, y_f16, saved->uvqk, saved->z, saved->o, saved->g, w->W1, w->W2};
+    for (const void* p : v16)
+      if (p && !aligned16(p)) return HSTU_ERR_UNSUPPORTED;
+  }
   cudaStream_t st = stream;
   int* status = ws_status(ws);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -658,6 +663,13 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   }
   if (!x || !dy || !dx || !saved->uvqk || !saved->z || !saved->o || !saved->g || !saved->mu || !saved->rstd)
     return HSTU_ERR_INVALID_ARG;
+  // 16-byte vector loads, stores and atomics (dW1 and dW2 are accumulated by float4 atomics)
+  {
+    const void* v16[] = {x, x_f16, dy, dy_f16, dx, dx_f16, saved->uvqk, saved->z, saved->o, saved->g,
+                         w->W1, w->W2, gr->dW1, gr->dW2};
+    for (const void* p : v16)
+      if (p && !aligned16(p)) return HSTU_ERR_UNSUPPORTED;
+  }
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   int* status = ws_status(ws);
   // fp16 operands: dy (of dG and dW2, next to fp16 G and W2), x (of dW1, next to fp16 dZ), W1, W2
@@ -1015,4 +1027,37 @@ extern "C" hstu_status_t hstu_falcon_fwd(const hstu_falcon_desc_t* desc, const h
     }
   }
   return HSTU_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Stochastic Length
+// ---------------------------------------------------------------------------------------------
+extern "C" hstu_status_t hstu_stochastic_length_offsets(const hstu_jagged_t* raw, double alpha, int64_t* new_offsets,
+                                                        void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  hstu_status_t s = check_jagged(raw);
+  if (s != HSTU_OK) return s;
+  if (!new_offsets || !ws || !(alpha >= 0.0) || !(alpha <= 2.0)) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < kWsHeader) return HSTU_ERR_WORKSPACE;
+  return cuda_status(launch_sl_lengths(raw->offsets, raw->B, alpha, new_offsets, ws_status(ws), stream));
+}
+
+extern "C" hstu_status_t hstu_stochastic_length_select(const hstu_jagged_t* raw, const int64_t* keys,
+                                                       const int64_t* new_offsets, const void* x, hstu_dtype_t x_dtype,
+                                                       int32_t D, int64_t* kept, void* x_out, int64_t* ts_out,
+                                                       void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  hstu_status_t s = check_jagged(raw);
+  if (s != HSTU_OK) return s;
+  if (!new_offsets || !kept || !ws || (raw->T > 0 && !keys)) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < kWsHeader) return HSTU_ERR_WORKSPACE;
+  int64_t row_bytes = 0;
+  if (x_out) {
+    if (!x || D <= 0) return HSTU_ERR_INVALID_ARG;
+    const int64_t es = x_dtype == HSTU_F32 ? 4 : (x_dtype == HSTU_BF16 || x_dtype == HSTU_F16) ? 2 : 0;
+    if (es == 0) return HSTU_ERR_UNSUPPORTED;
+    row_bytes = es * D;
+    if (row_bytes % 16 || !aligned16(x) || !aligned16(x_out)) return HSTU_ERR_UNSUPPORTED;
+  }
+  if (raw->T == 0) return HSTU_OK;
+  return cuda_status(launch_sl_select(raw->offsets, raw->B, raw->timestamps, keys, new_offsets, x, row_bytes, kept,
+                                      x_out, ts_out, ws_status(ws), stream));
 }

@@ -174,4 +174,13 @@ cudaError_t column_sum(const void* in, int dt, int64_t rows, int cols, int64_t l
 
 cudaError_t launch_timeout_probe(int* status, cudaStream_t st);
 
+// ---------------------------------------------------------------------------------------------
+// Stochastic Length (stochastic_length.cu)
+// ---------------------------------------------------------------------------------------------
+cudaError_t launch_sl_lengths(const int64_t* offsets, int B, double alpha, int64_t* new_offsets, int* status,
+                              cudaStream_t st);
+cudaError_t launch_sl_select(const int64_t* offsets, int B, const int64_t* ts, const int64_t* keys,
+                             const int64_t* new_offsets, const void* x, int64_t row_bytes, int64_t* kept, void* x_out,
+                             int64_t* ts_out, int* status, cudaStream_t st);
+
 }  // namespace hstu

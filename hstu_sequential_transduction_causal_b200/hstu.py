@@ -99,6 +99,9 @@ SIGNATURES = {
     "hstu_layer_workspace_size": (c_sz, [P(hstu_layer_desc_t), P(hstu_jagged_t)]),
     "hstu_layer_fwd": (c_i32, [P(hstu_layer_desc_t), P(hstu_jagged_t), P(hstu_layer_weights_t), c_vp, c_vp,
                                c_vp, c_vp, P(hstu_layer_saved_t), c_vp, c_sz, c_vp]),
+    "hstu_stochastic_length_offsets": (c_i32, [P(hstu_jagged_t), ctypes.c_double, c_vp, c_vp, c_sz, c_vp]),
+    "hstu_stochastic_length_select": (c_i32, [P(hstu_jagged_t), c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp,
+                                              c_vp, c_sz, c_vp]),
     "hstu_falcon_cache_size": (c_sz, [P(hstu_falcon_desc_t), P(hstu_jagged_t)]),
     "hstu_falcon_workspace_size": (c_sz, [P(hstu_falcon_desc_t), P(hstu_jagged_t)]),
     "hstu_falcon_fwd": (c_i32, [P(hstu_falcon_desc_t), P(hstu_layer_weights_t), P(hstu_jagged_t), c_vp, c_vp, c_i32,
@@ -344,3 +347,17 @@ def hstu_falcon_fwd(desc: hstu_falcon_desc_t, layers, prefix: hstu_jagged_t, pre
                                                     _ptr(kv_cache), int(cache_valid), _ptr(prefix_out),
                                                     _ptr(cand_x), _ptr(request_ts), _ptr(out), _ptr(ws),
                                                     ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def hstu_stochastic_length_offsets(raw: hstu_jagged_t, alpha: float, new_offsets, ws, stream=None) -> None:
+    _check("hstu_stochastic_length_offsets",
+           lib().hstu_stochastic_length_offsets(ctypes.byref(raw), float(alpha), _ptr(new_offsets), _ptr(ws),
+                                                ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def hstu_stochastic_length_select(raw: hstu_jagged_t, keys, new_offsets, x, x_dtype_code, D, kept, x_out, ts_out, ws,
+                                  stream=None) -> None:
+    _check("hstu_stochastic_length_select",
+           lib().hstu_stochastic_length_select(ctypes.byref(raw), _ptr(keys), _ptr(new_offsets), _ptr(x), x_dtype_code,
+                                               D, _ptr(kept), _ptr(x_out), _ptr(ts_out), _ptr(ws),
+                                               ws.numel() * ws.element_size(), _stream(stream)))

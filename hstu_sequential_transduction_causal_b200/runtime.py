@@ -116,3 +116,96 @@ class LayerRunner:
 
     def device_status(self) -> int:
         return H.hstu_sync_status(self.ws)
+
+
+class Encoder:
+    """A stack of HSTU layers on an fp32 residual stream (BF16 compute).
+
+    forward() keeps each layer's input and saved activations; backward() runs the layers in reverse
+    and returns dX of the stack, leaving each layer's parameter gradients in ``grads[l]``. Every
+    step is one hstu_layer_fwd / hstu_layer_bwd call; layer l hands layer l+1 the fp16 copy of its
+    output (the next f1 operand) and, going back, the fp16 copy of its dX (the next dy operand).
+    """
+
+    def __init__(self, layers, jag: JaggedBatch, inv_N: float, pos_max_len: int, device="cuda"):
+        self.layers, self.jag = list(layers), jag
+        L, D, T = len(self.layers), self.layers[0].D, jag.T
+        self.desc = H.make_layer_desc(D, self.layers[0].H, inv_N, pos_max_len, H.HSTU_BF16, H.HSTU_F32, H.HSTU_F32)
+        self.weights = [lay.weights() for lay in self.layers]
+        self.saved = [SavedActs.empty(T, D, torch.bfloat16, True, device) for _ in range(L)]
+        self.saved_structs = [sv.struct() for sv in self.saved]
+        self.xs = [None] + [torch.empty(T, D, dtype=torch.float32, device=device) for _ in range(L - 1)]
+        self.x16 = [None] + [torch.empty(T, D, dtype=torch.float16, device=device) for _ in range(L - 1)]
+        self.y = torch.empty(T, D, dtype=torch.float32, device=device)
+        self.dx = [torch.empty(T, D, dtype=torch.float32, device=device) for _ in range(2)]
+        self.dx16 = [torch.empty(T, D, dtype=torch.float16, device=device) for _ in range(2)]
+        self.ws = workspace(max(H.hstu_layer_workspace_size(self.desc, jag.struct),
+                                H.hstu_layer_bwd_workspace_size(self.desc, jag.struct)), device)
+        # one flat fp32 row per layer, every view starting on a 16-byte boundary (the weight
+        # gradients are accumulated with 16-byte vector atomics)
+        sizes = [4 * D * D, 4 * D, D * D, D, D, D, 2 * pos_max_len - 1, 128]
+        padded = [(n_ + 3) // 4 * 4 for n_ in sizes]
+        self.grad_flat = torch.zeros(L, sum(padded), dtype=torch.float32, device=device)
+        self.grads = []
+        for l in range(L):
+            views, o = [], 0
+            for n_, pn in zip(sizes, padded):
+                views.append(self.grad_flat[l, o:o + n_])
+                o += pn
+            self.grads.append(views)
+        self.grad_structs = [H.layer_grads(*g) for g in self.grads]
+
+    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        """x: fp32 [T, D] (kept by reference until backward)."""
+        self.xs[0] = x
+        L = len(self.layers)
+        for l in range(L):
+            last = l == L - 1
+            y = self.y if last else self.xs[l + 1]
+            H.hstu_layer_fwd(self.desc, self.jag.struct, self.weights[l], self.xs[l], self.x16[l], y,
+                             None if last else self.x16[l + 1], self.saved_structs[l], self.ws, stream)
+        return self.y
+
+    def backward(self, dy: torch.Tensor, stream=None) -> torch.Tensor:
+        g, g16 = dy, None
+        for l in reversed(range(len(self.layers))):
+            dx, dx16 = self.dx[l & 1], self.dx16[l & 1]
+            H.hstu_layer_bwd(self.desc, self.jag.struct, self.weights[l], self.xs[l], self.x16[l],
+                             self.saved_structs[l], g, g16, dx, dx16 if l > 0 else None, self.grad_structs[l],
+                             self.ws, stream)
+            g, g16 = dx, dx16
+        return g
+
+    def device_status(self) -> int:
+        return H.hstu_sync_status(self.ws)
+
+
+def stochastic_length(raw: JaggedBatch, keys: torch.Tensor, alpha: float, x: Optional[torch.Tensor] = None,
+                      device="cuda"):
+    """Subsamples a raw jagged batch on the GPU. Returns (JaggedBatch of the kept tokens, kept raw
+    indices, kept rows of x or None). One host read of the kept-token count sizes the outputs."""
+    ws = workspace(256, device)
+    new_off = torch.empty(raw.B + 1, dtype=torch.int64, device=device)
+    H.hstu_stochastic_length_offsets(raw.struct, alpha, new_off, ws)
+    off_host = new_off.cpu().numpy()
+    if H.hstu_sync_status(ws) != 0:
+        raise RuntimeError("malformed raw offsets")
+    T2 = int(off_host[-1])
+    kept = torch.empty(max(T2, 1), dtype=torch.int64, device=device)
+    ts = torch.empty(max(T2, 1), dtype=torch.int64, device=device)
+    x_out = None
+    code = None
+    if x is not None:
+        x_out = torch.empty(max(T2, 1), x.shape[1], dtype=x.dtype, device=device)
+        code = H._dtype_code(x)
+    H.hstu_stochastic_length_select(raw.struct, keys, new_off, x, code if code is not None else 0,
+                                    x.shape[1] if x is not None else 0, kept, x_out, ts, ws)
+    if H.hstu_sync_status(ws) != 0:
+        raise RuntimeError("stochastic length selection reported an error")
+    lens = np.diff(off_host)
+    jag = JaggedBatch.__new__(JaggedBatch)
+    jag.offsets_np, jag.B, jag.T = off_host, raw.B, T2
+    jag.max_len = int(lens.max()) if raw.B else 0
+    jag.offsets, jag.timestamps = new_off, ts[:T2]
+    jag.struct = H.make_jagged(jag.offsets, jag.timestamps, jag.max_len)
+    return jag, kept[:T2], (x_out[:T2] if x_out is not None else None)

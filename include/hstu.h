@@ -331,6 +331,32 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
                              size_t ws_bytes, hstu_stream_t stream);
 
 /* --------------------------------------------------------------------------------------------
+ * Stochastic Length ("HSTU: The First Exploration of the Scaling Law", 7.1.5 Stochastic Length):
+ * a history of n tokens keeps L = min(n, floor(n^(alpha/2) + 1/2)) tokens, the L tokens with the
+ * smallest random keys (ties broken by position), in their original order; positions are
+ * renumbered 0..L-1 and timestamps travel with their tokens. The random keys are an input: one
+ * int64 per raw token (a uniformly random subset follows from i.i.d. uniform keys).
+ * -------------------------------------------------------------------------------------------- */
+
+/* new_offsets (device, [B+1]) = exclusive prefix of L_b over raw's sequences. L is evaluated in
+ * double precision. ws: >= 256 bytes (status word; a malformed raw offsets array is reported as
+ * HSTU_ERR_DEVICE by hstu_sync_status). The caller reads new_offsets[B] = T' to size the outputs
+ * of hstu_stochastic_length_select. */
+hstu_status_t hstu_stochastic_length_offsets(const hstu_jagged_t* raw, double alpha, int64_t* new_offsets,
+                                             void* ws, size_t ws_bytes, hstu_stream_t stream);
+
+/* Selects the kept tokens of every sequence: kept (device int64 [T']) receives their global raw
+ * indices in order, ts_out (nullable, [T']) their timestamps, and x_out (nullable, [T', D] of
+ * x_dtype) their rows of x ([T_raw, D]). new_offsets must come from
+ * hstu_stochastic_length_offsets with the same raw batch and alpha. Rows are copied as bytes
+ * (D * element size must be a multiple of 16). */
+hstu_status_t hstu_stochastic_length_select(const hstu_jagged_t* raw, const int64_t* keys,
+                                            const int64_t* new_offsets, const void* x,
+                                            hstu_dtype_t x_dtype, int32_t D, int64_t* kept,
+                                            void* x_out, int64_t* ts_out, void* ws, size_t ws_bytes,
+                                            hstu_stream_t stream);
+
+/* --------------------------------------------------------------------------------------------
  * M-FALCON candidate scoring ("HSTU: The First Exploration of the Scaling Law", 7.1.5 M-FALCON).
  *
  * A stack of L layers (all BF16 mode, one hstu_layer_weights_t each) scores m candidates per

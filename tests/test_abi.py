@@ -80,3 +80,23 @@ def test_host_validation_without_gpu(lib):
     r = L.hstu_attn_fwd(ctypes.byref(desc), ctypes.byref(jag), 4096, 4096, 4096, 4096, 4096, 4096, 4096, 1 << 20,
                         None)
     assert r == 2
+
+
+def test_layer_bwd_rejects_misaligned_gradients_on_host(lib):
+    """dW1 / dW2 are accumulated with 16-byte vector atomics: a pointer off that boundary is refused
+    (HSTU_ERR_UNSUPPORTED) before anything reaches the GPU."""
+    Hb._lib = None
+    L = Hb.lib()
+    D, T = 256, 300
+    jag = Hb.hstu_jagged_t(B=1, max_len=T, T=T, offsets=1 << 20, timestamps=2 << 20)
+    desc = Hb.make_layer_desc(D, 4, 1.0 / 512, 512, Hb.HSTU_BF16, Hb.HSTU_BF16, Hb.HSTU_BF16)
+    need = L.hstu_layer_bwd_workspace_size(ctypes.byref(desc), ctypes.byref(jag))
+    w = Hb.hstu_layer_weights_t(*[(i + 3) << 20 for i in range(8)])
+    saved = Hb.hstu_layer_saved_t(*[(i + 20) << 20 for i in range(6)])
+    good = [(i + 40) << 20 for i in range(8)]
+    bad = list(good)
+    bad[0] += 4                                    # dW1 4 bytes off a 16-byte boundary
+    r = L.hstu_layer_bwd(ctypes.byref(desc), ctypes.byref(jag), ctypes.byref(w), 60 << 20, None, ctypes.byref(saved),
+                         61 << 20, None, 62 << 20, None, ctypes.byref(Hb.hstu_layer_grads_t(*bad)), 63 << 20, need,
+                         None)
+    assert r == 2
