@@ -27,6 +27,7 @@
 
 #include "hstu_internal.h"
 #include "sm100_ptx.cuh"
+#include "tile_pairs.cuh"
 #include "time_bucket_dev.cuh"
 
 namespace hstu {
@@ -49,29 +50,25 @@ __device__ __forceinline__ int pos_index_b(long long r, int L) {
 // ----------------------------------------------------------------------------------------------
 // transposed bias and bucket tiles
 // ----------------------------------------------------------------------------------------------
+// One block per causal tile pair. Thread t writes 8 consecutive queries [8 (t % 16), +8) of key
+// rows t / 16 + 16 p, p = 0..7: 16-byte half-bias and 8-byte bucket stores.
 __global__ void __launch_bounds__(256)
 attn_bias_t_kernel(AttnBwdArgs A) {
   const AttnArgs& a = A.f;
-  const int item = blockIdx.x;
-  const int kt = blockIdx.y;
-  if (item >= *a.count) return;
-  const int b = a.items[2 * item];
-  const int qt = a.items[2 * item + 1];
-  if (kt > qt) return;
+  int b, qt, kt;
+  if (!decode_tile_pair(blockIdx.x, a.pair_base, a.B, &b, &qt, &kt)) return;
   const long long seq0 = a.offsets[b];
   const int n = static_cast<int>(a.offsets[b + 1] - seq0);
-  const long long pair = a.pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2 + kt;
-
-  __shared__ long long s_qts[128];
+  __shared__ long long s_kts[128];
+  __shared__ long long s_tau[kTauEntries];
   __shared__ float s_win[256];
   __shared__ float s_rt[128];
-  __shared__ long long s_tau[kTauEntries];
   const int tid = threadIdx.x;
   const int L = a.pos_max_len;
   const int nb = a.n_buckets;
   if (tid < 128) {
-    const int qi = qt * kQTile + tid;
-    s_qts[tid] = a.ts[seq0 + (qi < n ? qi : n - 1)];
+    const int kj = kt * kQTile + tid;
+    s_kts[tid] = a.ts[seq0 + (kj < n ? kj : n - 1)];
     if (tid < nb) s_rt[tid] = a.rab_time[tid];
   }
   {
@@ -79,37 +76,37 @@ attn_bias_t_kernel(AttnBwdArgs A) {
     if (tid < 255) s_win[tid] = a.rab_pos[pos_index_b(rel0 + tid, L)];
   }
   for (int e = tid; e < kTauEntries; e += 256) s_tau[e] = c_time_taus[e];
-  __syncthreads();
-
-  const int j = blockIdx.z * 32 + (tid >> 3);   // key row within the tile
-  const int cg = tid & 7;                        // queries [16 cg, 16 cg + 16)
-  const int kj = kt * kQTile + j;
-  const long long t_j = a.ts[seq0 + (kj < n ? kj : n - 1)];
-  uint16_t* dst = reinterpret_cast<uint16_t*>(A.bias_t) + (pair * kQTile + j) * kQTile + 16 * cg;
-  uint8_t* dstb = reinterpret_cast<uint8_t*>(A.bucket_t) + (pair * kQTile + j) * kQTile + 16 * cg;
-  uint32_t bw[4];
+  const int c0 = 8 * (tid & 15);
+  long long qts[8];
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    uint32_t w[4];
+  for (int e = 0; e < 8; ++e) {
+    const int qi = qt * kQTile + c0 + e;
+    qts[e] = a.ts[seq0 + (qi < n ? qi : n - 1)];
+  }
+  __syncthreads();
+  const long long tile0 = blockIdx.x * static_cast<long long>(kQTile * kQTile);
+  uint16_t* tile = reinterpret_cast<uint16_t*>(A.bias_t) + tile0;
+  uint8_t* btile = reinterpret_cast<uint8_t*>(A.bucket_t) + tile0;
+#pragma unroll 1
+  for (int pass = 0; pass < 8; ++pass) {
+    const int j = (tid >> 4) + 16 * pass;   // key row within the tile
+    const long long t_j = s_kts[j];
+    uint32_t w[4], bw[2] = {0u, 0u};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       float v2[2];
-      int k2[2];
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        const int col = 16 * cg + 8 * u + 2 * e + x;
-        k2[x] = time_bucket_dev(s_qts[col] - t_j, s_tau, nb);
-        v2[x] = 0.5f * (s_win[col - j + 127] + s_rt[k2[x]]);
+        const int col = c0 + 2 * e + x;     // query column
+        const int bkt = time_bucket_dev(qts[2 * e + x] - t_j, s_tau, nb);
+        v2[x] = 0.5f * (s_win[col - j + 127] + s_rt[bkt]);
+        bw[e >> 1] |= static_cast<uint32_t>(bkt) << (8 * (2 * (e & 1) + x));
       }
       w[e] = pack_f16x2(v2[0], v2[1]);
-      const int byte = 8 * u + 2 * e;       // position of k2[0] among the 16 buckets
-      if ((byte & 3) == 0) bw[byte >> 2] = 0;
-      bw[byte >> 2] |= (static_cast<uint32_t>(k2[0]) << (8 * (byte & 3))) |
-                       (static_cast<uint32_t>(k2[1]) << (8 * ((byte & 3) + 1)));
     }
-    reinterpret_cast<uint4*>(dst)[u] = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(tile + j * kQTile + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint2*>(btile + j * kQTile + c0) = make_uint2(bw[0], bw[1]);
   }
-  *reinterpret_cast<uint4*>(dstb) = make_uint4(bw[0], bw[1], bw[2], bw[3]);
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -151,9 +148,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const long long pbase = a.pair_base[b];
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lb::kBar);
-  // 0 kv_full | 1,2 qdo_full | 3,4 qdo_empty | 5,6 bb_full | 7,8 bb_empty | 9 s_full | 10 p_ready |
-  // 11 dq_full | 12 fin
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  // 0 kv_full | 1,2 qdo_full | 3,4 qdo_empty | 5,6 bb_full | 7,8 bb_empty | 9,10 s_full (query half
+  // a, b) | 11,12 p_ready (half a, b) | 13 dq_full | 14 fin
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
@@ -173,10 +170,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(BAR(5 + s), 1);
       mbar_init(BAR(7 + s), 1);
     }
-    mbar_init(BAR(9), 1);
-    mbar_init(BAR(10), kSiluThreadsB);
-    mbar_init(BAR(11), 1);
-    mbar_init(BAR(12), 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(BAR(9 + h), 1);
+      mbar_init(BAR(11 + h), kSiluThreadsB / 2);
+    }
+    mbar_init(BAR(13), 1);
+    mbar_init(BAR(14), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -198,7 +197,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tDA = tmem + 128, tDV = tmem + 256, tDK = tmem + 320, tDQ = tmem + 384;
+  // query half h: S^T_h at columns [128 h, 128 h + 64) (P^T_h packed over its first 32), dA^T_h at
+  // [128 h + 64, 128 h + 128); accumulators dV, dK and the dQ tile of one query tile
+  const uint32_t tDV = tmem + 256, tDK = tmem + 320, tDQ = tmem + 384;
 
   const uint32_t sK = smem_u32(smem + Lb::kK), sV = smem_u32(smem + Lb::kV);
   const uint32_t sQ0 = smem_u32(smem + Lb::kQ0);
@@ -229,45 +230,65 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
   } else if (warp == kSiluWarpsB + 1) {
     // ---------------- tcgen05 issuer ----------------
+    // Per query tile s, in two halves of 64 queries: S^T_h = K Q_h^T and dA^T_h = V dO_h^T, then,
+    // once the elementwise warps of half h have written P^T_h (TMEM) and dX^T_h (shared memory),
+    // dV += P^T_h dO_h and dK += dX^T_h Q_h; after half b also dQ_tile = dX K. The next tile's half a
+    // is issued between the two halves, so each half's elementwise work overlaps MMAs.
     if (lane == 0) {
-      constexpr uint32_t id_ss = make_idesc_f16kind(128, 128, 0, 0, F16);
+      constexpr uint32_t id_s = make_idesc_f16kind(128, 64, 0, 0, F16);
       constexpr uint32_t id_kmn = make_idesc_f16kind(128, 64, 0, 1, F16);
       constexpr uint32_t id_mnmn = make_idesc_f16kind(128, 64, 1, 1, F16);
       bool ok = mbar_wait(BAR(0), 0, abort_flag, ctl);
+      auto issue_s = [&](int s, int h) -> bool {
+        const int st = s & 1;
+        if (h == 0 && !mbar_wait(BAR(1 + st), (s >> 1) & 1, abort_flag, ctl)) return false;
+        tc_fence_after();
+        const uint32_t sQ = sQ0 + st * 32768 + 8192 * h, sDO = sQ0 + st * 32768 + 16384 + 8192 * h;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_f16_ss(tmem + 128 * h, make_sdesc_sw128(sK + kk * 32, 16, 1024),
+                      make_sdesc_sw128(sQ + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_f16_ss(tmem + 128 * h + 64, make_sdesc_sw128(sV + kk * 32, 16, 1024),
+                      make_sdesc_sw128(sDO + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+        umma_commit(BAR(9 + h));
+        return true;
+      };
+      auto issue_grad = [&](int s, int h) -> bool {
+        if (!mbar_wait(BAR(11 + h), s & 1, abort_flag, ctl)) return false;
+        tc_fence_after();
+        const int st = s & 1;
+        const uint32_t sQ = sQ0 + st * 32768, sDO = sQ + 16384, sDX = sBT0 + st * 32768;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4)   // dV += P^T_h dO_h
+          umma_f16_ts(tDV, tmem + 128 * h + 8 * k4, make_sdesc_sw128(sDO + (4 * h + k4) * 2048, 16384, 1024),
+                      id_kmn, (s > 0 || h > 0 || k4 > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4)   // dK += dX^T_h Q_h
+          umma_f16_ss(tDK, make_sdesc_sw128(sDX + h * 16384 + k4 * 32, 16, 1024),
+                      make_sdesc_sw128(sQ + (4 * h + k4) * 2048, 16384, 1024), id_kmn,
+                      (s > 0 || h > 0 || k4 > 0) ? 1u : 0u);
+        return true;
+      };
+      if (ok && nsteps > 0) ok = issue_s(0, 0) && issue_s(0, 1);
       for (int s = 0; ok && s < nsteps; ++s) {
         const int st = s & 1;
-        if (!mbar_wait(BAR(1 + st), (s >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sQ = sQ0 + st * 32768, sDO = sQ + 16384;
+        if (!issue_grad(s, 0) || (s + 1 < nsteps && !issue_s(s + 1, 0)) || !issue_grad(s, 1)) {
+          ok = false;
+          break;
+        }
         const uint32_t sDX = sBT0 + st * 32768;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_f16_ss(tS, make_sdesc_sw128(sK + kk * 32, 16, 1024), make_sdesc_sw128(sQ + kk * 32, 16, 1024), id_ss,
-                      kk > 0 ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_f16_ss(tDA, make_sdesc_sw128(sV + kk * 32, 16, 1024), make_sdesc_sw128(sDO + kk * 32, 16, 1024),
-                      id_ss, kk > 0 ? 1u : 0u);
-        umma_commit(BAR(9));
-        if (!mbar_wait(BAR(10), s & 1, abort_flag, ctl)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)   // dV += P^T dO
-          umma_f16_ts(tDV, tS + 64 * (kk >> 2) + 8 * (kk & 3), make_sdesc_sw128(sDO + kk * 2048, 16384, 1024),
-                      id_kmn, (s > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)   // dK += dX^T Q
-          umma_f16_ss(tDK, make_sdesc_sw128(sDX + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                      make_sdesc_sw128(sQ + kk * 2048, 16384, 1024), id_kmn, (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)   // dQ_tile = dX K
           umma_f16_ss(tDQ, make_sdesc_sw128(sDX + kk * 2048, 16384, 1024),
                       make_sdesc_sw128(sK + kk * 2048, 16384, 1024), id_mnmn, kk > 0 ? 1u : 0u);
-        umma_commit(BAR(11));
+        umma_commit(BAR(13));
         umma_commit(BAR(3 + st));
         umma_commit(BAR(7 + st));
+        if (s + 1 < nsteps && !issue_s(s + 1, 1)) { ok = false; break; }
       }
-      if (ok) umma_commit(BAR(12));
+      if (ok) umma_commit(BAR(14));
     }
   } else {
     // ---------------- elementwise warps ----------------
@@ -277,32 +298,39 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const bool key_ok = kt * kQTile + rj < n;
     const float inv_N = a.inv_N;
+    // d rab_time: each thread sums runs of equal bucket along its key row; a closed run is added to
+    // the lane's own copy of the histogram (lanes of a warp never collide)
     int cur_b = -1;
     uint32_t cur_rep = 0xFFFFFFFFu;
     float acc_t = 0.0f;
     bool ok = true;
     auto flush_dq = [&](int s_prev) {
-      // dQ tile of query tile kt + s_prev: TMEM lane = query row, columns [32 hq, 32 hq + 32)
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tDQ + lane_base + 32 * hq, v);
-      tmem_ld_wait();
+      // (half-b warps) dQ tile of query tile kt + s_prev: TMEM lane = query row, all 64 columns
       const int qi = (kt + s_prev) * kQTile + quad * 32 + lane;
-      if (qi < n) {
-        float4* dst = reinterpret_cast<float4*>(A.dq + (seq0 + qi) * A.ld_g + h * kD + 32 * hq);
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tDQ + lane_base + 32 * c, v);
+        tmem_ld_wait();
+        if (qi < n) {
+          float4* dst = reinterpret_cast<float4*>(A.dq + (seq0 + qi) * A.ld_g + h * kD + 32 * c);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          atomicAdd(dst + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                         __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+          for (int q = 0; q < 8; ++q)
+            atomicAdd(dst + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                           __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+        }
       }
     };
     for (int s = 0; ok && s < nsteps; ++s) {
       const int qt = kt + s, st = s & 1;
-      if (!mbar_wait(BAR(5 + st), (s >> 1) & 1, abort_flag, ctl) || !mbar_wait(BAR(9), s & 1, abort_flag, ctl)) {
+      if (!mbar_wait(BAR(5 + st), (s >> 1) & 1, abort_flag, ctl) ||
+          !mbar_wait(BAR(9 + hq), s & 1, abort_flag, ctl)) {
         ok = false;
         break;
       }
-      if (s >= 1) {
-        if (!mbar_wait(BAR(11), (s - 1) & 1, abort_flag, ctl)) { ok = false; break; }
+      // half b starts after the MMAs of the previous tile's dQ: flushing it here costs no wait
+      if (hq == 1 && s >= 1) {
+        if (!mbar_wait(BAR(13), (s - 1) & 1, abort_flag, ctl)) { ok = false; break; }
         tc_fence_after();
         flush_dq(s - 1);
       }
@@ -318,8 +346,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       for (int hc = 0; hc < 2; ++hc) {
         const int c0 = 64 * hq + 32 * hc;   // first query column of the chunk
         uint32_t sv[32], dav[32];
-        tmem_ld_32x32b_x32(tS + lane_base + c0, sv);
-        tmem_ld_32x32b_x32(tDA + lane_base + c0, dav);
+        tmem_ld_32x32b_x32(tmem + lane_base + 128 * hq + 32 * hc, sv);
+        tmem_ld_32x32b_x32(tmem + lane_base + 128 * hq + 64 + 32 * hc, dav);
         uint32_t hb[16], bk[8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -379,7 +407,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             xf[2 * e2 + 1] = dv2[1];
           }
         }
-        tmem_st_32x32b_x16(tS + lane_base + 64 * hq + 16 * hc, pp);
+        tmem_st_32x32b_x16(tmem + lane_base + 128 * hq + 16 * hc, pp);
         // dX^T replaces the half-bias just read: same row, same swizzled 16-byte units
 #pragma unroll
         for (int q = 0; q < 4; ++q)
@@ -416,27 +444,26 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             for (int x = 0; x < 4; ++x) {
               const int bkt = static_cast<int>((wd >> (8 * x)) & 0xFFu);
               if (bkt != cur_b) {
-                // each lane owns a copy of the histogram: lanes of a warp never collide
                 if (acc_t != 0.0f) atomicAdd(s_dtime + cur_b * 32 + lane, acc_t);
                 acc_t = 0.0f;
                 cur_b = bkt;
-                cur_rep = 0x01010101u * static_cast<uint32_t>(bkt);
               }
               acc_t += xf[4 * wq + x];
             }
+            cur_rep = 0x01010101u * static_cast<uint32_t>(cur_b);
           }
         }
       }
       tmem_st_wait();
       tc_fence_before();
       fence_proxy_async_smem();
-      mbar_arrive(BAR(10));    // P^T in TMEM, dX^T in shared memory
+      mbar_arrive(BAR(11 + hq));    // P^T_h in TMEM, dX^T_h in shared memory
     }
-    if (ok && nsteps > 0 && mbar_wait(BAR(11), (nsteps - 1) & 1, abort_flag, ctl)) {
+    if (ok && hq == 1 && nsteps > 0 && mbar_wait(BAR(13), (nsteps - 1) & 1, abort_flag, ctl)) {
       tc_fence_after();
       flush_dq(nsteps - 1);
     }
-    if (ok && mbar_wait(BAR(12), 0, abort_flag, ctl)) {
+    if (ok && mbar_wait(BAR(14), 0, abort_flag, ctl)) {
       tc_fence_after();
       uint32_t vk[32], vv[32];
       tmem_ld_32x32b_x32(tDK + lane_base + 32 * hq, vk);
@@ -483,7 +510,7 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  attn_bias_t_kernel<<<dim3(static_cast<unsigned>(a.capacity), static_cast<unsigned>(mt), 4), 256, 0, st>>>(A);
+  attn_bias_t_kernel<<<static_cast<unsigned>(a.max_pairs), 256, 0, st>>>(A);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv, tdo, tbt, tbk;

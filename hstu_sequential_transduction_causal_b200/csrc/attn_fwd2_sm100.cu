@@ -29,6 +29,7 @@
 
 #include "hstu_internal.h"
 #include "sm100_ptx.cuh"
+#include "tile_pairs.cuh"
 #include "time_bucket_dev.cuh"
 
 namespace hstu {
@@ -50,28 +51,24 @@ __device__ __forceinline__ int pos_index2(long long r, int L) {
 // ----------------------------------------------------------------------------------------------
 // 1. bias tiles
 // ----------------------------------------------------------------------------------------------
+// One block per causal tile pair (blocks past the batch's last pair exit at once). Thread t writes
+// 8 consecutive keys [8 (t % 16), +8) of rows t / 16 + 16 p, p = 0..7: 16-byte coalesced stores.
 __global__ void __launch_bounds__(256)
 attn_bias_kernel(AttnArgs a) {
-  const int item = blockIdx.x;
-  const int kt = blockIdx.y;
-  if (item >= *a.count) return;
-  const int b = a.items[2 * item];
-  const int qt = a.items[2 * item + 1];
-  if (kt > qt) return;
+  int b, qt, kt;
+  if (!decode_tile_pair(blockIdx.x, a.pair_base, a.B, &b, &qt, &kt)) return;
   const long long seq0 = a.offsets[b];
   const int n = static_cast<int>(a.offsets[b + 1] - seq0);
-  const long long pair = a.pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2 + kt;
-
-  __shared__ long long s_kts[128];
+  __shared__ long long s_qts[128];
+  __shared__ long long s_tau[kTauEntries];
   __shared__ float s_win[256];
   __shared__ float s_rt[128];
-  __shared__ long long s_tau[kTauEntries];
   const int tid = threadIdx.x;
   const int L = a.pos_max_len;
   const int nb = a.n_buckets;
   if (tid < 128) {
-    const int kj = kt * kQTile + tid;
-    s_kts[tid] = kj < n ? a.ts[seq0 + kj] : 0;
+    const int qi = qt * kQTile + tid;
+    s_qts[tid] = a.ts[seq0 + (qi < n ? qi : n - 1)];
     if (tid < nb) s_rt[tid] = a.rab_time[tid];
   }
   {
@@ -79,28 +76,32 @@ attn_bias_kernel(AttnArgs a) {
     if (tid < 255) s_win[tid] = a.rab_pos[pos_index2(rel0 + tid, L)];
   }
   for (int e = tid; e < kTauEntries; e += 256) s_tau[e] = c_time_taus[e];
-  __syncthreads();
-
-  const int r = blockIdx.z * 32 + (tid >> 3);   // query row within the tile (32 rows per block)
-  const int cg = tid & 7;                        // 16 keys [16 cg, 16 cg + 16)
-  const int qi = qt * kQTile + r;
-  const long long t_i = a.ts[seq0 + (qi < n ? qi : n - 1)];
-  uint16_t* dst = reinterpret_cast<uint16_t*>(a.bias) + (pair * kQTile + r) * kQTile + 16 * cg;
+  const int c0 = 8 * (tid & 15);
+  long long kts[8];
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
+  for (int e = 0; e < 8; ++e) {
+    const int kj = kt * kQTile + c0 + e;
+    kts[e] = a.ts[seq0 + (kj < n ? kj : n - 1)];
+  }
+  __syncthreads();
+  uint16_t* tile = reinterpret_cast<uint16_t*>(a.bias) + blockIdx.x * static_cast<long long>(kQTile * kQTile);
+#pragma unroll 1
+  for (int pass = 0; pass < 8; ++pass) {
+    const int r = (tid >> 4) + 16 * pass;   // query row within the tile
+    const long long t_i = s_qts[r];
     uint32_t w[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       float v2[2];
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
-        const int col = 16 * cg + 8 * u + 2 * e + x;
-        const int bkt = time_bucket_dev(t_i - s_kts[col], s_tau, nb);
+        const int col = c0 + 2 * e + x;
+        const int bkt = time_bucket_dev(t_i - kts[2 * e + x], s_tau, nb);
         v2[x] = 0.5f * (s_win[r - col + 127] + s_rt[bkt]);
       }
       w[e] = pack_f16x2(v2[0], v2[1]);
     }
-    reinterpret_cast<uint4*>(dst)[u] = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(tile + r * kQTile + c0) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -482,7 +483,7 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  attn_bias_kernel<<<dim3(static_cast<unsigned>(a.capacity), static_cast<unsigned>(mt), 4), 256, 0, st>>>(a);
+  attn_bias_kernel<<<static_cast<unsigned>(a.max_pairs), 256, 0, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv, tb;

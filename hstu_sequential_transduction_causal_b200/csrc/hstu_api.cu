@@ -151,9 +151,8 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
   A.bias_t = w + lay.bias_t; A.bucket_t = w + lay.bucket_t;
   A.kitems = reinterpret_cast<int32_t*>(w + lay.kitems); A.kcount = kcount;
   e = launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, a.status, st,
-                      reinterpret_cast<long long*>(w + lay.f.pairs));
-  if (e == cudaSuccess)
-    e = launch_bwd_worklist(jag->offsets, jag->B, count, reinterpret_cast<int32_t*>(w + lay.kitems), kcount, st);
+                      reinterpret_cast<long long*>(w + lay.f.pairs), reinterpret_cast<int32_t*>(w + lay.kitems),
+                      kcount);
   if (e == cudaSuccess) e = attn_bwd_tc(A, st);
   return cuda_status(e);
 }

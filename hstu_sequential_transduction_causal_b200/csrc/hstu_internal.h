@@ -70,8 +70,11 @@ cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
 // ---------------------------------------------------------------------------------------------
 // Builds the (sequence, query tile) work list; with pair_base (device, [B+1]) also the index of
 // each sequence's first causal (query tile, key tile) pair and, in pair_base[B], their total.
+// With kitems, also the attention backward's (sequence, key tile) list in the same cost order: the
+// key tile that visits t + 1 query tiles sits where the forward list has query tile t.
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
-                            int32_t* count, int* status, cudaStream_t st, long long* pair_base = nullptr);
+                            int32_t* count, int* status, cudaStream_t st, long long* pair_base = nullptr,
+                            int32_t* kitems = nullptr, int32_t* kcount = nullptr);
 cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T,
                                 int n_buckets, const int64_t* sq_offsets, uint8_t* out,
                                 cudaStream_t st);
@@ -127,8 +130,6 @@ struct AttnBwdArgs {
   const int32_t* kcount;
 };
 
-cudaError_t launch_bwd_worklist(const int64_t* offsets, int B, const int32_t* fwd_count, int32_t* items,
-                                int32_t* count, cudaStream_t st);
 cudaError_t attn_bwd_tc(const AttnBwdArgs& a, cudaStream_t st);
 
 // Bound on the number of causal (query tile, key tile) pairs of a batch.

@@ -23,7 +23,7 @@ namespace {
 // ----------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
 worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items,
-                int32_t* count, int* status, long long* pair_base) {
+                int32_t* count, int* status, long long* pair_base, int32_t* kitems, int32_t* kcount) {
   __shared__ int s_warp[32];
   __shared__ int s_max_tiles;
   __shared__ int s_bad;
@@ -44,6 +44,7 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
   if (s_bad) {
     if (tid == 0) {
       *count = 0;
+      if (kcount) *kcount = 0;
       report_error(status, kDevBadInput);
       if (pair_base) pair_base[B > 0 ? B : 0] = 0;
     }
@@ -87,6 +88,10 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
           const int p = pos + __popc(m & ((1u << lane) - 1u));
           items[2 * p] = b;
           items[2 * p + 1] = t;
+          if (kitems) {   // the key tile that visits t + 1 query tiles: the same cost order
+            kitems[2 * p] = b;
+            kitems[2 * p + 1] = s_nt[b] - 1 - t;
+          }
         }
         pos += __popc(m);
       }
@@ -115,13 +120,20 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
       if (flag) {
         items[2 * pos] = b;
         items[2 * pos + 1] = t;
+        if (kitems) {
+          kitems[2 * pos] = b;
+          kitems[2 * pos + 1] = static_cast<int>((off[b + 1] - off[b] + kQTile - 1) / kQTile) - 1 - t;
+        }
       }
       __syncthreads();
       if (tid == blockDim.x - 1) s_base = pos + (flag ? 1 : 0);
       __syncthreads();
     }
   }
-  if (tid == 0) *count = s_base;
+  if (tid == 0) {
+    *count = s_base;
+    if (kcount) *kcount = s_base;
+  }
   if (!pair_base) return;
   // pair_base[b] = sum_{b' < b} nt_b' (nt_b' + 1) / 2: index of sequence b's first causal
   // (query tile, key tile) pair; pair_base[B] is the total.
@@ -162,63 +174,6 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
     __syncthreads();
   }
   if (tid == 0) pair_base[B] = s_run;
-}
-
-// Key-tile work list of the attention backward: every (sequence b, key tile t) pair ordered by the
-// number of query tiles it visits (nt_b - t, largest first), ties by increasing b. Runs after
-// worklist_kernel (which validated the offsets); an empty forward list gives an empty list here.
-__global__ void __launch_bounds__(1024)
-bwd_worklist_kernel(const int64_t* __restrict__ off, int B, const int32_t* fwd_count, int32_t* items,
-                    int32_t* count) {
-  __shared__ int s_max;
-  __shared__ int s_base;
-  __shared__ int s_warp[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) {
-    s_max = 0;
-    s_base = 0;
-  }
-  __syncthreads();
-  if (*fwd_count == 0) {
-    if (tid == 0) *count = 0;
-    return;
-  }
-  for (int b = tid; b < B; b += blockDim.x)
-    atomicMax(&s_max, static_cast<int>((off[b + 1] - off[b] + kQTile - 1) / kQTile));
-  __syncthreads();
-  const int max_tiles = s_max;
-  // classes c = max_tiles .. 1; class c holds (b, nt_b - c) for every b with nt_b >= c
-  for (int c = max_tiles; c >= 1; --c) {
-    for (int c0 = 0; c0 < B; c0 += blockDim.x) {
-      const int b = c0 + tid;
-      int nt = 0;
-      if (b < B) nt = static_cast<int>((off[b + 1] - off[b] + kQTile - 1) / kQTile);
-      const bool flag = b < B && nt >= c;
-      const unsigned m = __ballot_sync(0xffffffffu, flag);
-      if (lane == 0) s_warp[warp] = __popc(m);
-      __syncthreads();
-      if (warp == 0) {
-        const int v = s_warp[lane];
-        int inc = v;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, inc, d);
-          if (lane >= d) inc += y;
-        }
-        s_warp[lane] = inc - v;
-      }
-      __syncthreads();
-      const int pos = s_base + s_warp[warp] + __popc(m & ((1u << lane) - 1u));
-      if (flag) {
-        items[2 * pos] = b;
-        items[2 * pos + 1] = nt - c;
-      }
-      __syncthreads();
-      if (tid == blockDim.x - 1) s_base = pos + (flag ? 1 : 0);
-      __syncthreads();
-    }
-  }
-  if (tid == 0) *count = s_base;
 }
 
 // One warp per query row: writes bucket(t_i - t_j) for every key j of the row's sequence.
@@ -324,14 +279,9 @@ cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int
 }  // namespace
 
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
-                            int32_t* count, int* status, cudaStream_t st, long long* pair_base) {
-  worklist_kernel<<<1, 1024, 0, st>>>(offsets, B, T, max_len, items, count, status, pair_base);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_bwd_worklist(const int64_t* offsets, int B, const int32_t* fwd_count, int32_t* items,
-                                int32_t* count, cudaStream_t st) {
-  bwd_worklist_kernel<<<1, 1024, 0, st>>>(offsets, B, fwd_count, items, count);
+                            int32_t* count, int* status, cudaStream_t st, long long* pair_base, int32_t* kitems,
+                            int32_t* kcount) {
+  worklist_kernel<<<1, 1024, 0, st>>>(offsets, B, T, max_len, items, count, status, pair_base, kitems, kcount);
   return cudaGetLastError();
 }
 

@@ -152,13 +152,30 @@ convert_kernel(const void* __restrict__ in, void* __restrict__ out, int64_t n) {
   }
 }
 
+// Sums `parts` partial rows: block of 256 threads = 32 columns x 8 interleaved slices of the rows,
+// then a shared-memory sum of the slices (the loads are independent and coalesced per warp).
 __global__ void __launch_bounds__(256)
 colsum_final_kernel(const float* __restrict__ partial, int parts, int cols, float* __restrict__ out) {
-  const int c = blockIdx.x * 256 + threadIdx.x;
-  if (c >= cols) return;
-  float s = 0.0f;
-  for (int p = 0; p < parts; ++p) s += partial[static_cast<int64_t>(p) * cols + c];
-  out[c] = s;
+  __shared__ float s_part[8][33];
+  const int cl = threadIdx.x & 31, slice = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + cl;
+  float s0 = 0.0f, s1 = 0.0f;
+  if (c < cols) {
+    int p = slice;
+    for (; p + 8 < parts; p += 16) {
+      s0 += partial[static_cast<int64_t>(p) * cols + c];
+      s1 += partial[static_cast<int64_t>(p + 8) * cols + c];
+    }
+    if (p < parts) s0 += partial[static_cast<int64_t>(p) * cols + c];
+  }
+  s_part[slice][cl] = s0 + s1;
+  __syncthreads();
+  if (slice == 0 && c < cols) {
+    float t = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += s_part[k][cl];
+    out[c] = t;
+  }
 }
 
 }  // namespace
@@ -191,7 +208,7 @@ cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const f
 #undef HSTU_NGB
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  colsum_final_kernel<<<(2 * D + 255) / 256, 256, 0, st>>>(partial, G, 2 * D, dgamma_dbeta_out);
+  colsum_final_kernel<<<(2 * D + 31) / 32, 256, 0, st>>>(partial, G, 2 * D, dgamma_dbeta_out);
   return cudaGetLastError();
 }
 
@@ -237,7 +254,7 @@ cudaError_t column_sum(const void* in, int dt, int64_t rows, int cols, int64_t l
   else colsum_partial_kernel<kDtF16><<<grid, 256, 0, st>>>(in, rows, cols, ld, rows_per, partial);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  colsum_final_kernel<<<(cols + 255) / 256, 256, 0, st>>>(partial, parts, cols, out);
+  colsum_final_kernel<<<(cols + 31) / 32, 256, 0, st>>>(partial, parts, cols, out);
   return cudaGetLastError();
 }
 
