@@ -38,8 +38,6 @@ constexpr int kD = 64;
 constexpr int kSiluWarpsB = 8;
 constexpr int kThreadsB = 32 * (kSiluWarpsB + 2);
 constexpr int kSiluThreadsB = 32 * kSiluWarpsB;
-constexpr uint32_t kHalf2HalfB = 0x38003800u;       // (0.5, 0.5) in fp16
-constexpr uint32_t kHalf2MinusHalfB = 0xB800B800u;  // (-0.5, -0.5)
 
 __device__ __forceinline__ int pos_index_b(long long r, int L) {
   r = r > L - 1 ? L - 1 : r;
@@ -360,9 +358,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           bk[4 * q] = w.x; bk[4 * q + 1] = w.y; bk[4 * q + 2] = w.z; bk[4 * q + 3] = w.w;
         }
         tmem_ld_wait();
-        // F16: packed fp16 per pair of queries: h = x/2, t = tanh(h), sigma(x) = (1 + t)/2,
-        // P = SiLU(x) = h (1 + t), SiLU'(x) = sigma + P (1 - sigma), dX = dA inv_N SiLU'(x).
-        // BF16 operands (8x coarser P and dX for the MMAs): the same in fp32, rounded once.
+        // per query, in fp32: x = s + bias, sigma(x) = (1 + tanh(x/2)) / 2, P = SiLU(x) = x sigma,
+        // dX = dA inv_N SiLU'(x) with SiLU' = sigma + P (1 - sigma); P and dX are rounded once to the
+        // MMA operand type. (A packed-fp16 evaluation of SiLU' quantises 1 - sigma near x = 8 and
+        // biases the table-gradient sums.)
         uint32_t pp[16], dxp[16];
         float xf[32];
 #pragma unroll
@@ -373,39 +372,26 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             m = ((col >= lo_col && col < hi_col) ? 0x0000FFFFu : 0u) |
                 ((col + 1 >= lo_col && col + 1 < hi_col) ? 0xFFFF0000u : 0u);
           }
-          if constexpr (F16) {
-            const uint32_t s2 = pack_f16x2(__uint_as_float(sv[2 * e2]), __uint_as_float(sv[2 * e2 + 1]));
-            const uint32_t h2 = hfma2_u32(s2, kHalf2HalfB, hb[e2]);
-            const uint32_t t2 = tanh_f16x2(h2);
-            const uint32_t p2 = hfma2_u32(h2, t2, h2);
-            const uint32_t sg = hfma2_u32(t2, kHalf2HalfB, kHalf2HalfB);        // sigma
-            const uint32_t osg = hfma2_u32(t2, kHalf2MinusHalfB, kHalf2HalfB);  // 1 - sigma
-            const uint32_t g2 = hfma2_u32(p2, osg, sg);                          // SiLU'(x)
-            const uint32_t da2 =
-                pack_f16x2(__uint_as_float(dav[2 * e2]) * inv_N, __uint_as_float(dav[2 * e2 + 1]) * inv_N);
-            const uint32_t x2 = hmul2_u32(da2, g2) & m;
-            const float2 xv = unpack_f16x2(x2);
-            xf[2 * e2] = xv.x;
-            xf[2 * e2 + 1] = xv.y;
-            pp[e2] = p2 & m;
-            dxp[e2] = x2;
-          } else {
-            const float2 hbf = unpack_f16x2(hb[e2]);
-            float pv[2], dv2[2];
+          const float2 hbf = unpack_f16x2(hb[e2]);
+          float pv[2], dv2[2];
 #pragma unroll
-            for (int x = 0; x < 2; ++x) {
-              const float xs = __uint_as_float(sv[2 * e2 + x]) + 2.0f * (x ? hbf.y : hbf.x);
-              const float sg = fmaf(0.5f, tanh_f32_approx(0.5f * xs), 0.5f);
-              const float av = xs * sg;
-              const bool keep = (m >> (16 * x)) & 1u;
-              pv[x] = keep ? av : 0.0f;
-              dv2[x] = keep ? __uint_as_float(dav[2 * e2 + x]) * inv_N * fmaf(av, 1.0f - sg, sg) : 0.0f;
-            }
+          for (int x = 0; x < 2; ++x) {
+            const float xs = __uint_as_float(sv[2 * e2 + x]) + 2.0f * (x ? hbf.y : hbf.x);
+            const float sg = fmaf(0.5f, tanh_f32_approx(0.5f * xs), 0.5f);
+            const float av = xs * sg;
+            const bool keep = (m >> (16 * x)) & 1u;
+            pv[x] = keep ? av : 0.0f;
+            dv2[x] = keep ? __uint_as_float(dav[2 * e2 + x]) * inv_N * fmaf(av, 1.0f - sg, sg) : 0.0f;
+          }
+          if (F16) {
+            pp[e2] = pack_f16x2(pv[0], pv[1]);
+            dxp[e2] = pack_f16x2(dv2[0], dv2[1]);
+          } else {   // the MMAs take A and B of one type: P and dX as bf16 next to bf16 dO, Q, K
             pp[e2] = pack_bf16x2(pv[0], pv[1]);
             dxp[e2] = pack_bf16x2(dv2[0], dv2[1]);
-            xf[2 * e2] = dv2[0];
-            xf[2 * e2 + 1] = dv2[1];
           }
+          xf[2 * e2] = dv2[0];     // the table gradients sum dX in fp32
+          xf[2 * e2 + 1] = dv2[1];
         }
         tmem_st_32x32b_x16(tmem + lane_base + 128 * hq + 16 * hc, pp);
         // dX^T replaces the half-bias just read: same row, same swizzled 16-byte units

@@ -26,6 +26,7 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kThreads = 192;   // warps 0-3 epilogue, warp 4 TMA, warp 5 MMA
+constexpr int kBoxBytes = 4096; // one epilogue staging box: 32 rows x 128 bytes
 
 template <int BN, int STAGES>
 struct GemmSmem {
@@ -33,31 +34,18 @@ struct GemmSmem {
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTileBytes = STAGES * kStageBytes;
-  static constexpr int kBarOff = kTileBytes;
-  static constexpr int kTotal = kTileBytes + 256 + 1024;   // barriers + alignment slack
+  static constexpr int kOut = kTileBytes;            // 4 warps x 2 staging boxes
+  static constexpr int kBarOff = kOut + 4 * 2 * kBoxBytes;
+  static constexpr int kTotal = kBarOff + 256 + 1024;   // barriers + alignment slack
 };
 
 __host__ __device__ __forceinline__ int dt_size(int dt) { return dt == kDtF32 ? 4 : 2; }
 
-// 32 consecutive values of one row, stored as fp32, bf16 or fp16 (16-byte vector stores).
-__device__ __forceinline__ void store_row32(void* out, int dt, const float* v) {
-  if (dt == kDtF32) {
-    float4* o = reinterpret_cast<float4*>(out);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-  } else {
-    uint4* o = reinterpret_cast<uint4*>(out);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        w[e] = dt == kDtBF16 ? pack_bf16x2(v[8 * q + 2 * e], v[8 * q + 2 * e + 1])
-                             : pack_f16x2(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]);
-      o[q] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  }
-}
+struct GemmParams {
+  int M, N, num_kb, kb_per, tiles_n, splits, total;
+  uint32_t idesc;
+  GemmEpilogue epi;
+};
 
 __device__ __forceinline__ void load_row32(const void* in, int dt, float* v) {
   if (dt == kDtF32) {
@@ -95,28 +83,80 @@ __device__ __forceinline__ float load_one(const void* base, int dt, int64_t idx)
   return __half2float(reinterpret_cast<const __half*>(base)[idx]);
 }
 
+// Per-warp epilogue staging: boxes of 32 rows x 128 bytes in the 128-byte swizzled layout of the
+// output tensor maps, written row-per-lane (16-byte units XOR-ed with the row: conflict-free) and
+// sent by TMA (store or fp32 reduce-add), two boxes in flight per warp.
+struct EpiStage {
+  uint8_t* base;   // this warp's 2 boxes
+  int slot;
+  __device__ __forceinline__ void emit(const CUtensorMap* map, bool reduce, int x, int y, const uint32_t* w) {
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) bulk_wait_group_read<1>();   // the box written two emissions ago has been read
+    __syncwarp();
+    uint8_t* box = base + slot * kBoxBytes;
+    uint8_t* row = box + lane * 128;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      *reinterpret_cast<uint4*>(row + ((u ^ (lane & 7)) << 4)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if (reduce) tma_reduce_add_2d(map, smem_u32(box), x, y);
+      else tma_store_2d(map, smem_u32(box), x, y);
+      bulk_commit_group();
+    }
+    slot ^= 1;
+  }
+};
+
+// 64 values of one row -> the output's boxes: one 64-column box for 2-byte types, two 32-column
+// boxes for fp32.
+__device__ __forceinline__ void emit64(EpiStage& es, const CUtensorMap* map, int dt, bool reduce, int x, int y,
+                                       const float* v, int xlim) {
+  uint32_t w[32];
+  if (dt == kDtF32) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (x + 32 * h >= xlim) break;   // (warp-uniform) a box wholly past the last column
+#pragma unroll
+      for (int j = 0; j < 32; ++j) w[j] = __float_as_uint(v[32 * h + j]);
+      es.emit(map, reduce, x + 32 * h, y, w);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      w[j] = dt == kDtBF16 ? pack_bf16x2(v[2 * j], v[2 * j + 1]) : pack_f16x2(v[2 * j], v[2 * j + 1]);
+    es.emit(map, false, x, y, w);
+  }
+}
+
+// Persistent tensor-core GEMM: CTAs stride over (m tile, n tile, k split) work items; the
+// accumulator is double-buffered in TMEM so the epilogue of one tile overlaps the next tile's
+// mainloop.
 template <int BN, int STAGES, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    int M, int N, int num_kb, int kb_per_split, uint32_t idesc, GemmEpilogue epi, WaitCtl ctl) {
+                    const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
+                    GemmParams P, WaitCtl ctl) {
   using L = GemmSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  // bars[0..STAGES): full, [STAGES..2*STAGES): empty, [2*STAGES]: accumulator ready
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 1);
+  // [0, STAGES) full | [STAGES, 2 STAGES) empty | 2 STAGES + b: accumulator b full | + 2: empty
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto acc_full = [&](int b) { return smem_u32(&bars[2 * STAGES + b]); };
+  auto acc_empty = [&](int b) { return smem_u32(&bars[2 * STAGES + 2 + b]); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
-  const int m0 = blockIdx.y * kBM;
-  const int kb_begin = blockIdx.z * kb_per_split;
-  const int kb_end = min(num_kb, kb_begin + kb_per_split);
-  const int nkb = max(0, kb_end - kb_begin);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2 * STAGES + 1; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    for (int i = 0; i < 2 * STAGES; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(acc_full(b), 1);
+      mbar_init(acc_empty(b), 128);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -125,7 +165,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     tma_prefetch_desc(&tmB);
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), BN);
+    tmem_alloc(smem_u32(tmem_slot), 2 * BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -133,118 +173,155 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   tc_fence_after();
   const uint32_t tmem_acc = *tmem_slot;
 
+  auto decode = [&](int t, int& m0, int& n0, int& kb0, int& kb1) {
+    const int ks = t % P.splits;
+    const int rest = t / P.splits;
+    n0 = (rest % P.tiles_n) * BN;
+    m0 = (rest / P.tiles_n) * kBM;
+    kb0 = ks * P.kb_per;
+    kb1 = min(P.num_kb, kb0 + P.kb_per);
+  };
+
   if (warp == 4) {
     if (lane == 0) {
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % STAGES;
-        if (i >= STAGES && !mbar_wait(smem_u32(&bars[STAGES + s]), ((i / STAGES) - 1) & 1, abort_flag, ctl)) break;
-        const uint32_t full = smem_u32(&bars[s]);
-        const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
-        const uint32_t sb = sa + L::kABytes;
-        const int kx = (kb_begin + i) * kBK;
-        mbar_arrive_expect_tx(full, L::kStageBytes);
-        if (!A_MN) {
-          tma_load_2d(sa, &tmA, full, kx, m0);
-        } else {
-          tma_load_2d(sa, &tmA, full, m0, kx);
-          tma_load_2d(sa + 8192, &tmA, full, m0 + 64, kx);
-        }
-        if (!B_MN) {
-          tma_load_2d(sb, &tmB, full, kx, n0);
-        } else {
+      int g = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < P.total; t += gridDim.x) {
+        int m0, n0, kb0, kb1;
+        decode(t, m0, n0, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
+          const int s = g % STAGES;
+          if (g >= STAGES && !mbar_wait(smem_u32(&bars[STAGES + s]), ((g / STAGES) - 1) & 1, abort_flag, ctl)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = smem_u32(&bars[s]);
+          const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
+          const uint32_t sb = sa + L::kABytes;
+          const int kx = kb * kBK;
+          mbar_arrive_expect_tx(full, L::kStageBytes);
+          if (!A_MN) {
+            tma_load_2d(sa, &tmA, full, kx, m0);
+          } else {
+            tma_load_2d(sa, &tmA, full, m0, kx);
+            tma_load_2d(sa + 8192, &tmA, full, m0 + 64, kx);
+          }
+          if (!B_MN) {
+            tma_load_2d(sb, &tmB, full, kx, n0);
+          } else {
 #pragma unroll
-          for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * 8192, &tmB, full, n0 + 64 * c, kx);
+            for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * 8192, &tmB, full, n0 + 64 * c, kx);
+          }
         }
       }
     }
   } else if (warp == 5) {
     if (lane == 0) {
+      int g = 0, it = 0;
       bool ok = true;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % STAGES;
-        if (!mbar_wait(smem_u32(&bars[s]), (i / STAGES) & 1, abort_flag, ctl)) { ok = false; break; }
+      for (int t = blockIdx.x; ok && t < P.total; t += gridDim.x, ++it) {
+        int m0, n0, kb0, kb1;
+        decode(t, m0, n0, kb0, kb1);
+        const int buf = it & 1;
+        if (it >= 2 && !mbar_wait(acc_empty(buf), ((it >> 1) - 1) & 1, abort_flag, ctl)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
-        const uint32_t sb = sa + L::kABytes;
+        const uint32_t acc = tmem_acc + buf * BN;
+        for (int kb = kb0; kb < kb1; ++kb, ++g) {
+          const int s = g % STAGES;
+          if (!mbar_wait(smem_u32(&bars[s]), (g / STAGES) & 1, abort_flag, ctl)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
+          const uint32_t sb = sa + L::kABytes;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          const uint64_t ad = A_MN ? make_sdesc_sw128(sa + kk * 2048, 8192, 1024)
-                                   : make_sdesc_sw128(sa + kk * 32, 16, 1024);
-          const uint64_t bd = B_MN ? make_sdesc_sw128(sb + kk * 2048, 8192, 1024)
-                                   : make_sdesc_sw128(sb + kk * 32, 16, 1024);
-          umma_f16_ss(tmem_acc, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = A_MN ? make_sdesc_sw128(sa + kk * 2048, 8192, 1024)
+                                     : make_sdesc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? make_sdesc_sw128(sb + kk * 2048, 8192, 1024)
+                                     : make_sdesc_sw128(sb + kk * 32, 16, 1024);
+            umma_f16_ss(acc, ad, bd, P.idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&bars[STAGES + s]));
         }
-        umma_commit(smem_u32(&bars[STAGES + s]));
+        if (ok) umma_commit(acc_full(buf));
       }
-      if (ok) umma_commit(smem_u32(&bars[2 * STAGES]));
     }
   } else {
-    // epilogue warps 0-3: thread owns output row m0 + 32*warp + lane
-    bool have_acc = nkb > 0;
-    if (have_acc) have_acc = mbar_wait(smem_u32(&bars[2 * STAGES]), 0, abort_flag, ctl);
-    if (have_acc || nkb == 0) {
+    // epilogue warps 0-3: TMEM lanes 32 warp .. +31 = output rows m0 + 32 warp + lane
+    const GemmEpilogue& epi = P.epi;
+    EpiStage es{smem + L::kOut + warp * 2 * kBoxBytes, 0};
+    int it = 0;
+    for (int t = blockIdx.x; t < P.total; t += gridDim.x, ++it) {
+      int m0, n0, kb0, kb1;
+      decode(t, m0, n0, kb0, kb1);
+      const int buf = it & 1;
+      if (!mbar_wait(acc_full(buf), (it >> 1) & 1, abort_flag, ctl)) break;
       tc_fence_after();
       const int row = m0 + warp * 32 + lane;
-      const bool row_ok = row < M;
+      const bool row_ok = row < P.M;
+      const int ybox = m0 + warp * 32;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        if (nkb > 0) {
+      for (int c = 0; c < BN / 64; ++c) {
+        const int n = n0 + c * 64;
+        float v[64];
+        {
           uint32_t r[32];
-          tmem_ld_32x32b_x32(tmem_acc + (static_cast<uint32_t>(warp * 32) << 16) + c * 32, r);
-          tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        } else {
+          for (int h = 0; h < 2; ++h) {
+            tmem_ld_32x32b_x32(tmem_acc + buf * BN + (static_cast<uint32_t>(warp * 32) << 16) + c * 64 + 32 * h, r);
+            tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+            for (int j = 0; j < 32; ++j) v[32 * h + j] = __uint_as_float(r[j]);
+          }
         }
-        const int n = n0 + c * 32;
-        if (!row_ok || n >= N) continue;
+        if (c == BN / 64 - 1) {   // the whole accumulator is in registers: release it to the MMA
+          tc_fence_before();
+          mbar_arrive(acc_empty(buf));
+        }
+        if (n >= P.N) continue;
         if (epi.kind == kEpiAtomic) {
-          float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(epi.out0) +
-                                                static_cast<int64_t>(row) * epi.ld_out0 + n);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) atomicAdd(o + j, make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+          emit64(es, &tmO0, kDtF32, true, n, ybox, v, P.N);
           continue;
         }
         if (epi.bias) {
+          const float4* bp = reinterpret_cast<const float4*>(epi.bias + n);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] += __ldg(epi.bias + n + j);
+          for (int q = 0; q < 16; ++q) {
+            const float4 b4 = (n + 4 * q < P.N) ? __ldg(bp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * q] += b4.x; v[4 * q + 1] += b4.y; v[4 * q + 2] += b4.z; v[4 * q + 3] += b4.w;
+          }
         }
         if (epi.kind == kEpiSilu) {
-          if (epi.out1) {
-            uint8_t* o1 = reinterpret_cast<uint8_t*>(epi.out1) +
-                          (static_cast<int64_t>(row) * epi.ld_out1 + n) * dt_size(epi.out1_dt);
-            store_row32(o1, epi.out1_dt, v);
-          }
+          if (epi.out1) emit64(es, &tmO1, epi.out1_dt, false, n, ybox, v, P.N);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = silu_fast(v[j]);
+          for (int j = 0; j < 64; ++j) v[j] = silu_fast(v[j]);
         } else if (epi.resid) {
-          float rv[32];
-          const uint8_t* rp = reinterpret_cast<const uint8_t*>(epi.resid) +
-                              (static_cast<int64_t>(row) * epi.ld_resid + n) * dt_size(epi.resid_dt);
-          load_row32(rp, epi.resid_dt, rv);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] += rv[j];
+          for (int h = 0; h < 2; ++h) {
+            float rv[32];
+            if (row_ok && n + 32 * h < P.N) {
+              const uint8_t* rp = reinterpret_cast<const uint8_t*>(epi.resid) +
+                                  (static_cast<int64_t>(row) * epi.ld_resid + n + 32 * h) * dt_size(epi.resid_dt);
+              load_row32(rp, epi.resid_dt, rv);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) rv[j] = 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[32 * h + j] += rv[j];
+          }
         }
-        uint8_t* o0 = reinterpret_cast<uint8_t*>(epi.out0) +
-                      (static_cast<int64_t>(row) * epi.ld_out0 + n) * dt_size(epi.out0_dt);
-        store_row32(o0, epi.out0_dt, v);
-        if (epi.kind == kEpiLinear && epi.out1) {
-          uint8_t* o1 = reinterpret_cast<uint8_t*>(epi.out1) +
-                        (static_cast<int64_t>(row) * epi.ld_out1 + n) * dt_size(epi.out1_dt);
-          store_row32(o1, epi.out1_dt, v);
-        }
+        emit64(es, &tmO0, epi.out0_dt, false, n, ybox, v, P.N);
+        if (epi.kind == kEpiLinear && epi.out1) emit64(es, &tmO1, epi.out1_dt, false, n, ybox, v, P.N);
       }
     }
+    if (lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem_acc, BN);
+    tmem_dealloc(tmem_acc, 2 * BN);
   }
 }
 
@@ -310,10 +387,20 @@ gemm_f32_simt_kernel(const float* __restrict__ A, int64_t sam, int64_t sak, cons
   }
 }
 
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      n = 148;
+  }
+  return n;
+}
+
 template <int BN, int STAGES, bool A_MN, bool B_MN>
 cudaError_t launch_tc(const GemmArgs& g, cudaStream_t st) {
   using L = GemmSmem<BN, STAGES>;
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmO0, tmO1;
   // A: K-major -> [M rows, K] box {64, 128}; MN-major -> [K rows, M] box {64, 64}
   if (!A_MN) {
     if (!encode_tmap_2d_bf16(&tmA, g.A, g.K, g.M, g.lda, 64, kBM, g.f16)) return cudaErrorInvalidValue;
@@ -325,18 +412,33 @@ cudaError_t launch_tc(const GemmArgs& g, cudaStream_t st) {
   } else {
     if (!encode_tmap_2d_bf16(&tmB, g.B, g.N, g.K, g.ldb, 64, 64, g.f16)) return cudaErrorInvalidValue;
   }
+  // outputs: boxes of 32 rows x 128 bytes
+  const int dt0 = g.epi.kind == kEpiAtomic ? kDtF32 : g.epi.out0_dt;
+  if (!encode_tmap_2d_out(&tmO0, g.epi.out0, dt0, g.N, g.M, g.epi.ld_out0, 128 / dt_size(dt0), 32))
+    return cudaErrorInvalidValue;
+  if (g.epi.out1) {
+    if (!encode_tmap_2d_out(&tmO1, g.epi.out1, g.epi.out1_dt, g.N, g.M, g.epi.ld_out1, 128 / dt_size(g.epi.out1_dt), 32))
+      return cudaErrorInvalidValue;
+  } else {
+    tmO1 = tmO0;
+  }
   auto kern = gemm_bf16_tc_kernel<BN, STAGES, A_MN, B_MN>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kTotal);
   if (e != cudaSuccess) return e;
-  const int num_kb = static_cast<int>((g.K + kBK - 1) / kBK);
+  GemmParams P{};
+  P.M = static_cast<int>(g.M);
+  P.N = static_cast<int>(g.N);
+  P.num_kb = static_cast<int>((g.K + kBK - 1) / kBK);
   const int splits = g.splits < 1 ? 1 : g.splits;
-  const int kb_per = (num_kb + splits - 1) / splits;
-  const int zdim = (num_kb + kb_per - 1) / kb_per;
-  dim3 grid(static_cast<unsigned>((g.N + BN - 1) / BN), static_cast<unsigned>((g.M + kBM - 1) / kBM),
-            static_cast<unsigned>(zdim < 1 ? 1 : zdim));
-  const uint32_t idesc = make_idesc_f16kind(kBM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0, g.f16);
-  kern<<<grid, kThreads, L::kTotal, st>>>(tmA, tmB, static_cast<int>(g.M), static_cast<int>(g.N), num_kb,
-                                          kb_per, idesc, g.epi, wait_ctl(g.status));
+  P.kb_per = (P.num_kb + splits - 1) / splits;
+  P.splits = (P.num_kb + P.kb_per - 1) / P.kb_per;
+  P.tiles_n = static_cast<int>((g.N + BN - 1) / BN);
+  const int tiles_m = static_cast<int>((g.M + kBM - 1) / kBM);
+  P.total = tiles_m * P.tiles_n * P.splits;
+  P.idesc = make_idesc_f16kind(kBM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0, g.f16);
+  P.epi = g.epi;
+  const int grid = P.total < sm_count() ? P.total : sm_count();
+  kern<<<grid, kThreads, L::kTotal, st>>>(tmA, tmB, tmO0, tmO1, P, wait_ctl(g.status));
   return cudaGetLastError();
 }
 
@@ -352,7 +454,8 @@ cudaError_t dispatch_major(const GemmArgs& g, cudaStream_t st) {
 
 cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0) return cudaSuccess;
-  if (g.N % 256 == 0 && g.N >= 1024) return dispatch_major<256, 4>(g, st);
+  if (g.K <= 0) return cudaErrorInvalidValue;
+  if (g.N % 256 == 0 && g.N >= 1024) return dispatch_major<256, 3>(g, st);
   return dispatch_major<128, 4>(g, st);
 }
 

@@ -295,6 +295,23 @@ bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int6
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tmap_2d_out(CUtensorMap* map, const void* base, int dt, int64_t inner, int64_t outer, int64_t ld_elems,
+                        int box_inner, int box_outer) {
+  EncodeTiledFn fn = get_encode_fn();
+  const int64_t es = dt == kDtF32 ? 4 : 2;
+  if (!fn || !aligned16(base) || inner <= 0 || outer <= 0 || (ld_elems * es) % 16) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld_elems * es)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType t = dt == kDtF32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                : dt == kDtF16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = fn(map, t, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld_bytes,
                        int box_inner, int box_outer) {
   EncodeTiledFn fn = get_encode_fn();

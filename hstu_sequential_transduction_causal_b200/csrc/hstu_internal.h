@@ -55,6 +55,10 @@ struct GemmArgs {
 // 2D tensor map of a 2-byte element matrix (bf16, or fp16 when f16), 128-byte swizzle.
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t outer,
                          int64_t ld_elems, int box_inner, int box_outer, bool f16 = false);
+// 2D tensor map of an output matrix of element code dt (fp32, bf16, fp16), 128-byte swizzle, for
+// TMA stores and reduce-adds (box_inner * element size == 128).
+bool encode_tmap_2d_out(CUtensorMap* map, const void* base, int dt, int64_t inner, int64_t outer, int64_t ld_elems,
+                        int box_inner, int box_outer);
 // 2D tensor map of a u8 matrix, 128-byte swizzle (box_inner * 1 byte <= 128).
 bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld_bytes,
                        int box_inner, int box_outer);
