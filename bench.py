@@ -248,17 +248,23 @@ def main():
     weights = layer.weights()
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     # kernels of ours per step (cross-checked against the ncu launch list in profiles/)
-    n_fwd_kernels = 6          # f1 GEMM | work list, bias tiles, attention | LN-gate | f2 GEMM
-    n_bwd_kernels = 18         # 4 GEMMs, 2 column sums x 2, LN-gate bwd x 2, attention bwd x 4, dZ, 2 converts
+    # f1 GEMM | work list, bias tiles, attention | LN-gate | fp16 W2 copy, f2 GEMM
+    n_fwd_kernels = 7
+    # fp16 copies of dy, x, W1, W2 | dG, dW2 GEMMs | db2 (2) | LN-gate bwd + its finish | work list, transposed
+    # bias tiles, attention bwd | dZ | db1 (2) | dW1, dX GEMMs
+    n_bwd_kernels = 18
     names = ["uvqk", "attn", "norm_gate", "out_proj"] + (["backward"] if backward else [])
 
-    def step(ev=None):
+    def attention_forward():
+        H.hstu_attn_fwd(adesc, jag.struct, sv.uvqk[:, 2 * D:], sv.uvqk[:, 3 * D:], sv.uvqk[:, D:], layer.rab_pos,
+                        layer.rab_time, sv.o, ws)
+
+    def step(ev=None, all_reduce=True):
         rec = (lambda i: ev[i].record(stream)) if ev else (lambda i: None)
         rec(0)
         H.hstu_uvqk_fwd(T, D, H.HSTU_BF16, H.HSTU_F16, x, D, layer.W1, layer.b1, sv.uvqk, sv.z, ws)
         rec(1)
-        H.hstu_attn_fwd(adesc, jag.struct, sv.uvqk[:, 2 * D:], sv.uvqk[:, 3 * D:], sv.uvqk[:, D:], layer.rab_pos,
-                        layer.rab_time, sv.o, ws)
+        attention_forward()
         rec(2)
         H.hstu_norm_gate_fwd(T, D, H.HSTU_F32, H.HSTU_F16, H.HSTU_F16, sv.o, D, sv.uvqk, 4 * D, layer.gamma,
                              layer.beta, 1e-5, sv.g, sv.mu, sv.rstd)
@@ -268,7 +274,7 @@ def main():
         rec(4)
         if backward:
             H.hstu_layer_bwd(ldesc, jag.struct, weights, x, None, svs, dy, None, dx, None, grads, ws)
-            if world > 1:
+            if world > 1 and all_reduce:
                 dist.all_reduce(flat)
             rec(5)
 
@@ -281,18 +287,52 @@ def main():
         torch.cuda.synchronize()
         if H.hstu_sync_status(ws) != 0:
             raise RuntimeError("device status error during warm-up")
+        # per-piece device times of eagerly launched steps (the breakdown in the JSON line)
         nev = len(names) + 1
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+        n_eager = min(args.steps, 20)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n_eager)]
+        for i in range(n_eager):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+        seg = np.array([[e[k].elapsed_time(e[k + 1]) for k in range(nev - 1)] for e in evs])   # ms
+        # the timed steps replay one CUDA graph of the whole step (no host launch cost inside); the
+        # gradient all-reduce of a multi-GPU run follows each replay on the same stream
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step(all_reduce=False)
+        attn_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(attn_graph):
+            attention_forward()
+        for _ in range(3):
+            flush.zero_()
+            graph.replay()
+            attn_graph.replay()
+        torch.cuda.synchronize()
+        e_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         t_start = time.time()
         for i in range(args.steps):
             flush.zero_()
-            step(evs[i])
+            e_step[i][0].record(stream)
+            graph.replay()
+            if world > 1 and backward:
+                dist.all_reduce(flat)
+            e_step[i][1].record(stream)
         torch.cuda.synchronize()
         t_end = time.time()
         clk.window = (t_start, t_end)
+        n_attn = 20
+        e_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_attn)]
+        for i in range(n_attn):
+            flush.zero_()
+            e_attn[i][0].record(stream)
+            attn_graph.replay()
+            e_attn[i][1].record(stream)
+        torch.cuda.synchronize()
     finally:
         clk.__exit__()
     if world > 1:
@@ -300,9 +340,8 @@ def main():
     st = H.hstu_sync_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {st} in the timed region")
-    seg = np.array([[e[k].elapsed_time(e[k + 1]) for k in range(nev - 1)] for e in evs])   # ms
-    total_ms = float(seg.sum())
-    attn_ms = float(seg[:, 1].mean())
+    total_ms = float(sum(a.elapsed_time(b) for a, b in e_step))
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in e_attn]))
     t_tensor = torch.tensor([total_ms, attn_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t_tensor, op=dist.ReduceOp.MAX)
@@ -382,6 +421,8 @@ def main():
                          "peak_kind": f"{peak_kind} bf16 sustained (dense)", "traffic": traffic_record(args.workload),
                          "algorithmic_flops_per_launch": flops},
             "step_breakdown_ms": {k: float(seg[:, i].mean()) for i, k in enumerate(names)},
+            "timing": "device time of CUDA-graph replays of the whole step (events on the launching stream); "
+                      "step_breakdown_ms from eager launches",
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": int(h_y.numel() * 2)},
