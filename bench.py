@@ -180,6 +180,33 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def grad_buffer(D: int, pos_max_len: int, device):
+    """One flat fp32 buffer holding a layer's eight gradients (dW1, db1, dW2, db2, dgamma, dbeta,
+    drab_pos, drab_time), each view on a 16-byte boundary; a data-parallel step all-reduces it once."""
+    import torch
+    sizes = [4 * D * D, 4 * D, D * D, D, D, D, 2 * pos_max_len - 1, 128]
+    padded = [(n_ + 3) // 4 * 4 for n_ in sizes]
+    flat = torch.zeros(sum(padded), dtype=torch.float32, device=device)
+    views, o = [], 0
+    for n_, pn in zip(sizes, padded):
+        views.append(flat[o:o + n_])
+        o += pn
+    return flat, views
+
+
+def reduce_over_ranks(total_ms: float, attn_ms: float, tokens: int, world: int, device):
+    """Max over ranks of the device times, sum over ranks of the tokens (weak scaling: each rank
+    processes its own batch)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([total_ms, attn_ms], dtype=torch.float64, device=device)
+    n = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(n)
+    return float(t[0]), float(t[1]), float(n.item())
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -237,13 +264,7 @@ def main():
     ldesc = H.make_layer_desc(D, Hh, 1.0 / wl.N, wl.pos_max_len, H.HSTU_BF16, H.HSTU_BF16, H.HSTU_BF16)
     ws = workspace(max(H.hstu_attn_workspace_size(adesc, jag.struct),
                        H.hstu_layer_bwd_workspace_size(ldesc, jag.struct) if backward else 0), dev)
-    sizes = [4 * D * D, 4 * D, D * D, D, D, D, 2 * wl.pos_max_len - 1, 128]
-    padded = [(n_ + 3) // 4 * 4 for n_ in sizes]      # every gradient view 16-byte aligned
-    flat = torch.zeros(sum(padded), dtype=torch.float32, device=dev)
-    views, o = [], 0
-    for n_, pn in zip(sizes, padded):
-        views.append(flat[o:o + n_])
-        o += pn
+    flat, views = grad_buffer(D, wl.pos_max_len, dev)
     grads = H.layer_grads(*views)
     weights = layer.weights()
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -342,14 +363,7 @@ def main():
         raise RuntimeError(f"device status {st} in the timed region")
     total_ms = float(sum(a.elapsed_time(b) for a, b in e_step))
     attn_ms = float(np.mean([a.elapsed_time(b) for a, b in e_attn]))
-    t_tensor = torch.tensor([total_ms, attn_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_tensor, op=dist.ReduceOp.MAX)
-    total_ms, attn_ms_max = float(t_tensor[0]), float(t_tensor[1])
-    tt = torch.tensor([float(T)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tt)
-    tokens_all = float(tt.item())
+    total_ms, attn_ms_max, tokens_all = reduce_over_ranks(total_ms, attn_ms, T, world, dev)
     value = tokens_all * args.steps / (total_ms / 1e3)
 
     # End to end through the public layer API: per step the host->device copy of the step's inputs
