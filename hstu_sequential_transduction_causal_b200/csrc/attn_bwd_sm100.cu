@@ -48,8 +48,9 @@ __device__ __forceinline__ int pos_index_b(long long r, int L) {
 // ----------------------------------------------------------------------------------------------
 // transposed bias and bucket tiles
 // ----------------------------------------------------------------------------------------------
-// One block per causal tile pair. Thread t writes 8 consecutive queries [8 (t % 16), +8) of key
-// rows t / 16 + 16 p, p = 0..7: 16-byte half-bias and 8-byte bucket stores.
+// Four blocks per causal tile pair, 32 key rows each. Thread t writes 8 consecutive queries
+// [8 (t % 16), +8) of key rows 32 y + t / 16 + 16 p, p = 0, 1: 16-byte half-bias and 8-byte bucket
+// stores.
 __global__ void __launch_bounds__(256)
 attn_bias_t_kernel(AttnBwdArgs A) {
   const AttnArgs& a = A.f;
@@ -85,9 +86,9 @@ attn_bias_t_kernel(AttnBwdArgs A) {
   const long long tile0 = blockIdx.x * static_cast<long long>(kQTile * kQTile);
   uint16_t* tile = reinterpret_cast<uint16_t*>(A.bias_t) + tile0;
   uint8_t* btile = reinterpret_cast<uint8_t*>(A.bucket_t) + tile0;
-#pragma unroll 1
-  for (int pass = 0; pass < 8; ++pass) {
-    const int j = (tid >> 4) + 16 * pass;   // key row within the tile
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int j = 32 * blockIdx.y + (tid >> 4) + 16 * pass;   // key row within the tile
     const long long t_j = s_kts[j];
     uint32_t w[4], bw[2] = {0u, 0u};
 #pragma unroll
@@ -496,7 +497,7 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  attn_bias_t_kernel<<<static_cast<unsigned>(a.max_pairs), 256, 0, st>>>(A);
+  attn_bias_t_kernel<<<dim3(static_cast<unsigned>(a.max_pairs), 4), 256, 0, st>>>(A);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv, tdo, tbt, tbk;

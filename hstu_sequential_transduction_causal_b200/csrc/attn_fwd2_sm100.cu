@@ -51,8 +51,9 @@ __device__ __forceinline__ int pos_index2(long long r, int L) {
 // ----------------------------------------------------------------------------------------------
 // 1. bias tiles
 // ----------------------------------------------------------------------------------------------
-// One block per causal tile pair (blocks past the batch's last pair exit at once). Thread t writes
-// 8 consecutive keys [8 (t % 16), +8) of rows t / 16 + 16 p, p = 0..7: 16-byte coalesced stores.
+// Four blocks per causal tile pair, 32 query rows each (blocks past the batch's last pair exit at
+// once). Thread t writes 8 consecutive keys [8 (t % 16), +8) of rows 32 y + t / 16 + 16 p, p = 0, 1:
+// 16-byte coalesced stores.
 __global__ void __launch_bounds__(256)
 attn_bias_kernel(AttnArgs a) {
   int b, qt, kt;
@@ -85,9 +86,9 @@ attn_bias_kernel(AttnArgs a) {
   }
   __syncthreads();
   uint16_t* tile = reinterpret_cast<uint16_t*>(a.bias) + blockIdx.x * static_cast<long long>(kQTile * kQTile);
-#pragma unroll 1
-  for (int pass = 0; pass < 8; ++pass) {
-    const int r = (tid >> 4) + 16 * pass;   // query row within the tile
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int r = 32 * blockIdx.y + (tid >> 4) + 16 * pass;   // query row within the tile
     const long long t_i = s_qts[r];
     uint32_t w[4];
 #pragma unroll
@@ -483,7 +484,7 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  attn_bias_kernel<<<static_cast<unsigned>(a.max_pairs), 256, 0, st>>>(a);
+  attn_bias_kernel<<<dim3(static_cast<unsigned>(a.max_pairs), 4), 256, 0, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv, tb;
@@ -493,7 +494,11 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
       !encode_tmap_2d_bf16(&tv, a.v, static_cast<int64_t>(a.H) * kD, a.T, a.ld_v, 64, 128, f16) ||
       !encode_tmap_2d_bf16(&tb, a.bias, kQTile, a.max_pairs * kQTile, kQTile, 64, 128, true))
     return cudaErrorInvalidValue;
-  const int G = (a.H % 2 == 0) ? 2 : 1;
+  // Two heads per CTA share the Q-independent bias tile, but double the longest CTA's work: with
+  // long sequences (many key tiles in one query tile) the longest chain sets the kernel time, so one
+  // head per CTA is used there.
+  const int max_tiles = (a.max_len + kQTile - 1) / kQTile;
+  const int G = (a.H % 2 == 0 && max_tiles <= 8) ? 2 : 1;
   if (f16)
     return G == 2 ? launch_attn2<true, 2, false>(tq, tk, tv, tb, a, st)
                   : launch_attn2<true, 1, false>(tq, tk, tv, tb, a, st);
