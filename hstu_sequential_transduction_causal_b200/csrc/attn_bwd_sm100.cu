@@ -50,7 +50,7 @@ __device__ __forceinline__ int pos_index_b(long long r, int L) {
 // ----------------------------------------------------------------------------------------------
 // Four blocks per causal tile pair, 32 key rows each. Thread t writes 8 consecutive queries
 // [8 (t % 16), +8) of key rows 32 y + t / 16 + 16 p, p = 0, 1: 16-byte half-bias and 8-byte bucket
-// stores.
+// stores. Differences within a tile that fit in int32 take 32-bit bucket arithmetic.
 __global__ void __launch_bounds__(256)
 attn_bias_t_kernel(AttnBwdArgs A) {
   const AttnArgs& a = A.f;
@@ -58,38 +58,53 @@ attn_bias_t_kernel(AttnBwdArgs A) {
   if (!decode_tile_pair(blockIdx.x, a.pair_base, a.B, &b, &qt, &kt)) return;
   const long long seq0 = a.offsets[b];
   const int n = static_cast<int>(a.offsets[b + 1] - seq0);
-  __shared__ long long s_kts[128];
-  __shared__ long long s_tau[kTauEntries];
-  __shared__ float s_win[256];
-  __shared__ float s_rt[128];
-  const int tid = threadIdx.x;
+  __shared__ long long s_qts[128], s_kts[128], s_tau[kTauEntries], s_red[16];
+  __shared__ int s_tau32[kTauEntries];
+  __shared__ float s_win[256], s_rt[128];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = a.pos_max_len;
   const int nb = a.n_buckets;
+  long long t;
   if (tid < 128) {
-    const int kj = kt * kQTile + tid;
-    s_kts[tid] = a.ts[seq0 + (kj < n ? kj : n - 1)];
-    if (tid < nb) s_rt[tid] = a.rab_time[tid];
+    const int qi = qt * kQTile + tid;
+    t = a.ts[seq0 + (qi < n ? qi : n - 1)];
+    s_qts[tid] = t;
+  } else {
+    const int kj = kt * kQTile + tid - 128;
+    t = a.ts[seq0 + (kj < n ? kj : n - 1)];
+    s_kts[tid - 128] = t;
   }
-  {
-    const long long rel0 = static_cast<long long>(qt - kt) * kQTile - 127;
-    if (tid < 255) s_win[tid] = a.rab_pos[pos_index_b(rel0 + tid, L)];
+  if (tid < nb) s_rt[tid] = 0.5f * a.rab_time[tid];
+  if (tid < 255) s_win[tid] = 0.5f * a.rab_pos[pos_index_b(static_cast<long long>(qt - kt) * kQTile - 127 + tid, L)];
+  for (int e = tid; e < kTauEntries; e += 256) {
+    s_tau[e] = c_time_taus[e];
+    s_tau32[e] = c_time_taus32[e];
   }
-  for (int e = tid; e < kTauEntries; e += 256) s_tau[e] = c_time_taus[e];
-  const int c0 = 8 * (tid & 15);
-  long long qts[8];
+  long long mn = t, mx = t;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int qi = qt * kQTile + c0 + e;
-    qts[e] = a.ts[seq0 + (qi < n ? qi : n - 1)];
+  for (int d = 16; d > 0; d >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, d));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+  }
+  if (lane == 0) {
+    s_red[warp] = mn;
+    s_red[8 + warp] = mx;
   }
   __syncthreads();
+  long long lo = s_red[0], hi = s_red[8];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) {
+    lo = min(lo, s_red[w]);
+    hi = max(hi, s_red[8 + w]);
+  }
+  const bool fast = hi - lo < 0x7fffffffLL;
+  const int c0 = 8 * (tid & 15);
   const long long tile0 = blockIdx.x * static_cast<long long>(kQTile * kQTile);
   uint16_t* tile = reinterpret_cast<uint16_t*>(A.bias_t) + tile0;
   uint8_t* btile = reinterpret_cast<uint8_t*>(A.bucket_t) + tile0;
 #pragma unroll
   for (int pass = 0; pass < 2; ++pass) {
     const int j = 32 * blockIdx.y + (tid >> 4) + 16 * pass;   // key row within the tile
-    const long long t_j = s_kts[j];
     uint32_t w[4], bw[2] = {0u, 0u};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -97,8 +112,10 @@ attn_bias_t_kernel(AttnBwdArgs A) {
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
         const int col = c0 + 2 * e + x;     // query column
-        const int bkt = time_bucket_dev(qts[2 * e + x] - t_j, s_tau, nb);
-        v2[x] = 0.5f * (s_win[col - j + 127] + s_rt[bkt]);
+        const int bkt = fast ? time_bucket32(static_cast<int>(s_qts[col] - lo) - static_cast<int>(s_kts[j] - lo),
+                                             s_tau32, nb)
+                             : time_bucket_dev(s_qts[col] - s_kts[j], s_tau, nb);
+        v2[x] = s_win[col - j + 127] + s_rt[bkt];
         bw[e >> 1] |= static_cast<uint32_t>(bkt) << (8 * (2 * (e & 1) + x));
       }
       w[e] = pack_f16x2(v2[0], v2[1]);

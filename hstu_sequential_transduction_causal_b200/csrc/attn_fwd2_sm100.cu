@@ -38,8 +38,8 @@ namespace {
 
 constexpr int kD = 64;
 constexpr int kNS = 3;                 // K/V stages
-constexpr int kSiluWarps = 8;
-constexpr int kThreads2 = 32 * (kSiluWarps + 2);
+constexpr int kSiluWarps = 8;     // one group of SiLU warps: 4 TMEM lane quadrants x 2 key halves
+__host__ __device__ constexpr int threads2(int ng) { return 32 * (kSiluWarps * ng + 2); }
 constexpr uint32_t kHalf2Half = 0x38003800u;   // (0.5, 0.5) in fp16
 
 __device__ __forceinline__ int pos_index2(long long r, int L) {
@@ -51,6 +51,52 @@ __device__ __forceinline__ int pos_index2(long long r, int L) {
 // ----------------------------------------------------------------------------------------------
 // 1. bias tiles
 // ----------------------------------------------------------------------------------------------
+// Stages a tile pair's query and key timestamps (q_ts, k_ts: 128 each, clamped to the sequence),
+// the rab_pos window of its diagonals and rab_time, both pre-halved, and the bucket thresholds; returns
+// through lo / fast whether every difference of the tile fits in int32 (then offsets from lo are used).
+__device__ __forceinline__ void stage_tile_pair(const AttnArgs& a, long long seq0, int n, int qt, int kt,
+                                                long long* s_qts, long long* s_kts, float* s_win, float* s_rt,
+                                                long long* s_tau, int* s_tau32, long long* s_red, long long& lo,
+                                                bool& fast) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  long long t;
+  if (tid < 128) {
+    const int qi = qt * kQTile + tid;
+    t = a.ts[seq0 + (qi < n ? qi : n - 1)];
+    s_qts[tid] = t;
+  } else {
+    const int kj = kt * kQTile + tid - 128;
+    t = a.ts[seq0 + (kj < n ? kj : n - 1)];
+    s_kts[tid - 128] = t;
+  }
+  if (tid < a.n_buckets) s_rt[tid] = 0.5f * a.rab_time[tid];
+  if (tid < 255) s_win[tid] = 0.5f * a.rab_pos[pos_index2(static_cast<long long>(qt - kt) * kQTile - 127 + tid,
+                                                          a.pos_max_len)];
+  for (int e = tid; e < kTauEntries; e += 256) {
+    s_tau[e] = c_time_taus[e];
+    s_tau32[e] = c_time_taus32[e];
+  }
+  long long mn = t, mx = t;
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, d));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+  }
+  if (lane == 0) {
+    s_red[warp] = mn;
+    s_red[8 + warp] = mx;
+  }
+  __syncthreads();
+  long long bmn = s_red[0], bmx = s_red[8];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) {
+    bmn = min(bmn, s_red[w]);
+    bmx = max(bmx, s_red[8 + w]);
+  }
+  lo = bmn;
+  fast = bmx - bmn < 0x7fffffffLL;
+}
+
 // Four blocks per causal tile pair, 32 query rows each (blocks past the batch's last pair exit at
 // once). Thread t writes 8 consecutive keys [8 (t % 16), +8) of rows 32 y + t / 16 + 16 p, p = 0, 1:
 // 16-byte coalesced stores.
@@ -60,47 +106,46 @@ attn_bias_kernel(AttnArgs a) {
   if (!decode_tile_pair(blockIdx.x, a.pair_base, a.B, &b, &qt, &kt)) return;
   const long long seq0 = a.offsets[b];
   const int n = static_cast<int>(a.offsets[b + 1] - seq0);
-  __shared__ long long s_qts[128];
-  __shared__ long long s_tau[kTauEntries];
-  __shared__ float s_win[256];
-  __shared__ float s_rt[128];
+  __shared__ long long s_qts[128], s_kts[128], s_tau[kTauEntries], s_red[16];
+  __shared__ int s_tau32[kTauEntries];
+  __shared__ float s_win[256], s_rt[128];
+  long long lo;
+  bool fast;
+  stage_tile_pair(a, seq0, n, qt, kt, s_qts, s_kts, s_win, s_rt, s_tau, s_tau32, s_red, lo, fast);
   const int tid = threadIdx.x;
-  const int L = a.pos_max_len;
   const int nb = a.n_buckets;
-  if (tid < 128) {
-    const int qi = qt * kQTile + tid;
-    s_qts[tid] = a.ts[seq0 + (qi < n ? qi : n - 1)];
-    if (tid < nb) s_rt[tid] = a.rab_time[tid];
-  }
-  {
-    const long long rel0 = static_cast<long long>(qt - kt) * kQTile - 127;
-    if (tid < 255) s_win[tid] = a.rab_pos[pos_index2(rel0 + tid, L)];
-  }
-  for (int e = tid; e < kTauEntries; e += 256) s_tau[e] = c_time_taus[e];
   const int c0 = 8 * (tid & 15);
-  long long kts[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int kj = kt * kQTile + c0 + e;
-    kts[e] = a.ts[seq0 + (kj < n ? kj : n - 1)];
-  }
-  __syncthreads();
   uint16_t* tile = reinterpret_cast<uint16_t*>(a.bias) + blockIdx.x * static_cast<long long>(kQTile * kQTile);
 #pragma unroll
   for (int pass = 0; pass < 2; ++pass) {
     const int r = 32 * blockIdx.y + (tid >> 4) + 16 * pass;   // query row within the tile
-    const long long t_i = s_qts[r];
     uint32_t w[4];
+    if (fast) {
+      const int ti = static_cast<int>(s_qts[r] - lo);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float v2[2];
+      for (int e = 0; e < 4; ++e) {
+        float v2[2];
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        const int col = c0 + 2 * e + x;
-        const int bkt = time_bucket_dev(t_i - kts[2 * e + x], s_tau, nb);
-        v2[x] = 0.5f * (s_win[r - col + 127] + s_rt[bkt]);
+        for (int x = 0; x < 2; ++x) {
+          const int col = c0 + 2 * e + x;
+          const int bkt = time_bucket32(ti - static_cast<int>(s_kts[col] - lo), s_tau32, nb);
+          v2[x] = s_win[r - col + 127] + s_rt[bkt];
+        }
+        w[e] = pack_f16x2(v2[0], v2[1]);
       }
-      w[e] = pack_f16x2(v2[0], v2[1]);
+    } else {
+      const long long t_i = s_qts[r];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v2[2];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int col = c0 + 2 * e + x;
+          const int bkt = time_bucket_dev(t_i - s_kts[col], s_tau, nb);
+          v2[x] = s_win[r - col + 127] + s_rt[bkt];
+        }
+        w[e] = pack_f16x2(v2[0], v2[1]);
+      }
     }
     *reinterpret_cast<uint4*>(tile + r * kQTile + c0) = make_uint4(w[0], w[1], w[2], w[3]);
   }
@@ -111,19 +156,24 @@ attn_bias_kernel(AttnArgs a) {
 // ----------------------------------------------------------------------------------------------
 template <int G>
 struct Smem2 {
+  static constexpr int kBS = G == 1 ? 3 : 2;   // bias stages (one head per CTA: a bias tile per unit)
   static constexpr int kQ = 0;
   static constexpr int kKV = G * 16384;
   static constexpr int kBias = kKV + kNS * 32768;
-  static constexpr int kBar = kBias + 2 * 32768;
+  static constexpr int kBar = kBias + kBS * 32768;
   static constexpr int kTotal = kBar + 256 + 1024;
 };
 
-template <bool F16, int G, bool FALCON>
-__global__ void __launch_bounds__(kThreads2, 1)
+// NG = 2 (one head per CTA only): two groups of SiLU warps take alternate key tiles, so one group's
+// SiLU of tile t overlaps the other's of tile t + 1 (each group owns one S buffer and one bias stage).
+template <bool F16, int G, bool FALCON, int NG>
+__global__ void __launch_bounds__(threads2(NG), 1)
 attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB, AttnArgs a,
                     WaitCtl ctl) {
   using L = Smem2<G>;
+  static_assert(NG == 1 || G == 1, "two SiLU groups need one head per CTA");
+  constexpr int kTmaWarp = kSiluWarps * NG, kMmaWarp = kTmaWarp + 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int HG = a.H / G;
@@ -148,20 +198,21 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const int nsteps = nkt * G;
   const long long pair0 = FALCON ? 0 : a.pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2;
 
+  constexpr int BS = L::kBS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  // 0 q_full | 1..3 kv_full | 4..6 kv_empty | 7,8 b_full | 9,10 b_empty | 11,12 s_full |
-  // 13,14 p_full | 15 o_full
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  // 0 q_full | 1..3 kv_full | 4..6 kv_empty | b_full [BS] | b_empty [BS] | s_full [2] | p_full [2] |
+  // o_full
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12 + 2 * BS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  const uint32_t bar_q = BAR(0), bar_o = BAR(15);
+  const uint32_t bar_q = BAR(0), bar_o = BAR(11 + 2 * BS);
   auto bar_kv_full = [&](int s) { return BAR(1 + s); };
   auto bar_kv_empty = [&](int s) { return BAR(4 + s); };
   auto bar_b_full = [&](int s) { return BAR(7 + s); };
-  auto bar_b_empty = [&](int s) { return BAR(9 + s); };
-  auto bar_s_full = [&](int s) { return BAR(11 + s); };
-  auto bar_p_full = [&](int s) { return BAR(13 + s); };
+  auto bar_b_empty = [&](int s) { return BAR(7 + BS + s); };
+  auto bar_s_full = [&](int s) { return BAR(7 + 2 * BS + s); };
+  auto bar_p_full = [&](int s) { return BAR(9 + 2 * BS + s); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -173,9 +224,11 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       mbar_init(bar_kv_full(s), 1);
       mbar_init(bar_kv_empty(s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < BS; ++s) {
       mbar_init(bar_b_full(s), 1);
       mbar_init(bar_b_empty(s), kSiluThreads);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(bar_s_full(s), 1);
       mbar_init(bar_p_full(s), kSiluThreads);
     }
@@ -183,7 +236,7 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kSiluWarps && lane == 0) {
+  if (warp == kTmaWarp && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -203,7 +256,7 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const uint32_t sB = smem_u32(smem + L::kBias);
   const int qrow0 = FALCON ? b * a.cand_rows + qt * kQTile : static_cast<int>(seq0) + qt * kQTile;
 
-  if (warp == kSiluWarps) {
+  if (warp == kTmaWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_q, G * 16384);
@@ -212,8 +265,8 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       int s = 0;
       for (int kt = 0; ok && kt < nkt; ++kt) {
         if constexpr (!FALCON) {
-          const int bs = kt & 1;
-          if (kt >= 2 && !mbar_wait(bar_b_empty(bs), ((kt >> 1) & 1) ^ 1, abort_flag, ctl)) break;
+          const int bs = kt % BS;
+          if (kt >= BS && !mbar_wait(bar_b_empty(bs), ((kt / BS) - 1) & 1, abort_flag, ctl)) break;
           const int brow = static_cast<int>((pair0 + kt) * kQTile);
           mbar_arrive_expect_tx(bar_b_full(bs), 32768);
           tma_load_2d(sB + bs * 32768, &tmB, bar_b_full(bs), 0, brow);
@@ -232,7 +285,7 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         }
       }
     }
-  } else if (warp == kSiluWarps + 1) {
+  } else if (warp == kMmaWarp) {
     // ---------------- tcgen05 issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc_f16kind(128, 128, 0, 0, F16);
@@ -269,32 +322,17 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     }
   } else {
     // ---------------- SiLU warps ----------------
+    const int grp = warp / kSiluWarps;   // NG == 2: group g takes key tiles g, g + 2, ...
     const int quad = warp & 3;
-    const int half = warp >> 2;          // keys [64 half, 64 half + 64)
+    const int half = (warp >> 2) & 1;    // keys [64 half, 64 half + 64)
     const int r = quad * 32 + lane;      // query row within the tile == TMEM lane
     const int qi = qt * kQTile + r;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     bool ok = true;
-    for (int kt = 0; ok && kt < nkt; ++kt) {
-      uint32_t hb[32];
-      if constexpr (FALCON) {
-        // the bias depends on the key only: one 64-key row shared by every query row
-        const uint4* src = reinterpret_cast<const uint4*>(a.kbias + b * a.kbias_ld + kt * kQTile + 64 * half);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 v = __ldg(src + u);
-          hb[4 * u] = v.x; hb[4 * u + 1] = v.y; hb[4 * u + 2] = v.z; hb[4 * u + 3] = v.w;
-        }
-      } else {
-        const int bs = kt & 1;
-        if (!mbar_wait(bar_b_full(bs), (kt >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
-        const uint8_t* brow = smem + L::kBias + bs * 32768 + half * 16384 + r * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint4 v = *reinterpret_cast<const uint4*>(brow + ((u ^ (r & 7)) << 4));
-          hb[4 * u] = v.x; hb[4 * u + 1] = v.y; hb[4 * u + 2] = v.z; hb[4 * u + 3] = v.w;
-        }
-        mbar_arrive(bar_b_empty(bs));
+    for (int kt = grp; ok && kt < nkt; kt += NG) {
+      const int bs = kt % BS;
+      if constexpr (!FALCON) {
+        if (!mbar_wait(bar_b_full(bs), (kt / BS) & 1, abort_flag, ctl)) { ok = false; break; }
       }
       // FALCON: keys past the user's prefix (last tile) are masked; causal: the diagonal tile
       const int key_lim = FALCON ? n - kt * kQTile : 0;
@@ -304,16 +342,36 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int buf = s & 1;
         if (!mbar_wait(bar_s_full(buf), (s >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
         tc_fence_after();
-        uint32_t p[32];
 #pragma unroll
         for (int hc = 0; hc < 2; ++hc) {
           uint32_t sv[32];
           tmem_ld_32x32b_x32(tmem + lane_base + buf * 128 + 64 * half + 32 * hc, sv);
+          uint32_t hb[16];   // half-bias of keys [64 half + 32 hc, +32)
+          if constexpr (FALCON) {
+            // the bias depends on the key only: one row shared by every query row
+            const uint4* src =
+                reinterpret_cast<const uint4*>(a.kbias + b * a.kbias_ld + kt * kQTile + 64 * half + 32 * hc);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint4 v = __ldg(src + u);
+              hb[4 * u] = v.x; hb[4 * u + 1] = v.y; hb[4 * u + 2] = v.z; hb[4 * u + 3] = v.w;
+            }
+          } else {
+            const uint8_t* brow = smem + L::kBias + bs * 32768 + half * 16384 + r * 128;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint4 v = *reinterpret_cast<const uint4*>(brow + (((4 * hc + u) ^ (r & 7)) << 4));
+              hb[4 * u] = v.x; hb[4 * u + 1] = v.y; hb[4 * u + 2] = v.z; hb[4 * u + 3] = v.w;
+            }
+            // one head: the bias stage is free once both halves of its row are in registers
+            if (G == 1 && hc == 1) mbar_arrive(bar_b_empty(bs));
+          }
           tmem_ld_wait();
+          uint32_t p[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const uint32_t s2 = pack_f16x2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1]));
-            const uint32_t h2 = hfma2_u32(s2, kHalf2Half, hb[16 * hc + j]);
+            const uint32_t h2 = hfma2_u32(s2, kHalf2Half, hb[j]);
             const uint32_t t2 = tanh_f16x2(h2);
             uint32_t y2 = hfma2_u32(h2, t2, h2);
             if (!F16) {   // the P V MMA takes A and B of one type: P as bf16 next to bf16 V
@@ -326,15 +384,18 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
               const uint32_t m = (col + 1 <= lim) ? 0xFFFFFFFFu : ((col <= lim) ? 0x0000FFFFu : 0u);
               y2 &= m;
             }
-            p[16 * hc + j] = y2;
+            p[j] = y2;
           }
+          // P of these 32 keys packed into 16 columns over S chunk 0 (already read)
+          tmem_st_32x32b_x16(tmem + lane_base + buf * 128 + 64 * half + 16 * hc, p);
         }
-        tmem_st_32x32b_x32(tmem + lane_base + buf * 128 + 64 * half, p);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar_p_full(buf));
       }
+      if constexpr (!FALCON && G > 1) mbar_arrive(bar_b_empty(bs));
     }
+    if (grp > 0) ok = false;   // the epilogue is group 0's
     if (ok && (nkt == 0 || mbar_wait(bar_o, 0, abort_flag, ctl))) {
       tc_fence_after();
       // G == 1: both key halves split head 0's 64 columns; G >= 2: half c handles heads c, c+2, ...
@@ -461,13 +522,14 @@ falcon_key_bias_kernel(const int64_t* __restrict__ off, const int64_t* __restric
 template <bool F16, int G, bool FALCON>
 cudaError_t launch_attn2(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tb,
                          const AttnArgs& a, cudaStream_t st) {
-  auto kern = attn_fwd_tc2_kernel<F16, G, FALCON>;
+  constexpr int NG = G == 1 ? 2 : 1;
+  auto kern = attn_fwd_tc2_kernel<F16, G, FALCON, NG>;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), Smem2<G>::kTotal);
   if (e != cudaSuccess) return e;
   const long long blocks =
       (FALCON ? static_cast<long long>(a.B) * ((a.cand_rows + kQTile - 1) / kQTile) : a.capacity) * (a.H / G);
   if (blocks == 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(blocks), kThreads2, Smem2<G>::kTotal, st>>>(tq, tk, tv, tb, a, wait_ctl(a.status));
+  kern<<<static_cast<unsigned>(blocks), threads2(NG), Smem2<G>::kTotal, st>>>(tq, tk, tv, tb, a, wait_ctl(a.status));
   return cudaGetLastError();
 }
 

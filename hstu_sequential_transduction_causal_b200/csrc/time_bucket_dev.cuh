@@ -26,6 +26,20 @@ __device__ __forceinline__ int time_bucket_dev(long long dt, const long long* ta
   return min(k, nb - 1);
 }
 
+// The same for a difference known to fit in int32 (timestamps of a tile within 2^31 of each other):
+// tau32 holds tau_k saturated to INT32_MAX (tau_72 > 2^31 > every int32 dt, so no bucket past 71 is
+// reached) and tau32[0] = INT32_MIN; all arithmetic is 32-bit.
+__constant__ int c_time_taus32[kTauEntries];
+
+__device__ __forceinline__ int time_bucket32(int dt, const int* tau, int nb) {
+  if (dt <= 1) return 0;
+  constexpr float kLn2Over0301 = 0.693147180559945f / 0.301f;
+  const float lf = __log2f(static_cast<float>(dt)) * kLn2Over0301;
+  int k = min(static_cast<int>(lf), 126);
+  k += (dt >= tau[k + 1] ? 1 : 0) - (dt < tau[k] ? 1 : 0);
+  return min(k, nb - 1);
+}
+
 // Copies tau_0..tau_128 to this translation unit's constant bank, once per device.
 inline cudaError_t upload_time_taus() {
   static bool done[64] = {};
@@ -38,6 +52,10 @@ inline cudaError_t upload_time_taus() {
   for (int k = 1; k <= HSTU_TB_NUM_THRESHOLDS; ++k) taus[k] = kHstuTimeThresholds[k - 1];
   for (int k = HSTU_TB_NUM_THRESHOLDS + 1; k < kTauEntries; ++k) taus[k] = 0x7fffffffffffffffLL;
   e = cudaMemcpyToSymbol(c_time_taus, taus, sizeof(taus));
+  int taus32[kTauEntries];
+  for (int k = 0; k < kTauEntries; ++k)
+    taus32[k] = k == 0 ? (-0x7fffffff - 1) : (taus[k] > 0x7fffffffLL ? 0x7fffffff : static_cast<int>(taus[k]));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_time_taus32, taus32, sizeof(taus32));
   if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
   return e;
 }
