@@ -25,7 +25,8 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kThreads = 192;   // warps 0-3 epilogue, warp 4 TMA, warp 5 MMA
+constexpr int kEpiWarps = 8;    // 2 per TMEM lane quadrant, each on half of the tile's columns
+constexpr int kThreads = 32 * (kEpiWarps + 2);   // warps 0-7 epilogue, warp 8 TMA, warp 9 MMA
 constexpr int kBoxBytes = 4096; // one epilogue staging box: 32 rows x 128 bytes
 
 template <int BN, int STAGES>
@@ -34,8 +35,8 @@ struct GemmSmem {
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTileBytes = STAGES * kStageBytes;
-  static constexpr int kOut = kTileBytes;            // 4 warps x 2 staging boxes
-  static constexpr int kBarOff = kOut + 4 * 2 * kBoxBytes;
+  static constexpr int kOut = kTileBytes;            // 8 epilogue warps x 2 staging boxes
+  static constexpr int kBarOff = kOut + kEpiWarps * 2 * kBoxBytes;
   static constexpr int kTotal = kBarOff + 256 + 1024;   // barriers + alignment slack
 };
 
@@ -155,12 +156,12 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     for (int i = 0; i < 2 * STAGES; ++i) mbar_init(smem_u32(&bars[i]), 1);
     for (int b = 0; b < 2; ++b) {
       mbar_init(acc_full(b), 1);
-      mbar_init(acc_empty(b), 128);
+      mbar_init(acc_empty(b), 32 * kEpiWarps);
     }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kEpiWarps && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
@@ -182,7 +183,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     kb1 = min(P.num_kb, kb0 + P.kb_per);
   };
 
-  if (warp == 4) {
+  if (warp == kEpiWarps) {
     if (lane == 0) {
       int g = 0;
       bool ok = true;
@@ -215,7 +216,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kEpiWarps + 1) {
     if (lane == 0) {
       int g = 0, it = 0;
       bool ok = true;
@@ -246,8 +247,10 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       }
     }
   } else {
-    // epilogue warps 0-3: TMEM lanes 32 warp .. +31 = output rows m0 + 32 warp + lane
+    // epilogue warps 0-7: TMEM lanes 32 (warp % 4) .. +31 = output rows m0 + 32 (warp % 4) + lane,
+    // columns [BN/2 (warp / 4), +BN/2)
     const GemmEpilogue& epi = P.epi;
+    const int quad = warp & 3, chalf = warp >> 2;
     EpiStage es{smem + L::kOut + warp * 2 * kBoxBytes, 0};
     int it = 0;
     for (int t = blockIdx.x; t < P.total; t += gridDim.x, ++it) {
@@ -256,24 +259,26 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const int buf = it & 1;
       if (!mbar_wait(acc_full(buf), (it >> 1) & 1, abort_flag, ctl)) break;
       tc_fence_after();
-      const int row = m0 + warp * 32 + lane;
+      const int row = m0 + quad * 32 + lane;
       const bool row_ok = row < P.M;
-      const int ybox = m0 + warp * 32;
+      const int ybox = m0 + quad * 32;
+      constexpr int kChunks = BN / 128;   // 64-column chunks per warp
 #pragma unroll 1
-      for (int c = 0; c < BN / 64; ++c) {
-        const int n = n0 + c * 64;
+      for (int c = 0; c < kChunks; ++c) {
+        const int col = chalf * (BN / 2) + c * 64;   // within the tile
+        const int n = n0 + col;
         float v[64];
         {
           uint32_t r[32];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            tmem_ld_32x32b_x32(tmem_acc + buf * BN + (static_cast<uint32_t>(warp * 32) << 16) + c * 64 + 32 * h, r);
+            tmem_ld_32x32b_x32(tmem_acc + buf * BN + (static_cast<uint32_t>(quad * 32) << 16) + col + 32 * h, r);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[32 * h + j] = __uint_as_float(r[j]);
           }
         }
-        if (c == BN / 64 - 1) {   // the whole accumulator is in registers: release it to the MMA
+        if (c == kChunks - 1) {   // this warp's part of the accumulator is in registers: release it
           tc_fence_before();
           mbar_arrive(acc_empty(buf));
         }
