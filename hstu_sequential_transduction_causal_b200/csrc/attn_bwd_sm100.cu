@@ -12,14 +12,17 @@
 // [key][query] and the u8 time-bucket tile [key][query] (head independent, computed once).
 // attn_bwd_tc_kernel<F16>: one CTA per (sequence, 128-key tile, head), key tiles that visit the
 // most query tiles first; it walks the query tiles t >= its key tile:
-//   warp 8   : TMA: K, V once; Q and dO of each query tile (2 stages); bias and bucket tiles.
+//   warp 8   : TMA: K, V once; Q and dO of each query tile (2 stages); the half-bias tile.
 //   warp 9   : tcgen05: S^T = K Q^T and dA^T = V dO^T into TMEM; after the elementwise step
 //              dV += P^T dO (P^T from TMEM), dK += dX^T Q and dQ_tile = dX K (dX^T from shared
 //              memory, read K-major for dK and MN-major for dQ).
+//   warp 10  : TMA store of each tile's dX^T (16-bit, from shared memory) to the workspace.
 //   warps 0-7: key row = TMEM lane (warp & 3), query half (warp >> 2): x = s + bias,
-//              P^T = SiLU(x), dX^T = dA SiLU'(x) inv_N in fp32, causal and length masks; the
-//              position-bias gradient by shared atomics (one window per query tile), the time-bias
-//              gradient by runs of equal bucket; dQ_tile added to the fp32 dQ by vector atomics.
+//              P^T = SiLU(x), dX^T = dA SiLU'(x) inv_N in fp32, causal and length masks;
+//              dQ_tile added to the fp32 dQ by vector atomics.
+// attn_table_grad_kernel<F16>: per causal tile pair, sums the H heads' dX^T tiles and adds them to
+// d rab_pos (by diagonal) and d rab_time (by bucket): the tables are shared by the heads, so the
+// head sum comes first and each table entry takes one atomic per tile pair.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -36,7 +39,7 @@ namespace {
 
 constexpr int kD = 64;
 constexpr int kSiluWarpsB = 8;
-constexpr int kThreadsB = 32 * (kSiluWarpsB + 2);
+constexpr int kThreadsB = 32 * (kSiluWarpsB + 3);   // + TMA producer, MMA issuer, dX^T store warp
 constexpr int kSiluThreadsB = 32 * kSiluWarpsB;
 
 __device__ __forceinline__ int pos_index_b(long long r, int L) {
@@ -133,11 +136,7 @@ struct BwdSmem {
   static constexpr int kV = 16384;              // V tile (16 KB)
   static constexpr int kQ0 = 32768;             // stage st: Q at kQ0 + st * 32768, dO at +16384
   static constexpr int kBT0 = kQ0 + 2 * 32768;  // stage st: half-bias^T, overwritten in place by dX^T
-  static constexpr int kBK0 = kBT0 + 2 * 32768; // stage st: bucket^T (16 KB)
-  static constexpr int kTime = kBK0 + 2 * 16384;   // d rab_time partial sums, one copy per lane [128][32]
-  static constexpr int kPos = kTime + 128 * 32 * 4;  // d rab_pos partial sums of the CTA's diagonals
-  static constexpr int kPosWin = 4352;          // diagonals 128 s + d, -127 <= d <= 127, s <= 32
-  static constexpr int kBar = kPos + kPosWin * 4;
+  static constexpr int kBar = kBT0 + 2 * 32768;
   static constexpr int kTotal = kBar + 256 + 1024;
 };
 static_assert(BwdSmem::kTotal <= 232448, "shared memory of the backward kernel");
@@ -146,8 +145,8 @@ template <bool F16>
 __global__ void __launch_bounds__(kThreadsB, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                   const __grid_constant__ CUtensorMap tmBT, const __grid_constant__ CUtensorMap tmBK, AttnBwdArgs A,
-                   WaitCtl ctl) {
+                   const __grid_constant__ CUtensorMap tmBT, const __grid_constant__ CUtensorMap tmDX,
+                   AttnBwdArgs A, WaitCtl ctl) {
   using Lb = BwdSmem;
   const AttnArgs& a = A.f;
   extern __shared__ uint8_t smem_raw[];
@@ -165,14 +164,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lb::kBar);
   // 0 kv_full | 1,2 qdo_full | 3,4 qdo_empty | 5,6 bb_full | 7,8 bb_empty | 9,10 s_full (query half
-  // a, b) | 11,12 p_ready (half a, b) | 13 dq_full | 14 fin
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  // a, b) | 11,12 p_ready (half a, b) | 13 dq_full | 14 fin | 15,16 dx_full (stage)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  float* s_dtime = reinterpret_cast<float*>(smem + Lb::kTime);
-  float* s_dpos = reinterpret_cast<float*>(smem + Lb::kPos);
-  const int pos_used = min(Lb::kPosWin, 128 * nsteps + 255);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -184,7 +180,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(BAR(1 + s), 1);
       mbar_init(BAR(3 + s), 1);
       mbar_init(BAR(5 + s), 1);
-      mbar_init(BAR(7 + s), 1);
+      mbar_init(BAR(7 + s), 2);   // bias/dX stage free: the MMAs read dX^T and the store warp sent it
+      mbar_init(BAR(15 + s), kSiluThreadsB);   // both query halves of dX^T written
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(BAR(9 + h), 1);
@@ -195,15 +192,13 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     *abort_flag = 0;
     fence_barrier_init();
   }
-  for (int e = tid; e < 128 * 32; e += kThreadsB) s_dtime[e] = 0.0f;
-  for (int e = tid; e < pos_used; e += kThreadsB) s_dpos[e] = 0.0f;
   if (warp == kSiluWarpsB && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmDO);
     tma_prefetch_desc(&tmBT);
-    tma_prefetch_desc(&tmBK);
+    tma_prefetch_desc(&tmDX);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -219,7 +214,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   const uint32_t sK = smem_u32(smem + Lb::kK), sV = smem_u32(smem + Lb::kV);
   const uint32_t sQ0 = smem_u32(smem + Lb::kQ0);
-  const uint32_t sBT0 = smem_u32(smem + Lb::kBT0), sBK0 = smem_u32(smem + Lb::kBK0);
+  const uint32_t sBT0 = smem_u32(smem + Lb::kBT0);
   const int krow = static_cast<int>(seq0) + kt * kQTile;
 
   if (warp == kSiluWarpsB) {
@@ -238,10 +233,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tma_load_2d(sQ0 + st * 32768 + 16384, &tmDO, BAR(1 + st), h * kD, qrow);
         if (s >= 2 && !mbar_wait(BAR(7 + st), ph_free, abort_flag, ctl)) break;
         const int prow = static_cast<int>((pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt) * kQTile);
-        mbar_arrive_expect_tx(BAR(5 + st), 32768 + 16384);
+        mbar_arrive_expect_tx(BAR(5 + st), 32768);
         tma_load_2d(sBT0 + st * 32768, &tmBT, BAR(5 + st), 0, prow);
         tma_load_2d(sBT0 + st * 32768 + 16384, &tmBT, BAR(5 + st), 64, prow);
-        tma_load_2d(sBK0 + st * 16384, &tmBK, BAR(5 + st), 0, prow);
       }
     }
   } else if (warp == kSiluWarpsB + 1) {
@@ -306,6 +300,25 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       if (ok) umma_commit(BAR(14));
     }
+  } else if (warp == kSiluWarpsB + 2) {
+    // ---------------- dX^T store ----------------
+    // Once both query halves of tile s are done, dX^T (the fp16 operand of dK and dQ, in the stage's
+    // bias slot) goes to the workspace; the table gradients are summed from there over the heads.
+    if (lane == 0) {
+      for (int s = 0; s < nsteps; ++s) {
+        const int st = s & 1;
+        if (!mbar_wait(BAR(15 + st), (s >> 1) & 1, abort_flag, ctl)) break;
+        const int qt = kt + s;
+        const long long pair = pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt;
+        const int y = static_cast<int>((pair * a.H + h) * kQTile);
+        tma_store_2d(&tmDX, sBT0 + st * 32768, 0, y);
+        tma_store_2d(&tmDX, sBT0 + st * 32768 + 16384, 64, y);
+        bulk_commit_group();
+        bulk_wait_group_read<0>();
+        mbar_arrive(BAR(7 + st));
+      }
+      bulk_wait_group_all();
+    }
   } else {
     // ---------------- elementwise warps ----------------
     const int quad = warp & 3;
@@ -314,11 +327,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const bool key_ok = kt * kQTile + rj < n;
     const float inv_N = a.inv_N;
-    // d rab_time: each thread sums runs of equal bucket along its key row; a closed run is added to
-    // the lane's own copy of the histogram (lanes of a warp never collide)
-    int cur_b = -1;
-    uint32_t cur_rep = 0xFFFFFFFFu;
-    float acc_t = 0.0f;
     bool ok = true;
     auto flush_dq = [&](int s_prev) {
       // (half-b warps) dQ tile of query tile kt + s_prev: TMEM lane = query row, all 64 columns
@@ -357,23 +365,17 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int lo_col = (s == 0) ? rj : 0;
       const int hi_col = key_ok ? min(kQTile, n - qt * kQTile) : 0;
       uint8_t* bt_row = smem + Lb::kBT0 + st * 32768 + hq * 16384 + rj * 128;
-      const uint8_t* bk_row = smem + Lb::kBK0 + st * 16384 + rj * 128;
 #pragma unroll 1
       for (int hc = 0; hc < 2; ++hc) {
         const int c0 = 64 * hq + 32 * hc;   // first query column of the chunk
         uint32_t sv[32], dav[32];
         tmem_ld_32x32b_x32(tmem + lane_base + 128 * hq + 32 * hc, sv);
         tmem_ld_32x32b_x32(tmem + lane_base + 128 * hq + 64 + 32 * hc, dav);
-        uint32_t hb[16], bk[8];
+        uint32_t hb[16];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint4 w = *reinterpret_cast<const uint4*>(bt_row + (((4 * hc + q) ^ (rj & 7)) << 4));
           hb[4 * q] = w.x; hb[4 * q + 1] = w.y; hb[4 * q + 2] = w.z; hb[4 * q + 3] = w.w;
-        }
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const uint4 w = *reinterpret_cast<const uint4*>(bk_row + (((4 * hq + 2 * hc + q) ^ (rj & 7)) << 4));
-          bk[4 * q] = w.x; bk[4 * q + 1] = w.y; bk[4 * q + 2] = w.z; bk[4 * q + 3] = w.w;
         }
         tmem_ld_wait();
         // per query, in fp32: x = s + bias, sigma(x) = (1 + tanh(x/2)) / 2, P = SiLU(x) = x sigma,
@@ -381,7 +383,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         // MMA operand type. (A packed-fp16 evaluation of SiLU' quantises 1 - sigma near x = 8 and
         // biases the table-gradient sums.)
         uint32_t pp[16], dxp[16];
-        float xf[32];
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
           uint32_t m = 0xFFFFFFFFu;
@@ -408,8 +409,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             pp[e2] = pack_bf16x2(pv[0], pv[1]);
             dxp[e2] = pack_bf16x2(dv2[0], dv2[1]);
           }
-          xf[2 * e2] = dv2[0];     // the table gradients sum dX in fp32
-          xf[2 * e2 + 1] = dv2[1];
         }
         tmem_st_32x32b_x16(tmem + lane_base + 128 * hq + 16 * hc, pp);
         // dX^T replaces the half-bias just read: same row, same swizzled 16-byte units
@@ -417,51 +416,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int q = 0; q < 4; ++q)
           *reinterpret_cast<uint4*>(bt_row + (((4 * hc + q) ^ (rj & 7)) << 4)) =
               make_uint4(dxp[4 * q], dxp[4 * q + 1], dxp[4 * q + 2], dxp[4 * q + 3]);
-        // d rab_pos: the chunk is a 32x32 block (key rows 32 quad + l, query columns c0 + e); lane L
-        // gathers diagonal e - l = L from lane e - L and diagonal L - 32 from lane e - L + 32
-        {
-          float up = 0.0f, lo = 0.0f;
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float v = __shfl_sync(0xffffffffu, xf[e], (e - lane) & 31);
-            if (e >= lane) up += v;
-            else lo += v;
-          }
-          // window index of relative position r = 128 s + (c0 + d) - 32 quad, stored at r + 127
-          const int w_up = 128 * s + c0 - 32 * quad + 127 + lane;
-          const int w_lo = w_up - 32;
-          if (w_up < Lb::kPosWin) atomicAdd(s_dpos + w_up, up);
-          else atomicAdd(A.drab_pos + pos_index_b(w_up - 127, a.pos_max_len), up);
-          if (lane > 0) {
-            if (w_lo < Lb::kPosWin) atomicAdd(s_dpos + w_lo, lo);
-            else atomicAdd(A.drab_pos + pos_index_b(w_lo - 127, a.pos_max_len), lo);
-          }
-        }
-        // d rab_time: runs of equal bucket along the row (4 buckets per word)
-#pragma unroll
-        for (int wq = 0; wq < 8; ++wq) {
-          const uint32_t wd = bk[wq];
-          if (wd == cur_rep) {
-            acc_t += (xf[4 * wq] + xf[4 * wq + 1]) + (xf[4 * wq + 2] + xf[4 * wq + 3]);
-          } else {
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-              const int bkt = static_cast<int>((wd >> (8 * x)) & 0xFFu);
-              if (bkt != cur_b) {
-                if (acc_t != 0.0f) atomicAdd(s_dtime + cur_b * 32 + lane, acc_t);
-                acc_t = 0.0f;
-                cur_b = bkt;
-              }
-              acc_t += xf[4 * wq + x];
-            }
-            cur_rep = 0x01010101u * static_cast<uint32_t>(cur_b);
-          }
-        }
       }
       tmem_st_wait();
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(BAR(11 + hq));    // P^T_h in TMEM, dX^T_h in shared memory
+      mbar_arrive(BAR(15 + st));
     }
     if (ok && hq == 1 && nsteps > 0 && mbar_wait(BAR(13), (nsteps - 1) & 1, abort_flag, ctl)) {
       tc_fence_after();
@@ -486,7 +446,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
     }
-    if (acc_t != 0.0f) atomicAdd(s_dtime + cur_b * 32 + lane, acc_t);
   }
 
   tc_fence_before();
@@ -495,14 +454,136 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  for (int t = tid; t < a.n_buckets; t += kThreadsB) {
+}
+
+// ----------------------------------------------------------------------------------------------
+// table gradients from the per-head dX^T tiles
+// ----------------------------------------------------------------------------------------------
+// Two blocks per causal tile pair, 64 key rows each. Thread (warp w, lane l) holds the fp32 head
+// sum of key rows j_k = 64 y + 8 w + 2 k + l / 16 (k < 4), queries [c0, c0 + 8), c0 = 8 (l % 16).
+//  d rab_pos: element (j, i) of the tile lies on diagonal i - j + 127 (relative position
+//   128 (qt - kt) + i - j). A thread's 32 elements fall on 14 diagonals (e - 2k = const), summed in
+//   registers first; in each of the 14 steps the 32 lanes of a warp touch 32 distinct diagonals, so
+//   every warp adds into its own window without atomics. The 8 windows are summed and added to
+//   the table, one atomic per diagonal.
+//  d rab_time: each thread's elements in row-major order form runs of equal bucket (along a key
+//   row the bucket only grows when timestamps are sorted); a run is added to column l of a
+//   [bucket][lane] shared histogram, whose rows are then summed and added to the table.
+constexpr int kTgThreads = 256;
+
+template <bool F16>
+__global__ void __launch_bounds__(kTgThreads)
+attn_table_grad_kernel(AttnBwdArgs A) {
+  const AttnArgs& a = A.f;
+  int b, qt, kt;
+  if (!decode_tile_pair(blockIdx.x, a.pair_base, a.B, &b, &qt, &kt)) return;
+  __shared__ float s_win[8][256];
+  __shared__ float s_hist[128][32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int e = tid; e < 8 * 256; e += kTgThreads) (&s_win[0][0])[e] = 0.0f;
+  for (int e = tid; e < 128 * 32; e += kTgThreads) (&s_hist[0][0])[e] = 0.0f;
+  const int g = lane >> 4, c0 = 8 * (lane & 15);
+  const int j0 = 64 * static_cast<int>(blockIdx.y) + 8 * w + g;   // row of k = 0; row k is j0 + 2k
+  const long long pair = blockIdx.x;
+  const uint16_t* src = reinterpret_cast<const uint16_t*>(A.dxt) + pair * a.H * (kQTile * kQTile) +
+                        static_cast<long long>(j0) * kQTile + c0;
+  float acc[4][8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[k][e] = 0.0f;
+  auto add = [&](int k, const uint4& v) {
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float2 f;
+      if (F16) {
+        f = unpack_f16x2(u[q]);
+      } else {
+        f = make_float2(__uint_as_float(u[q] << 16), __uint_as_float(u[q] & 0xFFFF0000u));
+      }
+      acc[k][2 * q] += f.x;
+      acc[k][2 * q + 1] += f.y;
+    }
+  };
+  int h = 0;
+  for (; h + 2 <= a.H; h += 2) {
+    uint4 v0[4], v1[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v0[k] = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<long long>(h) * kQTile + 2 * k) * kQTile));
+      v1[k] = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<long long>(h + 1) * kQTile + 2 * k) * kQTile));
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      add(k, v0[k]);
+      add(k, v1[k]);
+    }
+  }
+  if (h < a.H) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      add(k, __ldg(reinterpret_cast<const uint4*>(src + (static_cast<long long>(h) * kQTile + 2 * k) * kQTile)));
+  }
+  // buckets of the same 32 elements
+  const uint8_t* bsrc = reinterpret_cast<const uint8_t*>(A.bucket_t) + pair * (kQTile * kQTile) +
+                        static_cast<long long>(j0) * kQTile + c0;
+  uint32_t bk[4][2];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(bsrc + 2 * k * kQTile));
+    bk[k][0] = v.x;
+    bk[k][1] = v.y;
+  }
+  __syncthreads();   // windows and histogram zeroed
+  // d rab_pos: diagonal of (k, e) is c0 - j0 + 127 + (e - 2k)
+  float pd[14];
+#pragma unroll
+  for (int m = 0; m < 14; ++m) pd[m] = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pd[e - 2 * k + 6] += acc[k][e];
+  const int dbase = c0 - j0 + 127 - 6;   // diagonal of slot 0, in [-6, 254 - 13]
+#pragma unroll
+  for (int m = 0; m < 14; ++m) {
+    const int d = dbase + m;
+    if (d >= 0 && d < 255) s_win[w][d] += pd[m];
+    __syncwarp();
+  }
+  // d rab_time: runs of equal bucket, in row-major order
+  {
+    int cur = static_cast<int>(bk[0][0] & 0x7Fu);
+    float run = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int bb = static_cast<int>((bk[k][e >> 2] >> (8 * (e & 3))) & 0x7Fu);   // buckets < 128
+        if (bb != cur) {
+          if (run != 0.0f) atomicAdd(&s_hist[cur][lane], run);
+          cur = bb;
+          run = 0.0f;
+        }
+        run += acc[k][e];
+      }
+    if (run != 0.0f) atomicAdd(&s_hist[cur][lane], run);
+  }
+  __syncthreads();
+  const int L = a.pos_max_len;
+  if (tid < 255) {
+    float v = 0.0f;
+#pragma unroll
+    for (int ww = 0; ww < 8; ++ww) v += s_win[ww][tid];
+    if (v != 0.0f)
+      atomicAdd(A.drab_pos + pos_index_b(static_cast<long long>(qt - kt) * kQTile + tid - 127, L), v);
+  }
+  if (tid < a.n_buckets) {
     float v = 0.0f;
 #pragma unroll 8
-    for (int l = 0; l < 32; ++l) v += s_dtime[t * 32 + ((l + t) & 31)];
-    if (v != 0.0f) atomicAdd(A.drab_time + t, v);
+    for (int l = 0; l < 32; ++l) v += s_hist[tid][(l + tid) & 31];
+    if (v != 0.0f) atomicAdd(A.drab_time + tid, v);
   }
-  for (int w = tid; w < pos_used; w += kThreadsB)
-    if (s_dpos[w] != 0.0f) atomicAdd(A.drab_pos + pos_index_b(w - 127, a.pos_max_len), s_dpos[w]);
 }
 
 }  // namespace
@@ -517,7 +598,9 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   attn_bias_t_kernel<<<dim3(static_cast<unsigned>(a.max_pairs), 4), 256, 0, st>>>(A);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap tq, tk, tv, tdo, tbt, tbk;
+  // TMA row coordinates of the bias and dX^T tiles are 32-bit
+  if (a.max_pairs * a.H * kQTile > 0x7fffffffLL) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv, tdo, tbt, tdx;
   const bool f16 = a.in_f16 != 0;
   const int64_t W = static_cast<int64_t>(a.H) * kD;
   if (!encode_tmap_2d_bf16(&tq, a.q, W, a.T, a.ld_q, 64, 128, f16) ||
@@ -525,14 +608,18 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
       !encode_tmap_2d_bf16(&tv, a.v, W, a.T, a.ld_v, 64, 128, f16) ||
       !encode_tmap_2d_bf16(&tdo, A.dout, W, a.T, A.ld_do, 64, 128, f16) ||
       !encode_tmap_2d_bf16(&tbt, A.bias_t, kQTile, a.max_pairs * kQTile, kQTile, 64, 128, true) ||
-      !encode_tmap_2d_u8(&tbk, A.bucket_t, kQTile, a.max_pairs * kQTile, kQTile, 128, 128))
+      !encode_tmap_2d_bf16(&tdx, A.dxt, kQTile, a.max_pairs * a.H * kQTile, kQTile, 64, 128, f16))
     return cudaErrorInvalidValue;
   auto kern = f16 ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), BwdSmem::kTotal);
   if (e != cudaSuccess) return e;
   const long long blocks = a.capacity * a.H;
-  kern<<<static_cast<unsigned>(blocks), kThreadsB, BwdSmem::kTotal, st>>>(tq, tk, tv, tdo, tbt, tbk, A,
+  kern<<<static_cast<unsigned>(blocks), kThreadsB, BwdSmem::kTotal, st>>>(tq, tk, tv, tdo, tbt, tdx, A,
                                                                           wait_ctl(a.status));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  auto tg = f16 ? attn_table_grad_kernel<true> : attn_table_grad_kernel<false>;
+  tg<<<dim3(static_cast<unsigned>(a.max_pairs), 2), kTgThreads, 0, st>>>(A);
   return cudaGetLastError();
 }
 

@@ -70,20 +70,23 @@ AttnWs attn_ws_layout(const hstu_jagged_t* j) {
 size_t attn_ws_bytes(const hstu_jagged_t* j) { return attn_ws_layout(j).total; }
 
 // attention-backward workspace: the forward layout up to pair_base, then the key-tile work list,
-// the transposed fp16 bias tiles (32 KB per pair) and the u8 bucket tiles (16 KB per pair).
+// the transposed fp16 bias tiles (32 KB per pair), the u8 bucket tiles (16 KB per pair) and the fp16
+// dX^T tiles of every (pair, head) (32 KB each) the table gradients are summed from.
 struct AttnBwdWs {
   AttnWs f;
-  size_t kitems, bias_t, bucket_t, total;
+  size_t kitems, bias_t, bucket_t, dxt, total;
 };
 
-AttnBwdWs attn_bwd_ws_layout(const hstu_jagged_t* j) {
+AttnBwdWs attn_bwd_ws_layout(const hstu_jagged_t* j, int H) {
   AttnBwdWs w{};
   w.f = attn_ws_layout(j);
   const int64_t cap = capacity_of(j);
+  const size_t tile = static_cast<size_t>(kQTile) * kQTile;
   w.kitems = w.f.bias;   // the forward bias region is not used by the backward
   w.bias_t = align_up(w.kitems + align_up(static_cast<size_t>(cap) * 8, 256), 1024);
-  w.bucket_t = w.bias_t + static_cast<size_t>(w.f.max_pairs) * kQTile * kQTile * 2;
-  w.total = w.bucket_t + static_cast<size_t>(w.f.max_pairs) * kQTile * kQTile;
+  w.bucket_t = w.bias_t + static_cast<size_t>(w.f.max_pairs) * tile * 2;
+  w.dxt = align_up(w.bucket_t + static_cast<size_t>(w.f.max_pairs) * tile, 1024);
+  w.total = w.dxt + static_cast<size_t>(w.f.max_pairs) * (H > 0 ? H : 0) * tile * 2;
   return w;
 }
 
@@ -97,7 +100,7 @@ struct LayerBwdWs {
 LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) {
   LayerBwdWs w{};
   const size_t T = static_cast<size_t>(j->T), D = static_cast<size_t>(d->D);
-  size_t off = align_up(attn_bwd_ws_layout(j).total, 1024);
+  size_t off = align_up(attn_bwd_ws_layout(j, d->H).total, 1024);
   auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes, 1024); return o; };
   w.dg = take(T * D * 4);
   w.dO = take(T * D * 2);
@@ -123,7 +126,7 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
                            const void* v, const void* d_out, const float* rab_pos, const float* rab_time, float* dq,
                            float* dk, float* dv, int64_t ld_g, float* d_rab_pos, float* d_rab_time, void* ws,
                            cudaStream_t st) {
-  const AttnBwdWs lay = attn_bwd_ws_layout(jag);
+  const AttnBwdWs lay = attn_bwd_ws_layout(jag, desc->H);
   cudaError_t e = cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (2 * static_cast<size_t>(desc->pos_max_len) - 1), st);
   if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, sizeof(float) * desc->n_time_buckets, st);
   if (e != cudaSuccess) return cuda_status(e);
@@ -148,7 +151,7 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
   A.dout = d_out; A.ld_do = desc->ld_o;
   A.dq = dq; A.dk = dk; A.dv = dv; A.ld_g = ld_g;
   A.drab_pos = d_rab_pos; A.drab_time = d_rab_time;
-  A.bias_t = w + lay.bias_t; A.bucket_t = w + lay.bucket_t;
+  A.bias_t = w + lay.bias_t; A.bucket_t = w + lay.bucket_t; A.dxt = w + lay.dxt;
   A.kitems = reinterpret_cast<int32_t*>(w + lay.kitems); A.kcount = kcount;
   e = launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, a.status, st,
                       reinterpret_cast<long long*>(w + lay.f.pairs), reinterpret_cast<int32_t*>(w + lay.kitems),
@@ -446,9 +449,8 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
 }
 
 size_t hstu_attn_bwd_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag) {
-  (void)desc;
-  if (check_jagged(jag) != HSTU_OK) return 0;
-  return attn_bwd_ws_layout(jag).total;
+  if (!desc || check_jagged(jag) != HSTU_OK) return 0;
+  return attn_bwd_ws_layout(jag, desc->H).total;
 }
 
 hstu_status_t hstu_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const void* q, const void* k,
@@ -459,7 +461,7 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
   if (s != HSTU_OK) return s;
   if (!is_tc_dtype(desc->dtype)) return HSTU_ERR_UNSUPPORTED;
   if (!ws) return HSTU_ERR_INVALID_ARG;
-  if (ws_bytes < attn_bwd_ws_layout(jag).total) return HSTU_ERR_WORKSPACE;
+  if (ws_bytes < attn_bwd_ws_layout(jag, desc->H).total) return HSTU_ERR_WORKSPACE;
   if (!d_rab_pos || !d_rab_time) return HSTU_ERR_INVALID_ARG;
   if (jag->T > 0) {
     if (!q || !k || !v || !d_out || !rab_pos || !rab_time || !dq || !dk || !dv) return HSTU_ERR_INVALID_ARG;

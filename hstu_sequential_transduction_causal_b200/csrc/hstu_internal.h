@@ -130,6 +130,7 @@ struct AttnBwdArgs {
   float* drab_pos; float* drab_time; // accumulated (must be zero on entry)
   void* bias_t;                // fp16 [max_pairs, 128 keys, 128 queries] half-bias, transposed
   void* bucket_t;              // u8   [max_pairs, 128 keys, 128 queries] time bucket, transposed
+  void* dxt;                   // fp16 [max_pairs, H, 128 keys, 128 queries] dX^T of every (pair, head)
   const int32_t* kitems;       // backward work list (b, key tile)
   const int32_t* kcount;
 };
