@@ -12,14 +12,15 @@
 // [key][query] and the u8 time-bucket tile [key][query] (head independent, computed once).
 // attn_bwd_tc_kernel<F16>: one CTA per (sequence, 128-key tile, head), key tiles that visit the
 // most query tiles first; it walks the query tiles t >= its key tile:
-//   warp 8   : TMA: K, V once; Q and dO of each query tile (2 stages); the half-bias tile.
-//   warp 9   : tcgen05: S^T = K Q^T and dA^T = V dO^T into TMEM; after the elementwise step
+//   warp 16  : TMA: K, V once; Q and dO of each query tile (2 stages); the half-bias tile.
+//   warp 17  : tcgen05: S^T = K Q^T and dA^T = V dO^T into TMEM; after the elementwise step
 //              dV += P^T dO (P^T from TMEM), dK += dX^T Q and dQ_tile = dX K (dX^T from shared
 //              memory, read K-major for dK and MN-major for dQ).
-//   warp 10  : TMA store of each tile's dX^T (16-bit, from shared memory) to the workspace.
-//   warps 0-7: key row = TMEM lane (warp & 3), query half (warp >> 2): x = s + bias,
-//              P^T = SiLU(x), dX^T = dA SiLU'(x) inv_N in fp32, causal and length masks;
-//              dQ_tile added to the fp32 dQ by vector atomics.
+//   warp 18  : TMA stores: each dQ tile (staged in shared memory) reduce-added into the fp32 dQ,
+//              each tile's dX^T (16-bit, from shared memory) to the workspace.
+//   warps 0-15: key row = TMEM lane (warp & 3), query half (warp >> 2) & 1, 32 of its 64 queries
+//              (warp >> 3): x = s + bias, P^T = SiLU(x), dX^T = dA SiLU'(x) inv_N in fp32, causal
+//              and length masks; the half-b warps also stage the previous tile's dQ.
 // attn_table_grad_kernel<F16>: per causal tile pair, sums the H heads' dX^T tiles and adds them to
 // d rab_pos (by diagonal) and d rab_time (by bucket): the tables are shared by the heads, so the
 // head sum comes first and each table entry takes one atomic per tile pair.
@@ -32,100 +33,26 @@
 #include "sm100_ptx.cuh"
 #include "tile_pairs.cuh"
 #include "time_bucket_dev.cuh"
+#include "bias_tile.cuh"
 
 namespace hstu {
 
 namespace {
 
 constexpr int kD = 64;
-constexpr int kSiluWarpsB = 8;
-constexpr int kThreadsB = 32 * (kSiluWarpsB + 3);   // + TMA producer, MMA issuer, dX^T store warp
+constexpr int kSiluWarpsB = 16;
+constexpr int kThreadsB = 32 * (kSiluWarpsB + 3);   // + TMA producer, MMA issuer, TMA store warp
 constexpr int kSiluThreadsB = 32 * kSiluWarpsB;
-
-__device__ __forceinline__ int pos_index_b(long long r, int L) {
-  r = r > L - 1 ? L - 1 : r;
-  r = r < -(L - 1) ? -(L - 1) : r;
-  return static_cast<int>(r) + L - 1;
-}
 
 // ----------------------------------------------------------------------------------------------
 // transposed bias and bucket tiles
 // ----------------------------------------------------------------------------------------------
-// Four blocks per causal tile pair, 32 key rows each. Thread t writes 8 consecutive queries
-// [8 (t % 16), +8) of key rows 32 y + t / 16 + 16 p, p = 0, 1: 16-byte half-bias and 8-byte bucket
-// stores. Differences within a tile that fit in int32 take 32-bit bucket arithmetic.
-__global__ void __launch_bounds__(256)
+// One block per causal tile pair: the [key][query] half-bias and u8 bucket tiles of bias_tile.cuh.
+__global__ void __launch_bounds__(kBiasThreads)
 attn_bias_t_kernel(AttnBwdArgs A) {
-  const AttnArgs& a = A.f;
-  int b, qt, kt;
-  if (!decode_tile_pair(blockIdx.x, a.pair_base, a.B, &b, &qt, &kt)) return;
-  const long long seq0 = a.offsets[b];
-  const int n = static_cast<int>(a.offsets[b + 1] - seq0);
-  __shared__ long long s_qts[128], s_kts[128], s_tau[kTauEntries], s_red[16];
-  __shared__ int s_tau32[kTauEntries];
-  __shared__ float s_win[256], s_rt[128];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int L = a.pos_max_len;
-  const int nb = a.n_buckets;
-  long long t;
-  if (tid < 128) {
-    const int qi = qt * kQTile + tid;
-    t = a.ts[seq0 + (qi < n ? qi : n - 1)];
-    s_qts[tid] = t;
-  } else {
-    const int kj = kt * kQTile + tid - 128;
-    t = a.ts[seq0 + (kj < n ? kj : n - 1)];
-    s_kts[tid - 128] = t;
-  }
-  if (tid < nb) s_rt[tid] = 0.5f * a.rab_time[tid];
-  if (tid < 255) s_win[tid] = 0.5f * a.rab_pos[pos_index_b(static_cast<long long>(qt - kt) * kQTile - 127 + tid, L)];
-  for (int e = tid; e < kTauEntries; e += 256) {
-    s_tau[e] = c_time_taus[e];
-    s_tau32[e] = c_time_taus32[e];
-  }
-  long long mn = t, mx = t;
-#pragma unroll
-  for (int d = 16; d > 0; d >>= 1) {
-    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, d));
-    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-  }
-  if (lane == 0) {
-    s_red[warp] = mn;
-    s_red[8 + warp] = mx;
-  }
-  __syncthreads();
-  long long lo = s_red[0], hi = s_red[8];
-#pragma unroll
-  for (int w = 1; w < 8; ++w) {
-    lo = min(lo, s_red[w]);
-    hi = max(hi, s_red[8 + w]);
-  }
-  const bool fast = hi - lo < 0x7fffffffLL;
-  const int c0 = 8 * (tid & 15);
   const long long tile0 = blockIdx.x * static_cast<long long>(kQTile * kQTile);
-  uint16_t* tile = reinterpret_cast<uint16_t*>(A.bias_t) + tile0;
-  uint8_t* btile = reinterpret_cast<uint8_t*>(A.bucket_t) + tile0;
-#pragma unroll
-  for (int pass = 0; pass < 2; ++pass) {
-    const int j = 32 * blockIdx.y + (tid >> 4) + 16 * pass;   // key row within the tile
-    uint32_t w[4], bw[2] = {0u, 0u};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float v2[2];
-#pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        const int col = c0 + 2 * e + x;     // query column
-        const int bkt = fast ? time_bucket32(static_cast<int>(s_qts[col] - lo) - static_cast<int>(s_kts[j] - lo),
-                                             s_tau32, nb)
-                             : time_bucket_dev(s_qts[col] - s_kts[j], s_tau, nb);
-        v2[x] = s_win[col - j + 127] + s_rt[bkt];
-        bw[e >> 1] |= static_cast<uint32_t>(bkt) << (8 * (2 * (e & 1) + x));
-      }
-      w[e] = pack_f16x2(v2[0], v2[1]);
-    }
-    *reinterpret_cast<uint4*>(tile + j * kQTile + c0) = make_uint4(w[0], w[1], w[2], w[3]);
-    *reinterpret_cast<uint2*>(btile + j * kQTile + c0) = make_uint2(bw[0], bw[1]);
-  }
+  bias_tile_block<true, true>(A.f, blockIdx.x, reinterpret_cast<uint16_t*>(A.bias_t) + tile0,
+                              reinterpret_cast<uint8_t*>(A.bucket_t) + tile0);
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -134,9 +61,10 @@ attn_bias_t_kernel(AttnBwdArgs A) {
 struct BwdSmem {
   static constexpr int kK = 0;                  // K tile of the CTA (16 KB)
   static constexpr int kV = 16384;              // V tile (16 KB)
-  static constexpr int kQ0 = 32768;             // stage st: Q at kQ0 + st * 32768, dO at +16384
-  static constexpr int kBT0 = kQ0 + 2 * 32768;  // stage st: half-bias^T, overwritten in place by dX^T
-  static constexpr int kBar = kBT0 + 2 * 32768;
+  static constexpr int kQ0 = 32768;             // stage st (of 3): Q at kQ0 + st * 32768, dO at +16384
+  static constexpr int kBT0 = kQ0 + 3 * 32768;  // stage st (of 2): half-bias^T, overwritten in place by dX^T
+  static constexpr int kDQ = kBT0 + 2 * 32768;  // dQ tile staging for the TMA reduce-add: 2 x [128][32] fp32
+  static constexpr int kBar = kDQ + 32768;
   static constexpr int kTotal = kBar + 256 + 1024;
 };
 static_assert(BwdSmem::kTotal <= 232448, "shared memory of the backward kernel");
@@ -146,7 +74,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                    const __grid_constant__ CUtensorMap tmBT, const __grid_constant__ CUtensorMap tmDX,
-                   AttnBwdArgs A, WaitCtl ctl) {
+                   const __grid_constant__ CUtensorMap tmDQ, AttnBwdArgs A, WaitCtl ctl) {
   using Lb = BwdSmem;
   const AttnArgs& a = A.f;
   extern __shared__ uint8_t smem_raw[];
@@ -164,11 +92,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lb::kBar);
   // 0 kv_full | 1,2 qdo_full | 3,4 qdo_empty | 5,6 bb_full | 7,8 bb_empty | 9,10 s_full (query half
-  // a, b) | 11,12 p_ready (half a, b) | 13 dq_full | 14 fin | 15,16 dx_full (stage)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  // a, b) | 11,12 p_ready (half a, b) | 13 dq_full | 14 fin | 15,16 dx_full (stage) | 17 dq_staged |
+  // 18 dq_stage_free | 19,20 p_free (half a, b: the dV MMA has read P^T_h) | 21 qdo_full, 22 qdo_empty
+  // of the third Q/dO stage
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  auto qdo_full = [&](int sq) { return sq < 2 ? BAR(1 + sq) : BAR(21); };
+  auto qdo_empty = [&](int sq) { return sq < 2 ? BAR(3 + sq) : BAR(22); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -183,12 +115,17 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(BAR(7 + s), 2);   // bias/dX stage free: the MMAs read dX^T and the store warp sent it
       mbar_init(BAR(15 + s), kSiluThreadsB);   // both query halves of dX^T written
     }
-    for (int h = 0; h < 2; ++h) {
-      mbar_init(BAR(9 + h), 1);
-      mbar_init(BAR(11 + h), kSiluThreadsB / 2);
+    for (int hh = 0; hh < 2; ++hh) {
+      mbar_init(BAR(9 + hh), 1);
+      mbar_init(BAR(11 + hh), kSiluThreadsB / 2);
+      mbar_init(BAR(19 + hh), 1);
     }
     mbar_init(BAR(13), 1);
     mbar_init(BAR(14), 1);
+    mbar_init(BAR(21), 1);
+    mbar_init(BAR(22), 1);
+    mbar_init(BAR(17), kSiluThreadsB / 2);     // the half-b warps staged a dQ tile
+    mbar_init(BAR(18), 1);                     // the store warp's reduce-add has read the staging
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -199,6 +136,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tma_prefetch_desc(&tmDO);
     tma_prefetch_desc(&tmBT);
     tma_prefetch_desc(&tmDX);
+    tma_prefetch_desc(&tmDQ);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -208,13 +146,15 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // query half h: S^T_h at columns [128 h, 128 h + 64) (P^T_h packed over its first 32), dA^T_h at
-  // [128 h + 64, 128 h + 128); accumulators dV, dK and the dQ tile of one query tile
-  const uint32_t tDV = tmem + 256, tDK = tmem + 320, tDQ = tmem + 384;
+  // query half h: S^T_h at columns [128 h, 128 h + 64), dA^T_h at [128 h + 64, 128 h + 128);
+  // accumulators dV, dK and the dQ tile of one query tile; P^T_h packed two per column at
+  // [448 + 32 h, 448 + 32 h + 32)
+  const uint32_t tDV = tmem + 256, tDK = tmem + 320, tDQ = tmem + 384, tP = tmem + 448;
 
   const uint32_t sK = smem_u32(smem + Lb::kK), sV = smem_u32(smem + Lb::kV);
   const uint32_t sQ0 = smem_u32(smem + Lb::kQ0);
   const uint32_t sBT0 = smem_u32(smem + Lb::kBT0);
+  const uint32_t sDQ = smem_u32(smem + Lb::kDQ);
   const int krow = static_cast<int>(seq0) + kt * kQTile;
 
   if (warp == kSiluWarpsB) {
@@ -223,91 +163,117 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_arrive_expect_tx(BAR(0), 32768);
       tma_load_2d(sK, &tmK, BAR(0), h * kD, krow);
       tma_load_2d(sV, &tmV, BAR(0), h * kD, krow);
-      for (int s = 0; s < nsteps; ++s) {
-        const int qt = kt + s, st = s & 1;
-        const uint32_t ph_free = ((s >> 1) & 1) ^ 1;
-        if (s >= 2 && !mbar_wait(BAR(3 + st), ph_free, abort_flag, ctl)) break;
-        const int qrow = static_cast<int>(seq0) + qt * kQTile;
-        mbar_arrive_expect_tx(BAR(1 + st), 32768);
-        tma_load_2d(sQ0 + st * 32768, &tmQ, BAR(1 + st), h * kD, qrow);
-        tma_load_2d(sQ0 + st * 32768 + 16384, &tmDO, BAR(1 + st), h * kD, qrow);
-        if (s >= 2 && !mbar_wait(BAR(7 + st), ph_free, abort_flag, ctl)) break;
+      // Q and dO of tile s (3 stages) run one tile ahead of its bias (2 stages): waiting for a bias
+      // stage never delays the next Q / dO load
+      auto load_bias = [&](int s) -> bool {
+        const int st = s & 1, qt = kt + s;
+        if (s >= 2 && !mbar_wait(BAR(7 + st), ((s >> 1) & 1) ^ 1, abort_flag, ctl)) return false;
         const int prow = static_cast<int>((pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt) * kQTile);
         mbar_arrive_expect_tx(BAR(5 + st), 32768);
         tma_load_2d(sBT0 + st * 32768, &tmBT, BAR(5 + st), 0, prow);
         tma_load_2d(sBT0 + st * 32768 + 16384, &tmBT, BAR(5 + st), 64, prow);
+        return true;
+      };
+      bool ok = true;
+      for (int s = 0; ok && s < nsteps; ++s) {
+        const int qt = kt + s, sq = s % 3;
+        if (s >= 3 && !mbar_wait(qdo_empty(sq), ((s / 3) & 1) ^ 1, abort_flag, ctl)) break;
+        const int qrow = static_cast<int>(seq0) + qt * kQTile;
+        mbar_arrive_expect_tx(qdo_full(sq), 32768);
+        tma_load_2d(sQ0 + sq * 32768, &tmQ, qdo_full(sq), h * kD, qrow);
+        tma_load_2d(sQ0 + sq * 32768 + 16384, &tmDO, qdo_full(sq), h * kD, qrow);
+        if (s >= 1) ok = load_bias(s - 1);
       }
+      if (ok && nsteps > 0) load_bias(nsteps - 1);
     }
   } else if (warp == kSiluWarpsB + 1) {
     // ---------------- tcgen05 issuer ----------------
     // Per query tile s, in two halves of 64 queries: S^T_h = K Q_h^T and dA^T_h = V dO_h^T, then,
     // once the elementwise warps of half h have written P^T_h (TMEM) and dX^T_h (shared memory),
-    // dV += P^T_h dO_h and dK += dX^T_h Q_h; after half b also dQ_tile = dX K. The next tile's half a
-    // is issued between the two halves, so each half's elementwise work overlaps MMAs.
+    // dV += P^T_h dO_h and dK += dX^T_h Q_h; after half b also dQ_tile = dX K. P^T has TMEM columns
+    // of its own, so the next tile's S^T_h, dA^T_h go first, as soon as half h has read this tile's:
+    // the elementwise warps of half h start the next tile while the gradient MMAs run.
     if (lane == 0) {
       constexpr uint32_t id_s = make_idesc_f16kind(128, 64, 0, 0, F16);
       constexpr uint32_t id_kmn = make_idesc_f16kind(128, 64, 0, 1, F16);
       constexpr uint32_t id_mnmn = make_idesc_f16kind(128, 64, 1, 1, F16);
       bool ok = mbar_wait(BAR(0), 0, abort_flag, ctl);
-      auto issue_s = [&](int s, int h) -> bool {
-        const int st = s & 1;
-        if (h == 0 && !mbar_wait(BAR(1 + st), (s >> 1) & 1, abort_flag, ctl)) return false;
+      // base descriptors: K-major (lbo 16) and MN-major (lbo 16384, the 64-element block stride)
+      const uint64_t k_km = make_sdesc_sw128(sK, 16, 1024), v_km = make_sdesc_sw128(sV, 16, 1024);
+      const uint64_t k_mn = make_sdesc_sw128(sK, 16384, 1024);
+      const uint64_t q_km = make_sdesc_sw128(sQ0, 16, 1024), q_mn = make_sdesc_sw128(sQ0, 16384, 1024);
+      const uint64_t x_km = make_sdesc_sw128(sBT0, 16, 1024), x_mn = make_sdesc_sw128(sBT0, 16384, 1024);
+      auto issue_s = [&](int s, int hh) -> bool {
+        const int sq = s % 3;
+        if (hh == 0 && !mbar_wait(qdo_full(sq), (s / 3) & 1, abort_flag, ctl)) return false;
         tc_fence_after();
-        const uint32_t sQ = sQ0 + st * 32768 + 8192 * h, sDO = sQ0 + st * 32768 + 16384 + 8192 * h;
+        const uint64_t qd = sdesc_add(q_km, sq * 32768 + 8192 * hh), dod = sdesc_add(qd, 16384);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_f16_ss(tmem + 128 * h, make_sdesc_sw128(sK + kk * 32, 16, 1024),
-                      make_sdesc_sw128(sQ + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + 128 * hh, sdesc_add(k_km, kk * 32), sdesc_add(qd, kk * 32), id_s, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_f16_ss(tmem + 128 * h + 64, make_sdesc_sw128(sV + kk * 32, 16, 1024),
-                      make_sdesc_sw128(sDO + kk * 32, 16, 1024), id_s, kk > 0 ? 1u : 0u);
-        umma_commit(BAR(9 + h));
+          umma_f16_ss(tmem + 128 * hh + 64, sdesc_add(v_km, kk * 32), sdesc_add(dod, kk * 32), id_s,
+                      kk > 0 ? 1u : 0u);
+        umma_commit(BAR(9 + hh));
         return true;
       };
-      auto issue_grad = [&](int s, int h) -> bool {
-        if (!mbar_wait(BAR(11 + h), s & 1, abort_flag, ctl)) return false;
-        tc_fence_after();
-        const int st = s & 1;
-        const uint32_t sQ = sQ0 + st * 32768, sDO = sQ + 16384, sDX = sBT0 + st * 32768;
+      auto issue_grad = [&](int s, int hh) {
+        const int st = s & 1, sq = s % 3;
+        const uint64_t qd = sdesc_add(q_mn, sq * 32768 + hh * 8192), dod = sdesc_add(qd, 16384);
+        const uint64_t xd = sdesc_add(x_km, st * 32768 + hh * 16384);
+        const uint32_t acc0 = (s > 0 || hh > 0) ? 1u : 0u;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4)   // dV += P^T_h dO_h
-          umma_f16_ts(tDV, tmem + 128 * h + 8 * k4, make_sdesc_sw128(sDO + (4 * h + k4) * 2048, 16384, 1024),
-                      id_kmn, (s > 0 || h > 0 || k4 > 0) ? 1u : 0u);
+          umma_f16_ts(tDV, tP + 32 * hh + 8 * k4, sdesc_add(dod, k4 * 2048), id_kmn, k4 > 0 ? 1u : acc0);
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4)   // dK += dX^T_h Q_h
-          umma_f16_ss(tDK, make_sdesc_sw128(sDX + h * 16384 + k4 * 32, 16, 1024),
-                      make_sdesc_sw128(sQ + (4 * h + k4) * 2048, 16384, 1024), id_kmn,
-                      (s > 0 || h > 0 || k4 > 0) ? 1u : 0u);
-        return true;
+          umma_f16_ss(tDK, sdesc_add(xd, k4 * 32), sdesc_add(qd, k4 * 2048), id_kmn, k4 > 0 ? 1u : acc0);
+        umma_commit(BAR(19 + hh));
       };
       if (ok && nsteps > 0) ok = issue_s(0, 0) && issue_s(0, 1);
       for (int s = 0; ok && s < nsteps; ++s) {
         const int st = s & 1;
-        if (!issue_grad(s, 0) || (s + 1 < nsteps && !issue_s(s + 1, 0)) || !issue_grad(s, 1)) {
-          ok = false;
-          break;
+        for (int hh = 0; ok && hh < 2; ++hh) {
+          ok = mbar_wait(BAR(11 + hh), s & 1, abort_flag, ctl) && (s + 1 >= nsteps || issue_s(s + 1, hh));
+          if (ok) {
+            tc_fence_after();
+            issue_grad(s, hh);
+          }
         }
-        const uint32_t sDX = sBT0 + st * 32768;
+        if (!ok) break;
+        const uint64_t xd = sdesc_add(x_mn, st * 32768);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)   // dQ_tile = dX K
-          umma_f16_ss(tDQ, make_sdesc_sw128(sDX + kk * 2048, 16384, 1024),
-                      make_sdesc_sw128(sK + kk * 2048, 16384, 1024), id_mnmn, kk > 0 ? 1u : 0u);
+          umma_f16_ss(tDQ, sdesc_add(xd, kk * 2048), sdesc_add(k_mn, kk * 2048), id_mnmn, kk > 0 ? 1u : 0u);
         umma_commit(BAR(13));
-        umma_commit(BAR(3 + st));
+        umma_commit(qdo_empty(s % 3));
         umma_commit(BAR(7 + st));
-        if (s + 1 < nsteps && !issue_s(s + 1, 1)) { ok = false; break; }
       }
       if (ok) umma_commit(BAR(14));
     }
   } else if (warp == kSiluWarpsB + 2) {
-    // ---------------- dX^T store ----------------
-    // Once both query halves of tile s are done, dX^T (the fp16 operand of dK and dQ, in the stage's
-    // bias slot) goes to the workspace; the table gradients are summed from there over the heads.
+    // ---------------- TMA stores ----------------
+    // dQ tile j (staged in shared memory by the half-b warps) is added to the fp32 dQ with one
+    // TMA reduce-add per 32 columns; once both query halves of tile s are done, dX^T (the 16-bit
+    // operand of dK and dQ, in the stage's bias slot) goes to the workspace, from which the table
+    // gradients are summed over the heads.
     if (lane == 0) {
-      for (int s = 0; s < nsteps; ++s) {
+      auto reduce_dq = [&](int j) -> bool {
+        if (!mbar_wait(BAR(17), j & 1, abort_flag, ctl)) return false;
+        const int y = static_cast<int>(seq0) + (kt + j) * kQTile;
+        tma_reduce_add_2d(&tmDQ, sDQ, h * kD, y);
+        tma_reduce_add_2d(&tmDQ, sDQ + 16384, h * kD + 32, y);
+        bulk_commit_group();
+        bulk_wait_group_read<0>();
+        mbar_arrive(BAR(18));
+        return true;
+      };
+      bool ok = true;
+      for (int s = 0; ok && s < nsteps; ++s) {
         const int st = s & 1;
-        if (!mbar_wait(BAR(15 + st), (s >> 1) & 1, abort_flag, ctl)) break;
+        if (s >= 1 && !reduce_dq(s - 1)) { ok = false; break; }
+        if (!mbar_wait(BAR(15 + st), (s >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
         const int qt = kt + s;
         const long long pair = pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt;
         const int y = static_cast<int>((pair * a.H + h) * kQTile);
@@ -317,31 +283,72 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         bulk_wait_group_read<0>();
         mbar_arrive(BAR(7 + st));
       }
+      if (ok && nsteps > 0) reduce_dq(nsteps - 1);
       bulk_wait_group_all();
     }
   } else {
     // ---------------- elementwise warps ----------------
+    // warp w: key rows [32 (w & 3), +32) (TMEM lane quadrant), query half hq = (w >> 2) & 1,
+    // queries [64 hq + 32 sub, +32) with sub = w >> 3
     const int quad = warp & 3;
-    const int hq = warp >> 2;             // queries [64 hq, 64 hq + 64)
+    const int hq = (warp >> 2) & 1;
+    const int sub = warp >> 3;
     const int rj = quad * 32 + lane;      // key row == TMEM lane of S^T, dA^T, dV, dK
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const bool key_ok = kt * kQTile + rj < n;
     const float inv_N = a.inv_N;
+    const float cN = 0.5f * inv_N;
     bool ok = true;
-    auto flush_dq = [&](int s_prev) {
-      // (half-b warps) dQ tile of query tile kt + s_prev: TMEM lane = query row, all 64 columns
-      const int qi = (kt + s_prev) * kQTile + quad * 32 + lane;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tDQ + lane_base + 32 * c, v);
-        tmem_ld_wait();
-        if (qi < n) {
-          float4* dst = reinterpret_cast<float4*>(A.dq + (seq0 + qi) * A.ld_g + h * kD + 32 * c);
+    // (half-b warps) dQ tile j: TMEM lane = query row, columns [32 sub, +32) staged as box sub of
+    // the reduce-add, 128-byte swizzled rows
+    auto stage_dq = [&](int j) -> bool {
+      if (!mbar_wait(BAR(13), j & 1, abort_flag, ctl)) return false;
+      if (j >= 1 && !mbar_wait(BAR(18), (j - 1) & 1, abort_flag, ctl)) return false;
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tDQ + lane_base + 32 * sub, v);
+      tmem_ld_wait();
+      uint8_t* row = smem + Lb::kDQ + sub * 16384 + rj * 128;
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            atomicAdd(dst + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                           __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+      for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4*>(row + ((u ^ (rj & 7)) << 4)) = make_uint4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(17));
+      return true;
+    };
+    // one 16-query piece: x = s + bias, sigma(x) = (1 + tanh(x/2)) / 2, P = SiLU(x) = x sigma,
+    // dX = dA inv_N SiLU'(x) = dA (inv_N sigma + P inv_N (1 - sigma)), all in fp32; P and dX are
+    // rounded once to the MMA operand type. (A packed-fp16 evaluation of SiLU' quantises 1 - sigma
+    // near x = 8 and biases the table-gradient sums.)
+    auto piece = [&](const uint32_t (&sv)[16], const uint32_t (&dav)[16], const uint32_t* hb, uint32_t* pp,
+                     uint32_t* dxp, bool masked, int col0, int lo_col, int hi_col) {
+#pragma unroll
+      for (int e2 = 0; e2 < 8; ++e2) {
+        const float2 hbf = unpack_f16x2(hb[e2]);
+        float pv[2], dv2[2];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const float hx = fmaf(__uint_as_float(sv[2 * e2 + x]), 0.5f, x ? hbf.y : hbf.x);
+          const float t = tanh_f32_approx(hx);
+          const float av = fmaf(hx, t, hx);
+          const float sgN = fmaf(cN, t, cN);
+          const float w = fmaf(av, inv_N - sgN, sgN);
+          float dxv = __uint_as_float(dav[2 * e2 + x]) * w;
+          float pvv = av;
+          if (masked) {
+            const int col = col0 + 2 * e2 + x;
+            const bool keep = col >= lo_col && col < hi_col;
+            pvv = keep ? pvv : 0.0f;
+            dxv = keep ? dxv : 0.0f;
+          }
+          pv[x] = pvv;
+          dv2[x] = dxv;
+        }
+        if (F16) {
+          pp[e2] = pack_f16x2(pv[0], pv[1]);
+          dxp[e2] = pack_f16x2(dv2[0], dv2[1]);
+        } else {   // the MMAs take A and B of one type: P and dX as bf16 next to bf16 dO, Q, K
+          pp[e2] = pack_bf16x2(pv[0], pv[1]);
+          dxp[e2] = pack_bf16x2(dv2[0], dv2[1]);
         }
       }
     };
@@ -352,93 +359,65 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         ok = false;
         break;
       }
-      // half b starts after the MMAs of the previous tile's dQ: flushing it here costs no wait
-      if (hq == 1 && s >= 1) {
-        if (!mbar_wait(BAR(13), (s - 1) & 1, abort_flag, ctl)) { ok = false; break; }
-        tc_fence_after();
-        flush_dq(s - 1);
-      }
       tc_fence_after();
       // masks: the diagonal tile keeps queries >= key; the last query tile keeps queries < n; a key
       // row past n keeps nothing (it only occurs in the diagonal tile of the last key tile)
       const bool need_mask = (s == 0) || (qt == nt - 1);
       const int lo_col = (s == 0) ? rj : 0;
-      const int hi_col = key_ok ? min(kQTile, n - qt * kQTile) : 0;
+      const int hi_col = (kt * kQTile + rj < n) ? min(kQTile, n - qt * kQTile) : 0;
       uint8_t* bt_row = smem + Lb::kBT0 + st * 32768 + hq * 16384 + rj * 128;
-#pragma unroll 1
-      for (int hc = 0; hc < 2; ++hc) {
-        const int c0 = 64 * hq + 32 * hc;   // first query column of the chunk
-        uint32_t sv[32], dav[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + 128 * hq + 32 * hc, sv);
-        tmem_ld_32x32b_x32(tmem + lane_base + 128 * hq + 64 + 32 * hc, dav);
-        uint32_t hb[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 w = *reinterpret_cast<const uint4*>(bt_row + (((4 * hc + q) ^ (rj & 7)) << 4));
+      for (int pc = 0; pc < 2; ++pc) {
+        const int c0 = 64 * hq + 32 * sub + 16 * pc;   // first query column of the piece
+        uint32_t sv[16], dav[16];
+        tmem_ld_32x32b_x16(tmem + lane_base + 128 * hq + 32 * sub + 16 * pc, sv);
+        tmem_ld_32x32b_x16(tmem + lane_base + 128 * hq + 64 + 32 * sub + 16 * pc, dav);
+        const int u0 = 4 * sub + 2 * pc;   // first 16-byte unit of the piece in the bias row
+        uint32_t hb[8];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const uint4 w = *reinterpret_cast<const uint4*>(bt_row + (((u0 + q) ^ (rj & 7)) << 4));
           hb[4 * q] = w.x; hb[4 * q + 1] = w.y; hb[4 * q + 2] = w.z; hb[4 * q + 3] = w.w;
         }
         tmem_ld_wait();
-        // per query, in fp32: x = s + bias, sigma(x) = (1 + tanh(x/2)) / 2, P = SiLU(x) = x sigma,
-        // dX = dA inv_N SiLU'(x) with SiLU' = sigma + P (1 - sigma); P and dX are rounded once to the
-        // MMA operand type. (A packed-fp16 evaluation of SiLU' quantises 1 - sigma near x = 8 and
-        // biases the table-gradient sums.)
-        uint32_t pp[16], dxp[16];
-#pragma unroll
-        for (int e2 = 0; e2 < 16; ++e2) {
-          uint32_t m = 0xFFFFFFFFu;
-          if (need_mask) {
-            const int col = c0 + 2 * e2;
-            m = ((col >= lo_col && col < hi_col) ? 0x0000FFFFu : 0u) |
-                ((col + 1 >= lo_col && col + 1 < hi_col) ? 0xFFFF0000u : 0u);
-          }
-          const float2 hbf = unpack_f16x2(hb[e2]);
-          float pv[2], dv2[2];
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            const float xs = __uint_as_float(sv[2 * e2 + x]) + 2.0f * (x ? hbf.y : hbf.x);
-            const float sg = fmaf(0.5f, tanh_f32_approx(0.5f * xs), 0.5f);
-            const float av = xs * sg;
-            const bool keep = (m >> (16 * x)) & 1u;
-            pv[x] = keep ? av : 0.0f;
-            dv2[x] = keep ? __uint_as_float(dav[2 * e2 + x]) * inv_N * fmaf(av, 1.0f - sg, sg) : 0.0f;
-          }
-          if (F16) {
-            pp[e2] = pack_f16x2(pv[0], pv[1]);
-            dxp[e2] = pack_f16x2(dv2[0], dv2[1]);
-          } else {   // the MMAs take A and B of one type: P and dX as bf16 next to bf16 dO, Q, K
-            pp[e2] = pack_bf16x2(pv[0], pv[1]);
-            dxp[e2] = pack_bf16x2(dv2[0], dv2[1]);
-          }
+        uint32_t pp[8], dxp[8];
+        if (need_mask) piece(sv, dav, hb, pp, dxp, true, c0, lo_col, hi_col);
+        else piece(sv, dav, hb, pp, dxp, false, c0, lo_col, hi_col);
+        if (pc == 0 && s >= 1) {   // the previous tile's dV MMA has read P^T_h
+          if (!mbar_wait(BAR(19 + hq), (s - 1) & 1, abort_flag, ctl)) { ok = false; break; }
+          tc_fence_after();
         }
-        tmem_st_32x32b_x16(tmem + lane_base + 128 * hq + 16 * hc, pp);
+        tmem_st_32x32b_x8(tP + lane_base + 32 * hq + 16 * sub + 8 * pc, pp);
         // dX^T replaces the half-bias just read: same row, same swizzled 16-byte units
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(bt_row + (((4 * hc + q) ^ (rj & 7)) << 4)) =
+        for (int q = 0; q < 2; ++q)
+          *reinterpret_cast<uint4*>(bt_row + (((u0 + q) ^ (rj & 7)) << 4)) =
               make_uint4(dxp[4 * q], dxp[4 * q + 1], dxp[4 * q + 2], dxp[4 * q + 3]);
       }
+      if (!ok) break;
+      // (half b) the previous tile's dQ: its MMAs were issued after this tile's S^T_b
+      if (hq == 1 && s >= 1 && !stage_dq(s - 1)) { ok = false; break; }
       tmem_st_wait();
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(BAR(11 + hq));    // P^T_h in TMEM, dX^T_h in shared memory
       mbar_arrive(BAR(15 + st));
     }
-    if (ok && hq == 1 && nsteps > 0 && mbar_wait(BAR(13), (nsteps - 1) & 1, abort_flag, ctl)) {
-      tc_fence_after();
-      flush_dq(nsteps - 1);
-    }
+    if (ok && hq == 1 && nsteps > 0 && !stage_dq(nsteps - 1)) ok = false;
     if (ok && mbar_wait(BAR(14), 0, abort_flag, ctl)) {
       tc_fence_after();
-      uint32_t vk[32], vv[32];
-      tmem_ld_32x32b_x32(tDK + lane_base + 32 * hq, vk);
-      tmem_ld_32x32b_x32(tDV + lane_base + 32 * hq, vv);
+      // dK, dV: key row = TMEM lane, columns [16 (2 hq + sub), +16)
+      const int cc = 16 * (2 * hq + sub);
+      uint32_t vk[16], vv[16];
+      tmem_ld_32x32b_x16(tDK + lane_base + cc, vk);
+      tmem_ld_32x32b_x16(tDV + lane_base + cc, vv);
       tmem_ld_wait();
-      if (key_ok) {
+      if (kt * kQTile + rj < n) {
         const long long row = seq0 + kt * kQTile + rj;
-        float4* dk = reinterpret_cast<float4*>(A.dk + row * A.ld_g + h * kD + 32 * hq);
-        float4* dvp = reinterpret_cast<float4*>(A.dv + row * A.ld_g + h * kD + 32 * hq);
+        float4* dk = reinterpret_cast<float4*>(A.dk + row * A.ld_g + h * kD + cc);
+        float4* dvp = reinterpret_cast<float4*>(A.dv + row * A.ld_g + h * kD + cc);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < 4; ++q) {
           dk[q] = make_float4(__uint_as_float(vk[4 * q]), __uint_as_float(vk[4 * q + 1]),
                               __uint_as_float(vk[4 * q + 2]), __uint_as_float(vk[4 * q + 3]));
           dvp[q] = make_float4(__uint_as_float(vv[4 * q]) * inv_N, __uint_as_float(vv[4 * q + 1]) * inv_N,
@@ -576,7 +555,7 @@ attn_table_grad_kernel(AttnBwdArgs A) {
 #pragma unroll
     for (int ww = 0; ww < 8; ++ww) v += s_win[ww][tid];
     if (v != 0.0f)
-      atomicAdd(A.drab_pos + pos_index_b(static_cast<long long>(qt - kt) * kQTile + tid - 127, L), v);
+      atomicAdd(A.drab_pos + bias_pos_index(static_cast<long long>(qt - kt) * kQTile + tid - 127, L), v);
   }
   if (tid < a.n_buckets) {
     float v = 0.0f;
@@ -595,12 +574,12 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  attn_bias_t_kernel<<<dim3(static_cast<unsigned>(a.max_pairs), 4), 256, 0, st>>>(A);
+  attn_bias_t_kernel<<<static_cast<unsigned>(a.max_pairs), kBiasThreads, 0, st>>>(A);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // TMA row coordinates of the bias and dX^T tiles are 32-bit
   if (a.max_pairs * a.H * kQTile > 0x7fffffffLL) return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv, tdo, tbt, tdx;
+  CUtensorMap tq, tk, tv, tdo, tbt, tdx, tdq;
   const bool f16 = a.in_f16 != 0;
   const int64_t W = static_cast<int64_t>(a.H) * kD;
   if (!encode_tmap_2d_bf16(&tq, a.q, W, a.T, a.ld_q, 64, 128, f16) ||
@@ -608,13 +587,14 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
       !encode_tmap_2d_bf16(&tv, a.v, W, a.T, a.ld_v, 64, 128, f16) ||
       !encode_tmap_2d_bf16(&tdo, A.dout, W, a.T, A.ld_do, 64, 128, f16) ||
       !encode_tmap_2d_bf16(&tbt, A.bias_t, kQTile, a.max_pairs * kQTile, kQTile, 64, 128, true) ||
-      !encode_tmap_2d_bf16(&tdx, A.dxt, kQTile, a.max_pairs * a.H * kQTile, kQTile, 64, 128, f16))
+      !encode_tmap_2d_bf16(&tdx, A.dxt, kQTile, a.max_pairs * a.H * kQTile, kQTile, 64, 128, f16) ||
+      !encode_tmap_2d_out(&tdq, A.dq, kDtF32, W, a.T, A.ld_g, 32, 128))
     return cudaErrorInvalidValue;
   auto kern = f16 ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), BwdSmem::kTotal);
   if (e != cudaSuccess) return e;
   const long long blocks = a.capacity * a.H;
-  kern<<<static_cast<unsigned>(blocks), kThreadsB, BwdSmem::kTotal, st>>>(tq, tk, tv, tdo, tbt, tdx, A,
+  kern<<<static_cast<unsigned>(blocks), kThreadsB, BwdSmem::kTotal, st>>>(tq, tk, tv, tdo, tbt, tdx, tdq, A,
                                                                           wait_ctl(a.status));
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

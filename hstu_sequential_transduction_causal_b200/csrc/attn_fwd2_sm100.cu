@@ -13,11 +13,17 @@
 //     instead of once per pair and head; buckets are exact integer evaluations.
 //  2. attn_fwd_tc2_kernel<F16, G>: one CTA per (sequence, 128-row query tile, group of G heads),
 //     longest causal rows first; only key tiles 0..t of the tile's own sequence are visited.
-//       warp 8   : TMA producer: Q of the G heads once; per key tile the bias tile (2 stages);
-//                  per (key tile, head) K and V (3 stages); all 128-byte swizzled.
-//       warp 9   : tcgen05 issuer: S = Q K^T into one of two TMEM tiles; then O_h += P V with the
-//                  A operand P read from TMEM (P overwrites the S tile it came from).
-//       warps 0-7: TMEM lane quadrant (warp & 3), key half (warp >> 2). Per element, in packed
+//       K/V warp : TMA producer: Q of the G heads once; per (key tile, head) K and V in separate
+//                  rings: a K stage is free once its S MMA has run and a V stage once its P V MMA
+//                  has, so K loads run several tiles ahead of the (later) V loads and TMA latency
+//                  stays hidden; all 128-byte swizzled.
+//       bias warp: TMA producer of the bias tiles (one per key tile), so that waiting for a bias
+//                  stage (freed by the SiLU warps) never delays a K or V load.
+//       MMA warp : tcgen05 issuer: S = Q K^T into one of three TMEM tiles; O_h += P V two units
+//                  later, with the A operand P read from TMEM (P overwrites the S tile it came
+//                  from), so the S MMAs of the next units never wait for a P V MMA.
+//       SiLU warps (8 per group, NG groups, numbered first; then the K/V, MMA and bias warps):
+//                  TMEM lane quadrant (warp & 3), key half (warp >> 2) & 1. Per element, in packed
 //                  fp16: h = 0.5 s + 0.5 bias, P = h + h tanh(h) = SiLU(s + bias); causal mask on
 //                  the diagonal tile only; P back into TMEM.
 //     1/N is applied to the fp32 accumulator in the epilogue; O is written in fp32 (or bf16).
@@ -31,124 +37,27 @@
 #include "sm100_ptx.cuh"
 #include "tile_pairs.cuh"
 #include "time_bucket_dev.cuh"
+#include "bias_tile.cuh"
 
 namespace hstu {
 
 namespace {
 
 constexpr int kD = 64;
-constexpr int kNS = 3;                 // K/V stages
 constexpr int kSiluWarps = 8;     // one group of SiLU warps: 4 TMEM lane quadrants x 2 key halves
-__host__ __device__ constexpr int threads2(int ng) { return 32 * (kSiluWarps * ng + 2); }
+__host__ __device__ constexpr int threads2(int ng) { return 32 * (kSiluWarps * ng + 3); }
 constexpr uint32_t kHalf2Half = 0x38003800u;   // (0.5, 0.5) in fp16
-
-__device__ __forceinline__ int pos_index2(long long r, int L) {
-  r = r > L - 1 ? L - 1 : r;
-  r = r < -(L - 1) ? -(L - 1) : r;
-  return static_cast<int>(r) + L - 1;
-}
 
 // ----------------------------------------------------------------------------------------------
 // 1. bias tiles
 // ----------------------------------------------------------------------------------------------
-// Stages a tile pair's query and key timestamps (q_ts, k_ts: 128 each, clamped to the sequence),
-// the rab_pos window of its diagonals and rab_time, both pre-halved, and the bucket thresholds; returns
-// through lo / fast whether every difference of the tile fits in int32 (then offsets from lo are used).
-__device__ __forceinline__ void stage_tile_pair(const AttnArgs& a, long long seq0, int n, int qt, int kt,
-                                                long long* s_qts, long long* s_kts, float* s_win, float* s_rt,
-                                                long long* s_tau, int* s_tau32, long long* s_red, long long& lo,
-                                                bool& fast) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  long long t;
-  if (tid < 128) {
-    const int qi = qt * kQTile + tid;
-    t = a.ts[seq0 + (qi < n ? qi : n - 1)];
-    s_qts[tid] = t;
-  } else {
-    const int kj = kt * kQTile + tid - 128;
-    t = a.ts[seq0 + (kj < n ? kj : n - 1)];
-    s_kts[tid - 128] = t;
-  }
-  if (tid < a.n_buckets) s_rt[tid] = 0.5f * a.rab_time[tid];
-  if (tid < 255) s_win[tid] = 0.5f * a.rab_pos[pos_index2(static_cast<long long>(qt - kt) * kQTile - 127 + tid,
-                                                          a.pos_max_len)];
-  for (int e = tid; e < kTauEntries; e += 256) {
-    s_tau[e] = c_time_taus[e];
-    s_tau32[e] = c_time_taus32[e];
-  }
-  long long mn = t, mx = t;
-#pragma unroll
-  for (int d = 16; d > 0; d >>= 1) {
-    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, d));
-    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-  }
-  if (lane == 0) {
-    s_red[warp] = mn;
-    s_red[8 + warp] = mx;
-  }
-  __syncthreads();
-  long long bmn = s_red[0], bmx = s_red[8];
-#pragma unroll
-  for (int w = 1; w < 8; ++w) {
-    bmn = min(bmn, s_red[w]);
-    bmx = max(bmx, s_red[8 + w]);
-  }
-  lo = bmn;
-  fast = bmx - bmn < 0x7fffffffLL;
-}
-
-// Four blocks per causal tile pair, 32 query rows each (blocks past the batch's last pair exit at
-// once). Thread t writes 8 consecutive keys [8 (t % 16), +8) of rows 32 y + t / 16 + 16 p, p = 0, 1:
-// 16-byte coalesced stores.
-__global__ void __launch_bounds__(256)
+// One block per causal tile pair (blocks past the batch's last pair exit at once): the [query][key]
+// half-bias tile of bias_tile.cuh.
+__global__ void __launch_bounds__(kBiasThreads)
 attn_bias_kernel(AttnArgs a) {
-  int b, qt, kt;
-  if (!decode_tile_pair(blockIdx.x, a.pair_base, a.B, &b, &qt, &kt)) return;
-  const long long seq0 = a.offsets[b];
-  const int n = static_cast<int>(a.offsets[b + 1] - seq0);
-  __shared__ long long s_qts[128], s_kts[128], s_tau[kTauEntries], s_red[16];
-  __shared__ int s_tau32[kTauEntries];
-  __shared__ float s_win[256], s_rt[128];
-  long long lo;
-  bool fast;
-  stage_tile_pair(a, seq0, n, qt, kt, s_qts, s_kts, s_win, s_rt, s_tau, s_tau32, s_red, lo, fast);
-  const int tid = threadIdx.x;
-  const int nb = a.n_buckets;
-  const int c0 = 8 * (tid & 15);
-  uint16_t* tile = reinterpret_cast<uint16_t*>(a.bias) + blockIdx.x * static_cast<long long>(kQTile * kQTile);
-#pragma unroll
-  for (int pass = 0; pass < 2; ++pass) {
-    const int r = 32 * blockIdx.y + (tid >> 4) + 16 * pass;   // query row within the tile
-    uint32_t w[4];
-    if (fast) {
-      const int ti = static_cast<int>(s_qts[r] - lo);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v2[2];
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const int col = c0 + 2 * e + x;
-          const int bkt = time_bucket32(ti - static_cast<int>(s_kts[col] - lo), s_tau32, nb);
-          v2[x] = s_win[r - col + 127] + s_rt[bkt];
-        }
-        w[e] = pack_f16x2(v2[0], v2[1]);
-      }
-    } else {
-      const long long t_i = s_qts[r];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v2[2];
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const int col = c0 + 2 * e + x;
-          const int bkt = time_bucket_dev(t_i - s_kts[col], s_tau, nb);
-          v2[x] = s_win[r - col + 127] + s_rt[bkt];
-        }
-        w[e] = pack_f16x2(v2[0], v2[1]);
-      }
-    }
-    *reinterpret_cast<uint4*>(tile + r * kQTile + c0) = make_uint4(w[0], w[1], w[2], w[3]);
-  }
+  bias_tile_block<false, false>(a, blockIdx.x,
+                                reinterpret_cast<uint16_t*>(a.bias) + blockIdx.x * static_cast<long long>(kQTile * kQTile),
+                                nullptr);
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -157,12 +66,16 @@ attn_bias_kernel(AttnArgs a) {
 template <int G>
 struct Smem2 {
   static constexpr int kBS = G == 1 ? 3 : 2;   // bias stages (one head per CTA: a bias tile per unit)
+  static constexpr int kNK = G == 1 ? 4 : 3;   // K stages (16 KB)
+  static constexpr int kNV = 3;                // V stages (16 KB)
   static constexpr int kQ = 0;
-  static constexpr int kKV = G * 16384;
-  static constexpr int kBias = kKV + kNS * 32768;
+  static constexpr int kK = G * 16384;
+  static constexpr int kV = kK + kNK * 16384;
+  static constexpr int kBias = kV + kNV * 16384;
   static constexpr int kBar = kBias + kBS * 32768;
   static constexpr int kTotal = kBar + 256 + 1024;
 };
+static_assert(Smem2<1>::kTotal <= 232448 && Smem2<2>::kTotal <= 232448, "shared memory of the attention kernel");
 
 // NG = 2 (one head per CTA only): two groups of SiLU warps take alternate key tiles, so one group's
 // SiLU of tile t overlaps the other's of tile t + 1 (each group owns one S buffer and one bias stage).
@@ -173,7 +86,7 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     WaitCtl ctl) {
   using L = Smem2<G>;
   static_assert(NG == 1 || G == 1, "two SiLU groups need one head per CTA");
-  constexpr int kTmaWarp = kSiluWarps * NG, kMmaWarp = kTmaWarp + 1;
+  constexpr int kTmaWarp = kSiluWarps * NG, kMmaWarp = kTmaWarp + 1, kBiasWarp = kTmaWarp + 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int HG = a.H / G;
@@ -198,21 +111,26 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const int nsteps = nkt * G;
   const long long pair0 = FALCON ? 0 : a.pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2;
 
-  constexpr int BS = L::kBS;
+  constexpr int BS = L::kBS, NK = L::kNK, NV = L::kNV;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  // 0 q_full | 1..3 kv_full | 4..6 kv_empty | b_full [BS] | b_empty [BS] | s_full [2] | p_full [2] |
-  // o_full
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12 + 2 * BS);
+  // 0 q_full | k_full [NK] | k_empty [NK] | v_full [NV] | v_empty [NV] | b_full [BS] | b_empty [BS] |
+  // s_full [3] | p_full [3] | o_full
+  constexpr int kBarK = 1, kBarV = kBarK + 2 * NK, kBarB = kBarV + 2 * NV, kBarS = kBarB + 2 * BS;
+  constexpr int kBarP = kBarS + 3, kBarO = kBarP + 3, kNumBars = kBarO + 1;
+  static_assert(kNumBars * 8 + 8 <= 256, "barrier region");
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  const uint32_t bar_q = BAR(0), bar_o = BAR(11 + 2 * BS);
-  auto bar_kv_full = [&](int s) { return BAR(1 + s); };
-  auto bar_kv_empty = [&](int s) { return BAR(4 + s); };
-  auto bar_b_full = [&](int s) { return BAR(7 + s); };
-  auto bar_b_empty = [&](int s) { return BAR(7 + BS + s); };
-  auto bar_s_full = [&](int s) { return BAR(7 + 2 * BS + s); };
-  auto bar_p_full = [&](int s) { return BAR(9 + 2 * BS + s); };
+  const uint32_t bar_q = BAR(0), bar_o = BAR(kBarO);
+  auto bar_k_full = [&](int s) { return BAR(kBarK + s); };
+  auto bar_k_empty = [&](int s) { return BAR(kBarK + NK + s); };
+  auto bar_v_full = [&](int s) { return BAR(kBarV + s); };
+  auto bar_v_empty = [&](int s) { return BAR(kBarV + NV + s); };
+  auto bar_b_full = [&](int s) { return BAR(kBarB + s); };
+  auto bar_b_empty = [&](int s) { return BAR(kBarB + BS + s); };
+  auto bar_s_full = [&](int s) { return BAR(kBarS + s); };
+  auto bar_p_full = [&](int s) { return BAR(kBarP + s); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -220,15 +138,19 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < kNS; ++s) {
-      mbar_init(bar_kv_full(s), 1);
-      mbar_init(bar_kv_empty(s), 1);
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(bar_k_full(s), 1);
+      mbar_init(bar_k_empty(s), 1);
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(bar_v_full(s), 1);
+      mbar_init(bar_v_empty(s), 1);
     }
     for (int s = 0; s < BS; ++s) {
       mbar_init(bar_b_full(s), 1);
       mbar_init(bar_b_empty(s), kSiluThreads);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 3; ++s) {
       mbar_init(bar_s_full(s), 1);
       mbar_init(bar_p_full(s), kSiluThreads);
     }
@@ -249,10 +171,13 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;    // S0 cols [0,128), S1 [128,256), O_h [256 + 64h, +64)
+  // S / P tiles of units s = 0, 1, 2 (mod 3) at columns [128 (s % 3), +128): with three of them the S
+  // MMA of unit s is issued before the P V MMA of unit s - 2; O_h at [384 + 64 h, +64)
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t kOCol = 384;
 
   const uint32_t sQ = smem_u32(smem + L::kQ);
-  const uint32_t sKV = smem_u32(smem + L::kKV);
+  const uint32_t sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
   const uint32_t sB = smem_u32(smem + L::kBias);
   const int qrow0 = FALCON ? b * a.cand_rows + qt * kQTile : static_cast<int>(seq0) + qt * kQTile;
 
@@ -261,28 +186,37 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_q, G * 16384);
       for (int h = 0; h < G; ++h) tma_load_2d(sQ + h * 16384, &tmQ, bar_q, (hg * G + h) * kD, qrow0);
+      // unit s = (key tile s / G, head s % G): K(s) first, V(s - 1) after it, so waiting for a V
+      // stage (freed late, by a P V MMA) never delays a K load
+      auto load_v = [&](int s) -> bool {
+        const int st = s % NV;
+        if (s >= NV && !mbar_wait(bar_v_empty(st), ((s / NV) - 1) & 1, abort_flag, ctl)) return false;
+        mbar_arrive_expect_tx(bar_v_full(st), 16384);
+        tma_load_2d(sV + st * 16384, &tmV, bar_v_full(st), (hg * G + s % G) * kD,
+                    static_cast<int>(seq0) + (s / G) * kQTile);
+        return true;
+      };
       bool ok = true;
-      int s = 0;
-      for (int kt = 0; ok && kt < nkt; ++kt) {
-        if constexpr (!FALCON) {
-          const int bs = kt % BS;
-          if (kt >= BS && !mbar_wait(bar_b_empty(bs), ((kt / BS) - 1) & 1, abort_flag, ctl)) break;
-          const int brow = static_cast<int>((pair0 + kt) * kQTile);
-          mbar_arrive_expect_tx(bar_b_full(bs), 32768);
-          tma_load_2d(sB + bs * 32768, &tmB, bar_b_full(bs), 0, brow);
-          tma_load_2d(sB + bs * 32768 + 16384, &tmB, bar_b_full(bs), 64, brow);
-        }
-        const int krow = static_cast<int>(seq0) + kt * kQTile;
-        for (int h = 0; h < G; ++h, ++s) {
-          const int st = s % kNS;
-          if (s >= kNS && !mbar_wait(bar_kv_empty(st), ((s / kNS) - 1) & 1, abort_flag, ctl)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar_kv_full(st), 32768);
-          tma_load_2d(sKV + st * 32768, &tmK, bar_kv_full(st), (hg * G + h) * kD, krow);
-          tma_load_2d(sKV + st * 32768 + 16384, &tmV, bar_kv_full(st), (hg * G + h) * kD, krow);
-        }
+      for (int s = 0; ok && s < nsteps; ++s) {
+        const int kt = s / G, h = s % G;
+        const int st = s % NK;
+        if (s >= NK && !mbar_wait(bar_k_empty(st), ((s / NK) - 1) & 1, abort_flag, ctl)) break;
+        mbar_arrive_expect_tx(bar_k_full(st), 16384);
+        tma_load_2d(sK + st * 16384, &tmK, bar_k_full(st), (hg * G + h) * kD, static_cast<int>(seq0) + kt * kQTile);
+        if (s >= 1) ok = load_v(s - 1);
+      }
+      if (ok && nsteps > 0) load_v(nsteps - 1);
+    }
+  } else if (warp == kBiasWarp) {
+    // ---------------- bias tiles ----------------
+    if (!FALCON && lane == 0) {
+      for (int kt = 0; kt < nkt; ++kt) {
+        const int bs = kt % BS;
+        if (kt >= BS && !mbar_wait(bar_b_empty(bs), ((kt / BS) - 1) & 1, abort_flag, ctl)) break;
+        const int brow = static_cast<int>((pair0 + kt) * kQTile);
+        mbar_arrive_expect_tx(bar_b_full(bs), 32768);
+        tma_load_2d(sB + bs * 32768, &tmB, bar_b_full(bs), 0, brow);
+        tma_load_2d(sB + bs * 32768 + 16384, &tmB, bar_b_full(bs), 64, brow);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -291,34 +225,61 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       constexpr uint32_t idesc_qk = make_idesc_f16kind(128, 128, 0, 0, F16);
       constexpr uint32_t idesc_pv = make_idesc_f16kind(128, 64, 0, 1, F16);
       bool ok = mbar_wait(bar_q, 0, abort_flag, ctl);
-      auto issue_pv = [&](int t) -> bool {
-        const int buf = t & 1, st = t % kNS, h = t % G;
-        if (!mbar_wait(bar_p_full(buf), (t >> 1) & 1, abort_flag, ctl)) return false;
+      const uint64_t q_desc0 = make_sdesc_sw128(sQ, 16, 1024), k_desc0 = make_sdesc_sw128(sK, 16, 1024);
+      const uint64_t v_desc0 = make_sdesc_sw128(sV, 16384, 1024);
+      auto issue_s = [&](int s) {
+        const int buf = s % 3, st = s % NK, h = s % G;
         tc_fence_after();
-        const uint32_t v = sKV + st * 32768 + 16384;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t a_tmem = tmem + buf * 128 + 64 * (kk >> 2) + 8 * (kk & 3);
-          umma_f16_ts(tmem + 256 + 64 * h, a_tmem, make_sdesc_sw128(v + kk * 2048, 16384, 1024), idesc_pv,
-                      (t >= G || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(bar_kv_empty(st));
-        return true;
-      };
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int buf = s & 1, st = s % kNS, h = s % G;
-        if (!mbar_wait(bar_kv_full(st), (s / kNS) & 1, abort_flag, ctl)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kb = sKV + st * 32768;
-        const uint32_t qb = sQ + h * 16384;
+        const uint64_t qd = sdesc_add(q_desc0, h * 16384), kd = sdesc_add(k_desc0, st * 16384);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_f16_ss(tmem + buf * 128, make_sdesc_sw128(qb + kk * 32, 16, 1024),
-                      make_sdesc_sw128(kb + kk * 32, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          umma_f16_ss(tmem + buf * 128, sdesc_add(qd, kk * 32), sdesc_add(kd, kk * 32), idesc_qk, kk > 0 ? 1u : 0u);
         umma_commit(bar_s_full(buf));
-        if (s >= 1 && !issue_pv(s - 1)) { ok = false; break; }
+        umma_commit(bar_k_empty(st));
+      };
+      auto issue_pv = [&](int t) {
+        const int buf = t % 3, st = t % NV, h = t % G;
+        tc_fence_after();
+        const uint64_t vd = sdesc_add(v_desc0, st * 16384);
+        const uint32_t a_tmem = tmem + buf * 128, o_tmem = tmem + kOCol + 64 * h;
+        const uint32_t acc0 = t >= G ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_ts(o_tmem, a_tmem + 64 * (kk >> 2) + 8 * (kk & 3), sdesc_add(vd, kk * 2048), idesc_pv,
+                      kk > 0 ? 1u : acc0);
+        umma_commit(bar_v_empty(st));
+      };
+      // S of unit sn goes first whenever its K tile has landed and its TMEM tile is free (the P V of
+      // unit sn - 3 has been issued: MMAs run in issue order); otherwise P V of unit tn once its P
+      // and V are ready. Neither waits for the other, so the next units' S overlaps this unit's
+      // SiLU. Polling is bounded like every wait: no progress for ctl.limit cycles aborts.
+      int sn = 0, tn = 0;
+      unsigned long long t_prog = clock64();
+      uint32_t idle = 0;
+      while (ok && tn < nsteps) {
+        bool progressed = false;
+        if (sn < nsteps && sn - tn < 3 && mbar_test(bar_k_full(sn % NK), (sn / NK) & 1)) {
+          issue_s(sn++);
+          progressed = true;
+        } else if (tn < sn && mbar_test(bar_p_full(tn % 3), (tn / 3) & 1) &&
+                   mbar_test(bar_v_full(tn % NV), (tn / NV) & 1)) {
+          issue_pv(tn++);
+          progressed = true;
+        }
+        if (progressed) {
+          t_prog = clock64();
+          idle = 0;
+        } else if ((++idle & 15u) == 0u) {
+          if (*abort_flag) {
+            ok = false;
+          } else if (clock64() - t_prog > ctl.limit) {
+            *abort_flag = 1;
+            report_error(ctl.status, kDevTimeout);
+            ok = false;
+          }
+        }
       }
-      if (ok && nsteps > 0 && issue_pv(nsteps - 1)) umma_commit(bar_o);
+      if (ok && nsteps > 0) umma_commit(bar_o);
     }
   } else {
     // ---------------- SiLU warps ----------------
@@ -339,8 +300,8 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       const bool diag = FALCON ? key_lim < kQTile : (kt == qt);
       for (int h = 0; h < G; ++h) {
         const int s = kt * G + h;
-        const int buf = s & 1;
-        if (!mbar_wait(bar_s_full(buf), (s >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
+        const int buf = s % 3;
+        if (!mbar_wait(bar_s_full(buf), (s / 3) & 1, abort_flag, ctl)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int hc = 0; hc < 2; ++hc) {
@@ -435,7 +396,7 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         for (int cc = 0; cc < kCols; cc += 32) {
           uint32_t ov[32];
           if (nkt > 0) {
-            tmem_ld_32x32b_x32(tmem + lane_base + 256 + 64 * h + col0 + cc, ov);
+            tmem_ld_32x32b_x32(tmem + lane_base + kOCol + 64 * h + col0 + cc, ov);
             tmem_ld_wait();
           } else {
 #pragma unroll
@@ -513,7 +474,7 @@ falcon_key_bias_kernel(const int64_t* __restrict__ off, const int64_t* __restric
     float v = 0.0f;
     if (j < n) {
       const int bkt = time_bucket_dev(treq - ts[s0 + j], s_tau, nb);
-      v = 0.5f * (rab_pos[pos_index2(n - j, L)] + rab_time[bkt]);
+      v = 0.5f * (rab_pos[bias_pos_index(n - j, L)] + rab_time[bkt]);
     }
     kbias[u * ld + j] = __half_as_ushort(__float2half_rn(v));
   }
@@ -546,7 +507,7 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  attn_bias_kernel<<<dim3(static_cast<unsigned>(a.max_pairs), 4), 256, 0, st>>>(a);
+  attn_bias_kernel<<<static_cast<unsigned>(a.max_pairs), kBiasThreads, 0, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv, tb;

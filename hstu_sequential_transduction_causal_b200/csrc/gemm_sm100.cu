@@ -218,6 +218,10 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
   } else if (warp == kEpiWarps + 1) {
     if (lane == 0) {
+      // descriptors of stage 0's A and B tiles; stages and K steps are offsets from them
+      const uint32_t sa0 = smem_u32(smem), sb0 = sa0 + L::kABytes;
+      const uint64_t a_desc0 = A_MN ? make_sdesc_sw128(sa0, 8192, 1024) : make_sdesc_sw128(sa0, 16, 1024);
+      const uint64_t b_desc0 = B_MN ? make_sdesc_sw128(sb0, 8192, 1024) : make_sdesc_sw128(sb0, 16, 1024);
       int g = 0, it = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < P.total; t += gridDim.x, ++it) {
@@ -231,16 +235,12 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           const int s = g % STAGES;
           if (!mbar_wait(smem_u32(&bars[s]), (g / STAGES) & 1, abort_flag, ctl)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
-          const uint32_t sb = sa + L::kABytes;
+          const uint64_t ad0 = sdesc_add(a_desc0, s * L::kStageBytes);
+          const uint64_t bd0 = sdesc_add(b_desc0, s * L::kStageBytes);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = A_MN ? make_sdesc_sw128(sa + kk * 2048, 8192, 1024)
-                                     : make_sdesc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bd = B_MN ? make_sdesc_sw128(sb + kk * 2048, 8192, 1024)
-                                     : make_sdesc_sw128(sb + kk * 32, 16, 1024);
-            umma_f16_ss(acc, ad, bd, P.idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_f16_ss(acc, sdesc_add(ad0, A_MN ? kk * 2048 : kk * 32), sdesc_add(bd0, B_MN ? kk * 2048 : kk * 32),
+                        P.idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
           umma_commit(smem_u32(&bars[STAGES + s]));
         }
         if (ok) umma_commit(acc_full(buf));
