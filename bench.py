@@ -268,6 +268,14 @@ def main():
     grads = H.layer_grads(*views)
     weights = layer.weights()
     flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():
+        """Evicts the step's data from the 126 MB L2: a 512 MB write, then a 256 MB read so that the
+        lines left behind are clean (the step does not pay the flush's own write-backs)."""
+        flush.zero_()
+        torch.sum(flush_rd, dim=0, out=flush_sink)
     # kernels of ours per step (cross-checked against the ncu launch list in profiles/)
     # f1 GEMM | work list, bias tiles, attention | LN-gate | fp16 W2 copy, f2 GEMM
     n_fwd_kernels = 7
@@ -303,7 +311,7 @@ def main():
     clk.__enter__()
     try:
         for _ in range(args.warmup):
-            flush.zero_()
+            flush_l2()
             step()
         torch.cuda.synchronize()
         if H.hstu_sync_status(ws) != 0:
@@ -313,7 +321,7 @@ def main():
         n_eager = min(args.steps, 20)
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n_eager)]
         for i in range(n_eager):
-            flush.zero_()
+            flush_l2()
             step(evs[i])
         torch.cuda.synchronize()
         seg = np.array([[e[k].elapsed_time(e[k + 1]) for k in range(nev - 1)] for e in evs])   # ms
@@ -326,7 +334,7 @@ def main():
         with torch.cuda.graph(attn_graph):
             attention_forward()
         for _ in range(3):
-            flush.zero_()
+            flush_l2()
             graph.replay()
             attn_graph.replay()
         torch.cuda.synchronize()
@@ -337,7 +345,7 @@ def main():
         torch.cuda.synchronize()
         t_start = time.time()
         for i in range(args.steps):
-            flush.zero_()
+            flush_l2()
             e_step[i][0].record(stream)
             graph.replay()
             if world > 1 and backward:
@@ -349,7 +357,7 @@ def main():
         n_attn = 20
         e_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_attn)]
         for i in range(n_attn):
-            flush.zero_()
+            flush_l2()
             e_attn[i][0].record(stream)
             attn_graph.replay()
             e_attn[i][1].record(stream)
@@ -400,7 +408,7 @@ def main():
     e2e_ms = 0.0
     n_e2e = max(10, args.steps // 4)
     for _ in range(n_e2e):
-        flush.zero_()
+        flush_l2()
         e0.record(stream)
         e2e_step()
         e1.record(stream)
@@ -429,7 +437,7 @@ def main():
             "config": {"workload": WORKLOADS[args.workload]["desc"], "global_batch": wl.B * world,
                        "tokens_per_rank": T, "seq_len": "jagged", "parallelism": f"dp{world}",
                        "attention_operands": "fp16 U|V|Q|K, P and G, fp32 accumulation and O",
-                       "l2": "flushed (512 MB write) before every timed step"},
+                       "l2": "flushed before every timed step (512 MB written, then 256 MB read)"},
             "roofline": {"bound": "tensor", "kernel": "jagged attention forward (bias tiles + attn_fwd_tc2_kernel)",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_kind": f"{peak_kind} bf16 sustained (dense)", "traffic": traffic_record(args.workload),

@@ -13,9 +13,9 @@
 // attn_bwd_tc_kernel<F16>: one CTA per (sequence, 128-key tile, head), key tiles that visit the
 // most query tiles first; it walks the query tiles t >= its key tile:
 //   warp 16  : TMA: K, V once; Q and dO of each query tile (2 stages); the half-bias tile.
-//   warp 17  : tcgen05: S^T = K Q^T and dA^T = V dO^T into TMEM; after the elementwise step
-//              dV += P^T dO (P^T from TMEM), dK += dX^T Q and dQ_tile = dX K (dX^T from shared
-//              memory, read K-major for dK and MN-major for dQ).
+//   warp 17  : tcgen05: S^T = K Q^T and dA^T = V dO^T into TMEM.
+//   warp 19  : tcgen05: after the elementwise step dV += P^T dO (P^T from TMEM), dK += dX^T Q and
+//              dQ_tile = dX K (dX^T from shared memory, read K-major for dK and MN-major for dQ).
 //   warp 18  : TMA stores: each dQ tile (staged in shared memory) reduce-added into the fp32 dQ,
 //              each tile's dX^T (16-bit, from shared memory) to the workspace.
 //   warps 0-15: key row = TMEM lane (warp & 3), query half (warp >> 2) & 1, 32 of its 64 queries
@@ -41,7 +41,7 @@ namespace {
 
 constexpr int kD = 64;
 constexpr int kSiluWarpsB = 16;
-constexpr int kThreadsB = 32 * (kSiluWarpsB + 3);   // + TMA producer, MMA issuer, TMA store warp
+constexpr int kThreadsB = 32 * (kSiluWarpsB + 4);   // + TMA producer, 2 MMA issuers, TMA store warp
 constexpr int kSiluThreadsB = 32 * kSiluWarpsB;
 
 // ----------------------------------------------------------------------------------------------
@@ -50,6 +50,7 @@ constexpr int kSiluThreadsB = 32 * kSiluWarpsB;
 // One block per causal tile pair: the [key][query] half-bias and u8 bucket tiles of bias_tile.cuh.
 __global__ void __launch_bounds__(kBiasThreads)
 attn_bias_t_kernel(AttnBwdArgs A) {
+  pdl_enter();
   const long long tile0 = blockIdx.x * static_cast<long long>(kQTile * kQTile);
   bias_tile_block<true, true>(A.f, blockIdx.x, reinterpret_cast<uint16_t*>(A.bias_t) + tile0,
                               reinterpret_cast<uint8_t*>(A.bucket_t) + tile0);
@@ -75,6 +76,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                    const __grid_constant__ CUtensorMap tmBT, const __grid_constant__ CUtensorMap tmDX,
                    const __grid_constant__ CUtensorMap tmDQ, AttnBwdArgs A, WaitCtl ctl) {
+  pdl_enter();
   using Lb = BwdSmem;
   const AttnArgs& a = A.f;
   extern __shared__ uint8_t smem_raw[];
@@ -110,7 +112,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     mbar_init(BAR(0), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(1 + s), 1);
-      mbar_init(BAR(3 + s), 1);
+      mbar_init(BAR(3 + s), 2);   // Q/dO stage free: both MMA issuers are done with it
       mbar_init(BAR(5 + s), 1);
       mbar_init(BAR(7 + s), 2);   // bias/dX stage free: the MMAs read dX^T and the store warp sent it
       mbar_init(BAR(15 + s), kSiluThreadsB);   // both query halves of dX^T written
@@ -123,7 +125,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     mbar_init(BAR(13), 1);
     mbar_init(BAR(14), 1);
     mbar_init(BAR(21), 1);
-    mbar_init(BAR(22), 1);
+    mbar_init(BAR(22), 2);
     mbar_init(BAR(17), kSiluThreadsB / 2);     // the half-b warps staged a dQ tile
     mbar_init(BAR(18), 1);                     // the store warp's reduce-add has read the staging
     *abort_flag = 0;
@@ -158,41 +160,45 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const int krow = static_cast<int>(seq0) + kt * kQTile;
 
   if (warp == kSiluWarpsB) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      mbar_arrive_expect_tx(BAR(0), 32768);
-      tma_load_2d(sK, &tmK, BAR(0), h * kD, krow);
-      tma_load_2d(sV, &tmV, BAR(0), h * kD, krow);
-      // Q and dO of tile s (3 stages) run one tile ahead of its bias (2 stages): waiting for a bias
-      // stage never delays the next Q / dO load
-      auto load_bias = [&](int s) -> bool {
-        const int st = s & 1, qt = kt + s;
-        if (s >= 2 && !mbar_wait(BAR(7 + st), ((s >> 1) & 1) ^ 1, abort_flag, ctl)) return false;
-        const int prow = static_cast<int>((pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt) * kQTile);
-        mbar_arrive_expect_tx(BAR(5 + st), 32768);
-        tma_load_2d(sBT0 + st * 32768, &tmBT, BAR(5 + st), 0, prow);
-        tma_load_2d(sBT0 + st * 32768 + 16384, &tmBT, BAR(5 + st), 64, prow);
-        return true;
-      };
-      bool ok = true;
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int qt = kt + s, sq = s % 3;
-        if (s >= 3 && !mbar_wait(qdo_empty(sq), ((s / 3) & 1) ^ 1, abort_flag, ctl)) break;
-        const int qrow = static_cast<int>(seq0) + qt * kQTile;
-        mbar_arrive_expect_tx(qdo_full(sq), 32768);
-        tma_load_2d(sQ0 + sq * 32768, &tmQ, qdo_full(sq), h * kD, qrow);
-        tma_load_2d(sQ0 + sq * 32768 + 16384, &tmDO, qdo_full(sq), h * kD, qrow);
-        if (s >= 1) ok = load_bias(s - 1);
-      }
-      if (ok && nsteps > 0) load_bias(nsteps - 1);
+    // ---------------- TMA producer: K, V once; Q / dO of stage sq from lanes 2 sq, 2 sq + 1; the bias
+    // halves of stage st from lanes 8 + 2 st, 9 + 2 st (consecutive stages load from different threads)
+    if (lane == 0) mbar_arrive_expect_tx(BAR(0), 32768);
+    __syncwarp();
+    if (lane == 0) tma_load_2d(sK, &tmK, BAR(0), h * kD, krow);
+    if (lane == 1) tma_load_2d(sV, &tmV, BAR(0), h * kD, krow);
+    // Q and dO of tile s (3 stages) run one tile ahead of its bias (2 stages): waiting for a bias
+    // stage never delays the next Q / dO load
+    auto load_bias = [&](int s) -> bool {
+      const int st = s & 1, qt = kt + s;
+      if (s >= 2 && !mbar_wait_warp(BAR(7 + st), ((s >> 1) & 1) ^ 1, abort_flag, ctl)) return false;
+      const int prow = static_cast<int>((pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt) * kQTile);
+      if (lane == 0) mbar_arrive_expect_tx(BAR(5 + st), 32768);
+      __syncwarp();
+      const int hx = lane - 8 - 2 * st;
+      if (hx == 0 || hx == 1) tma_load_2d(sBT0 + st * 32768 + hx * 16384, &tmBT, BAR(5 + st), 64 * hx, prow);
+      return true;
+    };
+    bool ok = true;
+    for (int s = 0; ok && s < nsteps; ++s) {
+      const int qt = kt + s, sq = s % 3;
+      if (s >= 3 && !mbar_wait_warp(qdo_empty(sq), ((s / 3) & 1) ^ 1, abort_flag, ctl)) break;
+      const int qrow = static_cast<int>(seq0) + qt * kQTile;
+      if (lane == 0) mbar_arrive_expect_tx(qdo_full(sq), 32768);
+      __syncwarp();
+      if (lane == 2 * sq) tma_load_2d(sQ0 + sq * 32768, &tmQ, qdo_full(sq), h * kD, qrow);
+      if (lane == 2 * sq + 1) tma_load_2d(sQ0 + sq * 32768 + 16384, &tmDO, qdo_full(sq), h * kD, qrow);
+      if (s >= 1) ok = load_bias(s - 1);
     }
-  } else if (warp == kSiluWarpsB + 1) {
-    // ---------------- tcgen05 issuer ----------------
+    if (ok && nsteps > 0) load_bias(nsteps - 1);
+  } else if (warp == kSiluWarpsB + 1 || warp == kSiluWarpsB + 3) {
+    // ---------------- tcgen05 issuers: S / dA (warp 17) and the gradient MMAs (warp 19) ----------------
     // Per query tile s, in two halves of 64 queries: S^T_h = K Q_h^T and dA^T_h = V dO_h^T, then,
     // once the elementwise warps of half h have written P^T_h (TMEM) and dX^T_h (shared memory),
     // dV += P^T_h dO_h and dK += dX^T_h Q_h; after half b also dQ_tile = dX K. P^T has TMEM columns
-    // of its own, so the next tile's S^T_h, dA^T_h go first, as soon as half h has read this tile's:
-    // the elementwise warps of half h start the next tile while the gradient MMAs run.
+    // of its own, so the next tile's S^T_h, dA^T_h are issued (by their own thread) as soon as half
+    // h has read this tile's: the elementwise warps of half h start the next tile while the
+    // gradient MMAs (the other thread) run. Both threads' MMAs read Q / dO, so its stage is freed
+    // by two commits.
     if (lane == 0) {
       constexpr uint32_t id_s = make_idesc_f16kind(128, 64, 0, 0, F16);
       constexpr uint32_t id_kmn = make_idesc_f16kind(128, 64, 0, 1, F16);
@@ -231,26 +237,37 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           umma_f16_ss(tDK, sdesc_add(xd, k4 * 32), sdesc_add(qd, k4 * 2048), id_kmn, k4 > 0 ? 1u : acc0);
         umma_commit(BAR(19 + hh));
       };
-      if (ok && nsteps > 0) ok = issue_s(0, 0) && issue_s(0, 1);
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int st = s & 1;
-        for (int hh = 0; ok && hh < 2; ++hh) {
-          ok = mbar_wait(BAR(11 + hh), s & 1, abort_flag, ctl) && (s + 1 >= nsteps || issue_s(s + 1, hh));
-          if (ok) {
-            tc_fence_after();
-            issue_grad(s, hh);
-          }
+      if (warp == kSiluWarpsB + 1) {
+        if (ok && nsteps > 0) {
+          ok = issue_s(0, 0) && issue_s(0, 1);
+          if (ok) umma_commit(qdo_empty(0));
         }
-        if (!ok) break;
-        const uint64_t xd = sdesc_add(x_mn, st * 32768);
+        for (int s = 0; ok && s + 1 < nsteps; ++s) {
+          for (int hh = 0; ok && hh < 2; ++hh)
+            ok = mbar_wait(BAR(11 + hh), s & 1, abort_flag, ctl) && issue_s(s + 1, hh);
+          if (ok) umma_commit(qdo_empty((s + 1) % 3));
+        }
+      } else {
+        for (int s = 0; ok && s < nsteps; ++s) {
+          const int st = s & 1;
+          for (int hh = 0; ok && hh < 2; ++hh) {
+            ok = mbar_wait(BAR(11 + hh), s & 1, abort_flag, ctl);
+            if (ok) {
+              tc_fence_after();
+              issue_grad(s, hh);
+            }
+          }
+          if (!ok) break;
+          const uint64_t xd = sdesc_add(x_mn, st * 32768);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)   // dQ_tile = dX K
-          umma_f16_ss(tDQ, sdesc_add(xd, kk * 2048), sdesc_add(k_mn, kk * 2048), id_mnmn, kk > 0 ? 1u : 0u);
-        umma_commit(BAR(13));
-        umma_commit(qdo_empty(s % 3));
-        umma_commit(BAR(7 + st));
+          for (int kk = 0; kk < 8; ++kk)   // dQ_tile = dX K
+            umma_f16_ss(tDQ, sdesc_add(xd, kk * 2048), sdesc_add(k_mn, kk * 2048), id_mnmn, kk > 0 ? 1u : 0u);
+          umma_commit(BAR(13));
+          umma_commit(qdo_empty(s % 3));
+          umma_commit(BAR(7 + st));
+        }
+        if (ok) umma_commit(BAR(14));
       }
-      if (ok) umma_commit(BAR(14));
     }
   } else if (warp == kSiluWarpsB + 2) {
     // ---------------- TMA stores ----------------
@@ -258,34 +275,38 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // TMA reduce-add per 32 columns; once both query halves of tile s are done, dX^T (the 16-bit
     // operand of dK and dQ, in the stage's bias slot) goes to the workspace, from which the table
     // gradients are summed over the heads.
-    if (lane == 0) {
-      auto reduce_dq = [&](int j) -> bool {
-        if (!mbar_wait(BAR(17), j & 1, abort_flag, ctl)) return false;
+    // dQ reduce-adds from lanes 0 and 1, dX^T stores from lanes 2 and 3 (each lane waits for its own
+    // bulk group; lane 0 then signals the barrier)
+    auto reduce_dq = [&](int j) -> bool {
+      if (!mbar_wait_warp(BAR(17), j & 1, abort_flag, ctl)) return false;
+      if (lane < 2) {
         const int y = static_cast<int>(seq0) + (kt + j) * kQTile;
-        tma_reduce_add_2d(&tmDQ, sDQ, h * kD, y);
-        tma_reduce_add_2d(&tmDQ, sDQ + 16384, h * kD + 32, y);
+        tma_reduce_add_2d(&tmDQ, sDQ + lane * 16384, h * kD + 32 * lane, y);
         bulk_commit_group();
         bulk_wait_group_read<0>();
-        mbar_arrive(BAR(18));
-        return true;
-      };
-      bool ok = true;
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int st = s & 1;
-        if (s >= 1 && !reduce_dq(s - 1)) { ok = false; break; }
-        if (!mbar_wait(BAR(15 + st), (s >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(18));
+      return true;
+    };
+    bool ok = true;
+    for (int s = 0; ok && s < nsteps; ++s) {
+      const int st = s & 1;
+      if (s >= 1 && !reduce_dq(s - 1)) { ok = false; break; }
+      if (!mbar_wait_warp(BAR(15 + st), (s >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
+      if (lane == 2 || lane == 3) {
         const int qt = kt + s;
         const long long pair = pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt;
         const int y = static_cast<int>((pair * a.H + h) * kQTile);
-        tma_store_2d(&tmDX, sBT0 + st * 32768, 0, y);
-        tma_store_2d(&tmDX, sBT0 + st * 32768 + 16384, 64, y);
+        tma_store_2d(&tmDX, sBT0 + st * 32768 + (lane - 2) * 16384, 64 * (lane - 2), y);
         bulk_commit_group();
         bulk_wait_group_read<0>();
-        mbar_arrive(BAR(7 + st));
       }
-      if (ok && nsteps > 0) reduce_dq(nsteps - 1);
-      bulk_wait_group_all();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(7 + st));
     }
+    if (ok && nsteps > 0) reduce_dq(nsteps - 1);
+    bulk_wait_group_all();
   } else {
     // ---------------- elementwise warps ----------------
     // warp w: key rows [32 (w & 3), +32) (TMEM lane quadrant), query half hq = (w >> 2) & 1,
@@ -453,6 +474,7 @@ constexpr int kTgThreads = 256;
 template <bool F16>
 __global__ void __launch_bounds__(kTgThreads)
 attn_table_grad_kernel(AttnBwdArgs A) {
+  pdl_enter();
   const AttnArgs& a = A.f;
   int b, qt, kt;
   if (!decode_tile_pair(blockIdx.x, a.pair_base, a.B, &b, &qt, &kt)) return;
@@ -574,8 +596,7 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  attn_bias_t_kernel<<<static_cast<unsigned>(a.max_pairs), kBiasThreads, 0, st>>>(A);
-  e = cudaGetLastError();
+  e = launch_pdl(attn_bias_t_kernel, dim3(static_cast<unsigned>(a.max_pairs)), dim3(kBiasThreads), 0, st, A);
   if (e != cudaSuccess) return e;
   // TMA row coordinates of the bias and dX^T tiles are 32-bit
   if (a.max_pairs * a.H * kQTile > 0x7fffffffLL) return cudaErrorInvalidValue;
@@ -594,13 +615,11 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), BwdSmem::kTotal);
   if (e != cudaSuccess) return e;
   const long long blocks = a.capacity * a.H;
-  kern<<<static_cast<unsigned>(blocks), kThreadsB, BwdSmem::kTotal, st>>>(tq, tk, tv, tdo, tbt, tdx, tdq, A,
-                                                                          wait_ctl(a.status));
-  e = cudaGetLastError();
+  e = launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(kThreadsB), BwdSmem::kTotal, st, tq, tk, tv, tdo, tbt,
+                 tdx, tdq, A, wait_ctl(a.status));
   if (e != cudaSuccess) return e;
   auto tg = f16 ? attn_table_grad_kernel<true> : attn_table_grad_kernel<false>;
-  tg<<<dim3(static_cast<unsigned>(a.max_pairs), 2), kTgThreads, 0, st>>>(A);
-  return cudaGetLastError();
+  return launch_pdl(tg, dim3(static_cast<unsigned>(a.max_pairs), 2), dim3(kTgThreads), 0, st, A);
 }
 
 }  // namespace hstu

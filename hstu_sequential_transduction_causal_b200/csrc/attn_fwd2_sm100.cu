@@ -19,9 +19,10 @@
 //                  stays hidden; all 128-byte swizzled.
 //       bias warp: TMA producer of the bias tiles (one per key tile), so that waiting for a bias
 //                  stage (freed by the SiLU warps) never delays a K or V load.
-//       MMA warp : tcgen05 issuer: S = Q K^T into one of three TMEM tiles; O_h += P V two units
-//                  later, with the A operand P read from TMEM (P overwrites the S tile it came
-//                  from), so the S MMAs of the next units never wait for a P V MMA.
+//       MMA warps: two tcgen05 issuing threads. One issues S = Q K^T into one of three TMEM tiles
+//                  (the tile of unit s - 3 once its P V has completed), the other O_h += P V with
+//                  the A operand P read from TMEM (P overwrites the S tile it came from); neither
+//                  waits behind the other's barriers, so the S MMAs of later units overlap SiLU.
 //       SiLU warps (8 per group, NG groups, numbered first; then the K/V, MMA and bias warps):
 //                  TMEM lane quadrant (warp & 3), key half (warp >> 2) & 1. Per element, in packed
 //                  fp16: h = 0.5 s + 0.5 bias, P = h + h tanh(h) = SiLU(s + bias); causal mask on
@@ -45,7 +46,7 @@ namespace {
 
 constexpr int kD = 64;
 constexpr int kSiluWarps = 8;     // one group of SiLU warps: 4 TMEM lane quadrants x 2 key halves
-__host__ __device__ constexpr int threads2(int ng) { return 32 * (kSiluWarps * ng + 3); }
+__host__ __device__ constexpr int threads2(int ng) { return 32 * (kSiluWarps * ng + 4); }
 constexpr uint32_t kHalf2Half = 0x38003800u;   // (0.5, 0.5) in fp16
 
 // ----------------------------------------------------------------------------------------------
@@ -55,6 +56,7 @@ constexpr uint32_t kHalf2Half = 0x38003800u;   // (0.5, 0.5) in fp16
 // half-bias tile of bias_tile.cuh.
 __global__ void __launch_bounds__(kBiasThreads)
 attn_bias_kernel(AttnArgs a) {
+  pdl_enter();
   bias_tile_block<false, false>(a, blockIdx.x,
                                 reinterpret_cast<uint16_t*>(a.bias) + blockIdx.x * static_cast<long long>(kQTile * kQTile),
                                 nullptr);
@@ -84,9 +86,11 @@ __global__ void __launch_bounds__(threads2(NG), 1)
 attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB, AttnArgs a,
                     WaitCtl ctl) {
+  pdl_enter();
   using L = Smem2<G>;
   static_assert(NG == 1 || G == 1, "two SiLU groups need one head per CTA");
   constexpr int kTmaWarp = kSiluWarps * NG, kMmaWarp = kTmaWarp + 1, kBiasWarp = kTmaWarp + 2;
+  constexpr int kPvWarp = kTmaWarp + 3;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int HG = a.H / G;
@@ -116,13 +120,14 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   // 0 q_full | k_full [NK] | k_empty [NK] | v_full [NV] | v_empty [NV] | b_full [BS] | b_empty [BS] |
   // s_full [3] | p_full [3] | o_full
   constexpr int kBarK = 1, kBarV = kBarK + 2 * NK, kBarB = kBarV + 2 * NV, kBarS = kBarB + 2 * BS;
-  constexpr int kBarP = kBarS + 3, kBarO = kBarP + 3, kNumBars = kBarO + 1;
+  constexpr int kBarP = kBarS + 3, kBarO = kBarP + 3, kBarPv = kBarO + 1, kNumBars = kBarPv + 3;
   static_assert(kNumBars * 8 + 8 <= 256, "barrier region");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = smem_u32(bars);
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   const uint32_t bar_q = BAR(0), bar_o = BAR(kBarO);
+  auto bar_pv_done = [&](int b) { return BAR(kBarPv + b); };   // P V of the unit in TMEM tile b done
   auto bar_k_full = [&](int s) { return BAR(kBarK + s); };
   auto bar_k_empty = [&](int s) { return BAR(kBarK + NK + s); };
   auto bar_v_full = [&](int s) { return BAR(kBarV + s); };
@@ -155,6 +160,7 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
       mbar_init(bar_p_full(s), kSiluThreads);
     }
     mbar_init(bar_o, 1);
+    for (int b3 = 0; b3 < 3; ++b3) mbar_init(bar_pv_done(b3), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -182,104 +188,95 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   const int qrow0 = FALCON ? b * a.cand_rows + qt * kQTile : static_cast<int>(seq0) + qt * kQTile;
 
   if (warp == kTmaWarp) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q, G * 16384);
-      for (int h = 0; h < G; ++h) tma_load_2d(sQ + h * 16384, &tmQ, bar_q, (hg * G + h) * kD, qrow0);
-      // unit s = (key tile s / G, head s % G): K(s) first, V(s - 1) after it, so waiting for a V
-      // stage (freed late, by a P V MMA) never delays a K load
-      auto load_v = [&](int s) -> bool {
-        const int st = s % NV;
-        if (s >= NV && !mbar_wait(bar_v_empty(st), ((s / NV) - 1) & 1, abort_flag, ctl)) return false;
+    // ---------------- TMA producer: K stage st from lane st, V stage st from lane 8 + st ----------------
+    if (lane == 0) mbar_arrive_expect_tx(bar_q, G * 16384);
+    __syncwarp();
+    if (lane < G) tma_load_2d(sQ + lane * 16384, &tmQ, bar_q, (hg * G + lane) * kD, qrow0);
+    // unit s = (key tile s / G, head s % G): K(s) first, V(s - 1) after it, so waiting for a V
+    // stage (freed late, by a P V MMA) never delays a K load
+    auto load_v = [&](int s) -> bool {
+      const int st = s % NV;
+      if (s >= NV && !mbar_wait_warp(bar_v_empty(st), ((s / NV) - 1) & 1, abort_flag, ctl)) return false;
+      if (lane == 8 + st) {
         mbar_arrive_expect_tx(bar_v_full(st), 16384);
         tma_load_2d(sV + st * 16384, &tmV, bar_v_full(st), (hg * G + s % G) * kD,
                     static_cast<int>(seq0) + (s / G) * kQTile);
-        return true;
-      };
-      bool ok = true;
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int kt = s / G, h = s % G;
-        const int st = s % NK;
-        if (s >= NK && !mbar_wait(bar_k_empty(st), ((s / NK) - 1) & 1, abort_flag, ctl)) break;
+      }
+      return true;
+    };
+    bool ok = true;
+    for (int s = 0; ok && s < nsteps; ++s) {
+      const int kt = s / G, h = s % G;
+      const int st = s % NK;
+      if (s >= NK && !mbar_wait_warp(bar_k_empty(st), ((s / NK) - 1) & 1, abort_flag, ctl)) break;
+      if (lane == st) {
         mbar_arrive_expect_tx(bar_k_full(st), 16384);
         tma_load_2d(sK + st * 16384, &tmK, bar_k_full(st), (hg * G + h) * kD, static_cast<int>(seq0) + kt * kQTile);
-        if (s >= 1) ok = load_v(s - 1);
       }
-      if (ok && nsteps > 0) load_v(nsteps - 1);
+      if (s >= 1) ok = load_v(s - 1);
     }
+    if (ok && nsteps > 0) load_v(nsteps - 1);
   } else if (warp == kBiasWarp) {
-    // ---------------- bias tiles ----------------
-    if (!FALCON && lane == 0) {
+    // ---------------- bias tiles (stage bs: its two 64-column halves from lanes 2 bs, 2 bs + 1) ----
+    if (!FALCON) {
       for (int kt = 0; kt < nkt; ++kt) {
         const int bs = kt % BS;
-        if (kt >= BS && !mbar_wait(bar_b_empty(bs), ((kt / BS) - 1) & 1, abort_flag, ctl)) break;
+        if (kt >= BS && !mbar_wait_warp(bar_b_empty(bs), ((kt / BS) - 1) & 1, abort_flag, ctl)) break;
         const int brow = static_cast<int>((pair0 + kt) * kQTile);
-        mbar_arrive_expect_tx(bar_b_full(bs), 32768);
-        tma_load_2d(sB + bs * 32768, &tmB, bar_b_full(bs), 0, brow);
-        tma_load_2d(sB + bs * 32768 + 16384, &tmB, bar_b_full(bs), 64, brow);
+        if (lane == 0) mbar_arrive_expect_tx(bar_b_full(bs), 32768);
+        __syncwarp();
+        const int hx = lane - 2 * bs;
+        if (hx == 0 || hx == 1) tma_load_2d(sB + bs * 32768 + hx * 16384, &tmB, bar_b_full(bs), 64 * hx, brow);
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ---------------- tcgen05 issuer ----------------
+  } else if (warp == kMmaWarp || warp == kPvWarp) {
+    // ---------------- tcgen05 issuers: S = Q K^T (one thread), O_h += P V (another) ----------------
+    // Two issuing threads keep the tensor pipe fed: neither waits behind the other's barrier. S of
+    // unit s reuses the TMEM tile of unit s - 3, so it waits for that unit's P V to have completed.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc_f16kind(128, 128, 0, 0, F16);
       constexpr uint32_t idesc_pv = make_idesc_f16kind(128, 64, 0, 1, F16);
-      bool ok = mbar_wait(bar_q, 0, abort_flag, ctl);
-      const uint64_t q_desc0 = make_sdesc_sw128(sQ, 16, 1024), k_desc0 = make_sdesc_sw128(sK, 16, 1024);
-      const uint64_t v_desc0 = make_sdesc_sw128(sV, 16384, 1024);
-      auto issue_s = [&](int s) {
-        const int buf = s % 3, st = s % NK, h = s % G;
-        tc_fence_after();
-        const uint64_t qd = sdesc_add(q_desc0, h * 16384), kd = sdesc_add(k_desc0, st * 16384);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_f16_ss(tmem + buf * 128, sdesc_add(qd, kk * 32), sdesc_add(kd, kk * 32), idesc_qk, kk > 0 ? 1u : 0u);
-        umma_commit(bar_s_full(buf));
-        umma_commit(bar_k_empty(st));
-      };
-      auto issue_pv = [&](int t) {
-        const int buf = t % 3, st = t % NV, h = t % G;
-        tc_fence_after();
-        const uint64_t vd = sdesc_add(v_desc0, st * 16384);
-        const uint32_t a_tmem = tmem + buf * 128, o_tmem = tmem + kOCol + 64 * h;
-        const uint32_t acc0 = t >= G ? 1u : 0u;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_f16_ts(o_tmem, a_tmem + 64 * (kk >> 2) + 8 * (kk & 3), sdesc_add(vd, kk * 2048), idesc_pv,
-                      kk > 0 ? 1u : acc0);
-        umma_commit(bar_v_empty(st));
-      };
-      // S of unit sn goes first whenever its K tile has landed and its TMEM tile is free (the P V of
-      // unit sn - 3 has been issued: MMAs run in issue order); otherwise P V of unit tn once its P
-      // and V are ready. Neither waits for the other, so the next units' S overlaps this unit's
-      // SiLU. Polling is bounded like every wait: no progress for ctl.limit cycles aborts.
-      int sn = 0, tn = 0;
-      unsigned long long t_prog = clock64();
-      uint32_t idle = 0;
-      while (ok && tn < nsteps) {
-        bool progressed = false;
-        if (sn < nsteps && sn - tn < 3 && mbar_test(bar_k_full(sn % NK), (sn / NK) & 1)) {
-          issue_s(sn++);
-          progressed = true;
-        } else if (tn < sn && mbar_test(bar_p_full(tn % 3), (tn / 3) & 1) &&
-                   mbar_test(bar_v_full(tn % NV), (tn / NV) & 1)) {
-          issue_pv(tn++);
-          progressed = true;
-        }
-        if (progressed) {
-          t_prog = clock64();
-          idle = 0;
-        } else if ((++idle & 15u) == 0u) {
-          if (*abort_flag) {
+      bool ok = true;
+      if (warp == kMmaWarp) {
+        ok = mbar_wait(bar_q, 0, abort_flag, ctl);
+        const uint64_t q_desc0 = make_sdesc_sw128(sQ, 16, 1024), k_desc0 = make_sdesc_sw128(sK, 16, 1024);
+        for (int s = 0; ok && s < nsteps; ++s) {
+          const int buf = s % 3, st = s % NK, h = s % G;
+          if (!mbar_wait(bar_k_full(st), (s / NK) & 1, abort_flag, ctl) ||
+              (s >= 3 && !mbar_wait(bar_pv_done(buf), ((s / 3) - 1) & 1, abort_flag, ctl))) {
             ok = false;
-          } else if (clock64() - t_prog > ctl.limit) {
-            *abort_flag = 1;
-            report_error(ctl.status, kDevTimeout);
-            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint64_t qd = sdesc_add(q_desc0, h * 16384), kd = sdesc_add(k_desc0, st * 16384);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f16_ss(tmem + buf * 128, sdesc_add(qd, kk * 32), sdesc_add(kd, kk * 32), idesc_qk, kk > 0 ? 1u : 0u);
+          umma_commit(bar_s_full(buf));
+          umma_commit(bar_k_empty(st));
         }
+      } else {
+        const uint64_t v_desc0 = make_sdesc_sw128(sV, 16384, 1024);
+        for (int t = 0; ok && t < nsteps; ++t) {
+          const int buf = t % 3, st = t % NV, h = t % G;
+          if (!mbar_wait(bar_p_full(buf), (t / 3) & 1, abort_flag, ctl) ||
+              !mbar_wait(bar_v_full(st), (t / NV) & 1, abort_flag, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t vd = sdesc_add(v_desc0, st * 16384);
+          const uint32_t a_tmem = tmem + buf * 128, o_tmem = tmem + kOCol + 64 * h;
+          const uint32_t acc0 = t >= G ? 1u : 0u;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ts(o_tmem, a_tmem + 64 * (kk >> 2) + 8 * (kk & 3), sdesc_add(vd, kk * 2048), idesc_pv,
+                        kk > 0 ? 1u : acc0);
+          umma_commit(bar_v_empty(st));
+          umma_commit(bar_pv_done(buf));
+        }
+        if (ok && nsteps > 0) umma_commit(bar_o);
       }
-      if (ok && nsteps > 0) umma_commit(bar_o);
     }
   } else {
     // ---------------- SiLU warps ----------------
@@ -490,8 +487,8 @@ cudaError_t launch_attn2(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   const long long blocks =
       (FALCON ? static_cast<long long>(a.B) * ((a.cand_rows + kQTile - 1) / kQTile) : a.capacity) * (a.H / G);
   if (blocks == 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(blocks), threads2(NG), Smem2<G>::kTotal, st>>>(tq, tk, tv, tb, a, wait_ctl(a.status));
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(threads2(NG)), Smem2<G>::kTotal, st, tq, tk, tv, tb,
+                    a, wait_ctl(a.status));
 }
 
 }  // namespace
@@ -507,8 +504,7 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  attn_bias_kernel<<<static_cast<unsigned>(a.max_pairs), kBiasThreads, 0, st>>>(a);
-  e = cudaGetLastError();
+  e = launch_pdl(attn_bias_kernel, dim3(static_cast<unsigned>(a.max_pairs)), dim3(kBiasThreads), 0, st, a);
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv, tb;
   const bool f16 = a.in_f16 != 0;

@@ -5,9 +5,9 @@
 // the buckets of time_bucket_dev.cuh). The bias does not depend on the head, so a pair's tile is
 // computed once and read by every head.
 //
-// Thread t takes 8 consecutive columns [8 (t % 16), +8) of the rows t / 16 + 16 p, p < 8: 64
-// elements, one 16-byte store per row (and an 8-byte bucket store). TRANSPOSED: rows are keys and
-// columns queries (the backward's [key][query] tiles); otherwise rows are queries. Timestamps past
+// Thread t takes the column pairs 2 (t % 16) + 32 e, e < 4, of the rows t / 16 + 16 p, p < 8: 64
+// elements, 4-byte half-bias (and 2-byte bucket) stores. TRANSPOSED: rows are keys and columns
+// queries (the backward's [key][query] tiles); otherwise rows are queries. Timestamps past
 // the sequence end are clamped to its last token (those elements are masked by the attention).
 // When every difference of the tile fits in int32 (spans under 68 years of seconds) the bucket
 // arithmetic is 32-bit.
@@ -78,55 +78,59 @@ __device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pai
   if (fast) s_ts32[tid] = static_cast<int>(s_ts[tid] - lo);
   __syncthreads();
   const int nb = a.n_buckets;
-  const int c0 = 8 * (tid & 15);
+  // thread: column pairs c = 2 (tid % 16) + 32 e + x (e < 4, x < 2) of rows r = tid / 16 + 16 p (p < 8).
+  // The 16 lanes of a half-warp read 32 consecutive diagonals of the rab_pos window (no bank
+  // conflicts) and store 64 contiguous bytes of one row.
+  const int cl = 2 * (tid & 15), rr = tid >> 4;
   // the query / key timestamp arrays of rows and columns
   const int row_base = TRANSPOSED ? 128 : 0, col_base = TRANSPOSED ? 0 : 128;
   if (fast) {
     int tc[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) tc[e] = s_ts32[col_base + c0 + e];
+    for (int e = 0; e < 4; ++e) {
+      tc[2 * e] = s_ts32[col_base + cl + 32 * e];
+      tc[2 * e + 1] = s_ts32[col_base + cl + 32 * e + 1];
+    }
 #pragma unroll 2
     for (int p = 0; p < 8; ++p) {
-      const int r = (tid >> 4) + 16 * p;
+      const int r = rr + 16 * p;
       const int tr = s_ts32[row_base + r];
-      uint32_t w[4], bw[2] = {0u, 0u};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         float v2[2];
+        uint32_t bw = 0u;
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-          const int c = c0 + 2 * e + x;
+          const int c = cl + 32 * e + x;
           const int dt = TRANSPOSED ? tc[2 * e + x] - tr : tr - tc[2 * e + x];   // t_query - t_key
           const int bkt = time_bucket32(dt, s_tau32, nb);
           v2[x] = s_win[TRANSPOSED ? c - r + 127 : r - c + 127] + s_rt[bkt];
-          if (BUCKETS) bw[e >> 1] |= static_cast<uint32_t>(bkt) << (8 * (2 * (e & 1) + x));
+          bw |= static_cast<uint32_t>(bkt) << (8 * x);
         }
-        w[e] = pack_f16x2(v2[0], v2[1]);
+        *reinterpret_cast<uint32_t*>(tile + r * kQTile + cl + 32 * e) = pack_f16x2(v2[0], v2[1]);
+        if (BUCKETS) *reinterpret_cast<uint16_t*>(btile + r * kQTile + cl + 32 * e) = static_cast<uint16_t>(bw);
       }
-      *reinterpret_cast<uint4*>(tile + r * kQTile + c0) = make_uint4(w[0], w[1], w[2], w[3]);
-      if (BUCKETS) *reinterpret_cast<uint2*>(btile + r * kQTile + c0) = make_uint2(bw[0], bw[1]);
     }
   } else {
 #pragma unroll 1
     for (int p = 0; p < 8; ++p) {
-      const int r = (tid >> 4) + 16 * p;
+      const int r = rr + 16 * p;
       const long long tr = s_ts[row_base + r];
-      uint32_t w[4], bw[2] = {0u, 0u};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         float v2[2];
+        uint32_t bw = 0u;
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
-          const int c = c0 + 2 * e + x;
+          const int c = cl + 32 * e + x;
           const long long tcv = s_ts[col_base + c];
           const int bkt = time_bucket_dev(TRANSPOSED ? tcv - tr : tr - tcv, s_tau, nb);
           v2[x] = s_win[TRANSPOSED ? c - r + 127 : r - c + 127] + s_rt[bkt];
-          if (BUCKETS) bw[e >> 1] |= static_cast<uint32_t>(bkt) << (8 * (2 * (e & 1) + x));
+          bw |= static_cast<uint32_t>(bkt) << (8 * x);
         }
-        w[e] = pack_f16x2(v2[0], v2[1]);
+        *reinterpret_cast<uint32_t*>(tile + r * kQTile + cl + 32 * e) = pack_f16x2(v2[0], v2[1]);
+        if (BUCKETS) *reinterpret_cast<uint16_t*>(btile + r * kQTile + cl + 32 * e) = static_cast<uint16_t>(bw);
       }
-      *reinterpret_cast<uint4*>(tile + r * kQTile + c0) = make_uint4(w[0], w[1], w[2], w[3]);
-      if (BUCKETS) *reinterpret_cast<uint2*>(btile + r * kQTile + c0) = make_uint2(bw[0], bw[1]);
     }
   }
 }

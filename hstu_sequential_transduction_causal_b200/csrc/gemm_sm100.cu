@@ -86,13 +86,14 @@ __device__ __forceinline__ float load_one(const void* base, int dt, int64_t idx)
 
 // Per-warp epilogue staging: boxes of 32 rows x 128 bytes in the 128-byte swizzled layout of the
 // output tensor maps, written row-per-lane (16-byte units XOR-ed with the row: conflict-free) and
-// sent by TMA (store or fp32 reduce-add), two boxes in flight per warp.
+// sent by TMA (store or fp32 reduce-add), two boxes in flight per warp. Box slot i is sent by lane i
+// (a thread keeps about one bulk copy in flight, so the two slots' copies overlap).
 struct EpiStage {
   uint8_t* base;   // this warp's 2 boxes
   int slot;
   __device__ __forceinline__ void emit(const CUtensorMap* map, bool reduce, int x, int y, const uint32_t* w) {
     const int lane = threadIdx.x & 31;
-    if (lane == 0) bulk_wait_group_read<1>();   // the box written two emissions ago has been read
+    if (lane == slot) bulk_wait_group_read<0>();   // this slot's previous box has been read
     __syncwarp();
     uint8_t* box = base + slot * kBoxBytes;
     uint8_t* row = box + lane * 128;
@@ -101,7 +102,7 @@ struct EpiStage {
       *reinterpret_cast<uint4*>(row + ((u ^ (lane & 7)) << 4)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
     fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) {
+    if (lane == slot) {
       if (reduce) tma_reduce_add_2d(map, smem_u32(box), x, y);
       else tma_store_2d(map, smem_u32(box), x, y);
       bulk_commit_group();
@@ -139,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                     GemmParams P, WaitCtl ctl) {
+  pdl_enter();
   using L = GemmSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -184,35 +186,44 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   };
 
   if (warp == kEpiWarps) {
-    if (lane == 0) {
-      int g = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < P.total; t += gridDim.x) {
-        int m0, n0, kb0, kb1;
-        decode(t, m0, n0, kb0, kb1);
-        for (int kb = kb0; kb < kb1; ++kb, ++g) {
-          const int s = g % STAGES;
-          if (g >= STAGES && !mbar_wait(smem_u32(&bars[STAGES + s]), ((g / STAGES) - 1) & 1, abort_flag, ctl)) {
-            ok = false;
-            break;
-          }
-          const uint32_t full = smem_u32(&bars[s]);
-          const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
-          const uint32_t sb = sa + L::kABytes;
-          const int kx = kb * kBK;
-          mbar_arrive_expect_tx(full, L::kStageBytes);
-          if (!A_MN) {
-            tma_load_2d(sa, &tmA, full, kx, m0);
-          } else {
-            tma_load_2d(sa, &tmA, full, m0, kx);
-            tma_load_2d(sa + 8192, &tmA, full, m0 + 64, kx);
-          }
-          if (!B_MN) {
-            tma_load_2d(sb, &tmB, full, kx, n0);
-          } else {
-#pragma unroll
-            for (int c = 0; c < BN / 64; ++c) tma_load_2d(sb + c * 8192, &tmB, full, n0 + 64 * c, kx);
-          }
+    // TMA producer. A thread keeps about one tile load in flight (measured: one 16 KB box per
+    // ~550 cycles per issuing thread, 3x that from 4 lanes), so the boxes of a stage are issued by
+    // different lanes: box i of stage s by lane s * boxes + i (A: 1 K-major box or 2 MN-major halves;
+    // B: 1 K-major box or BN / 64 MN-major boxes). Lane 0 waits for the stage and registers the
+    // bytes first.
+    constexpr int kABoxes = A_MN ? 2 : 1;
+    constexpr int kBoxes = kABoxes + (B_MN ? BN / 64 : 1);
+    static_assert(kBoxes * STAGES <= 32, "one lane per box of every stage");
+    int g = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < P.total; t += gridDim.x) {
+      int m0, n0, kb0, kb1;
+      decode(t, m0, n0, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb, ++g) {
+        const int s = g % STAGES;
+        bool free_ok = true;   // lane 0 waits; the verdict is made warp-uniform
+        if (lane == 0 && g >= STAGES)
+          free_ok = mbar_wait(smem_u32(&bars[STAGES + s]), ((g / STAGES) - 1) & 1, abort_flag, ctl);
+        if (!__shfl_sync(0xffffffffu, free_ok ? 1 : 0, 0)) {
+          ok = false;
+          break;
+        }
+        const uint32_t full = smem_u32(&bars[s]);
+        const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
+        const uint32_t sb = sa + L::kABytes;
+        const int kx = kb * kBK;
+        if (lane == 0) mbar_arrive_expect_tx(full, L::kStageBytes);
+        __syncwarp();
+        // stage s's boxes come from lanes [s * kBoxes, (s + 1) * kBoxes): consecutive stages are in
+        // flight from different threads
+        const int bx = lane - s * kBoxes;
+        if (bx >= 0 && bx < kABoxes) {
+          if (!A_MN) tma_load_2d(sa, &tmA, full, kx, m0);
+          else tma_load_2d(sa + bx * 8192, &tmA, full, m0 + 64 * bx, kx);
+        } else if (bx >= kABoxes && bx < kBoxes) {
+          const int c = bx - kABoxes;
+          if (!B_MN) tma_load_2d(sb, &tmB, full, kx, n0);
+          else tma_load_2d(sb + c * 8192, &tmB, full, n0 + 64 * c, kx);
         }
       }
     }
@@ -298,7 +309,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (epi.kind == kEpiSilu) {
           if (epi.out1) emit64(es, &tmO1, epi.out1_dt, false, n, ybox, v, P.N);
 #pragma unroll
-          for (int j = 0; j < 64; ++j) v[j] = silu_fast(v[j]);
+          for (int j = 0; j < 64; ++j) v[j] = silu_tanh(v[j]);
         } else if (epi.resid) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -319,7 +330,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (epi.kind == kEpiLinear && epi.out1) emit64(es, &tmO1, epi.out1_dt, false, n, ybox, v, P.N);
       }
     }
-    if (lane == 0) bulk_wait_group_all();
+    if (lane < 2) bulk_wait_group_all();
   }
 
   tc_fence_before();
@@ -443,8 +454,7 @@ cudaError_t launch_tc(const GemmArgs& g, cudaStream_t st) {
   P.idesc = make_idesc_f16kind(kBM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0, g.f16);
   P.epi = g.epi;
   const int grid = P.total < sm_count() ? P.total : sm_count();
-  kern<<<grid, kThreads, L::kTotal, st>>>(tmA, tmB, tmO0, tmO1, P, wait_ctl(g.status));
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, tmA, tmB, tmO0, tmO1, P, wait_ctl(g.status));
 }
 
 template <int BN, int STAGES>

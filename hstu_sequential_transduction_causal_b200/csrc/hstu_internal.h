@@ -9,6 +9,28 @@
 
 namespace hstu {
 
+// Launches a kernel that begins with pdl_enter() with programmatic stream serialization: its CTAs
+// may become resident while the previous kernel of the stream drains (they wait in pdl_enter until
+// it has completed), which hides host launch latency between eagerly launched kernels. Under
+// stream capture the attribute is left off: a replayed graph already launches back to back, and
+// measured replays were slower with programmatic edges.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cfg.numAttrs = (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusNone) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------------------------------------
 // workspace layout: [0, 256) status word + padding, then per-call regions
 // ---------------------------------------------------------------------------------------------

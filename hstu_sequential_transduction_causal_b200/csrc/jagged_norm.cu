@@ -24,6 +24,7 @@ namespace {
 __global__ void __launch_bounds__(1024)
 worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items,
                 int32_t* count, int* status, long long* pair_base, int32_t* kitems, int32_t* kcount) {
+  pdl_enter();
   __shared__ int s_warp[32];
   __shared__ int s_max_tiles;
   __shared__ int s_bad;
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(256)
 norm_gate_kernel(int64_t T, const void* __restrict__ o, int64_t ld_o, const void* __restrict__ u,
                  int64_t ld_u, const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
                  void* __restrict__ g, float* __restrict__ mu_out, float* __restrict__ rstd_out) {
+  pdl_enter();
   constexpr int D = VPT * 32;
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -271,9 +273,8 @@ template <int VPT, int OT, int UT, int GT>
 cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int64_t ld_u, const float* gamma,
                       const float* beta, float eps, void* g, float* mu, float* rstd, cudaStream_t st) {
   const int64_t blocks = (T + 7) / 8;
-  norm_gate_kernel<VPT, OT, UT, GT><<<static_cast<unsigned>(blocks), 256, 0, st>>>(T, o, ld_o, u, ld_u, gamma, beta, eps,
-                                                                             g, mu, rstd);
-  return cudaGetLastError();
+  return launch_pdl(norm_gate_kernel<VPT, OT, UT, GT>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, T, o,
+                    ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd);
 }
 
 }  // namespace
@@ -281,8 +282,8 @@ cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
                             int32_t* count, int* status, cudaStream_t st, long long* pair_base, int32_t* kitems,
                             int32_t* kcount) {
-  worklist_kernel<<<1, 1024, 0, st>>>(offsets, B, T, max_len, items, count, status, pair_base, kitems, kcount);
-  return cudaGetLastError();
+  return launch_pdl(worklist_kernel, dim3(1), dim3(1024), 0, st, offsets, B, T, max_len, items, count, status,
+                    pair_base, kitems, kcount);
 }
 
 cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int n_buckets,

@@ -37,6 +37,7 @@ norm_gate_bwd_kernel(int64_t T, const float* __restrict__ dg, const float* __res
                      const void* __restrict__ zu, int64_t ld_act, const float* __restrict__ gamma,
                      const float* __restrict__ beta, const float* __restrict__ mu, const float* __restrict__ rstd,
                      void* __restrict__ d_o, void* __restrict__ dz, int64_t ld_dz, float* __restrict__ partial) {
+  pdl_enter();
   constexpr int D = VPT * 32;
   __shared__ float s_red[8][2][D];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(256)
 dz_assemble_kernel(int64_t T, int D, const float* __restrict__ dv, const float* __restrict__ dq,
                    const float* __restrict__ dk, const void* __restrict__ z, int64_t ld_z, void* __restrict__ dz,
                    int64_t ld_dz) {
+  pdl_enter();
   const int64_t idx = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;   // over T x 3D
   const int64_t per_row = 3ll * D;
   if (idx >= T * per_row) return;
@@ -119,6 +121,7 @@ template <int DT>
 __global__ void __launch_bounds__(256)
 colsum_partial_kernel(const void* __restrict__ in, int64_t rows, int cols, int64_t ld, int64_t rows_per,
                       float* __restrict__ partial) {
+  pdl_enter();
   const int c = blockIdx.x * 256 + threadIdx.x;
   if (c >= cols) return;
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per;
@@ -136,6 +139,7 @@ colsum_partial_kernel(const void* __restrict__ in, int64_t rows, int cols, int64
 template <int IT, int OT>
 __global__ void __launch_bounds__(256)
 convert_kernel(const void* __restrict__ in, void* __restrict__ out, int64_t n) {
+  pdl_enter();
   const int64_t i = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;
   if (i + 8 <= n) {
     float v[8];
@@ -156,6 +160,7 @@ convert_kernel(const void* __restrict__ in, void* __restrict__ out, int64_t n) {
 // then a shared-memory sum of the slices (the loads are independent and coalesced per warp).
 __global__ void __launch_bounds__(256)
 colsum_final_kernel(const float* __restrict__ partial, int parts, int cols, float* __restrict__ out) {
+  pdl_enter();
   __shared__ float s_part[8][33];
   const int cl = threadIdx.x & 31, slice = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + cl;
@@ -191,13 +196,14 @@ cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const f
                           float* dgamma_dbeta_out, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const int G = norm_gate_bwd_blocks(T);
+  cudaError_t e = cudaSuccess;
 #define HSTU_NGB(VPT)                                                                                            \
   if (act_dt == kDtF16)                                                                                          \
-    norm_gate_bwd_kernel<VPT, kDtF16><<<G, 256, 0, st>>>(T, dg, o, u, zu, ld_act, gamma, beta, mu, rstd, d_o, dz, \
-                                                         ld_dz, partial);                                        \
+    e = launch_pdl(norm_gate_bwd_kernel<VPT, kDtF16>, dim3(G), dim3(256), 0, st, T, dg, o, u, zu, ld_act, gamma,   \
+                   beta, mu, rstd, d_o, dz, ld_dz, partial);                                                      \
   else if (act_dt == kDtBF16)                                                                                    \
-    norm_gate_bwd_kernel<VPT, kDtBF16><<<G, 256, 0, st>>>(T, dg, o, u, zu, ld_act, gamma, beta, mu, rstd, d_o,   \
-                                                          dz, ld_dz, partial);                                   \
+    e = launch_pdl(norm_gate_bwd_kernel<VPT, kDtBF16>, dim3(G), dim3(256), 0, st, T, dg, o, u, zu, ld_act, gamma,  \
+                   beta, mu, rstd, d_o, dz, ld_dz, partial);                                                      \
   else                                                                                                           \
     return cudaErrorInvalidValue;
   switch (D) {
@@ -206,10 +212,9 @@ cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const f
     default: return cudaErrorInvalidValue;
   }
 #undef HSTU_NGB
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  colsum_final_kernel<<<(2 * D + 31) / 32, 256, 0, st>>>(partial, G, 2 * D, dgamma_dbeta_out);
-  return cudaGetLastError();
+  return launch_pdl(colsum_final_kernel, dim3((2 * D + 31) / 32), dim3(256), 0, st, static_cast<const float*>(partial), G,
+                    2 * D, dgamma_dbeta_out);
 }
 
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
@@ -217,17 +222,18 @@ cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const flo
   const int64_t threads = T * 3ll * D / 8;
   if (threads == 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
-  if (act_dt == kDtF16) dz_assemble_kernel<kDtF16><<<blocks, 256, 0, st>>>(T, D, dv, dq, dk, z, ld_z, dz, ld_dz);
-  else if (act_dt == kDtBF16) dz_assemble_kernel<kDtBF16><<<blocks, 256, 0, st>>>(T, D, dv, dq, dk, z, ld_z, dz, ld_dz);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (act_dt == kDtF16)
+    return launch_pdl(dz_assemble_kernel<kDtF16>, dim3(blocks), dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz);
+  if (act_dt == kDtBF16)
+    return launch_pdl(dz_assemble_kernel<kDtBF16>, dim3(blocks), dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t convert_dtype(const void* in, int in_dt, void* out, int out_dt, int64_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>(((n + 7) / 8 + 255) / 256);
 #define HSTU_CV(I, O) \
-  if (in_dt == I && out_dt == O) { convert_kernel<I, O><<<blocks, 256, 0, st>>>(in, out, n); return cudaGetLastError(); }
+  if (in_dt == I && out_dt == O) return launch_pdl(convert_kernel<I, O>, dim3(blocks), dim3(256), 0, st, in, out, n);
   HSTU_CV(kDtBF16, kDtF16)
   HSTU_CV(kDtF32, kDtF16)
   HSTU_CV(kDtF32, kDtBF16)
@@ -249,13 +255,14 @@ cudaError_t column_sum(const void* in, int dt, int64_t rows, int cols, int64_t l
   const int parts = rows == 0 ? 1 : static_cast<int>((rows + rows_per - 1) / rows_per);
   if (rows == 0) return cudaMemsetAsync(out, 0, sizeof(float) * cols, st);
   dim3 grid((cols + 255) / 256, parts);
-  if (dt == kDtF32) colsum_partial_kernel<kDtF32><<<grid, 256, 0, st>>>(in, rows, cols, ld, rows_per, partial);
-  else if (dt == kDtBF16) colsum_partial_kernel<kDtBF16><<<grid, 256, 0, st>>>(in, rows, cols, ld, rows_per, partial);
-  else colsum_partial_kernel<kDtF16><<<grid, 256, 0, st>>>(in, rows, cols, ld, rows_per, partial);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e;
+  if (dt == kDtF32) e = launch_pdl(colsum_partial_kernel<kDtF32>, grid, dim3(256), 0, st, in, rows, cols, ld, rows_per, partial);
+  else if (dt == kDtBF16)
+    e = launch_pdl(colsum_partial_kernel<kDtBF16>, grid, dim3(256), 0, st, in, rows, cols, ld, rows_per, partial);
+  else e = launch_pdl(colsum_partial_kernel<kDtF16>, grid, dim3(256), 0, st, in, rows, cols, ld, rows_per, partial);
   if (e != cudaSuccess) return e;
-  colsum_final_kernel<<<(cols + 31) / 32, 256, 0, st>>>(partial, parts, cols, out);
-  return cudaGetLastError();
+  return launch_pdl(colsum_final_kernel, dim3((cols + 31) / 32), dim3(256), 0, st, static_cast<const float*>(partial), parts,
+                    cols, out);
 }
 
 }  // namespace hstu

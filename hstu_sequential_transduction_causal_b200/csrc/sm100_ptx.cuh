@@ -92,6 +92,26 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// The same wait for a whole warp: lane 0 waits, every lane gets its verdict and the warp is
+// reconverged (a producer warp then issues TMA copies from several lanes: an issuing thread keeps
+// about one tile copy in flight, so spreading a stage's copies over lanes overlaps them).
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort,
+                                               const WaitCtl& ctl) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, ctl);
+  ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+  __syncwarp();
+  return ok;
+}
+
+// Programmatic dependent launch: lets the stream's next kernel start launching into SMs this grid
+// frees, then waits until every grid this one depends on has completed and its writes are
+// visible. First statement of every kernel launched with launch_pdl (a no-op otherwise).
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------------------------------------
 // Proxy fences, named barriers
 // ------------------------------------------------------------------------------------------------
@@ -359,6 +379,14 @@ __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
 // result is a denormal-sized value instead of exactly 0, far below bf16 resolution.
 __device__ __forceinline__ float silu_fast(float x) {
   return __fdividef(x, 1.0f + __expf(fminf(-x, 80.0f)));
+}
+
+// SiLU(x) = h + h tanh(h), h = x / 2, with one hardware tanh (one MUFU operation instead of the
+// exponential and the reciprocal above; tanh.approx.f32 has a relative error near 2^-11, the
+// resolution of the 16-bit activations it feeds).
+__device__ __forceinline__ float silu_tanh(float x) {
+  const float h = 0.5f * x;
+  return fmaf(h, tanh_f32_approx(h), h);
 }
 
 }  // namespace hstu
