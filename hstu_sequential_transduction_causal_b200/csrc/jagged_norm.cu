@@ -177,6 +177,63 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
   if (tid == 0) pair_base[B] = s_run;
 }
 
+// The same lists for batches of at most 32 sequences, from a single warp (no block barriers):
+// lane b owns sequence b; the items are written tile index by tile index, longest first, as above.
+__global__ void __launch_bounds__(32)
+worklist_warp_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items, int32_t* count,
+                     int* status, long long* pair_base, int32_t* kitems, int32_t* kcount) {
+  pdl_enter();
+  const int lane = threadIdx.x;
+  const bool mine = lane < B;
+  long long n = 0;
+  if (mine) n = off[lane + 1] - off[lane];
+  bool bad = (B < 0 || B > 32 || off[0] != 0 || off[B > 0 ? B : 0] != T || (mine && (n < 0 || n > max_len)));
+  bad = __any_sync(0xffffffffu, bad);
+  if (bad) {
+    if (lane == 0) {
+      *count = 0;
+      if (kcount) *kcount = 0;
+      report_error(status, kDevBadInput);
+      if (pair_base) pair_base[B > 0 && B <= 32 ? B : 0] = 0;
+    }
+    return;
+  }
+  const int nt = mine ? static_cast<int>((n + kQTile - 1) / kQTile) : 0;
+  int max_tiles = nt;
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) max_tiles = max(max_tiles, __shfl_xor_sync(0xffffffffu, max_tiles, d));
+  int base = 0;
+  for (int t = max_tiles - 1; t >= 0; --t) {
+    const bool flag = nt > t;
+    const unsigned m = __ballot_sync(0xffffffffu, flag);
+    if (flag) {
+      const int pos = base + __popc(m & ((1u << lane) - 1u));
+      items[2 * pos] = lane;
+      items[2 * pos + 1] = t;
+      if (kitems) {
+        kitems[2 * pos] = lane;
+        kitems[2 * pos + 1] = nt - 1 - t;
+      }
+    }
+    base += __popc(m);
+  }
+  if (lane == 0) {
+    *count = base;
+    if (kcount) *kcount = base;
+  }
+  if (!pair_base) return;
+  const long long v = static_cast<long long>(nt) * (nt + 1) / 2;
+  long long inc = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += y;
+  }
+  if (mine) pair_base[lane] = inc - v;
+  const long long total = __shfl_sync(0xffffffffu, inc, 31);
+  if (lane == 0) pair_base[B] = total;
+}
+
 // One warp per query row: writes bucket(t_i - t_j) for every key j of the row's sequence.
 __global__ void __launch_bounds__(256)
 time_bucket_kernel(const int64_t* __restrict__ off, const int64_t* __restrict__ ts, int B, int64_t T,
@@ -282,6 +339,9 @@ cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
                             int32_t* count, int* status, cudaStream_t st, long long* pair_base, int32_t* kitems,
                             int32_t* kcount) {
+  if (B >= 0 && B <= 32)
+    return launch_pdl(worklist_warp_kernel, dim3(1), dim3(32), 0, st, offsets, B, T, max_len, items, count, status,
+                      pair_base, kitems, kcount);
   return launch_pdl(worklist_kernel, dim3(1), dim3(1024), 0, st, offsets, B, T, max_len, items, count, status,
                     pair_base, kitems, kcount);
 }

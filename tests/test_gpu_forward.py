@@ -36,8 +36,12 @@ def _silu_like(rng, shape):
 # integer steps: bit-exact
 # ---------------------------------------------------------------------------------------------
 
-def test_worklist_bit_exact():
-    lengths = [0, 1, 127, 128, 129, 300, 1024, 5, 0, 700, 256, 257]
+@pytest.mark.parametrize("lengths", [
+    [0, 1, 127, 128, 129, 300, 1024, 5, 0, 700, 256, 257],                     # one-warp path (B <= 32)
+    [129 * (i % 7) + (i % 3) for i in range(32)],                              # one-warp path, B = 32
+    [37 * i % 1025 for i in range(45)],                                        # block path (B > 32)
+])
+def test_worklist_bit_exact(lengths):
     off = W.offsets_from_lengths(lengths)
     jag = JaggedBatch(off, np.zeros(off[-1], np.int64), max_len=1024)
     cap = H.hstu_worklist_capacity(jag.struct)
