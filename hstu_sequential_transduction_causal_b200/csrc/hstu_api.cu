@@ -697,10 +697,15 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   const void* x_op = x_f16 ? x_f16 : wsb + lay.x_f16;
   void* w1_f16 = wsb + lay.w1_f16;
   void* w2_f16 = wsb + lay.w2_f16;
-  if (!dy_f16) e = convert_dtype(dy, y_dt, wsb + lay.dy_f16, kDtF16, T * D, st);
-  if (e == cudaSuccess && !x_f16) e = convert_dtype(x, x_dt, wsb + lay.x_f16, kDtF16, T * D, st);
-  if (e == cudaSuccess) e = convert_dtype(w->W1, kDtBF16, w1_f16, kDtF16, 4ll * D * D, st);
-  if (e == cudaSuccess) e = convert_dtype(w->W2, kDtBF16, w2_f16, kDtF16, 1ll * D * D, st);
+  {   // the fp16 GEMM operand copies, one launch
+    ConvertJob jobs[4];
+    int nj = 0;
+    if (!dy_f16) jobs[nj++] = ConvertJob{dy, wsb + lay.dy_f16, T * D, y_dt};
+    if (!x_f16) jobs[nj++] = ConvertJob{x, wsb + lay.x_f16, T * D, x_dt};
+    jobs[nj++] = ConvertJob{w->W1, w1_f16, 4ll * D * D, kDtBF16};
+    jobs[nj++] = ConvertJob{w->W2, w2_f16, 1ll * D * D, kDtBF16};
+    e = convert_many_to_f16(jobs, nj, st);
+  }
   if (e != cudaSuccess) return cuda_status(e);
   float* dG = reinterpret_cast<float*>(wsb + lay.dg);
   void* dO = wsb + lay.dO;

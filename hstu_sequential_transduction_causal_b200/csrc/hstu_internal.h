@@ -197,6 +197,14 @@ cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const flo
                         const void* z, int64_t ld_z, void* dz, int64_t ld_dz, cudaStream_t st);
 size_t colsum_partial_floats(int cols);
 cudaError_t convert_dtype(const void* in, int in_dt, void* out, int out_dt, int64_t n, cudaStream_t st);
+// Up to four conversions to fp16 (inputs fp32, bf16 or fp16) in one launch.
+struct ConvertJob {
+  const void* in;
+  void* out;
+  int64_t n;
+  int in_dt;
+};
+cudaError_t convert_many_to_f16(const ConvertJob* jobs, int njobs, cudaStream_t st);
 cudaError_t column_sum(const void* in, int dt, int64_t rows, int cols, int64_t ld, float* partial, float* out,
                        cudaStream_t st);
 

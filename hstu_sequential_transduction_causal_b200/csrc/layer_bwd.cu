@@ -126,13 +126,22 @@ colsum_partial_kernel(const void* __restrict__ in, int64_t rows, int cols, int64
   if (c >= cols) return;
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per;
   const int64_t r1 = r0 + rows_per < rows ? r0 + rows_per : rows;
-  float s = 0.0f;
-  for (int64_t r = r0; r < r1; ++r) {
+  // four independent accumulators: four loads in flight per thread
+  float s[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  int64_t r = r0;
+  for (; r + 4 <= r1; r += 4) {
+    float v[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) load_vec<1, DT>(in, (r + q) * ld + c, &v[q]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) s[q] += v[q];
+  }
+  for (; r < r1; ++r) {
     float v;
     load_vec<1, DT>(in, r * ld + c, &v);
-    s += v;
+    s[0] += v;
   }
-  partial[static_cast<int64_t>(blockIdx.y) * cols + c] = s;
+  partial[static_cast<int64_t>(blockIdx.y) * cols + c] = (s[0] + s[1]) + (s[2] + s[3]);
 }
 
 // out[i] = in[i] converted between fp32 / bf16 / fp16, 8 elements per thread (scalar tail).
@@ -229,6 +238,58 @@ cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const flo
   return cudaErrorInvalidValue;
 }
 
+struct ConvertBatch {
+  ConvertJob job[4];
+  int first_block[5];   // block b converts job j with first_block[j] <= b < first_block[j + 1]
+  int njobs;
+};
+
+// Several tensors converted to fp16 by one launch: each block finds its job, then 8 elements per
+// thread as in convert_kernel.
+__global__ void __launch_bounds__(256)
+convert_many_kernel(ConvertBatch cb) {
+  pdl_enter();
+  int j = 0;
+  while (j + 1 < cb.njobs && static_cast<int>(blockIdx.x) >= cb.first_block[j + 1]) ++j;
+  const ConvertJob& jb = cb.job[j];
+  const int64_t i = (static_cast<int64_t>(blockIdx.x - cb.first_block[j]) * blockDim.x + threadIdx.x) * 8;
+  if (i >= jb.n) return;
+  const int cnt = jb.n - i >= 8 ? 8 : static_cast<int>(jb.n - i);
+  float v[8];
+  if (cnt == 8) {
+    if (jb.in_dt == kDtF32) load_vec<8, kDtF32>(jb.in, i, v);
+    else if (jb.in_dt == kDtBF16) load_vec<8, kDtBF16>(jb.in, i, v);
+    else load_vec<8, kDtF16>(jb.in, i, v);
+    store_vec<8, kDtF16>(jb.out, i, v);
+  } else {
+    for (int k = 0; k < cnt; ++k) {
+      if (jb.in_dt == kDtF32) load_vec<1, kDtF32>(jb.in, i + k, &v[0]);
+      else if (jb.in_dt == kDtBF16) load_vec<1, kDtBF16>(jb.in, i + k, &v[0]);
+      else load_vec<1, kDtF16>(jb.in, i + k, &v[0]);
+      reinterpret_cast<__half*>(jb.out)[i + k] = __float2half_rn(v[0]);
+    }
+  }
+}
+
+cudaError_t convert_many_to_f16(const ConvertJob* jobs, int njobs, cudaStream_t st) {
+  ConvertBatch cb{};
+  int nb = 0, k = 0;
+  for (int j = 0; j < njobs && j < 4; ++j) {
+    if (jobs[j].n <= 0) continue;
+    if (jobs[j].in_dt != kDtF32 && jobs[j].in_dt != kDtBF16 && jobs[j].in_dt != kDtF16) return cudaErrorInvalidValue;
+    cb.job[k] = jobs[j];
+    cb.first_block[k] = nb;
+    const int64_t blocks = ((jobs[j].n + 7) / 8 + 255) / 256;
+    if (nb + blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+    nb += static_cast<int>(blocks);
+    ++k;
+  }
+  if (k == 0) return cudaSuccess;
+  cb.first_block[k] = nb;
+  cb.njobs = k;
+  return launch_pdl(convert_many_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, st, cb);
+}
+
 cudaError_t convert_dtype(const void* in, int in_dt, void* out, int out_dt, int64_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const unsigned blocks = static_cast<unsigned>(((n + 7) / 8 + 255) / 256);
@@ -244,14 +305,18 @@ cudaError_t convert_dtype(const void* in, int in_dt, void* out, int out_dt, int6
   return cudaErrorInvalidValue;
 }
 
-constexpr int kColsumParts = 64;
+constexpr int kColsumParts = 256;   // most row slices of a column sum (the partial buffer's height)
 
 size_t colsum_partial_floats(int cols) { return static_cast<size_t>(kColsumParts) * cols; }
 
 cudaError_t column_sum(const void* in, int dt, int64_t rows, int cols, int64_t ld, float* partial, float* out,
                        cudaStream_t st) {
   if (cols == 0) return cudaSuccess;
-  const int64_t rows_per = (rows + kColsumParts - 1) / kColsumParts;
+  // about four blocks per SM: more row slices when there are few column blocks
+  const int col_blocks = (cols + 255) / 256;
+  int want = (4 * 148 + col_blocks - 1) / col_blocks;
+  want = want < 32 ? 32 : (want > kColsumParts ? kColsumParts : want);
+  const int64_t rows_per = (rows + want - 1) / want;
   const int parts = rows == 0 ? 1 : static_cast<int>((rows + rows_per - 1) / rows_per);
   if (rows == 0) return cudaMemsetAsync(out, 0, sizeof(float) * cols, st);
   dim3 grid((cols + 255) / 256, parts);

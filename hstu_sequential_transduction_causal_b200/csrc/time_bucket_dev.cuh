@@ -31,12 +31,14 @@ __device__ __forceinline__ int time_bucket_dev(long long dt, const long long* ta
 // reached) and tau32[0] = INT32_MIN; all arithmetic is 32-bit.
 __constant__ int c_time_taus32[kTauEntries];
 
+// Branch-free: dt <= 1 is clamped to 1, whose estimate is 0 and whose corrections are both 0
+// (tau[1] = 2 > 1, tau[0] = INT32_MIN), so bucket 0 falls out of the general path.
 __device__ __forceinline__ int time_bucket32(int dt, const int* tau, int nb) {
-  if (dt <= 1) return 0;
+  const int v = max(dt, 1);
   constexpr float kLn2Over0301 = 0.693147180559945f / 0.301f;
-  const float lf = __log2f(static_cast<float>(dt)) * kLn2Over0301;
+  const float lf = __log2f(static_cast<float>(v)) * kLn2Over0301;
   int k = min(static_cast<int>(lf), 126);
-  k += (dt >= tau[k + 1] ? 1 : 0) - (dt < tau[k] ? 1 : 0);
+  k += (v >= tau[k + 1] ? 1 : 0) - (v < tau[k] ? 1 : 0);
   return min(k, nb - 1);
 }
 
