@@ -28,7 +28,8 @@ __device__ __forceinline__ float silu_grad(float z) {
   return s * (1.0f + z * (1.0f - s));
 }
 
-// One warp per token row (grid-stride over rows); lane l holds features [l VPT, (l+1) VPT).
+// One warp per token row (grid-stride over rows); lane l holds features 128 k + 4 l + i (k < VPT / 4,
+// i < 4): every load and store of the warp covers 128 consecutive features (coalesced).
 // Writes dO (act dtype), dZ_U = dU (.) SiLU'(Z_U) (fp16, row stride ld_dz) and per-block partial
 // sums of dgamma | dbeta into partial[blockIdx.x][0 .. 2D).
 template <int VPT, int AT>
@@ -39,20 +40,29 @@ norm_gate_bwd_kernel(int64_t T, const float* __restrict__ dg, const float* __res
                      void* __restrict__ d_o, void* __restrict__ dz, int64_t ld_dz, float* __restrict__ partial) {
   pdl_enter();
   constexpr int D = VPT * 32;
+  constexpr int KG = VPT / 4;   // groups of 4 features per lane
   __shared__ float s_red[8][2][D];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  auto feat = [&](int e) { return 128 * (e >> 2) + 4 * lane + (e & 3); };
   float gacc[VPT], bacc[VPT];
 #pragma unroll
   for (int e = 0; e < VPT; ++e) gacc[e] = bacc[e] = 0.0f;
   float gm[VPT], bt[VPT];
-  load_vec<VPT, kDtF32>(gamma, lane * VPT, gm);
-  load_vec<VPT, kDtF32>(beta, lane * VPT, bt);
+#pragma unroll
+  for (int k = 0; k < KG; ++k) {
+    load_vec<4, kDtF32>(gamma, 128 * k + 4 * lane, gm + 4 * k);
+    load_vec<4, kDtF32>(beta, 128 * k + 4 * lane, bt + 4 * k);
+  }
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp; row < T; row += static_cast<int64_t>(gridDim.x) * 8) {
     float g[VPT], x[VPT], uu[VPT], z[VPT];
-    load_vec<VPT, kDtF32>(dg, row * D + lane * VPT, g);
-    load_vec<VPT, kDtF32>(o, row * D + lane * VPT, x);
-    load_vec<VPT, AT>(u, row * ld_act + lane * VPT, uu);
-    load_vec<VPT, AT>(zu, row * ld_act + lane * VPT, z);
+#pragma unroll
+    for (int k = 0; k < KG; ++k) {
+      const int c = 128 * k + 4 * lane;
+      load_vec<4, kDtF32>(dg, row * D + c, g + 4 * k);
+      load_vec<4, kDtF32>(o, row * D + c, x + 4 * k);
+      load_vec<4, AT>(u, row * ld_act + c, uu + 4 * k);
+      load_vec<4, AT>(zu, row * ld_act + c, z + 4 * k);
+    }
     const float m = mu[row], rs = rstd[row];
     float s1 = 0.0f, s2 = 0.0f;
 #pragma unroll
@@ -77,13 +87,17 @@ norm_gate_bwd_kernel(int64_t T, const float* __restrict__ dg, const float* __res
     const float m1 = s1 * (1.0f / D), m2 = s2 * (1.0f / D);
 #pragma unroll
     for (int e = 0; e < VPT; ++e) g[e] = rs * (g[e] - m1 - x[e] * m2);
-    store_vec<VPT, AT>(d_o, row * D + lane * VPT, g);
-    store_vec<VPT, kDtF16>(dz, row * ld_dz + lane * VPT, z);
+#pragma unroll
+    for (int k = 0; k < KG; ++k) {
+      const int c = 128 * k + 4 * lane;
+      store_vec<4, AT>(d_o, row * D + c, g + 4 * k);
+      store_vec<4, kDtF16>(dz, row * ld_dz + c, z + 4 * k);
+    }
   }
 #pragma unroll
   for (int e = 0; e < VPT; ++e) {
-    s_red[warp][0][lane * VPT + e] = gacc[e];
-    s_red[warp][1][lane * VPT + e] = bacc[e];
+    s_red[warp][0][feat(e)] = gacc[e];
+    s_red[warp][1][feat(e)] = bacc[e];
   }
   __syncthreads();
   for (int c = threadIdx.x; c < 2 * D; c += 256) {

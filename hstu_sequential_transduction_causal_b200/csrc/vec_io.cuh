@@ -42,6 +42,11 @@ __device__ __forceinline__ void load_vec(const void* base, int64_t idx, float* v
           v[8 * q + 2 * e + 1] = f.y;
         }
       }
+    } else if constexpr (VPT == 4) {   // one 8-byte load
+      const uint2 t = *reinterpret_cast<const uint2*>(p);
+      const float2 f0 = DT == kDtBF16 ? unpack_bf16x2(t.x) : unpack_f16x2(t.x);
+      const float2 f1 = DT == kDtBF16 ? unpack_bf16x2(t.y) : unpack_f16x2(t.y);
+      v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
     } else {
 #pragma unroll
       for (int e = 0; e < VPT; e += 2) {
@@ -74,6 +79,8 @@ __device__ __forceinline__ void store_vec(void* base, int64_t idx, const float* 
       for (int q = 0; q < VPT / 8; ++q)
         reinterpret_cast<uint4*>(p)[q] = make_uint4(pk(v[8 * q], v[8 * q + 1]), pk(v[8 * q + 2], v[8 * q + 3]),
                                                     pk(v[8 * q + 4], v[8 * q + 5]), pk(v[8 * q + 6], v[8 * q + 7]));
+    } else if constexpr (VPT == 4) {   // one 8-byte store
+      *reinterpret_cast<uint2*>(p) = make_uint2(pk(v[0], v[1]), pk(v[2], v[3]));
     } else {
 #pragma unroll
       for (int e = 0; e < VPT; e += 2) reinterpret_cast<uint32_t*>(p)[e / 2] = pk(v[e], v[e + 1]);
