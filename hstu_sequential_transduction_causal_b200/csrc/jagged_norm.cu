@@ -256,8 +256,9 @@ time_bucket_kernel(const int64_t* __restrict__ off, const int64_t* __restrict__ 
 // ----------------------------------------------------------------------------------------------
 // LayerNorm (.) U ("4.4 Scaling Recommendation Models", Generative Recommenders and HSTU, third
 // equation Norm(AV) (.) U; "HSTU: The First Exploration of the Scaling Law", 7.1.4 Innovation 3):
-// one warp per token, lane l holds features [l*VPT, (l+1)*VPT); mean and variance by warp
-// shuffles (two passes over registers), fp32 statistics stored for the backward.
+// one warp per token (lane l holds 4-feature groups 4 l + 128 k, or [l VPT, (l+1) VPT) for small D);
+// mean and variance by warp shuffles (two passes over registers), fp32 statistics stored for the
+// backward.
 // ----------------------------------------------------------------------------------------------
 template <int VPT, int OT, int UT, int GT>
 __global__ void __launch_bounds__(256)
@@ -269,9 +270,17 @@ norm_gate_kernel(int64_t T, const void* __restrict__ o, int64_t ld_o, const void
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= T) return;
+  // D >= 128: lane l holds features 128 k + 4 l + i (every warp access covers 128 consecutive
+  // features); smaller D: features [l VPT, (l+1) VPT)
+  constexpr bool kGrouped = VPT % 4 == 0;
+  auto col = [&](int k) { return kGrouped ? 128 * k + 4 * lane : lane * VPT; };
+  constexpr int KG = kGrouped ? VPT / 4 : 1, W = kGrouped ? 4 : VPT;
   float x[VPT], uu[VPT];
-  load_vec<VPT, OT>(o, row * ld_o + lane * VPT, x);
-  load_vec<VPT, UT>(u, row * ld_u + lane * VPT, uu);
+#pragma unroll
+  for (int k = 0; k < KG; ++k) {
+    load_vec<W, OT>(o, row * ld_o + col(k), x + W * k);
+    load_vec<W, UT>(u, row * ld_u + col(k), uu + W * k);
+  }
   float s = 0.0f;
 #pragma unroll
   for (int e = 0; e < VPT; ++e) s += x[e];
@@ -288,11 +297,15 @@ norm_gate_kernel(int64_t T, const void* __restrict__ o, int64_t ld_o, const void
   for (int m = 16; m > 0; m >>= 1) q += __shfl_xor_sync(0xffffffffu, q, m);
   const float rstd = rsqrtf(q * (1.0f / D) + eps);
   float gm[VPT], bt[VPT];
-  load_vec<VPT, kDtF32>(gamma, lane * VPT, gm);
-  load_vec<VPT, kDtF32>(beta, lane * VPT, bt);
+#pragma unroll
+  for (int k = 0; k < KG; ++k) {
+    load_vec<W, kDtF32>(gamma, col(k), gm + W * k);
+    load_vec<W, kDtF32>(beta, col(k), bt + W * k);
+  }
 #pragma unroll
   for (int e = 0; e < VPT; ++e) x[e] = fmaf((x[e] - mean) * rstd, gm[e], bt[e]) * uu[e];
-  store_vec<VPT, GT>(g, row * D + lane * VPT, x);
+#pragma unroll
+  for (int k = 0; k < KG; ++k) store_vec<W, GT>(g, row * D + col(k), x + W * k);
   if (lane == 0) {
     if (mu_out) mu_out[row] = mean;
     if (rstd_out) rstd_out[row] = rstd;
