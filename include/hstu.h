@@ -220,7 +220,12 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
                             const float* rab_time, void* out, void* ws, size_t ws_bytes,
                             hstu_stream_t stream);
 
-/* Workspace bytes hstu_attn_bwd needs for this batch. */
+/* Workspace bytes hstu_attn_bwd needs for this batch: the work lists, per causal (query tile, key
+ * tile) pair a transposed fp16 half-bias tile (32 KB) and a u8 bucket tile (16 KB), and per pair
+ * and head a 16-bit dX^T tile (32 KB) from which the table gradients are summed over the heads.
+ * The pair count is bounded from the batch's tile capacity and max_len (capacity (max_len/128 + 1)
+ * / 2 pairs), so the size grows with H, T and max_len: about 1.5 GB for 30k tokens, max_len 4096
+ * and 8 heads; 0.54 GB for 5.8k tokens, max_len 8192. */
 size_t hstu_attn_bwd_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag);
 
 /* Pointwise causal attention backward (derived from the forward's definition; tensor-core dtypes
