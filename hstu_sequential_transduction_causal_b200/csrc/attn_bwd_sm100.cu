@@ -12,7 +12,7 @@
 // [key][query] and the u8 time-bucket tile [key][query] (head independent, computed once).
 // attn_bwd_tc_kernel<F16>: one CTA per (sequence, 128-key tile, head), key tiles that visit the
 // most query tiles first; it walks the query tiles t >= its key tile:
-//   warp 16  : TMA: K, V once; Q and dO of each query tile (2 stages); the half-bias tile.
+//   warp 16  : TMA: K, V once; Q and dO of each query tile (3 stages); the half-bias tile (2).
 //   warp 17  : tcgen05: S^T = K Q^T and dA^T = V dO^T into TMEM.
 //   warp 19  : tcgen05: after the elementwise step dV += P^T dO (P^T from TMEM), dK += dX^T Q and
 //              dQ_tile = dX K (dX^T from shared memory, read K-major for dK and MN-major for dQ).
