@@ -201,7 +201,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       decode(t, m0, n0, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb, ++g) {
         const int s = g % STAGES;
-        bool free_ok = true;   // lane 0 waits; the verdict is made warp-uniform
+        bool free_ok = true;   // lane 0 waits; the result is made warp-uniform
         if (lane == 0 && g >= STAGES)
           free_ok = mbar_wait(smem_u32(&bars[STAGES + s]), ((g / STAGES) - 1) & 1, abort_flag, ctl);
         if (!__shfl_sync(0xffffffffu, free_ok ? 1 : 0, 0)) {

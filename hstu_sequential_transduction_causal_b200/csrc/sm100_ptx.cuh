@@ -92,7 +92,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// The same wait for a whole warp: lane 0 waits, every lane gets its verdict and the warp is
+// The same wait for a whole warp: lane 0 waits, every lane gets its result and the warp is
 // reconverged (a producer warp then issues TMA copies from several lanes: an issuing thread keeps
 // about one tile copy in flight, so spreading a stage's copies over lanes overlaps them).
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort,

@@ -24,7 +24,7 @@ Pages followed (cited by title and section):
   time differences), "Innovation 3" (Norm(AV) (.) U gating); section 7.1.5 "Stochastic
   Length" and "M-FALCON" (candidates see the cached history, not each other).
 
-Readings where the pages are silent, garbled or disagree (each is also listed in the design doc):
+Readings where the pages are silent, garbled or disagree:
 
 R1  No input LayerNorm before f1 (the equations have none; the sketch's extra one is a variant).
 R2  N is a constant runtime scalar (``inv_N`` = 1/N), never the per-batch maximum length.
