@@ -154,7 +154,7 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 }
 __device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// 2D tile load (no multicast). x is the innermost coordinate (elements), y the row.
+// 2D tile load into this CTA's shared memory. x is the innermost coordinate (elements), y the row.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int32_t x, int32_t y) {
   asm volatile(
