@@ -424,7 +424,8 @@ hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype
   if (ws_bytes < kWsHeader) return HSTU_ERR_WORKSPACE;
   if (T == 0) return HSTU_OK;
   if (!x || !W1 || !uvqk || ld_x < D) return HSTU_ERR_INVALID_ARG;
-  if (dtype == HSTU_BF16 && (ld_x % 8 || !aligned16(x) || !aligned16(W1) || !aligned16(uvqk) || (z && !aligned16(z))))
+  if (dtype == HSTU_BF16 && (ld_x % 8 || !aligned16(x) || !aligned16(W1) || !aligned16(uvqk) || (z && !aligned16(z)) ||
+                             (b1 && !aligned16(b1))))
     return HSTU_ERR_UNSUPPORTED;
   return run_uvqk(T, D, dtype, act_dtype, x, ld_x, W1, b1, uvqk, z, ws_status(ws), stream);
 }
@@ -512,7 +513,8 @@ hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_d
   if (dtype == HSTU_F32 && (x_dtype != HSTU_F32 || y_dtype != HSTU_F32 || y_f16)) return HSTU_ERR_UNSUPPORTED;
   if (T == 0) return HSTU_OK;
   if (!g || !W2 || !x || !y) return HSTU_ERR_INVALID_ARG;
-  if (!aligned16(g) || !aligned16(W2) || !aligned16(x) || !aligned16(y) || (y_f16 && !aligned16(y_f16)))
+  if (!aligned16(g) || !aligned16(W2) || !aligned16(x) || !aligned16(y) || (y_f16 && !aligned16(y_f16)) ||
+      (dtype == HSTU_BF16 && b2 && !aligned16(b2)))
     return HSTU_ERR_UNSUPPORTED;
   return run_out_proj(T, D, dtype, g_dtype, g, W2, b2, x, x_dtype, y, y_dtype, y_f16, ws_status(ws), stream,
                       static_cast<uint8_t*>(ws) + kWsHeader);
@@ -570,8 +572,9 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   if (!x || !y || !w->W1 || !w->b1 || !w->W2 || !w->b2 || !w->gamma || !w->beta || !w->rab_pos || !w->rab_time ||
       !saved->uvqk || !saved->o || !saved->g || !saved->mu || !saved->rstd)
     return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(w->gamma) || !aligned16(w->beta)) return HSTU_ERR_UNSUPPORTED;   // vector loads in both modes
   if (desc->dtype == HSTU_BF16) {   // 16-byte vector and TMA access
-    const void* v16[] = {x, x_f16, y, y_f16, saved->uvqk, saved->z, saved->o, saved->g, w->W1, w->W2};
+    const void* v16[] = {x, x_f16, y, y_f16, saved->uvqk, saved->z, saved->o, saved->g, w->W1, w->W2, w->b1, w->b2};
     for (const void* p : v16)
       if (p && !aligned16(p)) return HSTU_ERR_UNSUPPORTED;
   }
@@ -624,9 +627,14 @@ hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
   if (M >= (1ll << 31) || N >= (1ll << 31) || K >= (1ll << 31)) return HSTU_ERR_UNSUPPORTED;
   if (out_dtype != HSTU_F32 && out_dtype != HSTU_BF16 && out_dtype != HSTU_F16) return HSTU_ERR_UNSUPPORTED;
   if (accumulate && (out_dtype != HSTU_F32 || bias || resid)) return HSTU_ERR_UNSUPPORTED;
-  if (resid && (!aligned16(resid) || (resid_dtype != HSTU_F32 && resid_dtype != HSTU_BF16 &&
-                                      resid_dtype != HSTU_F16)))
-    return HSTU_ERR_UNSUPPORTED;
+  if (lda < (a_mn ? M : K) || ldb < (b_mn ? N : K) || ld_out < N) return HSTU_ERR_INVALID_ARG;
+  if (bias && !aligned16(bias)) return HSTU_ERR_UNSUPPORTED;   // 16-byte vector loads in the epilogue
+  if (resid) {
+    if (resid_dtype != HSTU_F32 && resid_dtype != HSTU_BF16 && resid_dtype != HSTU_F16) return HSTU_ERR_UNSUPPORTED;
+    if (ld_resid < N) return HSTU_ERR_INVALID_ARG;
+    // residual rows are read 32 elements at a time by 16-byte vector loads
+    if (!aligned16(resid) || (ld_resid * (resid_dtype == HSTU_F32 ? 4 : 2)) % 16) return HSTU_ERR_UNSUPPORTED;
+  }
   GemmArgs g{};
   g.A = A; g.lda = lda; g.a_mn = a_mn != 0;
   g.B = B; g.ldb = ldb; g.b_mn = b_mn != 0; g.f16 = false;
@@ -681,10 +689,12 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   }
   if (!x || !dy || !dx || !saved->uvqk || !saved->z || !saved->o || !saved->g || !saved->mu || !saved->rstd)
     return HSTU_ERR_INVALID_ARG;
+  // the weights the backward reads (b1 and b2 are not needed: Z and Y already hold them)
+  if (!w->W1 || !w->W2 || !w->gamma || !w->beta || !w->rab_pos || !w->rab_time) return HSTU_ERR_INVALID_ARG;
   // 16-byte vector loads, stores and atomics (dW1 and dW2 are accumulated by float4 atomics)
   {
     const void* v16[] = {x, x_f16, dy, dy_f16, dx, dx_f16, saved->uvqk, saved->z, saved->o, saved->g,
-                         w->W1, w->W2, gr->dW1, gr->dW2};
+                         w->W1, w->W2, w->gamma, w->beta, gr->dW1, gr->dW2};
     for (const void* p : v16)
       if (p && !aligned16(p)) return HSTU_ERR_UNSUPPORTED;
   }
@@ -941,6 +951,9 @@ extern "C" hstu_status_t hstu_falcon_fwd(const hstu_falcon_desc_t* desc, const h
     const hstu_layer_weights_t& w = layers[l];
     if (!w.W1 || !w.b1 || !w.W2 || !w.b2 || !w.gamma || !w.beta || !w.rab_pos || !w.rab_time)
       return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(w.W1) || !aligned16(w.W2) || !aligned16(w.b1) || !aligned16(w.b2) || !aligned16(w.gamma) ||
+        !aligned16(w.beta))
+      return HSTU_ERR_UNSUPPORTED;
   }
   cudaStream_t st = stream;
   uint8_t* base = static_cast<uint8_t*>(ws);

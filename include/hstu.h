@@ -106,7 +106,10 @@ typedef struct hstu_layer_desc_t {
 } hstu_layer_desc_t;
 
 /* Layer parameters. W1 [4D, D] rows ordered U|V|Q|K, W2 [D, D], both of the compute dtype;
- * the vectors are fp32: b1 [4D], b2 [D], gamma [D], beta [D], rab_pos [2L-1], rab_time [nb]. */
+ * the vectors are fp32: b1 [4D], b2 [D], gamma [D], beta [D], rab_pos [2L-1], rab_time [nb].
+ * gamma and beta (always) and W1, W2, b1, b2 (BF16 mode) are read by 16-byte vector loads and must
+ * be 16-byte aligned (HSTU_ERR_UNSUPPORTED otherwise). The backward reads W1, W2, gamma, beta and
+ * the two tables, not b1 or b2. */
 typedef struct hstu_layer_weights_t {
   const void* W1;
   const float* b1;
@@ -199,8 +202,8 @@ hstu_status_t hstu_time_buckets(const hstu_jagged_t* jag, int32_t n_buckets,
  * ------------------------------------------------------------------------------------------- */
 
 /* f1 + SiLU + split ("Generative Recommenders and HSTU", first equation):
- * uvqk[t, :] = SiLU(x[t, :] W1^T + b1), [T, 4D] with row stride 4D; z (nullable) receives the
- * pre-activation. x and W1 have `dtype` (BF16 or F32); uvqk and z have act_dtype (F16 or BF16
+ * uvqk[t, :] = SiLU(x[t, :] W1^T + b1), [T, 4D] with row stride 4D; b1 (nullable: no bias; 16-byte
+ * aligned for BF16); z (nullable) receives the pre-activation. x and W1 have `dtype` (BF16 or F32); uvqk and z have act_dtype (F16 or BF16
  * for BF16 operands, F32 for F32); ld_x is x's row stride. ws: any workspace of at least 256
  * bytes (its status word receives device-side errors). */
 hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t act_dtype, const void* x,
@@ -280,8 +283,9 @@ hstu_status_t hstu_norm_gate_fwd(int64_t T, int32_t D, hstu_dtype_t o_dtype, hst
  * sketch): y = g W2^T + b2 + x. W2 has the compute dtype `dtype`; g has g_dtype (F32 compute: F32;
  * BF16 compute: BF16, or F16 with W2 read through an fp16 copy made in the workspace); x has
  * x_dtype; y has y_dtype; y_f16 (nullable) receives a second, fp16 copy of y (the next layer's
- * f1 operand when the residual stream is fp32). ws: at least hstu_out_proj_workspace_size(D, g_dtype)
- * bytes (status word, fp16 W2). F32 compute needs F32 x and y. */
+ * f1 operand when the residual stream is fp32). b2: nullable (no bias; 16-byte aligned for BF16).
+ * ws: at least hstu_out_proj_workspace_size(D, g_dtype) bytes (status word, fp16 W2). F32 compute
+ * needs F32 x and y. */
 size_t hstu_out_proj_workspace_size(int32_t D, hstu_dtype_t g_dtype);
 hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t g_dtype,
                                 const void* g, const void* W2, const float* b2, const void* x,
@@ -310,7 +314,10 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
  * as [M or N rows, K] (K-major); 1: stored row-major as [K rows, M or N] (MN-major, a transpose
  * for free). accumulate = 0: out = A B^T (+ bias[N]) (+ resid), out_dtype F32/BF16/F16;
  * accumulate = 1: out += A B^T in fp32 by atomics over K splits (bias and resid must be NULL).
- * N must be a multiple of 32, lda/ldb multiples of 8, pointers 16-byte aligned. ws: >= 256 bytes. */
+ * N must be a multiple of 32, lda/ldb multiples of 8, pointers (bias included) 16-byte aligned.
+ * lda >= K (K-major) or M (MN-major), ldb >= K or N, ld_out >= N, and with resid, ld_resid >= N
+ * (HSTU_ERR_INVALID_ARG otherwise) with ld_resid rows starting on 16-byte boundaries
+ * (HSTU_ERR_UNSUPPORTED otherwise). ws: >= 256 bytes. */
 hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
                                int32_t a_mn, const void* B, int64_t ldb, int32_t b_mn,
                                const float* bias, const void* resid, hstu_dtype_t resid_dtype,
