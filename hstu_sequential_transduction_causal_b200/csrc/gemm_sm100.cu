@@ -16,6 +16,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "hstu_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -403,13 +405,16 @@ gemm_f32_simt_kernel(const float* __restrict__ A, int64_t sam, int64_t sak, cons
   }
 }
 
+// SM count of the current device, cached per device (148 if it cannot be read).
 int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      n = 148;
-  }
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  const bool tracked = dev >= 0 && dev < 64;
+  int n = tracked ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (tracked) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 

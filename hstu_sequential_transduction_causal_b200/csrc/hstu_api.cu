@@ -7,6 +7,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/hstu.h"
@@ -17,20 +18,24 @@ namespace hstu {
 namespace {
 
 thread_local int32_t g_last_cuda_error = 0;
-unsigned long long g_wait_limit = 1ull << 31;
+std::atomic<unsigned long long> g_wait_limit{1ull << 31};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up on first use (again after a failed lookup).
 EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cache{nullptr};
+  EncodeTiledFn fn = cache.load(std::memory_order_acquire);
   if (!fn) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess) {
       fn = reinterpret_cast<EncodeTiledFn>(p);
+      cache.store(fn, std::memory_order_release);
+    }
   }
   return fn;
 }
@@ -282,7 +287,7 @@ hstu_status_t check_dense(int64_t T, int32_t D, hstu_dtype_t dtype) {
 
 }  // namespace
 
-WaitCtl wait_ctl(int* status) { return WaitCtl{status, g_wait_limit}; }
+WaitCtl wait_ctl(int* status) { return WaitCtl{status, g_wait_limit.load(std::memory_order_relaxed)}; }
 
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld_elems,
                          int box_inner, int box_outer, bool f16) {
@@ -372,7 +377,9 @@ const char* hstu_status_string(hstu_status_t s) {
 
 int32_t hstu_last_cuda_error(void) { return g_last_cuda_error; }
 
-void hstu_set_wait_limit(uint64_t cycles) { g_wait_limit = cycles ? cycles : (1ull << 31); }
+void hstu_set_wait_limit(uint64_t cycles) {
+  g_wait_limit.store(cycles ? cycles : (1ull << 31), std::memory_order_relaxed);
+}
 
 hstu_status_t hstu_sync_status(void* ws, hstu_stream_t stream, int32_t* device_status) {
   if (!ws || !device_status) return HSTU_ERR_INVALID_ARG;

@@ -9,6 +9,9 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "time_bucket_table.h"
 
 namespace hstu {
@@ -42,13 +45,19 @@ __device__ __forceinline__ int time_bucket32(int dt, const int* tau, int nb) {
   return min(k, nb - 1);
 }
 
-// Copies tau_0..tau_128 to this translation unit's constant bank, once per device.
+// Copies tau_0..tau_128 to this translation unit's constant bank, once per device. The copies are
+// synchronous, so the first call on a device must come before any stream capture. Safe to call from
+// several host threads: the upload is serialised and later calls only read a flag.
 inline cudaError_t upload_time_taus() {
-  static bool done[64] = {};
+  static std::atomic<bool> done[64];
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  const bool tracked = dev >= 0 && dev < 64;
+  if (tracked && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(mu);
+  if (tracked && done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
   long long taus[kTauEntries];
   taus[0] = -0x7fffffffffffffffLL - 1;
   for (int k = 1; k <= HSTU_TB_NUM_THRESHOLDS; ++k) taus[k] = kHstuTimeThresholds[k - 1];
@@ -58,7 +67,7 @@ inline cudaError_t upload_time_taus() {
   for (int k = 0; k < kTauEntries; ++k)
     taus32[k] = k == 0 ? (-0x7fffffff - 1) : (taus[k] > 0x7fffffffLL ? 0x7fffffff : static_cast<int>(taus[k]));
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_time_taus32, taus32, sizeof(taus32));
-  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  if (e == cudaSuccess && tracked) done[dev].store(true, std::memory_order_release);
   return e;
 }
 

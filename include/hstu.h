@@ -23,6 +23,12 @@
  *    *_workspace_size() returns. A workspace must be zero-filled once before its first use
  *    (it holds the device status word) and must not be shared by calls that overlap on the GPU.
  *  - Work is enqueued on `stream` (a cudaStream_t); calls return once it is enqueued.
+ *  - The first call that needs them on each device sets kernel attributes and copies constant
+ *    tables (the time-bucket thresholds) with synchronous CUDA calls. Make that first call outside
+ *    any stream capture; after it, every call can be captured into a CUDA graph. Calls from
+ *    several host threads are safe: the one-time setup is serialised, and hstu_last_cuda_error()
+ *    is kept per host thread. The only exception is the workspace: calls that overlap on the GPU
+ *    need workspaces of their own.
  *  - Matrices are row-major; ld_* arguments are row strides in ELEMENTS. bf16 tensors use the
  *    bfloat16 bit layout (uint16). Pointers handed to the tensor-core kernels must be 16-byte
  *    aligned and their row strides multiples of 8 elements (16 bytes).

@@ -428,3 +428,22 @@ def test_status_and_probe(L):
     for code, name in Hb.STATUS.items():
         assert L.hstu_status_string(code).decode() == name
     assert L.hstu_status_string(99).decode() == "HSTU_ERR_UNKNOWN"
+
+
+def test_last_cuda_error_is_per_host_thread(L):
+    """A CUDA failure on one host thread is not reported on another (the header's threading rule)."""
+    import threading
+
+    seen = {}
+
+    def fresh_thread():
+        seen["before"] = L.hstu_last_cuda_error()
+        seen["marked"] = _mark_launch(L)
+
+    _mark_encode(L)
+    mine = L.hstu_last_cuda_error()
+    t = threading.Thread(target=fresh_thread)
+    t.start()
+    t.join()
+    assert seen["before"] == 0 and seen["marked"] != 0
+    assert L.hstu_last_cuda_error() == mine != seen["marked"]
