@@ -108,3 +108,43 @@ def test_layer_bwd_rejects_misaligned_gradients_on_host(lib):
                          61 << 20, None, 62 << 20, None, ctypes.byref(Hb.hstu_layer_grads_t(*bad)), 63 << 20, need,
                          None)
     assert r == 2
+
+
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    """The boundary is usable from plain C: a C99 program that includes only include/hstu.h builds
+    with -Wall -Werror, links against libhstu.so and makes the calls that need no GPU."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_hstu.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "hstu.h"
+
+int main(void) {
+  if (hstu_abi_version() != HSTU_ABI_VERSION) return 1;
+  if (strcmp(hstu_status_string(HSTU_ERR_WORKSPACE), "HSTU_ERR_WORKSPACE") != 0) return 2;
+  hstu_jagged_t jag;
+  memset(&jag, 0, sizeof jag);
+  jag.B = -1;                                       /* malformed: refused on the host */
+  if (hstu_worklist_capacity(&jag) != -1) return 3;
+  hstu_attn_desc_t desc;
+  memset(&desc, 0, sizeof desc);
+  if (hstu_attn_fwd(&desc, &jag, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL) != HSTU_ERR_INVALID_ARG)
+    return 4;
+  int32_t st = 0;
+  if (hstu_sync_status(NULL, NULL, &st) != HSTU_ERR_INVALID_ARG) return 5;
+  printf("ok\n");
+  return 0;
+}
+''')
+    exe = tmp_path / "use_hstu"
+    libdir = os.path.dirname(B.LIB)
+    cmd = ["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+           str(src), "-o", str(exe), f"-L{libdir}", "-lhstu", f"-Wl,-rpath,{libdir}"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
