@@ -12,6 +12,7 @@ import os
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 from oracle import hstu_oracle as O
 from oracle.bruteforce import layer_fwd_scalar
@@ -117,6 +118,24 @@ def test_layer_matches_scalar_bruteforce(spread):
                           p.rab_time.tolist(), wl.offsets.tolist(), wl.timestamps.tolist(),
                           wl.H, inv_N, wl.pos_max_len)
     assert np.allclose(y, np.array(yb), rtol=1e-10, atol=1e-10)
+
+
+@settings(max_examples=40, deadline=None, derandomize=True)
+@given(lengths=st.lists(st.integers(0, 9), min_size=1, max_size=4), L=st.integers(2, 6),
+       H=st.sampled_from([1, 2]), dh=st.sampled_from([2, 3]), seed=st.integers(0, 2 ** 16), spread=st.booleans(),
+       inv_N=st.sampled_from([1.0, 0.25, 1.0 / 9.0]))
+def test_layer_matches_scalar_bruteforce_random_shapes(lengths, L, H, dh, seed, spread, inv_N):
+    """Seeded random shapes: empty and single-token sequences, one or two heads, odd head widths,
+    and position tables shorter than the sequences, so that the relative-position clamp at +-(L-1)
+    is taken in both the oracle and the scalar loops."""
+    wl, p = _tiny(lengths, D=H * dh, H=H, seed=seed, L=L, spread=spread)
+    y, _ = O.layer_fwd(wl.x, p, wl.offsets, wl.timestamps, wl.H, inv_N, wl.pos_max_len, THR)
+    yb = layer_fwd_scalar(wl.x.astype(float).tolist(), p.W1.astype(float).tolist(),
+                          p.b1.tolist(), p.W2.astype(float).tolist(), p.b2.tolist(),
+                          p.gamma.tolist(), p.beta.tolist(), p.rab_pos.tolist(),
+                          p.rab_time.tolist(), wl.offsets.tolist(), wl.timestamps.tolist(),
+                          wl.H, inv_N, wl.pos_max_len)
+    assert np.allclose(y, np.array(yb).reshape(y.shape), rtol=1e-10, atol=1e-10)
 
 
 def test_causality_later_tokens_do_not_leak():
@@ -233,8 +252,12 @@ def test_dense_formulation_of_the_first_page():
 # backward: central finite differences of the oracle's own forward
 # ---------------------------------------------------------------------------------------------
 
-def test_backward_matches_finite_differences():
-    wl, p = _tiny([3, 5, 1], D=8, H=2, seed=7, L=8, spread=True)
+@pytest.mark.parametrize("lengths,L", [([3, 5, 1], 8), ([9, 4, 1], 3)])
+def test_backward_matches_finite_differences(lengths, L):
+    """Central differences for every gradient. The second case has sequences longer than the
+    position table (L = 3), so many pairs share the clamped entry rab_pos[2L-2]; there every entry
+    of rab_pos is checked."""
+    wl, p = _tiny(lengths, D=8, H=2, seed=7, L=L, spread=True)
     inv_N = 0.5
     rng = np.random.default_rng(8)
     dy = rng.standard_normal((wl.T, wl.D))
@@ -259,6 +282,8 @@ def test_backward_matches_finite_differences():
             used = np.unique(O.time_bucket(
                 wl.timestamps[:, None] - wl.timestamps[None, :], THR))
             idx = np.union1d(idx[:5], used)
+        if pname == "rab_pos":
+            idx = np.arange(flat.size)
         for t in idx:
             old = flat[t]
             flat[t] = old + h
