@@ -2,7 +2,8 @@
 
 Pure Python loops over (token, feature), (sequence, head, i, j) with ``math.exp`` and exact
 ``decimal`` logarithms for the time buckets, written independently of ``hstu_oracle`` (no shared
-helper) so that it can pin that module on tiny inputs. Same readings R1-R9 as ``hstu_oracle``:
+helper) so that it can pin that module on tiny inputs. Same readings R1-R9 as ``hstu_oracle`` (listed
+in its header):
 no input LayerNorm, constant 1/N, causal j <= i, tables shared by heads,
 bucket = min(nb-1, floor(ln(max(dt,1))/0.301)), rab_pos index clip(i-j) + L - 1, U|V|Q|K split,
 affine LayerNorm over d_model with eps 1e-5, residual after f2.

@@ -215,7 +215,8 @@ def test_constant_v_hand_values():
 def test_dense_formulation_of_the_first_page():
     """The first page's sketch formulates one padded sequence densely: a per-head [n, n]
     position bias, causal lower triangle, division by n, LayerNorm over d_model, gate with U,
-    f2 and the residual (its extra input LayerNorm left out, reading R1; no time bias).
+    f2 and the residual (its extra input LayerNorm left out, reading R1 of oracle/hstu_oracle.py;
+    no time bias).
     Restated here with torch CPU ops and torch's LayerNorm; the oracle must agree."""
     n, D, H, L = 12, 16, 2, 16
     rng = np.random.default_rng(11)
@@ -300,9 +301,10 @@ def test_backward_matches_finite_differences(lengths, L):
 # M-FALCON, Stochastic Length, work list
 # ---------------------------------------------------------------------------------------------
 
-def test_falcon_equals_naive_last_row():
-    fw = W.make_falcon_workload(seed=4, users=2, prefix=6, m=3, b_m=2, D=8, H=2, layers=2,
-                                N=7, pos_max_len=8)
+def _check_falcon_against_naive(fw):
+    """Candidate c of user u must equal the last row of a plain causal stack run on the user's
+    prefix followed by that one candidate (timestamp = the request time), and the prefix outputs
+    the other rows."""
     yc, yp = O.falcon_fwd(fw.layers, fw.prefix_offsets, fw.prefix_ts, fw.prefix_x, fw.cand_x,
                           fw.request_ts, fw.m, fw.H, 1 / fw.N, fw.pos_max_len, THR)
     for u in range(fw.users):
@@ -315,6 +317,22 @@ def test_falcon_equals_naive_last_row():
                 xs, _ = O.layer_fwd(xs, p, off, ts, fw.H, 1 / fw.N, fw.pos_max_len, THR)
             assert np.allclose(yc[u * fw.m + c], xs[-1], rtol=1e-12, atol=1e-12)
             assert np.allclose(yp[s:e], xs[:-1], rtol=1e-12, atol=1e-12)
+
+
+def test_falcon_equals_naive_last_row():
+    _check_falcon_against_naive(W.make_falcon_workload(seed=4, users=2, prefix=6, m=3, b_m=2, D=8, H=2,
+                                                       layers=2, N=7, pos_max_len=8))
+
+
+@settings(max_examples=20, deadline=None, derandomize=True)
+@given(prefix_lengths=st.lists(st.integers(0, 7), min_size=1, max_size=3), m=st.integers(1, 3),
+       L=st.integers(2, 9), layers=st.integers(1, 2), seed=st.integers(0, 2 ** 16))
+def test_falcon_equals_naive_last_row_random_shapes(prefix_lengths, m, L, layers, seed):
+    """Ragged prefixes (empty and single-token ones included) and position tables shorter than a
+    prefix, so that a candidate's distance n - j to early prefix tokens is clamped as in a plain
+    causal sequence."""
+    _check_falcon_against_naive(W.make_falcon_workload(seed=seed, prefix_lengths=prefix_lengths, m=m, b_m=m,
+                                                       D=8, H=2, layers=layers, N=7, pos_max_len=L))
 
 
 def test_stochastic_length_counts_and_selection():
