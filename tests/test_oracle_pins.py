@@ -360,6 +360,33 @@ def test_stochastic_length_counts_and_selection():
             assert (j in sel) == (rank < L)
 
 
+@settings(max_examples=40, deadline=None, derandomize=True)
+@given(lens=st.lists(st.integers(0, 60), min_size=0, max_size=6), alpha=st.sampled_from([1.2, 1.6, 2.0]),
+       key_max=st.sampled_from([3, 1000, 2 ** 62]), seed=st.integers(0, 2 ** 16))
+def test_stochastic_length_random_shapes(lens, alpha, key_max, seed):
+    """Random jagged batches (empty ones included), few or many distinct keys: each sequence keeps
+    exactly stochastic_length_keep(n) tokens, in order, and they are the lowest in (key, position)."""
+    off = W.offsets_from_lengths(lens)
+    keys = np.random.default_rng(seed).integers(0, key_max, off[-1], dtype=np.int64)
+    new_off, kept = O.stochastic_length(off, keys, alpha)
+    assert len(new_off) == len(lens) + 1 and new_off[0] == 0 and new_off[-1] == len(kept)
+    for b, n_ in enumerate(lens):
+        L = O.stochastic_length_keep(n_, alpha)
+        sel = list(kept[new_off[b]:new_off[b + 1]] - off[b])
+        order = sorted(range(n_), key=lambda i: (keys[off[b] + i], i))
+        assert sel == sorted(order[:L])
+
+
+@settings(max_examples=40, deadline=None, derandomize=True)
+@given(lens=st.lists(st.integers(0, 700), min_size=0, max_size=8))
+def test_work_list_random_shapes(lens):
+    """Every (sequence, 128-row tile) once; longest remaining key range first, ties by sequence."""
+    off = W.offsets_from_lengths(lens)
+    wlst = O.tile_work_list(off, 128)
+    expect = sorted(((b, t) for b, n in enumerate(lens) for t in range(-(-n // 128))), key=lambda r: (-r[1], r[0]))
+    assert [tuple(int(v) for v in r) for r in wlst] == expect
+
+
 def test_work_list_invariants():
     off = W.offsets_from_lengths([0, 1, 128, 129, 700, 256])
     wlst = O.tile_work_list(off, 128)
