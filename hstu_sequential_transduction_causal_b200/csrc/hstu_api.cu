@@ -74,6 +74,16 @@ AttnWs attn_ws_layout(const hstu_jagged_t* j) {
 
 size_t attn_ws_bytes(const hstu_jagged_t* j) { return attn_ws_layout(j).total; }
 
+// The tile-pair kernels address their per-pair tiles by 32-bit TMA row coordinates: the forward's
+// bias tiles span max_pairs * 128 rows, the backward's dX^T tiles max_pairs * H * 128. A batch
+// beyond that (hundreds of GB of workspace) is refused on the host, before any size is computed
+// in size_t or anything is enqueued.
+constexpr int64_t kMaxTmaRows = 0x7fffffffLL;
+bool fwd_pairs_fit(const hstu_jagged_t* j) { return attn_ws_layout(j).max_pairs <= kMaxTmaRows / kQTile; }
+bool bwd_pairs_fit(const hstu_jagged_t* j, int H) {
+  return H > 0 && attn_ws_layout(j).max_pairs <= kMaxTmaRows / (static_cast<int64_t>(H) * kQTile);
+}
+
 // attention-backward workspace: the forward layout up to pair_base, then the key-tile work list,
 // the transposed fp16 bias tiles (32 KB per pair), the u8 bucket tiles (16 KB per pair) and the fp16
 // dX^T tiles of every (pair, head) (32 KB each) the table gradients are summed from.
@@ -438,8 +448,8 @@ hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype
 }
 
 size_t hstu_attn_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag) {
+  if (check_jagged(jag) != HSTU_OK || !fwd_pairs_fit(jag)) return 0;
   (void)desc;
-  if (check_jagged(jag) != HSTU_OK) return 0;
   return attn_ws_bytes(jag);
 }
 
@@ -448,6 +458,7 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
                             size_t ws_bytes, hstu_stream_t stream) {
   hstu_status_t s = check_attn(desc, jag);
   if (s != HSTU_OK) return s;
+  if (!fwd_pairs_fit(jag)) return HSTU_ERR_UNSUPPORTED;
   if (!ws) return HSTU_ERR_INVALID_ARG;
   if (ws_bytes < attn_ws_bytes(jag)) return HSTU_ERR_WORKSPACE;
   if (jag->T > 0 && (!q || !k || !v || !rab_pos || !rab_time || !out)) return HSTU_ERR_INVALID_ARG;
@@ -457,7 +468,7 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
 }
 
 size_t hstu_attn_bwd_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag) {
-  if (!desc || check_jagged(jag) != HSTU_OK) return 0;
+  if (!desc || check_jagged(jag) != HSTU_OK || !bwd_pairs_fit(jag, desc->H)) return 0;
   return attn_bwd_ws_layout(jag, desc->H).total;
 }
 
@@ -468,6 +479,7 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
   hstu_status_t s = check_attn(desc, jag);
   if (s != HSTU_OK) return s;
   if (!is_tc_dtype(desc->dtype)) return HSTU_ERR_UNSUPPORTED;
+  if (!bwd_pairs_fit(jag, desc->H)) return HSTU_ERR_UNSUPPORTED;
   if (!ws) return HSTU_ERR_INVALID_ARG;
   if (ws_bytes < attn_bwd_ws_layout(jag, desc->H).total) return HSTU_ERR_WORKSPACE;
   if (!d_rab_pos || !d_rab_time) return HSTU_ERR_INVALID_ARG;
@@ -550,7 +562,7 @@ LayerFwdWs layer_fwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) 
 }
 
 size_t hstu_layer_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag) {
-  if (!desc || check_jagged(jag) != HSTU_OK || desc->D <= 0) return 0;
+  if (!desc || check_jagged(jag) != HSTU_OK || desc->D <= 0 || !fwd_pairs_fit(jag)) return 0;
   return layer_fwd_layout(desc, jag).total;
 }
 
@@ -570,6 +582,7 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   ad.ld_q = ad.ld_k = ad.ld_v = 4ll * D; ad.ld_o = D;
   s = check_attn(&ad, jag);
   if (s != HSTU_OK) return s;
+  if (!fwd_pairs_fit(jag)) return HSTU_ERR_UNSUPPORTED;
   if (desc->dtype == HSTU_F32 && (desc->x_dtype != HSTU_F32 || desc->y_dtype != HSTU_F32 || y_f16))
     return HSTU_ERR_UNSUPPORTED;
   if (!ws) return HSTU_ERR_INVALID_ARG;
@@ -656,7 +669,7 @@ hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
 }
 
 size_t hstu_layer_bwd_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag) {
-  if (!desc || check_jagged(jag) != HSTU_OK) return 0;
+  if (!desc || check_jagged(jag) != HSTU_OK || !bwd_pairs_fit(jag, desc->H)) return 0;
   return layer_bwd_layout(desc, jag).total;
 }
 
@@ -677,6 +690,7 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   ad.ld_q = ad.ld_k = ad.ld_v = 4ll * D; ad.ld_o = D;
   s = check_attn(&ad, jag);
   if (s != HSTU_OK) return s;
+  if (!bwd_pairs_fit(jag, H)) return HSTU_ERR_UNSUPPORTED;
   if ((desc->x_dtype != HSTU_F32 && desc->x_dtype != HSTU_BF16) || (desc->y_dtype != HSTU_F32 && desc->y_dtype != HSTU_BF16))
     return HSTU_ERR_UNSUPPORTED;
   if (!ws) return HSTU_ERR_INVALID_ARG;
@@ -920,6 +934,7 @@ hstu_status_t check_falcon(const hstu_falcon_desc_t* d, const hstu_jagged_t* p) 
   if (d->pos_max_len <= 0 || !isfinite(d->inv_N)) return HSTU_ERR_INVALID_ARG;
   if (d->n_time_buckets < 1 || d->n_time_buckets > 128) return HSTU_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(d->users) * d->m >= (1ll << 31)) return HSTU_ERR_UNSUPPORTED;
+  if (!fwd_pairs_fit(p)) return HSTU_ERR_UNSUPPORTED;   // the prefix pass runs the causal layer
   return HSTU_OK;
 }
 

@@ -216,7 +216,10 @@ hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype
                             int64_t ld_x, const void* W1, const float* b1, void* uvqk, void* z,
                             void* ws, size_t ws_bytes, hstu_stream_t stream);
 
-/* Workspace bytes hstu_attn_fwd / hstu_attn_bwd need for this batch. */
+/* Workspace bytes hstu_attn_fwd needs for this batch; 0 when the batch is malformed or so large
+ * that its causal tile-pair bound times 128 rows exceeds 2^31 - 1 (the tile kernels' 32-bit row
+ * coordinates; such a batch would need hundreds of GB of workspace), which the calls refuse with
+ * HSTU_ERR_UNSUPPORTED. */
 size_t hstu_attn_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag);
 
 /* Pointwise causal attention forward ("Generative Recommenders and HSTU", second equation and
@@ -236,6 +239,8 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
  * / 2 pairs), so the size grows with H, T and max_len: about 1.5 GB for 30k tokens, max_len 4096
  * and 8 heads; 0.54 GB for 5.8k tokens, max_len 8192. */
 size_t hstu_attn_bwd_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag);
+/* (0 when the pair bound times H x 128 rows exceeds 2^31 - 1, which hstu_attn_bwd refuses with
+ * HSTU_ERR_UNSUPPORTED; same for hstu_layer_bwd_workspace_size.) */
 
 /* Pointwise causal attention backward (derived from the forward's definition; tensor-core dtypes
  * F16 / BF16 only). With x_ij = q_i.k_j + rab(i, j) and A_ij = SiLU(x_ij) inv_N on causal pairs:
@@ -298,7 +303,7 @@ hstu_status_t hstu_out_proj_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_d
                                 hstu_dtype_t x_dtype, void* y, hstu_dtype_t y_dtype,
                                 void* y_f16, void* ws, size_t ws_bytes, hstu_stream_t stream);
 
-/* Workspace bytes hstu_layer_fwd / hstu_layer_bwd need. */
+/* Workspace bytes hstu_layer_fwd needs (0 for a batch hstu_attn_workspace_size refuses). */
 size_t hstu_layer_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
 
 /* Whole layer forward: uvqk -> attention -> norm-gate -> out-projection, on `stream`.

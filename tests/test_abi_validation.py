@@ -39,6 +39,13 @@ def L():
     return Hb.lib()
 
 
+# Batches whose causal tile-pair bound exceeds the tile kernels' 32-bit row coordinates: 200M tokens at
+# max_len 8192 (51M pairs, beyond 2^31 / 128 for the forward), and 40M tokens (10M pairs: within the
+# forward's bound, beyond 2^31 / (H 128) for the backward with H = 2).
+HUGE_FWD = dict(T=200_000_000, max_len=8192)
+HUGE_BWD = dict(T=40_000_000, max_len=8192)
+
+
 def jag(B=2, T=300, max_len=200, **kw):
     j = Hb.hstu_jagged_t(B=B, max_len=max_len, T=T, offsets=fake(0), timestamps=fake(1))
     for k, v in kw.items():
@@ -179,7 +186,11 @@ def test_attn_fwd(L):
         ("out off 16 bytes", dict(out=fake(7) + 8), UNSUPPORTED),
         ("k off 16 bytes", dict(k=fake(3) + 2), UNSUPPORTED),
         ("no timestamps", dict(j=jag(timestamps=None)), INVALID),
+        ("tile-pair rows beyond 32 bits", dict(j=jag(**HUGE_FWD)), UNSUPPORTED),
+        ("the same on the CUDA-core path", dict(j=jag(**HUGE_FWD), d=attn_desc(dtype=F32, o_dtype=F32)), UNSUPPORTED),
     ])
+    assert L.hstu_attn_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag(**HUGE_FWD))) == 0
+    assert L.hstu_attn_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag(**HUGE_BWD))) > 0
     assert passes_host_checks(L, call, d=attn_desc(dtype=F32, d_qk=48, d_v=48))   # CUDA-core path: any d <= 64
 
 
@@ -199,8 +210,9 @@ def test_attn_bwd(L):
     need = L.hstu_attn_bwd_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag()))
     assert need > L.hstu_attn_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag()))
 
-    def call(d=None, q=fake(2), do=fake(5), dq=fake(8), drp=fake(11), drt=fake(12), ws=fake(13), ws_bytes=need):
-        return L.hstu_attn_bwd(ctypes.byref(d or attn_desc()), ctypes.byref(jag()), q, fake(3), fake(4), do, fake(6),
+    def call(d=None, j=None, q=fake(2), do=fake(5), dq=fake(8), drp=fake(11), drt=fake(12), ws=fake(13),
+             ws_bytes=need):
+        return L.hstu_attn_bwd(ctypes.byref(d or attn_desc()), ctypes.byref(j or jag()), q, fake(3), fake(4), do, fake(6),
                                fake(7), dq, fake(9), fake(10), drp, drt, ws, ws_bytes, None)
     run_cases(L, call, [
         ("F32 inputs (tensor cores only)", dict(d=attn_desc(dtype=F32, o_dtype=F32)), UNSUPPORTED),
@@ -212,7 +224,12 @@ def test_attn_bwd(L):
         ("no dout", dict(do=None), INVALID),
         ("dq off 16 bytes", dict(dq=fake(8) + 4), UNSUPPORTED),
         ("d = 32", dict(d=attn_desc(d_qk=32, d_v=32)), UNSUPPORTED),
+        ("dX^T rows beyond 32 bits", dict(j=jag(**HUGE_BWD)), UNSUPPORTED),
     ])
+    assert L.hstu_attn_bwd_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag(**HUGE_BWD))) == 0
+    # with one head the same batch fits the backward's bound
+    assert L.hstu_attn_bwd_workspace_size(ctypes.byref(attn_desc(H=1, ld_q=64, ld_k=64, ld_v=64, ld_o=64)),
+                                          ctypes.byref(jag(**HUGE_BWD))) > 0
 
 
 def test_norm_gate_fwd(L):
@@ -310,8 +327,8 @@ def test_layer_fwd(L):
     need = L.hstu_layer_workspace_size(ctypes.byref(layer_desc()), ctypes.byref(jag()))
     assert need >= L.hstu_attn_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag()))
 
-    def call(d=None, w=None, x=fake(2), y=fake(3), y16=None, sv=None, ws=fake(4), ws_bytes=need):
-        return L.hstu_layer_fwd(ctypes.byref(d or layer_desc()), ctypes.byref(jag()), ctypes.byref(w or weights()), x,
+    def call(d=None, j=None, w=None, x=fake(2), y=fake(3), y16=None, sv=None, ws=fake(4), ws_bytes=need):
+        return L.hstu_layer_fwd(ctypes.byref(d or layer_desc()), ctypes.byref(j or jag()), ctypes.byref(w or weights()), x,
                                 None, y, y16, ctypes.byref(sv or saved()), ws, ws_bytes, None)
     run_cases(L, call, [
         ("D not divisible by H", dict(d=layer_desc(H=3)), INVALID),
@@ -331,7 +348,9 @@ def test_layer_fwd(L):
         ("b2 off 16 bytes", dict(w=weights(b2=fake(23) + 4)), UNSUPPORTED),
         ("W2 off 16 bytes", dict(w=weights(W2=fake(22) + 2)), UNSUPPORTED),
         ("x off 16 bytes", dict(x=fake(2) + 2), UNSUPPORTED),
+        ("tile-pair rows beyond 32 bits", dict(j=jag(**HUGE_FWD)), UNSUPPORTED),
     ])
+    assert L.hstu_layer_workspace_size(ctypes.byref(layer_desc()), ctypes.byref(jag(**HUGE_FWD))) == 0
     assert passes_host_checks(L, call, sv=saved(z=None))                   # z is optional in the forward
     # the CUDA-core path reads the biases one element at a time
     assert passes_host_checks(L, call, d=layer_desc(dtype=F32, x_dtype=F32, y_dtype=F32), w=weights(b1=fake(21) + 4))
@@ -347,8 +366,8 @@ def test_layer_bwd(L):
         vals.update(kw)
         return Hb.hstu_layer_grads_t(*[vals[n] for n in names])
 
-    def call(d=None, w=None, sv=None, gr=None, x=fake(2), dy=fake(3), dx=fake(4), ws=fake(5), ws_bytes=need):
-        return L.hstu_layer_bwd(ctypes.byref(d or layer_desc()), ctypes.byref(jag()), ctypes.byref(w or weights()), x,
+    def call(d=None, j=None, w=None, sv=None, gr=None, x=fake(2), dy=fake(3), dx=fake(4), ws=fake(5), ws_bytes=need):
+        return L.hstu_layer_bwd(ctypes.byref(d or layer_desc()), ctypes.byref(j or jag()), ctypes.byref(w or weights()), x,
                                 None, ctypes.byref(sv or saved()), dy, None, dx, None, ctypes.byref(gr or grads()), ws,
                                 ws_bytes, None)
     run_cases(L, call, [
@@ -366,7 +385,9 @@ def test_layer_bwd(L):
         ("gamma off 16 bytes", dict(w=weights(gamma=fake(24) + 4)), UNSUPPORTED),
         ("dW1 off 16 bytes", dict(gr=grads(dW1=fake(40) + 4)), UNSUPPORTED),
         ("dx off 16 bytes", dict(dx=fake(4) + 2), UNSUPPORTED),
+        ("dX^T rows beyond 32 bits", dict(j=jag(**HUGE_BWD)), UNSUPPORTED),
     ])
+    assert L.hstu_layer_bwd_workspace_size(ctypes.byref(layer_desc()), ctypes.byref(jag(**HUGE_BWD))) == 0
     assert passes_host_checks(L, call, w=weights(b1=None, b2=None))   # the backward does not read the biases
 
 
@@ -383,9 +404,9 @@ def test_falcon_fwd(L):
     assert need > 0
     assert L.hstu_falcon_cache_size(ctypes.byref(falcon_desc()), ctypes.byref(jag())) == 2 * 300 * 2 * 256 * 2
 
-    def call(d=None, layers=None, cand=fake(3), req=fake(4), out=fake(5), ws=fake(6), ws_bytes=need):
+    def call(d=None, j=None, layers=None, cand=fake(3), req=fake(4), out=fake(5), ws=fake(6), ws_bytes=need):
         arr = (Hb.hstu_layer_weights_t * 2)(*(layers or [weights(), weights()]))
-        return L.hstu_falcon_fwd(ctypes.byref(d or falcon_desc()), arr, ctypes.byref(jag()), fake(2), fake(7), 0,
+        return L.hstu_falcon_fwd(ctypes.byref(d or falcon_desc()), arr, ctypes.byref(j or jag()), fake(2), fake(7), 0,
                                  None, cand, req, out, ws, ws_bytes, None)
     run_cases(L, call, [
         ("users differ from the prefix batch", dict(d=falcon_desc(users=3)), INVALID),
@@ -401,7 +422,9 @@ def test_falcon_fwd(L):
         ("second layer without gamma", dict(layers=[weights(), weights(gamma=None)]), INVALID),
         ("second layer's gamma off 16 bytes", dict(layers=[weights(), weights(gamma=fake(24) + 4)]), UNSUPPORTED),
         ("second layer's b2 off 16 bytes", dict(layers=[weights(), weights(b2=fake(23) + 4)]), UNSUPPORTED),
+        ("prefix tile-pair rows beyond 32 bits", dict(j=jag(**HUGE_FWD)), UNSUPPORTED),
     ])
+    assert L.hstu_falcon_workspace_size(ctypes.byref(falcon_desc()), ctypes.byref(jag(**HUGE_FWD))) == 0
     assert attempt(L, call, d=falcon_desc(m=0)) == (OK, False)   # no candidates: nothing to do
 
 
