@@ -209,9 +209,9 @@ hstu_status_t hstu_time_buckets(const hstu_jagged_t* jag, int32_t n_buckets,
 
 /* f1 + SiLU + split ("Generative Recommenders and HSTU", first equation):
  * uvqk[t, :] = SiLU(x[t, :] W1^T + b1), [T, 4D] with row stride 4D; b1 (nullable: no bias; 16-byte
- * aligned for BF16); z (nullable) receives the pre-activation. x and W1 have `dtype` (BF16 or F32); uvqk and z have act_dtype (F16 or BF16
- * for BF16 operands, F32 for F32); ld_x is x's row stride. ws: any workspace of at least 256
- * bytes (its status word receives device-side errors). */
+ * aligned for BF16); z (nullable) receives the pre-activation. x and W1 have `dtype` (BF16 or
+ * F32); uvqk and z have act_dtype (F16 or BF16 for BF16 operands, F32 for F32); ld_x is x's row
+ * stride. ws: any workspace of at least 256 bytes (its status word receives device-side errors). */
 hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t act_dtype, const void* x,
                             int64_t ld_x, const void* W1, const float* b1, void* uvqk, void* z,
                             void* ws, size_t ws_bytes, hstu_stream_t stream);
@@ -237,10 +237,9 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
  * and head a 16-bit dX^T tile (32 KB) from which the table gradients are summed over the heads.
  * The pair count is bounded from the batch's tile capacity and max_len (capacity (max_len/128 + 1)
  * / 2 pairs), so the size grows with H, T and max_len: about 1.5 GB for 30k tokens, max_len 4096
- * and 8 heads; 0.54 GB for 5.8k tokens, max_len 8192. */
+ * and 8 heads; 0.54 GB for 5.8k tokens, max_len 8192. 0 when the pair bound times H x 128 rows
+ * exceeds 2^31 - 1, which hstu_attn_bwd refuses with HSTU_ERR_UNSUPPORTED. */
 size_t hstu_attn_bwd_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag);
-/* (0 when the pair bound times H x 128 rows exceeds 2^31 - 1, which hstu_attn_bwd refuses with
- * HSTU_ERR_UNSUPPORTED; same for hstu_layer_bwd_workspace_size.) */
 
 /* Pointwise causal attention backward (derived from the forward's definition; tensor-core dtypes
  * F16 / BF16 only). With x_ij = q_i.k_j + rab(i, j) and A_ij = SiLU(x_ij) inv_N on causal pairs:
@@ -335,7 +334,7 @@ hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
                                int64_t ld_resid, void* out, hstu_dtype_t out_dtype, int64_t ld_out,
                                int32_t accumulate, void* ws, size_t ws_bytes, hstu_stream_t stream);
 
-/* Workspace bytes hstu_layer_bwd needs. */
+/* Workspace bytes hstu_layer_bwd needs (0 for a batch hstu_attn_bwd_workspace_size refuses). */
 size_t hstu_layer_bwd_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
 
 /* Whole layer backward (BF16 mode, D in {256, 512}), from the activations hstu_layer_fwd saved
@@ -361,8 +360,8 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
  * int64 per raw token (a uniformly random subset follows from i.i.d. uniform keys).
  * -------------------------------------------------------------------------------------------- */
 
-/* new_offsets (device, [B+1]) = exclusive prefix of L_b over raw's sequences. L is evaluated in
- * double precision. ws: >= 256 bytes (status word; a malformed raw offsets array is reported as
+/* new_offsets (device, [B+1]) = exclusive prefix of L_b over raw's sequences, alpha in [0, 2]
+ * (HSTU_ERR_INVALID_ARG otherwise). L is evaluated in double precision. ws: >= 256 bytes (status word; a malformed raw offsets array is reported as
  * HSTU_ERR_DEVICE by hstu_sync_status). The caller reads new_offsets[B] = T' to size the outputs
  * of hstu_stochastic_length_select. */
 hstu_status_t hstu_stochastic_length_offsets(const hstu_jagged_t* raw, double alpha, int64_t* new_offsets,
@@ -371,8 +370,9 @@ hstu_status_t hstu_stochastic_length_offsets(const hstu_jagged_t* raw, double al
 /* Selects the kept tokens of every sequence: kept (device int64 [T']) receives their global raw
  * indices in order, ts_out (nullable, [T']) their timestamps, and x_out (nullable, [T', D] of
  * x_dtype) their rows of x ([T_raw, D]). new_offsets must come from
- * hstu_stochastic_length_offsets with the same raw batch and alpha. Rows are copied as bytes
- * (D * element size must be a multiple of 16). */
+ * hstu_stochastic_length_offsets with the same raw batch and alpha. Rows are copied as bytes in
+ * 16-byte units: with x_out, D * element size must be a multiple of 16 and x, x_out 16-byte
+ * aligned (HSTU_ERR_UNSUPPORTED otherwise). */
 hstu_status_t hstu_stochastic_length_select(const hstu_jagged_t* raw, const int64_t* keys,
                                             const int64_t* new_offsets, const void* x,
                                             hstu_dtype_t x_dtype, int32_t D, int64_t* kept,
@@ -424,8 +424,10 @@ size_t hstu_falcon_workspace_size(const hstu_falcon_desc_t* desc, const hstu_jag
  * cand_x: bf16 [users * m, D], user u's candidates in rows [u m, (u+1) m).
  * request_ts: device int64 [users], the request time of each user.
  * out: fp32 [users * m, D], the candidates' output of the last layer.
- * Errors: the host checks of hstu_layer_fwd (D % 64 == 0, D/H == 64) plus
- * HSTU_ERR_INVALID_ARG for users != prefix->B, L < 1 or b_m < 1. */
+ * Errors: the host checks of hstu_layer_fwd (D % 64 == 0, D/H == 64; every layer's W1, W2, b1,
+ * b2, gamma and beta present and 16-byte aligned; the prefix batch within the tile-pair bound of
+ * hstu_attn_workspace_size) plus HSTU_ERR_INVALID_ARG for users != prefix->B, L < 1 or b_m < 1.
+ * hstu_falcon_cache_size and hstu_falcon_workspace_size return 0 for a refused descriptor. */
 hstu_status_t hstu_falcon_fwd(const hstu_falcon_desc_t* desc, const hstu_layer_weights_t* layers,
                               const hstu_jagged_t* prefix, const void* prefix_x, void* kv_cache,
                               int32_t cache_valid, void* prefix_out, const void* cand_x,

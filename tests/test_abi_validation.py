@@ -442,6 +442,28 @@ def test_stochastic_length(L):
     ])
 
 
+def test_stochastic_length_select(L):
+    def call(keys=fake(2), new_off=fake(3), x=fake(4), xdt=BF16, D=256, kept=fake(5), x_out=fake(6), ws=fake(7),
+             ws_bytes=256, j=None):
+        return L.hstu_stochastic_length_select(ctypes.byref(j or jag()), keys, new_off, x, xdt, D, kept, x_out,
+                                               fake(8), ws, ws_bytes, None)
+    run_cases(L, call, [
+        ("no keys", dict(keys=None), INVALID),
+        ("no new offsets", dict(new_off=None), INVALID),
+        ("no kept indices", dict(kept=None), INVALID),
+        ("no workspace", dict(ws=None), INVALID),
+        ("workspace below 256 bytes", dict(ws_bytes=8), WORKSPACE),
+        ("rows out without rows in", dict(x=None), INVALID),
+        ("zero width", dict(D=0), INVALID),
+        ("unknown dtype", dict(xdt=7), UNSUPPORTED),
+        ("rows not a multiple of 16 bytes", dict(D=100), UNSUPPORTED),
+        ("x off 16 bytes", dict(x=fake(4) + 8), UNSUPPORTED),
+        ("x_out off 16 bytes", dict(x_out=fake(6) + 2), UNSUPPORTED),
+    ])
+    assert passes_host_checks(L, call, x=None, x_out=None, D=0)     # indices only: x is not read
+    assert attempt(L, call, j=jag(B=2, T=0)) == (OK, False)
+
+
 def test_status_and_probe(L):
     st = ctypes.c_int32(0)
     assert L.hstu_sync_status(None, None, ctypes.byref(st)) == INVALID
