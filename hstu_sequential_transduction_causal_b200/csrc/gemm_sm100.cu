@@ -1,12 +1,14 @@
 // gemm_sm100.cu - the layer's projection GEMMs on the 5th-generation tensor cores.
 //
-// C[M, N] = A[M, K] * B[N, K]^T with bf16 operands and fp32 accumulation in tensor memory.
+// C[M, N] = A[M, K] * B[N, K]^T with 16-bit operands (both bf16 or both fp16) and fp32 accumulation
+// in tensor memory.
 // Each operand is either K-major (row-major [rows, K]) or MN-major (row-major [K, rows]), so the
 // forward projections (X W1^T, G W2^T) and the backward ones (dY W2, dZ W1, dY^T G, dZ^T X)
 // share one kernel. Operand tiles arrive by TMA (128-byte swizzle) into a STAGES-deep ring; one
 // thread issues tcgen05.mma (M=128, N=BN, K=16) into TMEM; four warps run the fused epilogue:
 //   SILU:   Z = acc + b;  out0 = SiLU(Z) (the U|V|Q|K activations), out1 = Z (optional)
-//   LINEAR: Y = acc (+ b) (+ R);  out0 = Y, out1 = bf16 copy of Y (optional)
+//   LINEAR: Y = acc (+ b) (+ R);  out0 = Y, out1 = a second copy of Y in out1's dtype (optional;
+//           the fp16 copy a stacked layer's f1 reads)
 //   ATOMIC: out0 += acc (fp32 reductions for split-K weight gradients)
 // ("4.4 Scaling Recommendation Models", Generative Recommenders and HSTU: f1 with phi1 = SiLU
 // and the split into U, V, Q, K; f2 followed by the residual of the "Code" sketch.)
