@@ -297,6 +297,47 @@ def test_backward_matches_finite_differences(lengths, L):
             assert abs(fd - an) <= 1e-6 + 1e-5 * abs(fd), (gname, t, fd, an)
 
 
+@settings(max_examples=25, deadline=None, derandomize=True)
+@given(lengths=st.lists(st.integers(0, 7), min_size=1, max_size=3), L=st.integers(2, 5), H=st.sampled_from([1, 2]),
+       d=st.sampled_from([2, 3]), seed=st.integers(0, 2 ** 16))
+def test_attention_backward_finite_differences_random_shapes(lengths, L, H, d, seed):
+    """The attention backward alone against central differences of the attention forward, over
+    random jagged shapes whose sequences may outrun the position table (clamped entries), with
+    unsorted and widely spread timestamps: dq, dk, dv on sampled entries, every rab_pos entry and
+    every rab_time entry a pair reads."""
+    rng = np.random.default_rng(seed)
+    off = W.offsets_from_lengths(lengths)
+    T = int(off[-1])
+    ts = rng.integers(-5, 10 ** 7, T).astype(np.int64)
+    q, k, v, do = (0.7 * rng.standard_normal((T, H, d)) for _ in range(4))
+    rp, rt = rng.standard_normal(2 * L - 1), rng.standard_normal(128)
+    inv_N = 0.4
+
+    def loss():
+        return float((O.pointwise_attention_fwd(q, k, v, off, ts, rp, rt, inv_N, L, THR) * do).sum())
+
+    grads = O.pointwise_attention_bwd(q, k, v, do, off, ts, rp, rt, inv_N, L, THR)
+    used_buckets = set()
+    for b in range(len(lengths)):
+        tb = ts[off[b]:off[b + 1]]
+        used_buckets |= set(np.unique(O.time_bucket(tb[:, None] - tb[None, :], THR)).tolist())
+    h = 1e-6
+    for arr, g, idx in ((q, grads[0], None), (k, grads[1], None), (v, grads[2], None),
+                        (rp, grads[3], np.arange(rp.size)), (rt, grads[4], np.array(sorted(used_buckets), int))):
+        flat, gflat = arr.reshape(-1), g.reshape(-1)
+        if idx is None:
+            idx = rng.choice(flat.size, size=min(flat.size, 6), replace=False) if flat.size else np.array([], int)
+        for t in idx:
+            old = flat[t]
+            flat[t] = old + h
+            lp = loss()
+            flat[t] = old - h
+            lm = loss()
+            flat[t] = old
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - gflat[t]) <= 1e-6 + 1e-5 * abs(fd), (t, fd, gflat[t])
+
+
 # ---------------------------------------------------------------------------------------------
 # M-FALCON, Stochastic Length, work list
 # ---------------------------------------------------------------------------------------------
