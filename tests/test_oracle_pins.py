@@ -338,6 +338,32 @@ def test_attention_backward_finite_differences_random_shapes(lengths, L, H, d, s
             assert abs(fd - gflat[t]) <= 1e-6 + 1e-5 * abs(fd), (t, fd, gflat[t])
 
 
+@settings(max_examples=25, deadline=None, derandomize=True)
+@given(T=st.integers(1, 9), D=st.sampled_from([1, 2, 5, 16]), eps=st.sampled_from([1e-5, 1e-3, 0.5]),
+       scale=st.sampled_from([1e-3, 1.0, 1e3]), seed=st.integers(0, 2 ** 16))
+def test_norm_gate_matches_torch_layer_norm_and_autograd(T, D, eps, scale, seed):
+    """LayerNorm (.) U and its backward against torch's own layer_norm and autograd in float64 on
+    the CPU: a library routine written independently of the oracle's closed forms. Rows of very
+    small and very large spread exercise eps; D = 1 makes xhat zero."""
+    rng = np.random.default_rng(seed)
+    o = scale * rng.standard_normal((T, D)) + rng.standard_normal((T, 1))
+    u, dg = rng.standard_normal((T, D)), rng.standard_normal((T, D))
+    gamma, beta = 1 + 0.3 * rng.standard_normal(D), 0.3 * rng.standard_normal(D)
+    g, mu, rstd = O.norm_gate_fwd(o, u, gamma, beta, eps)
+    do, dgamma, dbeta = O.norm_gate_bwd(dg, o, u, gamma, mu, rstd)
+
+    to = torch.tensor(o, dtype=torch.float64, requires_grad=True)
+    tg = torch.tensor(gamma, dtype=torch.float64, requires_grad=True)
+    tb = torch.tensor(beta, dtype=torch.float64, requires_grad=True)
+    ln = torch.nn.functional.layer_norm(to, (D,), tg, tb, eps)
+    ref = ln * torch.tensor(u, dtype=torch.float64)
+    ref.backward(torch.tensor(dg, dtype=torch.float64))
+    assert np.allclose(g, ref.detach().numpy(), rtol=1e-12, atol=1e-12)
+    for got, want in ((do, to.grad), (dgamma, tg.grad), (dbeta, tb.grad)):
+        w = want.numpy()
+        assert np.allclose(got, w, rtol=1e-9, atol=1e-9 * max(1.0, float(np.abs(w).max()))), (got, w)
+
+
 # ---------------------------------------------------------------------------------------------
 # M-FALCON, Stochastic Length, work list
 # ---------------------------------------------------------------------------------------------
