@@ -106,6 +106,28 @@ def time_bucket(dt, thresholds: np.ndarray) -> np.ndarray:
     return np.searchsorted(thresholds, v, side="right").astype(np.int64)
 
 
+def time_diff(ts_q, ts_k) -> np.ndarray:
+    """All differences t_q - t_k ([len(ts_q), len(ts_k)], int64), exact for any int64 inputs.
+
+    The bias depends on the true difference of two timestamps ("HSTU: The First Exploration of the
+    Scaling Law", 7.1.4 Innovation 2). When two int64 timestamps are more than 2^63 apart their
+    difference has no int64 value; it is then formed in Python integers and saturated to the
+    int64 range, which keeps the bucket: every threshold tau_k lies in [2, 2^63), so a saturated
+    difference has the same count of thresholds <= max(dt, 1) as the exact one.
+    """
+    a = np.asarray(ts_q, np.int64).reshape(-1)
+    b = np.asarray(ts_k, np.int64).reshape(-1)
+    if a.size == 0 or b.size == 0:
+        return np.zeros((a.size, b.size), np.int64)
+    hi = int(a.max()) - int(b.min())
+    lo = int(a.min()) - int(b.max())
+    if -(2 ** 63) <= lo and hi < 2 ** 63:
+        return a[:, None] - b[None, :]
+    d = a.astype(object)[:, None] - b.astype(object)[None, :]
+    d = np.minimum(np.maximum(d, -(2 ** 63)), 2 ** 63 - 1)
+    return d.astype(np.int64)
+
+
 def rel_pos_index(i, j, pos_max_len: int) -> np.ndarray:
     """Index into rab_pos for the pair (i, j): clip(i - j, -(L-1), L-1) + L - 1 (reading R6)."""
     L = int(pos_max_len)
@@ -156,7 +178,7 @@ def pair_bias(ts_q, ts_k, pos_q, pos_k, rab_pos, rab_time, pos_max_len, threshol
     """rab^{p,t}(i, j) = rab_pos[idx(p_i - p_j)] + rab_time[bucket(t_i - t_j)] for all pairs."""
     pi = np.asarray(pos_q, np.int64)[:, None]
     pj = np.asarray(pos_k, np.int64)[None, :]
-    dt = np.asarray(ts_q, np.int64)[:, None] - np.asarray(ts_k, np.int64)[None, :]
+    dt = time_diff(ts_q, ts_k)
     rp = np.asarray(rab_pos, np.float64)
     rt = np.asarray(rab_time, np.float64)
     return rp[rel_pos_index(pi, pj, pos_max_len)] + rt[time_bucket(dt, thresholds)]
@@ -274,7 +296,7 @@ def pointwise_attention_bwd(q, k, v, do, offsets, timestamps, rab_pos, rab_time,
                          pos_max_len, thresholds)
         causal = li[None, :] <= li[:, None]
         pidx = rel_pos_index(li[:, None], li[None, :], pos_max_len)
-        tidx = time_bucket(timestamps[s:e][:, None] - timestamps[s:e][None, :], thresholds)
+        tidx = time_bucket(time_diff(timestamps[s:e], timestamps[s:e]), thresholds)
         dp_sum = np.zeros((n, n))
         for h in range(H):
             p = q[s:e, h] @ k[s:e, h].T + bias
@@ -404,7 +426,8 @@ def falcon_fwd(layers: List, prefix_offsets, prefix_ts, prefix_x, cand_x, reques
             n = e - s
             j = np.arange(n)
             bias_prefix = (rp[rel_pos_index(n, j, pos_max_len)]
-                           + rt[time_bucket(int(request_ts[u_]) - prefix_ts[s:e], thresholds)])
+                           + rt[time_bucket(time_diff([int(request_ts[u_])], prefix_ts[s:e])[0],
+                                            thresholds)])
             bias_self = rp[rel_pos_index(0, 0, pos_max_len)] + rt[time_bucket(0, thresholds)]
             rows = slice(u_ * m, (u_ + 1) * m)
             for h in range(H):

@@ -120,6 +120,56 @@ def test_layer_matches_scalar_bruteforce(spread):
     assert np.allclose(y, np.array(yb), rtol=1e-10, atol=1e-10)
 
 
+def test_layer_matches_scalar_bruteforce_extreme_timestamps():
+    """Timestamps near both ends of the int64 range: differences of up to 2^64 - 1, which have no
+    int64 value, must still give the bucket of the true difference (the scalar loops subtract
+    Python integers exactly)."""
+    wl, p = _tiny([4, 3, 2])
+    big = 2 ** 63 - 1
+    wl.timestamps = np.array([-(2 ** 63), -5, 2 ** 62, big,       # spans of 2^63 + 2^62 and 2^64 - 1
+                              big, -(2 ** 63), 0,                  # out of order, negative differences
+                              big - 40, big], np.int64)
+    inv_N = 0.5
+    y, _ = O.layer_fwd(wl.x, p, wl.offsets, wl.timestamps, wl.H, inv_N, wl.pos_max_len, THR)
+    yb = layer_fwd_scalar(wl.x.astype(float).tolist(), p.W1.astype(float).tolist(),
+                          p.b1.tolist(), p.W2.astype(float).tolist(), p.b2.tolist(),
+                          p.gamma.tolist(), p.beta.tolist(), p.rab_pos.tolist(),
+                          p.rab_time.tolist(), wl.offsets.tolist(), [int(t) for t in wl.timestamps],
+                          wl.H, inv_N, wl.pos_max_len)
+    assert np.allclose(y, np.array(yb), rtol=1e-10, atol=1e-10)
+    ts = [int(t) for t in wl.timestamps[:4]]
+    exp = [[min(127, max(0, _decimal_bucket(a - b))) for b in ts] for a in ts]
+    assert np.array_equal(O.time_bucket(O.time_diff(ts, ts), THR), np.array(exp))
+
+
+def _decimal_bucket(dt):
+    ctx = decimal.Context(prec=60)
+    ln = ctx.ln(decimal.Decimal(max(int(dt), 1)))
+    return int((ln / decimal.Decimal("0.301")).to_integral_value(decimal.ROUND_FLOOR))
+
+
+@settings(max_examples=25, deadline=None, derandomize=True)
+@given(lengths=st.lists(st.integers(0, 700), min_size=1, max_size=5), H=st.sampled_from([1, 3]),
+       seed=st.integers(0, 2 ** 16), frac=st.sampled_from([0.02, 0.3, 1.0]))
+def test_attention_row_subset_equals_full_evaluation(lengths, H, seed, frac):
+    """``rows=`` groups the selected rows (by 512) and reads keys up to the group's last row; every
+    selected row must equal the full evaluation's (up to the last bits of the matrix products,
+    whose blocking depends on their shapes: a wrong key range or grouping moves rows by O(1)), and
+    every other row must be NaN."""
+    rng = np.random.default_rng(seed)
+    off = W.offsets_from_lengths(lengths)
+    T, d, L = int(off[-1]), 4, 300
+    ts = W.draw_timestamps(rng, lengths)
+    q, k, v = (rng.standard_normal((T, H, d)) for _ in range(3))
+    rp, rt = rng.standard_normal(2 * L - 1), rng.standard_normal(128)
+    full = O.pointwise_attention_fwd(q, k, v, off, ts, rp, rt, 1 / 64, L, THR)
+    rows = np.nonzero(rng.random(T) < frac)[0]
+    part = O.pointwise_attention_fwd(q, k, v, off, ts, rp, rt, 1 / 64, L, THR, rows=rows)
+    assert np.allclose(part[rows], full[rows], rtol=1e-12, atol=1e-12)
+    rest = np.setdiff1d(np.arange(T), rows)
+    assert np.all(np.isnan(part[rest]))
+
+
 @settings(max_examples=40, deadline=None, derandomize=True)
 @given(lengths=st.lists(st.integers(0, 9), min_size=1, max_size=4), L=st.integers(2, 6),
        H=st.sampled_from([1, 2]), dh=st.sampled_from([2, 3]), seed=st.integers(0, 2 ** 16), spread=st.booleans(),
