@@ -470,7 +470,7 @@ falcon_key_bias_kernel(const int64_t* __restrict__ off, const int64_t* __restric
        j += static_cast<long long>(gridDim.x) * blockDim.x) {
     float v = 0.0f;
     if (j < n) {
-      const int bkt = time_bucket_dev(treq - ts[s0 + j], s_tau, nb);
+      const int bkt = time_bucket_pair64(treq, ts[s0 + j], s_tau, nb);
       v = 0.5f * (rab_pos[bias_pos_index(n - j, L)] + rab_time[bkt]);
     }
     kbias[u * ld + j] = __half_as_ushort(__float2half_rn(v));

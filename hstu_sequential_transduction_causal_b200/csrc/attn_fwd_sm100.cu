@@ -222,7 +222,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int col = c * 32 + j + e;
-            const int bkt = time_bucket_dev(t_i - kts[col], s_tau, nb);
+            const int bkt = time_bucket_pair64(t_i, kts[col], s_tau, nb);
             const float x = __uint_as_float(sv[j + e]) + pw[-col] + s_rab_time[bkt];
             y[e] = (!diag || col <= r) ? silu_fast(x) : 0.0f;
           }
@@ -314,7 +314,7 @@ attn_fwd_f32_kernel(AttnArgs a) {
     float part = (lane < a.dqk ? q0 * kr[lane] : 0.0f) + (lane + 32 < a.dqk ? q1 * kr[lane + 32] : 0.0f);
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
-    const int bkt = time_bucket_dev(t_i - a.ts[j], c_time_taus, a.n_buckets);
+    const int bkt = time_bucket_pair64(t_i, a.ts[j], c_time_taus, a.n_buckets);
     const float x = part + a.rab_pos[pos_index(i - j, L)] + a.rab_time[bkt];
     const float w = x / (1.0f + expf(-x)) * a.inv_N;
     const float* vr = reinterpret_cast<const float*>(a.v) + j * a.ld_v + h * a.dv;

@@ -427,8 +427,11 @@ hstu_status_t hstu_time_buckets(const hstu_jagged_t* jag, int32_t n_buckets, con
   if (s != HSTU_OK) return s;
   if (n_buckets < 1 || n_buckets > 128) return HSTU_ERR_UNSUPPORTED;
   if (jag->T > 0 && (!sq_offsets || !out)) return HSTU_ERR_INVALID_ARG;
-  return cuda_status(launch_time_buckets(jag->offsets, jag->timestamps, jag->B, jag->T, n_buckets, sq_offsets, out,
-                                         stream));
+  // one block per (query tile, key tile) of each sequence: grid (mt^2, B)
+  const int64_t mt = (static_cast<int64_t>(jag->max_len) + kQTile - 1) / kQTile;
+  if (jag->B > 65535 || mt * mt > 0x7fffffffLL) return HSTU_ERR_UNSUPPORTED;
+  return cuda_status(launch_time_buckets(jag->offsets, jag->timestamps, jag->B, jag->T, jag->max_len, n_buckets,
+                                         sq_offsets, out, stream));
 }
 
 hstu_status_t hstu_uvqk_fwd(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t act_dtype, const void* x,
@@ -861,6 +864,14 @@ extern "C" hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_desc_t* desc, con
   cudaError_t e = cudaMemsetAsync(scratch, 0, kWsHeader, stream);
   if (e != cudaSuccess) return cuda_status(e);
   return run_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, scratch, stream, false);
+}
+
+extern "C" hstu_status_t hstu_attn_fwd_noalloc_status(hstu_stream_t stream, int32_t* device_status) {
+  if (!device_status) return HSTU_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  hstu_status_t s = noalloc_scratch(&scratch);
+  if (s != HSTU_OK) return s;
+  return hstu_sync_status(scratch, stream, device_status);
 }
 
 // ---------------------------------------------------------------------------------------------

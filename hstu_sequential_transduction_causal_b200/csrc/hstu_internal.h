@@ -101,9 +101,9 @@ cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
                             int32_t* count, int* status, cudaStream_t st, long long* pair_base = nullptr,
                             int32_t* kitems = nullptr, int32_t* kcount = nullptr);
-cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T,
-                                int n_buckets, const int64_t* sq_offsets, uint8_t* out,
-                                cudaStream_t st);
+// The n_b x n_b time-bucket matrices of the test surface, tile by tile with the bias tiles' code.
+cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int max_len,
+                                int n_buckets, const int64_t* sq_offsets, uint8_t* out, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------------
 // attention

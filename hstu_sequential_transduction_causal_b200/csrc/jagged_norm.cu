@@ -8,6 +8,7 @@
 #include "hstu_internal.h"
 #include "sm100_ptx.cuh"
 #include "time_bucket_dev.cuh"
+#include "bias_tile.cuh"
 #include "vec_io.cuh"
 
 namespace hstu {
@@ -234,23 +235,35 @@ worklist_warp_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_
   if (lane == 0) pair_base[B] = total;
 }
 
-// One warp per query row: writes bucket(t_i - t_j) for every key j of the row's sequence.
-__global__ void __launch_bounds__(256)
-time_bucket_kernel(const int64_t* __restrict__ off, const int64_t* __restrict__ ts, int B, int64_t T,
-                   int nb, const int64_t* __restrict__ sq_off, uint8_t* __restrict__ out) {
-  const int lane = threadIdx.x & 31;
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (row >= T) return;
-  int lo = 0, hi = B;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (off[mid] <= row) lo = mid; else hi = mid;
+// Test surface of the attention's time-bucket index: block (x = qt * mt + kt, y = b) writes
+// bucket(t_i - t_j) of every query i of tile qt and key j of tile kt of sequence b (all tiles, not
+// only causal ones) into the n_b x n_b matrix at out + sq_off[b]. It stages the tile's timestamps,
+// takes the 32-bit or 64-bit path and evaluates each element with exactly the functions the
+// attention's bias tiles use (bias_tile.cuh), so a bit-exact check of this output checks theirs.
+__global__ void __launch_bounds__(kBiasThreads)
+time_bucket_tile_kernel(const int64_t* __restrict__ off, const int64_t* __restrict__ ts, int nb, int mt,
+                        const int64_t* __restrict__ sq_off, uint8_t* __restrict__ out) {
+  __shared__ TileTimes s_t;
+  __shared__ long long s_tau[kTauEntries];
+  __shared__ int s_tau32[kTauEntries];
+  const int b = blockIdx.y;
+  const int qt = blockIdx.x / mt, kt = blockIdx.x - qt * mt;
+  const long long seq0 = off[b];
+  const long long n = off[b + 1] - seq0;
+  if (static_cast<long long>(qt) * kQTile >= n || static_cast<long long>(kt) * kQTile >= n) return;
+  tile_times_load(s_t, ts, seq0, static_cast<int>(n), qt * kQTile, kt * kQTile);
+  for (int e = threadIdx.x; e < kTauEntries; e += kBiasThreads) {
+    s_tau[e] = c_time_taus[e];
+    s_tau32[e] = c_time_taus32[e];
   }
-  const long long s0 = off[lo];
-  const long long n = off[lo + 1] - s0;
-  const long long ti = ts[row];
-  uint8_t* dst = out + sq_off[lo] + (row - s0) * n;
-  for (long long j = lane; j < n; j += 32) dst[j] = static_cast<uint8_t>(time_bucket_dev(ti - ts[s0 + j], c_time_taus, nb));
+  __syncthreads();
+  const bool fast = tile_times_finish(s_t);
+  uint8_t* dst = out + sq_off[b];
+  for (int e = threadIdx.x; e < kQTile * kQTile; e += kBiasThreads) {
+    const int r = e >> 7, c = e & 127;
+    const long long i = static_cast<long long>(qt) * kQTile + r, j = static_cast<long long>(kt) * kQTile + c;
+    if (i < n && j < n) dst[i * n + j] = static_cast<uint8_t>(tile_bucket<false>(s_t, fast, r, c, s_tau, s_tau32, nb));
+  }
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -359,13 +372,15 @@ cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_le
                     pair_base, kitems, kcount);
 }
 
-cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int n_buckets,
-                                const int64_t* sq_offsets, uint8_t* out, cudaStream_t st) {
-  if (T == 0) return cudaSuccess;
+cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int max_len,
+                                int n_buckets, const int64_t* sq_offsets, uint8_t* out, cudaStream_t st) {
+  if (T == 0 || B == 0) return cudaSuccess;
   cudaError_t e = upload_time_taus();
   if (e != cudaSuccess) return e;
-  time_bucket_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, st>>>(offsets, ts, B, T, n_buckets,
-                                                                          sq_offsets, out);
+  const int mt = (max_len + kQTile - 1) / kQTile;
+  if (mt == 0) return cudaSuccess;
+  time_bucket_tile_kernel<<<dim3(static_cast<unsigned>(mt * mt), static_cast<unsigned>(B)), kBiasThreads, 0, st>>>(
+      offsets, ts, n_buckets, mt, sq_offsets, out);
   return cudaGetLastError();
 }
 

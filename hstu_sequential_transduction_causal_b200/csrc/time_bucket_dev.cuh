@@ -29,6 +29,16 @@ __device__ __forceinline__ int time_bucket_dev(long long dt, const long long* ta
   return min(k, nb - 1);
 }
 
+// bucket(t_q - t_k) for any two int64 timestamps. The difference is formed in unsigned 64-bit
+// arithmetic, so it never overflows: t_q <= t_k gives bucket 0, and a difference above INT64_MAX
+// exceeds every threshold (all are below 2^63), which gives the last bucket.
+__device__ __forceinline__ int time_bucket_pair64(long long tq, long long tk, const long long* tau, int nb) {
+  if (tq <= tk) return 0;
+  const unsigned long long u = static_cast<unsigned long long>(tq) - static_cast<unsigned long long>(tk);
+  if (u > 0x7fffffffffffffffULL) return nb - 1;
+  return time_bucket_dev(static_cast<long long>(u), tau, nb);
+}
+
 // The same for a difference known to fit in int32 (timestamps of a tile within 2^31 of each other):
 // tau32 holds tau_k saturated to INT32_MAX (tau_72 > 2^31 > every int32 dt, so no bucket past 71 is
 // reached) and tau32[0] = INT32_MIN; all arithmetic is 32-bit.

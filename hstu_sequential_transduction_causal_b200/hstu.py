@@ -91,6 +91,7 @@ SIGNATURES = {
                                c_vp]),
     "hstu_attn_fwd_noalloc": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                       c_vp]),
+    "hstu_attn_fwd_noalloc_status": (c_i32, [c_vp, P(c_i32)]),
     "hstu_norm_gate_fwd": (c_i32, [c_i64, c_i32, c_i32, c_i32, c_i32, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp,
                                    c_f32, c_vp, c_vp, c_vp, c_vp]),
     "hstu_out_proj_workspace_size": (c_sz, [c_i32, c_i32]),
@@ -261,6 +262,13 @@ def hstu_attn_fwd_noalloc(desc, jag, q, k, v, rab_pos, rab_time, out, stream=Non
     _check("hstu_attn_fwd_noalloc", lib().hstu_attn_fwd_noalloc(ctypes.byref(desc), ctypes.byref(jag), _ptr(q), _ptr(k),
                                                                 _ptr(v), _ptr(rab_pos), _ptr(rab_time), _ptr(out),
                                                                 _stream(stream)))
+
+
+def hstu_attn_fwd_noalloc_status(stream=None) -> int:
+    """Device status of the last hstu_attn_fwd_noalloc call on this device (read and reset)."""
+    out = c_i32(0)
+    _check("hstu_attn_fwd_noalloc_status", lib().hstu_attn_fwd_noalloc_status(_stream(stream), ctypes.byref(out)))
+    return out.value
 
 
 def hstu_norm_gate_fwd(T, D, o_dtype_code, u_dtype_code, g_dtype_code, o, ld_o, u, ld_u, gamma, beta, eps, g, mu,

@@ -199,7 +199,11 @@ hstu_status_t hstu_jagged_worklist(const hstu_jagged_t* jag, int32_t* items, int
 /* Debug surface of the relative-time bias index ("HSTU: The First Exploration of the Scaling
  * Law", 7.1.4 Innovation 2): for every sequence b writes the n_b x n_b matrix of bucket(t_i -
  * t_j) (row i query, column j key, u8) at out + sq_offsets[b]; sq_offsets: device int64 [B+1],
- * the prefix sums of n_b^2. n_buckets in 1..128. */
+ * the prefix sums of n_b^2. n_buckets in 1..128. It runs the attention's own bucket code tile by
+ * tile (128 x 128 tiles of query and key rows): a tile whose timestamps span less than 2^31 - 1
+ * takes 32-bit arithmetic, any other tile a 64-bit path that never overflows, exactly as in the
+ * attention's bias tiles. max_len must bound every n_b (tiles past it are not written).
+ * HSTU_ERR_UNSUPPORTED for B > 65535 or ceil(max_len / 128)^2 > 2^31 - 1. */
 hstu_status_t hstu_time_buckets(const hstu_jagged_t* jag, int32_t n_buckets,
                                 const int64_t* sq_offsets, uint8_t* out, hstu_stream_t stream);
 
@@ -271,12 +275,21 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
  *    current); make that first call before any stream capture.
  *  - All calls share the one array and each call clears its status word: calls that overlap on
  *    the GPU (other streams, other host threads) race and must be serialised by the caller.
- *    Device-side errors of this variant are not reported; use hstu_attn_fwd with a workspace and
- *    hstu_sync_status to diagnose. */
+ *    Device-side errors of the last call (offsets that violate the jagged contract, a bounded wait
+ *    that ran out) are read with hstu_attn_fwd_noalloc_status. */
 hstu_status_t hstu_attn_fwd_noalloc(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag,
                                     const void* q, const void* k, const void* v,
                                     const float* rab_pos, const float* rab_time, void* out,
                                     hstu_stream_t stream);
+
+/* The device status word of hstu_attn_fwd_noalloc's built-in scratch on the current device: after
+ * synchronising `stream` it is copied into *device_status (HSTU_OK, HSTU_ERR_DEVICE for offsets
+ * that violated the jagged contract, HSTU_ERR_TIMEOUT for a bounded wait that ran out) and reset
+ * to 0. Since every hstu_attn_fwd_noalloc call clears it first, it describes the last call
+ * enqueued on this device; a call still running on another stream races with the read. Returns
+ * HSTU_ERR_INVALID_ARG for a NULL device_status, HSTU_ERR_CUDA if a copy fails. Allocates
+ * nothing. */
+hstu_status_t hstu_attn_fwd_noalloc_status(hstu_stream_t stream, int32_t* device_status);
 
 /* LayerNorm (.) U gating ("Generative Recommenders and HSTU", third equation; "HSTU: The First
  * Exploration of the Scaling Law", 7.1.4 Innovation 3): g = (gamma (o - mu) rstd + beta) (.) u

@@ -203,7 +203,9 @@ def test_attn_fwd_noalloc(L):
         ("no q", dict(q=None), INVALID),
         ("out off 16 bytes", dict(out=fake(7) + 4), UNSUPPORTED),
         ("129 buckets", dict(d=attn_desc(n_time_buckets=129)), UNSUPPORTED),
+        ("one sequence of 70,000 tiles", dict(j=jag(B=1, T=128 * 70000, max_len=1 << 30)), WORKSPACE),
     ])
+    assert L.hstu_attn_fwd_noalloc_status(None, None) == INVALID
 
 
 def test_attn_bwd(L):

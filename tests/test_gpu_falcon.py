@@ -88,22 +88,15 @@ def test_falcon_cache_reuse_is_identical():
     assert np.array_equal(first, second)
 
 
-def test_falcon_ranking_workload_sampled():
+def test_falcon_ranking_workload_every_candidate():
     """16 users x 2048-token prefixes, 1024 candidates per user in micro-batches of 256, 4 layers,
-    d_model 512, H 8: the whole problem on the GPU, sampled users and candidates in the oracle."""
+    d_model 512, H 8: every one of the 16384 candidate outputs (and the prefix's last-layer
+    output) against the oracle, which needs about two minutes of host time."""
     fw = W.make_falcon_workload(seed=0)
     r = FalconRun(fw, fw.b_m)
     got = r.run()
-    users = [0, 9]
-    cands = [0, 255, 256, 777, 1023]
-    off = fw.prefix_offsets
-    sub_off = np.concatenate([[0], np.cumsum([off[u + 1] - off[u] for u in users])]).astype(np.int64)
-    sub_rows = np.concatenate([np.arange(off[u], off[u + 1]) for u in users])
-    sub = W.FalconWorkload(D=fw.D, H=fw.H, N=fw.N, pos_max_len=fw.pos_max_len, layers=fw.layers,
-                           prefix_offsets=sub_off, prefix_ts=fw.prefix_ts[sub_rows], prefix_x=fw.prefix_x[sub_rows],
-                           cand_x=np.concatenate([fw.cand_x[u * fw.m + np.array(cands)] for u in users]),
-                           request_ts=fw.request_ts[users], m=len(cands), b_m=len(cands))
-    yc_ref, _ = _oracle(sub)
-    sel = np.concatenate([u * fw.m + np.array(cands) for u in users])
-    assert_close(got[sel], yc_ref, *BF16_TOL, what="ranking workload candidates")
     assert np.all(np.isfinite(got))
+    yc_ref, yp_ref = _oracle(fw)
+    assert got.shape == yc_ref.shape == (16 * 1024, fw.D)
+    assert_close(got, yc_ref, *BF16_TOL, what="ranking workload candidates (all)")
+    assert_close(r.prefix_out.float().cpu().numpy(), yp_ref, *BF16_TOL, what="ranking workload prefix output")

@@ -10,7 +10,7 @@ from hstu_sequential_transduction_causal_b200 import hstu as H
 from hstu_sequential_transduction_causal_b200 import workloads as W
 from hstu_sequential_transduction_causal_b200.runtime import (DeviceLayer, JaggedBatch, LayerRunner, to_dev,
                                                               workspace)
-from tests._util import BF16_TOL, F32_TOL, THR, assert_close, layer_oracle, sample_rows
+from tests._util import BF16_TOL, F32_TOL, THR, assert_close, layer_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -54,47 +54,108 @@ def test_worklist_bit_exact(lengths):
     assert np.array_equal(items[:n].cpu().numpy().astype(np.int64), exp)
 
 
+def _tile_paths(ts, off):
+    """Which bucket arithmetic each 128 x 128 (query tile, key tile) of every sequence takes: the
+    kernels use 32 bits when the tile's timestamps (query and key rows, rows past the end clamped
+    to the last token) span less than 2^31 - 1, else the 64-bit path."""
+    paths = set()
+    for b in range(len(off) - 1):
+        s, e = int(off[b]), int(off[b + 1])
+        n = e - s
+        nt = -(-n // 128)
+        for qt in range(nt):
+            for kt in range(nt):
+                rows = [min(qt * 128 + r, n - 1) for r in range(128)] + [min(kt * 128 + c, n - 1) for c in range(128)]
+                v = [int(ts[s + r]) for r in rows]
+                paths.add("32" if max(v) - min(v) < 2 ** 31 - 1 else "64")
+    return paths
+
+
+def _bucket_surface(off, ts, max_len=None):
+    jag = JaggedBatch(off, ts, max_len=max_len)
+    lens = np.diff(off)
+    sq = W.offsets_from_lengths(lens ** 2)
+    out = torch.full((max(int(sq[-1]), 1),), 255, dtype=torch.uint8, device="cuda")
+    H.hstu_time_buckets(jag.struct, 128, to_dev(sq, torch.int64), out)
+    got = out.cpu().numpy()
+    res = []
+    for b in range(len(off) - 1):
+        s, e = int(off[b]), int(off[b + 1])
+        n = e - s
+        res.append((got[sq[b]:sq[b + 1]].astype(np.int64).reshape(n, n),
+                    O.time_bucket(O.time_diff(ts[s:e], ts[s:e]), THR)))
+    return res
+
+
 def test_time_buckets_bit_exact():
     rng = np.random.default_rng(3)
-    lengths = [3, 70, 0, 200, 1]
+    lengths = [3, 70, 0, 200, 1, 300]
     off = W.offsets_from_lengths(lengths)
-    T = int(off[-1])
     ts = W.draw_timestamps(rng, lengths)
     # sequence 1: out of order, negative and threshold-adjacent differences, huge gaps
     s1 = slice(int(off[1]), int(off[2]))
     taus = THR[rng.integers(0, 127, size=70)]
     ts[s1] = 10 ** 15 + np.where(rng.random(70) < 0.5, taus, taus - 1) * rng.choice([-1, 1], 70)
     ts[int(off[3]):int(off[3]) + 5] = [0, 2 ** 62, -(2 ** 61), 7, 7]
-    jag = JaggedBatch(off, ts)
-    lens = np.diff(off)
-    sq = W.offsets_from_lengths(lens ** 2)
-    out = torch.full((int(sq[-1]),), 255, dtype=torch.uint8, device="cuda")
-    H.hstu_time_buckets(jag.struct, 128, to_dev(sq, torch.int64), out)
-    got = out.cpu().numpy()
-    for b in range(len(lengths)):
-        s, e = off[b], off[b + 1]
-        exp = O.time_bucket(ts[s:e][:, None] - ts[s:e][None, :], THR).reshape(-1)
-        assert np.array_equal(got[sq[b]:sq[b + 1]].astype(np.int64), exp), b
+    assert _tile_paths(ts, off) == {"32", "64"}
+    for b, (got, exp) in enumerate(_bucket_surface(off, ts)):
+        assert np.array_equal(got, exp), b
 
 
-def test_time_buckets_every_threshold_edge():
-    """Differences tau_k - 1, tau_k, tau_k + 1 for every threshold (and 0, 1, 2, int64-sized gaps)
-    against the first token: each bucket edge is hit from both sides."""
+def test_time_buckets_every_threshold_edge_32_bit_path():
+    """Differences tau_k - 1, tau_k, tau_k + 1 for every threshold below 2^31 (and 0, 1, 2), all in
+    tiles whose timestamps span less than 2^31 - 1: the 32-bit path meets every bucket edge that an
+    int32 difference can reach, from both sides, with positive and negative differences."""
+    vals = [0, 1, 2]
+    for t in THR:
+        if int(t) + 1 < 2 ** 31 - 1:
+            vals += [int(t) - 1, int(t), int(t) + 1]
+    ts = np.array(vals, dtype=np.int64)
+    off = np.array([0, len(ts)], np.int64)
+    assert _tile_paths(ts, off) == {"32"}
+    (got, exp), = _bucket_surface(off, ts)
+    assert np.array_equal(got, exp)
+    # every bucket an int32 difference can reach appears, and each edge is crossed
+    assert set(np.unique(exp[:, 0])) >= set(range(2, 72)) - {1}
+    assert np.array_equal(got[:, 0], O.time_bucket(ts, THR))
+
+
+def test_time_buckets_every_threshold_edge_64_bit_path():
+    """The same edges for every threshold, together with int64-sized gaps, so that the tiles holding
+    the larger thresholds take the 64-bit path."""
     vals = [0, 1, 2]
     for t in THR:
         vals += [int(t) - 1, int(t), int(t) + 1]
     vals += [2 ** 40, 2 ** 55 + 3, 2 ** 62 - 1]
     ts = np.array(vals, dtype=np.int64)
-    n = len(ts)
-    off = np.array([0, n], np.int64)
-    jag = JaggedBatch(off, ts)
-    sq = np.array([0, n * n], np.int64)
-    out = torch.full((n * n,), 255, dtype=torch.uint8, device="cuda")
-    H.hstu_time_buckets(jag.struct, 128, to_dev(sq, torch.int64), out)
-    got = out.cpu().numpy().astype(np.int64).reshape(n, n)
-    exp = O.time_bucket(ts[:, None] - ts[None, :], THR)
+    off = np.array([0, len(ts)], np.int64)
+    assert _tile_paths(ts, off) == {"32", "64"}
+    (got, exp), = _bucket_surface(off, ts)
     assert np.array_equal(got, exp)
     assert np.array_equal(got[:, 0], O.time_bucket(ts, THR))
+
+
+def test_time_buckets_spans_around_2_31_and_int64_extremes():
+    """Tile spans just under and at the 32-bit limit (2^31 - 2 takes 32 bits, 2^31 - 1 and 2^31 take
+    64), and timestamps at both ends of the int64 range, whose differences (up to 2^64 - 1) have no
+    int64 value: they must give the bucket of the true difference."""
+    big = 2 ** 63 - 1
+    seqs = [
+        [0, 2 ** 31 - 2, 5, 2 ** 31 - 3],                 # span 2^31 - 2: 32-bit
+        [0, 2 ** 31 - 1, 1, 2 ** 31 - 2],                 # span 2^31 - 1: 64-bit
+        [2 ** 31, 0, 17, 2 ** 31 - 40],                   # span 2^31: 64-bit
+        [-(2 ** 63), big, 0, -5, big - 1, -(2 ** 63) + 3, 2 ** 62],
+        [big, big - 1, big - int(THR[126]), big - int(THR[126]) + 1, -(2 ** 63)],
+    ]
+    off = W.offsets_from_lengths([len(q) for q in seqs])
+    ts = np.array([t for q in seqs for t in q], dtype=np.int64)
+    paths = [_tile_paths(ts[int(off[b]):int(off[b + 1])], np.array([0, off[b + 1] - off[b]])) for b in range(5)]
+    assert paths == [{"32"}, {"64"}, {"64"}, {"64"}, {"64"}]
+    for b, (got, exp) in enumerate(_bucket_surface(off, ts)):
+        assert np.array_equal(got, exp), b
+    # the extreme pairs themselves: INT64_MAX - INT64_MIN lies above every threshold
+    got3, _ = _bucket_surface(off, ts)[3]
+    assert got3[1, 0] == 127 and got3[0, 1] == 0
 
 
 # ---------------------------------------------------------------------------------------------
@@ -286,13 +347,15 @@ def test_layer_fwd_bf16_32_sequences_full():
     assert_close(y, ye, *BF16_TOL, what="Y c2 bf16")
 
 
-def test_layer_fwd_long_sequences_sampled_rows():
+def test_layer_fwd_long_sequences_every_row():
+    """The long-sequence workload (8 Pareto-length sequences, T = 5759, d_model 512, H 8): all
+    5759 x 512 outputs against the oracle."""
     wl = W.make_workload("c3", seed=0)
     y, run = _run_layer(wl)
     assert run.device_status() == 0
-    rows = sample_rows(wl.offsets, per_seq=6)
-    ye, _ = layer_oracle(wl, rows=rows)
-    assert_close(y[rows], ye, *BF16_TOL, what="Y c3 bf16 (sampled rows)")
+    ye, _ = layer_oracle(wl)
+    assert y.shape == ye.shape == (wl.T, wl.D)
+    assert_close(y, ye, *BF16_TOL, what="Y c3 bf16 (every row)")
 
 
 def test_layer_fwd_fp32_residual_stream():

@@ -17,6 +17,7 @@ from hstu_sequential_transduction_causal_b200 import hstu as H
 from hstu_sequential_transduction_causal_b200 import workloads as W
 from hstu_sequential_transduction_causal_b200.runtime import (DeviceLayer, JaggedBatch, LayerRunner, to_dev,
                                                               workspace)
+from tests import _rounding as R
 from tests._util import BF16_TOL, THR, assert_close
 
 pytestmark = pytest.mark.gpu
@@ -81,41 +82,53 @@ def _oracle_grads(wl):
     return O.layer_bwd(wl.dy, p, sv, wl.offsets, wl.timestamps, wl.H, 1.0 / wl.N, wl.pos_max_len, THR)
 
 
+def _model_grads(wl):
+    """The oracle with fp16 rounding at the CUDA path's storage points (tests/_rounding.py)."""
+    p = wl.layers[0]
+    args = (wl.offsets, wl.timestamps, wl.H, 1.0 / wl.N, wl.pos_max_len)
+    _, sv = R.layer_fwd(wl.x, p, *args)
+    return R.layer_bwd(wl.dy, p, sv, *args)
+
+
 NAMES = ("dW1", "db1", "dW2", "db2", "dgamma", "dbeta", "drab_pos", "drab_time")
 
 
 STRICT_MISSES = {}
 
 
-def _compare(dx, grads, ref, tag=""):
-    """dx (an O(1) activation gradient) meets the bf16 bound verbatim. Weight and table gradients
-    are sums over all tokens with scale rms(ref) far from 1; the bound's absolute term is applied
-    in units of that scale, |d| <= 1e-2 max(1, rms(ref)) + 1e-2 |ref|, together with a norm-relative
-    error <= 1e-2. The number of elements outside the unscaled bound is recorded for the report."""
+def _compare(dx, grads, ref, model, tag=""):
+    """dx (an O(1) activation gradient) meets the bf16 bound |d| <= 1e-2 + 1e-2 |ref| element by
+    element. The weight and table gradients are sums over all tokens; with 16-bit attention operands
+    some of their elements cannot meet that bound (tests/test_rounding_floor.py). For each of them
+    the count of elements outside the bound must stay within R.miss_ceiling of the rounding model's
+    count on the same inputs, every element within the bound taken in units of the gradient's scale
+    (|d| <= 1e-2 max(1, rms(ref)) + 1e-2 |ref|), and the norm-relative error within 1e-2."""
     assert_close(dx, ref["dx"], *BF16_TOL, what="dx")
     for name, g in zip(NAMES, grads):
         e = np.asarray(ref[name], np.float64)
         scale = max(1.0, float(np.sqrt(np.mean(e ** 2)))) if e.size else 1.0
-        STRICT_MISSES[f"{tag}{name}"] = int((np.abs(g - e) > 1e-2 + 1e-2 * np.abs(e)).sum())
+        got_m, model_m = R.misses(g, e), R.misses(model[name], e)
+        STRICT_MISSES[f"{tag}{name}"] = (got_m, model_m)
+        assert got_m <= R.miss_ceiling(model_m, e.size), (name, got_m, model_m)
         assert_close(g, e, 1e-2 * scale, 1e-2, what=name)
         nrm = float(np.linalg.norm(e))
         if nrm > 0:
             rel = float(np.linalg.norm(g - e)) / nrm
             assert rel <= 1e-2, f"{name}: norm-relative error {rel:.3e}"
-    print(f"\n{tag} elements outside the unscaled bound:",
+    print(f"\n{tag} elements outside the stated bound (GPU, rounding model):",
           {k: v for k, v in STRICT_MISSES.items() if k.startswith(tag)})
 
 
 def test_layer_bwd_ragged_d512():
     wl = W.make_workload("c3", seed=2, lengths=[1, 130, 300, 0, 257, 64], pos_max_len=512, N=512)
     dx, grads = _run_layer_fwd_bwd(wl)
-    _compare(dx, grads, _oracle_grads(wl), "ragged-d512 ")
+    _compare(dx, grads, _oracle_grads(wl), _model_grads(wl), "ragged-d512 ")
 
 
 def test_layer_bwd_d256_four_heads():
     wl = W.make_workload("c2", seed=3, lengths=[200, 129, 7], backward=True)
     dx, grads = _run_layer_fwd_bwd(wl)
-    _compare(dx, grads, _oracle_grads(wl), "d256 ")
+    _compare(dx, grads, _oracle_grads(wl), _model_grads(wl), "d256 ")
 
 
 def test_layer_bwd_fp32_residual_stream():
@@ -124,10 +137,10 @@ def test_layer_bwd_fp32_residual_stream():
     wl.x = np.random.default_rng(5).standard_normal((wl.T, wl.D)).astype(np.float32)
     wl.dy = np.random.default_rng(6).standard_normal((wl.T, wl.D)).astype(np.float32)
     dx, grads = _run_layer_fwd_bwd(wl, torch.float32)
-    _compare(dx, grads, _oracle_grads(wl), "fp32-residual ")
+    _compare(dx, grads, _oracle_grads(wl), _model_grads(wl), "fp32-residual ")
 
 
 def test_layer_bwd_long_sequence_workload_full():
     wl = W.make_workload("c3", seed=0)
     dx, grads = _run_layer_fwd_bwd(wl)
-    _compare(dx, grads, _oracle_grads(wl), "long-sequence-full ")
+    _compare(dx, grads, _oracle_grads(wl), _model_grads(wl), "long-sequence-full ")
