@@ -79,3 +79,32 @@ def layer_fwd_scalar(x, W1, b1, W2, b2, gamma, beta, rab_pos, rab_time, offsets,
             row.append(acc)
         Y.append(row)
     return Y
+
+
+def attention_scalar_ext(q, k, v, offsets, ts, types, rab_pos, rab_time, rab_type, per_head, inv_N, L):
+    """Pointwise attention with the bias rab_pos[idx(i - j)] + rab_time[bucket(t_i - t_j)] +
+    rab_type[type_i][type_j] (reading R12 of hstu_oracle), tables per head (per_head: nested lists
+    indexed by head first) or shared; q, k, v: nested lists [T][H][d]; types: list of ints or None
+    (no type term). Returns out [T][H][d]."""
+    T = len(q)
+    H = len(q[0]) if T else 0
+    d = len(v[0][0]) if T else 0
+    out = [[[0.0] * d for _ in range(H)] for _ in range(T)]
+    for b in range(len(offsets) - 1):
+        s0, s1 = offsets[b], offsets[b + 1]
+        for i in range(s0, s1):
+            for j in range(s0, i + 1):
+                for h in range(H):
+                    rp = rab_pos[h] if per_head else rab_pos
+                    rt = rab_time[h] if per_head else rab_time
+                    bias = rp[_pos(i - s0, j - s0, L)] + rt[_bucket(ts[i] - ts[j], len(rt))]
+                    if types is not None:
+                        ty = rab_type[h] if per_head else rab_type
+                        bias += ty[types[i]][types[j]]
+                    dot = 0.0
+                    for c in range(len(q[i][h])):
+                        dot += q[i][h][c] * k[j][h][c]
+                    a = _silu(dot + bias) * inv_N
+                    for c in range(d):
+                        out[i][h][c] += a * v[j][h][c]
+    return out

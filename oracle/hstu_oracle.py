@@ -46,6 +46,11 @@ R10 Stochastic Length keeps L = min(n, floor(n**(alpha/2) + 1/2)) tokens, the L 
 R11 M-FALCON: a candidate attends to every token of its user's prefix and to itself; it sits at
     position n (the prefix length) with the request timestamp, so its result equals the last
     row of a causal forward over prefix + [candidate].
+R12 The richer bias f(p_i - p_j, t_i - t_j, type_i, type_j) of "HSTU: The First Exploration of
+    the Scaling Law", 7.1.4 Innovation 2, whose form the page does not give, is read as the sum of
+    three looked-up terms: rab_pos[idx(p_i - p_j)] + rab_time[bucket(t_i - t_j)] +
+    rab_type[type_i, type_j], each table either shared by the heads or with one slice per head
+    (the first page's sketch keeps a per-head bias table). Token types are small integers.
 
 Parity pins for every function live in ``tests/test_oracle_pins.py``; none is unpinned.
 """
@@ -224,6 +229,94 @@ def pointwise_attention_fwd(q, k, v, offsets, timestamps, rab_pos, rab_time, inv
                 a = np.where(causal, silu(p) * inv_N, 0.0)
                 out[s + li, h, :] = a @ v[s:s + nk, h, :]
     return out
+
+
+def pair_bias_ext(ts_q, ts_k, pos_q, pos_k, type_q, type_k, rab_pos_h, rab_time_h, rab_type_h, pos_max_len,
+                  thresholds):
+    """f(p_i - p_j, t_i - t_j, type_i, type_j) with one head's tables (reading R12):
+    rab_pos_h[idx(p_i - p_j)] + rab_time_h[bucket(t_i - t_j)] + rab_type_h[type_i, type_j]; the type
+    term is left out when rab_type_h is None."""
+    b = pair_bias(ts_q, ts_k, pos_q, pos_k, rab_pos_h, rab_time_h, pos_max_len, thresholds)
+    if rab_type_h is not None:
+        tt = np.asarray(rab_type_h, np.float64)
+        b = b + tt[np.asarray(type_q, np.int64)[:, None], np.asarray(type_k, np.int64)[None, :]]
+    return b
+
+
+def pointwise_attention_fwd_ext(q, k, v, offsets, timestamps, rab_pos, rab_time, inv_N, pos_max_len,
+                                thresholds, token_type=None, rab_type=None, per_head=False):
+    """The pointwise attention of ``pointwise_attention_fwd`` with the bias of reading R12: with
+    per_head, rab_pos [H, 2L-1], rab_time [H, nb] and rab_type [H, nt, nt] give head h its own
+    slices, else they are shared ([2L-1], [nb], [nt, nt]); token_type [T] holds each token's type
+    (needed with rab_type)."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    T, H, _ = q.shape
+    out = np.zeros((T, H, v.shape[2]))
+    ty = None if token_type is None else np.asarray(token_type, np.int64)
+    for b in range(len(offsets) - 1):
+        s, e = int(offsets[b]), int(offsets[b + 1])
+        if e == s:
+            continue
+        li = np.arange(e - s)
+        causal = li[None, :] <= li[:, None]
+        for h in range(H):
+            sl = (lambda t: None if t is None else np.asarray(t, np.float64)[h]) if per_head else \
+                (lambda t: None if t is None else np.asarray(t, np.float64))
+            bias = pair_bias_ext(timestamps[s:e], timestamps[s:e], li, li,
+                                 None if ty is None else ty[s:e], None if ty is None else ty[s:e],
+                                 sl(rab_pos), sl(rab_time), sl(rab_type), pos_max_len, thresholds)
+            p = q[s:e, h] @ k[s:e, h].T + bias
+            a = np.where(causal, silu(p) * inv_N, 0.0)
+            out[s:e, h] = a @ v[s:e, h]
+    return out
+
+
+def pointwise_attention_bwd_ext(q, k, v, do, offsets, timestamps, rab_pos, rab_time, inv_N, pos_max_len,
+                                thresholds, token_type=None, rab_type=None, per_head=False):
+    """Gradients of ``pointwise_attention_fwd_ext``: dq, dk, dv and the gradients of rab_pos,
+    rab_time and rab_type (same shapes as the tables; None for an absent rab_type). Each table
+    entry receives dP of every pair (of every head sharing it) that reads it."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    do = np.asarray(do, np.float64)
+    T, H, _ = q.shape
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    drp = np.zeros(np.asarray(rab_pos).shape)
+    drt = np.zeros(np.asarray(rab_time).shape)
+    dty = None if rab_type is None else np.zeros(np.asarray(rab_type).shape)
+    ty = None if token_type is None else np.asarray(token_type, np.int64)
+    for b in range(len(offsets) - 1):
+        s, e = int(offsets[b]), int(offsets[b + 1])
+        if e == s:
+            continue
+        li = np.arange(e - s)
+        causal = li[None, :] <= li[:, None]
+        pidx = rel_pos_index(li[:, None], li[None, :], pos_max_len)
+        tidx = time_bucket(time_diff(timestamps[s:e], timestamps[s:e]), thresholds)
+        for h in range(H):
+            sl = (lambda t: None if t is None else np.asarray(t, np.float64)[h]) if per_head else \
+                (lambda t: None if t is None else np.asarray(t, np.float64))
+            bias = pair_bias_ext(timestamps[s:e], timestamps[s:e], li, li,
+                                 None if ty is None else ty[s:e], None if ty is None else ty[s:e],
+                                 sl(rab_pos), sl(rab_time), sl(rab_type), pos_max_len, thresholds)
+            p = q[s:e, h] @ k[s:e, h].T + bias
+            a = np.where(causal, silu(p) * inv_N, 0.0)
+            dv[s:e, h] = a.T @ do[s:e, h]
+            dp = np.where(causal, (do[s:e, h] @ v[s:e, h].T) * silu_grad(p) * inv_N, 0.0)
+            dq[s:e, h] = dp @ k[s:e, h]
+            dk[s:e, h] = dp.T @ q[s:e, h]
+            tp = drp[h] if per_head else drp
+            tt = drt[h] if per_head else drt
+            np.add.at(tp, pidx[causal], dp[causal])
+            np.add.at(tt, tidx[causal], dp[causal])
+            if dty is not None:
+                ti = np.broadcast_to(ty[s:e][:, None], (e - s, e - s))
+                tj = np.broadcast_to(ty[s:e][None, :], (e - s, e - s))
+                np.add.at(dty[h] if per_head else dty, (ti[causal], tj[causal]), dp[causal])
+    return dq, dk, dv, drp, drt, dty
 
 
 def norm_gate_fwd(o, u, gamma, beta, eps: float = LN_EPS):

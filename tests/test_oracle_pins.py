@@ -511,3 +511,80 @@ def test_work_list_invariants():
     assert {tuple(r) for r in wlst} == expect and len(wlst) == len(expect)
     for a, b in zip(wlst[:-1], wlst[1:]):
         assert a[1] > b[1] or (a[1] == b[1] and a[0] < b[0])
+
+
+# ---------------------------------------------------------------------------------------------
+# the richer bias: per-head tables and the token-type term (reading R12)
+# ---------------------------------------------------------------------------------------------
+
+def _ext_case(lengths, H=2, d=3, L=6, n_types=3, seed=0, spread=True):
+    rng = np.random.default_rng(seed)
+    off = W.offsets_from_lengths(lengths)
+    T = int(off[-1])
+    ts = W.draw_timestamps(rng, lengths)
+    if spread:
+        ts = (ts + rng.integers(-5, 10 ** 8, T)).astype(np.int64)
+    q, k, v = (rng.standard_normal((T, H, d)) for _ in range(3))
+    types = rng.integers(0, n_types, T)
+    rp = rng.standard_normal((H, 2 * L - 1))
+    rt = rng.standard_normal((H, 128))
+    ty = rng.standard_normal((H, n_types, n_types))
+    return off, ts, q, k, v, types, rp, rt, ty
+
+
+@pytest.mark.parametrize("per_head,with_types", [(True, True), (True, False), (False, True)])
+def test_attention_ext_matches_scalar_bruteforce(per_head, with_types):
+    from oracle.bruteforce import attention_scalar_ext
+    off, ts, q, k, v, types, rp, rt, ty = _ext_case([4, 0, 9, 1, 7], seed=5)
+    if not per_head:
+        rp, rt, ty = rp[0], rt[0], ty[0]
+    inv_N = 0.2
+    got = O.pointwise_attention_fwd_ext(q, k, v, off, ts, rp, rt, inv_N, 6, THR,
+                                        token_type=types if with_types else None,
+                                        rab_type=ty if with_types else None, per_head=per_head)
+    exp = attention_scalar_ext(q.tolist(), k.tolist(), v.tolist(), off.tolist(), [int(t) for t in ts],
+                               [int(t) for t in types] if with_types else None, rp.tolist(), rt.tolist(),
+                               ty.tolist(), per_head, inv_N, 6)
+    assert np.allclose(got, np.array(exp), rtol=1e-11, atol=1e-11)
+
+
+def test_attention_ext_reduces_to_the_shared_tables():
+    """Equal per-head slices and no type term give the shared-table attention; a type table holding
+    one constant c everywhere gives the shared attention with c added to every rab_pos entry."""
+    off, ts, q, k, v, types, rp, rt, ty = _ext_case([5, 11, 2], H=3, seed=7)
+    base = O.pointwise_attention_fwd(q, k, v, off, ts, rp[0], rt[0], 0.3, 6, THR)
+    same = O.pointwise_attention_fwd_ext(q, k, v, off, ts, np.repeat(rp[:1], 3, 0), np.repeat(rt[:1], 3, 0), 0.3, 6,
+                                         THR, per_head=True)
+    assert np.allclose(same, base, rtol=1e-13, atol=1e-13)
+    c = 0.37
+    shifted = O.pointwise_attention_fwd(q, k, v, off, ts, rp[0] + c, rt[0], 0.3, 6, THR)
+    const = O.pointwise_attention_fwd_ext(q, k, v, off, ts, rp[0], rt[0], 0.3, 6, THR, token_type=types,
+                                          rab_type=np.full((3, 3), c))
+    assert np.allclose(const, shifted, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("per_head", [True, False])
+def test_attention_ext_backward_finite_differences(per_head):
+    off, ts, q, k, v, types, rp, rt, ty = _ext_case([3, 6, 1], H=2, d=2, L=4, seed=9)
+    if not per_head:
+        rp, rt, ty = rp[0], rt[0], ty[0]
+    rng = np.random.default_rng(1)
+    do = rng.standard_normal(q.shape)
+    kw = dict(token_type=types, per_head=per_head)
+
+    def loss(q_=q, k_=k, v_=v, rp_=rp, rt_=rt, ty_=ty):
+        o = O.pointwise_attention_fwd_ext(q_, k_, v_, off, ts, rp_, rt_, 0.5, 4, THR, rab_type=ty_, **kw)
+        return float(np.sum(o * do))
+
+    dq, dk, dv, drp, drt, dty = O.pointwise_attention_bwd_ext(q, k, v, do, off, ts, rp, rt, 0.5, 4, THR,
+                                                              rab_type=ty, **kw)
+    eps = 1e-6
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv), ("rp", rp, drp), ("rt", rt, drt),
+                            ("ty", ty, dty)):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            a1, a2 = arr.copy(), arr.copy()
+            a1[idx] += eps
+            a2[idx] -= eps
+            fd[idx] = (loss(**{f"{name}_": a1}) - loss(**{f"{name}_": a2})) / (2 * eps)
+        assert np.allclose(grad, fd, rtol=1e-5, atol=1e-7), name
