@@ -26,7 +26,8 @@ Pages followed (cited by title and section):
 
 Readings where the pages are silent, garbled or disagree:
 
-R1  No input LayerNorm before f1 (the equations have none; the sketch's extra one is a variant).
+R1  No input LayerNorm before f1 (the equations have none); the sketch's extra one is the
+    variant ``layer_fwd_norm_in`` (f1 reads LayerNorm_in(X), the residual adds X).
 R2  N is a constant runtime scalar (``inv_N`` = 1/N), never the per-batch maximum length.
 R3  The causal mask keeps j <= i (diagonal included), as in the sketch.
 R4  rab_pos and rab_time are shared by all heads.
@@ -360,6 +361,27 @@ def layer_fwd(x, p, offsets, timestamps, H, inv_N, pos_max_len, thresholds, eps=
     return y, dict(x=x, z=z, s=s, o=o, g=g, mu=mu, rstd=rstd)
 
 
+def layer_fwd_norm_in(x, p, gamma_in, beta_in, offsets, timestamps, H, inv_N, pos_max_len, thresholds,
+                      eps=LN_EPS):
+    """The variant of the first page's "Code" sketch that normalises the layer input first: f1 reads
+    Xn = LayerNorm_in(X) (affine, over d_model, eps 1e-5), the residual adds X itself (the sketch
+    returns x + f2(norm_av(av) * u) with u, v, q, k from f1(norm_in(x))). Returns (Y, saved) with
+    saved["x"] = Xn, the LayerNorm_in statistics in saved["mu_in"], saved["rstd_in"] and the raw
+    input in saved["x_raw"]."""
+    x = np.asarray(x, np.float64)
+    T, D = x.shape
+    xn, mu_in, rstd_in = norm_gate_fwd(x, np.ones_like(x), gamma_in, beta_in, eps)
+    d = D // H
+    z, s = uvqk_fwd(xn, p.W1, p.b1)
+    u, v, q, k = split_uvqk(s, D)
+    o = pointwise_attention_fwd(q.reshape(T, H, d), k.reshape(T, H, d), v.reshape(T, H, d),
+                                offsets, timestamps, p.rab_pos, p.rab_time, inv_N, pos_max_len,
+                                thresholds).reshape(T, D)
+    g, mu, rstd = norm_gate_fwd(o, u, p.gamma, p.beta, eps)
+    y = out_proj_fwd(g, p.W2, p.b2, x)
+    return y, dict(x=xn, z=z, s=s, o=o, g=g, mu=mu, rstd=rstd, x_raw=x, mu_in=mu_in, rstd_in=rstd_in)
+
+
 # ----------------------------------------------------------------------------------------------
 # Backward (closed form, derived from the forward equations; no autograd)
 # ----------------------------------------------------------------------------------------------
@@ -455,6 +477,22 @@ def layer_bwd(dy, p, saved, offsets, timestamps, H, inv_N, pos_max_len, threshol
     dx = dy + dz @ W1
     return dict(dx=dx, dW1=dW1, db1=db1, dW2=dW2, db2=db2, dgamma=dgamma, dbeta=dbeta,
                 drab_pos=drp, drab_time=drt, dz=dz, do=do)
+
+
+def layer_bwd_norm_in(dy, p, gamma_in, saved, offsets, timestamps, H, inv_N, pos_max_len, thresholds):
+    """Backward of ``layer_fwd_norm_in``: the layer's own gradients with Xn as f1's input (dW1 =
+    dZ^T Xn), then d Xn = dZ W1 through LayerNorm_in back to X, dX = dY + LN_in^T(d Xn); also
+    dgamma_in and dbeta_in."""
+    r = layer_bwd(dy, p, saved, offsets, timestamps, H, inv_N, pos_max_len, thresholds)
+    dxn = r["dz"] @ np.asarray(p.W1, np.float64)
+    x = saved["x_raw"]
+    dx_in, dgamma_in, dbeta_in = norm_gate_bwd(dxn, x, np.ones_like(x), gamma_in, saved["mu_in"],
+                                               saved["rstd_in"])
+    r = dict(r)
+    r["dx"] = np.asarray(dy, np.float64) + dx_in
+    r["dgamma_in"] = dgamma_in
+    r["dbeta_in"] = dbeta_in
+    return r
 
 
 # ----------------------------------------------------------------------------------------------

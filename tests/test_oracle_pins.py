@@ -588,3 +588,68 @@ def test_attention_ext_backward_finite_differences(per_head):
             a2[idx] -= eps
             fd[idx] = (loss(**{f"{name}_": a1}) - loss(**{f"{name}_": a2})) / (2 * eps)
         assert np.allclose(grad, fd, rtol=1e-5, atol=1e-7), name
+
+
+# ---------------------------------------------------------------------------------------------
+# the sketch's input LayerNorm (the norm_in variant of reading R1)
+# ---------------------------------------------------------------------------------------------
+
+def test_norm_in_variant_matches_the_first_page_sketch():
+    """The first page's sketch with its input LayerNorm kept (f1 reads norm_in(x), the residual adds
+    x), restated with torch ops and torch's LayerNorm, against layer_fwd_norm_in."""
+    n, D, H, L = 10, 16, 2, 16
+    rng = np.random.default_rng(12)
+    wl = W.make_workload("c1", seed=4, lengths=[n], D=D, H=H, pos_max_len=L, N=n)
+    p = wl.layers[0]
+    p.rab_time = np.zeros(128, np.float32)
+    p.rab_pos = rng.standard_normal(2 * L - 1).astype(np.float32)
+    g_in, b_in = 1 + 0.3 * rng.standard_normal(D), 0.3 * rng.standard_normal(D)
+    x_np = 3.0 + 2.0 * rng.standard_normal((n, D))          # far from normalised, so norm_in matters
+    y, _ = O.layer_fwd_norm_in(x_np, p, g_in, b_in, wl.offsets, wl.timestamps, H, 1.0 / n, L, THR)
+    x = torch.tensor(x_np, dtype=torch.float64)[None]
+    f1 = torch.nn.Linear(D, 4 * D).double()
+    f2 = torch.nn.Linear(D, D).double()
+    with torch.no_grad():
+        f1.weight.copy_(torch.tensor(p.W1))
+        f1.bias.copy_(torch.tensor(p.b1))
+        f2.weight.copy_(torch.tensor(p.W2))
+        f2.bias.copy_(torch.tensor(p.b2))
+    ii, jj = torch.arange(n)[:, None], torch.arange(n)[None, :]
+    dense = torch.tensor(p.rab_pos, dtype=torch.float64)[(ii - jj).clamp(-(L - 1), L - 1) + L - 1][None].expand(H, n, n)
+    xn = torch.nn.functional.layer_norm(x, (D,), torch.tensor(g_in), torch.tensor(b_in), eps=1e-5)
+    u, v, q, k = torch.nn.functional.silu(f1(xn)).chunk(4, dim=-1)
+    heads = lambda t: t.view(1, n, H, D // H).transpose(1, 2)
+    sc = heads(q) @ heads(k).transpose(-1, -2) + dense
+    a = torch.nn.functional.silu(sc).masked_fill(~torch.ones(n, n, dtype=torch.bool).tril(), 0) / n
+    av = (a @ heads(v)).transpose(1, 2).reshape(1, n, D)
+    ln = torch.nn.functional.layer_norm(av, (D,), torch.tensor(p.gamma, dtype=torch.float64),
+                                        torch.tensor(p.beta, dtype=torch.float64), eps=1e-5)
+    yt = (x + f2(ln * u))[0].detach().numpy()
+    assert np.allclose(y, yt, rtol=1e-12, atol=1e-12)
+
+
+def test_norm_in_backward_finite_differences():
+    wl, p = _tiny([3, 4, 1], D=8, H=2, seed=6)
+    rng = np.random.default_rng(3)
+    x = 1.5 + rng.standard_normal((wl.T, wl.D))
+    g_in, b_in = 1 + 0.3 * rng.standard_normal(wl.D), 0.3 * rng.standard_normal(wl.D)
+    dy = rng.standard_normal((wl.T, wl.D))
+    args = (wl.offsets, wl.timestamps, wl.H, 0.2, wl.pos_max_len, THR)
+
+    def loss(x_=x, g_=g_in, b_=b_in, W1=None):
+        pp = p if W1 is None else type(p)(**{**p.__dict__, "W1": W1})
+        return float(np.sum(O.layer_fwd_norm_in(x_, pp, g_, b_, *args)[0] * dy))
+
+    _, sv = O.layer_fwd_norm_in(x, p, g_in, b_in, *args)
+    r = O.layer_bwd_norm_in(dy, p, g_in, sv, *args)
+    eps = 1e-6
+    for name, arr, grad, kw in (("dx", x, r["dx"], "x_"), ("dgamma_in", g_in, r["dgamma_in"], "g_"),
+                                ("dbeta_in", b_in, r["dbeta_in"], "b_"), ("dW1", np.asarray(p.W1, np.float64),
+                                                                          r["dW1"], "W1")):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            a1, a2 = arr.copy(), arr.copy()
+            a1[idx] += eps
+            a2[idx] -= eps
+            fd[idx] = (loss(**{kw: a1}) - loss(**{kw: a2})) / (2 * eps)
+        assert np.allclose(grad, fd, rtol=1e-5, atol=1e-7), name
