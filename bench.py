@@ -32,13 +32,14 @@ sys.path.insert(0, ROOT)
 
 METRIC = "HSTU layer jagged tokens/sec (bf16 fwd/bwd); attention TFLOP/s as % of bf16 peak"
 WORKLOADS = {
-    "c3": dict(backward=True,
-               desc="HSTU layer forward+backward bf16: B=8 jagged sequences, lengths Pareto(alpha=1.2) clipped "
-                    "to [256,8192], d_model 512, H 8, d_qk=d_v=64, N=8192, rab_pos for max_len 8192, "
-                    "seed = rank"),
-    "c2": dict(backward=False,
-               desc="HSTU layer forward bf16: B=32 jagged sequences, lengths U[64,1024], d_model 256, H 4, "
-                    "d_qk=d_v=64, N=1024, seed = rank"),
+    "c3": dict(backward=True, B=8,
+               desc="HSTU layer forward+backward bf16: B=8 jagged sequences per GPU, lengths Pareto(alpha=1.2) "
+                    "clipped to [256,8192], d_model 512, H 8, d_qk=d_v=64, N=8192, rab_pos for max_len 8192; one "
+                    "global batch of 8 x n_gpus sequences (seed 0) split over the GPUs by hstu_dp_partition"),
+    "c2": dict(backward=False, B=32,
+               desc="HSTU layer forward bf16: B=32 jagged sequences per GPU, lengths U[64,1024], d_model 256, H 4, "
+                    "d_qk=d_v=64, N=1024; one global batch of 32 x n_gpus sequences (seed 0) split over the GPUs "
+                    "by hstu_dp_partition"),
 }
 
 
@@ -212,6 +213,82 @@ def reduce_over_ranks(total_ms: float, attn_ms: float, tokens: int, world: int, 
     return float(t[0]), float(t[1]), float(n.item())
 
 
+def measure_other_workloads(dev):
+    """Throughput of the two other workloads the hot path serves, on this GPU (CUDA events):
+    the 8-layer encoder forward+backward with Stochastic Length (64 raw sequences U[512, 4096],
+    alpha 1.6, d_model 512, H 8; tokens/s after subsampling) and M-FALCON ranking (16 users x
+    2048-token prefixes, 1024 candidates each in micro-batches of 256, 4 layers; candidates/s with
+    the prefix K/V built in the call, and with it reused from the cache)."""
+    import torch
+    from hstu_sequential_transduction_causal_b200 import hstu as H
+    from hstu_sequential_transduction_causal_b200 import workloads as W
+    from hstu_sequential_transduction_causal_b200.runtime import (DeviceLayer, Encoder, JaggedBatch, stochastic_length,
+                                                                  to_dev, workspace)
+    out = {}
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, warm=2, reps=5):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        ms = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        return float(np.median(ms))
+
+    wl = W.make_workload("c4", seed=0)
+    rng = np.random.default_rng(9)
+    raw = JaggedBatch(wl.offsets, wl.timestamps, device=dev)
+    raw_x = to_dev(rng.standard_normal((wl.T, wl.D)).astype(np.float32), torch.float32, dev)
+    jag, kept, xk = stochastic_length(raw, to_dev(wl.extra["sl_keys"], torch.int64, dev), wl.extra["sl_alpha"],
+                                      raw_x, device=dev)
+    layers = [DeviceLayer.upload(p, wl.D, wl.H, True, device=dev) for p in wl.layers]
+    enc = Encoder(layers, jag, 1.0 / wl.N, wl.pos_max_len, device=dev)
+    dy = torch.randn(jag.T, wl.D, dtype=torch.float32, device=dev)
+
+    def enc_step():
+        enc.forward(xk)
+        enc.backward(dy)
+    ms = timed(enc_step)
+    if enc.device_status() != 0:
+        raise RuntimeError("device status error in the encoder leg")
+    out["encoder_8_layers_fwd_bwd"] = {"value": jag.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+                                       "tokens": jag.T, "raw_tokens": wl.T,
+                                       "workload": "64 sequences U[512,4096] -> Stochastic Length alpha 1.6, "
+                                                   "8 layers, d_model 512, H 8, fp32 residual stream, eager launches"}
+    del enc, layers, raw_x, xk, dy
+    fw = W.make_falcon_workload(seed=0)
+    lens = np.diff(fw.prefix_offsets)
+    pj = JaggedBatch(fw.prefix_offsets, fw.prefix_ts, max_len=int(lens.max()), device=dev)
+    fl = [DeviceLayer.upload(p, fw.D, fw.H, True, device=dev) for p in fw.layers]
+    fws = [x.weights() for x in fl]
+    desc = H.make_falcon_desc(len(fl), fw.users, fw.m, fw.b_m, fw.D, fw.H, 1.0 / fw.N, fw.pos_max_len)
+    px, cx = to_dev(fw.prefix_x, torch.bfloat16, dev), to_dev(fw.cand_x, torch.bfloat16, dev)
+    req = to_dev(fw.request_ts, torch.int64, dev)
+    cache = torch.empty(H.hstu_falcon_cache_size(desc, pj.struct) // 2, dtype=torch.float16, device=dev)
+    fws_ws = workspace(H.hstu_falcon_workspace_size(desc, pj.struct), dev)
+    fout = torch.empty(fw.users * fw.m, fw.D, dtype=torch.float32, device=dev)
+
+    def falcon(valid):
+        return lambda: H.hstu_falcon_fwd(desc, fws, pj.struct, px, cache, valid, None, cx, req, fout, fws_ws)
+    ms_build = timed(falcon(0), reps=3)
+    ms_reuse = timed(falcon(1), reps=3)
+    if H.hstu_sync_status(fws_ws) != 0:
+        raise RuntimeError("device status error in the M-FALCON leg")
+    n_c = fw.users * fw.m
+    out["falcon_ranking"] = {"value": n_c / (ms_build / 1e3), "unit": "candidates/s", "ms_per_request_batch": ms_build,
+                             "cached_prefix": {"value": n_c / (ms_reuse / 1e3), "unit": "candidates/s",
+                                               "ms": ms_reuse},
+                             "workload": "16 users x 2048-token prefixes, 1024 candidates per user, micro-batches "
+                                         "of 256, 4 layers, d_model 512, H 8"}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -221,6 +298,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=15.0)
+    ap.add_argument("--no-extra", action="store_true", help="skip the encoder and M-FALCON throughput legs")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -253,9 +331,17 @@ def main():
     stream = torch.cuda.current_stream()
     backward = WORKLOADS[args.workload]["backward"]
 
-    wl = W.make_workload(args.workload, seed=rank)
-    if wl.dy is None:
-        wl.dy = W.round_bf16(np.random.default_rng(1000 + rank).standard_normal((wl.T, wl.D)))
+    # one global batch, split over the ranks by whole sequences (cost-balanced, the same split on
+    # every rank); per-rank work stays about constant as the number of GPUs grows
+    from hstu_sequential_transduction_causal_b200.runtime import shard_rows
+    gwl = W.make_workload(args.workload, seed=0, B=WORKLOADS[args.workload]["B"] * world)
+    if gwl.dy is None:
+        gwl.dy = W.round_bf16(np.random.default_rng(1000).standard_normal((gwl.T, gwl.D)))
+    rank_of, rank_cost = H.hstu_dp_partition(np.diff(gwl.offsets), gwl.D, world)
+    shard_off, shard = shard_rows(gwl.offsets, rank_of, rank)
+    wl = W.Workload(name=gwl.name, D=gwl.D, H=gwl.H, dtype=gwl.dtype, N=gwl.N, pos_max_len=gwl.pos_max_len,
+                    offsets=shard_off, timestamps=gwl.timestamps[shard], x=gwl.x[shard], layers=gwl.layers,
+                    dy=gwl.dy[shard])
     D, Hh, T = wl.D, wl.H, wl.T
     jag = JaggedBatch(wl.offsets, wl.timestamps, device=dev)
     layer = DeviceLayer.upload(wl.layers[0], D, Hh, True, device=dev)
@@ -293,6 +379,30 @@ def main():
         H.hstu_attn_fwd(adesc, jag.struct, sv.uvqk[:, 2 * D:], sv.uvqk[:, 3 * D:], sv.uvqk[:, D:], layer.rab_pos,
                         layer.rab_time, sv.o, ws)
 
+    # CUDA events the library records right around its dominant kernels (hstu_profile_events); captured
+    # into the step graph as event nodes, read after every timed replay
+    prof_kernels = [H.PROFILE_ATTN_FWD, H.PROFILE_NORM_FWD] + ([H.PROFILE_ATTN_BWD, H.PROFILE_NORM_BWD]
+                                                                if backward else [])
+    prof_ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in prof_kernels}
+    prof_ms = {k: [] for k in prof_kernels}
+
+    # data parallelism: the gradient sum runs on a side stream, started by the events hstu_layer_bwd
+    # records when dW2, db2, dgamma, dbeta and the tables are final (reduced while dZ, db1, dW1 and dX
+    # are computed) and when dW1, db1 are final (reduced while the dX GEMM runs)
+    comm = torch.cuda.Stream(device=dev) if world > 1 else None
+    n_late = 4 * D * D + 4 * D             # dW1, db1 lead the flat buffer
+    if comm is not None and backward:
+        ev_early, ev_w1 = torch.cuda.Event(), torch.cuda.Event()
+        H.hstu_layer_bwd_ready_events(ev_early, ev_w1)
+
+    def reduce_grads():
+        with torch.cuda.stream(comm):
+            comm.wait_event(ev_early)
+            dist.all_reduce(flat[n_late:])
+            comm.wait_event(ev_w1)
+            dist.all_reduce(flat[:n_late])
+        stream.wait_stream(comm)
+
     def step(ev=None, all_reduce=True):
         rec = (lambda i: ev[i].record(stream)) if ev else (lambda i: None)
         rec(0)
@@ -309,7 +419,7 @@ def main():
         if backward:
             H.hstu_layer_bwd(ldesc, jag.struct, weights, x, None, svs, dy, None, dx, None, grads, ws)
             if world > 1 and all_reduce:
-                dist.all_reduce(flat)
+                reduce_grads()
             rec(5)
 
     clk = ClockSampler(local_rank)
@@ -332,15 +442,31 @@ def main():
         seg = np.array([[e[k].elapsed_time(e[k + 1]) for k in range(nev - 1)] for e in evs])   # ms
         # the timed steps replay one CUDA graph of the whole step (no host launch cost inside); the
         # gradient all-reduce of a multi-GPU run follows each replay on the same stream
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            step(all_reduce=False)
+        # one GPU: the timed steps replay one CUDA graph of the whole step (no host launch cost
+        # inside); several GPUs: eager steps, so that the gradient all-reduce on the side stream
+        # overlaps the end of the backward
+        graph = torch.cuda.CUDAGraph() if world == 1 else None
+        if graph is not None:
+            with torch.cuda.graph(graph):
+                step(all_reduce=False)
         attn_graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(attn_graph):
             attention_forward()
+        # the same step with the library's kernel events recorded around its dominant kernels (event
+        # nodes cost some time between kernels, so the headline replays the graph without them)
+        for k, (e0_, e1_) in prof_ev.items():
+            H.hstu_profile_events(k, e0_, e1_)
+        prof_graph = torch.cuda.CUDAGraph() if world == 1 else None
+        if prof_graph is not None:
+            with torch.cuda.graph(prof_graph):
+                step(all_reduce=False)
+            for k in prof_ev:
+                H.hstu_profile_events(k)
+        run_prof = prof_graph.replay if prof_graph is not None else step
+        run_step = graph.replay if graph is not None else step
         for _ in range(3):
             flush_l2()
-            graph.replay()
+            run_step()
             attn_graph.replay()
         torch.cuda.synchronize()
         e_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -349,16 +475,30 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
         t_start = time.time()
+        if world > 1:
+            for k in prof_ev:
+                H.hstu_profile_events(k)
         for i in range(args.steps):
             flush_l2()
             e_step[i][0].record(stream)
-            graph.replay()
-            if world > 1 and backward:
-                dist.all_reduce(flat)
+            run_step()
             e_step[i][1].record(stream)
         torch.cuda.synchronize()
         t_end = time.time()
         clk.window = (t_start, t_end)
+        # per-kernel device times: as many steps again, each followed by a read of the kernel events
+        # (the next replay records them anew)
+        if world > 1:
+            for k, (e0_, e1_) in prof_ev.items():
+                H.hstu_profile_events(k, e0_, e1_)
+        for i in range(args.steps):
+            flush_l2()
+            run_prof()
+            torch.cuda.synchronize()
+            for k, (e0_, e1_) in prof_ev.items():
+                prof_ms[k].append(e0_.elapsed_time(e1_))
+        for k in prof_ev:
+            H.hstu_profile_events(k)
         n_attn = 20
         e_attn = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_attn)]
         for i in range(n_attn):
@@ -389,6 +529,8 @@ def main():
     h_off = torch.from_numpy(wl.offsets).pin_memory()
     h_ts = torch.from_numpy(wl.timestamps).pin_memory()
     h_y = torch.empty(T, D, dtype=torch.bfloat16).pin_memory()
+    h_dx = torch.empty(T, D, dtype=torch.bfloat16).pin_memory()
+    h_grads = torch.empty_like(flat, device="cpu").pin_memory()
     d_x = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
     d_dy = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
     e2e_ws = workspace(H.hstu_layer_bwd_workspace_size(run.desc, jag.struct) if backward else 256, dev)
@@ -403,8 +545,11 @@ def main():
             H.hstu_layer_bwd(run.desc, jag.struct, run.weights, d_x, None, run.saved_struct, d_dy, None, dx, None,
                              grads, e2e_ws)
             if world > 1:
-                dist.all_reduce(flat)
+                reduce_grads()
         h_y.copy_(run.y, non_blocking=True)
+        if backward:
+            h_dx.copy_(dx, non_blocking=True)
+            h_grads.copy_(flat, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
@@ -426,33 +571,72 @@ def main():
     if run.device_status() != 0 or H.hstu_sync_status(e2e_ws) != 0:
         raise RuntimeError("device status error in the end-to-end pass")
 
+    kern_ms = {k: float(np.mean(v)) for k, v in prof_ms.items()}
+    if world > 1:
+        tk = torch.tensor([kern_ms[k] for k in prof_kernels], dtype=torch.float64, device=dev)
+        dist.all_reduce(tk, op=dist.ReduceOp.MAX)
+        kern_ms = {k: float(tk[i]) for i, k in enumerate(prof_kernels)}
+    extra = measure_other_workloads(dev) if (world == 1 and not args.no_extra) else None
+
     if rank == 0:
         peaks, peak_kind = load_peaks()
         flops = attn_flops(wl.offsets, D)
-        achieved = flops / (attn_ms_max / 1e3) / 1e12
-        peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+        tf_peak = float(peaks.get("bf16_tflops"))
+        hbm_peak = float(peaks.get("hbm_gbs"))
+        achieved = flops / (kern_ms[H.PROFILE_ATTN_FWD] / 1e3) / 1e12
+        whole_fwd = flops / (attn_ms_max / 1e3) / 1e12
+        # LayerNorm (.) U: O fp32 and U fp16 read, G fp16 written, mu and rstd fp32 written
+        ln_bytes = T * (4 * D + 2 * D + 2 * D + 8)
+        rooflines = {
+            "attention_forward_whole": {
+                "what": "work list + bias tiles + attention kernel (its own graph, L2 flushed before each replay)",
+                "achieved": whole_fwd, "peak": tf_peak, "unit": "TFLOP/s", "frac": whole_fwd / tf_peak,
+                "ms": attn_ms_max},
+            "norm_gate_fwd": {"bound": "hbm", "achieved": ln_bytes / (kern_ms[H.PROFILE_NORM_FWD] / 1e3) / 1e9,
+                              "peak": hbm_peak, "unit": "GB/s", "algorithmic_bytes_per_launch": ln_bytes,
+                              "ms": kern_ms[H.PROFILE_NORM_FWD]}}
+        rooflines["norm_gate_fwd"]["frac"] = rooflines["norm_gate_fwd"]["achieved"] / hbm_peak
+        if backward:
+            # attention backward: four contractions (P recompute not counted) = 2x the forward's flops
+            bw = 2 * flops / (kern_ms[H.PROFILE_ATTN_BWD] / 1e3) / 1e12
+            rooflines["attention_backward"] = {"bound": "tensor", "achieved": bw, "peak": tf_peak, "unit": "TFLOP/s",
+                                               "frac": bw / tf_peak, "algorithmic_flops_per_launch": 2 * flops,
+                                               "ms": kern_ms[H.PROFILE_ATTN_BWD]}
+            # its backward: dG fp32, O fp32, U and Z_U fp16, mu and rstd read; dO and dZ_U fp16 written
+            lnb_bytes = T * (4 * D + 4 * D + 2 * D + 2 * D + 8 + 2 * D + 2 * D)
+            a_ = lnb_bytes / (kern_ms[H.PROFILE_NORM_BWD] / 1e3) / 1e9
+            rooflines["norm_gate_bwd"] = {"bound": "hbm", "achieved": a_, "peak": hbm_peak, "unit": "GB/s",
+                                          "frac": a_ / hbm_peak, "algorithmic_bytes_per_launch": lnb_bytes,
+                                          "ms": kern_ms[H.PROFILE_NORM_BWD]}
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_oracle_sample(wl, backward)
         h2d = int((h_x.numel() + h_dy.numel()) * 2 + h_off.numel() * 8 + h_ts.numel() * 8)
+        d2h = int(h_y.numel() * 2 + ((h_dx.numel() * 2 + h_grads.numel() * 4) if backward else 0))
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": WORKLOADS[args.workload]["desc"], "global_batch": wl.B * world,
                        "tokens_per_rank": T, "seq_len": "jagged", "parallelism": f"dp{world}",
+                       "rank_cost_imbalance": float(rank_cost.max() / rank_cost.mean()) if world > 1 else 1.0,
                        "attention_operands": "fp16 U|V|Q|K, P and G, fp32 accumulation and O",
                        "l2": "flushed before every timed step (512 MB written, then 256 MB read)"},
-            "roofline": {"bound": "tensor", "kernel": "jagged attention forward (bias tiles + attn_fwd_tc2_kernel)",
-                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_kind": f"{peak_kind} bf16 sustained (dense)", "traffic": traffic_record(args.workload),
-                         "algorithmic_flops_per_launch": flops},
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_persistent_kernel (jagged pointwise attention forward)",
+                         "achieved": achieved, "peak": tf_peak, "unit": "TFLOP/s", "frac": achieved / tf_peak,
+                         "peak_kind": f"{peak_kind} bf16 burst (dense)", "traffic": traffic_record(args.workload),
+                         "algorithmic_flops_per_launch": flops, "ms": kern_ms[H.PROFILE_ATTN_FWD],
+                         "timing": "CUDA events recorded by the library right around the kernel, inside as many "
+                                   "timed replays of the step (a graph with those event nodes) as the headline"},
+            "rooflines": rooflines,
+            "workloads": extra,
             "step_breakdown_ms": {k: float(seg[:, i].mean()) for i, k in enumerate(names)},
-            "timing": "device time of CUDA-graph replays of the whole step (events on the launching stream); "
-                      "step_breakdown_ms from eager launches",
+            "timing": ("device time of CUDA-graph replays of the whole step" if world == 1 else
+                       "device time of eagerly launched steps, gradient all-reduce overlapped on a side stream") +
+                      " (events on the launching stream); step_breakdown_ms from eager launches",
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": int(h_y.numel() * 2)},
+                    "d2h_bytes_per_step": d2h, "d2h": "Y" + (", dX and the eight gradients" if backward else "")},
             "gpu_launches": int((n_fwd_kernels + (n_bwd_kernels if backward else 0)) * args.steps),
             "clocks": clk.summary(),
         }

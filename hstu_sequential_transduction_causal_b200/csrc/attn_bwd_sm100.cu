@@ -47,12 +47,13 @@ constexpr int kSiluThreadsB = 32 * kSiluWarpsB;
 // ----------------------------------------------------------------------------------------------
 // transposed bias and bucket tiles
 // ----------------------------------------------------------------------------------------------
-// One block per causal tile pair: the [key][query] half-bias and u8 bucket tiles of bias_tile.cuh.
+// Four blocks per causal tile pair: the [key][query] half-bias and u8 bucket tiles of bias_tile.cuh.
 __global__ void __launch_bounds__(kBiasThreads)
 attn_bias_t_kernel(AttnBwdArgs A) {
   pdl_enter();
   const long long tile0 = blockIdx.x * static_cast<long long>(kQTile * kQTile);
-  bias_tile_block<true, true>(A.f, blockIdx.x, reinterpret_cast<uint16_t*>(A.bias_t) + tile0,
+  const long long btile = (blockIdx.x * static_cast<long long>(A.f.bias_heads) + blockIdx.z) * (kQTile * kQTile);
+  bias_tile_block<true, true>(A.f, blockIdx.x, blockIdx.y, blockIdx.z, reinterpret_cast<uint16_t*>(A.bias_t) + btile,
                               reinterpret_cast<uint8_t*>(A.bucket_t) + tile0);
 }
 
@@ -85,9 +86,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const int h = blockIdx.x - item * a.H;
   if (item >= *A.kcount) return;
   const int b = A.kitems[2 * item];
-  const int kt = A.kitems[2 * item + 1];
-  const long long seq0 = a.offsets[b];
-  const int n = static_cast<int>(a.offsets[b + 1] - seq0);
+  const int kt_item = A.kitems[2 * item + 1];
+  const bool packed = kt_item < 0;         // a pack of -kt_item short sequences: one diagonal tile
+  const int kt = packed ? 0 : kt_item;
+  long long seq0;
+  int n;
+  pair_rows(a.offsets, a.pack, b, &seq0, &n);
   const int nt = (n + kQTile - 1) / kQTile;
   const int nsteps = nt - kt;              // query tiles kt .. nt-1
   const long long pbase = a.pair_base[b];
@@ -171,7 +175,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     auto load_bias = [&](int s) -> bool {
       const int st = s & 1, qt = kt + s;
       if (s >= 2 && !mbar_wait_warp(BAR(7 + st), ((s >> 1) & 1) ^ 1, abort_flag, ctl)) return false;
-      const int prow = static_cast<int>((pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt) * kQTile);
+      const long long pair = pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt;
+      const int prow = static_cast<int>((pair * a.bias_heads + (a.bias_heads > 1 ? h : 0)) * kQTile);
       if (lane == 0) mbar_arrive_expect_tx(BAR(5 + st), 32768);
       __syncwarp();
       const int hx = lane - 8 - 2 * st;
@@ -316,6 +321,18 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int sub = warp >> 3;
     const int rj = quad * 32 + lane;      // key row == TMEM lane of S^T, dA^T, dV, dK
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    // in a pack, queries past the end of the key row's own sequence are masked
+    int seg_end = n;
+    if (packed && rj < n) {
+      const long long g = seq0 + rj;
+      int s0 = b, s1 = b - kt_item;
+      while (s1 - s0 > 1) {
+        const int mid = (s0 + s1) >> 1;
+        if (a.offsets[mid] <= g) s0 = mid;
+        else s1 = mid;
+      }
+      seg_end = static_cast<int>(a.offsets[s0 + 1] - seq0);
+    }
     const float inv_N = a.inv_N;
     const float cN = 0.5f * inv_N;
     bool ok = true;
@@ -385,7 +402,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       // row past n keeps nothing (it only occurs in the diagonal tile of the last key tile)
       const bool need_mask = (s == 0) || (qt == nt - 1);
       const int lo_col = (s == 0) ? rj : 0;
-      const int hi_col = (kt * kQTile + rj < n) ? min(kQTile, n - qt * kQTile) : 0;
+      const int hi_col = (kt * kQTile + rj < n) ? min(kQTile, seg_end - qt * kQTile) : 0;
       uint8_t* bt_row = smem + Lb::kBT0 + st * 32768 + hq * 16384 + rj * 128;
 #pragma unroll
       for (int pc = 0; pc < 2; ++pc) {
@@ -478,11 +495,26 @@ attn_table_grad_kernel(AttnBwdArgs A) {
   const AttnArgs& a = A.f;
   int b, qt, kt;
   if (!decode_tile_pair(blockIdx.x, a.pair_base, a.B, &b, &qt, &kt)) return;
+  if (a.pack && a.pack[b] == 0) return;   // a packed sequence's own pair: its pack's tile holds its rows
   __shared__ float s_win[8][256];
   __shared__ float s_hist[128][32];
+  __shared__ float s_thist[16 * 16];
+  __shared__ int s_ty[256];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  // table slice hb: with tables shared by the heads (bias_heads 1) the block sums all H heads, with
+  // per-head tables only head hb
+  const int hb = blockIdx.z;
+  const int h_lo = a.bias_heads > 1 ? hb : 0, h_hi = a.bias_heads > 1 ? hb + 1 : a.H;
+  const int nt = a.n_types;
   for (int e = tid; e < 8 * 256; e += kTgThreads) (&s_win[0][0])[e] = 0.0f;
   for (int e = tid; e < 128 * 32; e += kTgThreads) (&s_hist[0][0])[e] = 0.0f;
+  if (nt > 0) {
+    s_thist[tid] = 0.0f;   // 256 threads, 16 x 16 entries
+    long long seq0;
+    int n;
+    if (pair_rows(a.offsets, a.pack, b, &seq0, &n))
+      tile_types_load(s_ty, a.token_type, seq0, n, qt * kQTile, kt * kQTile, nt, nullptr);
+  }
   const int g = lane >> 4, c0 = 8 * (lane & 15);
   const int j0 = 64 * static_cast<int>(blockIdx.y) + 8 * w + g;   // row of k = 0; row k is j0 + 2k
   const long long pair = blockIdx.x;
@@ -507,8 +539,8 @@ attn_table_grad_kernel(AttnBwdArgs A) {
       acc[k][2 * q + 1] += f.y;
     }
   };
-  int h = 0;
-  for (; h + 2 <= a.H; h += 2) {
+  int h = h_lo;
+  for (; h + 2 <= h_hi; h += 2) {
     uint4 v0[4], v1[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -521,7 +553,7 @@ attn_table_grad_kernel(AttnBwdArgs A) {
       add(k, v1[k]);
     }
   }
-  if (h < a.H) {
+  if (h < h_hi) {
 #pragma unroll
     for (int k = 0; k < 4; ++k)
       add(k, __ldg(reinterpret_cast<const uint4*>(src + (static_cast<long long>(h) * kQTile + 2 * k) * kQTile)));
@@ -570,21 +602,35 @@ attn_table_grad_kernel(AttnBwdArgs A) {
       }
     if (run != 0.0f) atomicAdd(&s_hist[cur][lane], run);
   }
+  // d rab_type[type_query][type_key]: element (key row j_k, query c0 + e)
+  if (nt > 0) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int tk = s_ty[128 + j0 + 2 * k];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (acc[k][e] != 0.0f) atomicAdd(&s_thist[s_ty[c0 + e] * nt + tk], acc[k][e]);
+    }
+  }
   __syncthreads();
   const int L = a.pos_max_len;
+  float* drab_pos = A.drab_pos + static_cast<long long>(hb) * (2 * L - 1);
+  float* drab_time = A.drab_time + static_cast<long long>(hb) * a.n_buckets;
   if (tid < 255) {
     float v = 0.0f;
 #pragma unroll
     for (int ww = 0; ww < 8; ++ww) v += s_win[ww][tid];
     if (v != 0.0f)
-      atomicAdd(A.drab_pos + bias_pos_index(static_cast<long long>(qt - kt) * kQTile + tid - 127, L), v);
+      atomicAdd(drab_pos + bias_pos_index(static_cast<long long>(qt - kt) * kQTile + tid - 127, L), v);
   }
   if (tid < a.n_buckets) {
     float v = 0.0f;
 #pragma unroll 8
     for (int l = 0; l < 32; ++l) v += s_hist[tid][(l + tid) & 31];
-    if (v != 0.0f) atomicAdd(A.drab_time + tid, v);
+    if (v != 0.0f) atomicAdd(drab_time + tid, v);
   }
+  if (nt > 0 && tid < nt * nt && s_thist[tid] != 0.0f)
+    atomicAdd(A.drab_type + static_cast<long long>(hb) * nt * nt + tid, s_thist[tid]);
 }
 
 }  // namespace
@@ -596,7 +642,8 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  e = launch_pdl(attn_bias_t_kernel, dim3(static_cast<unsigned>(a.max_pairs)), dim3(kBiasThreads), 0, st, A);
+  e = launch_pdl(attn_bias_t_kernel, dim3(static_cast<unsigned>(a.max_pairs), 4, static_cast<unsigned>(a.bias_heads)),
+                 dim3(kBiasThreads), 0, st, A);
   if (e != cudaSuccess) return e;
   // TMA row coordinates of the bias and dX^T tiles are 32-bit
   if (a.max_pairs * a.H * kQTile > 0x7fffffffLL) return cudaErrorInvalidValue;
@@ -607,7 +654,7 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
       !encode_tmap_2d_bf16(&tk, a.k, W, a.T, a.ld_k, 64, 128, f16) ||
       !encode_tmap_2d_bf16(&tv, a.v, W, a.T, a.ld_v, 64, 128, f16) ||
       !encode_tmap_2d_bf16(&tdo, A.dout, W, a.T, A.ld_do, 64, 128, f16) ||
-      !encode_tmap_2d_bf16(&tbt, A.bias_t, kQTile, a.max_pairs * kQTile, kQTile, 64, 128, true) ||
+      !encode_tmap_2d_bf16(&tbt, A.bias_t, kQTile, a.max_pairs * a.bias_heads * kQTile, kQTile, 64, 128, true) ||
       !encode_tmap_2d_bf16(&tdx, A.dxt, kQTile, a.max_pairs * a.H * kQTile, kQTile, 64, 128, f16) ||
       !encode_tmap_2d_out(&tdq, A.dq, kDtF32, W, a.T, A.ld_g, 32, 128))
     return cudaErrorInvalidValue;
@@ -615,11 +662,15 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), BwdSmem::kTotal);
   if (e != cudaSuccess) return e;
   const long long blocks = a.capacity * a.H;
-  e = launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(kThreadsB), BwdSmem::kTotal, st, tq, tk, tv, tdo, tbt,
-                 tdx, tdq, A, wait_ctl(a.status));
+  e = prof_record(kProfAttnBwd, false, st);
+  if (e == cudaSuccess)
+    e = launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(kThreadsB), BwdSmem::kTotal, st, tq, tk, tv, tdo,
+                   tbt, tdx, tdq, A, wait_ctl(a.status));
+  if (e == cudaSuccess) e = prof_record(kProfAttnBwd, true, st);
   if (e != cudaSuccess) return e;
   auto tg = f16 ? attn_table_grad_kernel<true> : attn_table_grad_kernel<false>;
-  return launch_pdl(tg, dim3(static_cast<unsigned>(a.max_pairs), 2), dim3(kTgThreads), 0, st, A);
+  return launch_pdl(tg, dim3(static_cast<unsigned>(a.max_pairs), 2, static_cast<unsigned>(a.bias_heads)),
+                    dim3(kTgThreads), 0, st, A);
 }
 
 }  // namespace hstu

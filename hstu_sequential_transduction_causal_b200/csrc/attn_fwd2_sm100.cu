@@ -52,13 +52,13 @@ constexpr uint32_t kHalf2Half = 0x38003800u;   // (0.5, 0.5) in fp16
 // ----------------------------------------------------------------------------------------------
 // 1. bias tiles
 // ----------------------------------------------------------------------------------------------
-// One block per causal tile pair (blocks past the batch's last pair exit at once): the [query][key]
+// Four blocks per causal tile pair (blocks past the batch's last pair exit at once): the [query][key]
 // half-bias tile of bias_tile.cuh.
 __global__ void __launch_bounds__(kBiasThreads)
 attn_bias_kernel(AttnArgs a) {
   pdl_enter();
-  bias_tile_block<false, false>(a, blockIdx.x,
-                                reinterpret_cast<uint16_t*>(a.bias) + blockIdx.x * static_cast<long long>(kQTile * kQTile),
+  const long long tile = (blockIdx.x * static_cast<long long>(a.bias_heads) + blockIdx.z) * (kQTile * kQTile);
+  bias_tile_block<false, false>(a, blockIdx.x, blockIdx.y, blockIdx.z, reinterpret_cast<uint16_t*>(a.bias) + tile,
                                 nullptr);
 }
 
@@ -448,6 +448,422 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
   }
 }
 
+// ----------------------------------------------------------------------------------------------
+// 3. persistent attention: one CTA per SM pulling (work item, head) units, longest first
+// ----------------------------------------------------------------------------------------------
+// Unit u = (work item u / H, head u % H): query tile qt of sequence b against key tiles 0..qt. CTAs
+// take units from a global counter in list order, so the longest causal rows go first and a CTA that
+// finishes early takes the next unit (list scheduling). Every ring below is indexed by the CTA's
+// running step count s (one step = one key tile of one unit), so the pipelines run across unit
+// boundaries: the next unit's Q and K loads and its first S MMAs are issued while the current
+// unit's last tiles are still in SiLU or P V, and the epilogue of a unit (O from TMEM, scaled by
+// 1/N) overlaps the next unit's MMAs through a second O accumulator.
+//   warps 0-15 : SiLU, two groups of 8 taking alternate steps (group s % 2); each warp one TMEM lane
+//                quadrant (warp & 3) and one key half ((warp >> 2) & 1). The group that runs a
+//                unit's last step also writes its output.
+//   warp 16    : scheduler (lane 0 takes the next unit, publishes it in a two-slot ring) and TMA
+//                producer of Q (two buffers), K and V (three stages each).
+//   warp 17    : tcgen05 issuer of S = Q K^T into three TMEM tiles.
+//   warp 18    : TMA producer of the bias tiles (three stages).
+//   warp 19    : tcgen05 issuer of O += P V, P read from TMEM, into two alternating O accumulators.
+struct Smem3 {
+  static constexpr int kNQ = 2, kNK = 3, kNV = 3, kBS = 3;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kNQ * 16384;
+  static constexpr int kV = kK + kNK * 16384;
+  static constexpr int kBias = kV + kNV * 16384;
+  static constexpr int kBar = kBias + kBS * 32768;
+  static constexpr int kTotal = kBar + 512 + 1024;
+};
+static_assert(Smem3::kTotal <= 232448, "shared memory of the persistent attention kernel");
+
+constexpr int kThreads3 = 32 * (2 * kSiluWarps + 4);
+constexpr int kUnitConsumers = 2 * kSiluWarps + 3;   // SiLU warps, S issuer, bias warp, P V issuer
+
+struct UnitRec {
+  int b, qt, h, valid;
+};
+
+template <bool F16>
+__global__ void __launch_bounds__(kThreads3, 1)
+attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB,
+                           AttnArgs a, WaitCtl ctl) {
+  pdl_enter();
+  using L = Smem3;
+  constexpr int NK = L::kNK, NV = L::kNV, BS = L::kBS;
+  static_assert(NK == 3 && NV == 3 && BS == 3, "the rings share the step index modulo 3");
+  constexpr int kTmaWarp = 2 * kSiluWarps, kSWarp = kTmaWarp + 1, kBiasWarp = kTmaWarp + 2, kPvWarp = kTmaWarp + 3;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  // 0 u_full[2] | 2 u_empty[2] | 4 q_full[2] | 6 q_empty[2] | 8 k_full[3] | 11 k_empty[3] | 14 v_full[3] |
+  // 17 v_empty[3] | 20 b_full[3] | 23 b_empty[3] | 26 s_full[3] | 29 p_full[3] | 32 pv_done[3] | 35 o_full[2] |
+  // 37 o_empty[2]
+  constexpr int kNumBars = 39;
+  UnitRec* ring = reinterpret_cast<UnitRec*>(smem + L::kBar + 320);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + 352);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBar + 356);
+  const uint32_t bar0 = smem_u32(bars);
+  auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  auto u_full = [&](int i) { return BAR(0 + i); };
+  auto u_empty = [&](int i) { return BAR(2 + i); };
+  auto q_full = [&](int i) { return BAR(4 + i); };
+  auto q_empty = [&](int i) { return BAR(6 + i); };
+  auto k_full = [&](int i) { return BAR(8 + i); };
+  auto k_empty = [&](int i) { return BAR(11 + i); };
+  auto v_full = [&](int i) { return BAR(14 + i); };
+  auto v_empty = [&](int i) { return BAR(17 + i); };
+  auto b_full = [&](int i) { return BAR(20 + i); };
+  auto b_empty = [&](int i) { return BAR(23 + i); };
+  auto s_full = [&](int i) { return BAR(26 + i); };
+  auto p_full = [&](int i) { return BAR(29 + i); };
+  auto pv_done = [&](int i) { return BAR(32 + i); };
+  auto o_full = [&](int i) { return BAR(35 + i); };
+  auto o_empty = [&](int i) { return BAR(37 + i); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr int kGroupThreads = 32 * kSiluWarps;
+  // a unit's query tile and key-tile count: a pack of short sequences (qt = -k) is one diagonal tile
+  auto unit_qt = [](int qt) { return qt < 0 ? 0 : qt; };
+  auto unit_nkt = [](int qt) { return qt < 0 ? 1 : qt + 1; };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(u_full(i), 1);
+      mbar_init(u_empty(i), kUnitConsumers);
+      mbar_init(q_full(i), 1);
+      mbar_init(q_empty(i), 1);
+      mbar_init(o_full(i), 1);
+      mbar_init(o_empty(i), kGroupThreads);
+    }
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(k_full(i), 1);
+      mbar_init(k_empty(i), 1);
+      mbar_init(v_full(i), 1);
+      mbar_init(v_empty(i), 1);
+      mbar_init(b_full(i), 1);
+      mbar_init(b_empty(i), kGroupThreads);
+      mbar_init(s_full(i), 1);
+      mbar_init(p_full(i), kGroupThreads);
+      mbar_init(pv_done(i), 1);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  static_assert(kNumBars * 8 <= 320, "barrier region");
+  if (warp == kTmaWarp && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // S / P tiles of steps s = 0, 1, 2 (mod 3) at columns [128 (s % 3), +128); O of units 0, 1 (mod 2) at
+  // [384 + 64 (u % 2), +64)
+  const uint32_t tmem = *tmem_slot;
+  constexpr uint32_t kOCol = 384;
+  const uint32_t sQ = smem_u32(smem + L::kQ), sK = smem_u32(smem + L::kK), sV = smem_u32(smem + L::kV);
+  const uint32_t sB = smem_u32(smem + L::kBias);
+
+  // The unit published in ring slot uc % 2 (consumers): lane 0 waits and reads, the warp gets it by
+  // shuffles, lane 0 then frees the slot.
+  auto take_unit = [&](int uc, UnitRec& r) -> bool {
+    const int slot = uc & 1;
+    if (!mbar_wait_warp(u_full(slot), (uc >> 1) & 1, abort_flag, ctl)) return false;
+    int v[4] = {0, 0, 0, 0};
+    if (lane == 0) {
+      const UnitRec x = ring[slot];
+      v[0] = x.b; v[1] = x.qt; v[2] = x.h; v[3] = x.valid;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __shfl_sync(0xffffffffu, v[i], 0);
+    r.b = v[0]; r.qt = v[1]; r.h = v[2]; r.valid = v[3];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(u_empty(slot));
+    return true;
+  };
+
+  if (warp == kTmaWarp) {
+    // ---------------- scheduler + Q / K / V producer ----------------
+    const long long total = static_cast<long long>(*a.count) * a.H;
+    int sg = 0;
+    bool ok = true;
+    auto load_v = [&](int s, int vrow, int h) -> bool {
+      const int st = s % NV;
+      if (s >= NV && !mbar_wait_warp(v_empty(st), ((s / NV) - 1) & 1, abort_flag, ctl)) return false;
+      if (lane == 8 + st) {
+        mbar_arrive_expect_tx(v_full(st), 16384);
+        tma_load_2d(sV + st * 16384, &tmV, v_full(st), h * kD, vrow);
+      }
+      return true;
+    };
+    for (int uc = 0; ok; ++uc) {
+      const int slot = uc & 1;
+      if (uc >= 2 && !mbar_wait_warp(u_empty(slot), ((uc >> 1) - 1) & 1, abort_flag, ctl)) break;
+      int v[4] = {0, 0, 0, 0};
+      if (lane == 0) {
+        for (;;) {
+          const long long u = atomicAdd(a.unit_counter, 1);
+          if (u >= total) break;
+          const int item = static_cast<int>(u / a.H);
+          const int b = a.items[2 * item], qt = a.items[2 * item + 1];
+          // prefix append: a query tile wholly inside the old prefix has nothing to write
+          if (a.q_from && static_cast<long long>(unit_qt(qt) + 1) * kQTile <= a.q_from[b + 1] - a.q_from[b]) continue;
+          v[0] = b;
+          v[1] = qt;
+          v[2] = static_cast<int>(u - static_cast<long long>(item) * a.H);
+          v[3] = 1;
+          break;
+        }
+        ring[slot] = UnitRec{v[0], v[1], v[2], v[3]};
+        mbar_arrive(u_full(slot));
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = __shfl_sync(0xffffffffu, v[i], 0);
+      if (!v[3]) break;
+      const int b = v[0], qt = unit_qt(v[1]), h = v[2];
+      const int row0 = static_cast<int>(a.offsets[b]);
+      const int nkt = unit_nkt(v[1]);
+      const int qb = uc & 1;
+      if (uc >= 2 && !mbar_wait_warp(q_empty(qb), ((uc >> 1) - 1) & 1, abort_flag, ctl)) break;
+      if (lane == 0) mbar_arrive_expect_tx(q_full(qb), 16384);
+      __syncwarp();
+      if (lane == 16 + qb) tma_load_2d(sQ + qb * 16384, &tmQ, q_full(qb), h * kD, row0 + qt * kQTile);
+      // K of step s first, V of step s - 1 after it: waiting for a V stage (freed late, by a P V MMA)
+      // never delays a K load
+      for (int kt = 0; ok && kt < nkt; ++kt) {
+        const int s = sg + kt, st = s % NK;
+        if (s >= NK && !mbar_wait_warp(k_empty(st), ((s / NK) - 1) & 1, abort_flag, ctl)) { ok = false; break; }
+        if (lane == st) {
+          mbar_arrive_expect_tx(k_full(st), 16384);
+          tma_load_2d(sK + st * 16384, &tmK, k_full(st), h * kD, row0 + kt * kQTile);
+        }
+        if (kt >= 1) ok = load_v(s - 1, row0 + (kt - 1) * kQTile, h);
+      }
+      if (ok) ok = load_v(sg + nkt - 1, row0 + (nkt - 1) * kQTile, h);
+      sg += nkt;
+    }
+  } else if (warp == kBiasWarp) {
+    // ---------------- bias tiles (stage bs: its two 64-column halves from lanes 2 bs, 2 bs + 1) ----
+    int sg = 0;
+    bool ok = true;
+    UnitRec r;
+    for (int uc = 0; ok && take_unit(uc, r) && r.valid; ++uc) {
+      const int qt = unit_qt(r.qt);
+      const long long pair0 = a.pair_base[r.b] + static_cast<long long>(qt) * (qt + 1) / 2;
+      const int nkt = unit_nkt(r.qt);
+      const int hb = a.bias_heads > 1 ? r.h : 0;
+      for (int kt = 0; kt < nkt; ++kt) {
+        const int s = sg + kt, bs = s % BS;
+        if (s >= BS && !mbar_wait_warp(b_empty(bs), ((s / BS) - 1) & 1, abort_flag, ctl)) { ok = false; break; }
+        const int brow = static_cast<int>(((pair0 + kt) * a.bias_heads + hb) * kQTile);
+        if (lane == 0) mbar_arrive_expect_tx(b_full(bs), 32768);
+        __syncwarp();
+        const int hx = lane - 2 * bs;
+        if (hx == 0 || hx == 1) tma_load_2d(sB + bs * 32768 + hx * 16384, &tmB, b_full(bs), 64 * hx, brow);
+      }
+      sg += nkt;
+    }
+  } else if (warp == kSWarp) {
+    // ---------------- S = Q K^T ----------------
+    constexpr uint32_t idesc_qk = make_idesc_f16kind(128, 128, 0, 0, F16);
+    const uint64_t q_desc0 = make_sdesc_sw128(sQ, 16, 1024), k_desc0 = make_sdesc_sw128(sK, 16, 1024);
+    int sg = 0;
+    bool ok = true;
+    UnitRec r;
+    for (int uc = 0; ok && take_unit(uc, r) && r.valid; ++uc) {
+      if (lane == 0) {
+        const int qb = uc & 1, nkt = unit_nkt(r.qt);
+        ok = mbar_wait(q_full(qb), (uc >> 1) & 1, abort_flag, ctl);
+        const uint64_t qd = sdesc_add(q_desc0, qb * 16384);
+        for (int kt = 0; ok && kt < nkt; ++kt) {
+          const int s = sg + kt, buf = s % 3;
+          if (!mbar_wait(k_full(buf), (s / 3) & 1, abort_flag, ctl) ||
+              (s >= 3 && !mbar_wait(pv_done(buf), ((s / 3) - 1) & 1, abort_flag, ctl))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t kd = sdesc_add(k_desc0, buf * 16384);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f16_ss(tmem + buf * 128, sdesc_add(qd, kk * 32), sdesc_add(kd, kk * 32), idesc_qk, kk > 0 ? 1u : 0u);
+          umma_commit(s_full(buf));
+          umma_commit(k_empty(buf));
+        }
+        if (ok) umma_commit(q_empty(qb));
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      sg += unit_nkt(r.qt);
+    }
+  } else if (warp == kPvWarp) {
+    // ---------------- O += P V ----------------
+    constexpr uint32_t idesc_pv = make_idesc_f16kind(128, 64, 0, 1, F16);
+    const uint64_t v_desc0 = make_sdesc_sw128(sV, 16384, 1024);
+    int sg = 0;
+    bool ok = true;
+    UnitRec r;
+    for (int uc = 0; ok && take_unit(uc, r) && r.valid; ++uc) {
+      if (lane == 0) {
+        const int ob = uc & 1, nkt = unit_nkt(r.qt);
+        if (uc >= 2) ok = mbar_wait(o_empty(ob), ((uc >> 1) - 1) & 1, abort_flag, ctl);
+        const uint32_t o_tmem = tmem + kOCol + 64 * ob;
+        for (int kt = 0; ok && kt < nkt; ++kt) {
+          const int s = sg + kt, buf = s % 3;
+          if (!mbar_wait(p_full(buf), (s / 3) & 1, abort_flag, ctl) ||
+              !mbar_wait(v_full(buf), (s / 3) & 1, abort_flag, ctl)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t vd = sdesc_add(v_desc0, buf * 16384);
+          const uint32_t a_tmem = tmem + buf * 128;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ts(o_tmem, a_tmem + 64 * (kk >> 2) + 8 * (kk & 3), sdesc_add(vd, kk * 2048), idesc_pv,
+                        (kk > 0 || kt > 0) ? 1u : 0u);
+          umma_commit(v_empty(buf));
+          umma_commit(pv_done(buf));
+        }
+        if (ok) umma_commit(o_full(ob));
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      sg += unit_nkt(r.qt);
+    }
+  } else {
+    // ---------------- SiLU warps ----------------
+    const int grp = warp / kSiluWarps;   // takes the steps s with s % 2 == grp
+    const int quad = warp & 3;
+    const int half = (warp >> 2) & 1;    // keys [64 half, 64 half + 64)
+    const int r = quad * 32 + lane;      // query row within the tile == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    int sg = 0;
+    bool ok = true;
+    UnitRec u;
+    for (int uc = 0; ok && take_unit(uc, u) && u.valid; ++uc) {
+      const int nkt = unit_nkt(u.qt), qt = unit_qt(u.qt);
+      // first key column this row may see: its own sequence's start inside a pack, else 0
+      int lo = 0;
+      if (u.qt < 0) {
+        const long long g = a.offsets[u.b] + r;
+        int s0 = u.b, s1 = u.b - u.qt;   // pack members b .. b + k - 1
+        while (s1 - s0 > 1) {
+          const int mid = (s0 + s1) >> 1;
+          if (a.offsets[mid] <= g) s0 = mid;
+          else s1 = mid;
+        }
+        lo = static_cast<int>(a.offsets[s0] - a.offsets[u.b]);
+      }
+      for (int kt = (sg & 1) == grp ? 0 : 1; ok && kt < nkt; kt += 2) {
+        const int s = sg + kt, buf = s % 3;
+        if (!mbar_wait(b_full(buf), (s / 3) & 1, abort_flag, ctl) ||
+            !mbar_wait(s_full(buf), (s / 3) & 1, abort_flag, ctl)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool diag = kt == qt;
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc) {
+          uint32_t sv[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + buf * 128 + 64 * half + 32 * hc, sv);
+          uint32_t hb[16];   // half-bias of keys [64 half + 32 hc, +32)
+          const uint8_t* brow = smem + L::kBias + buf * 32768 + half * 16384 + r * 128;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const uint4 v = *reinterpret_cast<const uint4*>(brow + (((4 * hc + q4) ^ (r & 7)) << 4));
+            hb[4 * q4] = v.x; hb[4 * q4 + 1] = v.y; hb[4 * q4 + 2] = v.z; hb[4 * q4 + 3] = v.w;
+          }
+          // the bias stage is free once both halves of this row are in registers
+          if (hc == 1) mbar_arrive(b_empty(buf));
+          tmem_ld_wait();
+          uint32_t p[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const uint32_t s2 = pack_f16x2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1]));
+            const uint32_t h2 = hfma2_u32(s2, kHalf2Half, hb[j]);
+            const uint32_t t2 = tanh_f16x2(h2);
+            uint32_t y2 = hfma2_u32(h2, t2, h2);
+            if (!F16) {   // the P V MMA takes A and B of one type: P as bf16 next to bf16 V
+              const float2 f = unpack_f16x2(y2);
+              y2 = pack_bf16x2(f.x, f.y);
+            }
+            if (diag) {   // keys lo <= col <= r
+              const int col = 64 * half + 32 * hc + 2 * j;
+              const uint32_t m = ((col <= r && col >= lo) ? 0x0000FFFFu : 0u) |
+                                 ((col + 1 <= r && col + 1 >= lo) ? 0xFFFF0000u : 0u);
+              y2 &= m;
+            }
+            p[j] = y2;
+          }
+          // P of these 32 keys packed into 16 columns over S chunk 0 (already read)
+          tmem_st_32x32b_x16(tmem + lane_base + buf * 128 + 64 * half + 16 * hc, p);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_full(buf));
+      }
+      // the group that ran the unit's last step writes its output: rows of this quadrant, columns
+      // [32 half, +32) of the head, times 1/N
+      if (ok && ((sg + nkt - 1) & 1) == grp) {
+        const int ob = uc & 1;
+        if (!mbar_wait(o_full(ob), (uc >> 1) & 1, abort_flag, ctl)) {
+          ok = false;
+        } else {
+          tc_fence_after();
+          uint32_t ov[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + kOCol + 64 * ob + 32 * half, ov);
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(o_empty(ob));
+          long long seq0;
+          int n;
+          pair_rows(a.offsets, a.pack, u.b, &seq0, &n);   // a pack's rows, or sequence b's
+          const int qi = qt * kQTile + r;
+          const long long q_lo = a.q_from ? a.q_from[u.b + 1] - a.q_from[u.b] : 0;
+          if (qi < n && qi >= q_lo) {
+            const float sc = a.inv_N;
+            const long long orow = seq0 + qi;
+            const int ocol = u.h * kD + 32 * half;
+            if (a.o_f32) {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + orow * a.ld_o + ocol);
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(__uint_as_float(ov[4 * q]) * sc, __uint_as_float(ov[4 * q + 1]) * sc,
+                                     __uint_as_float(ov[4 * q + 2]) * sc, __uint_as_float(ov[4 * q + 3]) * sc);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + orow * a.ld_o + ocol);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                dst[q] = make_uint4(
+                    pack_bf16x2(__uint_as_float(ov[8 * q]) * sc, __uint_as_float(ov[8 * q + 1]) * sc),
+                    pack_bf16x2(__uint_as_float(ov[8 * q + 2]) * sc, __uint_as_float(ov[8 * q + 3]) * sc),
+                    pack_bf16x2(__uint_as_float(ov[8 * q + 4]) * sc, __uint_as_float(ov[8 * q + 5]) * sc),
+                    pack_bf16x2(__uint_as_float(ov[8 * q + 6]) * sc, __uint_as_float(ov[8 * q + 7]) * sc));
+            }
+          }
+        }
+      }
+      sg += nkt;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // M-FALCON per-key half-bias: kbias[u * ld + j] = 0.5 (rab_pos[idx(n_u - j)] +
 // rab_time[bucket(request_ts[u] - t_j)]) for j < n_u, 0 up to ld. A prefix longer than ld is a
 // contract violation: recorded in the status word (the attention then stops at ld keys).
@@ -498,31 +914,54 @@ int64_t attn_max_pairs(int64_t capacity, int max_len) {
   return capacity * (mt + 1) / 2;
 }
 
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <bool F16>
+cudaError_t launch_attn_persistent(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                   const CUtensorMap& tb, const AttnArgs& a, cudaStream_t st) {
+  auto kern = attn_fwd_persistent_kernel<F16>;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), Smem3::kTotal);
+  if (e != cudaSuccess) return e;
+  const long long units = a.capacity * a.H;
+  const long long blocks = units < sm_count() ? units : sm_count();
+  if (blocks == 0) return cudaSuccess;
+  e = prof_record(kProfAttnFwd, false, st);
+  if (e == cudaSuccess)
+    e = launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(kThreads3), Smem3::kTotal, st, tq, tk, tv, tb, a,
+                   wait_ctl(a.status));
+  if (e == cudaSuccess) e = prof_record(kProfAttnFwd, true, st);
+  return e;
+}
+
 cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
   cudaError_t e = upload_time_taus();
   if (e != cudaSuccess) return e;
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  e = launch_pdl(attn_bias_kernel, dim3(static_cast<unsigned>(a.max_pairs)), dim3(kBiasThreads), 0, st, a);
+  e = launch_pdl(attn_bias_kernel, dim3(static_cast<unsigned>(a.max_pairs), 4, static_cast<unsigned>(a.bias_heads)),
+                 dim3(kBiasThreads), 0, st, a);
   if (e != cudaSuccess) return e;
   CUtensorMap tq, tk, tv, tb;
   const bool f16 = a.in_f16 != 0;
   if (!encode_tmap_2d_bf16(&tq, a.q, static_cast<int64_t>(a.H) * kD, a.T, a.ld_q, 64, 128, f16) ||
       !encode_tmap_2d_bf16(&tk, a.k, static_cast<int64_t>(a.H) * kD, a.T, a.ld_k, 64, 128, f16) ||
       !encode_tmap_2d_bf16(&tv, a.v, static_cast<int64_t>(a.H) * kD, a.T, a.ld_v, 64, 128, f16) ||
-      !encode_tmap_2d_bf16(&tb, a.bias, kQTile, a.max_pairs * kQTile, kQTile, 64, 128, true))
+      !encode_tmap_2d_bf16(&tb, a.bias, kQTile, a.max_pairs * a.bias_heads * kQTile, kQTile, 64, 128, true))
     return cudaErrorInvalidValue;
-  // Two heads per CTA share the Q-independent bias tile, but double the longest CTA's work: with
-  // long sequences (many key tiles in one query tile) the longest chain sets the kernel time, so one
-  // head per CTA is used there.
-  const int max_tiles = (a.max_len + kQTile - 1) / kQTile;
-  const int G = (a.H % 2 == 0 && max_tiles <= 8) ? 2 : 1;
-  if (f16)
-    return G == 2 ? launch_attn2<true, 2, false>(tq, tk, tv, tb, a, st)
-                  : launch_attn2<true, 1, false>(tq, tk, tv, tb, a, st);
-  return G == 2 ? launch_attn2<false, 2, false>(tq, tk, tv, tb, a, st)
-                : launch_attn2<false, 1, false>(tq, tk, tv, tb, a, st);
+  // the persistent kernel's unit counter lives in the workspace header (reset by the work list)
+  if (!a.unit_counter) return cudaErrorInvalidValue;
+  return f16 ? launch_attn_persistent<true>(tq, tk, tv, tb, a, st) : launch_attn_persistent<false>(tq, tk, tv, tb, a, st);
 }
 
 cudaError_t falcon_key_bias(const int64_t* offsets, const int64_t* ts, int users, int max_len,

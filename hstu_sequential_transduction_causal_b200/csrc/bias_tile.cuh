@@ -1,12 +1,12 @@
-// bias_tile.cuh - the relative half-bias of one causal (query tile, key tile) pair, computed by one
-// block of 256 threads:
+// bias_tile.cuh - the relative half-bias of one causal (query tile, key tile) pair, computed by four
+// blocks of 256 threads (32 rows each):
 //   bias(i, j) = 0.5 (rab_pos[clamp(i - j)] + rab_time[bucket(t_i - t_j)])
 // ("HSTU: The First Exploration of the Scaling Law", 7.1.4 Innovation 2: position and time bias;
 // the buckets of time_bucket_dev.cuh). The bias does not depend on the head, so a pair's tile is
 // computed once and read by every head.
 //
-// Thread t takes the column pairs 2 (t % 16) + 32 e, e < 4, of the rows t / 16 + 16 p, p < 8: 64
-// elements, 4-byte half-bias (and 2-byte bucket) stores. TRANSPOSED: rows are keys and columns
+// Thread t of block rb takes the column pairs 2 (t % 16) + 32 e, e < 4, of the rows 32 rb + t / 16 +
+// 16 p, p < 2: 16 elements, 4-byte half-bias (and 2-byte bucket) stores. TRANSPOSED: rows are keys and columns
 // queries (the backward's [key][query] tiles); otherwise rows are queries. Timestamps past
 // the sequence end are clamped to its last token (those elements are masked by the attention).
 // When every difference of the tile fits in int32 (spans under 68 years of seconds) the bucket
@@ -95,22 +95,49 @@ __device__ __forceinline__ int tile_bucket(const TileTimes& s, bool fast, int r,
               : time_bucket_pair64(s.ts[qi], s.ts[128 + kj], tau, nb);
 }
 
+// Token types of a staged tile, clamped into [0, nt) (a type outside it is reported): ty[0, 128) the
+// query rows, ty[128, 256) the key rows, like TileTimes.
+__device__ __forceinline__ void tile_types_load(int* ty, const int32_t* __restrict__ types, long long seq0, int n,
+                                                int q0, int k0, int nt, int* status) {
+  const int tid = threadIdx.x;
+  const int idx = (tid < 128 ? q0 : k0) + (tid & 127);
+  int t = types[seq0 + (idx < n ? idx : n - 1)];
+  if (t < 0 || t >= nt) {
+    if (idx < n) report_error(status, kDevBadInput);
+    t = t < 0 ? 0 : nt - 1;
+  }
+  ty[tid] = t;
+}
+
+// Rows [32 rb, 32 rb + 32) of the tile of causal pair `pair` for bias head slice hb (four blocks cover
+// a tile, so that a batch of a few hundred pairs still puts several blocks on every SM). With per-head
+// tables (bias_heads = H) every head has its own tile; with a type term each element also adds
+// rab_type[type_query][type_key]. BUCKETS: also the u8 bucket tile (head-independent, written by the
+// hb = 0 blocks).
 template <bool TRANSPOSED, bool BUCKETS>
-__device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pair, uint16_t* __restrict__ tile,
-                                                uint8_t* __restrict__ btile) {
+__device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pair, int rb, int hb,
+                                                uint16_t* __restrict__ tile, uint8_t* __restrict__ btile) {
   __shared__ TileTimes s_t;
   __shared__ long long s_tau[kTauEntries];
   __shared__ int s_tau32[kTauEntries];
   __shared__ float s_win[256], s_rt[128];
-  int b, qt, kt;
+  __shared__ int s_ty[256];
+  __shared__ float s_tt[16 * 16];
+  int b, qt, kt, n;
+  long long seq0;
   if (!decode_tile_pair(pair, a.pair_base, a.B, &b, &qt, &kt)) return;
-  const long long seq0 = a.offsets[b];
-  const int n = static_cast<int>(a.offsets[b + 1] - seq0);
+  if (!pair_rows(a.offsets, a.pack, b, &seq0, &n)) return;   // a packed sequence's own pair: unused
   const int tid = threadIdx.x;
+  const int L = a.pos_max_len, nt = a.n_types;
+  const float* rab_pos = a.rab_pos + static_cast<long long>(hb) * (2 * L - 1);
+  const float* rab_time = a.rab_time + static_cast<long long>(hb) * a.n_buckets;
   tile_times_load(s_t, a.ts, seq0, n, qt * kQTile, kt * kQTile);
-  if (tid < a.n_buckets) s_rt[tid] = 0.5f * a.rab_time[tid];
-  if (tid < 255) s_win[tid] = 0.5f * a.rab_pos[bias_pos_index(static_cast<long long>(qt - kt) * kQTile - 127 + tid,
-                                                               a.pos_max_len)];
+  if (tid < a.n_buckets) s_rt[tid] = 0.5f * rab_time[tid];
+  if (tid < 255) s_win[tid] = 0.5f * rab_pos[bias_pos_index(static_cast<long long>(qt - kt) * kQTile - 127 + tid, L)];
+  if (nt > 0) {
+    tile_types_load(s_ty, a.token_type, seq0, n, qt * kQTile, kt * kQTile, nt, a.status);
+    if (tid < nt * nt) s_tt[tid] = 0.5f * a.rab_type[static_cast<long long>(hb) * nt * nt + tid];
+  }
   for (int e = tid; e < kTauEntries; e += kBiasThreads) {
     s_tau[e] = c_time_taus[e];
     s_tau32[e] = c_time_taus32[e];
@@ -118,14 +145,15 @@ __device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pai
   __syncthreads();
   const bool fast = tile_times_finish(s_t);
   const int nb = a.n_buckets;
-  // thread: column pairs c = 2 (tid % 16) + 32 e + x (e < 4, x < 2) of rows r = tid / 16 + 16 p (p < 8).
-  // The 16 lanes of a half-warp read 32 consecutive diagonals of the rab_pos window (no bank
+  const bool buckets = BUCKETS && hb == 0;
+  // thread: column pairs c = 2 (tid % 16) + 32 e + x (e < 4, x < 2) of rows r = 32 rb + tid / 16 + 16 p
+  // (p < 2). The 16 lanes of a half-warp read 32 consecutive diagonals of the rab_pos window (no bank
   // conflicts) and store 64 contiguous bytes of one row.
-  const int cl = 2 * (tid & 15), rr = tid >> 4;
+  const int cl = 2 * (tid & 15), rr = 32 * rb + (tid >> 4);
   auto row_pass = [&](auto fast_tag) {
     constexpr bool kFast = decltype(fast_tag)::value;
-#pragma unroll 2
-    for (int p = 0; p < 8; ++p) {
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
       const int r = rr + 16 * p;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -135,11 +163,13 @@ __device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pai
         for (int x = 0; x < 2; ++x) {
           const int c = cl + 32 * e + x;
           const int bkt = tile_bucket<TRANSPOSED>(s_t, kFast, r, c, s_tau, s_tau32, nb);
-          v2[x] = s_win[TRANSPOSED ? c - r + 127 : r - c + 127] + s_rt[bkt];
+          float v = s_win[TRANSPOSED ? c - r + 127 : r - c + 127] + s_rt[bkt];
+          if (nt > 0) v += s_tt[s_ty[TRANSPOSED ? c : r] * nt + s_ty[128 + (TRANSPOSED ? r : c)]];
+          v2[x] = v;
           bw |= static_cast<uint32_t>(bkt) << (8 * x);
         }
         *reinterpret_cast<uint32_t*>(tile + r * kQTile + cl + 32 * e) = pack_f16x2(v2[0], v2[1]);
-        if (BUCKETS) *reinterpret_cast<uint16_t*>(btile + r * kQTile + cl + 32 * e) = static_cast<uint16_t>(bw);
+        if (buckets) *reinterpret_cast<uint16_t*>(btile + r * kQTile + cl + 32 * e) = static_cast<uint16_t>(bw);
       }
     }
   };

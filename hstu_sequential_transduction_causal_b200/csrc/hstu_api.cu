@@ -18,6 +18,8 @@ namespace hstu {
 namespace {
 
 thread_local int32_t g_last_cuda_error = 0;
+thread_local cudaEvent_t g_prof_events[kProfKernels][2] = {};
+thread_local cudaEvent_t g_ready_events[2] = {};   // hstu_layer_bwd_ready_events: early, w1
 std::atomic<unsigned long long> g_wait_limit{1ull << 31};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -53,22 +55,26 @@ int* ws_status(void* ws) { return static_cast<int*>(ws); }
 // attention workspace: [0,256) status | [256,512) count | [512, ...) items (int32 x 2 x capacity)
 int64_t capacity_of(const hstu_jagged_t* j) { return static_cast<int64_t>(j->B) + (j->T + kQTile - 1) / kQTile; }
 
-// attention workspace: [0,256) status | [256,512) work-list count | items (int32 x 2 x capacity) |
-// pair_base (int64 x (B+1)) | fp16 bias tiles (32 KB per causal tile pair, 1024-aligned)
+// attention workspace: [0,256) status | [256,512) work-list counts (256: forward items, 260: backward
+// items, 272: the persistent forward's unit counter) | items (int32 x 2 x capacity) |
+// pair_base (int64 x (B+1)) | pack (int32 x B: short sequences sharing a tile) | fp16 bias tiles
+// (32 KB per causal tile pair and bias slice, 1024-aligned)
 struct AttnWs {
-  size_t items, pairs, bias, items_end, total;
+  size_t items, pairs, pack, bias, items_end, total;
   int64_t max_pairs;
 };
 
-AttnWs attn_ws_layout(const hstu_jagged_t* j) {
+// hb: bias tiles per causal pair (1, or H for per-head bias tables)
+AttnWs attn_ws_layout(const hstu_jagged_t* j, int hb = 1) {
   AttnWs w{};
   const int64_t cap = capacity_of(j);
   w.items = kWsHeader + 256;
   w.items_end = w.items + align_up(static_cast<size_t>(cap) * 8, 256);
   w.pairs = w.items_end;
-  w.bias = align_up(w.pairs + align_up(static_cast<size_t>(j->B + 1) * 8, 256), 1024);
+  w.pack = w.pairs + align_up(static_cast<size_t>(j->B + 1) * 8, 256);
+  w.bias = align_up(w.pack + align_up(static_cast<size_t>(j->B) * 4, 256), 1024);
   w.max_pairs = attn_max_pairs(cap, j->max_len);
-  w.total = w.bias + static_cast<size_t>(w.max_pairs) * kQTile * kQTile * 2;
+  w.total = w.bias + static_cast<size_t>(w.max_pairs) * hb * kQTile * kQTile * 2;
   return w;
 }
 
@@ -79,7 +85,9 @@ size_t attn_ws_bytes(const hstu_jagged_t* j) { return attn_ws_layout(j).total; }
 // beyond that (hundreds of GB of workspace) is refused on the host, before any size is computed
 // in size_t or anything is enqueued.
 constexpr int64_t kMaxTmaRows = 0x7fffffffLL;
-bool fwd_pairs_fit(const hstu_jagged_t* j) { return attn_ws_layout(j).max_pairs <= kMaxTmaRows / kQTile; }
+bool fwd_pairs_fit(const hstu_jagged_t* j, int hb = 1) {
+  return attn_ws_layout(j).max_pairs <= kMaxTmaRows / (static_cast<int64_t>(hb) * kQTile);
+}
 bool bwd_pairs_fit(const hstu_jagged_t* j, int H) {
   return H > 0 && attn_ws_layout(j).max_pairs <= kMaxTmaRows / (static_cast<int64_t>(H) * kQTile);
 }
@@ -92,14 +100,14 @@ struct AttnBwdWs {
   size_t kitems, bias_t, bucket_t, dxt, total;
 };
 
-AttnBwdWs attn_bwd_ws_layout(const hstu_jagged_t* j, int H) {
+AttnBwdWs attn_bwd_ws_layout(const hstu_jagged_t* j, int H, int hb = 1) {
   AttnBwdWs w{};
   w.f = attn_ws_layout(j);
   const int64_t cap = capacity_of(j);
   const size_t tile = static_cast<size_t>(kQTile) * kQTile;
   w.kitems = w.f.bias;   // the forward bias region is not used by the backward
   w.bias_t = align_up(w.kitems + align_up(static_cast<size_t>(cap) * 8, 256), 1024);
-  w.bucket_t = w.bias_t + static_cast<size_t>(w.f.max_pairs) * tile * 2;
+  w.bucket_t = w.bias_t + static_cast<size_t>(w.f.max_pairs) * hb * tile * 2;
   w.dxt = align_up(w.bucket_t + static_cast<size_t>(w.f.max_pairs) * tile, 1024);
   w.total = w.dxt + static_cast<size_t>(w.f.max_pairs) * (H > 0 ? H : 0) * tile * 2;
   return w;
@@ -140,10 +148,14 @@ LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) 
 hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const void* q, const void* k,
                            const void* v, const void* d_out, const float* rab_pos, const float* rab_time, float* dq,
                            float* dk, float* dv, int64_t ld_g, float* d_rab_pos, float* d_rab_time, void* ws,
-                           cudaStream_t st) {
-  const AttnBwdWs lay = attn_bwd_ws_layout(jag, desc->H);
-  cudaError_t e = cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * (2 * static_cast<size_t>(desc->pos_max_len) - 1), st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, sizeof(float) * desc->n_time_buckets, st);
+                           cudaStream_t st, const hstu_rab_ext_t* ext = nullptr, float* d_rab_type = nullptr) {
+  const int hb = ext && ext->per_head ? desc->H : 1;
+  const int nt = ext ? ext->n_types : 0;
+  const AttnBwdWs lay = attn_bwd_ws_layout(jag, desc->H, hb);
+  cudaError_t e =
+      cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * hb * (2 * static_cast<size_t>(desc->pos_max_len) - 1), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, sizeof(float) * hb * desc->n_time_buckets, st);
+  if (e == cudaSuccess && nt > 0) e = cudaMemsetAsync(d_rab_type, 0, sizeof(float) * hb * nt * nt, st);
   if (e != cudaSuccess) return cuda_status(e);
   if (jag->T == 0) return HSTU_OK;
   e = cudaMemsetAsync(dq, 0, sizeof(float) * static_cast<size_t>(jag->T) * ld_g, st);
@@ -165,12 +177,15 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
   a.max_pairs = lay.f.max_pairs;
   A.dout = d_out; A.ld_do = desc->ld_o;
   A.dq = dq; A.dk = dk; A.dv = dv; A.ld_g = ld_g;
-  A.drab_pos = d_rab_pos; A.drab_time = d_rab_time;
+  A.drab_pos = d_rab_pos; A.drab_time = d_rab_time; A.drab_type = d_rab_type;
+  a.bias_heads = hb; a.n_types = nt;
+  if (nt > 0) { a.token_type = ext->token_type; a.rab_type = ext->rab_type; }
   A.bias_t = w + lay.bias_t; A.bucket_t = w + lay.bucket_t; A.dxt = w + lay.dxt;
   A.kitems = reinterpret_cast<int32_t*>(w + lay.kitems); A.kcount = kcount;
+  a.pack = reinterpret_cast<const int32_t*>(w + lay.f.pack);
   e = launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, a.status, st,
                       reinterpret_cast<long long*>(w + lay.f.pairs), reinterpret_cast<int32_t*>(w + lay.kitems),
-                      kcount);
+                      kcount, nullptr, reinterpret_cast<int32_t*>(w + lay.f.pack));
   if (e == cudaSuccess) e = attn_bwd_tc(A, st);
   return cuda_status(e);
 }
@@ -210,9 +225,11 @@ hstu_status_t check_attn(const hstu_attn_desc_t* d, const hstu_jagged_t* j) {
 // fits and the tensor-core path runs the kernel that evaluates the bias per element and head.
 hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, const void* q, const void* k,
                            const void* v, const float* rab_pos, const float* rab_time, void* out, void* ws,
-                           cudaStream_t st, bool tile_pairs = true) {
+                           cudaStream_t st, bool tile_pairs = true, const hstu_rab_ext_t* ext = nullptr,
+                           const int64_t* q_from = nullptr) {
   const int64_t cap = capacity_of(j);
-  const AttnWs lay = attn_ws_layout(j);
+  const int hb = ext && ext->per_head ? d->H : 1;
+  const AttnWs lay = attn_ws_layout(j, hb);
   uint8_t* w = static_cast<uint8_t*>(ws);
   int32_t* count = reinterpret_cast<int32_t*>(w + kWsHeader);
   int32_t* items = reinterpret_cast<int32_t*>(w + lay.items);
@@ -225,14 +242,23 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
   a.in_f16 = d->dtype == HSTU_F16;
   a.rab_pos = rab_pos; a.rab_time = rab_time; a.items = items; a.count = count; a.capacity = cap;
   a.status = ws_status(ws);
+  a.bias_heads = hb;
+  a.q_from = q_from;
+  if (ext && ext->n_types > 0) {
+    a.n_types = ext->n_types; a.token_type = ext->token_type; a.rab_type = ext->rab_type;
+  }
   const bool pairs = tile_pairs && is_tc_dtype(d->dtype);
   if (pairs) {
     a.pair_base = reinterpret_cast<const long long*>(w + lay.pairs);
     a.bias = w + lay.bias;
     a.max_pairs = lay.max_pairs;
+    a.unit_counter = count + 4;   // [272, 276) of the workspace header region
+    // short sequences share tiles, except in a prefix append (whose rows start mid-sequence)
+    if (!q_from) a.pack = reinterpret_cast<const int32_t*>(w + lay.pack);
   }
   cudaError_t e = launch_worklist(j->offsets, j->B, j->T, j->max_len, items, count, a.status, st,
-                                  pairs ? reinterpret_cast<long long*>(w + lay.pairs) : nullptr);
+                                  pairs ? reinterpret_cast<long long*>(w + lay.pairs) : nullptr, nullptr, nullptr,
+                                  pairs ? a.unit_counter : nullptr, const_cast<int32_t*>(a.pack));
   if (e != cudaSuccess) return cuda_status(e);
   if (j->T == 0) return HSTU_OK;
   if (!is_tc_dtype(d->dtype)) e = attn_fwd_f32_simt(a, st);
@@ -298,6 +324,16 @@ hstu_status_t check_dense(int64_t T, int32_t D, hstu_dtype_t dtype) {
 }  // namespace
 
 WaitCtl wait_ctl(int* status) { return WaitCtl{status, g_wait_limit.load(std::memory_order_relaxed)}; }
+
+cudaError_t prof_record(int kernel, bool stop, cudaStream_t st) {
+  if (kernel < 0 || kernel >= kProfKernels) return cudaSuccess;
+  cudaEvent_t ev = g_prof_events[kernel][stop ? 1 : 0];
+  if (!ev) return cudaSuccess;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(st, &cs);
+  if (e != cudaSuccess) return e;
+  return cs == cudaStreamCaptureStatusNone ? cudaEventRecord(ev, st) : cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+}
 
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld_elems,
                          int box_inner, int box_outer, bool f16) {
@@ -403,6 +439,20 @@ hstu_status_t hstu_sync_status(void* ws, hstu_stream_t stream, int32_t* device_s
   return HSTU_OK;
 }
 
+hstu_status_t hstu_profile_events(int32_t kernel, void* start, void* stop) {
+  if (kernel < 0 || kernel >= kProfKernels || (start == nullptr) != (stop == nullptr)) return HSTU_ERR_INVALID_ARG;
+  g_prof_events[kernel][0] = static_cast<cudaEvent_t>(start);
+  g_prof_events[kernel][1] = static_cast<cudaEvent_t>(stop);
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_layer_bwd_ready_events(void* early, void* w1) {
+  if ((early == nullptr) != (w1 == nullptr)) return HSTU_ERR_INVALID_ARG;
+  g_ready_events[0] = static_cast<cudaEvent_t>(early);
+  g_ready_events[1] = static_cast<cudaEvent_t>(w1);
+  return HSTU_OK;
+}
+
 hstu_status_t hstu_debug_timeout_probe(void* ws, size_t ws_bytes, hstu_stream_t stream) {
   if (!ws) return HSTU_ERR_INVALID_ARG;
   if (ws_bytes < kWsHeader) return HSTU_ERR_WORKSPACE;
@@ -468,6 +518,68 @@ hstu_status_t hstu_attn_fwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
   if (is_tc_dtype(desc->dtype) && jag->T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)))
     return HSTU_ERR_UNSUPPORTED;
   return run_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, ws, stream);
+}
+
+// ext: per_head 0 or 1, n_types 0..16 with its pointers when T > 0; tensor-core dtypes only
+hstu_status_t check_rab_ext(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const hstu_rab_ext_t* ext) {
+  if (!ext || (ext->per_head != 0 && ext->per_head != 1) || ext->n_types < 0) return HSTU_ERR_INVALID_ARG;
+  if (ext->n_types > 16) return HSTU_ERR_UNSUPPORTED;
+  if (ext->n_types > 0 && jag->T > 0 && (!ext->token_type || !ext->rab_type)) return HSTU_ERR_INVALID_ARG;
+  if (!is_tc_dtype(desc->dtype)) return HSTU_ERR_UNSUPPORTED;
+  return HSTU_OK;
+}
+
+size_t hstu_attn_ext_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const hstu_rab_ext_t* ext) {
+  if (!desc || !ext || check_jagged(jag) != HSTU_OK || desc->H <= 0) return 0;
+  const int hb = ext->per_head ? desc->H : 1;
+  if (!fwd_pairs_fit(jag, hb)) return 0;
+  return attn_ws_layout(jag, hb).total;
+}
+
+hstu_status_t hstu_attn_fwd_ext(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const hstu_rab_ext_t* ext,
+                                const void* q, const void* k, const void* v, const float* rab_pos,
+                                const float* rab_time, void* out, void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  hstu_status_t s = check_attn(desc, jag);
+  if (s != HSTU_OK) return s;
+  s = check_rab_ext(desc, jag, ext);
+  if (s != HSTU_OK) return s;
+  const int hb = ext->per_head ? desc->H : 1;
+  if (!fwd_pairs_fit(jag, hb)) return HSTU_ERR_UNSUPPORTED;
+  if (!ws) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < attn_ws_layout(jag, hb).total) return HSTU_ERR_WORKSPACE;
+  if (jag->T > 0 && (!q || !k || !v || !rab_pos || !rab_time || !out)) return HSTU_ERR_INVALID_ARG;
+  if (jag->T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))) return HSTU_ERR_UNSUPPORTED;
+  return run_attn_fwd(desc, jag, q, k, v, rab_pos, rab_time, out, ws, stream, true, ext);
+}
+
+size_t hstu_attn_bwd_ext_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag,
+                                        const hstu_rab_ext_t* ext) {
+  if (!desc || !ext || check_jagged(jag) != HSTU_OK || !bwd_pairs_fit(jag, desc->H)) return 0;
+  return attn_bwd_ws_layout(jag, desc->H, ext->per_head ? desc->H : 1).total;
+}
+
+hstu_status_t hstu_attn_bwd_ext(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const hstu_rab_ext_t* ext,
+                                const void* q, const void* k, const void* v, const void* d_out,
+                                const float* rab_pos, const float* rab_time, float* dq, float* dk, float* dv,
+                                float* d_rab_pos, float* d_rab_time, float* d_rab_type, void* ws,
+                                size_t ws_bytes, hstu_stream_t stream) {
+  hstu_status_t s = check_attn(desc, jag);
+  if (s != HSTU_OK) return s;
+  s = check_rab_ext(desc, jag, ext);
+  if (s != HSTU_OK) return s;
+  if (!bwd_pairs_fit(jag, desc->H)) return HSTU_ERR_UNSUPPORTED;
+  if (!ws) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < attn_bwd_ws_layout(jag, desc->H, ext->per_head ? desc->H : 1).total) return HSTU_ERR_WORKSPACE;
+  if (!d_rab_pos || !d_rab_time || (ext->n_types > 0 && !d_rab_type)) return HSTU_ERR_INVALID_ARG;
+  if (jag->T > 0) {
+    if (!q || !k || !v || !d_out || !rab_pos || !rab_time || !dq || !dk || !dv) return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_out) || !aligned16(dq) || !aligned16(dk) ||
+        !aligned16(dv))
+      return HSTU_ERR_UNSUPPORTED;
+  }
+  const int64_t W = static_cast<int64_t>(desc->H) * desc->d_qk;
+  return run_attn_bwd(desc, jag, q, k, v, d_out, rab_pos, rab_time, dq, dk, dv, W, d_rab_pos, d_rab_time, ws, stream,
+                      ext, d_rab_type);
 }
 
 size_t hstu_attn_bwd_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag) {
@@ -569,9 +681,16 @@ size_t hstu_layer_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagge
   return layer_fwd_layout(desc, jag).total;
 }
 
-hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag, const hstu_layer_weights_t* w,
-                             const void* x, const void* x_f16, void* y, void* y_f16, const hstu_layer_saved_t* saved,
-                             void* ws, size_t ws_bytes, hstu_stream_t stream) {
+}  // extern "C"
+
+namespace hstu {
+namespace {
+
+// The layer forward. resid_dtype: the dtype of x as the residual (desc->x_dtype, except for the
+// norm_in variant, which passes an F32 descriptor so that f1 reads x_f16 = Xn, with a bf16 or fp32 X).
+hstu_status_t run_layer_fwd(const hstu_layer_desc_t* desc, hstu_dtype_t resid_dtype, const hstu_jagged_t* jag,
+                            const hstu_layer_weights_t* w, const void* x, const void* x_f16, void* y, void* y_f16,
+                            const hstu_layer_saved_t* saved, void* ws, size_t ws_bytes, hstu_stream_t stream) {
   if (!desc || !w || !saved) return HSTU_ERR_INVALID_ARG;
   hstu_status_t s = check_jagged(jag);
   if (s != HSTU_OK) return s;
@@ -634,8 +753,19 @@ hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   cudaError_t e = norm_gate_fwd(T, D, kDtF32, act, g_dt, saved->o, D, uvqk, 4ll * D, w->gamma, w->beta,
                                 desc->ln_eps, saved->g, saved->mu, saved->rstd, st);
   if (e != cudaSuccess) return cuda_status(e);
-  return run_out_proj(T, D, desc->dtype, g_dt, saved->g, w->W2, w->b2, x, desc->x_dtype, y, desc->y_dtype, y_f16,
+  return run_out_proj(T, D, desc->dtype, g_dt, saved->g, w->W2, w->b2, x, resid_dtype, y, desc->y_dtype, y_f16,
                       status, st, wsb + lay.w2_f16);
+}
+
+}  // namespace
+}  // namespace hstu
+
+extern "C" {
+
+hstu_status_t hstu_layer_fwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag, const hstu_layer_weights_t* w,
+                             const void* x, const void* x_f16, void* y, void* y_f16, const hstu_layer_saved_t* saved,
+                             void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  return run_layer_fwd(desc, desc ? desc->x_dtype : HSTU_F32, jag, w, x, x_f16, y, y_f16, saved, ws, ws_bytes, stream);
 }
 
 hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, int64_t lda, int32_t a_mn,
@@ -676,10 +806,18 @@ size_t hstu_layer_bwd_workspace_size(const hstu_layer_desc_t* desc, const hstu_j
   return layer_bwd_layout(desc, jag).total;
 }
 
-hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag, const hstu_layer_weights_t* w,
-                             const void* x, const void* x_f16, const hstu_layer_saved_t* saved, const void* dy,
-                             const void* dy_f16, void* dx, void* dx_f16, const hstu_layer_grads_t* gr, void* ws,
-                             size_t ws_bytes, hstu_stream_t stream) {
+}  // extern "C"
+
+namespace hstu {
+namespace {
+
+// The layer backward; with nin (the norm_in variant) dW1 reads the saved Xn and the last GEMM writes
+// dXn = dZ W1 (fp32, no residual) after the layer workspace, from which the input LayerNorm's
+// backward forms dX = dY + LN_in^T(dXn), dgamma_in and dbeta_in.
+hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag, const hstu_layer_weights_t* w,
+                            const void* x, const void* x_f16, const hstu_layer_saved_t* saved, const void* dy,
+                            const void* dy_f16, void* dx, void* dx_f16, const hstu_layer_grads_t* gr, void* ws,
+                            size_t ws_bytes, hstu_stream_t stream, const hstu_norm_in_t* nin) {
   if (!desc || !w || !saved || !gr) return HSTU_ERR_INVALID_ARG;
   hstu_status_t s = check_jagged(jag);
   if (s != HSTU_OK) return s;
@@ -698,7 +836,9 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
     return HSTU_ERR_UNSUPPORTED;
   if (!ws) return HSTU_ERR_INVALID_ARG;
   const LayerBwdWs lay = layer_bwd_layout(desc, jag);
-  if (ws_bytes < lay.total) return HSTU_ERR_WORKSPACE;
+  const size_t nin_dxn = lay.total;
+  const size_t nin_part = align_up(nin_dxn + static_cast<size_t>(jag->T) * D * 4, 1024);
+  if (ws_bytes < (nin ? nin_part + ln_in_bwd_partial_floats(D) * 4 : lay.total)) return HSTU_ERR_WORKSPACE;
   if (!gr->dW1 || !gr->db1 || !gr->dW2 || !gr->db2 || !gr->dgamma || !gr->dbeta || !gr->drab_pos || !gr->drab_time)
     return HSTU_ERR_INVALID_ARG;
   const int64_t T = jag->T;
@@ -709,6 +849,8 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
                           (2ull * desc->pos_max_len - 1) * 4, 1ull * desc->n_time_buckets * 4};
     float* ps[8] = {gr->dW1, gr->db1, gr->dW2, gr->db2, gr->dgamma, gr->dbeta, gr->drab_pos, gr->drab_time};
     for (int i = 0; i < 8 && e == cudaSuccess; ++i) e = cudaMemsetAsync(ps[i], 0, zs[i], st);
+    if (nin && e == cudaSuccess) e = cudaMemsetAsync(nin->dgamma, 0, 4ull * D, st);
+    if (nin && e == cudaSuccess) e = cudaMemsetAsync(nin->dbeta, 0, 4ull * D, st);
     return cuda_status(e);
   }
   if (!x || !dy || !dx || !saved->uvqk || !saved->z || !saved->o || !saved->g || !saved->mu || !saved->rstd)
@@ -728,6 +870,7 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   const int x_dt = desc->x_dtype == HSTU_F32 ? kDtF32 : kDtBF16;
   const int y_dt = desc->y_dtype == HSTU_F32 ? kDtF32 : kDtBF16;
   const void* dy_op = dy_f16 ? dy_f16 : wsb + lay.dy_f16;
+  if (nin) x_f16 = nin->xn;   // f1 read Xn: dW1 = dZ^T Xn
   const void* x_op = x_f16 ? x_f16 : wsb + lay.x_f16;
   void* w1_f16 = wsb + lay.w1_f16;
   void* w2_f16 = wsb + lay.w2_f16;
@@ -776,6 +919,10 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
   s = run_attn_bwd(&ad, jag, uvqk + 2 * D * 2, uvqk + 3 * D * 2, uvqk + 1 * D * 2, dO, w->rab_pos, w->rab_time, dq, dk,
                    dv, D, gr->drab_pos, gr->drab_time, ws, st);
   if (s != HSTU_OK) return s;
+  if (g_ready_events[0]) {   // dW2, db2, dgamma, dbeta and the table gradients are final
+    e = cudaEventRecord(g_ready_events[0], st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
   // 4. SiLU backward into dZ[:, D:4D], db1 = sum_t dZ
   e = dz_assemble(T, D, kDtF16, dv, dq, dk, saved->z, 4ll * D, dz, 4ll * D, st);
   if (e == cudaSuccess) e = column_sum(dz, kDtF16, T, 4 * D, 4ll * D, part, gr->db1, st);
@@ -788,16 +935,90 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
     g3.epi.kind = kEpiAtomic; g3.epi.out0 = gr->dW1; g3.epi.out0_dt = kDtF32; g3.epi.ld_out0 = D; g3.status = status;
     e = gemm_bf16(g3, st);
   }
+  if (e == cudaSuccess && g_ready_events[1]) e = cudaEventRecord(g_ready_events[1], st);   // dW1, db1 final
   if (e == cudaSuccess) {
     GemmArgs g4{};
     g4.A = dz; g4.lda = 4ll * D; g4.a_mn = false; g4.B = w1_f16; g4.ldb = D; g4.b_mn = true; g4.f16 = true;
     g4.M = T; g4.N = D; g4.K = 4ll * D; g4.splits = 1;
-    g4.epi.kind = kEpiLinear; g4.epi.resid = dy; g4.epi.resid_dt = desc->y_dtype; g4.epi.ld_resid = D;
-    g4.epi.out0 = dx; g4.epi.out0_dt = desc->x_dtype; g4.epi.ld_out0 = D;
-    g4.epi.out1 = dx_f16; g4.epi.out1_dt = kDtF16; g4.epi.ld_out1 = D; g4.status = status;
+    g4.epi.kind = kEpiLinear;
+    if (nin) {   // dXn = dZ W1, then through the input LayerNorm
+      g4.epi.out0 = wsb + nin_dxn; g4.epi.out0_dt = kDtF32; g4.epi.ld_out0 = D;
+    } else {
+      g4.epi.resid = dy; g4.epi.resid_dt = desc->y_dtype; g4.epi.ld_resid = D;
+      g4.epi.out0 = dx; g4.epi.out0_dt = desc->x_dtype; g4.epi.ld_out0 = D;
+      g4.epi.out1 = dx_f16; g4.epi.out1_dt = kDtF16; g4.epi.ld_out1 = D;
+    }
+    g4.status = status;
     e = gemm_bf16(g4, st);
   }
+  if (nin && e == cudaSuccess)
+    e = ln_in_bwd(T, D, desc->x_dtype == HSTU_F32 ? kDtF32 : kDtBF16, desc->y_dtype == HSTU_F32 ? kDtF32 : kDtBF16,
+                  reinterpret_cast<const float*>(wsb + nin_dxn), x, dy, nin->gamma, nin->mu, nin->rstd, dx, dx_f16,
+                  reinterpret_cast<float*>(wsb + nin_part), nin->dgamma, nin->dbeta, st);
   return cuda_status(e);
+}
+
+}  // namespace
+}  // namespace hstu
+
+extern "C" {
+
+hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag, const hstu_layer_weights_t* w,
+                             const void* x, const void* x_f16, const hstu_layer_saved_t* saved, const void* dy,
+                             const void* dy_f16, void* dx, void* dx_f16, const hstu_layer_grads_t* grads, void* ws,
+                             size_t ws_bytes, hstu_stream_t stream) {
+  return run_layer_bwd(desc, jag, w, x, x_f16, saved, dy, dy_f16, dx, dx_f16, grads, ws, ws_bytes, stream, nullptr);
+}
+
+size_t hstu_layer_norm_in_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag) {
+  if (!desc || desc->D <= 0 || desc->H <= 0) return 0;
+  hstu_layer_desc_t d32 = *desc;   // the forward's fp16 W1 copy region
+  d32.x_dtype = HSTU_F32;
+  const size_t f = hstu_layer_workspace_size(&d32, jag);
+  const size_t b = hstu_layer_bwd_workspace_size(desc, jag);
+  if (f == 0 || b == 0) return 0;
+  const size_t nb = align_up(align_up(b, 1024) + static_cast<size_t>(jag->T) * desc->D * 4, 1024) +
+                    ln_in_bwd_partial_floats(desc->D) * 4;
+  return f > nb ? f : nb;
+}
+
+hstu_status_t hstu_layer_fwd_norm_in(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag,
+                                     const hstu_layer_weights_t* w, const hstu_norm_in_t* nin, const void* x, void* y,
+                                     void* y_f16, const hstu_layer_saved_t* saved, void* ws, size_t ws_bytes,
+                                     hstu_stream_t stream) {
+  if (!desc || !w || !saved || !nin) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t s = check_jagged(jag);
+  if (s != HSTU_OK) return s;
+  if (desc->dtype != HSTU_BF16) return HSTU_ERR_UNSUPPORTED;
+  if (desc->D != 256 && desc->D != 512) return HSTU_ERR_UNSUPPORTED;
+  if (desc->x_dtype != HSTU_F32 && desc->x_dtype != HSTU_BF16) return HSTU_ERR_UNSUPPORTED;
+  if (!ws) return HSTU_ERR_INVALID_ARG;
+  if (ws_bytes < hstu_layer_norm_in_workspace_size(desc, jag)) return HSTU_ERR_WORKSPACE;
+  if (jag->T == 0) return HSTU_OK;
+  if (!x || !nin->gamma || !nin->beta || !nin->xn || !nin->mu || !nin->rstd) return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(nin->gamma) || !aligned16(nin->beta) || !aligned16(nin->xn))
+    return HSTU_ERR_UNSUPPORTED;
+  // Xn = LayerNorm_in(X) in fp16: f1 reads it (with an fp16 copy of W1), the residual adds X itself
+  cudaError_t e = norm_gate_fwd(jag->T, desc->D, desc->x_dtype == HSTU_F32 ? kDtF32 : kDtBF16, kDtOne, kDtF16, x,
+                                desc->D, nullptr, 0, nin->gamma, nin->beta, desc->ln_eps, nin->xn, nin->mu, nin->rstd,
+                                stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  hstu_layer_desc_t d32 = *desc;
+  d32.x_dtype = HSTU_F32;
+  return run_layer_fwd(&d32, desc->x_dtype, jag, w, x, nin->xn, y, y_f16, saved, ws, ws_bytes, stream);
+}
+
+hstu_status_t hstu_layer_bwd_norm_in(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag,
+                                     const hstu_layer_weights_t* w, const hstu_norm_in_t* nin, const void* x,
+                                     const hstu_layer_saved_t* saved, const void* dy, void* dx, void* dx_f16,
+                                     const hstu_layer_grads_t* grads, void* ws, size_t ws_bytes,
+                                     hstu_stream_t stream) {
+  if (!nin || !desc) return HSTU_ERR_INVALID_ARG;
+  if (jag && jag->T > 0 && (!nin->gamma || !nin->xn || !nin->mu || !nin->rstd)) return HSTU_ERR_INVALID_ARG;
+  if (!nin->dgamma || !nin->dbeta) return HSTU_ERR_INVALID_ARG;
+  if (nin->xn && !aligned16(nin->xn)) return HSTU_ERR_UNSUPPORTED;
+  if (ws_bytes < hstu_layer_norm_in_workspace_size(desc, jag)) return HSTU_ERR_WORKSPACE;
+  return run_layer_bwd(desc, jag, w, x, nullptr, saved, dy, nullptr, dx, dx_f16, grads, ws, ws_bytes, stream, nin);
 }
 
 }  // extern "C"
@@ -1065,6 +1286,7 @@ extern "C" hstu_status_t hstu_falcon_fwd(const hstu_falcon_desc_t* desc, const h
       }
       if (s != HSTU_OK) return s;
       AttnArgs a{};
+      a.bias_heads = 1;
       a.B = users; a.T = Tp; a.max_len = prefix->max_len; a.offsets = prefix->offsets; a.ts = prefix->timestamps;
       a.H = desc->H; a.dqk = 64; a.dv = 64; a.inv_N = desc->inv_N; a.pos_max_len = desc->pos_max_len;
       a.n_buckets = desc->n_time_buckets;
@@ -1094,6 +1316,143 @@ extern "C" hstu_status_t hstu_falcon_fwd(const hstu_falcon_desc_t* desc, const h
                                         static_cast<size_t>(rows) * D * 4, users, cudaMemcpyDeviceToDevice, st);
       if (e != cudaSuccess) return cuda_status(e);
     }
+  }
+  return HSTU_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// M-FALCON prefix append ("HSTU: The First Exploration of the Scaling Law", 7.1.5 M-FALCON: the
+// history's K, V cache is reused across requests)
+// ---------------------------------------------------------------------------------------------
+namespace hstu {
+namespace {
+
+// Workspace: the attention workspace of the combined prefixes first (its status word is the call's),
+// then the combined query buffer and attention output, and the appended rows' U|V|Q|K, O, G, mu,
+// rstd, fp32 stream (two buffers) and its fp16 copy, and fp16 copies of W1, W2.
+struct AppendWs {
+  size_t qbuf, o_comb, a_uvqk, a_o, a_g, a_mu, a_rstd, a_x0, a_x1, a_x16, w1_f16, w2_f16, total;
+};
+
+AppendWs append_layout(const hstu_falcon_desc_t* d, const hstu_jagged_t* pnew, int64_t A) {
+  AppendWs w{};
+  const size_t Tn = static_cast<size_t>(pnew->T), D = static_cast<size_t>(d->D), a = static_cast<size_t>(A);
+  size_t off = align_up(attn_ws_bytes(pnew), 1024);
+  auto take = [&](size_t bytes) { const size_t o = off; off = align_up(off + bytes, 1024); return o; };
+  w.qbuf = take(Tn * D * 2);
+  w.o_comb = take(Tn * D * 4);
+  w.a_uvqk = take(a * 4 * D * 2);
+  w.a_o = take(a * D * 4);
+  w.a_g = take(a * D * 2);
+  w.a_mu = take(a * 4);
+  w.a_rstd = take(a * 4);
+  w.a_x0 = take(a * D * 4);
+  w.a_x1 = take(a * D * 4);
+  w.a_x16 = take(a * D * 2);
+  w.w1_f16 = take(4 * D * D * 2);
+  w.w2_f16 = take(D * D * 2);
+  w.total = off;
+  return w;
+}
+
+hstu_status_t check_append(const hstu_falcon_desc_t* d, const hstu_jagged_t* pold, const hstu_jagged_t* app,
+                           const hstu_jagged_t* pnew) {
+  hstu_status_t s = check_falcon(d, pnew);
+  if (s != HSTU_OK) return s;
+  if (check_jagged(pold) != HSTU_OK || !app || app->B < 0 || app->T < 0 || !app->offsets) return HSTU_ERR_INVALID_ARG;
+  if (pold->B != d->users || app->B != d->users || pold->T + app->T != pnew->T) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+}  // namespace
+}  // namespace hstu
+
+extern "C" size_t hstu_falcon_append_workspace_size(const hstu_falcon_desc_t* desc, const hstu_jagged_t* prefix_old,
+                                                    const hstu_jagged_t* appended, const hstu_jagged_t* prefix_new) {
+  if (check_append(desc, prefix_old, appended, prefix_new) != HSTU_OK) return 0;
+  return append_layout(desc, prefix_new, appended->T).total;
+}
+
+extern "C" hstu_status_t hstu_falcon_append(const hstu_falcon_desc_t* desc, const hstu_layer_weights_t* layers,
+                                            const hstu_jagged_t* prefix_old, const void* kv_cache_old,
+                                            const hstu_jagged_t* appended, const void* app_x,
+                                            const hstu_jagged_t* prefix_new, void* kv_cache_new, void* app_out,
+                                            void* ws, size_t ws_bytes, hstu_stream_t stream) {
+  hstu_status_t s = check_append(desc, prefix_old, appended, prefix_new);
+  if (s != HSTU_OK) return s;
+  if (!layers || !ws) return HSTU_ERR_INVALID_ARG;
+  const int64_t A = appended->T, Tn = prefix_new->T, To = prefix_old->T;
+  const AppendWs lay = append_layout(desc, prefix_new, A);
+  if (ws_bytes < lay.total) return HSTU_ERR_WORKSPACE;
+  if (Tn == 0) return HSTU_OK;
+  if (!kv_cache_new || (To > 0 && !kv_cache_old) || (A > 0 && !app_x)) return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(kv_cache_new) || (kv_cache_old && !aligned16(kv_cache_old)) || (app_x && !aligned16(app_x)) ||
+      (app_out && !aligned16(app_out)))
+    return HSTU_ERR_UNSUPPORTED;
+  const int32_t D = desc->D, L = desc->L, users = desc->users;
+  for (int l = 0; l < L; ++l) {
+    const hstu_layer_weights_t& w = layers[l];
+    if (!w.W1 || !w.b1 || !w.W2 || !w.b2 || !w.gamma || !w.beta || !w.rab_pos || !w.rab_time)
+      return HSTU_ERR_INVALID_ARG;
+    if (!aligned16(w.W1) || !aligned16(w.W2) || !aligned16(w.b1) || !aligned16(w.b2) || !aligned16(w.gamma) ||
+        !aligned16(w.beta))
+      return HSTU_ERR_UNSUPPORTED;
+  }
+  cudaStream_t st = stream;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  int* status = ws_status(ws);
+  const size_t old_layer = static_cast<size_t>(To) * 2 * D, new_layer = static_cast<size_t>(Tn) * 2 * D;
+  const uint16_t* cache_old = static_cast<const uint16_t*>(kv_cache_old);
+  uint16_t* cache_new = static_cast<uint16_t*>(kv_cache_new);
+  uint16_t* a_uvqk = reinterpret_cast<uint16_t*>(base + lay.a_uvqk);
+  void* a_x[2] = {base + lay.a_x0, base + lay.a_x1};
+  void* a_x16 = base + lay.a_x16;
+  hstu_attn_desc_t ad{};
+  ad.H = desc->H; ad.d_qk = 64; ad.d_v = 64; ad.inv_N = desc->inv_N; ad.pos_max_len = desc->pos_max_len;
+  ad.n_time_buckets = desc->n_time_buckets; ad.dtype = HSTU_F16; ad.o_dtype = HSTU_F32;
+  ad.ld_q = D; ad.ld_k = 2ll * D; ad.ld_v = 2ll * D; ad.ld_o = D;
+  const void* xin = app_x;
+  for (int l = 0; l < L; ++l) {
+    const hstu_layer_weights_t& w = layers[l];
+    const bool last = l == L - 1;
+    // 1. U|V|Q|K of the appended rows (layer 0 reads the bf16 input, later layers the fp16 copy of
+    //    the fp32 stream)
+    if (A > 0) {
+      if (l == 0) {
+        s = run_uvqk(A, D, HSTU_BF16, HSTU_F16, xin, D, w.W1, w.b1, a_uvqk, nullptr, status, st);
+      } else {
+        cudaError_t e = convert_dtype(w.W1, kDtBF16, base + lay.w1_f16, kDtF16, 4ll * D * D, st);
+        if (e != cudaSuccess) return cuda_status(e);
+        s = run_uvqk(A, D, HSTU_BF16, HSTU_F16, a_x16, D, base + lay.w1_f16, w.b1, a_uvqk, nullptr, status, st, true);
+      }
+      if (s != HSTU_OK) return s;
+    }
+    // 2. this layer's combined cache and the combined query buffer
+    uint16_t* cl = cache_new + l * new_layer;
+    cudaError_t e = falcon_append_scatter(prefix_old->offsets, appended->offsets, prefix_new->offsets, users, Tn, D,
+                                          cache_old ? cache_old + l * old_layer : nullptr, a_uvqk, cl,
+                                          reinterpret_cast<uint16_t*>(base + lay.qbuf), status, st);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (A == 0) continue;
+    // 3. causal attention of the appended rows over the combined prefix (rows of the old prefix are
+    //    neither computed nor written)
+    s = run_attn_fwd(&ad, prefix_new, base + lay.qbuf, cl, cl + D, w.rab_pos, w.rab_time, base + lay.o_comb, ws, st,
+                     true, nullptr, prefix_old->offsets);
+    if (s != HSTU_OK) return s;
+    e = falcon_append_gather(prefix_old->offsets, appended->offsets, prefix_new->offsets, users, A, D,
+                             reinterpret_cast<const float*>(base + lay.o_comb), reinterpret_cast<float*>(base + lay.a_o),
+                             st);
+    // 4. LayerNorm (.) U, f2 + residual
+    if (e == cudaSuccess)
+      e = norm_gate_fwd(A, D, kDtF32, kDtF16, kDtF16, base + lay.a_o, D, a_uvqk, 4ll * D, w.gamma, w.beta,
+                        desc->ln_eps, base + lay.a_g, reinterpret_cast<float*>(base + lay.a_mu),
+                        reinterpret_cast<float*>(base + lay.a_rstd), st);
+    if (e != cudaSuccess) return cuda_status(e);
+    void* y = (last && app_out) ? app_out : a_x[l & 1];
+    s = run_out_proj(A, D, HSTU_BF16, HSTU_F16, base + lay.a_g, w.W2, w.b2, xin, l == 0 ? HSTU_BF16 : HSTU_F32, y,
+                     HSTU_F32, last ? nullptr : a_x16, status, st, base + lay.w2_f16);
+    if (s != HSTU_OK) return s;
+    xin = y;
   }
   return HSTU_OK;
 }

@@ -32,6 +32,14 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 // ---------------------------------------------------------------------------------------------
+// Timing hook (hstu_profile_events): caller-owned CUDA events recorded on the launching stream right
+// before and right after the dominant kernel of a call; under stream capture they become external
+// event-record nodes, so graph replays time the kernel too. Per host thread; no-op when unset.
+// ---------------------------------------------------------------------------------------------
+enum : int { kProfAttnFwd = 0, kProfAttnBwd = 1, kProfNormFwd = 2, kProfNormBwd = 3, kProfKernels = 4 };
+cudaError_t prof_record(int kernel, bool stop, cudaStream_t st);
+
+// ---------------------------------------------------------------------------------------------
 // workspace layout: [0, 256) status word + padding, then per-call regions
 // ---------------------------------------------------------------------------------------------
 constexpr size_t kWsHeader = 256;
@@ -97,10 +105,14 @@ cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
 // Builds the (sequence, query tile) work list; with pair_base (device, [B+1]) also the index of
 // each sequence's first causal (query tile, key tile) pair and, in pair_base[B], their total.
 // With kitems, also the attention backward's (sequence, key tile) list in the same cost order: the
-// key tile that visits t + 1 query tiles sits where the forward list has query tile t.
+// key tile that visits t + 1 query tiles sits where the forward list has query tile t. With sched,
+// sched[0] (the persistent attention kernel's unit counter) is reset to 0. With pack (int32 [B]),
+// runs of short sequences share a tile: pack[b] = k >= 2 marks the first of k packed sequences
+// (one item (b, -k) in both lists), 0 the other members, 1 a sequence on its own.
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
                             int32_t* count, int* status, cudaStream_t st, long long* pair_base = nullptr,
-                            int32_t* kitems = nullptr, int32_t* kcount = nullptr);
+                            int32_t* kitems = nullptr, int32_t* kcount = nullptr, int32_t* sched = nullptr,
+                            int32_t* pack = nullptr);
 // The n_b x n_b time-bucket matrices of the test surface, tile by tile with the bias tiles' code.
 cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int max_len,
                                 int n_buckets, const int64_t* sq_offsets, uint8_t* out, cudaStream_t st);
@@ -142,6 +154,20 @@ struct AttnArgs {
   const uint16_t* kbias;        // fp16 half-bias per prefix key: [B, kbias_ld], user u at u * kbias_ld
   int64_t kbias_ld;             // multiple of 128 >= every prefix length
   const float* self_bias;       // device: rab_pos[idx(0)] + rab_time[bucket(0)]
+  int32_t* unit_counter;        // persistent forward: next (work item, head) unit, reset by the work list
+  // the richer bias (hstu_rab_ext_t): bias_heads tiles per causal pair (1: tables shared by the heads,
+  // H: one slice per head, rab_pos / rab_time / rab_type indexed by head first); n_types > 0 adds
+  // rab_type[type_i][type_j]
+  int bias_heads;
+  int n_types;
+  const int32_t* token_type;
+  const float* rab_type;
+  // prefix append: only query rows at or past q_from[b + 1] - q_from[b] of sequence b (the old
+  // prefix length, from the old prefix offsets) are computed and written; null = every row
+  const int64_t* q_from;
+  // packed short sequences (launch_worklist's pack array) or null: an item (b, -k) is one tile over
+  // the rows of sequences b .. b + k - 1, keys masked to the query row's own sequence
+  const int32_t* pack;
 };
 
 struct AttnBwdArgs {
@@ -150,7 +176,8 @@ struct AttnBwdArgs {
   float* dq; float* dk; float* dv;   // fp32 [T, H*64], dq accumulated (must be zero on entry)
   int64_t ld_g;                      // row stride of dq, dk, dv
   float* drab_pos; float* drab_time; // accumulated (must be zero on entry)
-  void* bias_t;                // fp16 [max_pairs, 128 keys, 128 queries] half-bias, transposed
+  float* drab_type;                  // [bias_heads, n_types, n_types], accumulated; null without types
+  void* bias_t;                // fp16 [max_pairs, bias_heads, 128 keys, 128 queries] half-bias, transposed
   void* bucket_t;              // u8   [max_pairs, 128 keys, 128 queries] time bucket, transposed
   void* dxt;                   // fp16 [max_pairs, H, 128 keys, 128 queries] dX^T of every (pair, head)
   const int32_t* kitems;       // backward work list (b, key tile)
@@ -172,6 +199,13 @@ cudaError_t falcon_key_bias(const int64_t* offsets, const int64_t* ts, int users
                             int pos_max_len, int n_buckets, uint16_t* kbias, int64_t kbias_ld, float* self_bias,
                             int* status, cudaStream_t st);
 cudaError_t attn_falcon_tc(const AttnArgs& a, cudaStream_t st);
+// M-FALCON prefix append (falcon_append.cu): one layer of the combined K|V cache and the combined
+// query buffer; the appended rows' attention output back in their own order.
+cudaError_t falcon_append_scatter(const int64_t* old_off, const int64_t* app_off, const int64_t* new_off, int users,
+                                  int64_t T_new, int D, const uint16_t* old_cache, const uint16_t* uvqk,
+                                  uint16_t* new_cache, uint16_t* qbuf, int* status, cudaStream_t st);
+cudaError_t falcon_append_gather(const int64_t* old_off, const int64_t* app_off, const int64_t* new_off, int users,
+                                 int64_t A, int D, const float* o_comb, float* o_app, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------------
 // LayerNorm (.) U
@@ -209,6 +243,14 @@ cudaError_t column_sum(const void* in, int dt, int64_t rows, int cols, int64_t l
                        cudaStream_t st);
 
 cudaError_t launch_timeout_probe(int* status, cudaStream_t st);
+
+// Backward of the input LayerNorm of the norm_in layer variant (norm_in.cu): dx = dy + LN_in^T(dxn)
+// in x's dtype (and an fp16 copy when dx_f16), dgamma / dbeta through `partial`
+// (ln_in_bwd_partial_floats(D) floats). x and dy: fp32 / fp32 or bf16 / bf16; D in {256, 512}.
+size_t ln_in_bwd_partial_floats(int D);
+cudaError_t ln_in_bwd(int64_t T, int D, int x_dt, int y_dt, const float* dxn, const void* x, const void* dy,
+                      const float* gamma, const float* mu, const float* rstd, void* dx, void* dx_f16, float* partial,
+                      float* dgamma, float* dbeta, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------------
 // Stochastic Length (stochastic_length.cu)

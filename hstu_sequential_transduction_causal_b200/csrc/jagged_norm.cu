@@ -15,17 +15,49 @@ namespace hstu {
 
 namespace {
 
+// Short sequences share a tile: a run of consecutive sequences of at most kPackMaxLen tokens each
+// (empty ones included) whose rows add up to at most 128 becomes one 128-row tile, so a batch of
+// short histories does not leave most of every tile empty. Greedy in batch order inside chunks of 32
+// sequences (chunks are packed independently, so a block packs them in parallel). pack[b]: k >= 2
+// for the first sequence of a pack of k, 0 for the other members, 1 for a sequence on its own.
+constexpr int kPackMaxLen = 64;
+
+__device__ void pack_chunk(const int64_t* __restrict__ off, int b0, int b1, int32_t* pack) {
+  int i = b0;
+  while (i < b1) {
+    const long long n = off[i + 1] - off[i];
+    if (n <= 0 || n > kPackMaxLen) {
+      pack[i++] = 1;
+      continue;
+    }
+    long long total = n;
+    int k = 1;
+    while (i + k < b1) {
+      const long long m = off[i + k + 1] - off[i + k];
+      if (m > kPackMaxLen || total + m > kQTile) break;
+      total += m;
+      ++k;
+    }
+    pack[i] = k;
+    for (int j = 1; j < k; ++j) pack[i + j] = 0;
+    i += k;
+  }
+}
+
 // ----------------------------------------------------------------------------------------------
 // Jagged tile work list ("4.4 Scaling Recommendation Models", Efficiency tricks: kernels over
 // variable-length sequences). One block: emits (b, t) for every query tile t of every sequence,
-// tiles with more causal key tiles first, ties by increasing b. Also validates the offsets:
+// tiles with more causal key tiles first, ties by increasing b; with `pack`, a pack of k >= 2 short
+// sequences is one item (b, -k) among the one-tile items. Also validates the offsets:
 // offsets[0] == 0, non-decreasing, every length <= max_len, offsets[B] == T; a violation records
 // kDevBadInput and empties the list so no later kernel reads out of bounds.
 // ----------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024)
 worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items,
-                int32_t* count, int* status, long long* pair_base, int32_t* kitems, int32_t* kcount) {
+                int32_t* count, int* status, long long* pair_base, int32_t* kitems, int32_t* kcount,
+                int32_t* sched, int32_t* pack) {
   pdl_enter();
+  if (sched && threadIdx.x == 0) sched[0] = 0;   // the persistent attention's unit counter
   __shared__ int s_warp[32];
   __shared__ int s_max_tiles;
   __shared__ int s_bad;
@@ -57,9 +89,14 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
   __shared__ int s_nt[kStageSeqs];
   __shared__ int s_start[kStageTiles];
   if (B <= kStageSeqs && max_tiles <= kStageTiles) {
-    // Fast path. Tile counts staged in shared memory; warp w owns the tile indices t = w, w+32, ...
+    // Fast path. Tile counts staged in shared memory (0 for a pack member, whose rows the pack's
+    // first sequence covers); warp w owns the tile indices t = w, w+32, ...
+    if (pack) {
+      for (int c = tid; c * 32 < B; c += blockDim.x) pack_chunk(off, 32 * c, min(B, 32 * c + 32), pack);
+      __syncthreads();
+    }
     for (int b = tid; b < B; b += blockDim.x)
-      s_nt[b] = static_cast<int>((off[b + 1] - off[b] + kQTile - 1) / kQTile);
+      s_nt[b] = (pack && pack[b] == 0) ? 0 : static_cast<int>((off[b + 1] - off[b] + kQTile - 1) / kQTile);
     __syncthreads();
     for (int t = warp; t < max_tiles; t += 32) {
       int c = 0;
@@ -88,11 +125,12 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
         const unsigned m = __ballot_sync(0xffffffffu, flag);
         if (flag) {
           const int p = pos + __popc(m & ((1u << lane) - 1u));
+          const int pk = pack ? pack[b] : 1;
           items[2 * p] = b;
-          items[2 * p + 1] = t;
+          items[2 * p + 1] = pk >= 2 ? -pk : t;
           if (kitems) {   // the key tile that visits t + 1 query tiles: the same cost order
             kitems[2 * p] = b;
-            kitems[2 * p + 1] = s_nt[b] - 1 - t;
+            kitems[2 * p + 1] = pk >= 2 ? -pk : s_nt[b] - 1 - t;
           }
         }
         pos += __popc(m);
@@ -100,6 +138,9 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
     }
     __syncthreads();
   } else for (int t = max_tiles - 1; t >= 0; --t) {
+    // (large batches: no packing)
+    if (pack && t == max_tiles - 1)
+      for (int b = tid; b < B; b += blockDim.x) pack[b] = 1;
     for (int c0 = 0; c0 < B; c0 += blockDim.x) {
       const int b = c0 + tid;
       bool flag = false;
@@ -182,8 +223,10 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
 // lane b owns sequence b; the items are written tile index by tile index, longest first, as above.
 __global__ void __launch_bounds__(32)
 worklist_warp_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items, int32_t* count,
-                     int* status, long long* pair_base, int32_t* kitems, int32_t* kcount) {
+                     int* status, long long* pair_base, int32_t* kitems, int32_t* kcount, int32_t* sched,
+                     int32_t* pack) {
   pdl_enter();
+  if (sched && threadIdx.x == 0) sched[0] = 0;   // the persistent attention's unit counter
   const int lane = threadIdx.x;
   const bool mine = lane < B;
   long long n = 0;
@@ -199,7 +242,14 @@ worklist_warp_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_
     }
     return;
   }
-  const int nt = mine ? static_cast<int>((n + kQTile - 1) / kQTile) : 0;
+  const int nt_all = mine ? static_cast<int>((n + kQTile - 1) / kQTile) : 0;
+  int pk = 1;
+  if (pack) {
+    if (lane == 0) pack_chunk(off, 0, B, pack);
+    __syncwarp();
+    if (mine) pk = pack[lane];
+  }
+  const int nt = pk == 0 ? 0 : nt_all;   // a pack member's rows are in its pack's tile
   int max_tiles = nt;
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) max_tiles = max(max_tiles, __shfl_xor_sync(0xffffffffu, max_tiles, d));
@@ -210,10 +260,10 @@ worklist_warp_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_
     if (flag) {
       const int pos = base + __popc(m & ((1u << lane) - 1u));
       items[2 * pos] = lane;
-      items[2 * pos + 1] = t;
+      items[2 * pos + 1] = pk >= 2 ? -pk : t;
       if (kitems) {
         kitems[2 * pos] = lane;
-        kitems[2 * pos + 1] = nt - 1 - t;
+        kitems[2 * pos + 1] = pk >= 2 ? -pk : nt - 1 - t;
       }
     }
     base += __popc(m);
@@ -223,7 +273,7 @@ worklist_warp_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_
     if (kcount) *kcount = base;
   }
   if (!pair_base) return;
-  const long long v = static_cast<long long>(nt) * (nt + 1) / 2;
+  const long long v = static_cast<long long>(nt_all) * (nt_all + 1) / 2;
   long long inc = v;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -356,20 +406,24 @@ template <int VPT, int OT, int UT, int GT>
 cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int64_t ld_u, const float* gamma,
                       const float* beta, float eps, void* g, float* mu, float* rstd, cudaStream_t st) {
   const int64_t blocks = (T + 7) / 8;
-  return launch_pdl(norm_gate_kernel<VPT, OT, UT, GT>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, T, o,
-                    ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd);
+  cudaError_t e = prof_record(kProfNormFwd, false, st);
+  if (e == cudaSuccess)
+    e = launch_pdl(norm_gate_kernel<VPT, OT, UT, GT>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, T, o,
+                   ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd);
+  if (e == cudaSuccess) e = prof_record(kProfNormFwd, true, st);
+  return e;
 }
 
 }  // namespace
 
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
                             int32_t* count, int* status, cudaStream_t st, long long* pair_base, int32_t* kitems,
-                            int32_t* kcount) {
+                            int32_t* kcount, int32_t* sched, int32_t* pack) {
   if (B >= 0 && B <= 32)
     return launch_pdl(worklist_warp_kernel, dim3(1), dim3(32), 0, st, offsets, B, T, max_len, items, count, status,
-                      pair_base, kitems, kcount);
+                      pair_base, kitems, kcount, sched, pack);
   return launch_pdl(worklist_kernel, dim3(1), dim3(1024), 0, st, offsets, B, T, max_len, items, count, status,
-                    pair_base, kitems, kcount);
+                    pair_base, kitems, kcount, sched, pack);
 }
 
 cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int max_len,
@@ -389,7 +443,8 @@ cudaError_t norm_gate_fwd(int64_t T, int D, int o_dt, int u_dt, int g_dt, const 
                           float* rstd, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   // supported (o, u, g) combinations: exact fp32; fp32 O with fp16 U and fp16 G (tensor-core
-  // layer); fp32 O with fp16 or bf16 U and bf16 G; all bf16.
+  // layer); fp32 O with fp16 or bf16 U and bf16 G; all bf16; fp32 or bf16 O without a gate and fp16
+  // G (the input LayerNorm of the norm_in layer variant).
 #define HSTU_NG(VPT)                                                                                     \
   if (o_dt == kDtF32 && u_dt == kDtF32 && g_dt == kDtF32)                                               \
     return launch_ng<VPT, kDtF32, kDtF32, kDtF32>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
@@ -401,6 +456,10 @@ cudaError_t norm_gate_fwd(int64_t T, int D, int o_dt, int u_dt, int g_dt, const 
     return launch_ng<VPT, kDtF32, kDtBF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
   if (o_dt == kDtBF16 && u_dt == kDtBF16 && g_dt == kDtBF16)                                            \
     return launch_ng<VPT, kDtBF16, kDtBF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+  if (o_dt == kDtF32 && u_dt == kDtOne && g_dt == kDtF16)                                               \
+    return launch_ng<VPT, kDtF32, kDtOne, kDtF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st);  \
+  if (o_dt == kDtBF16 && u_dt == kDtOne && g_dt == kDtF16)                                              \
+    return launch_ng<VPT, kDtBF16, kDtOne, kDtF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
   return cudaErrorInvalidValue
   switch (D) {
     case 64: HSTU_NG(2);

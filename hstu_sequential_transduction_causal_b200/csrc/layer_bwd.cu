@@ -219,7 +219,8 @@ cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const f
                           float* dgamma_dbeta_out, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   const int G = norm_gate_bwd_blocks(T);
-  cudaError_t e = cudaSuccess;
+  cudaError_t e = prof_record(kProfNormBwd, false, st);
+  if (e != cudaSuccess) return e;
 #define HSTU_NGB(VPT)                                                                                            \
   if (act_dt == kDtF16)                                                                                          \
     e = launch_pdl(norm_gate_bwd_kernel<VPT, kDtF16>, dim3(G), dim3(256), 0, st, T, dg, o, u, zu, ld_act, gamma,   \
@@ -235,6 +236,7 @@ cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const f
     default: return cudaErrorInvalidValue;
   }
 #undef HSTU_NGB
+  if (e == cudaSuccess) e = prof_record(kProfNormBwd, true, st);
   if (e != cudaSuccess) return e;
   return launch_pdl(colsum_final_kernel, dim3((2 * D + 31) / 32), dim3(256), 0, st, static_cast<const float*>(partial), G,
                     2 * D, dgamma_dbeta_out);

@@ -348,8 +348,9 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
 // small numeric helpers
 // ------------------------------------------------------------------------------------------------
 
-// element types of activations and operands (same codes as hstu_dtype_t)
-enum : int { kDtF32 = 0, kDtBF16 = 1, kDtF16 = 2 };
+// element types of activations and operands (same codes as hstu_dtype_t); kDtOne: no array, every
+// element reads as 1 (the LayerNorm kernel without its gate)
+enum : int { kDtF32 = 0, kDtBF16 = 1, kDtF16 = 2, kDtOne = 3 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

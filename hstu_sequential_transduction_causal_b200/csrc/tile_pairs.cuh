@@ -28,4 +28,19 @@ __device__ __forceinline__ bool decode_tile_pair(long long p, const long long* _
   return true;
 }
 
+// Rows covered by the tiles of causal pair (b, qt, kt): sequence b (from row seq0, n rows), or,
+// for the only pair of the first sequence of a pack of k >= 2 short sequences (pack[b] = k), the
+// pack's rows. False for the pair of a pack member, which no tile uses.
+__device__ __forceinline__ bool pair_rows(const int64_t* __restrict__ offsets, const int32_t* __restrict__ pack,
+                                          int b, long long* seq0, int* n) {
+  *seq0 = offsets[b];
+  int k = 1;
+  if (pack) {
+    k = pack[b];
+    if (k == 0) return false;
+  }
+  *n = static_cast<int>(offsets[b + k] - *seq0);
+  return true;
+}
+
 }  // namespace hstu

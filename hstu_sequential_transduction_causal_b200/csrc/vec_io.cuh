@@ -12,7 +12,10 @@ namespace hstu {
 
 template <int VPT, int DT>
 __device__ __forceinline__ void load_vec(const void* base, int64_t idx, float* v) {
-  if constexpr (VPT == 1) {
+  if constexpr (DT == kDtOne) {
+#pragma unroll
+    for (int e = 0; e < VPT; ++e) v[e] = 1.0f;
+  } else if constexpr (VPT == 1) {
     if constexpr (DT == kDtF32) v[0] = reinterpret_cast<const float*>(base)[idx];
     else if constexpr (DT == kDtBF16) v[0] = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[idx]);
     else v[0] = __half2float(reinterpret_cast<const __half*>(base)[idx]);

@@ -64,6 +64,15 @@ class hstu_falcon_desc_t(ctypes.Structure):
                 ("inv_N", c_f32), ("pos_max_len", c_i32), ("n_time_buckets", c_i32), ("ln_eps", c_f32)]
 
 
+class hstu_rab_ext_t(ctypes.Structure):
+    _fields_ = [("per_head", c_i32), ("n_types", c_i32), ("token_type", c_vp), ("rab_type", c_vp)]
+
+
+class hstu_norm_in_t(ctypes.Structure):
+    _fields_ = [("gamma", c_vp), ("beta", c_vp), ("xn", c_vp), ("mu", c_vp), ("rstd", c_vp), ("dgamma", c_vp),
+                ("dbeta", c_vp)]
+
+
 P = ctypes.POINTER
 # name -> (restype, argtypes); the list every test checks against include/hstu.h
 SIGNATURES = {
@@ -73,6 +82,10 @@ SIGNATURES = {
     "hstu_sync_status": (c_i32, [c_vp, c_vp, P(c_i32)]),
     "hstu_set_wait_limit": (None, [ctypes.c_uint64]),
     "hstu_debug_timeout_probe": (c_i32, [c_vp, c_sz, c_vp]),
+    "hstu_profile_events": (c_i32, [c_i32, c_vp, c_vp]),
+    "hstu_dp_sequence_cost": (ctypes.c_double, [c_i64, c_i32]),
+    "hstu_dp_partition": (c_i32, [c_vp, c_i32, c_i32, c_i32, c_vp, c_vp]),
+    "hstu_layer_bwd_ready_events": (c_i32, [c_vp, c_vp]),
     "hstu_worklist_capacity": (c_i64, [P(hstu_jagged_t)]),
     "hstu_jagged_worklist": (c_i32, [P(hstu_jagged_t), c_vp, c_vp, c_vp]),
     "hstu_time_buckets": (c_i32, [P(hstu_jagged_t), c_i32, c_vp, c_vp, c_vp]),
@@ -89,6 +102,12 @@ SIGNATURES = {
     "hstu_layer_bwd": (c_i32, [P(hstu_layer_desc_t), P(hstu_jagged_t), P(hstu_layer_weights_t), c_vp, c_vp,
                                P(hstu_layer_saved_t), c_vp, c_vp, c_vp, c_vp, P(hstu_layer_grads_t), c_vp, c_sz,
                                c_vp]),
+    "hstu_attn_ext_workspace_size": (c_sz, [P(hstu_attn_desc_t), P(hstu_jagged_t), P(hstu_rab_ext_t)]),
+    "hstu_attn_fwd_ext": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), P(hstu_rab_ext_t), c_vp, c_vp, c_vp, c_vp,
+                                  c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "hstu_attn_bwd_ext_workspace_size": (c_sz, [P(hstu_attn_desc_t), P(hstu_jagged_t), P(hstu_rab_ext_t)]),
+    "hstu_attn_bwd_ext": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), P(hstu_rab_ext_t), c_vp, c_vp, c_vp, c_vp,
+                                  c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "hstu_attn_fwd_noalloc": (c_i32, [P(hstu_attn_desc_t), P(hstu_jagged_t), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                       c_vp]),
     "hstu_attn_fwd_noalloc_status": (c_i32, [c_vp, P(c_i32)]),
@@ -105,6 +124,16 @@ SIGNATURES = {
                                               c_vp, c_sz, c_vp]),
     "hstu_falcon_cache_size": (c_sz, [P(hstu_falcon_desc_t), P(hstu_jagged_t)]),
     "hstu_falcon_workspace_size": (c_sz, [P(hstu_falcon_desc_t), P(hstu_jagged_t)]),
+    "hstu_layer_norm_in_workspace_size": (c_sz, [P(hstu_layer_desc_t), P(hstu_jagged_t)]),
+    "hstu_layer_fwd_norm_in": (c_i32, [P(hstu_layer_desc_t), P(hstu_jagged_t), P(hstu_layer_weights_t),
+                                       P(hstu_norm_in_t), c_vp, c_vp, c_vp, P(hstu_layer_saved_t), c_vp, c_sz, c_vp]),
+    "hstu_layer_bwd_norm_in": (c_i32, [P(hstu_layer_desc_t), P(hstu_jagged_t), P(hstu_layer_weights_t),
+                                       P(hstu_norm_in_t), c_vp, P(hstu_layer_saved_t), c_vp, c_vp, c_vp,
+                                       P(hstu_layer_grads_t), c_vp, c_sz, c_vp]),
+    "hstu_falcon_append_workspace_size": (c_sz, [P(hstu_falcon_desc_t), P(hstu_jagged_t), P(hstu_jagged_t),
+                                                  P(hstu_jagged_t)]),
+    "hstu_falcon_append": (c_i32, [P(hstu_falcon_desc_t), P(hstu_layer_weights_t), P(hstu_jagged_t), c_vp,
+                                   P(hstu_jagged_t), c_vp, P(hstu_jagged_t), c_vp, c_vp, c_vp, c_sz, c_vp]),
     "hstu_falcon_fwd": (c_i32, [P(hstu_falcon_desc_t), P(hstu_layer_weights_t), P(hstu_jagged_t), c_vp, c_vp, c_i32,
                                 c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
 }
@@ -207,6 +236,46 @@ def hstu_set_wait_limit(cycles: int) -> None:
     lib().hstu_set_wait_limit(int(cycles))
 
 
+PROFILE_ATTN_FWD, PROFILE_ATTN_BWD, PROFILE_NORM_FWD, PROFILE_NORM_BWD = 0, 1, 2, 3
+
+
+def hstu_profile_events(kernel: int, start=None, stop=None) -> None:
+    """Records the two torch.cuda.Event objects (timing enabled) around the given kernel of later
+    calls on this host thread; no events disables. The events are recorded once first so that
+    their CUDA handles exist."""
+    if start is None or stop is None:
+        _check("hstu_profile_events", lib().hstu_profile_events(kernel, None, None))
+        return
+    for ev in (start, stop):
+        ev.record()
+    _check("hstu_profile_events", lib().hstu_profile_events(kernel, ctypes.c_void_p(start.cuda_event),
+                                                            ctypes.c_void_p(stop.cuda_event)))
+
+
+def hstu_dp_partition(lengths, D: int, world: int):
+    """(rank of each sequence int32 [B], cost of each rank float64 [world]) of the library's
+    cost-balanced split of one global batch (host arrays; no GPU needed)."""
+    import numpy as np
+    lens = np.ascontiguousarray(lengths, dtype=np.int64)
+    rank_of = np.zeros(lens.shape[0], dtype=np.int32)
+    cost = np.zeros(world, dtype=np.float64)
+    _check("hstu_dp_partition", lib().hstu_dp_partition(lens.ctypes.data, lens.shape[0], D, world,
+                                                        rank_of.ctypes.data, cost.ctypes.data))
+    return rank_of, cost
+
+
+def hstu_layer_bwd_ready_events(early=None, w1=None) -> None:
+    """torch.cuda.Event objects recorded by later hstu_layer_bwd calls on this thread when their
+    early gradients (dW2, db2, dgamma, dbeta, tables) and then dW1, db1 are final; none disables."""
+    if early is None or w1 is None:
+        _check("hstu_layer_bwd_ready_events", lib().hstu_layer_bwd_ready_events(None, None))
+        return
+    for ev in (early, w1):
+        ev.record()
+    _check("hstu_layer_bwd_ready_events", lib().hstu_layer_bwd_ready_events(ctypes.c_void_p(early.cuda_event),
+                                                                            ctypes.c_void_p(w1.cuda_event)))
+
+
 def hstu_debug_timeout_probe(ws: torch.Tensor, stream=None) -> None:
     _check("hstu_debug_timeout_probe", lib().hstu_debug_timeout_probe(_ptr(ws), ws.numel() * ws.element_size(),
                                                                       _stream(stream)))
@@ -254,6 +323,35 @@ def hstu_attn_bwd(desc, jag, q, k, v, d_out, rab_pos, rab_time, dq, dk, dv, d_ra
                                                 _ptr(d_out), _ptr(rab_pos), _ptr(rab_time), _ptr(dq), _ptr(dk),
                                                 _ptr(dv), _ptr(d_rab_pos), _ptr(d_rab_time), _ptr(ws),
                                                 ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def make_rab_ext(per_head: bool, n_types: int = 0, token_type=None, rab_type=None) -> hstu_rab_ext_t:
+    return hstu_rab_ext_t(per_head=int(per_head), n_types=n_types, token_type=_ptr(token_type),
+                          rab_type=_ptr(rab_type))
+
+
+def hstu_attn_ext_workspace_size(desc, jag, ext) -> int:
+    return lib().hstu_attn_ext_workspace_size(ctypes.byref(desc), ctypes.byref(jag), ctypes.byref(ext))
+
+
+def hstu_attn_fwd_ext(desc, jag, ext, q, k, v, rab_pos, rab_time, out, ws, stream=None) -> None:
+    _check("hstu_attn_fwd_ext", lib().hstu_attn_fwd_ext(ctypes.byref(desc), ctypes.byref(jag), ctypes.byref(ext),
+                                                        _ptr(q), _ptr(k), _ptr(v), _ptr(rab_pos), _ptr(rab_time),
+                                                        _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                                        _stream(stream)))
+
+
+def hstu_attn_bwd_ext_workspace_size(desc, jag, ext) -> int:
+    return lib().hstu_attn_bwd_ext_workspace_size(ctypes.byref(desc), ctypes.byref(jag), ctypes.byref(ext))
+
+
+def hstu_attn_bwd_ext(desc, jag, ext, q, k, v, d_out, rab_pos, rab_time, dq, dk, dv, d_rab_pos, d_rab_time,
+                      d_rab_type, ws, stream=None) -> None:
+    _check("hstu_attn_bwd_ext", lib().hstu_attn_bwd_ext(ctypes.byref(desc), ctypes.byref(jag), ctypes.byref(ext),
+                                                        _ptr(q), _ptr(k), _ptr(v), _ptr(d_out), _ptr(rab_pos),
+                                                        _ptr(rab_time), _ptr(dq), _ptr(dk), _ptr(dv),
+                                                        _ptr(d_rab_pos), _ptr(d_rab_time), _ptr(d_rab_type),
+                                                        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def hstu_attn_fwd_noalloc(desc, jag, q, k, v, rab_pos, rab_time, out, stream=None) -> None:
@@ -369,3 +467,43 @@ def hstu_stochastic_length_select(raw: hstu_jagged_t, keys, new_offsets, x, x_dt
            lib().hstu_stochastic_length_select(ctypes.byref(raw), _ptr(keys), _ptr(new_offsets), _ptr(x), x_dtype_code,
                                                D, _ptr(kept), _ptr(x_out), _ptr(ts_out), _ptr(ws),
                                                ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def hstu_falcon_append_workspace_size(desc, prefix_old, appended, prefix_new) -> int:
+    return lib().hstu_falcon_append_workspace_size(ctypes.byref(desc), ctypes.byref(prefix_old), ctypes.byref(appended),
+                                                   ctypes.byref(prefix_new))
+
+
+def hstu_falcon_append(desc, layers, prefix_old, kv_cache_old, appended, app_x, prefix_new, kv_cache_new, app_out,
+                       ws, stream=None) -> None:
+    """layers: a sequence of hstu_layer_weights_t (marshalled into the host array the call reads)."""
+    arr = (hstu_layer_weights_t * len(layers))(*layers)
+    _check("hstu_falcon_append", lib().hstu_falcon_append(ctypes.byref(desc), arr, ctypes.byref(prefix_old),
+                                                          _ptr(kv_cache_old), ctypes.byref(appended), _ptr(app_x),
+                                                          ctypes.byref(prefix_new), _ptr(kv_cache_new),
+                                                          _ptr(app_out), _ptr(ws), ws.numel() * ws.element_size(),
+                                                          _stream(stream)))
+
+
+def make_norm_in(gamma, beta, xn, mu, rstd, dgamma=None, dbeta=None) -> hstu_norm_in_t:
+    return hstu_norm_in_t(gamma=_ptr(gamma), beta=_ptr(beta), xn=_ptr(xn), mu=_ptr(mu), rstd=_ptr(rstd),
+                          dgamma=_ptr(dgamma), dbeta=_ptr(dbeta))
+
+
+def hstu_layer_norm_in_workspace_size(desc, jag) -> int:
+    return lib().hstu_layer_norm_in_workspace_size(ctypes.byref(desc), ctypes.byref(jag))
+
+
+def hstu_layer_fwd_norm_in(desc, jag, weights, nin, x, y, y_f16, saved, ws, stream=None) -> None:
+    _check("hstu_layer_fwd_norm_in", lib().hstu_layer_fwd_norm_in(ctypes.byref(desc), ctypes.byref(jag),
+                                                                  ctypes.byref(weights), ctypes.byref(nin), _ptr(x),
+                                                                  _ptr(y), _ptr(y_f16), ctypes.byref(saved), _ptr(ws),
+                                                                  ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def hstu_layer_bwd_norm_in(desc, jag, weights, nin, x, saved, dy, dx, dx_f16, grads, ws, stream=None) -> None:
+    _check("hstu_layer_bwd_norm_in", lib().hstu_layer_bwd_norm_in(ctypes.byref(desc), ctypes.byref(jag),
+                                                                  ctypes.byref(weights), ctypes.byref(nin), _ptr(x),
+                                                                  ctypes.byref(saved), _ptr(dy), _ptr(dx),
+                                                                  _ptr(dx_f16), ctypes.byref(grads), _ptr(ws),
+                                                                  ws.numel() * ws.element_size(), _stream(stream)))

@@ -87,6 +87,20 @@ class JaggedBatch:
         self.struct = H.make_jagged(self.offsets, self.timestamps, self.max_len)
 
 
+def shard_rows(offsets: np.ndarray, rank_of: np.ndarray, rank: int):
+    """The sequences a data-parallel split (hstu_dp_partition) gives `rank`, in batch order: their
+    offsets (int64 [B_r + 1], starting at 0) and the global rows they own (int64 [T_r]), for
+    gathering x, dy and timestamps of the rank's shard from the global batch."""
+    offsets = np.asarray(offsets, np.int64)
+    mine = np.nonzero(np.asarray(rank_of) == rank)[0]
+    lens = offsets[mine + 1] - offsets[mine]
+    off = np.zeros(mine.shape[0] + 1, np.int64)
+    np.cumsum(lens, out=off[1:])
+    rows = (np.concatenate([np.arange(offsets[b], offsets[b + 1], dtype=np.int64) for b in mine])
+            if mine.size else np.zeros(0, np.int64))
+    return off, rows
+
+
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
     """A zero-filled workspace (its first word is the device status word)."""
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)

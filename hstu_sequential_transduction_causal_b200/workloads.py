@@ -148,7 +148,7 @@ def _draw_lengths(rng: np.random.Generator, cfg: dict) -> np.ndarray:
 
 
 def make_workload(name: str, seed: int = 0, *, lengths=None, D=None, H=None, dtype=None,
-                  N=None, pos_max_len=None, layers=None, backward=None) -> Workload:
+                  N=None, pos_max_len=None, layers=None, backward=None, B=None) -> Workload:
     """Draw one of the named workloads (``c1``..``c4``), optionally overriding its shape.
 
     ``c4`` returns the *raw* sequences plus the Stochastic Length random keys in
@@ -157,7 +157,7 @@ def make_workload(name: str, seed: int = 0, *, lengths=None, D=None, H=None, dty
     """
     cfg = dict(CONFIGS[name])
     for k, v in dict(lengths=lengths, D=D, H=H, dtype=dtype, N=N, pos_max_len=pos_max_len,
-                     layers=layers, backward=backward).items():
+                     layers=layers, backward=backward, B=B).items():
         if v is not None:
             cfg[k] = v
     rng = np.random.default_rng(seed)

@@ -177,6 +177,16 @@ hstu_status_t hstu_sync_status(void* ws, hstu_stream_t stream, int32_t* device_s
  * (2^31 cycles, about a second). Process-wide; affects launches made after the call. */
 void hstu_set_wait_limit(uint64_t cycles);
 
+/* Kernel timing hook: `start` and `stop` are cudaEvent_t handles created by the caller (timing
+ * enabled). Until the next call with the same `kernel`, every call of this host thread that launches
+ * that kernel records `start` on its stream right before the launch and `stop` right after, so
+ * cudaEventElapsedTime(start, stop) is that kernel's device time (under stream capture the records
+ * become external event nodes of the graph, re-recorded at each replay). kernel: 0 the attention
+ * forward (hstu_attn_fwd, hstu_layer_fwd), 1 the attention backward (hstu_attn_bwd,
+ * hstu_layer_bwd), 2 the LayerNorm (.) U forward, 3 its backward. start = stop = NULL disables.
+ * HSTU_ERR_INVALID_ARG for another kernel number or only one NULL event. */
+hstu_status_t hstu_profile_events(int32_t kernel, void* start, void* stop);
+
 /* Test surface for the failure path: launches one CTA that waits on an mbarrier nothing ever
  * arrives at, bounded by the wait limit; it records HSTU_ERR_TIMEOUT in the status word of `ws`
  * and returns. Lets a test check the timeout path without a hang. */
@@ -257,6 +267,49 @@ hstu_status_t hstu_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* j
                             const float* rab_pos, const float* rab_time, float* dq, float* dk,
                             float* dv, float* d_rab_pos, float* d_rab_time, void* ws,
                             size_t ws_bytes, hstu_stream_t stream);
+
+/* The richer relative bias of "HSTU: The First Exploration of the Scaling Law", 7.1.4 Innovation 2,
+ * f(p_i - p_j, t_i - t_j, type_i, type_j), whose form the page does not give, read as the sum
+ *   rab_pos[idx(i - j)] + rab_time[bucket(t_i - t_j)] + rab_type[type_i][type_j]
+ * with every table either shared by the heads or given one slice per head (the first page's sketch
+ * keeps a per-head bias table). */
+typedef struct hstu_rab_ext_t {
+  int32_t per_head;           /* 0: rab_pos [2L-1], rab_time [nb], rab_type [nt][nt] shared by the heads;
+                                 1: rab_pos [H][2L-1], rab_time [H][nb], rab_type [H][nt][nt] */
+  int32_t n_types;            /* nt: 0 = no type term, else 1..16 token types */
+  const int32_t* token_type;  /* device int32 [T], each in [0, nt); NULL when nt = 0. A type outside
+                                 that range is clamped into it and reported as HSTU_ERR_DEVICE. */
+  const float* rab_type;      /* device fp32, query token's type first; NULL when nt = 0 */
+} hstu_rab_ext_t;
+
+/* Workspace bytes of hstu_attn_fwd_ext: hstu_attn_workspace_size with one bias tile per causal tile
+ * pair and head when ext->per_head (H times the tile region); 0 for a batch or descriptor it
+ * refuses (as hstu_attn_workspace_size, with the pair bound taken times H for per-head tables). */
+size_t hstu_attn_ext_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag,
+                                    const hstu_rab_ext_t* ext);
+
+/* hstu_attn_fwd with the bias of hstu_rab_ext_t (tensor-core dtypes F16 / BF16 only). rab_pos and
+ * rab_time have the shapes ext->per_head selects. HSTU_ERR_INVALID_ARG for per_head not 0 or 1, a
+ * NULL ext, or nt > 0 with a NULL token_type / rab_type; HSTU_ERR_UNSUPPORTED for nt > 16 or an F32
+ * descriptor; otherwise the errors of hstu_attn_fwd. */
+hstu_status_t hstu_attn_fwd_ext(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const hstu_rab_ext_t* ext,
+                                const void* q, const void* k, const void* v, const float* rab_pos,
+                                const float* rab_time, void* out, void* ws, size_t ws_bytes, hstu_stream_t stream);
+
+/* Workspace bytes of hstu_attn_bwd_ext (the transposed bias tiles per pair and head when
+ * per_head); 0 for a refused batch. */
+size_t hstu_attn_bwd_ext_workspace_size(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag,
+                                        const hstu_rab_ext_t* ext);
+
+/* hstu_attn_bwd with the bias of hstu_rab_ext_t: d_rab_pos, d_rab_time and d_rab_type (fp32, the
+ * shapes of the tables, overwritten; d_rab_type NULL when nt = 0) receive, per entry, the sum of
+ * dX_ij over every pair (and every head sharing the entry) that reads it. Errors as
+ * hstu_attn_fwd_ext and hstu_attn_bwd. */
+hstu_status_t hstu_attn_bwd_ext(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const hstu_rab_ext_t* ext,
+                                const void* q, const void* k, const void* v, const void* d_out,
+                                const float* rab_pos, const float* rab_time, float* dq, float* dk, float* dv,
+                                float* d_rab_pos, float* d_rab_time, float* d_rab_type, void* ws,
+                                size_t ws_bytes, hstu_stream_t stream);
 
 /* Largest number of (sequence, 128-row tile) work items, B + ceil(T / 128), that
  * hstu_attn_fwd_noalloc accepts. */
@@ -366,6 +419,71 @@ hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t*
                              size_t ws_bytes, hstu_stream_t stream);
 
 /* --------------------------------------------------------------------------------------------
+ * The input-LayerNorm variant of the layer ("4.4 Scaling Recommendation Models", section Code: the
+ * sketch normalises the layer input before f1, Xn = LayerNorm_in(X) over d_model with gamma_in,
+ * beta_in and eps = desc->ln_eps, and adds the raw X as the residual):
+ *   U, V, Q, K = Split(SiLU(Xn W1^T + b1)),  Y = f2(LayerNorm(A V) (.) U) + X.
+ * BF16 compute, D in {256, 512}; X of desc->x_dtype (BF16 or F32), Y of desc->y_dtype.
+ * -------------------------------------------------------------------------------------------- */
+typedef struct hstu_norm_in_t {
+  const float* gamma;   /* [D], 16-byte aligned */
+  const float* beta;    /* [D], 16-byte aligned */
+  void* xn;             /* fp16 [T, D], 16-byte aligned: Xn, written by the forward, read by the backward */
+  float* mu;            /* [T]: LayerNorm_in statistics, written by the forward */
+  float* rstd;          /* [T] */
+  float* dgamma;        /* [D]: the backward's gradients of gamma and beta (fp32, overwritten) */
+  float* dbeta;         /* [D] */
+} hstu_norm_in_t;
+
+/* Workspace bytes of both hstu_layer_fwd_norm_in and hstu_layer_bwd_norm_in (0 for a batch they refuse). */
+size_t hstu_layer_norm_in_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
+
+/* Forward: Xn, mu, rstd into nin; the layer on Xn as in hstu_layer_fwd (saved as there), with X as
+ * the residual. Errors of hstu_layer_fwd, plus HSTU_ERR_INVALID_ARG for a NULL nin member the call
+ * writes or reads and HSTU_ERR_UNSUPPORTED for another compute dtype, D or an unaligned pointer. */
+hstu_status_t hstu_layer_fwd_norm_in(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag,
+                                     const hstu_layer_weights_t* w, const hstu_norm_in_t* nin, const void* x, void* y,
+                                     void* y_f16, const hstu_layer_saved_t* saved, void* ws, size_t ws_bytes,
+                                     hstu_stream_t stream);
+
+/* Backward: as hstu_layer_bwd with dW1 = dZ^T Xn, then dXn = dZ W1 through the input LayerNorm:
+ * dX = dY + LN_in^T(dXn) (dx of desc->x_dtype, dx_f16 nullable fp16 copy), nin->dgamma and
+ * nin->dbeta overwritten. dy: [T, D] of desc->y_dtype, which must equal desc->x_dtype. */
+hstu_status_t hstu_layer_bwd_norm_in(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag,
+                                     const hstu_layer_weights_t* w, const hstu_norm_in_t* nin, const void* x,
+                                     const hstu_layer_saved_t* saved, const void* dy, void* dx, void* dx_f16,
+                                     const hstu_layer_grads_t* grads, void* ws, size_t ws_bytes,
+                                     hstu_stream_t stream);
+
+/* --------------------------------------------------------------------------------------------
+ * Data parallelism ("4.4 Scaling Recommendation Models", Generative Recommenders and HSTU,
+ * Efficiency tricks: the sequences of a batch are independent, so one global batch is split over
+ * ranks by whole sequences and the only exchange is the gradient sum). Host functions; no CUDA.
+ * -------------------------------------------------------------------------------------------- */
+
+/* Work of one layer step on a sequence of n tokens, in units of 2 D flops: n (n + 1) + 5 D n (the
+ * attention's 2 D n (n + 1) flops plus the projections' 10 D^2 n). */
+double hstu_dp_sequence_cost(int64_t n, int32_t D);
+
+/* Assigns each of B sequences (lengths: HOST int64 [B]) to one of `world` ranks, balancing
+ * hstu_dp_sequence_cost: sequences by decreasing cost (ties by index), each to the least loaded rank
+ * (ties by lowest rank); deterministic, so every rank computes the same split. The largest rank load
+ * is at most 4/3 of the best split's. rank_of: HOST int32 [B], receives the rank of each sequence;
+ * rank_cost: HOST double [world] or NULL, receives each rank's summed cost. HSTU_ERR_INVALID_ARG for
+ * B < 0, world < 1, D < 1, a negative length or a NULL array when B > 0. */
+hstu_status_t hstu_dp_partition(const int64_t* lengths, int32_t B, int32_t D, int32_t world, int32_t* rank_of,
+                                double* rank_cost);
+
+/* Events for overlapping the gradient all-reduce of data parallelism with the rest of a backward:
+ * until the next call, every hstu_layer_bwd of this host thread records `early` on its stream once
+ * dW2, db2, dgamma, dbeta, drab_pos and drab_time are final (before the SiLU and f1 backward), and
+ * `w1` once dW1 and db1 are final (before the dX GEMM). A communication stream that waits on them
+ * can reduce those gradients while the remaining kernels run. Under stream capture they are
+ * recorded as capture dependencies, so a stream that waits on them forks from the captured graph.
+ * Both NULL disables; HSTU_ERR_INVALID_ARG when only one is NULL. */
+hstu_status_t hstu_layer_bwd_ready_events(void* early, void* w1);
+
+/* --------------------------------------------------------------------------------------------
  * Stochastic Length ("HSTU: The First Exploration of the Scaling Law", 7.1.5 Stochastic Length):
  * a history of n tokens keeps L = min(n, floor(n^(alpha/2) + 1/2)) tokens, the L tokens with the
  * smallest random keys (ties broken by position), in their original order; positions are
@@ -446,6 +564,32 @@ hstu_status_t hstu_falcon_fwd(const hstu_falcon_desc_t* desc, const hstu_layer_w
                               int32_t cache_valid, void* prefix_out, const void* cand_x,
                               const int64_t* request_ts, void* out, void* ws, size_t ws_bytes,
                               hstu_stream_t stream);
+
+/* M-FALCON prefix append ("HSTU: The First Exploration of the Scaling Law", 7.1.5 M-FALCON: the
+ * history's K, V cache is reused across requests): extends every user's cached prefix by new actions
+ * without recomputing the old prefix. In a causal layer a token's K and V do not depend on later
+ * tokens, so the old rows' cache entries are kept and only the appended tokens run through the L
+ * layers, each attending to the whole cached prefix and to the appended tokens before it (their
+ * positions continue from n_old, their timestamps are those of prefix_new).
+ *  prefix_old: the cached prefixes (users = B, n_old_u tokens each); kv_cache_old as written by
+ *    hstu_falcon_fwd (cache_valid = 0) or an earlier append for them.
+ *  appended: B = users jagged rows of the new actions (offsets: device [users+1]; timestamps unused),
+ *    their bf16 input rows in app_x [appended->T, D].
+ *  prefix_new: the combined prefixes, n_old_u + a_u tokens per user (old tokens first), with the
+ *    combined timestamps; kv_cache_new (hstu_falcon_cache_size(desc, prefix_new) bytes, not
+ *    overlapping kv_cache_old) receives the combined cache, ready for hstu_falcon_fwd with
+ *    cache_valid = 1 on prefix_new.
+ *  app_out: fp32 [appended->T, D] or NULL, the appended tokens' last-layer output (equal to the rows
+ *    a full causal forward over prefix_new gives them).
+ * Errors: those of hstu_falcon_fwd for prefix_new, HSTU_ERR_INVALID_ARG when prefix_old or appended
+ * do not have `users` sequences or prefix_old->T + appended->T != prefix_new->T; a user whose
+ * combined length is not n_old + a is reported as HSTU_ERR_DEVICE and left out. */
+size_t hstu_falcon_append_workspace_size(const hstu_falcon_desc_t* desc, const hstu_jagged_t* prefix_old,
+                                         const hstu_jagged_t* appended, const hstu_jagged_t* prefix_new);
+hstu_status_t hstu_falcon_append(const hstu_falcon_desc_t* desc, const hstu_layer_weights_t* layers,
+                                 const hstu_jagged_t* prefix_old, const void* kv_cache_old,
+                                 const hstu_jagged_t* appended, const void* app_x, const hstu_jagged_t* prefix_new,
+                                 void* kv_cache_new, void* app_out, void* ws, size_t ws_bytes, hstu_stream_t stream);
 
 #ifdef __cplusplus
 }

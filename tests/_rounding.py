@@ -91,12 +91,12 @@ def attention_bwd(q, k, v, do, off, ts, rab_pos, rab_time, inv_N, L, r=rounder()
     return dq, dk, dv, drp, drt
 
 
-def layer_fwd(x, p, off, ts, H, inv_N, L, r=rounder()):
-    """Y and the saved intermediates; f1 reads r(x), the residual adds x itself."""
+def layer_fwd(x, p, off, ts, H, inv_N, L, r=rounder(), x_f1=None):
+    """Y and the saved intermediates; f1 reads r(x) (or x_f1 when given), the residual adds x itself."""
     x = _same(x)
     T, D = x.shape
     d = D // H
-    z, s = O.uvqk_fwd(r("x", x), p.W1, p.b1)
+    z, s = O.uvqk_fwd(r("x", x) if x_f1 is None else x_f1, p.W1, p.b1)
     z, s = r("z", z), r("uvqk", s)
     u, v, q, k = O.split_uvqk(s, D)
     o = attention_fwd(q.reshape(T, H, d), k.reshape(T, H, d), v.reshape(T, H, d), off, ts, p.rab_pos,
@@ -104,7 +104,7 @@ def layer_fwd(x, p, off, ts, H, inv_N, L, r=rounder()):
     g, mu, rstd = O.norm_gate_fwd(o, u, p.gamma, p.beta)
     g = r("g", g)
     y = O.out_proj_fwd(g, p.W2, p.b2, x)
-    return y, dict(x=x, z=z, s=s, o=o, g=g, mu=mu, rstd=rstd)
+    return y, dict(x=x if x_f1 is None else x_f1, z=z, s=s, o=o, g=g, mu=mu, rstd=rstd)
 
 
 def layer_bwd(dy, p, sv, off, ts, H, inv_N, L, r=rounder()):
@@ -127,8 +127,28 @@ def layer_bwd(dy, p, sv, off, ts, H, inv_N, L, r=rounder()):
                                          r("do", do).reshape(T, H, d), off, ts, p.rab_pos, p.rab_time, inv_N, L, r)
     ds = np.concatenate([du, dv.reshape(T, D), dq.reshape(T, D), dk.reshape(T, D)], axis=1)
     dz = r("dz", ds * O.silu_grad(z))
-    return dict(dx=dy + dz @ W1, dW1=dz.T @ r("x", x), db1=dz.sum(axis=0), dW2=dW2, db2=db2, dgamma=dgamma,
+    return dict(dx=dy + dz @ W1, dz=dz, dW1=dz.T @ r("x", x), db1=dz.sum(axis=0), dW2=dW2, db2=db2, dgamma=dgamma,
                 dbeta=dbeta, drab_pos=drp, drab_time=drt)
+
+
+def layer_fwd_norm_in(x, p, gamma_in, beta_in, off, ts, H, inv_N, L, r=rounder()):
+    """The norm_in variant: f1 reads Xn = LayerNorm_in(x) stored in fp16, the residual adds x."""
+    x = _same(x)
+    xn, mu, rstd = O.norm_gate_fwd(x, np.ones_like(x), gamma_in, beta_in)
+    y, sv = layer_fwd(x, p, off, ts, H, inv_N, L, r, x_f1=r("x", xn))
+    sv.update(x_raw=x, mu_in=mu, rstd_in=rstd)
+    return y, sv
+
+
+def layer_bwd_norm_in(dy, p, gamma_in, sv, off, ts, H, inv_N, L, r=rounder()):
+    """Its backward: dW1 = dZ^T Xn (fp16 Xn), dXn = dZ W1 in fp32, dX = dY + LN_in^T(dXn)."""
+    g = layer_bwd(dy, p, sv, off, ts, H, inv_N, L, r)
+    dxn = g["dz"] @ _same(p.W1)
+    x = sv["x_raw"]
+    dx_in, dgi, dbi = O.norm_gate_bwd(dxn, x, np.ones_like(x), gamma_in, sv["mu_in"], sv["rstd_in"])
+    g = dict(g)
+    g.update(dx=_same(dy) + dx_in, dgamma_in=dgi, dbeta_in=dbi)
+    return g
 
 
 def stack_fwd_bwd(x, layers, off, ts, H, inv_N, L, dy, r=rounder()):

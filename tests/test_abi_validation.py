@@ -494,3 +494,85 @@ def test_last_cuda_error_is_per_host_thread(L):
     t.join()
     assert seen["before"] == 0 and seen["marked"] != 0
     assert L.hstu_last_cuda_error() == mine != seen["marked"]
+
+
+def test_profile_events(L):
+    assert L.hstu_profile_events(4, fake(0), fake(1)) == INVALID        # no such kernel
+    assert L.hstu_profile_events(-1, None, None) == INVALID
+    assert L.hstu_profile_events(0, fake(0), None) == INVALID           # one event only
+    assert L.hstu_profile_events(0, None, fake(1)) == INVALID
+    for k in range(4):
+        assert L.hstu_profile_events(k, None, None) == OK               # disabling is always fine
+
+
+def rab_ext(**kw):
+    e = Hb.hstu_rab_ext_t(per_head=1, n_types=3, token_type=fake(20), rab_type=fake(21))
+    for k, v in kw.items():
+        setattr(e, k, v)
+    return e
+
+
+def test_attn_fwd_ext(L):
+    need = L.hstu_attn_ext_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag()), ctypes.byref(rab_ext()))
+    shared = L.hstu_attn_ext_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag()),
+                                            ctypes.byref(rab_ext(per_head=0)))
+    assert need > shared == L.hstu_attn_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag()))
+
+    def call(d=None, j=None, e="default", q=fake(2), ws_bytes=need):
+        ext = ctypes.byref(rab_ext()) if e == "default" else (None if e is None else ctypes.byref(e))
+        return L.hstu_attn_fwd_ext(ctypes.byref(d or attn_desc()), ctypes.byref(j or jag()), ext, q, fake(3), fake(4),
+                                   fake(5), fake(6), fake(7), fake(8), ws_bytes, None)
+    run_cases(L, call, [
+        ("no ext", dict(e=None), INVALID),
+        ("per_head 2", dict(e=rab_ext(per_head=2)), INVALID),
+        ("17 types", dict(e=rab_ext(n_types=17)), UNSUPPORTED),
+        ("types without a type array", dict(e=rab_ext(token_type=None)), INVALID),
+        ("types without a type table", dict(e=rab_ext(rab_type=None)), INVALID),
+        ("workspace sized for shared tables", dict(ws_bytes=shared), WORKSPACE),
+        ("fp32 descriptor", dict(d=attn_desc(dtype=F32, o_dtype=F32)), UNSUPPORTED),
+        ("no q", dict(q=None), INVALID),
+    ])
+    assert passes_host_checks(L, call, e=rab_ext(n_types=0, token_type=None, rab_type=None))
+
+
+def test_attn_bwd_ext(L):
+    need = L.hstu_attn_bwd_ext_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag()), ctypes.byref(rab_ext()))
+    assert need > L.hstu_attn_bwd_workspace_size(ctypes.byref(attn_desc()), ctypes.byref(jag()))
+
+    def call(e="default", drty=fake(14), ws_bytes=need):
+        ext = ctypes.byref(rab_ext()) if e == "default" else (None if e is None else ctypes.byref(e))
+        return L.hstu_attn_bwd_ext(ctypes.byref(attn_desc()), ctypes.byref(jag()), ext, fake(2), fake(3), fake(4),
+                                   fake(5), fake(6), fake(7), fake(8), fake(9), fake(10), fake(11), fake(12), drty,
+                                   fake(13), ws_bytes, None)
+    run_cases(L, call, [
+        ("no ext", dict(e=None), INVALID),
+        ("types without d_rab_type", dict(drty=None), INVALID),
+        ("small workspace", dict(ws_bytes=need - 1), WORKSPACE),
+    ])
+    assert passes_host_checks(L, call, e=rab_ext(n_types=0, token_type=None, rab_type=None), drty=None)
+
+
+def test_falcon_append(L):
+    old, app, new = jag(T=200), jag(T=100), jag(T=300)
+    need = L.hstu_falcon_append_workspace_size(ctypes.byref(falcon_desc()), ctypes.byref(old), ctypes.byref(app),
+                                               ctypes.byref(new))
+    assert need > 0
+
+    def call(d=None, o=None, a=None, n=None, layers=None, cache_old=fake(2), app_x=fake(3), cache_new=fake(4),
+             out=fake(5), ws_bytes=need):
+        arr = (Hb.hstu_layer_weights_t * 2)(*(layers or [weights(), weights()]))
+        return L.hstu_falcon_append(ctypes.byref(d or falcon_desc()), arr, ctypes.byref(o or old), cache_old,
+                                    ctypes.byref(a or app), app_x, ctypes.byref(n or new), cache_new, out, fake(6),
+                                    ws_bytes, None)
+    run_cases(L, call, [
+        ("old and appended rows do not add up", dict(a=jag(T=99)), INVALID),
+        ("appended batch with another user count", dict(a=jag(B=3, T=100)), INVALID),
+        ("users differ from the combined batch", dict(d=falcon_desc(users=3)), INVALID),
+        ("workspace one byte short", dict(ws_bytes=need - 1), WORKSPACE),
+        ("no new cache", dict(cache_new=None), INVALID),
+        ("no old cache", dict(cache_old=None), INVALID),
+        ("no appended rows", dict(app_x=None), INVALID),
+        ("new cache off 16 bytes", dict(cache_new=fake(4) + 2), UNSUPPORTED),
+        ("second layer without W2", dict(layers=[weights(), weights(W2=None)]), INVALID),
+        ("head width 32", dict(d=falcon_desc(H=8)), UNSUPPORTED),
+    ])

@@ -75,3 +75,15 @@ def test_attn_bwd_odd_heads_long_sequence():
     st, got, exp = _run_attn_bwd([1100, 3], 3, 1200, 1.0 / 2048, seed=5)
     assert st == 0
     _check(got, exp)
+
+
+@pytest.mark.parametrize("lengths", [
+    [17, 64, 3, 1, 0, 40, 60, 5, 12, 64, 64, 1, 33, 130, 2],
+    [(7 * i) % 66 for i in range(45)] + [200, 3],
+])
+def test_attn_bwd_packed_short_sequences(lengths):
+    """The backward over packs of short sequences (one key tile per pack, queries limited to the key's
+    own sequence, the packed members' own pairs skipped by the table gradients)."""
+    st, got, exp = _run_attn_bwd(lengths, 2, 300, 1.0 / 128, seed=9, spread=True)
+    assert st == 0
+    _check(got, exp)

@@ -100,3 +100,57 @@ def test_falcon_ranking_workload_every_candidate():
     assert got.shape == yc_ref.shape == (16 * 1024, fw.D)
     assert_close(got, yc_ref, *BF16_TOL, what="ranking workload candidates (all)")
     assert_close(r.prefix_out.float().cpu().numpy(), yp_ref, *BF16_TOL, what="ranking workload prefix output")
+
+
+def test_falcon_prefix_append_matches_a_rebuilt_prefix():
+    """hstu_falcon_append grows cached prefixes of 130, 0, 1 and 257 tokens by 5, 3, 0 and 130 new
+    actions. The combined cache must be bit-identical to one built from scratch over the combined
+    prefixes (each row's K, V come from the same per-row arithmetic), the appended tokens' output
+    must equal the rows a full causal forward over the combined prefixes gives them (bit-identical
+    on the GPU, and within the bf16 bound of the oracle), and candidates scored from the appended
+    cache must match the oracle's M-FALCON over the combined prefixes."""
+    old_lens, app_lens = [130, 0, 1, 257], [5, 3, 0, 130]
+    fw = W.make_falcon_workload(seed=14, prefix_lengths=[o + a for o, a in zip(old_lens, app_lens)], m=7, b_m=7,
+                                D=128, H=2, layers=2, N=400, pos_max_len=400)
+    off = fw.prefix_offsets
+    rows_old = np.concatenate([np.arange(off[u], off[u] + old_lens[u]) for u in range(4)]).astype(np.int64)
+    rows_app = np.concatenate([np.arange(off[u] + old_lens[u], off[u + 1]) for u in range(4)]).astype(np.int64)
+    fw_old = W.FalconWorkload(D=fw.D, H=fw.H, N=fw.N, pos_max_len=fw.pos_max_len, layers=fw.layers,
+                              prefix_offsets=W.offsets_from_lengths(old_lens), prefix_ts=fw.prefix_ts[rows_old],
+                              prefix_x=fw.prefix_x[rows_old], cand_x=fw.cand_x, request_ts=fw.request_ts, m=fw.m,
+                              b_m=fw.b_m)
+    r_old = FalconRun(fw_old, fw.b_m)
+    r_old.run(cache_valid=0)
+    r_new = FalconRun(fw, fw.b_m)           # the combined prefixes, built from scratch
+    r_new.run(cache_valid=0)
+    jag_app = JaggedBatch(W.offsets_from_lengths(app_lens), fw.prefix_ts[rows_app], max_len=max(app_lens))
+    cache = torch.full_like(r_new.cache, float("nan"))
+    app_out = torch.full((len(rows_app), fw.D), float("nan"), dtype=torch.float32, device="cuda")
+    ws = workspace(H.hstu_falcon_append_workspace_size(r_new.desc, r_old.jag.struct, jag_app.struct,
+                                                       r_new.jag.struct))
+    H.hstu_falcon_append(r_new.desc, r_new.weights, r_old.jag.struct, r_old.cache, jag_app.struct,
+                         to_dev(fw.prefix_x[rows_app], torch.bfloat16), r_new.jag.struct, cache, app_out, ws)
+    torch.cuda.synchronize()
+    assert H.hstu_sync_status(ws) == 0
+    assert torch.equal(cache, r_new.cache)
+    assert torch.equal(app_out, r_new.prefix_out[torch.from_numpy(rows_app).cuda()])
+    yc_ref, yp_ref = _oracle(fw)
+    assert_close(app_out.cpu().numpy(), yp_ref[rows_app], *BF16_TOL, what="appended tokens' output")
+    r_new.cache.copy_(cache)
+    r_new.px.fill_(float("nan"))            # cache_valid = 1 does not read the prefix input
+    assert_close(r_new.run(cache_valid=1), yc_ref, *BF16_TOL, what="candidates on the appended cache")
+
+
+def test_falcon_append_of_nothing_keeps_the_cache():
+    lens = [64, 0, 200]
+    fw = W.make_falcon_workload(seed=15, prefix_lengths=lens, m=3, b_m=3, D=128, H=2, layers=2, N=300,
+                                pos_max_len=300)
+    r = FalconRun(fw, fw.b_m)
+    r.run(cache_valid=0)
+    jag_app = JaggedBatch(np.zeros(4, np.int64), np.zeros(0, np.int64), max_len=0)
+    cache = torch.full_like(r.cache, float("nan"))
+    ws = workspace(H.hstu_falcon_append_workspace_size(r.desc, r.jag.struct, jag_app.struct, r.jag.struct))
+    H.hstu_falcon_append(r.desc, r.weights, r.jag.struct, r.cache, jag_app.struct, None, r.jag.struct, cache, None, ws)
+    torch.cuda.synchronize()
+    assert H.hstu_sync_status(ws) == 0
+    assert torch.equal(cache, r.cache)

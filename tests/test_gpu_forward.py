@@ -418,3 +418,50 @@ def test_empty_sequences_only():
     got, st = _run_attn(off, np.zeros(0, np.int64), np.zeros((0, 64)), np.zeros((0, 64)), np.zeros((0, 64)),
                         np.zeros(15, np.float32), np.zeros(128, np.float32), 1, 64, 8, 1.0, True, max_len=1)
     assert st == 0 and got.shape == (0, 64)
+
+
+def test_profile_events_time_the_attention_kernel():
+    """The timing hook records its two events around the attention forward kernel only: the kernel's
+    time is positive and shorter than the whole call (work list and bias tiles included)."""
+    wl = W.make_workload("c2", seed=0)
+    Hh, d, L = wl.H, wl.D // wl.H, wl.pos_max_len
+    off, ts, q, k, v, rp, rt = _attn_case(list(np.diff(wl.offsets)), Hh, d, L, 1 / wl.N, True, seed=3, f16=True)
+    jag = JaggedBatch(off, ts)
+    desc = H.make_attn_desc(Hh, d, d, 1 / wl.N, L, H.HSTU_F16, Hh * d, Hh * d, Hh * d, Hh * d)
+    ws = workspace(H.hstu_attn_workspace_size(desc, jag.struct))
+    out = torch.empty(jag.T, Hh * d, dtype=torch.float32, device="cuda")
+    args = [to_dev(a, torch.float16) for a in (q, k, v)] + [to_dev(rp, torch.float32), to_dev(rt, torch.float32)]
+    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    H.hstu_profile_events(H.PROFILE_ATTN_FWD, k0, k1)
+    try:
+        for _ in range(3):
+            c0.record()
+            H.hstu_attn_fwd(desc, jag.struct, *args, out, ws)
+            c1.record()
+        torch.cuda.synchronize()
+    finally:
+        H.hstu_profile_events(H.PROFILE_ATTN_FWD)
+    assert H.hstu_sync_status(ws) == 0
+    kern, whole = k0.elapsed_time(k1), c0.elapsed_time(c1)
+    assert 0 < kern < whole, (kern, whole)
+
+
+@pytest.mark.parametrize("lengths", [
+    [17, 64, 3, 1, 0, 40, 60, 5, 12, 64, 64, 1, 33, 130, 2],                 # one-warp work list (B <= 32)
+    [(7 * i) % 66 for i in range(45)] + [200, 3],                              # block work list (B > 32)
+])
+def test_attn_fwd_packed_short_sequences(lengths):
+    """Runs of short sequences (at most 64 tokens each, at most 128 rows together) share one 128-row
+    tile, every row seeing only its own sequence's keys: the output must be the oracle's, with
+    sequences of length 0 and 1 inside packs, packs that end exactly at 128 rows and long sequences
+    between them."""
+    Hh, d, L, inv_N = 2, 64, 300, 1.0 / 128
+    off, ts, q, k, v, rp, rt = _attn_case(lengths, Hh, d, L, inv_N, True, seed=8, spread_ts=True, f16=True)
+    got, st = _run_attn(off, ts, q, k, v, rp, rt, Hh, d, L, inv_N, True, f16=True)
+    assert st == 0
+    T = int(off[-1])
+    exp = O.pointwise_attention_fwd(q.reshape(T, Hh, d), k.reshape(T, Hh, d), v.reshape(T, Hh, d), off, ts, rp, rt,
+                                    inv_N, L, THR).reshape(T, Hh * d)
+    scale = float(np.sqrt(np.mean(exp ** 2)))
+    assert_close(got, exp, 1e-2 * scale, 1e-2, what="O (packed short sequences)")

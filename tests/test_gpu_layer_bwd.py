@@ -2,11 +2,12 @@
 against the oracle's closed-form gradients (pinned to finite differences on the CPU).
 
 dx (an O(1) activation gradient) meets the bf16 bound |d| <= 1e-2 + 1e-2 |ref| element by element.
-Weight and table gradients are sums over all tokens whose scale rms(ref) is far from 1 (dW1 ~ 14 on
-the long-sequence workload); their bound applies the absolute term in units of that scale, and each
-tensor is also held to a norm-relative error <= 1e-2. Elements outside the unscaled bound are counted
-and printed: they come from fp16 rounding of the attention operands (inherent to tensor-core
-attention) meeting heavy cancellation in sums over thousands of tokens.
+Weight and table gradients are sums over all tokens whose scale rms(ref) is far from 1 (dW1 ~ 34 on
+the long-sequence workload). With 16-bit attention operands some of their elements cannot meet the
+stated bound (tests/test_rounding_floor.py), so for each of them the count outside it is held to a
+multiple of the count of the rounding model of tests/_rounding.py on the same inputs; every element
+is held to the bound taken in units of the tensor's scale, and the tensor to a norm-relative error
+<= 1e-2.
 """
 import numpy as np
 import pytest
@@ -15,8 +16,8 @@ import torch
 from oracle import hstu_oracle as O
 from hstu_sequential_transduction_causal_b200 import hstu as H
 from hstu_sequential_transduction_causal_b200 import workloads as W
-from hstu_sequential_transduction_causal_b200.runtime import (DeviceLayer, JaggedBatch, LayerRunner, to_dev,
-                                                              workspace)
+from hstu_sequential_transduction_causal_b200.runtime import (DeviceLayer, JaggedBatch, LayerRunner, SavedActs,
+                                                              to_dev, workspace)
 from tests import _rounding as R
 from tests._util import BF16_TOL, THR, assert_close
 
@@ -144,3 +145,59 @@ def test_layer_bwd_long_sequence_workload_full():
     wl = W.make_workload("c3", seed=0)
     dx, grads = _run_layer_fwd_bwd(wl)
     _compare(dx, grads, _oracle_grads(wl), _model_grads(wl), "long-sequence-full ")
+
+
+@pytest.mark.parametrize("x_dtype", [torch.bfloat16, torch.float32])
+def test_layer_norm_in_variant_fwd_bwd(x_dtype):
+    """The sketch's input-LayerNorm variant (hstu_layer_fwd_norm_in / _bwd_norm_in) against the
+    oracle's layer_fwd_norm_in / layer_bwd_norm_in: Y element by element within the bf16 bound, dX
+    and the gradients (dgamma_in and dbeta_in included) as in _compare, with the rounding model
+    (tests/_rounding.py) extended by the fp16 Xn."""
+    wl = W.make_workload("c3", seed=6, lengths=[1, 130, 300, 0, 257, 64], pos_max_len=512, N=512)
+    rng = np.random.default_rng(17)
+    x = 2.0 + 1.5 * rng.standard_normal((wl.T, wl.D))          # not normalised: the input LayerNorm matters
+    x = W.round_bf16(x) if x_dtype == torch.bfloat16 else x.astype(np.float32)
+    g_in = (1 + 0.2 * rng.standard_normal(wl.D)).astype(np.float32)
+    b_in = (0.2 * rng.standard_normal(wl.D)).astype(np.float32)
+    jag = JaggedBatch(wl.offsets, wl.timestamps)
+    layer = DeviceLayer.upload(wl.layers[0], wl.D, wl.H, True)
+    code = H.HSTU_BF16 if x_dtype == torch.bfloat16 else H.HSTU_F32
+    desc = H.make_layer_desc(wl.D, wl.H, 1.0 / wl.N, wl.pos_max_len, H.HSTU_BF16, code, code)
+    T, D = wl.T, wl.D
+    sv = SavedActs.empty(T, D, torch.bfloat16, True)
+    xn = torch.empty(T, D, dtype=torch.float16, device="cuda")
+    mu, rstd = (torch.empty(T, dtype=torch.float32, device="cuda") for _ in range(2))
+    dg_in, db_in = (torch.full((D,), float("nan"), dtype=torch.float32, device="cuda") for _ in range(2))
+    g_in_d, b_in_d = to_dev(g_in, torch.float32), to_dev(b_in, torch.float32)   # kept alive: nin holds pointers
+    nin = H.make_norm_in(g_in_d, b_in_d, xn, mu, rstd, dg_in, db_in)
+    ws = workspace(H.hstu_layer_norm_in_workspace_size(desc, jag.struct))
+    xd = to_dev(x, x_dtype)
+    y = torch.full((T, D), float("nan"), dtype=x_dtype, device="cuda")
+    weights = layer.weights()
+    H.hstu_layer_fwd_norm_in(desc, jag.struct, weights, nin, xd, y, None, sv.struct(), ws)
+    grads = [torch.full(s, float("nan"), dtype=torch.float32, device="cuda")
+             for s in [(4 * D, D), (4 * D,), (D, D), (D,), (D,), (D,), (2 * wl.pos_max_len - 1,), (128,)]]
+    dy_np = W.round_bf16(rng.standard_normal((T, D))) if x_dtype == torch.bfloat16 else \
+        rng.standard_normal((T, D)).astype(np.float32)
+    dx = torch.full((T, D), float("nan"), dtype=x_dtype, device="cuda")
+    H.hstu_layer_bwd_norm_in(desc, jag.struct, weights, nin, xd, sv.struct(), to_dev(dy_np, x_dtype), dx, None,
+                             H.layer_grads(*grads), ws)
+    torch.cuda.synchronize()
+    assert H.hstu_sync_status(ws) == 0
+    p = wl.layers[0]
+    args = (wl.offsets, wl.timestamps, wl.H, 1.0 / wl.N, wl.pos_max_len)
+    ye, sve = O.layer_fwd_norm_in(x, p, g_in, b_in, *args, THR)
+    assert_close(y.float().cpu().numpy(), ye, *BF16_TOL, what="Y (norm_in)")
+    ref = O.layer_bwd_norm_in(dy_np, p, g_in, sve, *args, THR)
+    _, svm = R.layer_fwd_norm_in(x, p, g_in, b_in, *args)
+    model = R.layer_bwd_norm_in(dy_np, p, g_in, svm, *args)
+    dxg = dx.float().cpu().numpy()
+    dscale = max(1.0, float(np.sqrt(np.mean(ref["dx"] ** 2))))
+    assert R.misses(dxg, ref["dx"]) <= R.miss_ceiling(R.misses(model["dx"], ref["dx"]), dxg.size)
+    assert_close(dxg, ref["dx"], 1e-2 * dscale, 1e-2, what="dX (norm_in)")
+    got = [g.cpu().numpy() for g in grads] + [dg_in.cpu().numpy(), db_in.cpu().numpy()]
+    for name, g in zip(NAMES + ("dgamma_in", "dbeta_in"), got):
+        e = np.asarray(ref[name], np.float64)
+        scale = max(1.0, float(np.sqrt(np.mean(e ** 2))))
+        assert R.misses(g, e) <= R.miss_ceiling(R.misses(model[name], e), e.size), name
+        assert_close(g, e, 1e-2 * scale, 1e-2, what=f"{name} (norm_in)")
