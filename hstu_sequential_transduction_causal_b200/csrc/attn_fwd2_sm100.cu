@@ -462,10 +462,17 @@ attn_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 //                quadrant (warp & 3) and one key half ((warp >> 2) & 1). The group that runs a
 //                unit's last step also writes its output.
 //   warp 16    : scheduler (lane 0 takes the next unit, publishes it in a two-slot ring) and TMA
-//                producer of Q (two buffers), K and V (three stages each).
+//                producer of Q (two buffers) and K (three stages); it takes the next unit as soon as
+//                it has issued the current unit's last K load, so the next unit's loads start while
+//                the current one computes.
 //   warp 17    : tcgen05 issuer of S = Q K^T into three TMEM tiles.
-//   warp 18    : TMA producer of the bias tiles (three stages).
+//   warp 18    : TMA producer of the bias tiles and of V (three stages each), per step the bias then
+//                V, so that waiting for a V stage (freed by a P V MMA) never holds back a K load or
+//                the next unit.
 //   warp 19    : tcgen05 issuer of O += P V, P read from TMEM, into two alternating O accumulators.
+// (20 warps: five per SM sub-partition leave 96 registers a thread.)
+// Every tile is loaded as 8 KB boxes of 64 rows from separate lanes: a thread keeps about one TMA
+// copy in flight, and tile loads take thousands of cycles when every SM is loading.
 struct Smem3 {
   static constexpr int kNQ = 2, kNK = 3, kNV = 3, kBS = 3;
   static constexpr int kQ = 0;
@@ -478,10 +485,15 @@ struct Smem3 {
 static_assert(Smem3::kTotal <= 232448, "shared memory of the persistent attention kernel");
 
 constexpr int kThreads3 = 32 * (2 * kSiluWarps + 4);
-constexpr int kUnitConsumers = 2 * kSiluWarps + 3;   // SiLU warps, S issuer, bias warp, P V issuer
+constexpr int kUnitConsumers = 2 * kSiluWarps + 3;   // SiLU warps, S issuer, bias / V warp, P V issuer
 
+// A unit as the scheduler publishes it, with everything the other roles need about it (reading
+// offsets, pair_base or the pack array from global memory inside the pipeline stalled it by thousands
+// of cycles): sequence b, query tile qt (-k for a pack of k short sequences), head h, first row and
+// row count of the sequence (or pack), its first causal pair, and the first query row to write.
 struct UnitRec {
   int b, qt, h, valid;
+  int row0, n, pair0, q_lo;
 };
 
 template <bool F16>
@@ -502,8 +514,8 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
   // 37 o_empty[2]
   constexpr int kNumBars = 39;
   UnitRec* ring = reinterpret_cast<UnitRec*>(smem + L::kBar + 320);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + 352);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBar + 356);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBar + 384);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBar + 388);
   const uint32_t bar0 = smem_u32(bars);
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   auto u_full = [&](int i) { return BAR(0 + i); };
@@ -578,37 +590,28 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
   auto take_unit = [&](int uc, UnitRec& r) -> bool {
     const int slot = uc & 1;
     if (!mbar_wait_warp(u_full(slot), (uc >> 1) & 1, abort_flag, ctl)) return false;
-    int v[4] = {0, 0, 0, 0};
+    int v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (lane == 0) {
       const UnitRec x = ring[slot];
-      v[0] = x.b; v[1] = x.qt; v[2] = x.h; v[3] = x.valid;
+      v[0] = x.b; v[1] = x.qt; v[2] = x.h; v[3] = x.valid; v[4] = x.row0; v[5] = x.n; v[6] = x.pair0; v[7] = x.q_lo;
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = __shfl_sync(0xffffffffu, v[i], 0);
-    r.b = v[0]; r.qt = v[1]; r.h = v[2]; r.valid = v[3];
+    for (int i = 0; i < 8; ++i) v[i] = __shfl_sync(0xffffffffu, v[i], 0);
+    r.b = v[0]; r.qt = v[1]; r.h = v[2]; r.valid = v[3]; r.row0 = v[4]; r.n = v[5]; r.pair0 = v[6]; r.q_lo = v[7];
     __syncwarp();
     if (lane == 0) mbar_arrive(u_empty(slot));
     return true;
   };
 
   if (warp == kTmaWarp) {
-    // ---------------- scheduler + Q / K / V producer ----------------
+    // ---------------- scheduler + Q / K producer ----------------
     const long long total = static_cast<long long>(*a.count) * a.H;
     int sg = 0;
     bool ok = true;
-    auto load_v = [&](int s, int vrow, int h) -> bool {
-      const int st = s % NV;
-      if (s >= NV && !mbar_wait_warp(v_empty(st), ((s / NV) - 1) & 1, abort_flag, ctl)) return false;
-      if (lane == 8 + st) {
-        mbar_arrive_expect_tx(v_full(st), 16384);
-        tma_load_2d(sV + st * 16384, &tmV, v_full(st), h * kD, vrow);
-      }
-      return true;
-    };
     for (int uc = 0; ok; ++uc) {
       const int slot = uc & 1;
       if (uc >= 2 && !mbar_wait_warp(u_empty(slot), ((uc >> 1) - 1) & 1, abort_flag, ctl)) break;
-      int v[4] = {0, 0, 0, 0};
+      int v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       if (lane == 0) {
         for (;;) {
           const long long u = atomicAdd(a.unit_counter, 1);
@@ -616,59 +619,79 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
           const int item = static_cast<int>(u / a.H);
           const int b = a.items[2 * item], qt = a.items[2 * item + 1];
           // prefix append: a query tile wholly inside the old prefix has nothing to write
-          if (a.q_from && static_cast<long long>(unit_qt(qt) + 1) * kQTile <= a.q_from[b + 1] - a.q_from[b]) continue;
+          const long long q_lo = a.q_from ? a.q_from[b + 1] - a.q_from[b] : 0;
+          if (static_cast<long long>(unit_qt(qt) + 1) * kQTile <= q_lo) continue;
+          long long seq0;
+          int n;
+          pair_rows(a.offsets, a.pack, b, &seq0, &n);
           v[0] = b;
           v[1] = qt;
           v[2] = static_cast<int>(u - static_cast<long long>(item) * a.H);
           v[3] = 1;
+          v[4] = static_cast<int>(seq0);
+          v[5] = n;
+          v[6] = static_cast<int>(a.pair_base[b] + static_cast<long long>(unit_qt(qt)) * (unit_qt(qt) + 1) / 2);
+          v[7] = static_cast<int>(q_lo);
           break;
         }
-        ring[slot] = UnitRec{v[0], v[1], v[2], v[3]};
+        ring[slot] = UnitRec{v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]};
         mbar_arrive(u_full(slot));
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = __shfl_sync(0xffffffffu, v[i], 0);
+      for (int i = 0; i < 8; ++i) v[i] = __shfl_sync(0xffffffffu, v[i], 0);
       if (!v[3]) break;
-      const int b = v[0], qt = unit_qt(v[1]), h = v[2];
-      const int row0 = static_cast<int>(a.offsets[b]);
+      const int qt = unit_qt(v[1]), h = v[2];
+      const int row0 = v[4];
       const int nkt = unit_nkt(v[1]);
       const int qb = uc & 1;
       if (uc >= 2 && !mbar_wait_warp(q_empty(qb), ((uc >> 1) - 1) & 1, abort_flag, ctl)) break;
       if (lane == 0) mbar_arrive_expect_tx(q_full(qb), 16384);
       __syncwarp();
-      if (lane == 16 + qb) tma_load_2d(sQ + qb * 16384, &tmQ, q_full(qb), h * kD, row0 + qt * kQTile);
-      // K of step s first, V of step s - 1 after it: waiting for a V stage (freed late, by a P V MMA)
-      // never delays a K load
-      for (int kt = 0; ok && kt < nkt; ++kt) {
+      if (lane == 16 + 2 * qb || lane == 17 + 2 * qb) {
+        const int ry = lane & 1;
+        tma_load_2d(sQ + qb * 16384 + ry * 8192, &tmQ, q_full(qb), h * kD, row0 + qt * kQTile + 64 * ry);
+      }
+      for (int kt = 0; kt < nkt; ++kt) {
         const int s = sg + kt, st = s % NK;
         if (s >= NK && !mbar_wait_warp(k_empty(st), ((s / NK) - 1) & 1, abort_flag, ctl)) { ok = false; break; }
-        if (lane == st) {
-          mbar_arrive_expect_tx(k_full(st), 16384);
-          tma_load_2d(sK + st * 16384, &tmK, k_full(st), h * kD, row0 + kt * kQTile);
+        if (lane == 0) mbar_arrive_expect_tx(k_full(st), 16384);
+        __syncwarp();
+        if (lane == 2 * st || lane == 2 * st + 1) {
+          const int ry = lane & 1;
+          tma_load_2d(sK + st * 16384 + ry * 8192, &tmK, k_full(st), h * kD, row0 + kt * kQTile + 64 * ry);
         }
-        if (kt >= 1) ok = load_v(s - 1, row0 + (kt - 1) * kQTile, h);
       }
-      if (ok) ok = load_v(sg + nkt - 1, row0 + (nkt - 1) * kQTile, h);
       sg += nkt;
     }
   } else if (warp == kBiasWarp) {
-    // ---------------- bias tiles (stage bs: its two 64-column halves from lanes 2 bs, 2 bs + 1) ----
+    // ---------------- bias tiles and V (bias stage: four 8 KB boxes from lanes 4 bs .. 4 bs + 3; V
+    // stage: two from lanes 12 + 2 st, 13 + 2 st) ----------------
     int sg = 0;
     bool ok = true;
     UnitRec r;
     for (int uc = 0; ok && take_unit(uc, r) && r.valid; ++uc) {
-      const int qt = unit_qt(r.qt);
-      const long long pair0 = a.pair_base[r.b] + static_cast<long long>(qt) * (qt + 1) / 2;
+      const long long pair0 = r.pair0;
       const int nkt = unit_nkt(r.qt);
       const int hb = a.bias_heads > 1 ? r.h : 0;
+      const int row0 = r.row0;
       for (int kt = 0; kt < nkt; ++kt) {
         const int s = sg + kt, bs = s % BS;
         if (s >= BS && !mbar_wait_warp(b_empty(bs), ((s / BS) - 1) & 1, abort_flag, ctl)) { ok = false; break; }
         const int brow = static_cast<int>(((pair0 + kt) * a.bias_heads + hb) * kQTile);
         if (lane == 0) mbar_arrive_expect_tx(b_full(bs), 32768);
         __syncwarp();
-        const int hx = lane - 2 * bs;
-        if (hx == 0 || hx == 1) tma_load_2d(sB + bs * 32768 + hx * 16384, &tmB, b_full(bs), 64 * hx, brow);
+        const int part = lane - 4 * bs;   // column half part >> 1, row half part & 1
+        if (part >= 0 && part < 4)
+          tma_load_2d(sB + bs * 32768 + (part >> 1) * 16384 + (part & 1) * 8192, &tmB, b_full(bs), 64 * (part >> 1),
+                      brow + 64 * (part & 1));
+        const int st = s % NV;
+        if (s >= NV && !mbar_wait_warp(v_empty(st), ((s / NV) - 1) & 1, abort_flag, ctl)) { ok = false; break; }
+        if (lane == 0) mbar_arrive_expect_tx(v_full(st), 16384);
+        __syncwarp();
+        if (lane == 12 + 2 * st || lane == 13 + 2 * st) {
+          const int ry = lane & 1;
+          tma_load_2d(sV + st * 16384 + ry * 8192, &tmV, v_full(st), r.h * kD, row0 + kt * kQTile + 64 * ry);
+        }
       }
       sg += nkt;
     }
@@ -753,14 +776,14 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
       // first key column this row may see: its own sequence's start inside a pack, else 0
       int lo = 0;
       if (u.qt < 0) {
-        const long long g = a.offsets[u.b] + r;
+        const long long g = static_cast<long long>(u.row0) + r;
         int s0 = u.b, s1 = u.b - u.qt;   // pack members b .. b + k - 1
         while (s1 - s0 > 1) {
           const int mid = (s0 + s1) >> 1;
           if (a.offsets[mid] <= g) s0 = mid;
           else s1 = mid;
         }
-        lo = static_cast<int>(a.offsets[s0] - a.offsets[u.b]);
+        lo = static_cast<int>(a.offsets[s0] - u.row0);
       }
       for (int kt = (sg & 1) == grp ? 0 : 1; ok && kt < nkt; kt += 2) {
         const int s = sg + kt, buf = s % 3;
@@ -771,23 +794,24 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
         }
         tc_fence_after();
         const bool diag = kt == qt;
+        // four chunks of 16 keys: [64 half + 16 hc, +16)
 #pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-          uint32_t sv[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + buf * 128 + 64 * half + 32 * hc, sv);
-          uint32_t hb[16];   // half-bias of keys [64 half + 32 hc, +32)
+        for (int hc = 0; hc < 4; ++hc) {
+          uint32_t sv[16];
+          tmem_ld_32x32b_x16(tmem + lane_base + buf * 128 + 64 * half + 16 * hc, sv);
+          uint32_t hb[8];   // half-bias of these keys
           const uint8_t* brow = smem + L::kBias + buf * 32768 + half * 16384 + r * 128;
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const uint4 v = *reinterpret_cast<const uint4*>(brow + (((4 * hc + q4) ^ (r & 7)) << 4));
-            hb[4 * q4] = v.x; hb[4 * q4 + 1] = v.y; hb[4 * q4 + 2] = v.z; hb[4 * q4 + 3] = v.w;
+          for (int q2 = 0; q2 < 2; ++q2) {
+            const uint4 v = *reinterpret_cast<const uint4*>(brow + (((2 * hc + q2) ^ (r & 7)) << 4));
+            hb[4 * q2] = v.x; hb[4 * q2 + 1] = v.y; hb[4 * q2 + 2] = v.z; hb[4 * q2 + 3] = v.w;
           }
-          // the bias stage is free once both halves of this row are in registers
-          if (hc == 1) mbar_arrive(b_empty(buf));
+          // the bias stage is free once the whole row is in registers
+          if (hc == 3) mbar_arrive(b_empty(buf));
           tmem_ld_wait();
-          uint32_t p[16];
+          uint32_t p[8];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 8; ++j) {
             const uint32_t s2 = pack_f16x2(__uint_as_float(sv[2 * j]), __uint_as_float(sv[2 * j + 1]));
             const uint32_t h2 = hfma2_u32(s2, kHalf2Half, hb[j]);
             const uint32_t t2 = tanh_f16x2(h2);
@@ -797,15 +821,15 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
               y2 = pack_bf16x2(f.x, f.y);
             }
             if (diag) {   // keys lo <= col <= r
-              const int col = 64 * half + 32 * hc + 2 * j;
+              const int col = 64 * half + 16 * hc + 2 * j;
               const uint32_t m = ((col <= r && col >= lo) ? 0x0000FFFFu : 0u) |
                                  ((col + 1 <= r && col + 1 >= lo) ? 0xFFFF0000u : 0u);
               y2 &= m;
             }
             p[j] = y2;
           }
-          // P of these 32 keys packed into 16 columns over S chunk 0 (already read)
-          tmem_st_32x32b_x16(tmem + lane_base + buf * 128 + 64 * half + 16 * hc, p);
+          // P of these 16 keys packed into 8 columns over S columns already read
+          tmem_st_32x32b_x8(tmem + lane_base + buf * 128 + 64 * half + 8 * hc, p);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -819,35 +843,38 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
           ok = false;
         } else {
           tc_fence_after();
-          uint32_t ov[32];
-          tmem_ld_32x32b_x32(tmem + lane_base + kOCol + 64 * ob + 32 * half, ov);
-          tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(o_empty(ob));
-          long long seq0;
-          int n;
-          pair_rows(a.offsets, a.pack, u.b, &seq0, &n);   // a pack's rows, or sequence b's
           const int qi = qt * kQTile + r;
-          const long long q_lo = a.q_from ? a.q_from[u.b + 1] - a.q_from[u.b] : 0;
-          if (qi < n && qi >= q_lo) {
-            const float sc = a.inv_N;
-            const long long orow = seq0 + qi;
-            const int ocol = u.h * kD + 32 * half;
-            if (a.o_f32) {
-              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + orow * a.ld_o + ocol);
+          const bool row_ok = qi < u.n && qi >= u.q_lo;
+          const float sc = a.inv_N;
+          const long long orow = static_cast<long long>(u.row0) + qi;
+          // columns [32 half + 16 c, +16) of the head, two chunks
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t ov[16];
+            tmem_ld_32x32b_x16(tmem + lane_base + kOCol + 64 * ob + 32 * half + 16 * c, ov);
+            tmem_ld_wait();
+            if (c == 1) {
+              tc_fence_before();
+              mbar_arrive(o_empty(ob));
+            }
+            if (row_ok) {
+              const int ocol = u.h * kD + 32 * half + 16 * c;
+              if (a.o_f32) {
+                float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + orow * a.ld_o + ocol);
 #pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dst[q] = make_float4(__uint_as_float(ov[4 * q]) * sc, __uint_as_float(ov[4 * q + 1]) * sc,
-                                     __uint_as_float(ov[4 * q + 2]) * sc, __uint_as_float(ov[4 * q + 3]) * sc);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + orow * a.ld_o + ocol);
+                for (int q = 0; q < 4; ++q)
+                  dst[q] = make_float4(__uint_as_float(ov[4 * q]) * sc, __uint_as_float(ov[4 * q + 1]) * sc,
+                                       __uint_as_float(ov[4 * q + 2]) * sc, __uint_as_float(ov[4 * q + 3]) * sc);
+              } else {
+                uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.o) + orow * a.ld_o + ocol);
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-                dst[q] = make_uint4(
-                    pack_bf16x2(__uint_as_float(ov[8 * q]) * sc, __uint_as_float(ov[8 * q + 1]) * sc),
-                    pack_bf16x2(__uint_as_float(ov[8 * q + 2]) * sc, __uint_as_float(ov[8 * q + 3]) * sc),
-                    pack_bf16x2(__uint_as_float(ov[8 * q + 4]) * sc, __uint_as_float(ov[8 * q + 5]) * sc),
-                    pack_bf16x2(__uint_as_float(ov[8 * q + 6]) * sc, __uint_as_float(ov[8 * q + 7]) * sc));
+                for (int q = 0; q < 2; ++q)
+                  dst[q] = make_uint4(
+                      pack_bf16x2(__uint_as_float(ov[8 * q]) * sc, __uint_as_float(ov[8 * q + 1]) * sc),
+                      pack_bf16x2(__uint_as_float(ov[8 * q + 2]) * sc, __uint_as_float(ov[8 * q + 3]) * sc),
+                      pack_bf16x2(__uint_as_float(ov[8 * q + 4]) * sc, __uint_as_float(ov[8 * q + 5]) * sc),
+                      pack_bf16x2(__uint_as_float(ov[8 * q + 6]) * sc, __uint_as_float(ov[8 * q + 7]) * sc));
+              }
             }
           }
         }
@@ -872,7 +899,7 @@ falcon_key_bias_kernel(const int64_t* __restrict__ off, const int64_t* __restric
                        const float* __restrict__ rab_pos, const float* __restrict__ rab_time, int L, int nb,
                        uint16_t* kbias, int64_t ld, float* self_bias, int* status) {
   __shared__ long long s_tau[kTauEntries];
-  for (int e = threadIdx.x; e < kTauEntries; e += blockDim.x) s_tau[e] = c_time_taus[e];
+  for (int e = threadIdx.x; e < kTauEntries; e += blockDim.x) s_tau[e] = g_time_taus[e];
   __syncthreads();
   const int u = blockIdx.y;
   if (u == 0 && blockIdx.x == 0 && threadIdx.x == 0) *self_bias = rab_pos[L - 1] + rab_time[0];
@@ -959,9 +986,17 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
       !encode_tmap_2d_bf16(&tv, a.v, static_cast<int64_t>(a.H) * kD, a.T, a.ld_v, 64, 128, f16) ||
       !encode_tmap_2d_bf16(&tb, a.bias, kQTile, a.max_pairs * a.bias_heads * kQTile, kQTile, 64, 128, true))
     return cudaErrorInvalidValue;
-  // the persistent kernel's unit counter lives in the workspace header (reset by the work list)
+  // the persistent kernel's unit counter lives in the workspace header (reset by the work list); it
+  // loads every tile as 64-row boxes
   if (!a.unit_counter) return cudaErrorInvalidValue;
-  return f16 ? launch_attn_persistent<true>(tq, tk, tv, tb, a, st) : launch_attn_persistent<false>(tq, tk, tv, tb, a, st);
+  CUtensorMap pq, pk, pv, pb;
+  if (!encode_tmap_2d_bf16(&pq, a.q, static_cast<int64_t>(a.H) * kD, a.T, a.ld_q, 64, 64, f16) ||
+      !encode_tmap_2d_bf16(&pk, a.k, static_cast<int64_t>(a.H) * kD, a.T, a.ld_k, 64, 64, f16) ||
+      !encode_tmap_2d_bf16(&pv, a.v, static_cast<int64_t>(a.H) * kD, a.T, a.ld_v, 64, 64, f16) ||
+      !encode_tmap_2d_bf16(&pb, a.bias, kQTile, a.max_pairs * a.bias_heads * kQTile, kQTile, 64, 64, true))
+    return cudaErrorInvalidValue;
+  (void)tq; (void)tk; (void)tv; (void)tb;
+  return f16 ? launch_attn_persistent<true>(pq, pk, pv, pb, a, st) : launch_attn_persistent<false>(pq, pk, pv, pb, a, st);
 }
 
 cudaError_t falcon_key_bias(const int64_t* offsets, const int64_t* ts, int users, int max_len,

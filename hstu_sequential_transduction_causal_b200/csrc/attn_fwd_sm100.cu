@@ -104,7 +104,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     fence_barrier_init();
   }
   for (int e = tid; e < a.n_buckets && e < 128; e += kThreads) s_rab_time[e] = a.rab_time[e];
-  for (int e = tid; e < kTauEntries; e += kThreads) s_tau[e] = c_time_taus[e];
+  for (int e = tid; e < kTauEntries; e += kThreads) s_tau[e] = g_time_taus[e];
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);

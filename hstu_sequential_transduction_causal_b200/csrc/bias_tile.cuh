@@ -139,8 +139,8 @@ __device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pai
     if (tid < nt * nt) s_tt[tid] = 0.5f * a.rab_type[static_cast<long long>(hb) * nt * nt + tid];
   }
   for (int e = tid; e < kTauEntries; e += kBiasThreads) {
-    s_tau[e] = c_time_taus[e];
-    s_tau32[e] = c_time_taus32[e];
+    s_tau[e] = g_time_taus[e];
+    s_tau32[e] = g_time_taus32[e];
   }
   __syncthreads();
   const bool fast = tile_times_finish(s_t);

@@ -303,8 +303,8 @@ time_bucket_tile_kernel(const int64_t* __restrict__ off, const int64_t* __restri
   if (static_cast<long long>(qt) * kQTile >= n || static_cast<long long>(kt) * kQTile >= n) return;
   tile_times_load(s_t, ts, seq0, static_cast<int>(n), qt * kQTile, kt * kQTile);
   for (int e = threadIdx.x; e < kTauEntries; e += kBiasThreads) {
-    s_tau[e] = c_time_taus[e];
-    s_tau32[e] = c_time_taus32[e];
+    s_tau[e] = g_time_taus[e];
+    s_tau32[e] = g_time_taus32[e];
   }
   __syncthreads();
   const bool fast = tile_times_finish(s_t);

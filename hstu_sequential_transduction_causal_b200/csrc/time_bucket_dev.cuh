@@ -55,7 +55,13 @@ __device__ __forceinline__ int time_bucket32(int dt, const int* tau, int nb) {
   return min(k, nb - 1);
 }
 
-// Copies tau_0..tau_128 to this translation unit's constant bank, once per device. The copies are
+// The same tables in global memory, for kernels that stage them into shared memory: a warp reads 32
+// consecutive entries in one request, where reads of different constant-bank entries by the lanes of
+// a warp are serialised (and, on an SM's first touch, each one misses the constant cache).
+__device__ long long g_time_taus[kTauEntries];
+__device__ int g_time_taus32[kTauEntries];
+
+// Copies tau_0..tau_128 to this translation unit's constant bank and global mirrors, once per device. The copies are
 // synchronous, so the first call on a device must come before any stream capture. Safe to call from
 // several host threads: the upload is serialised and later calls only read a flag.
 inline cudaError_t upload_time_taus() {
@@ -77,6 +83,8 @@ inline cudaError_t upload_time_taus() {
   for (int k = 0; k < kTauEntries; ++k)
     taus32[k] = k == 0 ? (-0x7fffffff - 1) : (taus[k] > 0x7fffffffLL ? 0x7fffffff : static_cast<int>(taus[k]));
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(c_time_taus32, taus32, sizeof(taus32));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_time_taus, taus, sizeof(taus));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_time_taus32, taus32, sizeof(taus32));
   if (e == cudaSuccess && tracked) done[dev].store(true, std::memory_order_release);
   return e;
 }
