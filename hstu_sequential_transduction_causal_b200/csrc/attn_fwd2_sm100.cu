@@ -501,7 +501,8 @@ __global__ void __launch_bounds__(kThreads3, 1)
 attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB,
                            AttnArgs a, WaitCtl ctl) {
-  pdl_enter();
+  // set-up below reads nothing an earlier grid writes: it overlaps that grid's tail
+  pdl_trigger();
   using L = Smem3;
   constexpr int NK = L::kNK, NV = L::kNV, BS = L::kBS;
   static_assert(NK == 3 && NV == 3 && BS == 3, "the rings share the step index modulo 3");
@@ -578,6 +579,7 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   // S / P tiles of steps s = 0, 1, 2 (mod 3) at columns [128 (s % 3), +128); O of units 0, 1 (mod 2) at
   // [384 + 64 (u % 2), +64)
   const uint32_t tmem = *tmem_slot;
@@ -605,7 +607,17 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
 
   if (warp == kTmaWarp) {
     // ---------------- scheduler + Q / K producer ----------------
-    const long long total = static_cast<long long>(*a.count) * a.H;
+    // Units u = item * H + h in work-list order: CTA x starts with unit x, later ones come from the
+    // counter (offset by the grid size). One 32-byte record per item (written by the work list)
+    // describes the unit; the first record is read together with the item count.
+    long long total = 0;
+    int4 first0 = make_int4(0, 0, 0, 0), first1 = first0;
+    if (lane == 0) {
+      const int4* rec = reinterpret_cast<const int4*>(a.urec) + 2 * (blockIdx.x / a.H);
+      first0 = rec[0];
+      first1 = rec[1];
+      total = static_cast<long long>(*a.count) * a.H;
+    }
     int sg = 0;
     bool ok = true;
     for (int uc = 0; ok; ++uc) {
@@ -613,24 +625,28 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
       if (uc >= 2 && !mbar_wait_warp(u_empty(slot), ((uc >> 1) - 1) & 1, abort_flag, ctl)) break;
       int v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       if (lane == 0) {
-        for (;;) {
-          const long long u = atomicAdd(a.unit_counter, 1);
+        for (bool first = uc == 0;; first = false) {
+          const long long u = first ? static_cast<long long>(blockIdx.x)
+                                    : static_cast<long long>(gridDim.x) + atomicAdd(a.unit_counter, 1);
           if (u >= total) break;
           const int item = static_cast<int>(u / a.H);
-          const int b = a.items[2 * item], qt = a.items[2 * item + 1];
+          int4 r0 = first0, r1 = first1;
+          if (!first) {
+            const int4* rec = reinterpret_cast<const int4*>(a.urec) + 2 * item;
+            r0 = rec[0];
+            r1 = rec[1];
+          }
+          const int b = r0.x, qt = r0.y;
           // prefix append: a query tile wholly inside the old prefix has nothing to write
           const long long q_lo = a.q_from ? a.q_from[b + 1] - a.q_from[b] : 0;
           if (static_cast<long long>(unit_qt(qt) + 1) * kQTile <= q_lo) continue;
-          long long seq0;
-          int n;
-          pair_rows(a.offsets, a.pack, b, &seq0, &n);
           v[0] = b;
           v[1] = qt;
           v[2] = static_cast<int>(u - static_cast<long long>(item) * a.H);
           v[3] = 1;
-          v[4] = static_cast<int>(seq0);
-          v[5] = n;
-          v[6] = static_cast<int>(a.pair_base[b] + static_cast<long long>(unit_qt(qt)) * (unit_qt(qt) + 1) / 2);
+          v[4] = r0.z;
+          v[5] = r0.w;
+          v[6] = r1.x;
           v[7] = static_cast<int>(q_lo);
           break;
         }
@@ -767,6 +783,8 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
     const int quad = warp & 3;
     const int half = (warp >> 2) & 1;    // keys [64 half, 64 half + 64)
     const int r = quad * 32 + lane;      // query row within the tile == TMEM lane
+    // fp32 output rows written as 32-byte stores when the base and the row stride allow them
+    const bool o_v8 = ((reinterpret_cast<uintptr_t>(a.o) | static_cast<uintptr_t>(a.ld_o * 4)) & 31) == 0;
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     int sg = 0;
     bool ok = true;
@@ -859,7 +877,16 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
             }
             if (row_ok) {
               const int ocol = u.h * kD + 32 * half + 16 * c;
-              if (a.o_f32) {
+              if (a.o_f32 && o_v8) {
+                float* dst = reinterpret_cast<float*>(a.o) + orow * a.ld_o + ocol;
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                  float f[8];
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * q + e]) * sc;
+                  st_global_v8(dst + 8 * q, f);
+                }
+              } else if (a.o_f32) {
                 float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.o) + orow * a.ld_o + ocol);
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -979,23 +1006,16 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
   e = launch_pdl(attn_bias_kernel, dim3(static_cast<unsigned>(a.max_pairs), 4, static_cast<unsigned>(a.bias_heads)),
                  dim3(kBiasThreads), 0, st, a);
   if (e != cudaSuccess) return e;
-  CUtensorMap tq, tk, tv, tb;
   const bool f16 = a.in_f16 != 0;
-  if (!encode_tmap_2d_bf16(&tq, a.q, static_cast<int64_t>(a.H) * kD, a.T, a.ld_q, 64, 128, f16) ||
-      !encode_tmap_2d_bf16(&tk, a.k, static_cast<int64_t>(a.H) * kD, a.T, a.ld_k, 64, 128, f16) ||
-      !encode_tmap_2d_bf16(&tv, a.v, static_cast<int64_t>(a.H) * kD, a.T, a.ld_v, 64, 128, f16) ||
-      !encode_tmap_2d_bf16(&tb, a.bias, kQTile, a.max_pairs * a.bias_heads * kQTile, kQTile, 64, 128, true))
-    return cudaErrorInvalidValue;
-  // the persistent kernel's unit counter lives in the workspace header (reset by the work list); it
-  // loads every tile as 64-row boxes
-  if (!a.unit_counter) return cudaErrorInvalidValue;
+  // the persistent kernel's unit counter lives in the workspace header (reset by the work list), its
+  // unit records next to the work list; it loads every tile as 64-row boxes
+  if (!a.unit_counter || !a.urec) return cudaErrorInvalidValue;
   CUtensorMap pq, pk, pv, pb;
   if (!encode_tmap_2d_bf16(&pq, a.q, static_cast<int64_t>(a.H) * kD, a.T, a.ld_q, 64, 64, f16) ||
       !encode_tmap_2d_bf16(&pk, a.k, static_cast<int64_t>(a.H) * kD, a.T, a.ld_k, 64, 64, f16) ||
       !encode_tmap_2d_bf16(&pv, a.v, static_cast<int64_t>(a.H) * kD, a.T, a.ld_v, 64, 64, f16) ||
       !encode_tmap_2d_bf16(&pb, a.bias, kQTile, a.max_pairs * a.bias_heads * kQTile, kQTile, 64, 64, true))
     return cudaErrorInvalidValue;
-  (void)tq; (void)tk; (void)tv; (void)tb;
   return f16 ? launch_attn_persistent<true>(pq, pk, pv, pb, a, st) : launch_attn_persistent<false>(pq, pk, pv, pb, a, st);
 }
 

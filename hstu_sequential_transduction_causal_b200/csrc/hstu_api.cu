@@ -60,7 +60,7 @@ int64_t capacity_of(const hstu_jagged_t* j) { return static_cast<int64_t>(j->B) 
 // pair_base (int64 x (B+1)) | pack (int32 x B: short sequences sharing a tile) | fp16 bias tiles
 // (32 KB per causal tile pair and bias slice, 1024-aligned)
 struct AttnWs {
-  size_t items, pairs, pack, bias, items_end, total;
+  size_t items, pairs, pack, urec, bias, items_end, total;
   int64_t max_pairs;
 };
 
@@ -72,7 +72,8 @@ AttnWs attn_ws_layout(const hstu_jagged_t* j, int hb = 1) {
   w.items_end = w.items + align_up(static_cast<size_t>(cap) * 8, 256);
   w.pairs = w.items_end;
   w.pack = w.pairs + align_up(static_cast<size_t>(j->B + 1) * 8, 256);
-  w.bias = align_up(w.pack + align_up(static_cast<size_t>(j->B) * 4, 256), 1024);
+  w.urec = w.pack + align_up(static_cast<size_t>(j->B) * 4, 256);
+  w.bias = align_up(w.urec + static_cast<size_t>(cap) * 32, 1024);
   w.max_pairs = attn_max_pairs(cap, j->max_len);
   w.total = w.bias + static_cast<size_t>(w.max_pairs) * hb * kQTile * kQTile * 2;
   return w;
@@ -253,12 +254,14 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
     a.bias = w + lay.bias;
     a.max_pairs = lay.max_pairs;
     a.unit_counter = count + 4;   // [272, 276) of the workspace header region
+    a.urec = reinterpret_cast<const int32_t*>(w + lay.urec);
     // short sequences share tiles, except in a prefix append (whose rows start mid-sequence)
     if (!q_from) a.pack = reinterpret_cast<const int32_t*>(w + lay.pack);
   }
   cudaError_t e = launch_worklist(j->offsets, j->B, j->T, j->max_len, items, count, a.status, st,
                                   pairs ? reinterpret_cast<long long*>(w + lay.pairs) : nullptr, nullptr, nullptr,
-                                  pairs ? a.unit_counter : nullptr, const_cast<int32_t*>(a.pack));
+                                  pairs ? a.unit_counter : nullptr, const_cast<int32_t*>(a.pack),
+                                  const_cast<int32_t*>(a.urec));
   if (e != cudaSuccess) return cuda_status(e);
   if (j->T == 0) return HSTU_OK;
   if (!is_tc_dtype(d->dtype)) e = attn_fwd_f32_simt(a, st);

@@ -108,11 +108,13 @@ cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
 // key tile that visits t + 1 query tiles sits where the forward list has query tile t. With sched,
 // sched[0] (the persistent attention kernel's unit counter) is reset to 0. With pack (int32 [B]),
 // runs of short sequences share a tile: pack[b] = k >= 2 marks the first of k packed sequences
-// (one item (b, -k) in both lists), 0 the other members, 1 a sequence on its own.
+// (one item (b, -k) in both lists), 0 the other members, 1 a sequence on its own. With urec (needs
+// pair_base; int32 [capacity, 8], 16-byte aligned), the persistent attention forward's record of
+// each item: {b, tile, first row, rows, first causal pair of the query tile, 0, 0, 0}.
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
                             int32_t* count, int* status, cudaStream_t st, long long* pair_base = nullptr,
                             int32_t* kitems = nullptr, int32_t* kcount = nullptr, int32_t* sched = nullptr,
-                            int32_t* pack = nullptr);
+                            int32_t* pack = nullptr, int32_t* urec = nullptr);
 // The n_b x n_b time-bucket matrices of the test surface, tile by tile with the bias tiles' code.
 cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int max_len,
                                 int n_buckets, const int64_t* sq_offsets, uint8_t* out, cudaStream_t st);
@@ -155,6 +157,7 @@ struct AttnArgs {
   int64_t kbias_ld;             // multiple of 128 >= every prefix length
   const float* self_bias;       // device: rab_pos[idx(0)] + rab_time[bucket(0)]
   int32_t* unit_counter;        // persistent forward: next (work item, head) unit, reset by the work list
+  const int32_t* urec;          // persistent forward: per-item unit records (launch_worklist's urec)
   // the richer bias (hstu_rab_ext_t): bias_heads tiles per causal pair (1: tables shared by the heads,
   // H: one slice per head, rab_pos / rab_time / rab_type indexed by head first); n_types > 0 adds
   // rab_type[type_i][type_j]

@@ -44,6 +44,28 @@ __device__ void pack_chunk(const int64_t* __restrict__ off, int b0, int b1, int3
   }
 }
 
+// Unit records of the persistent attention forward, one per work item p: {b, tile, row0, n, pair0,
+// 0, 0, 0} (int32): the item, the first row and row count its tiles cover (a pack's rows for a pack),
+// and the index of its query tile's first causal pair. Run by threads [tid, tid + nthreads) after
+// items, count and pair_base are written and visible to them.
+__device__ void write_unit_records(const int64_t* __restrict__ off, const int32_t* items, int count,
+                                   const long long* pair_base, int32_t* urec, int tid, int nthreads) {
+  for (int p = tid; p < count; p += nthreads) {
+    const int b = items[2 * p], t = items[2 * p + 1];
+    const int k = t < 0 ? -t : 1;
+    const int qt = t < 0 ? 0 : t;
+    int4 r0, r1;
+    r0.x = b;
+    r0.y = t;
+    r0.z = static_cast<int>(off[b]);
+    r0.w = static_cast<int>(off[b + k] - off[b]);
+    r1.x = static_cast<int>(pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2);
+    r1.y = r1.z = r1.w = 0;
+    reinterpret_cast<int4*>(urec)[2 * p] = r0;
+    reinterpret_cast<int4*>(urec)[2 * p + 1] = r1;
+  }
+}
+
 // ----------------------------------------------------------------------------------------------
 // Jagged tile work list ("4.4 Scaling Recommendation Models", Efficiency tricks: kernels over
 // variable-length sequences). One block: emits (b, t) for every query tile t of every sequence,
@@ -55,7 +77,7 @@ __device__ void pack_chunk(const int64_t* __restrict__ off, int b0, int b1, int3
 __global__ void __launch_bounds__(1024)
 worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items,
                 int32_t* count, int* status, long long* pair_base, int32_t* kitems, int32_t* kcount,
-                int32_t* sched, int32_t* pack) {
+                int32_t* sched, int32_t* pack, int32_t* urec) {
   pdl_enter();
   if (sched && threadIdx.x == 0) sched[0] = 0;   // the persistent attention's unit counter
   __shared__ int s_warp[32];
@@ -217,6 +239,9 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
     __syncthreads();
   }
   if (tid == 0) pair_base[B] = s_run;
+  if (!urec) return;
+  __syncthreads();
+  write_unit_records(off, items, s_base, pair_base, urec, tid, blockDim.x);
 }
 
 // The same lists for batches of at most 32 sequences, from a single warp (no block barriers):
@@ -224,7 +249,7 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
 __global__ void __launch_bounds__(32)
 worklist_warp_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items, int32_t* count,
                      int* status, long long* pair_base, int32_t* kitems, int32_t* kcount, int32_t* sched,
-                     int32_t* pack) {
+                     int32_t* pack, int32_t* urec) {
   pdl_enter();
   if (sched && threadIdx.x == 0) sched[0] = 0;   // the persistent attention's unit counter
   const int lane = threadIdx.x;
@@ -283,6 +308,9 @@ worklist_warp_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_
   if (mine) pair_base[lane] = inc - v;
   const long long total = __shfl_sync(0xffffffffu, inc, 31);
   if (lane == 0) pair_base[B] = total;
+  if (!urec) return;
+  __syncwarp();
+  write_unit_records(off, items, base, pair_base, urec, lane, 32);
 }
 
 // Test surface of the attention's time-bucket index: block (x = qt * mt + kt, y = b) writes
@@ -418,12 +446,13 @@ cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int
 
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
                             int32_t* count, int* status, cudaStream_t st, long long* pair_base, int32_t* kitems,
-                            int32_t* kcount, int32_t* sched, int32_t* pack) {
+                            int32_t* kcount, int32_t* sched, int32_t* pack, int32_t* urec) {
+  if (urec && !pair_base) return cudaErrorInvalidValue;
   if (B >= 0 && B <= 32)
     return launch_pdl(worklist_warp_kernel, dim3(1), dim3(32), 0, st, offsets, B, T, max_len, items, count, status,
-                      pair_base, kitems, kcount, sched, pack);
+                      pair_base, kitems, kcount, sched, pack, urec);
   return launch_pdl(worklist_kernel, dim3(1), dim3(1024), 0, st, offsets, B, T, max_len, items, count, status,
-                    pair_base, kitems, kcount, sched, pack);
+                    pair_base, kitems, kcount, sched, pack, urec);
 }
 
 cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int max_len,

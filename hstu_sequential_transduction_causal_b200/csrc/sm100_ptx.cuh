@@ -112,6 +112,18 @@ __device__ __forceinline__ void pdl_enter() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// One 32-byte store of eight floats (dst 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(float* dst, const float (&f)[8]) {
+  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "f"(f[0]), "f"(f[1]),
+               "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]), "f"(f[7])
+               : "memory");
+}
+
+// The two halves of pdl_enter, for a kernel whose set-up (barriers, tensor memory, descriptor
+// prefetch) touches nothing an earlier grid writes and can overlap that grid's tail.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------------------------------------
 // Proxy fences, named barriers
 // ------------------------------------------------------------------------------------------------
