@@ -395,6 +395,9 @@ cudaError_t ensure_smem_attr(const void* kernel, int bytes) {
   for (int i = 0; i < n_done; ++i)
     if (done[i] == kernel && done_dev[i] == dev) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  // the whole unified L1 / shared array as shared memory, so that the blocks per SM the kernel was
+  // sized for (two 96 KB blocks for the staged LayerNorm kernels) are resident together
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e == cudaSuccess && n_done < 256) {
     done[n_done] = kernel;
     done_dev[n_done] = dev;
@@ -754,7 +757,7 @@ hstu_status_t run_layer_fwd(const hstu_layer_desc_t* desc, hstu_dtype_t resid_dt
   // G in fp16 (BF16 mode): f2 then reads an fp16 copy of W2
   const hstu_dtype_t g_dt = desc->dtype == HSTU_BF16 ? HSTU_F16 : HSTU_F32;
   cudaError_t e = norm_gate_fwd(T, D, kDtF32, act, g_dt, saved->o, D, uvqk, 4ll * D, w->gamma, w->beta,
-                                desc->ln_eps, saved->g, saved->mu, saved->rstd, st);
+                                desc->ln_eps, saved->g, saved->mu, saved->rstd, st, status);
   if (e != cudaSuccess) return cuda_status(e);
   return run_out_proj(T, D, desc->dtype, g_dt, saved->g, w->W2, w->b2, x, resid_dtype, y, desc->y_dtype, y_f16,
                       status, st, wsb + lay.w2_f16);
@@ -913,7 +916,7 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   // 2. norm-gate backward: dO (fp16), dZ_U (bf16), dgamma | dbeta
   if (e == cudaSuccess)
     e = norm_gate_bwd(T, D, kDtF16, dG, static_cast<const float*>(saved->o), saved->uvqk, saved->z, 4ll * D, w->gamma,
-                      w->beta, saved->mu, saved->rstd, dO, dz, 4ll * D, part, gb, st);
+                      w->beta, saved->mu, saved->rstd, dO, dz, 4ll * D, part, gb, st, status);
   if (e == cudaSuccess) e = cudaMemcpyAsync(gr->dgamma, gb, sizeof(float) * D, cudaMemcpyDeviceToDevice, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(gr->dbeta, gb + D, sizeof(float) * D, cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return cuda_status(e);

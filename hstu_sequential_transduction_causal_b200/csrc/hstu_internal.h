@@ -95,6 +95,8 @@ bool encode_tmap_2d_u8(CUtensorMap* map, const void* base, int64_t inner, int64_
 
 // Sets a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t ensure_smem_attr(const void* kernel, int bytes);
+// Multiprocessors of the current device (cached per device; 148 when the query fails).
+int sm_count();
 
 cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st);
 cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
@@ -214,9 +216,10 @@ cudaError_t falcon_append_gather(const int64_t* old_off, const int64_t* app_off,
 // LayerNorm (.) U
 // ---------------------------------------------------------------------------------------------
 // o_dt: f32 or bf16; u_dt: any; g_dt: any (kDt* codes). g has row stride D.
+// status (device, optional): where a bounded wait of the staged kernel records a timeout.
 cudaError_t norm_gate_fwd(int64_t T, int D, int o_dt, int u_dt, int g_dt, const void* o, int64_t ld_o,
                           const void* u, int64_t ld_u, const float* gamma, const float* beta,
-                          float eps, void* g, float* mu, float* rstd, cudaStream_t st);
+                          float eps, void* g, float* mu, float* rstd, cudaStream_t st, int* status = nullptr);
 
 cudaError_t convert_f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t st);
 
@@ -229,7 +232,7 @@ int norm_gate_bwd_blocks(int64_t T);
 cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const float* o, const void* u,
                           const void* zu, int64_t ld_act, const float* gamma, const float* beta, const float* mu,
                           const float* rstd, void* d_o, void* dz, int64_t ld_dz, float* partial,
-                          float* dgamma_dbeta_out, cudaStream_t st);
+                          float* dgamma_dbeta_out, cudaStream_t st, int* status = nullptr);
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
                         const void* z, int64_t ld_z, void* dz, int64_t ld_dz, cudaStream_t st);
 size_t colsum_partial_floats(int cols);

@@ -352,12 +352,19 @@ time_bucket_tile_kernel(const int64_t* __restrict__ off, const int64_t* __restri
 // backward.
 // ----------------------------------------------------------------------------------------------
 template <int VPT, int OT, int UT, int GT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, VPT <= 16 ? 4 : 2)
 norm_gate_kernel(int64_t T, const void* __restrict__ o, int64_t ld_o, const void* __restrict__ u,
                  int64_t ld_u, const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
                  void* __restrict__ g, float* __restrict__ mu_out, float* __restrict__ rstd_out) {
-  pdl_enter();
   constexpr int D = VPT * 32;
+  // gamma | beta staged once per block (they are parameters, not written by an earlier grid)
+  __shared__ __align__(16) float s_gb[2 * D];
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    s_gb[c] = gamma[c];
+    s_gb[D + c] = beta[c];
+  }
+  pdl_enter();
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= T) return;
@@ -387,19 +394,113 @@ norm_gate_kernel(int64_t T, const void* __restrict__ o, int64_t ld_o, const void
 #pragma unroll
   for (int m = 16; m > 0; m >>= 1) q += __shfl_xor_sync(0xffffffffu, q, m);
   const float rstd = rsqrtf(q * (1.0f / D) + eps);
-  float gm[VPT], bt[VPT];
 #pragma unroll
   for (int k = 0; k < KG; ++k) {
-    load_vec<W, kDtF32>(gamma, col(k), gm + W * k);
-    load_vec<W, kDtF32>(beta, col(k), bt + W * k);
-  }
+    float gm[W], bt[W];
+    load_vec<W, kDtF32>(s_gb, col(k), gm);
+    load_vec<W, kDtF32>(s_gb + D, col(k), bt);
 #pragma unroll
-  for (int e = 0; e < VPT; ++e) x[e] = fmaf((x[e] - mean) * rstd, gm[e], bt[e]) * uu[e];
+    for (int e = 0; e < W; ++e) x[W * k + e] = fmaf((x[W * k + e] - mean) * rstd, gm[e], bt[e]) * uu[W * k + e];
+  }
 #pragma unroll
   for (int k = 0; k < KG; ++k) store_vec<W, GT>(g, row * D + col(k), x + W * k);
   if (lane == 0) {
     if (mu_out) mu_out[row] = mean;
     if (rstd_out) rstd_out[row] = rstd;
+  }
+}
+
+// Bytes of one element of a kDt* type in memory (kDtOne: none).
+__host__ __device__ constexpr int dt_bytes(int dt) { return dt == kDtF32 ? 4 : (dt == kDtOne ? 0 : 2); }
+
+// Row slots per warp of the staged kernel below.
+constexpr int kNgSlots = 4;
+
+// The same LayerNorm (.) U for D >= 128 with the rows staged by bulk copies: a persistent grid whose
+// warps each own kNgSlots row slots in shared memory (O row, then U row) and rows gw, gw + W, ...
+// (gw = the warp's global index, W = all warps); lane 0 keeps kNgSlots rows in flight, refilling a
+// slot as soon as the warp has read it, so the whole batch is requested at the speed the copy
+// engines take it instead of one round trip per warp. Every wait is bounded (ctl).
+template <int VPT, int OT, int UT, int GT>
+__global__ void __launch_bounds__(256)
+norm_gate_staged_kernel(int64_t T, const void* __restrict__ o, int64_t ld_o, const void* __restrict__ u,
+                        int64_t ld_u, const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
+                        void* __restrict__ g, float* __restrict__ mu_out, float* __restrict__ rstd_out, WaitCtl ctl) {
+  constexpr int D = VPT * 32, KG = VPT / 4;
+  constexpr int OB = D * dt_bytes(OT), UB = D * dt_bytes(UT), SLOT = OB + UB, S = kNgSlots;
+  static_assert(VPT % 4 == 0 && OB % 16 == 0 && UB % 16 == 0, "rows of whole 16-byte chunks");
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint64_t s_bar[8 * S];
+  __shared__ int s_abort;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 8 * S; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  float gm[VPT], bt[VPT];   // parameters: read before the wait for the earlier grid
+#pragma unroll
+  for (int k = 0; k < KG; ++k) {
+    load_vec<4, kDtF32>(gamma, 128 * k + 4 * lane, gm + 4 * k);
+    load_vec<4, kDtF32>(beta, 128 * k + 4 * lane, bt + 4 * k);
+  }
+  pdl_enter();
+  __syncthreads();
+  const long long W = static_cast<long long>(gridDim.x) * 8, gw = static_cast<long long>(blockIdx.x) * 8 + warp;
+  uint8_t* wslots = smem + static_cast<size_t>(warp) * S * SLOT;
+  auto issue = [&](long long i) {   // lane 0: row i of this warp into slot i % S
+    const long long row = gw + i * W;
+    if (row >= T) return;
+    const int sl = static_cast<int>(i % S);
+    const uint32_t bar = smem_u32(&s_bar[warp * S + sl]);
+    mbar_arrive_expect_tx(bar, SLOT);
+    bulk_load(smem_u32(wslots + sl * SLOT), static_cast<const uint8_t*>(o) + row * ld_o * dt_bytes(OT), OB, bar);
+    if constexpr (UB > 0)
+      bulk_load(smem_u32(wslots + sl * SLOT + OB), static_cast<const uint8_t*>(u) + row * ld_u * dt_bytes(UT), UB, bar);
+  };
+  if (lane == 0)
+    for (int i = 0; i < S; ++i) issue(i);
+  for (long long i = 0;; ++i) {
+    const long long row = gw + i * W;
+    if (row >= T) break;
+    const int sl = static_cast<int>(i % S);
+    if (!mbar_wait_warp(smem_u32(&s_bar[warp * S + sl]), static_cast<uint32_t>((i / S) & 1), &s_abort, ctl)) break;
+    const uint8_t* so = wslots + sl * SLOT;
+    float x[VPT], uu[VPT];
+#pragma unroll
+    for (int k = 0; k < KG; ++k) {
+      load_vec<4, OT>(so, 128 * k + 4 * lane, x + 4 * k);
+      load_vec<4, UT>(so + OB, 128 * k + 4 * lane, uu + 4 * k);
+    }
+    // every lane has read the slot: refill it (generic reads before the copy engine's writes)
+    __syncwarp();
+    if (lane == 0) {
+      fence_proxy_async_smem();
+      issue(i + S);
+    }
+    float s = 0.0f;
+#pragma unroll
+    for (int e = 0; e < VPT; ++e) s += x[e];
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+    const float mean = s * (1.0f / D);
+    float q = 0.0f;
+#pragma unroll
+    for (int e = 0; e < VPT; ++e) {
+      const float d = x[e] - mean;
+      q = fmaf(d, d, q);
+    }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) q += __shfl_xor_sync(0xffffffffu, q, m);
+    const float rstd = rsqrtf(q * (1.0f / D) + eps);
+#pragma unroll
+    for (int e = 0; e < VPT; ++e) x[e] = fmaf((x[e] - mean) * rstd, gm[e], bt[e]) * uu[e];
+#pragma unroll
+    for (int k = 0; k < KG; ++k) store_vec<4, GT>(g, row * D + 128 * k + 4 * lane, x + 4 * k);
+    if (lane == 0) {
+      if (mu_out) mu_out[row] = mean;
+      if (rstd_out) rstd_out[row] = rstd;
+    }
   }
 }
 
@@ -432,11 +533,31 @@ __global__ void timeout_probe_kernel(WaitCtl ctl) {
 
 template <int VPT, int OT, int UT, int GT>
 cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int64_t ld_u, const float* gamma,
-                      const float* beta, float eps, void* g, float* mu, float* rstd, cudaStream_t st) {
-  const int64_t blocks = (T + 7) / 8;
+                      const float* beta, float eps, void* g, float* mu, float* rstd, cudaStream_t st, int* status) {
+  const int64_t rows8 = (T + 7) / 8;
   cudaError_t e = prof_record(kProfNormFwd, false, st);
-  if (e == cudaSuccess)
-    e = launch_pdl(norm_gate_kernel<VPT, OT, UT, GT>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, T, o,
+  if (e != cudaSuccess) return e;
+  // staged rows (D >= 128) need 16-byte aligned row starts; their sizes are whole 16-byte chunks
+  bool staged = false;
+  if constexpr (VPT % 4 == 0) {
+    const auto al16 = [](const void* p, int64_t ld, int bytes) {
+      return bytes == 0 || ((reinterpret_cast<uintptr_t>(p) | static_cast<uintptr_t>(ld * bytes)) & 15) == 0;
+    };
+    if (al16(o, ld_o, dt_bytes(OT)) && al16(u, ld_u, dt_bytes(UT))) {
+      staged = true;
+      constexpr int kSmem = 8 * kNgSlots * VPT * 32 * (dt_bytes(OT) + dt_bytes(UT));
+      auto kern = norm_gate_staged_kernel<VPT, OT, UT, GT>;
+      e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kSmem);
+      if (e != cudaSuccess) return e;
+      const int per_sm = kSmem <= 100 * 1024 ? 2 : 1;
+      const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
+      const int64_t blocks = rows8 < cap ? rows8 : cap;
+      e = launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(256), kSmem, st, T, o, ld_o, u, ld_u, gamma,
+                     beta, eps, g, mu, rstd, wait_ctl(status));
+    }
+  }
+  if (!staged)
+    e = launch_pdl(norm_gate_kernel<VPT, OT, UT, GT>, dim3(static_cast<unsigned>(rows8)), dim3(256), 0, st, T, o,
                    ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd);
   if (e == cudaSuccess) e = prof_record(kProfNormFwd, true, st);
   return e;
@@ -469,26 +590,26 @@ cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B
 
 cudaError_t norm_gate_fwd(int64_t T, int D, int o_dt, int u_dt, int g_dt, const void* o, int64_t ld_o, const void* u,
                           int64_t ld_u, const float* gamma, const float* beta, float eps, void* g, float* mu,
-                          float* rstd, cudaStream_t st) {
+                          float* rstd, cudaStream_t st, int* status) {
   if (T == 0) return cudaSuccess;
   // supported (o, u, g) combinations: exact fp32; fp32 O with fp16 U and fp16 G (tensor-core
   // layer); fp32 O with fp16 or bf16 U and bf16 G; all bf16; fp32 or bf16 O without a gate and fp16
   // G (the input LayerNorm of the norm_in layer variant).
 #define HSTU_NG(VPT)                                                                                     \
   if (o_dt == kDtF32 && u_dt == kDtF32 && g_dt == kDtF32)                                               \
-    return launch_ng<VPT, kDtF32, kDtF32, kDtF32>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+    return launch_ng<VPT, kDtF32, kDtF32, kDtF32>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st, status); \
   if (o_dt == kDtF32 && u_dt == kDtF16 && g_dt == kDtF16)                                               \
-    return launch_ng<VPT, kDtF32, kDtF16, kDtF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+    return launch_ng<VPT, kDtF32, kDtF16, kDtF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st, status); \
   if (o_dt == kDtF32 && u_dt == kDtF16 && g_dt == kDtBF16)                                              \
-    return launch_ng<VPT, kDtF32, kDtF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+    return launch_ng<VPT, kDtF32, kDtF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st, status); \
   if (o_dt == kDtF32 && u_dt == kDtBF16 && g_dt == kDtBF16)                                             \
-    return launch_ng<VPT, kDtF32, kDtBF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+    return launch_ng<VPT, kDtF32, kDtBF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st, status); \
   if (o_dt == kDtBF16 && u_dt == kDtBF16 && g_dt == kDtBF16)                                            \
-    return launch_ng<VPT, kDtBF16, kDtBF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+    return launch_ng<VPT, kDtBF16, kDtBF16, kDtBF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st, status); \
   if (o_dt == kDtF32 && u_dt == kDtOne && g_dt == kDtF16)                                               \
-    return launch_ng<VPT, kDtF32, kDtOne, kDtF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st);  \
+    return launch_ng<VPT, kDtF32, kDtOne, kDtF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st, status);  \
   if (o_dt == kDtBF16 && u_dt == kDtOne && g_dt == kDtF16)                                              \
-    return launch_ng<VPT, kDtBF16, kDtOne, kDtF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st); \
+    return launch_ng<VPT, kDtBF16, kDtOne, kDtF16>(T, o, ld_o, u, ld_u, gamma, beta, eps, g, mu, rstd, st, status); \
   return cudaErrorInvalidValue
   switch (D) {
     case 64: HSTU_NG(2);

@@ -9,6 +9,8 @@
 //     dgamma = sum_t dLn (.) xhat,  dbeta = sum_t dLn;
 //   SiLU backward: dZ = dS (.) SiLU'(Z), SiLU'(z) = s(z)(1 + z(1 - s(z))), s = logistic;
 //   column sums for the bias gradients.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -24,35 +26,35 @@ namespace hstu {
 namespace {
 
 __device__ __forceinline__ float silu_grad(float z) {
-  const float s = 1.0f / (1.0f + __expf(fminf(-z, 80.0f)));
+  const float s = __fdividef(1.0f, 1.0f + __expf(fminf(-z, 80.0f)));
   return s * (1.0f + z * (1.0f - s));
 }
 
 // One warp per token row (grid-stride over rows); lane l holds features 128 k + 4 l + i (k < VPT / 4,
-// i < 4): every load and store of the warp covers 128 consecutive features (coalesced).
+// i < 4): every load and store of the warp covers 128 consecutive features (coalesced). gamma and
+// beta are staged in shared memory (registers for two blocks per SM).
 // Writes dO (act dtype), dZ_U = dU (.) SiLU'(Z_U) (fp16, row stride ld_dz) and per-block partial
 // sums of dgamma | dbeta into partial[blockIdx.x][0 .. 2D).
 template <int VPT, int AT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 norm_gate_bwd_kernel(int64_t T, const float* __restrict__ dg, const float* __restrict__ o, const void* __restrict__ u,
                      const void* __restrict__ zu, int64_t ld_act, const float* __restrict__ gamma,
                      const float* __restrict__ beta, const float* __restrict__ mu, const float* __restrict__ rstd,
                      void* __restrict__ d_o, void* __restrict__ dz, int64_t ld_dz, float* __restrict__ partial) {
-  pdl_enter();
   constexpr int D = VPT * 32;
   constexpr int KG = VPT / 4;   // groups of 4 features per lane
+  __shared__ __align__(16) float s_gb[2 * D];
   __shared__ float s_red[8][2][D];
+  for (int c = threadIdx.x; c < D; c += blockDim.x) {
+    s_gb[c] = gamma[c];
+    s_gb[D + c] = beta[c];
+  }
+  pdl_enter();
+  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  auto feat = [&](int e) { return 128 * (e >> 2) + 4 * lane + (e & 3); };
   float gacc[VPT], bacc[VPT];
 #pragma unroll
   for (int e = 0; e < VPT; ++e) gacc[e] = bacc[e] = 0.0f;
-  float gm[VPT], bt[VPT];
-#pragma unroll
-  for (int k = 0; k < KG; ++k) {
-    load_vec<4, kDtF32>(gamma, 128 * k + 4 * lane, gm + 4 * k);
-    load_vec<4, kDtF32>(beta, 128 * k + 4 * lane, bt + 4 * k);
-  }
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + warp; row < T; row += static_cast<int64_t>(gridDim.x) * 8) {
     float g[VPT], x[VPT], uu[VPT], z[VPT];
 #pragma unroll
@@ -66,18 +68,27 @@ norm_gate_bwd_kernel(int64_t T, const float* __restrict__ dg, const float* __res
     const float m = mu[row], rs = rstd[row];
     float s1 = 0.0f, s2 = 0.0f;
 #pragma unroll
-    for (int e = 0; e < VPT; ++e) {
-      const float xh = (x[e] - m) * rs;
-      const float dln = g[e] * uu[e];
-      const float dxh = dln * gm[e];
-      gacc[e] = fmaf(dln, xh, gacc[e]);
-      bacc[e] += dln;
-      s1 += dxh;
-      s2 = fmaf(dxh, xh, s2);
-      const float du = g[e] * fmaf(gm[e], xh, bt[e]);
-      z[e] = du * silu_grad(z[e]);        // dZ_U
-      x[e] = xh;                          // keep xhat
-      g[e] = dxh;                         // keep dxhat
+    for (int k = 0; k < KG; ++k) {
+      const int c = 128 * k + 4 * lane;
+      float gm[4], bt[4];
+      load_vec<4, kDtF32>(s_gb, c, gm);
+      load_vec<4, kDtF32>(s_gb + D, c, bt);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = 4 * k + i;
+        const float xh = (x[e] - m) * rs;
+        const float dln = g[e] * uu[e];
+        const float dxh = dln * gm[i];
+        gacc[e] = fmaf(dln, xh, gacc[e]);
+        bacc[e] += dln;
+        s1 += dxh;
+        s2 = fmaf(dxh, xh, s2);
+        const float du = g[e] * fmaf(gm[i], xh, bt[i]);
+        z[e] = du * silu_grad(z[e]);        // dZ_U
+        x[e] = xh;                          // keep xhat
+        g[e] = dxh;                         // keep dxhat
+      }
+      store_vec<4, kDtF16>(dz, row * ld_dz + c, z + 4 * k);
     }
 #pragma unroll
     for (int k = 16; k > 0; k >>= 1) {
@@ -88,16 +99,13 @@ norm_gate_bwd_kernel(int64_t T, const float* __restrict__ dg, const float* __res
 #pragma unroll
     for (int e = 0; e < VPT; ++e) g[e] = rs * (g[e] - m1 - x[e] * m2);
 #pragma unroll
-    for (int k = 0; k < KG; ++k) {
-      const int c = 128 * k + 4 * lane;
-      store_vec<4, AT>(d_o, row * D + c, g + 4 * k);
-      store_vec<4, kDtF16>(dz, row * ld_dz + c, z + 4 * k);
-    }
+    for (int k = 0; k < KG; ++k) store_vec<4, AT>(d_o, row * D + 128 * k + 4 * lane, g + 4 * k);
   }
 #pragma unroll
   for (int e = 0; e < VPT; ++e) {
-    s_red[warp][0][feat(e)] = gacc[e];
-    s_red[warp][1][feat(e)] = bacc[e];
+    const int f = 128 * (e >> 2) + 4 * lane + (e & 3);
+    s_red[warp][0][f] = gacc[e];
+    s_red[warp][1][f] = bacc[e];
   }
   __syncthreads();
   for (int c = threadIdx.x; c < 2 * D; c += 256) {
@@ -105,6 +113,140 @@ norm_gate_bwd_kernel(int64_t T, const float* __restrict__ dg, const float* __res
 #pragma unroll
     for (int w = 0; w < 8; ++w) s += s_red[w][c / D][c % D];
     partial[static_cast<int64_t>(blockIdx.x) * 2 * D + c] = s;
+  }
+}
+
+// Row slots per warp of the staged backward below.
+constexpr int kNgbSlots = 2;
+
+// The same backward with the rows staged by bulk copies (dG, O as fp32, then U and Z_U of the act
+// type): a persistent grid whose warps each own kNgbSlots row slots in shared memory and rows gw,
+// gw + W, ... (gw = the warp's global index, W = all warps); lane 0 refills a slot as soon as the
+// warp has read it. xhat and dxhat are recomputed from the slot after the row reductions instead of
+// being held in registers. The slot memory holds the block's dgamma | dbeta sums at the end.
+template <int VPT, int AT>
+__global__ void __launch_bounds__(256, 2)
+norm_gate_bwd_staged_kernel(int64_t T, const float* __restrict__ dg, const float* __restrict__ o,
+                            const void* __restrict__ u, const void* __restrict__ zu, int64_t ld_act,
+                            const float* __restrict__ gamma, const float* __restrict__ beta,
+                            const float* __restrict__ mu, const float* __restrict__ rstd, void* __restrict__ d_o,
+                            void* __restrict__ dz, int64_t ld_dz, float* __restrict__ partial, WaitCtl ctl) {
+  constexpr int D = VPT * 32, KG = VPT / 4;
+  constexpr int GB = D * 4, OB = D * 4, AB = D * 2, SLOT = GB + OB + 2 * AB, S = kNgbSlots;
+  static_assert(VPT % 4 == 0, "groups of four features per lane");
+  static_assert(8 * S * SLOT >= 8 * 2 * D * 4, "the slots hold the block's partial sums at the end");
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint64_t s_bar[8 * S];
+  __shared__ int s_abort;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 8 * S; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  float gm[VPT], bt[VPT];
+#pragma unroll
+  for (int k = 0; k < KG; ++k) {
+    load_vec<4, kDtF32>(gamma, 128 * k + 4 * lane, gm + 4 * k);
+    load_vec<4, kDtF32>(beta, 128 * k + 4 * lane, bt + 4 * k);
+  }
+  pdl_enter();
+  __syncthreads();
+  const long long W = static_cast<long long>(gridDim.x) * 8, gw = static_cast<long long>(blockIdx.x) * 8 + warp;
+  uint8_t* wslots = smem + static_cast<size_t>(warp) * S * SLOT;
+  auto issue = [&](long long i) {   // lane 0: row i of this warp into slot i % S
+    const long long row = gw + i * W;
+    if (row >= T) return;
+    const int sl = static_cast<int>(i % S);
+    const uint32_t bar = smem_u32(&s_bar[warp * S + sl]);
+    const uint32_t dst = smem_u32(wslots + sl * SLOT);
+    mbar_arrive_expect_tx(bar, SLOT);
+    bulk_load(dst, dg + row * D, GB, bar);
+    bulk_load(dst + GB, o + row * D, OB, bar);
+    bulk_load(dst + GB + OB, static_cast<const uint16_t*>(u) + row * ld_act, AB, bar);
+    bulk_load(dst + GB + OB + AB, static_cast<const uint16_t*>(zu) + row * ld_act, AB, bar);
+  };
+  if (lane == 0)
+    for (int i = 0; i < S; ++i) issue(i);
+  float gacc[VPT], bacc[VPT];
+#pragma unroll
+  for (int e = 0; e < VPT; ++e) gacc[e] = bacc[e] = 0.0f;
+  for (long long i = 0;; ++i) {
+    const long long row = gw + i * W;
+    if (row >= T) break;
+    const int sl = static_cast<int>(i % S);
+    if (!mbar_wait_warp(smem_u32(&s_bar[warp * S + sl]), static_cast<uint32_t>((i / S) & 1), &s_abort, ctl)) break;
+    const uint8_t* sg = wslots + sl * SLOT;
+    const uint8_t *so = sg + GB, *su = so + OB, *sz = su + AB;
+    const float m = mu[row], rs = rstd[row];
+    float s1 = 0.0f, s2 = 0.0f;
+#pragma unroll
+    for (int k = 0; k < KG; ++k) {
+      const int c = 128 * k + 4 * lane;
+      float g4[4], x4[4], u4[4], z4[4];
+      load_vec<4, kDtF32>(sg, c, g4);
+      load_vec<4, kDtF32>(so, c, x4);
+      load_vec<4, AT>(su, c, u4);
+      load_vec<4, AT>(sz, c, z4);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = 4 * k + q;
+        const float xh = (x4[q] - m) * rs;
+        const float dln = g4[q] * u4[q];
+        const float dxh = dln * gm[e];
+        gacc[e] = fmaf(dln, xh, gacc[e]);
+        bacc[e] += dln;
+        s1 += dxh;
+        s2 = fmaf(dxh, xh, s2);
+        z4[q] = g4[q] * fmaf(gm[e], xh, bt[e]) * silu_grad(z4[q]);   // dZ_U
+      }
+      store_vec<4, kDtF16>(dz, row * ld_dz + c, z4);
+    }
+#pragma unroll
+    for (int k = 16; k > 0; k >>= 1) {
+      s1 += __shfl_xor_sync(0xffffffffu, s1, k);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, k);
+    }
+    const float m1 = s1 * (1.0f / D), m2 = s2 * (1.0f / D);
+#pragma unroll
+    for (int k = 0; k < KG; ++k) {
+      const int c = 128 * k + 4 * lane;
+      float g4[4], x4[4], u4[4];
+      load_vec<4, kDtF32>(sg, c, g4);
+      load_vec<4, kDtF32>(so, c, x4);
+      load_vec<4, AT>(su, c, u4);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float xh = (x4[q] - m) * rs;
+        const float dxh = g4[q] * u4[q] * gm[4 * k + q];
+        g4[q] = rs * (dxh - m1 - xh * m2);
+      }
+      store_vec<4, AT>(d_o, row * D + c, g4);
+    }
+    // every lane has read the slot: refill it (generic reads before the copy engine's writes)
+    __syncwarp();
+    if (lane == 0) {
+      fence_proxy_async_smem();
+      issue(i + S);
+    }
+  }
+  // the block's partial sums, through the slot memory once every copy has landed and been read (a
+  // failed wait set s_abort, so every thread of the block takes the same branch)
+  __syncthreads();
+  if (s_abort) return;
+  float* s_red = reinterpret_cast<float*>(smem);   // [8][2][D]
+#pragma unroll
+  for (int e = 0; e < VPT; ++e) {
+    const int f = 128 * (e >> 2) + 4 * lane + (e & 3);
+    s_red[(warp * 2 + 0) * D + f] = gacc[e];
+    s_red[(warp * 2 + 1) * D + f] = bacc[e];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < 2 * D; c += 256) {
+    float t = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += s_red[(w * 2 + c / D) * D + c % D];
+    partial[static_cast<int64_t>(blockIdx.x) * 2 * D + c] = t;
   }
 }
 
@@ -208,6 +350,7 @@ colsum_final_kernel(const float* __restrict__ partial, int parts, int cols, floa
 
 }  // namespace
 
+// Two blocks of eight rows per SM of a 148-SM part (at most); one block per eight rows below that.
 int norm_gate_bwd_blocks(int64_t T) {
   const int64_t b = (T + 7) / 8;
   return static_cast<int>(b < 296 ? (b > 0 ? b : 1) : 296);
@@ -216,30 +359,50 @@ int norm_gate_bwd_blocks(int64_t T) {
 cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const float* o, const void* u,
                           const void* zu, int64_t ld_act, const float* gamma, const float* beta, const float* mu,
                           const float* rstd, void* d_o, void* dz, int64_t ld_dz, float* partial,
-                          float* dgamma_dbeta_out, cudaStream_t st) {
+                          float* dgamma_dbeta_out, cudaStream_t st, int* status) {
   if (T == 0) return cudaSuccess;
   const int G = norm_gate_bwd_blocks(T);
   cudaError_t e = prof_record(kProfNormBwd, false, st);
   if (e != cudaSuccess) return e;
+  // the staged kernel copies whole rows: 16-byte aligned row starts for U and Z_U (dG, O and the
+  // fp32 rows are [T, D] with D a multiple of 128)
+  const bool staged = (((reinterpret_cast<uintptr_t>(u) | reinterpret_cast<uintptr_t>(zu) |
+                         reinterpret_cast<uintptr_t>(dg) | reinterpret_cast<uintptr_t>(o) |
+                         static_cast<uintptr_t>(ld_act * 2)) & 15) == 0);
+  const int gs = static_cast<int>(std::min<int64_t>((T + 7) / 8, 2ll * sm_count()));
+  int parts = G;   // partial rows written
+#define HSTU_NGB_ONE(VPT, AT)                                                                                    \
+  if (staged && gs <= G) {                                                                                       \
+    constexpr int kSmem = 8 * kNgbSlots * VPT * 32 * 12;                                                         \
+    auto kern = norm_gate_bwd_staged_kernel<VPT, AT>;                                                            \
+    e = ensure_smem_attr(reinterpret_cast<const void*>(kern), kSmem);                                            \
+    if (e == cudaSuccess)                                                                                        \
+      e = launch_pdl(kern, dim3(gs), dim3(256), kSmem, st, T, dg, o, u, zu, ld_act, gamma, beta, mu, rstd, d_o, dz, \
+                     ld_dz, partial, wait_ctl(status));                                                           \
+    parts = gs;                                                                                                  \
+  } else {                                                                                                       \
+    e = launch_pdl(norm_gate_bwd_kernel<VPT, AT>, dim3(G), dim3(256), 0, st, T, dg, o, u, zu, ld_act, gamma, beta, \
+                   mu, rstd, d_o, dz, ld_dz, partial);                                                            \
+  }
 #define HSTU_NGB(VPT)                                                                                            \
-  if (act_dt == kDtF16)                                                                                          \
-    e = launch_pdl(norm_gate_bwd_kernel<VPT, kDtF16>, dim3(G), dim3(256), 0, st, T, dg, o, u, zu, ld_act, gamma,   \
-                   beta, mu, rstd, d_o, dz, ld_dz, partial);                                                      \
-  else if (act_dt == kDtBF16)                                                                                    \
-    e = launch_pdl(norm_gate_bwd_kernel<VPT, kDtBF16>, dim3(G), dim3(256), 0, st, T, dg, o, u, zu, ld_act, gamma,  \
-                   beta, mu, rstd, d_o, dz, ld_dz, partial);                                                      \
-  else                                                                                                           \
-    return cudaErrorInvalidValue;
+  if (act_dt == kDtF16) {                                                                                        \
+    HSTU_NGB_ONE(VPT, kDtF16)                                                                                    \
+  } else if (act_dt == kDtBF16) {                                                                                \
+    HSTU_NGB_ONE(VPT, kDtBF16)                                                                                   \
+  } else {                                                                                                       \
+    return cudaErrorInvalidValue;                                                                                \
+  }
   switch (D) {
     case 256: HSTU_NGB(8); break;
     case 512: HSTU_NGB(16); break;
     default: return cudaErrorInvalidValue;
   }
 #undef HSTU_NGB
+#undef HSTU_NGB_ONE
   if (e == cudaSuccess) e = prof_record(kProfNormBwd, true, st);
   if (e != cudaSuccess) return e;
-  return launch_pdl(colsum_final_kernel, dim3((2 * D + 31) / 32), dim3(256), 0, st, static_cast<const float*>(partial), G,
-                    2 * D, dgamma_dbeta_out);
+  return launch_pdl(colsum_final_kernel, dim3((2 * D + 31) / 32), dim3(256), 0, st, static_cast<const float*>(partial),
+                    parts, 2 * D, dgamma_dbeta_out);
 }
 
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,

@@ -112,6 +112,14 @@ __device__ __forceinline__ void pdl_enter() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// Untiled bulk copy of `bytes` (a multiple of 16) from global src into this CTA's shared memory at
+// dst, both 16-byte aligned; completes `bytes` transactions on the mbarrier bar. No multicast.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 // One 32-byte store of eight floats (dst 32-byte aligned).
 __device__ __forceinline__ void st_global_v8(float* dst, const float (&f)[8]) {
   asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "f"(f[0]), "f"(f[1]),
