@@ -34,6 +34,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "hstu_internal.h"
 #include "sm100_ptx.cuh"
 #include "tile_pairs.cuh"
@@ -875,7 +877,15 @@ attn_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid
               tc_fence_before();
               mbar_arrive(o_empty(ob));
             }
+            // P and the half-bias are fp16: a score beyond the fp16 range turns O non-finite, which
+            // is reported (HSTU_ERR_DEVICE) instead of passing silently
             if (row_ok) {
+              bool finite = true;
+#pragma unroll
+              for (int e = 0; e < 16; ++e) finite &= isfinite(__uint_as_float(ov[e]));
+              if (!finite) report_error(a.status, kDevBadInput);
+            }
+            if (row_ok && HSTU_DCHECK(orow >= 0 && orow < a.T, a.status)) {
               const int ocol = u.h * kD + 32 * half + 16 * c;
               if (a.o_f32 && o_v8) {
                 float* dst = reinterpret_cast<float*>(a.o) + orow * a.ld_o + ocol;
@@ -969,15 +979,15 @@ int64_t attn_max_pairs(int64_t capacity, int max_len) {
 }
 
 int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cache[64];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
-  }
-  return cached[dev];
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  const bool tracked = dev >= 0 && dev < 64;
+  int n = tracked ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (tracked) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 template <bool F16>

@@ -133,7 +133,10 @@ __device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pai
   const float* rab_time = a.rab_time + static_cast<long long>(hb) * a.n_buckets;
   tile_times_load(s_t, a.ts, seq0, n, qt * kQTile, kt * kQTile);
   if (tid < a.n_buckets) s_rt[tid] = 0.5f * rab_time[tid];
-  if (tid < 255) s_win[tid] = 0.5f * rab_pos[bias_pos_index(static_cast<long long>(qt - kt) * kQTile - 127 + tid, L)];
+  if (tid < 255) {
+    const int pi = bias_pos_index(static_cast<long long>(qt - kt) * kQTile - 127 + tid, L);
+    if (HSTU_DCHECK(pi >= 0 && pi < 2 * L - 1, a.status)) s_win[tid] = 0.5f * rab_pos[pi];
+  }
   if (nt > 0) {
     tile_types_load(s_ty, a.token_type, seq0, n, qt * kQTile, kt * kQTile, nt, a.status);
     if (tid < nt * nt) s_tt[tid] = 0.5f * a.rab_type[static_cast<long long>(hb) * nt * nt + tid];
@@ -163,8 +166,13 @@ __device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pai
         for (int x = 0; x < 2; ++x) {
           const int c = cl + 32 * e + x;
           const int bkt = tile_bucket<TRANSPOSED>(s_t, kFast, r, c, s_tau, s_tau32, nb);
-          float v = s_win[TRANSPOSED ? c - r + 127 : r - c + 127] + s_rt[bkt];
-          if (nt > 0) v += s_tt[s_ty[TRANSPOSED ? c : r] * nt + s_ty[128 + (TRANSPOSED ? r : c)]];
+          const int wi = TRANSPOSED ? c - r + 127 : r - c + 127;
+          float v = 0.0f;
+          if (HSTU_DCHECK(bkt >= 0 && bkt < nb && wi >= 0 && wi < 255, a.status)) v = s_win[wi] + s_rt[bkt];
+          if (nt > 0) {
+            const int ti = s_ty[TRANSPOSED ? c : r] * nt + s_ty[128 + (TRANSPOSED ? r : c)];
+            if (HSTU_DCHECK(ti >= 0 && ti < nt * nt, a.status)) v += s_tt[ti];
+          }
           v2[x] = v;
           bw |= static_cast<uint32_t>(bkt) << (8 * x);
         }

@@ -311,6 +311,14 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
         }
         if (epi.kind == kEpiSilu) {
+          // Z and SiLU(Z) stored in fp16: a pre-activation outside the fp16 range (or NaN) is reported
+          // (HSTU_ERR_DEVICE) instead of becoming inf silently
+          if (row_ok && (epi.out0_dt == kDtF16 || epi.out1_dt == kDtF16)) {
+            bool in_range = true;
+#pragma unroll
+            for (int j = 0; j < 64; ++j) in_range &= fabsf(v[j]) <= 65504.0f;
+            if (!in_range) report_error(ctl.status, kDevBadInput);
+          }
           if (epi.out1) emit64(es, &tmO1, epi.out1_dt, false, n, ybox, v, P.N);
 #pragma unroll
           for (int j = 0; j < 64; ++j) v[j] = silu_tanh(v[j]);
@@ -405,19 +413,6 @@ gemm_f32_simt_kernel(const float* __restrict__ A, int64_t sam, int64_t sak, cons
         store_one(epi.out1, epi.out1_dt, static_cast<int64_t>(m) * epi.ld_out1 + n, v);
     }
   }
-}
-
-// SM count of the current device, cached per device (148 if it cannot be read).
-int sm_count() {
-  static std::atomic<int> cache[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  const bool tracked = dev >= 0 && dev < 64;
-  int n = tracked ? cache[dev].load(std::memory_order_relaxed) : 0;
-  if (n > 0) return n;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  if (tracked) cache[dev].store(n, std::memory_order_relaxed);
-  return n;
 }
 
 template <int BN, int STAGES, bool A_MN, bool B_MN>

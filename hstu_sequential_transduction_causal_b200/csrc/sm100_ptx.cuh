@@ -25,6 +25,15 @@ __device__ __forceinline__ void report_error(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Checked indices of the debug build (compiled with -DHSTU_DEBUG: build.py --debug writes
+// libhstu_debug.so): a failed check records kDevBadInput (HSTU_ERR_DEVICE) in the status word and
+// the guarded access is skipped. The release build compiles every check to `true`.
+#ifdef HSTU_DEBUG
+#define HSTU_DCHECK(cond, status) ((cond) ? true : (::hstu::report_error((status), ::hstu::kDevBadInput), false))
+#else
+#define HSTU_DCHECK(cond, status) true
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

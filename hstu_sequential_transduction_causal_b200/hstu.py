@@ -13,11 +13,16 @@ from typing import Optional
 
 import torch
 
-from .build import LIB as _LIB_PATH
+from .build import LIB as _LIB_RELEASE, LIB_DEBUG as _LIB_DEBUG
+
+# HSTU_DEBUG=1 selects the checked-index build (build.py --debug)
+_LIB_PATH = _LIB_DEBUG if os.environ.get("HSTU_DEBUG", "0") not in ("", "0") else _LIB_RELEASE
 
 c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
 HSTU_F32, HSTU_BF16, HSTU_F16 = 0, 1, 2
+(HSTU_OK, HSTU_ERR_INVALID_ARG, HSTU_ERR_UNSUPPORTED, HSTU_ERR_WORKSPACE, HSTU_ERR_CUDA, HSTU_ERR_TIMEOUT,
+ HSTU_ERR_DEVICE) = range(7)
 STATUS = {0: "HSTU_OK", 1: "HSTU_ERR_INVALID_ARG", 2: "HSTU_ERR_UNSUPPORTED", 3: "HSTU_ERR_WORKSPACE",
           4: "HSTU_ERR_CUDA", 5: "HSTU_ERR_TIMEOUT", 6: "HSTU_ERR_DEVICE"}
 
@@ -146,7 +151,8 @@ def library_path() -> str:
 
 
 def lib() -> ctypes.CDLL:
-    """Loads libhstu.so (built in-tree by ``build.py``); raises if it is missing."""
+    """Loads libhstu.so (libhstu_debug.so under HSTU_DEBUG=1; built in-tree by ``build.py``); raises if
+    it is missing."""
     global _lib
     if _lib is None:
         if not os.path.exists(_LIB_PATH):

@@ -88,7 +88,10 @@ typedef struct hstu_attn_desc_t {
   float inv_N;             /* 1/N, the constant normaliser */
   int32_t pos_max_len;     /* L: rab_pos has 2L-1 entries */
   int32_t n_time_buckets;  /* 1..128 */
-  hstu_dtype_t dtype;      /* dtype of q, k, v: BF16 or F16 (tensor cores) or F32 (CUDA cores) */
+  hstu_dtype_t dtype;      /* dtype of q, k, v: BF16 or F16 (tensor cores) or F32 (CUDA cores). On
+                              the tensor cores the score, the half-bias and P are fp16: a score
+                              past 65504 makes O non-finite, which the forward records as
+                              HSTU_ERR_DEVICE in the status word */
   hstu_dtype_t o_dtype;    /* dtype of out: F32 (any dtype) or BF16 (BF16 inputs only) */
   int64_t ld_q, ld_k, ld_v, ld_o; /* row strides (elements); head h occupies columns [h*d, (h+1)*d) */
 } hstu_attn_desc_t;
@@ -104,7 +107,12 @@ typedef struct hstu_layer_desc_t {
   hstu_dtype_t dtype;      /* BF16: bf16 weights and activations on the tensor cores with fp32
                               accumulation: U|V|Q|K, Z, the attention weights P and G in fp16
                               (8x finer than bf16 at the same MMA rate), O in fp32; f2 reads an
-                              fp16 copy of W2 (exact for bf16 values in the fp16 range);
+                              fp16 copy of W2 (exact for bf16 values in the fp16 range).
+                              Range: fp16 holds |v| <= 65504. A pre-activation Z outside that
+                              range, or an attention score that drives O to inf / NaN, is recorded
+                              as HSTU_ERR_DEVICE in the status word (the call's outputs are then not
+                              meaningful); G = LayerNorm(O) (.) U is bounded by |gamma| sqrt(D) +
+                              |beta| times |U| and is not checked.
                               F32: every step in fp32 on the CUDA cores */
   hstu_dtype_t x_dtype;    /* dtype of X; F32 with BF16 compute = fp32 residual stream (f1 then
                               reads an fp16 copy of X and of W1) */

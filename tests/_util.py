@@ -60,3 +60,30 @@ def sample_rows(offsets, per_seq=6, seed=0):
         cand.update(int(r) for r in rng.integers(0, n, size=per_seq))
         rows.extend(s + r for r in sorted(cand))
     return np.array(sorted(set(rows)), np.int64)
+
+
+# Canary guard words (a stand-in for an out-of-bounds checker, which this pool does not offer): the
+# output tensor sits inside a larger allocation whose leading and trailing bytes hold a fixed pattern
+# that no kernel may change.
+CANARY = 0xA5
+
+
+def guarded(shape, dtype, fill=float("nan"), guard_bytes=4096, device="cuda"):
+    """(tensor, check): a device tensor of `shape` (filled with `fill`) between two guard regions of
+    `guard_bytes` holding CANARY; check(what) asserts both regions are intact."""
+    import torch
+    elt = torch.empty((), dtype=dtype).element_size()
+    n = int(np.prod(shape))
+    g = guard_bytes // elt
+    raw = torch.empty(n + 2 * g, dtype=dtype, device=device)
+    raw.view(torch.uint8).fill_(CANARY)
+    t = raw[g:g + n].view(*shape)
+    if fill is not None:
+        t.fill_(fill)
+
+    def check(what=""):
+        b = raw.view(torch.uint8)
+        head, tail = b[:g * elt], b[(g + n) * elt:]
+        assert bool((head == CANARY).all()), f"{what}: bytes before the output changed"
+        assert bool((tail == CANARY).all()), f"{what}: bytes after the output changed"
+    return t, check
