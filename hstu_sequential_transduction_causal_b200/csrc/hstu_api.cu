@@ -118,7 +118,7 @@ AttnBwdWs attn_bwd_ws_layout(const hstu_jagged_t* j, int H, int hb = 1) {
 // (fp32), dZ (fp16 [T, 4D]), reduction partials, dgamma | dbeta, and the fp16 GEMM operands: copies
 // of dy, x, W1 and W2 (both MMA operands share a type; G and dZ are fp16).
 struct LayerBwdWs {
-  size_t dg, dO, dq, dk, dv, dz, partial, gb, dy_f16, x_f16, w1_f16, w2_f16, total;
+  size_t dg, dO, dq, dk, dv, dz, part_dy, part_ln, part_dz, dy_f16, x_f16, w1_f16, w2_f16, total;
 };
 
 LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) {
@@ -132,10 +132,11 @@ LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) 
   w.dk = take(T * D * 4);
   w.dv = take(T * D * 4);
   w.dz = take(T * 4 * D * 2);
-  size_t pf = colsum_partial_floats(static_cast<int>(4 * D));
-  const size_t pl = static_cast<size_t>(norm_gate_bwd_blocks(j->T)) * 2 * D;
-  w.partial = take((pf > pl ? pf : pl) * 4);
-  w.gb = take(2 * D * 4);
+  // partial column sums: db2 (from the fp16 copy of dY), dgamma | dbeta (LayerNorm backward), db1
+  // (column sum of dZ)
+  w.part_dy = take(static_cast<size_t>(kTailParts) * D * 4);
+  w.part_ln = take(static_cast<size_t>(norm_gate_bwd_blocks(j->T)) * 2 * D * 4);
+  w.part_dz = take(colsum_partial_floats(static_cast<int>(4 * D)) * 4);
   w.dy_f16 = take(T * D * 2);
   w.x_f16 = take(T * D * 2);
   w.w1_f16 = take(4 * D * D * 2);
@@ -880,10 +881,16 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   const void* x_op = x_f16 ? x_f16 : wsb + lay.x_f16;
   void* w1_f16 = wsb + lay.w1_f16;
   void* w2_f16 = wsb + lay.w2_f16;
-  {   // the fp16 GEMM operand copies, one launch
+  float* part_dy = reinterpret_cast<float*>(wsb + lay.part_dy);
+  float* part_ln = reinterpret_cast<float*>(wsb + lay.part_ln);
+  float* part_dz = reinterpret_cast<float*>(wsb + lay.part_dz);
+  int parts_dy = 0, parts_ln = 0;
+  // the fp16 copy of dY (unless the caller passed one) together with the partial sums of db2
+  e = rows_to_f16_colsum(T, D, y_dt, dy, dy_f16 ? nullptr : wsb + lay.dy_f16, part_dy, &parts_dy, st);
+  if (e != cudaSuccess) return cuda_status(e);
+  {   // the other fp16 GEMM operand copies, one launch
     ConvertJob jobs[4];
     int nj = 0;
-    if (!dy_f16) jobs[nj++] = ConvertJob{dy, wsb + lay.dy_f16, T * D, y_dt};
     if (!x_f16) jobs[nj++] = ConvertJob{x, wsb + lay.x_f16, T * D, x_dt};
     jobs[nj++] = ConvertJob{w->W1, w1_f16, 4ll * D * D, kDtBF16};
     jobs[nj++] = ConvertJob{w->W2, w2_f16, 1ll * D * D, kDtBF16};
@@ -896,8 +903,6 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   float* dk = reinterpret_cast<float*>(wsb + lay.dk);
   float* dv = reinterpret_cast<float*>(wsb + lay.dv);
   void* dz = wsb + lay.dz;
-  float* part = reinterpret_cast<float*>(wsb + lay.partial);
-  float* gb = reinterpret_cast<float*>(wsb + lay.gb);
   // 1. f2 backward: dG = dY W2, dW2 = dY^T G, db2 = sum_t dY
   GemmArgs g{};
   g.A = dy_op; g.lda = D; g.a_mn = false; g.B = w2_f16; g.ldb = D; g.b_mn = true; g.f16 = true;
@@ -912,13 +917,17 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
     g2.epi.kind = kEpiAtomic; g2.epi.out0 = gr->dW2; g2.epi.out0_dt = kDtF32; g2.epi.ld_out0 = D; g2.status = status;
     e = gemm_bf16(g2, st);
   }
-  if (e == cudaSuccess) e = column_sum(dy, desc->y_dtype, T, D, D, part, gr->db2, st);
-  // 2. norm-gate backward: dO (fp16), dZ_U (bf16), dgamma | dbeta
+  // 2. norm-gate backward: dO (fp16), dZ_U (fp16), partial dgamma | dbeta; then db2, dgamma and dbeta
+  // finished by one launch straight into the caller's buffers
   if (e == cudaSuccess)
     e = norm_gate_bwd(T, D, kDtF16, dG, static_cast<const float*>(saved->o), saved->uvqk, saved->z, 4ll * D, w->gamma,
-                      w->beta, saved->mu, saved->rstd, dO, dz, 4ll * D, part, gb, st, status);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(gr->dgamma, gb, sizeof(float) * D, cudaMemcpyDeviceToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(gr->dbeta, gb + D, sizeof(float) * D, cudaMemcpyDeviceToDevice, st);
+                      w->beta, saved->mu, saved->rstd, dO, dz, 4ll * D, part_ln, &parts_ln, st, status);
+  if (e == cudaSuccess) {
+    const ColsumJob jobs[3] = {{part_dy, D, parts_dy, D, gr->db2},
+                               {part_ln, 2ll * D, parts_ln, D, gr->dgamma},
+                               {part_ln + D, 2ll * D, parts_ln, D, gr->dbeta}};
+    e = colsum_final_multi(jobs, 3, st);
+  }
   if (e != cudaSuccess) return cuda_status(e);
   // 3. attention backward
   const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
@@ -931,7 +940,7 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   }
   // 4. SiLU backward into dZ[:, D:4D], db1 = sum_t dZ
   e = dz_assemble(T, D, kDtF16, dv, dq, dk, saved->z, 4ll * D, dz, 4ll * D, st);
-  if (e == cudaSuccess) e = column_sum(dz, kDtF16, T, 4 * D, 4ll * D, part, gr->db1, st);
+  if (e == cudaSuccess) e = column_sum(dz, kDtF16, T, 4 * D, 4ll * D, part_dz, gr->db1, st);
   // 5. f1 backward: dW1 = dZ^T X, dX = dY + dZ W1 (fp16 dZ, x and W1)
   if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW1, 0, sizeof(float) * 4 * D * D, st);
   if (e == cudaSuccess) {

@@ -228,13 +228,34 @@ cudaError_t convert_f32_to_bf16(const float* in, void* out, int64_t n, cudaStrea
 // ---------------------------------------------------------------------------------------------
 int norm_gate_bwd_blocks(int64_t T);
 // dO = LayerNorm backward of dLn = dG (.) U; dZ_U = dG (.) Ln (.) SiLU'(Z_U) (fp16, stride ld_dz);
-// dgamma | dbeta -> dgamma_dbeta_out[0 .. 2D) via partial [norm_gate_bwd_blocks(T), 2D].
+// the partial sums of dgamma | dbeta into partial [*parts, 2D] (*parts <= norm_gate_bwd_blocks(T));
+// the caller finishes them (colsum_final_multi).
 cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const float* o, const void* u,
                           const void* zu, int64_t ld_act, const float* gamma, const float* beta, const float* mu,
-                          const float* rstd, void* d_o, void* dz, int64_t ld_dz, float* partial,
-                          float* dgamma_dbeta_out, cudaStream_t st, int* status = nullptr);
+                          const float* rstd, void* d_o, void* dz, int64_t ld_dz, float* partial, int* parts,
+                          cudaStream_t st, int* status = nullptr);
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
                         const void* z, int64_t ld_z, void* dz, int64_t ld_dz, cudaStream_t st);
+// [T, D] rows (fp32, bf16 or fp16) to fp16 (out may be null) and their partial column sums into
+// partial [*parts, D] (at most kTailParts rows).
+cudaError_t rows_to_f16_colsum(int64_t T, int D, int in_dt, const void* in, void* out, float* partial, int* parts,
+                               cudaStream_t st);
+// Most partial rows rows_to_f16_colsum writes.
+constexpr int kTailParts = 296;
+// Several column-sum finishes in one launch.
+struct ColsumJob {
+  const float* partial;   // parts rows of `ld` floats; the job reads columns [0, cols)
+  int64_t ld;
+  int parts;
+  int cols;
+  float* out;             // [cols]
+};
+struct ColsumJobs {
+  ColsumJob job[4];
+  int first_block[5];
+  int njobs;
+};
+cudaError_t colsum_final_multi(const ColsumJob* jobs, int njobs, cudaStream_t st);
 size_t colsum_partial_floats(int cols);
 cudaError_t convert_dtype(const void* in, int in_dt, void* out, int out_dt, int64_t n, cudaStream_t st);
 // Up to four conversions to fp16 (inputs fp32, bf16 or fp16) in one launch.

@@ -119,6 +119,9 @@ norm_gate_bwd_kernel(int64_t T, const float* __restrict__ dg, const float* __res
 // Row slots per warp of the staged backward below.
 constexpr int kNgbSlots = 2;
 
+// Threads of the fused conversion + column-sum kernel (rows_to_f16_colsum_kernel).
+constexpr int kTailThreads = 256;
+
 // The same backward with the rows staged by bulk copies (dG, O as fp32, then U and Z_U of the act
 // type): a persistent grid whose warps each own kNgbSlots row slots in shared memory and rows gw,
 // gw + W, ... (gw = the warp's global index, W = all warps); lane 0 refills a slot as soon as the
@@ -272,6 +275,86 @@ dz_assemble_kernel(int64_t T, int D, const float* __restrict__ dv, const float* 
   store_vec<8, kDtF16>(dz, row * ld_dz + D + c, gv);
 }
 
+// dY converted to fp16 (out, may be null when the caller holds an fp16 copy) and the partial column
+// sums of dY (the db2 of f2's bias): block b sums rows [b R, (b+1) R) into partial[b][0 .. D); its
+// threads own 8 columns each (D / 8 per row, 256 / (D / 8) rows side by side) and keep four rows'
+// loads in flight each.
+template <int D, int IT>
+__global__ void __launch_bounds__(kTailThreads)
+rows_to_f16_colsum_kernel(int64_t T, const void* __restrict__ in, void* __restrict__ out, int64_t rows_per,
+                          float* __restrict__ partial) {
+  constexpr int TPR = D / 8, RP = kTailThreads / TPR, U = 4;
+  static_assert(RP >= 1 && kTailThreads % TPR == 0, "whole rows per block");
+  __shared__ float s_red[RP > 1 ? RP - 1 : 1][D];
+  pdl_enter();
+  const int g = threadIdx.x % TPR, rp = threadIdx.x / TPR;
+  const int c = 8 * g;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per;
+  const int64_t r1 = r0 + rows_per < T ? r0 + rows_per : T;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+  for (int64_t row = r0 + rp; row < r1; row += U * RP) {
+    float v[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t r = row + static_cast<int64_t>(u) * RP;
+      if (r < r1) load_vec<8, IT>(in, r * D + c, v[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t r = row + static_cast<int64_t>(u) * RP;
+      if (r >= r1) continue;
+      if (out) store_vec<8, kDtF16>(out, r * D + c, v[u]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += v[u][e];
+    }
+  }
+  if constexpr (RP > 1) {
+    if (rp > 0)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_red[rp - 1][c + e] = acc[e];
+    __syncthreads();
+    if (rp == 0)
+      for (int q = 1; q < RP; ++q)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += s_red[q - 1][c + e];
+  }
+  if (rp == 0)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) partial[static_cast<int64_t>(blockIdx.x) * D + c + e] = acc[e];
+}
+
+// Several column-sum finishes in one launch: job j sums parts rows (row stride ld) of its partial
+// buffer into out[0 .. cols); each block takes 32 columns of one job (as colsum_final_kernel).
+__global__ void __launch_bounds__(256)
+colsum_final_multi_kernel(ColsumJobs jobs) {
+  pdl_enter();
+  __shared__ float s_part[8][33];
+  int j = 0;
+  while (j + 1 < jobs.njobs && static_cast<int>(blockIdx.x) >= jobs.first_block[j + 1]) ++j;
+  const ColsumJob& jb = jobs.job[j];
+  const int cl = threadIdx.x & 31, slice = threadIdx.x >> 5;
+  const int c = (static_cast<int>(blockIdx.x) - jobs.first_block[j]) * 32 + cl;
+  float s0 = 0.0f, s1 = 0.0f;
+  if (c < jb.cols) {
+    int p = slice;
+    for (; p + 8 < jb.parts; p += 16) {
+      s0 += jb.partial[static_cast<int64_t>(p) * jb.ld + c];
+      s1 += jb.partial[static_cast<int64_t>(p + 8) * jb.ld + c];
+    }
+    if (p < jb.parts) s0 += jb.partial[static_cast<int64_t>(p) * jb.ld + c];
+  }
+  s_part[slice][cl] = s0 + s1;
+  __syncthreads();
+  if (slice == 0 && c < jb.cols) {
+    float t = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += s_part[k][cl];
+    jb.out[c] = t;
+  }
+}
+
 // partial[y][c] = sum over rows [y R, (y+1) R) of in[row][c]; one thread per column.
 template <int DT>
 __global__ void __launch_bounds__(256)
@@ -358,8 +441,9 @@ int norm_gate_bwd_blocks(int64_t T) {
 
 cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const float* o, const void* u,
                           const void* zu, int64_t ld_act, const float* gamma, const float* beta, const float* mu,
-                          const float* rstd, void* d_o, void* dz, int64_t ld_dz, float* partial,
-                          float* dgamma_dbeta_out, cudaStream_t st, int* status) {
+                          const float* rstd, void* d_o, void* dz, int64_t ld_dz, float* partial, int* parts_out,
+                          cudaStream_t st, int* status) {
+  *parts_out = 0;
   if (T == 0) return cudaSuccess;
   const int G = norm_gate_bwd_blocks(T);
   cudaError_t e = prof_record(kProfNormBwd, false, st);
@@ -400,10 +484,19 @@ cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const f
 #undef HSTU_NGB
 #undef HSTU_NGB_ONE
   if (e == cudaSuccess) e = prof_record(kProfNormBwd, true, st);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(colsum_final_kernel, dim3((2 * D + 31) / 32), dim3(256), 0, st, static_cast<const float*>(partial),
-                    parts, 2 * D, dgamma_dbeta_out);
+  *parts_out = parts;
+  return e;
 }
+
+namespace {
+// Partial rows of the fused column sum: blocks of at least 16 rows, at most kTailParts of them.
+int tail_parts(int64_t T, int64_t* rows_per) {
+  int64_t g = (T + 15) / 16;
+  g = g < 1 ? 1 : (g > kTailParts ? kTailParts : g);
+  *rows_per = (T + g - 1) / g;
+  return static_cast<int>((T + *rows_per - 1) / *rows_per);
+}
+}  // namespace
 
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
                         const void* z, int64_t ld_z, void* dz, int64_t ld_dz, cudaStream_t st) {
@@ -415,6 +508,43 @@ cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const flo
   if (act_dt == kDtBF16)
     return launch_pdl(dz_assemble_kernel<kDtBF16>, dim3(blocks), dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t rows_to_f16_colsum(int64_t T, int D, int in_dt, const void* in, void* out, float* partial, int* parts,
+                               cudaStream_t st) {
+  *parts = 0;
+  if (T == 0) return cudaSuccess;
+  int64_t rows_per = 0;
+  const int g = tail_parts(T, &rows_per);
+  *parts = g;
+#define HSTU_RC(DD, IT)                                                                                          \
+  if (D == DD && in_dt == IT)                                                                                    \
+    return launch_pdl(rows_to_f16_colsum_kernel<DD, IT>, dim3(g), dim3(kTailThreads), 0, st, T, in, out, rows_per, \
+                      partial);
+  HSTU_RC(256, kDtF32)
+  HSTU_RC(512, kDtF32)
+  HSTU_RC(256, kDtBF16)
+  HSTU_RC(512, kDtBF16)
+  HSTU_RC(256, kDtF16)
+  HSTU_RC(512, kDtF16)
+#undef HSTU_RC
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t colsum_final_multi(const ColsumJob* jobs, int njobs, cudaStream_t st) {
+  ColsumJobs cj{};
+  int nb = 0, k = 0;
+  for (int j = 0; j < njobs && j < 4; ++j) {
+    if (jobs[j].cols <= 0) continue;
+    cj.job[k] = jobs[j];
+    cj.first_block[k] = nb;
+    nb += (jobs[j].cols + 31) / 32;
+    ++k;
+  }
+  if (k == 0) return cudaSuccess;
+  cj.first_block[k] = nb;
+  cj.njobs = k;
+  return launch_pdl(colsum_final_multi_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, st, cj);
 }
 
 struct ConvertBatch {
