@@ -51,10 +51,15 @@ constexpr int kSiluThreadsB = 32 * kSiluWarpsB;
 __global__ void __launch_bounds__(kBiasThreads)
 attn_bias_t_kernel(AttnBwdArgs A) {
   pdl_enter();
-  const long long tile0 = blockIdx.x * static_cast<long long>(kQTile * kQTile);
-  const long long btile = (blockIdx.x * static_cast<long long>(A.f.bias_heads) + blockIdx.z) * (kQTile * kQTile);
-  bias_tile_block<true, true>(A.f, blockIdx.x, blockIdx.y, blockIdx.z, reinterpret_cast<uint16_t*>(A.bias_t) + btile,
-                              reinterpret_cast<uint8_t*>(A.bucket_t) + tile0);
+  // pairs blockIdx.x, + gridDim.x, ... up to the batch's last one
+  for (long long p = blockIdx.x; p < A.f.max_pairs; p += gridDim.x) {
+    const long long tile0 = p * static_cast<long long>(kQTile * kQTile);
+    const long long btile = (p * A.f.bias_heads + blockIdx.z) * (kQTile * kQTile);
+    if (!bias_tile_block<true, true>(A.f, p, blockIdx.y, blockIdx.z, reinterpret_cast<uint16_t*>(A.bias_t) + btile,
+                                     reinterpret_cast<uint8_t*>(A.bucket_t) + tile0))
+      break;
+    __syncthreads();
+  }
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -488,14 +493,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 //   [bucket][lane] shared histogram, whose rows are then summed and added to the table.
 constexpr int kTgThreads = 256;
 
+// One causal tile pair (row block yblk, table slice hb) of attn_table_grad_kernel; false when `pair`
+// is past the batch's last pair.
 template <bool F16>
-__global__ void __launch_bounds__(kTgThreads)
-attn_table_grad_kernel(AttnBwdArgs A) {
-  pdl_enter();
+__device__ __forceinline__ bool table_grad_pair(const AttnBwdArgs& A, long long pair, int yblk, int hb) {
   const AttnArgs& a = A.f;
   int b, qt, kt;
-  if (!decode_tile_pair(blockIdx.x, a.pair_base, a.B, &b, &qt, &kt)) return;
-  if (a.pack && a.pack[b] == 0) return;   // a packed sequence's own pair: its pack's tile holds its rows
+  if (!decode_tile_pair(pair, a.pair_base, a.B, &b, &qt, &kt)) return false;
+  if (a.pack && a.pack[b] == 0) return true;   // a packed sequence's own pair: its pack's tile holds its rows
   __shared__ float s_win[8][256];
   __shared__ float s_hist[128][32];
   __shared__ float s_thist[16 * 16];
@@ -503,7 +508,6 @@ attn_table_grad_kernel(AttnBwdArgs A) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   // table slice hb: with tables shared by the heads (bias_heads 1) the block sums all H heads, with
   // per-head tables only head hb
-  const int hb = blockIdx.z;
   const int h_lo = a.bias_heads > 1 ? hb : 0, h_hi = a.bias_heads > 1 ? hb + 1 : a.H;
   const int nt = a.n_types;
   for (int e = tid; e < 8 * 256; e += kTgThreads) (&s_win[0][0])[e] = 0.0f;
@@ -516,8 +520,7 @@ attn_table_grad_kernel(AttnBwdArgs A) {
       tile_types_load(s_ty, a.token_type, seq0, n, qt * kQTile, kt * kQTile, nt, nullptr);
   }
   const int g = lane >> 4, c0 = 8 * (lane & 15);
-  const int j0 = 64 * static_cast<int>(blockIdx.y) + 8 * w + g;   // row of k = 0; row k is j0 + 2k
-  const long long pair = blockIdx.x;
+  const int j0 = 64 * yblk + 8 * w + g;   // row of k = 0; row k is j0 + 2k
   const uint16_t* src = reinterpret_cast<const uint16_t*>(A.dxt) + pair * a.H * (kQTile * kQTile) +
                         static_cast<long long>(j0) * kQTile + c0;
   float acc[4][8];
@@ -631,6 +634,18 @@ attn_table_grad_kernel(AttnBwdArgs A) {
   }
   if (nt > 0 && tid < nt * nt && s_thist[tid] != 0.0f)
     atomicAdd(A.drab_type + static_cast<long long>(hb) * nt * nt + tid, s_thist[tid]);
+  return true;
+}
+
+// Pairs blockIdx.x, + gridDim.x, ... up to the batch's last one (the grid is sized for the SMs).
+template <bool F16>
+__global__ void __launch_bounds__(kTgThreads)
+attn_table_grad_kernel(AttnBwdArgs A) {
+  pdl_enter();
+  for (long long p = blockIdx.x; p < A.f.max_pairs; p += gridDim.x) {
+    if (!table_grad_pair<F16>(A, p, static_cast<int>(blockIdx.y), static_cast<int>(blockIdx.z))) break;
+    __syncthreads();   // the shared windows and histograms are reused by the next pair
+  }
 }
 
 }  // namespace
@@ -642,7 +657,8 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  e = launch_pdl(attn_bias_t_kernel, dim3(static_cast<unsigned>(a.max_pairs), 4, static_cast<unsigned>(a.bias_heads)),
+  e = launch_pdl(attn_bias_t_kernel, dim3(static_cast<unsigned>(bias_grid_pairs(a.max_pairs, a.bias_heads)), 4,
+                                          static_cast<unsigned>(a.bias_heads)),
                  dim3(kBiasThreads), 0, st, A);
   if (e != cudaSuccess) return e;
   // TMA row coordinates of the bias and dX^T tiles are 32-bit
@@ -669,7 +685,8 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (e == cudaSuccess) e = prof_record(kProfAttnBwd, true, st);
   if (e != cudaSuccess) return e;
   auto tg = f16 ? attn_table_grad_kernel<true> : attn_table_grad_kernel<false>;
-  return launch_pdl(tg, dim3(static_cast<unsigned>(a.max_pairs), 2, static_cast<unsigned>(a.bias_heads)),
+  return launch_pdl(tg, dim3(static_cast<unsigned>(bias_grid_pairs(a.max_pairs, a.bias_heads) * 2), 2,
+                             static_cast<unsigned>(a.bias_heads)),
                     dim3(kTgThreads), 0, st, A);
 }
 

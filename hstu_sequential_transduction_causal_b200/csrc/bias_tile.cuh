@@ -113,9 +113,10 @@ __device__ __forceinline__ void tile_types_load(int* ty, const int32_t* __restri
 // a tile, so that a batch of a few hundred pairs still puts several blocks on every SM). With per-head
 // tables (bias_heads = H) every head has its own tile; with a type term each element also adds
 // rab_type[type_query][type_key]. BUCKETS: also the u8 bucket tile (head-independent, written by the
-// hb = 0 blocks).
+// hb = 0 blocks). False when `pair` is past the batch's last pair. A block that calls it again must
+// synchronise first (the staging arrays are reused).
 template <bool TRANSPOSED, bool BUCKETS>
-__device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pair, int rb, int hb,
+__device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, long long pair, int rb, int hb,
                                                 uint16_t* __restrict__ tile, uint8_t* __restrict__ btile) {
   __shared__ TileTimes s_t;
   __shared__ long long s_tau[kTauEntries];
@@ -125,8 +126,8 @@ __device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pai
   __shared__ float s_tt[16 * 16];
   int b, qt, kt, n;
   long long seq0;
-  if (!decode_tile_pair(pair, a.pair_base, a.B, &b, &qt, &kt)) return;
-  if (!pair_rows(a.offsets, a.pack, b, &seq0, &n)) return;   // a packed sequence's own pair: unused
+  if (!decode_tile_pair(pair, a.pair_base, a.B, &b, &qt, &kt)) return false;
+  if (!pair_rows(a.offsets, a.pack, b, &seq0, &n)) return true;   // a packed sequence's own pair: unused
   const int tid = threadIdx.x;
   const int L = a.pos_max_len, nt = a.n_types;
   const float* rab_pos = a.rab_pos + static_cast<long long>(hb) * (2 * L - 1);
@@ -183,6 +184,7 @@ __device__ __forceinline__ void bias_tile_block(const AttnArgs& a, long long pai
   };
   if (fast) row_pass(BoolTag<true>{});
   else row_pass(BoolTag<false>{});
+  return true;
 }
 
 }  // namespace
