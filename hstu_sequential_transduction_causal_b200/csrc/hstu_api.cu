@@ -133,10 +133,10 @@ LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) 
   w.dv = take(T * D * 4);
   w.dz = take(T * 4 * D * 2);
   // partial column sums: db2 (from the fp16 copy of dY), dgamma | dbeta (LayerNorm backward), db1
-  // (column sum of dZ)
+  // (dZ assembly, one row per 32 tokens)
   w.part_dy = take(static_cast<size_t>(kTailParts) * D * 4);
   w.part_ln = take(static_cast<size_t>(norm_gate_bwd_blocks(j->T)) * 2 * D * 4);
-  w.part_dz = take(colsum_partial_floats(static_cast<int>(4 * D)) * 4);
+  w.part_dz = take(static_cast<size_t>((j->T + 31) / 32) * 4 * D * 4);
   w.dy_f16 = take(T * D * 2);
   w.x_f16 = take(T * D * 2);
   w.w1_f16 = take(4 * D * D * 2);
@@ -938,9 +938,13 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
     e = cudaEventRecord(g_ready_events[0], st);
     if (e != cudaSuccess) return cuda_status(e);
   }
-  // 4. SiLU backward into dZ[:, D:4D], db1 = sum_t dZ
-  e = dz_assemble(T, D, kDtF16, dv, dq, dk, saved->z, 4ll * D, dz, 4ll * D, st);
-  if (e == cudaSuccess) e = column_sum(dz, kDtF16, T, 4 * D, 4ll * D, part_dz, gr->db1, st);
+  // 4. SiLU backward into dZ[:, D:4D] with the partial sums of db1 = sum_t dZ, then their finish
+  int parts_dz = 0;
+  e = dz_assemble(T, D, kDtF16, dv, dq, dk, saved->z, 4ll * D, dz, 4ll * D, part_dz, &parts_dz, st);
+  if (e == cudaSuccess) {
+    const ColsumJob job{part_dz, 4ll * D, parts_dz, 4 * D, gr->db1};
+    e = colsum_final_multi(&job, 1, st);
+  }
   // 5. f1 backward: dW1 = dZ^T X, dX = dY + dZ W1 (fp16 dZ, x and W1)
   if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW1, 0, sizeof(float) * 4 * D * D, st);
   if (e == cudaSuccess) {

@@ -236,8 +236,11 @@ cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const f
                           const void* zu, int64_t ld_act, const float* gamma, const float* beta, const float* mu,
                           const float* rstd, void* d_o, void* dz, int64_t ld_dz, float* partial, int* parts,
                           cudaStream_t st, int* status = nullptr);
+// dZ[:, D:4D] = [dV | dQ | dK] (.) SiLU'(Z[:, D:4D]) in fp16 and the partial column sums of all of
+// dZ (dZ[:, 0:D] already written) into partial [*parts = ceil(T / 32), 4D]; D a multiple of 64.
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
-                        const void* z, int64_t ld_z, void* dz, int64_t ld_dz, cudaStream_t st);
+                        const void* z, int64_t ld_z, void* dz, int64_t ld_dz, float* partial, int* parts,
+                        cudaStream_t st);
 // [T, D] rows (fp32, bf16 or fp16) to fp16 (out may be null) and their partial column sums into
 // partial [*parts, D] (at most kTailParts rows).
 cudaError_t rows_to_f16_colsum(int64_t T, int D, int in_dt, const void* in, void* out, float* partial, int* parts,

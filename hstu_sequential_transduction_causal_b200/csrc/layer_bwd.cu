@@ -253,26 +253,58 @@ norm_gate_bwd_staged_kernel(int64_t T, const float* __restrict__ dg, const float
   }
 }
 
-// dZ[:, D:4D] = [dV | dQ | dK] (.) SiLU'(Z[:, D:4D]) in fp16; g* are fp32 [T, D].
+// dZ[:, D:4D] = [dV | dQ | dK] (.) SiLU'(Z[:, D:4D]) in fp16 (g* are fp32 [T, D]), together with the
+// partial column sums of all of dZ (the db1 of f1's bias). A block covers 32 rows x 64 columns of
+// dZ: warp w takes rows 4w .. 4w+3, lane l row 4w + l / 8 and columns 8 (l % 8) .. +7, so each row's
+// 64 columns are one coalesced access. Columns [0, D) (dZ_U, written by the LayerNorm backward) are
+// only read back for their sums. The block's 32 rows are summed by shuffles (the 4 rows of a warp)
+// and shared memory (the 8 warps) into partial[row block][cols]; the sums are of the fp16 values
+// stored. Block b covers column block b % (4D / 64) of row block b / (4D / 64).
 template <int AT>
 __global__ void __launch_bounds__(256)
 dz_assemble_kernel(int64_t T, int D, const float* __restrict__ dv, const float* __restrict__ dq,
                    const float* __restrict__ dk, const void* __restrict__ z, int64_t ld_z, void* __restrict__ dz,
-                   int64_t ld_dz) {
+                   int64_t ld_dz, float* __restrict__ partial) {
+  __shared__ float s_red[8][64];
   pdl_enter();
-  const int64_t idx = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 8;   // over T x 3D
-  const int64_t per_row = 3ll * D;
-  if (idx >= T * per_row) return;
-  const int64_t row = idx / per_row;
-  const int c = static_cast<int>(idx - row * per_row);   // multiple of 8, block of 8 inside one of V|Q|K
-  const int blk = c / D, cc = c - blk * D;
-  const float* g = blk == 0 ? dv : (blk == 1 ? dq : dk);
-  float gv[8], zv[8];
-  load_vec<8, kDtF32>(g, row * D + cc, gv);
-  load_vec<8, AT>(z, row * ld_z + D + c, zv);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ncb = 4 * D / 64;
+  const int cb = static_cast<int>(blockIdx.x % ncb);
+  const int64_t rb = blockIdx.x / ncb;
+  const int c = 64 * cb + 8 * (lane & 7);   // column of dZ, in [0, 4D)
+  const int64_t row = 32 * rb + 4 * warp + (lane >> 3);
+  float v[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) gv[e] *= silu_grad(zv[e]);
-  store_vec<8, kDtF16>(dz, row * ld_dz + D + c, gv);
+  for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+  if (row < T) {
+    if (c < D) {
+      load_vec<8, kDtF16>(dz, row * ld_dz + c, v);
+    } else {
+      const int blk = (c - D) / D, cc = (c - D) - blk * D;
+      const float* g = blk == 0 ? dv : (blk == 1 ? dq : dk);
+      float zv[8];
+      load_vec<8, kDtF32>(g, row * D + cc, v);
+      load_vec<8, AT>(z, row * ld_z + c, zv);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __half2float(__float2half_rn(v[e] * silu_grad(zv[e])));
+      store_vec<8, kDtF16>(dz, row * ld_dz + c, v);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    v[e] += __shfl_xor_sync(0xffffffffu, v[e], 8);
+    v[e] += __shfl_xor_sync(0xffffffffu, v[e], 16);
+  }
+  if (lane < 8)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s_red[warp][8 * lane + e] = v[e];
+  __syncthreads();
+  if (threadIdx.x < 64) {
+    float t = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += s_red[w][threadIdx.x];
+    partial[rb * 4 * D + 64 * cb + threadIdx.x] = t;
+  }
 }
 
 // dY converted to fp16 (out, may be null when the caller holds an fp16 copy) and the partial column
@@ -499,14 +531,20 @@ int tail_parts(int64_t T, int64_t* rows_per) {
 }  // namespace
 
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
-                        const void* z, int64_t ld_z, void* dz, int64_t ld_dz, cudaStream_t st) {
-  const int64_t threads = T * 3ll * D / 8;
-  if (threads == 0) return cudaSuccess;
-  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+                        const void* z, int64_t ld_z, void* dz, int64_t ld_dz, float* partial, int* parts,
+                        cudaStream_t st) {
+  *parts = static_cast<int>((T + 31) / 32);
+  if (T == 0) return cudaSuccess;
+  if (D % 64) return cudaErrorInvalidValue;
+  const int64_t blocks = static_cast<int64_t>(4 * D / 64) * *parts;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(blocks));
   if (act_dt == kDtF16)
-    return launch_pdl(dz_assemble_kernel<kDtF16>, dim3(blocks), dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz);
+    return launch_pdl(dz_assemble_kernel<kDtF16>, grid, dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz,
+                      partial);
   if (act_dt == kDtBF16)
-    return launch_pdl(dz_assemble_kernel<kDtBF16>, dim3(blocks), dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz);
+    return launch_pdl(dz_assemble_kernel<kDtBF16>, grid, dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz,
+                      partial);
   return cudaErrorInvalidValue;
 }
 
