@@ -4,14 +4,17 @@
 // in tensor memory.
 // Each operand is either K-major (row-major [rows, K]) or MN-major (row-major [K, rows]), so the
 // forward projections (X W1^T, G W2^T) and the backward ones (dY W2, dZ W1, dY^T G, dZ^T X)
-// share one kernel. Operand tiles arrive by TMA (128-byte swizzle) into a STAGES-deep ring; one
-// thread issues tcgen05.mma (M=128, N=BN, K=16) into TMEM; four warps run the fused epilogue:
+// share one kernel. Operand tiles arrive by TMA (128-byte swizzle) into a 4-deep ring; one thread
+// issues tcgen05.mma (M=128, N=256, K=16) into TMEM; eight warps run the fused epilogue:
 //   SILU:   Z = acc + b;  out0 = SiLU(Z) (the U|V|Q|K activations), out1 = Z (optional)
 //   LINEAR: Y = acc (+ b) (+ R);  out0 = Y, out1 = a second copy of Y in out1's dtype (optional;
 //           the fp16 copy a stacked layer's f1 reads)
 //   ATOMIC: out0 += acc (fp32 reductions for split-K weight gradients)
 // ("4.4 Scaling Recommendation Models", Generative Recommenders and HSTU: f1 with phi1 = SiLU
 // and the split into U, V, Q, K; f2 followed by the residual of the "Code" sketch.)
+// One launch can run two independent products (the backward's dY W2 with dY^T G, and dZ W1 with
+// dZ^T X): their work units share the persistent CTAs, taken largest first from a global counter,
+// so neither product's last partial wave leaves SMs idle.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -28,29 +31,74 @@ namespace hstu {
 namespace {
 
 constexpr int kBM = 128;
+constexpr int kBN = 256;        // every tile is 128 x 256: one tcgen05.mma (M=128, K=16) costs the
+                                // same issue time at N = 64, 128 or 256, so N = 256 is the only
+                                // width that runs the tensor pipe at full rate
 constexpr int kBK = 64;
+constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;    // 2 per TMEM lane quadrant, each on half of the tile's columns
-constexpr int kThreads = 32 * (kEpiWarps + 2);   // warps 0-7 epilogue, warp 8 TMA, warp 9 MMA
+constexpr int kProdWarp0 = kEpiWarps;            // warps 8-11: TMA producers, one per stage slot
+constexpr int kMmaWarp = kProdWarp0 + kStages;   // warp 12: MMA issue
+constexpr int kSchedWarp = kMmaWarp + 1;         // warp 13: work-unit scheduler
+constexpr int kThreads = 32 * (kSchedWarp + 1);
 constexpr int kBoxBytes = 4096; // one epilogue staging box: 32 rows x 128 bytes
+constexpr int kRing = 8;        // work-unit ring between the scheduler and the other roles
+constexpr int kRingReaders = kStages + 1 + kEpiWarps;
 
-template <int BN, int STAGES>
 struct GemmSmem {
   static constexpr int kABytes = kBM * kBK * 2;      // 16 KB
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kBBytes = kBN * kBK * 2;      // 32 KB
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kTileBytes = STAGES * kStageBytes;
-  static constexpr int kOut = kTileBytes;            // 8 epilogue warps x 2 staging boxes
-  static constexpr int kBarOff = kOut + kEpiWarps * 2 * kBoxBytes;
-  static constexpr int kTotal = kBarOff + 256 + 1024;   // barriers + alignment slack
+  static constexpr int kOut = kStages * kStageBytes;  // one staging box per epilogue warp
+  static constexpr int kBarOff = kOut + kEpiWarps * kBoxBytes;
+  // full[S] | empty[S] | acc_full[2] | acc_empty[2] | ring_full[R] | ring_empty[R] | ring_got[R]
+  static constexpr int kNumBars = 2 * kStages + 4 + 3 * kRing;
+  static constexpr int kMiscOff = kBarOff + 8 * kNumBars;   // tmem slot, abort flag, ring[R]
+  static constexpr int kTotal = kMiscOff + 8 + 4 * kRing + 1024;   // + alignment slack
 };
+static_assert(GemmSmem::kTotal <= 232448, "shared memory per CTA");
 
 __host__ __device__ __forceinline__ int dt_size(int dt) { return dt == kDtF32 ? 4 : 2; }
 
-struct GemmParams {
-  int M, N, num_kb, kb_per, tiles_n, splits, total;
+// One GEMM of a launch. Its work units are (m tile, n tile, k split) triples, k split fastest.
+struct GemmProb {
+  int M, N, num_kb, kb_per, tiles_n, splits, units;
+  int a_mn, b_mn;
   uint32_t idesc;
   GemmEpilogue epi;
 };
+
+// The tensor maps of one problem (TMA reads them from kernel parameter space).
+struct GemmMaps {
+  CUtensorMap a, b, o0, o1;
+};
+
+// A launch runs one or two independent GEMMs: units [0, p[0].units) are the first problem's,
+// the rest the second's. With `sched` the CTAs take units from a global counter (largest units
+// should come first); without it CTA c runs units c, c + grid, c + 2 grid, ...
+struct GemmLaunch {
+  GemmProb p[2];
+  int nprob, total;
+  int* sched;   // [0] next unit, [1] CTAs finished; zero between launches (the last CTA resets them)
+};
+
+struct Unit {
+  int prob, m0, n0, kb0, kb1;
+};
+
+__device__ __forceinline__ Unit decode_unit(const GemmLaunch& L, int u) {
+  Unit w;
+  w.prob = (L.nprob > 1 && u >= L.p[0].units) ? 1 : 0;
+  const GemmProb& q = L.p[w.prob];
+  const int t = w.prob ? u - L.p[0].units : u;
+  const int ks = t % q.splits;
+  const int rest = t / q.splits;
+  w.n0 = (rest % q.tiles_n) * kBN;
+  w.m0 = (rest / q.tiles_n) * kBM;
+  w.kb0 = ks * q.kb_per;
+  w.kb1 = min(q.num_kb, w.kb0 + q.kb_per);
+  return w;
+}
 
 __device__ __forceinline__ void load_row32(const void* in, int dt, float* v) {
   if (dt == kDtF32) {
@@ -88,30 +136,27 @@ __device__ __forceinline__ float load_one(const void* base, int dt, int64_t idx)
   return __half2float(reinterpret_cast<const __half*>(base)[idx]);
 }
 
-// Per-warp epilogue staging: boxes of 32 rows x 128 bytes in the 128-byte swizzled layout of the
+// Per-warp epilogue staging: one box of 32 rows x 128 bytes in the 128-byte swizzled layout of the
 // output tensor maps, written row-per-lane (16-byte units XOR-ed with the row: conflict-free) and
-// sent by TMA (store or fp32 reduce-add), two boxes in flight per warp. Box slot i is sent by lane i
-// (a thread keeps about one bulk copy in flight, so the two slots' copies overlap).
+// sent by TMA (store or fp32 reduce-add) from lane 0, which first waits until its previous box has
+// been read out of shared memory.
 struct EpiStage {
-  uint8_t* base;   // this warp's 2 boxes
-  int slot;
+  uint8_t* box;
   __device__ __forceinline__ void emit(const CUtensorMap* map, bool reduce, int x, int y, const uint32_t* w) {
     const int lane = threadIdx.x & 31;
-    if (lane == slot) bulk_wait_group_read<0>();   // this slot's previous box has been read
+    if (lane == 0) bulk_wait_group_read<0>();
     __syncwarp();
-    uint8_t* box = base + slot * kBoxBytes;
     uint8_t* row = box + lane * 128;
 #pragma unroll
     for (int u = 0; u < 8; ++u)
       *reinterpret_cast<uint4*>(row + ((u ^ (lane & 7)) << 4)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
     fence_proxy_async_smem();
     __syncwarp();
-    if (lane == slot) {
+    if (lane == 0) {
       if (reduce) tma_reduce_add_2d(map, smem_u32(box), x, y);
       else tma_store_2d(map, smem_u32(box), x, y);
       bulk_commit_group();
     }
-    slot ^= 1;
   }
 };
 
@@ -136,43 +181,65 @@ __device__ __forceinline__ void emit64(EpiStage& es, const CUtensorMap* map, int
   }
 }
 
-// Persistent tensor-core GEMM: CTAs stride over (m tile, n tile, k split) work items; the
-// accumulator is double-buffered in TMEM so the epilogue of one tile overlaps the next tile's
-// mainloop.
-template <int BN, int STAGES, bool A_MN, bool B_MN>
+// Persistent tensor-core GEMM over the work units of one or two problems. Roles of a CTA:
+//   warps 0-7   epilogue: TMEM -> registers -> fused epilogue -> TMA stores
+//   warps 8-11  TMA producers, warp 8 + s filling stage slot s (separate warps keep the copies of
+//               several stages in flight at once; one issuing warp serialises them)
+//   warp 12     one thread issues tcgen05.mma (M=128, N=256, K=16) into a double-buffered TMEM
+//               accumulator, so the epilogue of one unit overlaps the next unit's mainloop
+//   warp 13     scheduler (dynamic mode): takes the CTA's next unit from the global counter one unit
+//               ahead of the producers and publishes it to the other roles through a ring
+// 14 warps put 4 warps on some SM sub-partitions (16,384 registers each): 128 registers a thread
 __global__ void __launch_bounds__(kThreads, 1)
-gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
-                    GemmParams P, WaitCtl ctl) {
+gemm_bf16_tc_kernel(const __grid_constant__ GemmMaps m0, const __grid_constant__ GemmMaps m1,
+                    const __grid_constant__ GemmLaunch L, WaitCtl ctl) {
   pdl_enter();
-  using L = GemmSmem<BN, STAGES>;
+  using S = GemmSmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  // [0, STAGES) full | [STAGES, 2 STAGES) empty | 2 STAGES + b: accumulator b full | + 2: empty
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
+  auto full = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty = [&](int s) { return smem_u32(&bars[kStages + s]); };
+  auto acc_full = [&](int b) { return smem_u32(&bars[2 * kStages + b]); };
+  auto acc_empty = [&](int b) { return smem_u32(&bars[2 * kStages + 2 + b]); };
+  auto ring_full = [&](int r) { return smem_u32(&bars[2 * kStages + 4 + r]); };
+  auto ring_empty = [&](int r) { return smem_u32(&bars[2 * kStages + 4 + kRing + r]); };
+  auto ring_got = [&](int r) { return smem_u32(&bars[2 * kStages + 4 + 2 * kRing + r]); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto acc_full = [&](int b) { return smem_u32(&bars[2 * STAGES + b]); };
-  auto acc_empty = [&](int b) { return smem_u32(&bars[2 * STAGES + 2 + b]); };
+  volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const bool dynamic = L.sched != nullptr;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2 * STAGES; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(full(i), 1);
+      mbar_init(empty(i), 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(acc_full(b), 1);
       mbar_init(acc_empty(b), 32 * kEpiWarps);
     }
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(ring_full(r), 1);
+      mbar_init(ring_empty(r), kRingReaders);
+      mbar_init(ring_got(r), 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kEpiWarps && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+  if (warp == kProdWarp0 && lane == 0) {
+    tma_prefetch_desc(&m0.a);
+    tma_prefetch_desc(&m0.b);
+    if (L.nprob > 1) {
+      tma_prefetch_desc(&m1.a);
+      tma_prefetch_desc(&m1.b);
+    }
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_slot), 2 * BN);
+    tmem_alloc(smem_u32(tmem_slot), 2 * kBN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -180,114 +247,149 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   tc_fence_after();
   const uint32_t tmem_acc = *tmem_slot;
 
-  auto decode = [&](int t, int& m0, int& n0, int& kb0, int& kb1) {
-    const int ks = t % P.splits;
-    const int rest = t / P.splits;
-    n0 = (rest % P.tiles_n) * BN;
-    m0 = (rest / P.tiles_n) * kBM;
-    kb0 = ks * P.kb_per;
-    kb1 = min(P.num_kb, kb0 + P.kb_per);
+  // Unit i of this CTA, for one reading thread (false: the wait gave up). In dynamic mode the
+  // reader frees the ring slot as soon as it holds the value; producer warp 0 also tells the
+  // scheduler that it started the unit, which paces the next take from the global counter.
+  auto take_unit = [&](int i, int& u) -> bool {
+    if (!dynamic) {
+      u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+      return true;
+    }
+    const int r = i % kRing;
+    if (!mbar_wait(ring_full(r), (i / kRing) & 1, abort_flag, ctl)) return false;
+    u = ring[r];
+    mbar_arrive(ring_empty(r));
+    if (warp == kProdWarp0) mbar_arrive(ring_got(r));
+    return true;
+  };
+  // the same for a whole warp (lane 0 reads, every lane gets the result)
+  auto take_unit_warp = [&](int i, int& u) -> bool {
+    int v = 0;
+    bool ok = true;
+    if (lane == 0) ok = take_unit(i, v);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    u = __shfl_sync(0xffffffffu, v, 0);
+    return ok;
   };
 
-  if (warp == kEpiWarps) {
-    // TMA producer. A thread keeps about one tile load in flight (measured: one 16 KB box per
-    // ~550 cycles per issuing thread, 3x that from 4 lanes), so the boxes of a stage are issued by
-    // different lanes: box i of stage s by lane s * boxes + i (A: 1 K-major box or 2 MN-major halves;
-    // B: 1 K-major box or BN / 64 MN-major boxes). Lane 0 waits for the stage and registers the
-    // bytes first.
-    constexpr int kABoxes = A_MN ? 2 : 1;
-    constexpr int kBoxes = kABoxes + (B_MN ? BN / 64 : 1);
-    static_assert(kBoxes * STAGES <= 32, "one lane per box of every stage");
+  if (warp >= kProdWarp0 && warp < kMmaWarp) {
+    // producer of stage slot s: the CTA's k-blocks g (counted over all its units) with g % S == s
+    const int s = warp - kProdWarp0;
     int g = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; ok && t < P.total; t += gridDim.x) {
-      int m0, n0, kb0, kb1;
-      decode(t, m0, n0, kb0, kb1);
-      for (int kb = kb0; kb < kb1; ++kb, ++g) {
-        const int s = g % STAGES;
+    for (int i = 0;; ++i) {
+      int u;
+      if (!take_unit_warp(i, u) || u >= L.total) break;
+      const Unit w = decode_unit(L, u);
+      const GemmProb& q = L.p[w.prob];
+      const GemmMaps& mp = w.prob ? m1 : m0;
+      const int nkb = w.kb1 - w.kb0;
+      const int a_boxes = q.a_mn ? 2 : 1;                 // A: 1 K-major box or 2 MN-major halves
+      const int boxes = a_boxes + (q.b_mn ? kBN / 64 : 1);   // B: 1 K-major box or 4 MN-major boxes
+      bool ok = true;
+      for (int j = (s - g % kStages + kStages) % kStages; j < nkb; j += kStages) {
+        const int gg = g + j;
         bool free_ok = true;   // lane 0 waits; the result is made warp-uniform
-        if (lane == 0 && g >= STAGES)
-          free_ok = mbar_wait(smem_u32(&bars[STAGES + s]), ((g / STAGES) - 1) & 1, abort_flag, ctl);
+        if (lane == 0 && gg >= kStages) free_ok = mbar_wait(empty(s), ((gg / kStages) - 1) & 1, abort_flag, ctl);
         if (!__shfl_sync(0xffffffffu, free_ok ? 1 : 0, 0)) {
           ok = false;
           break;
         }
-        const uint32_t full = smem_u32(&bars[s]);
-        const uint32_t sa = smem_u32(smem + s * L::kStageBytes);
-        const uint32_t sb = sa + L::kABytes;
-        const int kx = kb * kBK;
-        if (lane == 0) mbar_arrive_expect_tx(full, L::kStageBytes);
+        const uint32_t sa = smem_u32(smem + s * S::kStageBytes);
+        const uint32_t sb = sa + S::kABytes;
+        const int kx = (w.kb0 + j) * kBK;
+        if (lane == 0) mbar_arrive_expect_tx(full(s), S::kStageBytes);
         __syncwarp();
-        // stage s's boxes come from lanes [s * kBoxes, (s + 1) * kBoxes): consecutive stages are in
-        // flight from different threads
-        const int bx = lane - s * kBoxes;
-        if (bx >= 0 && bx < kABoxes) {
-          if (!A_MN) tma_load_2d(sa, &tmA, full, kx, m0);
-          else tma_load_2d(sa + bx * 8192, &tmA, full, m0 + 64 * bx, kx);
-        } else if (bx >= kABoxes && bx < kBoxes) {
-          const int c = bx - kABoxes;
-          if (!B_MN) tma_load_2d(sb, &tmB, full, kx, n0);
-          else tma_load_2d(sb + c * 8192, &tmB, full, n0 + 64 * c, kx);
+        if (lane < a_boxes) {
+          if (!q.a_mn) tma_load_2d(sa, &mp.a, full(s), kx, w.m0);
+          else tma_load_2d(sa + lane * 8192, &mp.a, full(s), w.m0 + 64 * lane, kx);
+        } else if (lane < boxes) {
+          const int c = lane - a_boxes;
+          if (!q.b_mn) tma_load_2d(sb, &mp.b, full(s), kx, w.n0);
+          else tma_load_2d(sb + c * 8192, &mp.b, full(s), w.n0 + 64 * c, kx);
         }
       }
+      if (!ok) break;
+      g += nkb;
     }
-  } else if (warp == kEpiWarps + 1) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      // descriptors of stage 0's A and B tiles; stages and K steps are offsets from them
-      const uint32_t sa0 = smem_u32(smem), sb0 = sa0 + L::kABytes;
-      const uint64_t a_desc0 = A_MN ? make_sdesc_sw128(sa0, 8192, 1024) : make_sdesc_sw128(sa0, 16, 1024);
-      const uint64_t b_desc0 = B_MN ? make_sdesc_sw128(sb0, 8192, 1024) : make_sdesc_sw128(sb0, 16, 1024);
-      int g = 0, it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < P.total; t += gridDim.x, ++it) {
-        int m0, n0, kb0, kb1;
-        decode(t, m0, n0, kb0, kb1);
-        const int buf = it & 1;
-        if (it >= 2 && !mbar_wait(acc_empty(buf), ((it >> 1) - 1) & 1, abort_flag, ctl)) { ok = false; break; }
+      const uint32_t sa0 = smem_u32(smem), sb0 = sa0 + S::kABytes;
+      int g = 0;
+      for (int i = 0;; ++i) {
+        int u;
+        if (!take_unit(i, u) || u >= L.total) break;
+        const Unit w = decode_unit(L, u);
+        const GemmProb& q = L.p[w.prob];
+        // descriptors of stage 0's A and B tiles; stages and K steps are offsets from them
+        const uint64_t a_desc0 = q.a_mn ? make_sdesc_sw128(sa0, 8192, 1024) : make_sdesc_sw128(sa0, 16, 1024);
+        const uint64_t b_desc0 = q.b_mn ? make_sdesc_sw128(sb0, 8192, 1024) : make_sdesc_sw128(sb0, 16, 1024);
+        const uint32_t a_kstep = q.a_mn ? 2048 : 32, b_kstep = q.b_mn ? 2048 : 32;
+        const int buf = i & 1;
+        if (i >= 2 && !mbar_wait(acc_empty(buf), ((i >> 1) - 1) & 1, abort_flag, ctl)) break;
         tc_fence_after();
-        const uint32_t acc = tmem_acc + buf * BN;
-        for (int kb = kb0; kb < kb1; ++kb, ++g) {
-          const int s = g % STAGES;
-          if (!mbar_wait(smem_u32(&bars[s]), (g / STAGES) & 1, abort_flag, ctl)) { ok = false; break; }
+        const uint32_t acc = tmem_acc + buf * kBN;
+        bool ok = true;
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++g) {
+          const int s = g % kStages;
+          if (!mbar_wait(full(s), (g / kStages) & 1, abort_flag, ctl)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint64_t ad0 = sdesc_add(a_desc0, s * L::kStageBytes);
-          const uint64_t bd0 = sdesc_add(b_desc0, s * L::kStageBytes);
+          const uint64_t ad0 = sdesc_add(a_desc0, s * S::kStageBytes);
+          const uint64_t bd0 = sdesc_add(b_desc0, s * S::kStageBytes);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_f16_ss(acc, sdesc_add(ad0, A_MN ? kk * 2048 : kk * 32), sdesc_add(bd0, B_MN ? kk * 2048 : kk * 32),
-                        P.idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
-          umma_commit(smem_u32(&bars[STAGES + s]));
+            umma_f16_ss(acc, sdesc_add(ad0, kk * a_kstep), sdesc_add(bd0, kk * b_kstep), q.idesc,
+                        (kb > w.kb0 || kk > 0) ? 1u : 0u);
+          umma_commit(empty(s));
         }
-        if (ok) umma_commit(acc_full(buf));
+        if (!ok) break;
+        umma_commit(acc_full(buf));
+      }
+    }
+  } else if (warp == kSchedWarp) {
+    if (dynamic && lane == 0) {
+      for (int i = 0;; ++i) {
+        const int r = i % kRing;
+        // pace: take unit i once the producers have started unit i - 1
+        if (i >= 1 && !mbar_wait(ring_got((i - 1) % kRing), ((i - 1) / kRing) & 1, abort_flag, ctl)) break;
+        const int u = i == 0 ? static_cast<int>(blockIdx.x) : static_cast<int>(gridDim.x) + atomicAdd(L.sched, 1);
+        if (i >= kRing && !mbar_wait(ring_empty(r), ((i / kRing) - 1) & 1, abort_flag, ctl)) break;
+        ring[r] = u;
+        mbar_arrive(ring_full(r));
+        if (u >= L.total) break;
       }
     }
   } else {
     // epilogue warps 0-7: TMEM lanes 32 (warp % 4) .. +31 = output rows m0 + 32 (warp % 4) + lane,
-    // columns [BN/2 (warp / 4), +BN/2)
-    const GemmEpilogue& epi = P.epi;
+    // columns [128 (warp / 4), +128) of the tile
     const int quad = warp & 3, chalf = warp >> 2;
-    EpiStage es{smem + L::kOut + warp * 2 * kBoxBytes, 0};
-    int it = 0;
-    for (int t = blockIdx.x; t < P.total; t += gridDim.x, ++it) {
-      int m0, n0, kb0, kb1;
-      decode(t, m0, n0, kb0, kb1);
-      const int buf = it & 1;
-      if (!mbar_wait(acc_full(buf), (it >> 1) & 1, abort_flag, ctl)) break;
+    EpiStage es{smem + S::kOut + warp * kBoxBytes};
+    for (int i = 0;; ++i) {
+      int u;
+      if (!take_unit_warp(i, u) || u >= L.total) break;
+      const Unit w = decode_unit(L, u);
+      const GemmProb& q = L.p[w.prob];
+      const GemmEpilogue& epi = q.epi;
+      const GemmMaps& mp = w.prob ? m1 : m0;
+      const int buf = i & 1;
+      if (!mbar_wait(acc_full(buf), (i >> 1) & 1, abort_flag, ctl)) break;
       tc_fence_after();
-      const int row = m0 + quad * 32 + lane;
-      const bool row_ok = row < P.M;
-      const int ybox = m0 + quad * 32;
-      constexpr int kChunks = BN / 128;   // 64-column chunks per warp
+      const int row = w.m0 + quad * 32 + lane;
+      const bool row_ok = row < q.M;
+      const int ybox = w.m0 + quad * 32;
+      constexpr int kChunks = kBN / 128;   // 64-column chunks per warp
 #pragma unroll 1
       for (int c = 0; c < kChunks; ++c) {
-        const int col = chalf * (BN / 2) + c * 64;   // within the tile
-        const int n = n0 + col;
+        const int col = chalf * (kBN / 2) + c * 64;   // within the tile
+        const int n = w.n0 + col;
         float v[64];
         {
           uint32_t r[32];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            tmem_ld_32x32b_x32(tmem_acc + buf * BN + (static_cast<uint32_t>(quad * 32) << 16) + col + 32 * h, r);
+            tmem_ld_32x32b_x32(tmem_acc + buf * kBN + (static_cast<uint32_t>(quad * 32) << 16) + col + 32 * h, r);
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[32 * h + j] = __uint_as_float(r[j]);
@@ -297,17 +399,17 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           tc_fence_before();
           mbar_arrive(acc_empty(buf));
         }
-        if (n >= P.N) continue;
+        if (n >= q.N) continue;
         if (epi.kind == kEpiAtomic) {
-          emit64(es, &tmO0, kDtF32, true, n, ybox, v, P.N);
+          emit64(es, &mp.o0, kDtF32, true, n, ybox, v, q.N);
           continue;
         }
         if (epi.bias) {
           const float4* bp = reinterpret_cast<const float4*>(epi.bias + n);
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const float4 b4 = (n + 4 * q < P.N) ? __ldg(bp + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-            v[4 * q] += b4.x; v[4 * q + 1] += b4.y; v[4 * q + 2] += b4.z; v[4 * q + 3] += b4.w;
+          for (int k4 = 0; k4 < 16; ++k4) {
+            const float4 b4 = (n + 4 * k4 < q.N) ? __ldg(bp + k4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * k4] += b4.x; v[4 * k4 + 1] += b4.y; v[4 * k4 + 2] += b4.z; v[4 * k4 + 3] += b4.w;
           }
         }
         if (epi.kind == kEpiSilu) {
@@ -319,14 +421,14 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int j = 0; j < 64; ++j) in_range &= fabsf(v[j]) <= 65504.0f;
             if (!in_range) report_error(ctl.status, kDevBadInput);
           }
-          if (epi.out1) emit64(es, &tmO1, epi.out1_dt, false, n, ybox, v, P.N);
+          if (epi.out1) emit64(es, &mp.o1, epi.out1_dt, false, n, ybox, v, q.N);
 #pragma unroll
           for (int j = 0; j < 64; ++j) v[j] = silu_tanh(v[j]);
         } else if (epi.resid) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             float rv[32];
-            if (row_ok && n + 32 * h < P.N) {
+            if (row_ok && n + 32 * h < q.N) {
               const uint8_t* rp = reinterpret_cast<const uint8_t*>(epi.resid) +
                                   (static_cast<int64_t>(row) * epi.ld_resid + n + 32 * h) * dt_size(epi.resid_dt);
               load_row32(rp, epi.resid_dt, rv);
@@ -338,18 +440,27 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int j = 0; j < 32; ++j) v[32 * h + j] += rv[j];
           }
         }
-        emit64(es, &tmO0, epi.out0_dt, false, n, ybox, v, P.N);
-        if (epi.kind == kEpiLinear && epi.out1) emit64(es, &tmO1, epi.out1_dt, false, n, ybox, v, P.N);
+        emit64(es, &mp.o0, epi.out0_dt, false, n, ybox, v, q.N);
+        if (epi.kind == kEpiLinear && epi.out1) emit64(es, &mp.o1, epi.out1_dt, false, n, ybox, v, q.N);
       }
     }
-    if (lane < 2) bulk_wait_group_all();
+    if (lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem_acc, 2 * BN);
+    tmem_dealloc(tmem_acc, 2 * kBN);
+  }
+  if (dynamic && threadIdx.x == 0) {
+    // every take from the counter of this launch happened before its CTA got here: the last CTA
+    // leaves both counters at zero for the next launch that uses them
+    __threadfence();
+    if (atomicAdd(L.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      atomicExch(L.sched, 0);
+      atomicExch(L.sched + 1, 0);
+    }
   }
 }
 
@@ -415,65 +526,84 @@ gemm_f32_simt_kernel(const float* __restrict__ A, int64_t sam, int64_t sak, cons
   }
 }
 
-template <int BN, int STAGES, bool A_MN, bool B_MN>
-cudaError_t launch_tc(const GemmArgs& g, cudaStream_t st) {
-  using L = GemmSmem<BN, STAGES>;
-  CUtensorMap tmA, tmB, tmO0, tmO1;
+bool encode_problem(const GemmArgs& g, GemmMaps& m) {
   // A: K-major -> [M rows, K] box {64, 128}; MN-major -> [K rows, M] box {64, 64}
-  if (!A_MN) {
-    if (!encode_tmap_2d_bf16(&tmA, g.A, g.K, g.M, g.lda, 64, kBM, g.f16)) return cudaErrorInvalidValue;
-  } else {
-    if (!encode_tmap_2d_bf16(&tmA, g.A, g.M, g.K, g.lda, 64, 64, g.f16)) return cudaErrorInvalidValue;
+  if (!g.a_mn) {
+    if (!encode_tmap_2d_bf16(&m.a, g.A, g.K, g.M, g.lda, 64, kBM, g.f16)) return false;
+  } else if (!encode_tmap_2d_bf16(&m.a, g.A, g.M, g.K, g.lda, 64, 64, g.f16)) {
+    return false;
   }
-  if (!B_MN) {
-    if (!encode_tmap_2d_bf16(&tmB, g.B, g.K, g.N, g.ldb, 64, BN, g.f16)) return cudaErrorInvalidValue;
-  } else {
-    if (!encode_tmap_2d_bf16(&tmB, g.B, g.N, g.K, g.ldb, 64, 64, g.f16)) return cudaErrorInvalidValue;
+  // B: K-major -> [N rows, K] box {64, 256}; MN-major -> [K rows, N] box {64, 64}
+  if (!g.b_mn) {
+    if (!encode_tmap_2d_bf16(&m.b, g.B, g.K, g.N, g.ldb, 64, kBN, g.f16)) return false;
+  } else if (!encode_tmap_2d_bf16(&m.b, g.B, g.N, g.K, g.ldb, 64, 64, g.f16)) {
+    return false;
   }
   // outputs: boxes of 32 rows x 128 bytes
   const int dt0 = g.epi.kind == kEpiAtomic ? kDtF32 : g.epi.out0_dt;
-  if (!encode_tmap_2d_out(&tmO0, g.epi.out0, dt0, g.N, g.M, g.epi.ld_out0, 128 / dt_size(dt0), 32))
-    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d_out(&m.o0, g.epi.out0, dt0, g.N, g.M, g.epi.ld_out0, 128 / dt_size(dt0), 32)) return false;
   if (g.epi.out1) {
-    if (!encode_tmap_2d_out(&tmO1, g.epi.out1, g.epi.out1_dt, g.N, g.M, g.epi.ld_out1, 128 / dt_size(g.epi.out1_dt), 32))
-      return cudaErrorInvalidValue;
+    if (!encode_tmap_2d_out(&m.o1, g.epi.out1, g.epi.out1_dt, g.N, g.M, g.epi.ld_out1, 128 / dt_size(g.epi.out1_dt), 32))
+      return false;
   } else {
-    tmO1 = tmO0;
+    m.o1 = m.o0;
   }
-  auto kern = gemm_bf16_tc_kernel<BN, STAGES, A_MN, B_MN>;
-  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), L::kTotal);
-  if (e != cudaSuccess) return e;
-  GemmParams P{};
+  return true;
+}
+
+GemmProb make_prob(const GemmArgs& g) {
+  GemmProb P{};
   P.M = static_cast<int>(g.M);
   P.N = static_cast<int>(g.N);
   P.num_kb = static_cast<int>((g.K + kBK - 1) / kBK);
   const int splits = g.splits < 1 ? 1 : g.splits;
   P.kb_per = (P.num_kb + splits - 1) / splits;
   P.splits = (P.num_kb + P.kb_per - 1) / P.kb_per;
-  P.tiles_n = static_cast<int>((g.N + BN - 1) / BN);
+  P.tiles_n = static_cast<int>((g.N + kBN - 1) / kBN);
   const int tiles_m = static_cast<int>((g.M + kBM - 1) / kBM);
-  P.total = tiles_m * P.tiles_n * P.splits;
-  P.idesc = make_idesc_f16kind(kBM, BN, A_MN ? 1 : 0, B_MN ? 1 : 0, g.f16);
+  P.units = tiles_m * P.tiles_n * P.splits;
+  P.a_mn = g.a_mn ? 1 : 0;
+  P.b_mn = g.b_mn ? 1 : 0;
+  P.idesc = make_idesc_f16kind(kBM, kBN, P.a_mn, P.b_mn, g.f16);
   P.epi = g.epi;
-  const int grid = P.total < sm_count() ? P.total : sm_count();
-  return launch_pdl(kern, dim3(grid), dim3(kThreads), L::kTotal, st, tmA, tmB, tmO0, tmO1, P, wait_ctl(g.status));
-}
-
-template <int BN, int STAGES>
-cudaError_t dispatch_major(const GemmArgs& g, cudaStream_t st) {
-  if (!g.a_mn && !g.b_mn) return launch_tc<BN, STAGES, false, false>(g, st);
-  if (!g.a_mn && g.b_mn) return launch_tc<BN, STAGES, false, true>(g, st);
-  if (g.a_mn && !g.b_mn) return launch_tc<BN, STAGES, true, false>(g, st);
-  return launch_tc<BN, STAGES, true, true>(g, st);
+  return P;
 }
 
 }  // namespace
 
+cudaError_t gemm_bf16_group(const GemmArgs* gs, int n, int* sched, cudaStream_t st) {
+  if (!gs || n < 1 || n > 2) return cudaErrorInvalidValue;
+  GemmMaps maps[2];
+  GemmLaunch L{};
+  int k = 0;
+  int* status = nullptr;
+  for (int i = 0; i < n; ++i) {
+    const GemmArgs& g = gs[i];
+    if (g.M <= 0 || g.N <= 0) continue;   // an empty product: nothing to compute
+    if (g.K <= 0 || (g.splits > 1 && g.epi.kind != kEpiAtomic)) return cudaErrorInvalidValue;
+    if (!encode_problem(g, maps[k])) return cudaErrorInvalidValue;
+    L.p[k] = make_prob(g);
+    if (!status) status = g.status;
+    ++k;
+  }
+  if (k == 0) return cudaSuccess;
+  if (k == 1) maps[1] = maps[0];
+  L.nprob = k;
+  const int64_t total = static_cast<int64_t>(L.p[0].units) + (k > 1 ? L.p[1].units : 0);
+  if (total >= (1ll << 30)) return cudaErrorInvalidValue;
+  L.total = static_cast<int>(total);
+  L.sched = sched;
+  auto kern = gemm_bf16_tc_kernel;
+  cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), GemmSmem::kTotal);
+  if (e != cudaSuccess) return e;
+  const int grid = L.total < sm_count() ? L.total : sm_count();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), GemmSmem::kTotal, st, maps[0], maps[1], L, wait_ctl(status));
+}
+
 cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st) {
   if (g.M <= 0 || g.N <= 0) return cudaSuccess;
   if (g.K <= 0) return cudaErrorInvalidValue;
-  if (g.N % 256 == 0 && g.N >= 1024) return dispatch_major<256, 3>(g, st);
-  return dispatch_major<128, 4>(g, st);
+  return gemm_bf16_group(&g, 1, nullptr, st);
 }
 
 cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st) {

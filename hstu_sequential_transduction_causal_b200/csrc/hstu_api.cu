@@ -7,6 +7,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -307,15 +308,28 @@ hstu_status_t run_out_proj(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_
   return cuda_status(dtype == HSTU_BF16 ? gemm_bf16(g, st) : gemm_f32(g, st));
 }
 
-// Split-K factor that gives the accumulating GEMM about two CTAs per SM.
+// Split-K factor of an accumulating GEMM run alone: about two work units per SM (128 x 256 tiles),
+// each of at least 4 k-blocks of 64.
 int auto_splits(int64_t M, int64_t N, int64_t K) {
-  const int64_t bn = (N % 256 == 0 && N >= 1024) ? 256 : 128;
-  const int64_t tiles = ((M + 127) / 128) * ((N + bn - 1) / bn);
+  const int64_t tiles = ((M + 127) / 128) * ((N + 255) / 256);
   const int64_t nkb = (K + 63) / 64;
   int64_t s = (296 + tiles - 1) / tiles;
-  if (s > nkb) s = nkb;
+  const int64_t s_max = (nkb + 3) / 4;
+  if (s > s_max) s = s_max;
   return static_cast<int>(s < 1 ? 1 : s);
 }
+
+// Split-K factor that cuts K into work units of about `unit_kb` k-blocks of 64 (an accumulating
+// GEMM sharing a launch with a product whose units are larger).
+int splits_for_unit(int64_t K, int64_t unit_kb) {
+  const int64_t nkb = (K + 63) / 64;
+  if (unit_kb < 1) unit_kb = 1;
+  const int64_t s = (nkb + unit_kb - 1) / unit_kb;
+  return static_cast<int>(s < 1 ? 1 : s);
+}
+
+// The two scheduling counters of the grouped backward GEMMs: bytes [64, 72) of the workspace header.
+int* gemm_sched(void* ws) { return static_cast<int*>(ws) + 16; }
 
 hstu_status_t check_dense(int64_t T, int32_t D, hstu_dtype_t dtype) {
   if (T < 0 || D <= 0) return HSTU_ERR_INVALID_ARG;
@@ -903,19 +917,20 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   float* dk = reinterpret_cast<float*>(wsb + lay.dk);
   float* dv = reinterpret_cast<float*>(wsb + lay.dv);
   void* dz = wsb + lay.dz;
-  // 1. f2 backward: dG = dY W2, dW2 = dY^T G, db2 = sum_t dY
-  GemmArgs g{};
-  g.A = dy_op; g.lda = D; g.a_mn = false; g.B = w2_f16; g.ldb = D; g.b_mn = true; g.f16 = true;
-  g.M = T; g.N = D; g.K = D; g.splits = 1;
-  g.epi.kind = kEpiLinear; g.epi.out0 = dG; g.epi.out0_dt = kDtF32; g.epi.ld_out0 = D; g.status = status;
-  e = gemm_bf16(g, st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW2, 0, sizeof(float) * D * D, st);
+  // 1. f2 backward: dG = dY W2 and dW2 = dY^T G in one launch (dW2 split over K = T into units of
+  //    about half a dG unit, reduced into the zeroed dW2); db2 = sum_t dY
+  e = cudaMemsetAsync(gr->dW2, 0, sizeof(float) * D * D, st);
   if (e == cudaSuccess) {
-    GemmArgs g2{};
+    GemmArgs gg[2] = {};
+    GemmArgs& g = gg[0];
+    g.A = dy_op; g.lda = D; g.a_mn = false; g.B = w2_f16; g.ldb = D; g.b_mn = true; g.f16 = true;
+    g.M = T; g.N = D; g.K = D; g.splits = 1;
+    g.epi.kind = kEpiLinear; g.epi.out0 = dG; g.epi.out0_dt = kDtF32; g.epi.ld_out0 = D; g.status = status;
+    GemmArgs& g2 = gg[1];
     g2.A = dy_op; g2.lda = D; g2.a_mn = true; g2.B = saved->g; g2.ldb = D; g2.b_mn = true; g2.f16 = true;
-    g2.M = D; g2.N = D; g2.K = T; g2.splits = auto_splits(D, D, T);
+    g2.M = D; g2.N = D; g2.K = T; g2.splits = splits_for_unit(T, std::max<int64_t>(4, D / 128));
     g2.epi.kind = kEpiAtomic; g2.epi.out0 = gr->dW2; g2.epi.out0_dt = kDtF32; g2.epi.ld_out0 = D; g2.status = status;
-    e = gemm_bf16(g2, st);
+    e = gemm_bf16_group(gg, 2, gemm_sched(ws), st);
   }
   // 2. norm-gate backward: dO (fp16), dZ_U (fp16), partial dgamma | dbeta; then db2, dgamma and dbeta
   // finished by one launch straight into the caller's buffers
@@ -945,18 +960,16 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
     const ColsumJob job{part_dz, 4ll * D, parts_dz, 4 * D, gr->db1};
     e = colsum_final_multi(&job, 1, st);
   }
-  // 5. f1 backward: dW1 = dZ^T X, dX = dY + dZ W1 (fp16 dZ, x and W1)
+  // 5. f1 backward in one launch: dX = dY + dZ W1 and dW1 = dZ^T X (fp16 dZ, x and W1; dW1 split
+  //    over K = T into units of about a third of a dX unit, reduced into the zeroed dW1)
   if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW1, 0, sizeof(float) * 4 * D * D, st);
   if (e == cudaSuccess) {
-    GemmArgs g3{};
+    GemmArgs gg[2] = {};
+    GemmArgs& g3 = gg[1];
     g3.A = dz; g3.lda = 4ll * D; g3.a_mn = true; g3.B = x_op; g3.ldb = D; g3.b_mn = true; g3.f16 = true;
-    g3.M = 4ll * D; g3.N = D; g3.K = T; g3.splits = auto_splits(4ll * D, D, T);
+    g3.M = 4ll * D; g3.N = D; g3.K = T; g3.splits = splits_for_unit(T, std::max<int64_t>(4, D / 48));
     g3.epi.kind = kEpiAtomic; g3.epi.out0 = gr->dW1; g3.epi.out0_dt = kDtF32; g3.epi.ld_out0 = D; g3.status = status;
-    e = gemm_bf16(g3, st);
-  }
-  if (e == cudaSuccess && g_ready_events[1]) e = cudaEventRecord(g_ready_events[1], st);   // dW1, db1 final
-  if (e == cudaSuccess) {
-    GemmArgs g4{};
+    GemmArgs& g4 = gg[0];
     g4.A = dz; g4.lda = 4ll * D; g4.a_mn = false; g4.B = w1_f16; g4.ldb = D; g4.b_mn = true; g4.f16 = true;
     g4.M = T; g4.N = D; g4.K = 4ll * D; g4.splits = 1;
     g4.epi.kind = kEpiLinear;
@@ -968,8 +981,9 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
       g4.epi.out1 = dx_f16; g4.epi.out1_dt = kDtF16; g4.epi.ld_out1 = D;
     }
     g4.status = status;
-    e = gemm_bf16(g4, st);
+    e = gemm_bf16_group(gg, 2, gemm_sched(ws), st);
   }
+  if (e == cudaSuccess && g_ready_events[1]) e = cudaEventRecord(g_ready_events[1], st);   // dW1, db1 final
   if (nin && e == cudaSuccess)
     e = ln_in_bwd(T, D, desc->x_dtype == HSTU_F32 ? kDtF32 : kDtBF16, desc->y_dtype == HSTU_F32 ? kDtF32 : kDtBF16,
                   reinterpret_cast<const float*>(wsb + nin_dxn), x, dy, nin->gamma, nin->mu, nin->rstd, dx, dx_f16,

@@ -99,6 +99,11 @@ cudaError_t ensure_smem_attr(const void* kernel, int bytes);
 int sm_count();
 
 cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st);
+// Two independent products in one launch (n = 1 or 2; empty products are skipped). With `sched`
+// (two ints, zero before the first launch; each launch leaves them zero) the CTAs take work units
+// from a global counter in order, so the caller lists the product with the larger units first;
+// without it every CTA runs a fixed stride of units.
+cudaError_t gemm_bf16_group(const GemmArgs* g, int n, int* sched, cudaStream_t st);
 cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------------

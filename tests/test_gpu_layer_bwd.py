@@ -32,11 +32,20 @@ def _lib():
     torch.cuda.init()
 
 
+# (M, N, K without / with split-K accumulation): one tile row; ragged M, N and K (partial 128 x 256
+# tiles, a partial last k-block); more work units than SMs (each CTA loops over several units and
+# reuses both TMEM accumulators)
+_LINEAR_SHAPES = {"one_tile_row": (296, 256, 320, 1000), "ragged": (312, 320, 264, 1096),
+                  "many_units": (5000, 1024, 128, 2000)}
+
+
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 0), (1, 1)])
 @pytest.mark.parametrize("accumulate", [0, 1])
-def test_linear_all_operand_layouts(a_mn, b_mn, accumulate):
+@pytest.mark.parametrize("shape", list(_LINEAR_SHAPES))
+def test_linear_all_operand_layouts(a_mn, b_mn, accumulate, shape):
     rng = np.random.default_rng(10 + 2 * a_mn + b_mn)
-    M, N, K = 296, 256, 1000 if accumulate else 320
+    M, N, K0, K1 = _LINEAR_SHAPES[shape]
+    K = K1 if accumulate else K0
     A = W.round_bf16(rng.standard_normal((M, K)))
     Bm = W.round_bf16(rng.standard_normal((N, K)) / np.sqrt(K))
     bias = (0.1 * rng.standard_normal(N)).astype(np.float32)
