@@ -13,9 +13,10 @@
 // attn_bwd_tc_kernel<F16>: one CTA per (sequence, 128-key tile, head), key tiles that visit the
 // most query tiles first; it walks the query tiles t >= its key tile:
 //   warp 16  : TMA: K, V once; Q and dO of each query tile (3 stages); the half-bias tile (2).
-//   warp 17  : tcgen05: S^T = K Q^T and dA^T = V dO^T into TMEM.
-//   warp 19  : tcgen05: after the elementwise step dV += P^T dO (P^T from TMEM), dK += dX^T Q and
-//              dQ_tile = dX K (dX^T from shared memory, read K-major for dK and MN-major for dQ).
+//   warp 17  : tcgen05: S^T = K Q^T and dA^T = V dO^T into TMEM (N = 128, the whole query tile);
+//              after the elementwise step, the next tile's S^T / dA^T first, then dV += P^T dO
+//              (P^T from TMEM), dK += dX^T Q and dQ_tile = dX K (dX^T from shared memory, read
+//              K-major for dK and MN-major for dQ). Warp 19 idles.
 //   warp 18  : TMA stores: each dQ tile (staged in shared memory) reduce-added into the fp32 dQ,
 //              each tile's dX^T (16-bit, from shared memory) to the workspace.
 //   warps 0-15: key row = TMEM lane (warp & 3), query half (warp >> 2) & 1, 32 of its 64 queries
@@ -47,19 +48,11 @@ constexpr int kSiluThreadsB = 32 * kSiluWarpsB;
 // ----------------------------------------------------------------------------------------------
 // transposed bias and bucket tiles
 // ----------------------------------------------------------------------------------------------
-// Four blocks per causal tile pair: the [key][query] half-bias and u8 bucket tiles of bias_tile.cuh.
+// One block per causal tile pair (grid-stride): the [key][query] half-bias and u8 bucket tiles of
+// bias_tile.cuh.
 __global__ void __launch_bounds__(kBiasThreads)
 attn_bias_t_kernel(AttnBwdArgs A) {
-  pdl_enter();
-  // pairs blockIdx.x, + gridDim.x, ... up to the batch's last one
-  for (long long p = blockIdx.x; p < A.f.max_pairs; p += gridDim.x) {
-    const long long tile0 = p * static_cast<long long>(kQTile * kQTile);
-    const long long btile = (p * A.f.bias_heads + blockIdx.z) * (kQTile * kQTile);
-    if (!bias_tile_block<true, true>(A.f, p, blockIdx.y, blockIdx.z, reinterpret_cast<uint16_t*>(A.bias_t) + btile,
-                                     reinterpret_cast<uint8_t*>(A.bucket_t) + tile0))
-      break;
-    __syncthreads();
-  }
+  bias_tiles<true, true>(A.f, reinterpret_cast<uint16_t*>(A.bias_t), reinterpret_cast<uint8_t*>(A.bucket_t));
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -157,7 +150,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // query half h: S^T_h at columns [128 h, 128 h + 64), dA^T_h at [128 h + 64, 128 h + 128);
+  // query q of the tile: S^T at column q, dA^T at column 128 + q;
   // accumulators dV, dK and the dQ tile of one query tile; P^T_h packed two per column at
   // [448 + 32 h, 448 + 32 h + 32)
   const uint32_t tDV = tmem + 256, tDK = tmem + 320, tDQ = tmem + 384, tP = tmem + 448;
@@ -200,17 +193,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (s >= 1) ok = load_bias(s - 1);
     }
     if (ok && nsteps > 0) load_bias(nsteps - 1);
-  } else if (warp == kSiluWarpsB + 1 || warp == kSiluWarpsB + 3) {
-    // ---------------- tcgen05 issuers: S / dA (warp 17) and the gradient MMAs (warp 19) ----------------
-    // Per query tile s, in two halves of 64 queries: S^T_h = K Q_h^T and dA^T_h = V dO_h^T, then,
-    // once the elementwise warps of half h have written P^T_h (TMEM) and dX^T_h (shared memory),
-    // dV += P^T_h dO_h and dK += dX^T_h Q_h; after half b also dQ_tile = dX K. P^T has TMEM columns
-    // of its own, so the next tile's S^T_h, dA^T_h are issued (by their own thread) as soon as half
-    // h has read this tile's: the elementwise warps of half h start the next tile while the
-    // gradient MMAs (the other thread) run. Both threads' MMAs read Q / dO, so its stage is freed
-    // by two commits.
+  } else if (warp == kSiluWarpsB + 1) {
+    // ---------------- tcgen05 issuer (warp 17; warp 19 idles) ----------------
+    // Per query tile s: S^T = K Q^T and dA^T = V dO^T over the whole tile (N = 128: a tcgen05.mma
+    // costs the same issue time at N = 64 and 128, so two 64-query halves would double it); once
+    // both query halves' elementwise warps have written P^T (TMEM) and dX^T (shared memory), first
+    // the next tile's S^T / dA^T (so that its elementwise work overlaps the gradient MMAs), then
+    // dV += P^T_h dO_h and dK += dX^T_h Q_h for both halves and dQ_tile = dX K. The Q / dO stage
+    // is freed by two commits: after S^T / dA^T and after the gradient MMAs.
     if (lane == 0) {
-      constexpr uint32_t id_s = make_idesc_f16kind(128, 64, 0, 0, F16);
+      constexpr uint32_t id_s = make_idesc_f16kind(128, 128, 0, 0, F16);
       constexpr uint32_t id_kmn = make_idesc_f16kind(128, 64, 0, 1, F16);
       constexpr uint32_t id_mnmn = make_idesc_f16kind(128, 64, 1, 1, F16);
       bool ok = mbar_wait(BAR(0), 0, abort_flag, ctl);
@@ -219,19 +211,20 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint64_t k_mn = make_sdesc_sw128(sK, 16384, 1024);
       const uint64_t q_km = make_sdesc_sw128(sQ0, 16, 1024), q_mn = make_sdesc_sw128(sQ0, 16384, 1024);
       const uint64_t x_km = make_sdesc_sw128(sBT0, 16, 1024), x_mn = make_sdesc_sw128(sBT0, 16384, 1024);
-      auto issue_s = [&](int s, int hh) -> bool {
+      auto issue_s = [&](int s) -> bool {
         const int sq = s % 3;
-        if (hh == 0 && !mbar_wait(qdo_full(sq), (s / 3) & 1, abort_flag, ctl)) return false;
+        if (!mbar_wait(qdo_full(sq), (s / 3) & 1, abort_flag, ctl)) return false;
         tc_fence_after();
-        const uint64_t qd = sdesc_add(q_km, sq * 32768 + 8192 * hh), dod = sdesc_add(qd, 16384);
+        const uint64_t qd = sdesc_add(q_km, sq * 32768), dod = sdesc_add(qd, 16384);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_f16_ss(tmem + 128 * hh, sdesc_add(k_km, kk * 32), sdesc_add(qd, kk * 32), id_s, kk > 0 ? 1u : 0u);
+          umma_f16_ss(tmem, sdesc_add(k_km, kk * 32), sdesc_add(qd, kk * 32), id_s, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_f16_ss(tmem + 128 * hh + 64, sdesc_add(v_km, kk * 32), sdesc_add(dod, kk * 32), id_s,
-                      kk > 0 ? 1u : 0u);
-        umma_commit(BAR(9 + hh));
+          umma_f16_ss(tmem + 128, sdesc_add(v_km, kk * 32), sdesc_add(dod, kk * 32), id_s, kk > 0 ? 1u : 0u);
+        umma_commit(BAR(9));
+        umma_commit(BAR(10));
+        umma_commit(qdo_empty(sq));
         return true;
       };
       auto issue_grad = [&](int s, int hh) {
@@ -247,37 +240,27 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           umma_f16_ss(tDK, sdesc_add(xd, k4 * 32), sdesc_add(qd, k4 * 2048), id_kmn, k4 > 0 ? 1u : acc0);
         umma_commit(BAR(19 + hh));
       };
-      if (warp == kSiluWarpsB + 1) {
-        if (ok && nsteps > 0) {
-          ok = issue_s(0, 0) && issue_s(0, 1);
-          if (ok) umma_commit(qdo_empty(0));
+      if (ok && nsteps > 0) ok = issue_s(0);
+      for (int s = 0; ok && s < nsteps; ++s) {
+        const int st = s & 1;
+        ok = mbar_wait(BAR(11), s & 1, abort_flag, ctl) && mbar_wait(BAR(12), s & 1, abort_flag, ctl);
+        if (!ok) break;
+        tc_fence_after();
+        if (s + 1 < nsteps && !issue_s(s + 1)) {
+          ok = false;
+          break;
         }
-        for (int s = 0; ok && s + 1 < nsteps; ++s) {
-          for (int hh = 0; ok && hh < 2; ++hh)
-            ok = mbar_wait(BAR(11 + hh), s & 1, abort_flag, ctl) && issue_s(s + 1, hh);
-          if (ok) umma_commit(qdo_empty((s + 1) % 3));
-        }
-      } else {
-        for (int s = 0; ok && s < nsteps; ++s) {
-          const int st = s & 1;
-          for (int hh = 0; ok && hh < 2; ++hh) {
-            ok = mbar_wait(BAR(11 + hh), s & 1, abort_flag, ctl);
-            if (ok) {
-              tc_fence_after();
-              issue_grad(s, hh);
-            }
-          }
-          if (!ok) break;
-          const uint64_t xd = sdesc_add(x_mn, st * 32768);
+        issue_grad(s, 0);
+        issue_grad(s, 1);
+        const uint64_t xd = sdesc_add(x_mn, st * 32768);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)   // dQ_tile = dX K
-            umma_f16_ss(tDQ, sdesc_add(xd, kk * 2048), sdesc_add(k_mn, kk * 2048), id_mnmn, kk > 0 ? 1u : 0u);
-          umma_commit(BAR(13));
-          umma_commit(qdo_empty(s % 3));
-          umma_commit(BAR(7 + st));
-        }
-        if (ok) umma_commit(BAR(14));
+        for (int kk = 0; kk < 8; ++kk)   // dQ_tile = dX K
+          umma_f16_ss(tDQ, sdesc_add(xd, kk * 2048), sdesc_add(k_mn, kk * 2048), id_mnmn, kk > 0 ? 1u : 0u);
+        umma_commit(BAR(13));
+        umma_commit(qdo_empty(s % 3));
+        umma_commit(BAR(7 + st));
       }
+      if (ok) umma_commit(BAR(14));
     }
   } else if (warp == kSiluWarpsB + 2) {
     // ---------------- TMA stores ----------------
@@ -317,7 +300,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
     if (ok && nsteps > 0) reduce_dq(nsteps - 1);
     bulk_wait_group_all();
-  } else {
+  } else if (warp < kSiluWarpsB) {
     // ---------------- elementwise warps ----------------
     // warp w: key rows [32 (w & 3), +32) (TMEM lane quadrant), query half hq = (w >> 2) & 1,
     // queries [64 hq + 32 sub, +32) with sub = w >> 3
@@ -413,8 +396,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       for (int pc = 0; pc < 2; ++pc) {
         const int c0 = 64 * hq + 32 * sub + 16 * pc;   // first query column of the piece
         uint32_t sv[16], dav[16];
-        tmem_ld_32x32b_x16(tmem + lane_base + 128 * hq + 32 * sub + 16 * pc, sv);
-        tmem_ld_32x32b_x16(tmem + lane_base + 128 * hq + 64 + 32 * sub + 16 * pc, dav);
+        tmem_ld_32x32b_x16(tmem + lane_base + 64 * hq + 32 * sub + 16 * pc, sv);
+        tmem_ld_32x32b_x16(tmem + lane_base + 128 + 64 * hq + 32 * sub + 16 * pc, dav);
         const int u0 = 4 * sub + 2 * pc;   // first 16-byte unit of the piece in the bias row
         uint32_t hb[8];
 #pragma unroll
@@ -657,8 +640,8 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  e = launch_pdl(attn_bias_t_kernel, dim3(static_cast<unsigned>(bias_grid_pairs(a.max_pairs, a.bias_heads)), 4,
-                                          static_cast<unsigned>(a.bias_heads)),
+  e = launch_pdl(attn_bias_t_kernel,
+                 dim3(static_cast<unsigned>(bias_tile_grid(a.max_pairs, a.bias_heads)), static_cast<unsigned>(a.bias_heads)),
                  dim3(kBiasThreads), 0, st, A);
   if (e != cudaSuccess) return e;
   // TMA row coordinates of the bias and dX^T tiles are 32-bit

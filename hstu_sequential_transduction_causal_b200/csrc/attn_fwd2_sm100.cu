@@ -58,16 +58,7 @@ constexpr uint32_t kHalf2Half = 0x38003800u;   // (0.5, 0.5) in fp16
 // half-bias tile of bias_tile.cuh.
 __global__ void __launch_bounds__(kBiasThreads)
 attn_bias_kernel(AttnArgs a) {
-  pdl_enter();
-  // pairs blockIdx.x, + gridDim.x, ... up to the batch's last one (the grid is sized for the SMs,
-  // not for the bound max_pairs)
-  for (long long p = blockIdx.x; p < a.max_pairs; p += gridDim.x) {
-    const long long tile = (p * a.bias_heads + blockIdx.z) * (kQTile * kQTile);
-    if (!bias_tile_block<false, false>(a, p, blockIdx.y, blockIdx.z, reinterpret_cast<uint16_t*>(a.bias) + tile,
-                                       nullptr))
-      break;
-    __syncthreads();
-  }
+  bias_tiles<false, false>(a, reinterpret_cast<uint16_t*>(a.bias), nullptr);
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -981,6 +972,12 @@ cudaError_t launch_attn2(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 // Pairs the bias-tile grids cover at once (they loop over the rest): eight 256-thread blocks per SM
 // across the 4 row blocks and the head slices.
+int64_t bias_tile_grid(int64_t max_pairs, int bias_heads) {
+  const int64_t fit = (4ll * sm_count()) / (bias_heads > 0 ? bias_heads : 1);
+  const int64_t g = fit < 1 ? 1 : fit;
+  return max_pairs < g ? max_pairs : g;
+}
+
 int64_t bias_grid_pairs(int64_t max_pairs, int bias_heads) {
   const int64_t fit = (8ll * sm_count()) / (4ll * (bias_heads > 0 ? bias_heads : 1));
   const int64_t g = fit < 1 ? 1 : fit;
@@ -1027,8 +1024,8 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  e = launch_pdl(attn_bias_kernel, dim3(static_cast<unsigned>(bias_grid_pairs(a.max_pairs, a.bias_heads)), 4,
-                                        static_cast<unsigned>(a.bias_heads)),
+  e = launch_pdl(attn_bias_kernel,
+                 dim3(static_cast<unsigned>(bias_tile_grid(a.max_pairs, a.bias_heads)), static_cast<unsigned>(a.bias_heads)),
                  dim3(kBiasThreads), 0, st, a);
   if (e != cudaSuccess) return e;
   const bool f16 = a.in_f16 != 0;

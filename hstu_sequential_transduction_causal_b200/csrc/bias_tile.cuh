@@ -1,12 +1,12 @@
-// bias_tile.cuh - the relative half-bias of one causal (query tile, key tile) pair, computed by four
-// blocks of 256 threads (32 rows each):
+// bias_tile.cuh - the relative half-bias of one causal (query tile, key tile) pair, computed by one
+// block of 256 threads:
 //   bias(i, j) = 0.5 (rab_pos[clamp(i - j)] + rab_time[bucket(t_i - t_j)])
 // ("HSTU: The First Exploration of the Scaling Law", 7.1.4 Innovation 2: position and time bias;
 // the buckets of time_bucket_dev.cuh). The bias does not depend on the head, so a pair's tile is
 // computed once and read by every head.
 //
-// Thread t of block rb takes the column pairs 2 (t % 16) + 32 e, e < 4, of the rows 32 rb + t / 16 +
-// 16 p, p < 2: 16 elements, 4-byte half-bias (and 2-byte bucket) stores. TRANSPOSED: rows are keys and columns
+// Thread t takes the column pairs 2 (t % 16) + 32 e, e < 4, of the rows t / 16 + 16 p, p < 8: 64
+// elements, 4-byte half-bias (and 2-byte bucket) stores. TRANSPOSED: rows are keys and columns
 // queries (the backward's [key][query] tiles); otherwise rows are queries. Timestamps past
 // the sequence end are clamped to its last token (those elements are masked by the attention).
 // When every difference of the tile fits in int32 (spans under 68 years of seconds) the bucket
@@ -109,56 +109,95 @@ __device__ __forceinline__ void tile_types_load(int* ty, const int32_t* __restri
   ty[tid] = t;
 }
 
-// Rows [32 rb, 32 rb + 32) of the tile of causal pair `pair` for bias head slice hb (four blocks cover
-// a tile, so that a batch of a few hundred pairs still puts several blocks on every SM). With per-head
-// tables (bias_heads = H) every head has its own tile; with a type term each element also adds
-// rab_type[type_query][type_key]. BUCKETS: also the u8 bucket tile (head-independent, written by the
-// hb = 0 blocks). False when `pair` is past the batch's last pair. A block that calls it again must
-// synchronise first (the staging arrays are reused).
+// The constant part of a block's bias work, staged once per block: the bucket thresholds and the
+// head slice's halved rab_time (n_buckets <= 128) and rab_type (n_types <= 16) tables. These are
+// inputs of the call, never written by the kernels before it, so a kernel may stage them before its
+// programmatic-dependency wait.
+struct BiasConst {
+  long long tau[kTauEntries];
+  int tau32[kTauEntries];
+  float rt[128];
+  float tt[16 * 16];
+};
+
+__device__ __forceinline__ void bias_const_load(BiasConst& c, const AttnArgs& a, int hb) {
+  const int tid = threadIdx.x;
+  for (int e = tid; e < kTauEntries; e += kBiasThreads) {
+    c.tau[e] = g_time_taus[e];
+    c.tau32[e] = g_time_taus32[e];
+  }
+  if (tid < a.n_buckets) c.rt[tid] = 0.5f * a.rab_time[static_cast<long long>(hb) * a.n_buckets + tid];
+  const int nt = a.n_types;
+  if (nt > 0 && tid < nt * nt) c.tt[tid] = 0.5f * a.rab_type[static_cast<long long>(hb) * nt * nt + tid];
+}
+
+// The batch's pair numbering, offsets and packing, read by every tile's decode: staged in shared
+// memory for batches of up to kSeqStage sequences (one round of loads instead of a binary search of
+// dependent global loads per tile), else the global arrays.
+constexpr int kSeqStage = 512;
+struct SeqTables {
+  const long long* pair_base;
+  const int64_t* offsets;
+  const int32_t* pack;
+};
+
+__device__ __forceinline__ SeqTables stage_seq_tables(const AttnArgs& a, long long* s_pb, int64_t* s_off,
+                                                      int32_t* s_pack) {
+  if (a.B > kSeqStage) return SeqTables{a.pair_base, a.offsets, a.pack};
+  for (int i = threadIdx.x; i <= a.B; i += kBiasThreads) {
+    s_pb[i] = a.pair_base[i];
+    s_off[i] = a.offsets[i];
+    if (a.pack && i < a.B) s_pack[i] = a.pack[i];
+  }
+  return SeqTables{s_pb, s_off, a.pack ? s_pack : nullptr};
+}
+
+// The whole tile of causal pair `pair` for bias head slice hb, by one block of kBiasThreads threads
+// (c staged and synchronised before). With per-head tables (bias_heads = H) every head has its own
+// tile; with a type term each element also adds rab_type[type_query][type_key]. BUCKETS: also the u8
+// bucket tile (head-independent, written by the hb = 0 blocks). False when `pair` is past the batch's
+// last pair. A block that calls it again must synchronise first (the staging arrays are reused).
 template <bool TRANSPOSED, bool BUCKETS>
-__device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, long long pair, int rb, int hb,
-                                                uint16_t* __restrict__ tile, uint8_t* __restrict__ btile) {
+__device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, const BiasConst& cst, const SeqTables& sq,
+                                                long long pair, int hb, uint16_t* __restrict__ tile,
+                                                uint8_t* __restrict__ btile) {
   __shared__ TileTimes s_t;
-  __shared__ long long s_tau[kTauEntries];
-  __shared__ int s_tau32[kTauEntries];
-  __shared__ float s_win[256], s_rt[128];
+  __shared__ float s_win[256];
   __shared__ int s_ty[256];
-  __shared__ float s_tt[16 * 16];
   int b, qt, kt, n;
   long long seq0;
-  if (!decode_tile_pair(pair, a.pair_base, a.B, &b, &qt, &kt)) return false;
-  if (!pair_rows(a.offsets, a.pack, b, &seq0, &n)) return true;   // a packed sequence's own pair: unused
+  if (!decode_tile_pair(pair, sq.pair_base, a.B, &b, &qt, &kt)) return false;
+  if (!pair_rows(sq.offsets, sq.pack, b, &seq0, &n)) return true;   // a packed sequence's own pair: unused
   const int tid = threadIdx.x;
   const int L = a.pos_max_len, nt = a.n_types;
   const float* rab_pos = a.rab_pos + static_cast<long long>(hb) * (2 * L - 1);
-  const float* rab_time = a.rab_time + static_cast<long long>(hb) * a.n_buckets;
   tile_times_load(s_t, a.ts, seq0, n, qt * kQTile, kt * kQTile);
-  if (tid < a.n_buckets) s_rt[tid] = 0.5f * rab_time[tid];
   if (tid < 255) {
     const int pi = bias_pos_index(static_cast<long long>(qt - kt) * kQTile - 127 + tid, L);
     if (HSTU_DCHECK(pi >= 0 && pi < 2 * L - 1, a.status)) s_win[tid] = 0.5f * rab_pos[pi];
   }
-  if (nt > 0) {
-    tile_types_load(s_ty, a.token_type, seq0, n, qt * kQTile, kt * kQTile, nt, a.status);
-    if (tid < nt * nt) s_tt[tid] = 0.5f * a.rab_type[static_cast<long long>(hb) * nt * nt + tid];
-  }
-  for (int e = tid; e < kTauEntries; e += kBiasThreads) {
-    s_tau[e] = g_time_taus[e];
-    s_tau32[e] = g_time_taus32[e];
-  }
+  if (nt > 0) tile_types_load(s_ty, a.token_type, seq0, n, qt * kQTile, kt * kQTile, nt, a.status);
   __syncthreads();
   const bool fast = tile_times_finish(s_t);
   const int nb = a.n_buckets;
   const bool buckets = BUCKETS && hb == 0;
-  // thread: column pairs c = 2 (tid % 16) + 32 e + x (e < 4, x < 2) of rows r = 32 rb + tid / 16 + 16 p
-  // (p < 2). The 16 lanes of a half-warp read 32 consecutive diagonals of the rab_pos window (no bank
+  // thread: column pairs c = 2 (tid % 16) + 32 e + x (e < 4, x < 2) of rows r = tid / 16 + 16 p
+  // (p < 8). The 16 lanes of a half-warp read 32 consecutive diagonals of the rab_pos window (no bank
   // conflicts) and store 64 contiguous bytes of one row.
-  const int cl = 2 * (tid & 15), rr = 32 * rb + (tid >> 4);
+  const int cl = 2 * (tid & 15), rr = tid >> 4;
+  // staging index of a row / column token: queries at [0, 128), keys at [128, 256)
+  constexpr int kRowBase = TRANSPOSED ? 128 : 0, kColBase = TRANSPOSED ? 0 : 128;
   auto row_pass = [&](auto fast_tag) {
     constexpr bool kFast = decltype(fast_tag)::value;
+    int tcol[8];   // (fast path) the 32-bit times of this thread's 8 columns
+    if (kFast) {
 #pragma unroll
-    for (int p = 0; p < 2; ++p) {
+      for (int j = 0; j < 8; ++j) tcol[j] = s_t.ts32[kColBase + cl + 32 * (j >> 1) + (j & 1)];
+    }
+#pragma unroll 2
+    for (int p = 0; p < 8; ++p) {
       const int r = rr + 16 * p;
+      const int trow = kFast ? s_t.ts32[kRowBase + r] : 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         float v2[2];
@@ -166,13 +205,15 @@ __device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, long long pai
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           const int c = cl + 32 * e + x;
-          const int bkt = tile_bucket<TRANSPOSED>(s_t, kFast, r, c, s_tau, s_tau32, nb);
+          // bucket(t_query - t_key)
+          const int bkt = kFast ? time_bucket32(TRANSPOSED ? tcol[2 * e + x] - trow : trow - tcol[2 * e + x], cst.tau32, nb)
+                                : tile_bucket<TRANSPOSED>(s_t, false, r, c, cst.tau, cst.tau32, nb);
           const int wi = TRANSPOSED ? c - r + 127 : r - c + 127;
           float v = 0.0f;
-          if (HSTU_DCHECK(bkt >= 0 && bkt < nb && wi >= 0 && wi < 255, a.status)) v = s_win[wi] + s_rt[bkt];
+          if (HSTU_DCHECK(bkt >= 0 && bkt < nb && wi >= 0 && wi < 255, a.status)) v = s_win[wi] + cst.rt[bkt];
           if (nt > 0) {
             const int ti = s_ty[TRANSPOSED ? c : r] * nt + s_ty[128 + (TRANSPOSED ? r : c)];
-            if (HSTU_DCHECK(ti >= 0 && ti < nt * nt, a.status)) v += s_tt[ti];
+            if (HSTU_DCHECK(ti >= 0 && ti < nt * nt, a.status)) v += cst.tt[ti];
           }
           v2[x] = v;
           bw |= static_cast<uint32_t>(bkt) << (8 * x);
@@ -185,6 +226,31 @@ __device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, long long pai
   if (fast) row_pass(BoolTag<true>{});
   else row_pass(BoolTag<false>{});
   return true;
+}
+
+// Grid-stride loop of a bias kernel: block (x, hb = blockIdx.y) stages its constants, waits for the
+// kernels before it (the pair numbering and packing come from the work list) and stages the sequence
+// tables, then computes the tiles of pairs x, x + gridDim.x, ... (tiles[pair * bias_heads + hb],
+// btiles[pair]).
+template <bool TRANSPOSED, bool BUCKETS>
+__device__ __forceinline__ void bias_tiles(const AttnArgs& a, uint16_t* __restrict__ tiles,
+                                           uint8_t* __restrict__ btiles) {
+  __shared__ BiasConst s_c;
+  __shared__ long long s_pb[kSeqStage + 1];
+  __shared__ int64_t s_off[kSeqStage + 1];
+  __shared__ int32_t s_pack[kSeqStage];
+  const int hb = blockIdx.y;
+  pdl_trigger();
+  bias_const_load(s_c, a, hb);
+  pdl_wait();
+  const SeqTables sq = stage_seq_tables(a, s_pb, s_off, s_pack);
+  __syncthreads();
+  for (long long p = blockIdx.x; p < a.max_pairs; p += gridDim.x) {
+    uint16_t* tile = tiles + (p * a.bias_heads + hb) * (kQTile * kQTile);
+    uint8_t* btile = BUCKETS ? btiles + p * (kQTile * kQTile) : nullptr;
+    if (!bias_tile_block<TRANSPOSED, BUCKETS>(a, s_c, sq, p, hb, tile, btile)) break;
+    __syncthreads();
+  }
 }
 
 }  // namespace

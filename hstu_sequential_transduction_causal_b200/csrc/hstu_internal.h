@@ -198,8 +198,10 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& a, cudaStream_t st);
 
 // Bound on the number of causal (query tile, key tile) pairs of a batch.
 int64_t attn_max_pairs(int64_t capacity, int max_len);
-// Pairs the bias-tile (and table-gradient) grids cover at once; they loop over the rest.
+// Pairs the table-gradient grid covers at once; it loops over the rest.
 int64_t bias_grid_pairs(int64_t max_pairs, int bias_heads);
+// Blocks (one tile each) of a bias-tile grid per head slice: four per SM; they loop over the rest.
+int64_t bias_tile_grid(int64_t max_pairs, int bias_heads);
 
 cudaError_t attn_fwd_bf16_tc(const AttnArgs& a, cudaStream_t st);     // work list only
 cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st);         // bias tiles + work list

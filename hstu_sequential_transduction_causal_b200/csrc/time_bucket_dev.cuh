@@ -45,12 +45,19 @@ __device__ __forceinline__ int time_bucket_pair64(long long tq, long long tk, co
 __constant__ int c_time_taus32[kTauEntries];
 
 // Branch-free: dt <= 1 is clamped to 1, whose estimate is 0 and whose corrections are both 0
-// (tau[1] = 2 > 1, tau[0] = INT32_MIN), so bucket 0 falls out of the general path.
+// (tau[1] = 2 > 1, tau[0] = INT32_MIN), so bucket 0 falls out of the general path. The estimate is
+// integer arithmetic (one leading-zero count, no conversions or logarithm on the special-function
+// unit): log2(v) is replaced by its chord on each octave, e + f with e the position of the leading
+// one and f the bits below it read as a fraction, which lies at most 0.0861 below log2(v); in 8.24
+// fixed point times 590 / 256 (for 1 / (0.301 log2 e) = 2.30284) the estimate of ln(v) / 0.301 is
+// within (-0.2, +0.06) of it for v < 2^31, so its floor is at most one bucket off and the two
+// threshold comparisons make the result exact.
 __device__ __forceinline__ int time_bucket32(int dt, const int* tau, int nb) {
   const int v = max(dt, 1);
-  constexpr float kLn2Over0301 = 0.693147180559945f / 0.301f;
-  const float lf = __log2f(static_cast<float>(v)) * kLn2Over0301;
-  int k = min(static_cast<int>(lf), 126);
+  const unsigned u = static_cast<unsigned>(v);
+  const int lz = __clz(v);
+  const unsigned fx = (static_cast<unsigned>(31 - lz) << 24) | (((u << lz) << 1) >> 8);
+  int k = min(static_cast<int>(__umulhi(fx, 590u)), 126);
   k += (v >= tau[k + 1] ? 1 : 0) - (v < tau[k] ? 1 : 0);
   return min(k, nb - 1);
 }
