@@ -380,10 +380,10 @@ def main():
     # kernels of ours per step (cross-checked against the ncu launch list in profiles/)
     # f1 GEMM | work list, bias tiles, attention | LN-gate | fp16 W2 copy, f2 GEMM
     n_fwd_kernels = 7
-    # fp16 dy with the db2 partial sums | fp16 copies of x, W1, W2 (one launch) | dG, dW2 GEMMs | LN-gate bwd |
-    # finish of db2, dgamma, dbeta | work list, transposed bias tiles, attention bwd, table gradients | dZ
-    # with the db1 partial sums | finish of db1 | dW1, dX GEMMs
-    n_bwd_kernels = 14
+    # fp16 dy with the db2 partial sums | fp16 copies of x, W1, W2 (one launch) | dG with dW2 (one grouped
+    # GEMM launch) | LN-gate bwd | finish of db2, dgamma, dbeta | work list, transposed bias tiles, attention
+    # bwd, table gradients | dZ with the db1 partial sums | finish of db1 | dX with dW1 (one grouped launch)
+    n_bwd_kernels = 12
     names = ["uvqk", "attn", "norm_gate", "out_proj"] + (["backward"] if backward else [])
 
     def attention_forward():

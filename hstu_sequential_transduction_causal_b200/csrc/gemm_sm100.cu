@@ -37,13 +37,15 @@ constexpr int kBN = 256;        // every tile is 128 x 256: one tcgen05.mma (M=1
 constexpr int kBK = 64;
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;    // 2 per TMEM lane quadrant, each on half of the tile's columns
-constexpr int kProdWarp0 = kEpiWarps;            // warps 8-11: TMA producers, one per stage slot
-constexpr int kMmaWarp = kProdWarp0 + kStages;   // warp 12: MMA issue
-constexpr int kSchedWarp = kMmaWarp + 1;         // warp 13: work-unit scheduler
-constexpr int kThreads = 32 * (kSchedWarp + 1);
+constexpr int kProdWarps = 2;                    // warps 8, 9: TMA producers of alternate stage slots
+constexpr int kProdWarp0 = kEpiWarps;
+constexpr int kMmaWarp = kProdWarp0 + kProdWarps;   // warp 10: MMA issue
+constexpr int kSchedWarp = kMmaWarp + 1;            // warp 11: work-unit scheduler
+constexpr int kThreads = 32 * (kSchedWarp + 1);     // 12 warps: 168 registers a thread
+static_assert(kStages % kProdWarps == 0, "each producer warp owns whole stage slots");
 constexpr int kBoxBytes = 4096; // one epilogue staging box: 32 rows x 128 bytes
 constexpr int kRing = 8;        // work-unit ring between the scheduler and the other roles
-constexpr int kRingReaders = kStages + 1 + kEpiWarps;
+constexpr int kRingReaders = kProdWarps + 1 + kEpiWarps;
 
 struct GemmSmem {
   static constexpr int kABytes = kBM * kBK * 2;      // 16 KB
@@ -183,13 +185,13 @@ __device__ __forceinline__ void emit64(EpiStage& es, const CUtensorMap* map, int
 
 // Persistent tensor-core GEMM over the work units of one or two problems. Roles of a CTA:
 //   warps 0-7   epilogue: TMEM -> registers -> fused epilogue -> TMA stores
-//   warps 8-11  TMA producers, warp 8 + s filling stage slot s (separate warps keep the copies of
-//               several stages in flight at once; one issuing warp serialises them)
-//   warp 12     one thread issues tcgen05.mma (M=128, N=256, K=16) into a double-buffered TMEM
+//   warps 8, 9  TMA producers, warp 8 + p filling the stage slots s with s % 2 == p (an issuing warp
+//               keeps about one stage's copies in flight; two warps stay ahead of the MMAs of
+//               128 x 256 x 64 k-blocks)
+//   warp 10     one thread issues tcgen05.mma (M=128, N=256, K=16) into a double-buffered TMEM
 //               accumulator, so the epilogue of one unit overlaps the next unit's mainloop
-//   warp 13     scheduler (dynamic mode): takes the CTA's next unit from the global counter one unit
+//   warp 11     scheduler (dynamic mode): takes the CTA's next unit from the global counter one unit
 //               ahead of the producers and publishes it to the other roles through a ring
-// 14 warps put 4 warps on some SM sub-partitions (16,384 registers each): 128 registers a thread
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_bf16_tc_kernel(const __grid_constant__ GemmMaps m0, const __grid_constant__ GemmMaps m1,
                     const __grid_constant__ GemmLaunch L, WaitCtl ctl) {
@@ -273,8 +275,8 @@ gemm_bf16_tc_kernel(const __grid_constant__ GemmMaps m0, const __grid_constant__
   };
 
   if (warp >= kProdWarp0 && warp < kMmaWarp) {
-    // producer of stage slot s: the CTA's k-blocks g (counted over all its units) with g % S == s
-    const int s = warp - kProdWarp0;
+    // producer p: the CTA's k-blocks g (counted over all its units) with g % 2 == p, stage slot g % S
+    const int p = warp - kProdWarp0;
     int g = 0;
     for (int i = 0;; ++i) {
       int u;
@@ -286,8 +288,9 @@ gemm_bf16_tc_kernel(const __grid_constant__ GemmMaps m0, const __grid_constant__
       const int a_boxes = q.a_mn ? 2 : 1;                 // A: 1 K-major box or 2 MN-major halves
       const int boxes = a_boxes + (q.b_mn ? kBN / 64 : 1);   // B: 1 K-major box or 4 MN-major boxes
       bool ok = true;
-      for (int j = (s - g % kStages + kStages) % kStages; j < nkb; j += kStages) {
+      for (int j = (p - g % kProdWarps + kProdWarps) % kProdWarps; j < nkb; j += kProdWarps) {
         const int gg = g + j;
+        const int s = gg % kStages;
         bool free_ok = true;   // lane 0 waits; the result is made warp-uniform
         if (lane == 0 && gg >= kStages) free_ok = mbar_wait(empty(s), ((gg / kStages) - 1) & 1, abort_flag, ctl);
         if (!__shfl_sync(0xffffffffu, free_ok ? 1 : 0, 0)) {
