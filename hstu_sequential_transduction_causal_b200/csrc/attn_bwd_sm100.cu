@@ -640,10 +640,12 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
-  e = launch_pdl(attn_bias_t_kernel,
-                 dim3(static_cast<unsigned>(bias_tile_grid(a.max_pairs, a.bias_heads)), static_cast<unsigned>(a.bias_heads)),
-                 dim3(kBiasThreads), 0, st, A);
-  if (e != cudaSuccess) return e;
+  if (!A.bias_cached) {
+    e = launch_pdl(attn_bias_t_kernel,
+                   dim3(static_cast<unsigned>(bias_tile_grid(a.max_pairs, a.bias_heads)), static_cast<unsigned>(a.bias_heads)),
+                   dim3(kBiasThreads), 0, st, A);
+    if (e != cudaSuccess) return e;
+  }
   // TMA row coordinates of the bias and dX^T tiles are 32-bit
   if (a.max_pairs * a.H * kQTile > 0x7fffffffLL) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv, tdo, tbt, tdx, tdq;

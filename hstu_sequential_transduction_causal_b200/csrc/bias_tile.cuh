@@ -160,7 +160,8 @@ __device__ __forceinline__ SeqTables stage_seq_tables(const AttnArgs& a, long lo
 template <bool TRANSPOSED, bool BUCKETS>
 __device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, const BiasConst& cst, const SeqTables& sq,
                                                 long long pair, int hb, uint16_t* __restrict__ tile,
-                                                uint8_t* __restrict__ btile) {
+                                                uint8_t* __restrict__ btile, uint16_t* __restrict__ tile_t,
+                                                uint8_t* __restrict__ btile_t) {
   __shared__ TileTimes s_t;
   __shared__ float s_win[256];
   __shared__ int s_ty[256];
@@ -180,15 +181,17 @@ __device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, const BiasCon
   __syncthreads();
   const bool fast = tile_times_finish(s_t);
   const int nb = a.n_buckets;
-  const bool buckets = BUCKETS && hb == 0;
   // thread: column pairs c = 2 (tid % 16) + 32 e + x (e < 4, x < 2) of rows r = tid / 16 + 16 p
   // (p < 8). The 16 lanes of a half-warp read 32 consecutive diagonals of the rab_pos window (no bank
   // conflicts) and store 64 contiguous bytes of one row.
   const int cl = 2 * (tid & 15), rr = tid >> 4;
-  // staging index of a row / column token: queries at [0, 128), keys at [128, 256)
-  constexpr int kRowBase = TRANSPOSED ? 128 : 0, kColBase = TRANSPOSED ? 0 : 128;
-  auto row_pass = [&](auto fast_tag) {
+  // one pass over the tile: query-major (KEY_MAJOR false) or key-major; bout (nullable) receives the
+  // buckets in the same layout
+  auto row_pass = [&](auto fast_tag, auto key_major_tag, uint16_t* __restrict__ out, uint8_t* __restrict__ bout) {
     constexpr bool kFast = decltype(fast_tag)::value;
+    constexpr bool kTr = decltype(key_major_tag)::value;
+    // staging index of a row / column token: queries at [0, 128), keys at [128, 256)
+    constexpr int kRowBase = kTr ? 128 : 0, kColBase = kTr ? 0 : 128;
     int tcol[8];   // (fast path) the 32-bit times of this thread's 8 columns
     if (kFast) {
 #pragma unroll
@@ -206,32 +209,37 @@ __device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, const BiasCon
         for (int x = 0; x < 2; ++x) {
           const int c = cl + 32 * e + x;
           // bucket(t_query - t_key)
-          const int bkt = kFast ? time_bucket32(TRANSPOSED ? tcol[2 * e + x] - trow : trow - tcol[2 * e + x], cst.tau32, nb)
-                                : tile_bucket<TRANSPOSED>(s_t, false, r, c, cst.tau, cst.tau32, nb);
-          const int wi = TRANSPOSED ? c - r + 127 : r - c + 127;
+          const int bkt = kFast ? time_bucket32(kTr ? tcol[2 * e + x] - trow : trow - tcol[2 * e + x], cst.tau32, nb)
+                                : tile_bucket<kTr>(s_t, false, r, c, cst.tau, cst.tau32, nb);
+          const int wi = kTr ? c - r + 127 : r - c + 127;
           float v = 0.0f;
           if (HSTU_DCHECK(bkt >= 0 && bkt < nb && wi >= 0 && wi < 255, a.status)) v = s_win[wi] + cst.rt[bkt];
           if (nt > 0) {
-            const int ti = s_ty[TRANSPOSED ? c : r] * nt + s_ty[128 + (TRANSPOSED ? r : c)];
+            const int ti = s_ty[kTr ? c : r] * nt + s_ty[128 + (kTr ? r : c)];
             if (HSTU_DCHECK(ti >= 0 && ti < nt * nt, a.status)) v += cst.tt[ti];
           }
           v2[x] = v;
           bw |= static_cast<uint32_t>(bkt) << (8 * x);
         }
-        *reinterpret_cast<uint32_t*>(tile + r * kQTile + cl + 32 * e) = pack_f16x2(v2[0], v2[1]);
-        if (buckets) *reinterpret_cast<uint16_t*>(btile + r * kQTile + cl + 32 * e) = static_cast<uint16_t>(bw);
+        *reinterpret_cast<uint32_t*>(out + r * kQTile + cl + 32 * e) = pack_f16x2(v2[0], v2[1]);
+        if (bout) *reinterpret_cast<uint16_t*>(bout + r * kQTile + cl + 32 * e) = static_cast<uint16_t>(bw);
       }
     }
   };
-  if (fast) row_pass(BoolTag<true>{});
-  else row_pass(BoolTag<false>{});
+  auto pass = [&](auto key_major_tag, uint16_t* out, uint8_t* bout) {
+    if (fast) row_pass(BoolTag<true>{}, key_major_tag, out, bout);
+    else row_pass(BoolTag<false>{}, key_major_tag, out, bout);
+  };
+  pass(BoolTag<TRANSPOSED>{}, tile, BUCKETS && hb == 0 ? btile : nullptr);
+  // the backward's key-major tile and buckets as well (a forward that caches them for its backward)
+  if (!TRANSPOSED && tile_t) pass(BoolTag<true>{}, tile_t, hb == 0 ? btile_t : nullptr);
   return true;
 }
 
 // Grid-stride loop of a bias kernel: block (x, hb = blockIdx.y) stages its constants, waits for the
 // kernels before it (the pair numbering and packing come from the work list) and stages the sequence
 // tables, then computes the tiles of pairs x, x + gridDim.x, ... (tiles[pair * bias_heads + hb],
-// btiles[pair]).
+// btiles[pair]; with a.bias_t_out / a.bucket_t_out also the key-major tiles and buckets there).
 template <bool TRANSPOSED, bool BUCKETS>
 __device__ __forceinline__ void bias_tiles(const AttnArgs& a, uint16_t* __restrict__ tiles,
                                            uint8_t* __restrict__ btiles) {
@@ -248,7 +256,10 @@ __device__ __forceinline__ void bias_tiles(const AttnArgs& a, uint16_t* __restri
   for (long long p = blockIdx.x; p < a.max_pairs; p += gridDim.x) {
     uint16_t* tile = tiles + (p * a.bias_heads + hb) * (kQTile * kQTile);
     uint8_t* btile = BUCKETS ? btiles + p * (kQTile * kQTile) : nullptr;
-    if (!bias_tile_block<TRANSPOSED, BUCKETS>(a, s_c, sq, p, hb, tile, btile)) break;
+    uint16_t* tile_t = a.bias_t_out ? static_cast<uint16_t*>(a.bias_t_out) + (p * a.bias_heads + hb) * (kQTile * kQTile)
+                                    : nullptr;
+    uint8_t* btile_t = a.bucket_t_out ? static_cast<uint8_t*>(a.bucket_t_out) + p * (kQTile * kQTile) : nullptr;
+    if (!bias_tile_block<TRANSPOSED, BUCKETS>(a, s_c, sq, p, hb, tile, btile, tile_t, btile_t)) break;
     __syncthreads();
   }
 }

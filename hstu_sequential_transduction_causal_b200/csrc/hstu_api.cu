@@ -94,6 +94,19 @@ bool bwd_pairs_fit(const hstu_jagged_t* j, int H) {
   return H > 0 && attn_ws_layout(j).max_pairs <= kMaxTmaRows / (static_cast<int64_t>(H) * kQTile);
 }
 
+// hstu_layer_saved_t.attn_bias: the backward's key-major fp16 half-bias tiles (32 KB per causal
+// pair), then the u8 bucket tiles (16 KB per pair), in the layout of the attention backward's own.
+struct BiasCache {
+  size_t bucket, total;
+};
+BiasCache bias_cache_layout(const hstu_jagged_t* j) {
+  const int64_t mp = attn_ws_layout(j).max_pairs;
+  BiasCache c{};
+  c.bucket = align_up(static_cast<size_t>(mp) * kQTile * kQTile * 2, 256);
+  c.total = c.bucket + align_up(static_cast<size_t>(mp) * kQTile * kQTile, 256);
+  return c;
+}
+
 // attention-backward workspace: the forward layout up to pair_base, then the key-tile work list,
 // the transposed fp16 bias tiles (32 KB per pair), the u8 bucket tiles (16 KB per pair) and the fp16
 // dX^T tiles of every (pair, head) (32 KB each) the table gradients are summed from.
@@ -151,7 +164,8 @@ LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) 
 hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const void* q, const void* k,
                            const void* v, const void* d_out, const float* rab_pos, const float* rab_time, float* dq,
                            float* dk, float* dv, int64_t ld_g, float* d_rab_pos, float* d_rab_time, void* ws,
-                           cudaStream_t st, const hstu_rab_ext_t* ext = nullptr, float* d_rab_type = nullptr) {
+                           cudaStream_t st, const hstu_rab_ext_t* ext = nullptr, float* d_rab_type = nullptr,
+                           void* bias_cache = nullptr) {
   const int hb = ext && ext->per_head ? desc->H : 1;
   const int nt = ext ? ext->n_types : 0;
   const AttnBwdWs lay = attn_bwd_ws_layout(jag, desc->H, hb);
@@ -184,6 +198,11 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
   a.bias_heads = hb; a.n_types = nt;
   if (nt > 0) { a.token_type = ext->token_type; a.rab_type = ext->rab_type; }
   A.bias_t = w + lay.bias_t; A.bucket_t = w + lay.bucket_t; A.dxt = w + lay.dxt;
+  if (bias_cache && hb == 1) {   // written by this batch's forward (shared tables only)
+    A.bias_t = bias_cache;
+    A.bucket_t = static_cast<uint8_t*>(bias_cache) + bias_cache_layout(jag).bucket;
+    A.bias_cached = 1;
+  }
   A.kitems = reinterpret_cast<int32_t*>(w + lay.kitems); A.kcount = kcount;
   a.pack = reinterpret_cast<const int32_t*>(w + lay.f.pack);
   e = launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, a.status, st,
@@ -229,7 +248,7 @@ hstu_status_t check_attn(const hstu_attn_desc_t* d, const hstu_jagged_t* j) {
 hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, const void* q, const void* k,
                            const void* v, const float* rab_pos, const float* rab_time, void* out, void* ws,
                            cudaStream_t st, bool tile_pairs = true, const hstu_rab_ext_t* ext = nullptr,
-                           const int64_t* q_from = nullptr) {
+                           const int64_t* q_from = nullptr, void* bias_cache = nullptr) {
   const int64_t cap = capacity_of(j);
   const int hb = ext && ext->per_head ? d->H : 1;
   const AttnWs lay = attn_ws_layout(j, hb);
@@ -259,6 +278,10 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
     a.urec = reinterpret_cast<const int32_t*>(w + lay.urec);
     // short sequences share tiles, except in a prefix append (whose rows start mid-sequence)
     if (!q_from) a.pack = reinterpret_cast<const int32_t*>(w + lay.pack);
+    if (bias_cache && hb == 1 && !q_from) {   // the backward's tiles too
+      a.bias_t_out = bias_cache;
+      a.bucket_t_out = static_cast<uint8_t*>(bias_cache) + bias_cache_layout(j).bucket;
+    }
   }
   cudaError_t e = launch_worklist(j->offsets, j->B, j->T, j->max_len, items, count, a.status, st,
                                   pairs ? reinterpret_cast<long long*>(w + lay.pairs) : nullptr, nullptr, nullptr,
@@ -740,6 +763,7 @@ hstu_status_t run_layer_fwd(const hstu_layer_desc_t* desc, hstu_dtype_t resid_dt
     const void* v16[] = {x, x_f16, y, y_f16, saved->uvqk, saved->z, saved->o, saved->g, w->W1, w->W2, w->b1, w->b2};
     for (const void* p : v16)
       if (p && !aligned16(p)) return HSTU_ERR_UNSUPPORTED;
+    if (saved->attn_bias && reinterpret_cast<uintptr_t>(saved->attn_bias) % 256) return HSTU_ERR_UNSUPPORTED;
   }
   cudaStream_t st = stream;
   int* status = ws_status(ws);
@@ -767,7 +791,7 @@ hstu_status_t run_layer_fwd(const hstu_layer_desc_t* desc, hstu_dtype_t resid_dt
   const size_t es = act == HSTU_F32 ? 4 : 2;
   const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
   s = run_attn_fwd(&ad, jag, uvqk + 2 * D * es, uvqk + 3 * D * es, uvqk + 1 * D * es, w->rab_pos, w->rab_time,
-                   saved->o, ws, st);
+                   saved->o, ws, st, true, nullptr, nullptr, saved->attn_bias);
   if (s != HSTU_OK) return s;
   // G in fp16 (BF16 mode): f2 then reads an fp16 copy of W2
   const hstu_dtype_t g_dt = desc->dtype == HSTU_BF16 ? HSTU_F16 : HSTU_F32;
@@ -827,6 +851,11 @@ size_t hstu_layer_bwd_workspace_size(const hstu_layer_desc_t* desc, const hstu_j
   return layer_bwd_layout(desc, jag).total;
 }
 
+size_t hstu_layer_bias_cache_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag) {
+  if (!desc || check_jagged(jag) != HSTU_OK || !bwd_pairs_fit(jag, desc->H)) return 0;
+  return bias_cache_layout(jag).total;
+}
+
 }  // extern "C"
 
 namespace hstu {
@@ -884,6 +913,7 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
                          w->W1, w->W2, w->gamma, w->beta, gr->dW1, gr->dW2};
     for (const void* p : v16)
       if (p && !aligned16(p)) return HSTU_ERR_UNSUPPORTED;
+    if (saved->attn_bias && reinterpret_cast<uintptr_t>(saved->attn_bias) % 256) return HSTU_ERR_UNSUPPORTED;
   }
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   int* status = ws_status(ws);
@@ -947,7 +977,7 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   // 3. attention backward
   const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
   s = run_attn_bwd(&ad, jag, uvqk + 2 * D * 2, uvqk + 3 * D * 2, uvqk + 1 * D * 2, dO, w->rab_pos, w->rab_time, dq, dk,
-                   dv, D, gr->drab_pos, gr->drab_time, ws, st);
+                   dv, D, gr->drab_pos, gr->drab_time, ws, st, nullptr, nullptr, saved->attn_bias);
   if (s != HSTU_OK) return s;
   if (g_ready_events[0]) {   // dW2, db2, dgamma, dbeta and the table gradients are final
     e = cudaEventRecord(g_ready_events[0], st);

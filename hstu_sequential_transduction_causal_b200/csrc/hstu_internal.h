@@ -178,6 +178,10 @@ struct AttnArgs {
   // packed short sequences (launch_worklist's pack array) or null: an item (b, -k) is one tile over
   // the rows of sequences b .. b + k - 1, keys masked to the query row's own sequence
   const int32_t* pack;
+  // (forward, nullable) the bias kernel also writes the backward's key-major tiles and buckets here,
+  // laid out as AttnBwdArgs::bias_t and ::bucket_t
+  void* bias_t_out;
+  void* bucket_t_out;
 };
 
 struct AttnBwdArgs {
@@ -192,6 +196,7 @@ struct AttnBwdArgs {
   void* dxt;                   // fp16 [max_pairs, H, 128 keys, 128 queries] dX^T of every (pair, head)
   const int32_t* kitems;       // backward work list (b, key tile)
   const int32_t* kcount;
+  int bias_cached;             // bias_t and bucket_t were written by the forward: no bias kernel
 };
 
 cudaError_t attn_bwd_tc(const AttnBwdArgs& a, cudaStream_t st);

@@ -57,7 +57,7 @@ class hstu_layer_weights_t(ctypes.Structure):
 
 
 class hstu_layer_saved_t(ctypes.Structure):
-    _fields_ = [(n, c_vp) for n in ("uvqk", "z", "o", "g", "mu", "rstd")]
+    _fields_ = [(n, c_vp) for n in ("uvqk", "z", "o", "g", "mu", "rstd", "attn_bias")]
 
 
 class hstu_layer_grads_t(ctypes.Structure):
@@ -104,6 +104,7 @@ SIGNATURES = {
     "hstu_linear_bf16": (c_i32, [c_i64, c_i64, c_i64, c_vp, c_i64, c_i32, c_vp, c_i64, c_i32, c_vp, c_vp, c_i32,
                                  c_i64, c_vp, c_i32, c_i64, c_i32, c_vp, c_sz, c_vp]),
     "hstu_layer_bwd_workspace_size": (c_sz, [P(hstu_layer_desc_t), P(hstu_jagged_t)]),
+    "hstu_layer_bias_cache_size": (c_sz, [P(hstu_layer_desc_t), P(hstu_jagged_t)]),
     "hstu_layer_bwd": (c_i32, [P(hstu_layer_desc_t), P(hstu_jagged_t), P(hstu_layer_weights_t), c_vp, c_vp,
                                P(hstu_layer_saved_t), c_vp, c_vp, c_vp, c_vp, P(hstu_layer_grads_t), c_vp, c_sz,
                                c_vp]),
@@ -410,8 +411,8 @@ def layer_weights(W1, b1, W2, b2, gamma, beta, rab_pos, rab_time) -> hstu_layer_
     return hstu_layer_weights_t(*[_ptr(t) for t in (W1, b1, W2, b2, gamma, beta, rab_pos, rab_time)])
 
 
-def layer_saved(uvqk, z, o, g, mu, rstd) -> hstu_layer_saved_t:
-    return hstu_layer_saved_t(*[_ptr(t) for t in (uvqk, z, o, g, mu, rstd)])
+def layer_saved(uvqk, z, o, g, mu, rstd, attn_bias=None) -> hstu_layer_saved_t:
+    return hstu_layer_saved_t(*[_ptr(t) for t in (uvqk, z, o, g, mu, rstd, attn_bias)])
 
 
 def hstu_linear_bf16(M, N, K, A, lda, a_mn, B, ldb, b_mn, bias, resid, resid_dtype_code, ld_resid, out,
@@ -424,6 +425,10 @@ def hstu_linear_bf16(M, N, K, A, lda, a_mn, B, ldb, b_mn, bias, resid, resid_dty
 
 def hstu_layer_bwd_workspace_size(desc: hstu_layer_desc_t, jag: hstu_jagged_t) -> int:
     return lib().hstu_layer_bwd_workspace_size(ctypes.byref(desc), ctypes.byref(jag))
+
+
+def hstu_layer_bias_cache_size(desc: hstu_layer_desc_t, jag: hstu_jagged_t) -> int:
+    return lib().hstu_layer_bias_cache_size(ctypes.byref(desc), ctypes.byref(jag))
 
 
 def hstu_layer_bwd(desc, jag, weights: hstu_layer_weights_t, x, x_f16, saved: hstu_layer_saved_t, dy, dy_f16, dx,

@@ -57,19 +57,23 @@ class SavedActs:
     g: torch.Tensor
     mu: torch.Tensor
     rstd: torch.Tensor
+    attn_bias: Optional[torch.Tensor] = None   # the backward's bias tiles, written by the forward
 
     @classmethod
-    def empty(cls, T: int, D: int, dtype: torch.dtype, keep_z: bool, device="cuda") -> "SavedActs":
+    def empty(cls, T: int, D: int, dtype: torch.dtype, keep_z: bool, device="cuda",
+              bias_cache_bytes: int = 0) -> "SavedActs":
         act = torch.float16 if dtype == torch.bfloat16 else dtype     # U|V|Q|K, Z and G in fp16
         return cls(uvqk=torch.empty(T, 4 * D, dtype=act, device=device),
                    z=torch.empty(T, 4 * D, dtype=act, device=device) if keep_z else None,
                    o=torch.empty(T, D, dtype=torch.float32, device=device),
                    g=torch.empty(T, D, dtype=act, device=device),
                    mu=torch.empty(T, dtype=torch.float32, device=device),
-                   rstd=torch.empty(T, dtype=torch.float32, device=device))
+                   rstd=torch.empty(T, dtype=torch.float32, device=device),
+                   attn_bias=(torch.empty(bias_cache_bytes, dtype=torch.uint8, device=device)
+                              if bias_cache_bytes > 0 else None))
 
     def struct(self) -> H.hstu_layer_saved_t:
-        return H.layer_saved(self.uvqk, self.z, self.o, self.g, self.mu, self.rstd)
+        return H.layer_saved(self.uvqk, self.z, self.o, self.g, self.mu, self.rstd, self.attn_bias)
 
 
 class JaggedBatch:
@@ -110,13 +114,19 @@ class LayerRunner:
     """Runs ``hstu_layer_fwd`` for one layer on a fixed jagged batch with reusable buffers."""
 
     def __init__(self, layer: DeviceLayer, jag: JaggedBatch, inv_N: float, pos_max_len: int,
-                 x_dtype: torch.dtype, y_dtype: torch.dtype, keep_z: bool = False, device="cuda"):
+                 x_dtype: torch.dtype, y_dtype: torch.dtype, keep_z: bool = False, device="cuda",
+                 bias_cache: Optional[bool] = None):
+        """keep_z: a backward follows (Z is kept); bias_cache (default: keep_z in BF16 mode): the forward
+        also writes the backward's attention bias tiles into saved.attn_bias."""
         self.layer, self.jag = layer, jag
         cdt = torch.bfloat16 if layer.dtype_code == H.HSTU_BF16 else torch.float32
         code = {torch.bfloat16: H.HSTU_BF16, torch.float32: H.HSTU_F32}
         self.desc = H.make_layer_desc(layer.D, layer.H, inv_N, pos_max_len, layer.dtype_code, code[x_dtype],
                                       code[y_dtype])
-        self.saved = SavedActs.empty(jag.T, layer.D, cdt, keep_z, device)
+        if bias_cache is None:
+            bias_cache = keep_z and layer.dtype_code == H.HSTU_BF16
+        nbias = H.hstu_layer_bias_cache_size(self.desc, jag.struct) if bias_cache else 0
+        self.saved = SavedActs.empty(jag.T, layer.D, cdt, keep_z, device, nbias)
         self.saved_struct = self.saved.struct()
         self.ws = workspace(H.hstu_layer_workspace_size(self.desc, jag.struct), device)
         self.y = torch.empty(jag.T, layer.D, dtype=y_dtype, device=device)
@@ -146,7 +156,8 @@ class Encoder:
         L, D, T = len(self.layers), self.layers[0].D, jag.T
         self.desc = H.make_layer_desc(D, self.layers[0].H, inv_N, pos_max_len, H.HSTU_BF16, H.HSTU_F32, H.HSTU_F32)
         self.weights = [lay.weights() for lay in self.layers]
-        self.saved = [SavedActs.empty(T, D, torch.bfloat16, True, device) for _ in range(L)]
+        nbias = H.hstu_layer_bias_cache_size(self.desc, jag.struct)
+        self.saved = [SavedActs.empty(T, D, torch.bfloat16, True, device, nbias) for _ in range(L)]
         self.saved_structs = [sv.struct() for sv in self.saved]
         self.xs = [None] + [torch.empty(T, D, dtype=torch.float32, device=device) for _ in range(L - 1)]
         self.x16 = [None] + [torch.empty(T, D, dtype=torch.float16, device=device) for _ in range(L - 1)]

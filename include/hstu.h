@@ -140,7 +140,12 @@ typedef struct hstu_layer_weights_t {
  * mode all are fp32.
  * o [T, D] attention output, always fp32 (LayerNorm divides by its spread across features,
  * which is far smaller than its mean, so bf16 storage would be amplified); g [T, D] =
- * LN(O) (.) U; mu, rstd [T] fp32 LayerNorm statistics. */
+ * LN(O) (.) U; mu, rstd [T] fp32 LayerNorm statistics.
+ * attn_bias (optional, BF16 mode; NULL = unused): hstu_layer_bias_cache_size(desc, jag) bytes,
+ * 256-byte aligned. The forward then also writes there the attention backward's relative-bias
+ * tiles (each causal 128 x 128 (query tile, key tile) pair's half-bias, key-major, and its time
+ * buckets), and a backward given the same struct reads them instead of recomputing them. Valid
+ * only for the batch and rab tables of the forward that wrote it. */
 typedef struct hstu_layer_saved_t {
   void* uvqk;
   void* z;
@@ -148,6 +153,7 @@ typedef struct hstu_layer_saved_t {
   void* g;
   float* mu;
   float* rstd;
+  void* attn_bias;
 } hstu_layer_saved_t;
 
 /* Weight gradients of one layer (fp32, overwritten): dW1 [4D, D], db1 [4D], dW2 [D, D], db2 [D],
@@ -410,6 +416,10 @@ hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
 
 /* Workspace bytes hstu_layer_bwd needs (0 for a batch hstu_attn_bwd_workspace_size refuses). */
 size_t hstu_layer_bwd_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
+
+/* Bytes of hstu_layer_saved_t.attn_bias for this batch (0 for a batch hstu_attn_workspace_size
+ * refuses): per causal tile pair a 32 KB fp16 half-bias tile and a 16 KB u8 bucket tile. */
+size_t hstu_layer_bias_cache_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
 
 /* Whole layer backward (BF16 mode, D in {256, 512}), from the activations hstu_layer_fwd saved
  * (z required). x_f16: nullable fp16 copy of x (the dW1 operand; converted when NULL). dy: [T, D]

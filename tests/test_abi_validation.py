@@ -319,8 +319,9 @@ def weights(**kw):
 
 
 def saved(**kw):
-    names = ("uvqk", "z", "o", "g", "mu", "rstd")
+    names = ("uvqk", "z", "o", "g", "mu", "rstd", "attn_bias")
     vals = {n: fake(30 + i) for i, n in enumerate(names)}
+    vals["attn_bias"] = None
     vals.update(kw)
     return Hb.hstu_layer_saved_t(*[vals[n] for n in names])
 
@@ -350,6 +351,7 @@ def test_layer_fwd(L):
         ("b2 off 16 bytes", dict(w=weights(b2=fake(23) + 4)), UNSUPPORTED),
         ("W2 off 16 bytes", dict(w=weights(W2=fake(22) + 2)), UNSUPPORTED),
         ("x off 16 bytes", dict(x=fake(2) + 2), UNSUPPORTED),
+        ("bias cache off 256 bytes", dict(sv=saved(attn_bias=fake(36) + 128)), UNSUPPORTED),
         ("tile-pair rows beyond 32 bits", dict(j=jag(**HUGE_FWD)), UNSUPPORTED),
     ])
     assert L.hstu_layer_workspace_size(ctypes.byref(layer_desc()), ctypes.byref(jag(**HUGE_FWD))) == 0
@@ -387,10 +389,24 @@ def test_layer_bwd(L):
         ("gamma off 16 bytes", dict(w=weights(gamma=fake(24) + 4)), UNSUPPORTED),
         ("dW1 off 16 bytes", dict(gr=grads(dW1=fake(40) + 4)), UNSUPPORTED),
         ("dx off 16 bytes", dict(dx=fake(4) + 2), UNSUPPORTED),
+        ("bias cache off 256 bytes", dict(sv=saved(attn_bias=fake(36) + 16)), UNSUPPORTED),
         ("dX^T rows beyond 32 bits", dict(j=jag(**HUGE_BWD)), UNSUPPORTED),
     ])
     assert L.hstu_layer_bwd_workspace_size(ctypes.byref(layer_desc()), ctypes.byref(jag(**HUGE_BWD))) == 0
     assert passes_host_checks(L, call, w=weights(b1=None, b2=None))   # the backward does not read the biases
+    assert passes_host_checks(L, call, sv=saved(attn_bias=fake(36)))   # the optional bias cache
+
+
+def test_layer_bias_cache_size(L):
+    """48 KB per causal tile pair (a 32 KB half-bias tile and a 16 KB bucket tile) of the batch's
+    pair bound; 0 for a refused descriptor or batch."""
+    size = L.hstu_layer_bias_cache_size
+    size.restype = ctypes.c_size_t
+    # B = 2 sequences of at most 200 rows: 2 tiles each, so at most 3 causal pairs per sequence
+    n = size(ctypes.byref(layer_desc()), ctypes.byref(jag()))
+    assert n >= 6 * 48 * 1024 and n % 256 == 0
+    assert size(None, ctypes.byref(jag())) == 0
+    assert size(ctypes.byref(layer_desc()), ctypes.byref(jag(**HUGE_BWD))) == 0
 
 
 def falcon_desc(**kw):

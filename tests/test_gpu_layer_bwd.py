@@ -66,10 +66,10 @@ def test_linear_all_operand_layouts(a_mn, b_mn, accumulate, shape):
     assert_close(got, ref, 1e-4 * np.sqrt(K), 1e-4, what=f"linear a_mn={a_mn} b_mn={b_mn} acc={accumulate}")
 
 
-def _run_layer_fwd_bwd(wl, x_dtype=torch.bfloat16):
+def _run_layer_fwd_bwd(wl, x_dtype=torch.bfloat16, bias_cache=None):
     jag = JaggedBatch(wl.offsets, wl.timestamps)
     layer = DeviceLayer.upload(wl.layers[0], wl.D, wl.H, True)
-    run = LayerRunner(layer, jag, 1.0 / wl.N, wl.pos_max_len, x_dtype, x_dtype, keep_z=True)
+    run = LayerRunner(layer, jag, 1.0 / wl.N, wl.pos_max_len, x_dtype, x_dtype, keep_z=True, bias_cache=bias_cache)
     x = to_dev(wl.x, x_dtype)
     run.forward(x)
     D, T = wl.D, wl.T
@@ -133,6 +133,19 @@ def test_layer_bwd_ragged_d512():
     wl = W.make_workload("c3", seed=2, lengths=[1, 130, 300, 0, 257, 64], pos_max_len=512, N=512)
     dx, grads = _run_layer_fwd_bwd(wl)
     _compare(dx, grads, _oracle_grads(wl), _model_grads(wl), "ragged-d512 ")
+
+
+def test_layer_bwd_bias_cache_matches_recompute():
+    """The backward reading the bias tiles its forward cached (hstu_layer_saved_t.attn_bias) computes
+    what it computes from tiles of its own: dx bit for bit (no reduction of unfixed order reaches
+    it), the gradients reduced by atomics up to the order of their fp32 additions."""
+    wl = W.make_workload("c3", seed=5, lengths=[300, 1, 129, 700, 64, 0, 400], pos_max_len=1024, N=1024)
+    dx_c, g_c = _run_layer_fwd_bwd(wl, bias_cache=True)
+    dx_r, g_r = _run_layer_fwd_bwd(wl, bias_cache=False)
+    np.testing.assert_array_equal(dx_c, dx_r)
+    for name, a, b in zip(("dW1", "db1", "dW2", "db2", "dgamma", "dbeta", "drab_pos", "drab_time"), g_c, g_r):
+        scale = max(float(np.abs(b).max()), 1e-30)
+        assert np.abs(a - b).max() <= 1e-5 * scale, name
 
 
 def test_layer_bwd_d256_four_heads():
