@@ -10,8 +10,9 @@
 //
 // attn_bias_t_kernel: per causal (query tile, key tile) pair, the transposed fp16 half-bias tile
 // [key][query] and the u8 time-bucket tile [key][query] (head independent, computed once).
-// attn_bwd_tc_kernel<F16>: one CTA per (sequence, 128-key tile, head), key tiles that visit the
-// most query tiles first; it walks the query tiles t >= its key tile:
+// attn_bwd_tc_kernel<F16>: persistent, one CTA per SM taking (sequence, 128-key tile, head) units
+// from a counter, key tiles that visit the most query tiles first; a unit walks the query tiles
+// t >= its key tile:
 //   warp 16  : TMA: K, V once; Q and dO of each query tile (3 stages); the half-bias tile (2).
 //   warp 17  : tcgen05: S^T = K Q^T and dA^T = V dO^T into TMEM (N = 128, the whole query tile);
 //              after the elementwise step, the next tile's S^T / dA^T first, then dV += P^T dO
@@ -65,10 +66,38 @@ struct BwdSmem {
   static constexpr int kBT0 = kQ0 + 3 * 32768;  // stage st (of 2): half-bias^T, overwritten in place by dX^T
   static constexpr int kDQ = kBT0 + 2 * 32768;  // dQ tile staging for the TMA reduce-add: 2 x [128][32] fp32
   static constexpr int kBar = kDQ + 32768;
-  static constexpr int kTotal = kBar + 256 + 1024;
+  static constexpr int kTotal = kBar + 512 + 1024;   // barriers, TMEM slot, abort flag, unit ring; alignment
 };
 static_assert(BwdSmem::kTotal <= 232448, "shared memory of the backward kernel");
 
+// One (key tile, head) unit of the persistent backward: the work-list item and head of unit u.
+struct BwdUnit {
+  int b, kt, kt_item, h, n, nt, nsteps;
+  bool packed;
+  long long seq0, pbase;
+};
+
+__device__ __forceinline__ BwdUnit bwd_unit(const AttnBwdArgs& A, int u) {
+  const AttnArgs& a = A.f;
+  BwdUnit w;
+  const int item = u / a.H;
+  w.h = u - item * a.H;
+  w.b = A.kitems[2 * item];
+  w.kt_item = A.kitems[2 * item + 1];
+  w.packed = w.kt_item < 0;   // a pack of -kt_item short sequences: one diagonal tile
+  w.kt = w.packed ? 0 : w.kt_item;
+  pair_rows(a.offsets, a.pack, w.b, &w.seq0, &w.n);
+  w.nt = (w.n + kQTile - 1) / kQTile;
+  w.nsteps = w.nt - w.kt;     // query tiles kt .. nt-1
+  w.pbase = a.pair_base[w.b];
+  return w;
+}
+
+constexpr int kRingB = 4;                        // unit ring between the scheduler warp and the others
+constexpr int kRingReadersB = kSiluWarpsB + 3;   // producer, MMA issuer, store warp, elementwise warps
+
+// Persistent: one CTA per SM takes (key tile, head) units, longest key tiles first, from a counter
+// the work list zeroes; barrier phases run on per-CTA counters of units (i) and query-tile steps (G).
 template <bool F16>
 __global__ void __launch_bounds__(kThreadsB, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -80,31 +109,25 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const AttnArgs& a = A.f;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int item = blockIdx.x / a.H;
-  const int h = blockIdx.x - item * a.H;
-  if (item >= *A.kcount) return;
-  const int b = A.kitems[2 * item];
-  const int kt_item = A.kitems[2 * item + 1];
-  const bool packed = kt_item < 0;         // a pack of -kt_item short sequences: one diagonal tile
-  const int kt = packed ? 0 : kt_item;
-  long long seq0;
-  int n;
-  pair_rows(a.offsets, a.pack, b, &seq0, &n);
-  const int nt = (n + kQTile - 1) / kQTile;
-  const int nsteps = nt - kt;              // query tiles kt .. nt-1
-  const long long pbase = a.pair_base[b];
+  const int total = *A.kcount * a.H;
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lb::kBar);
   // 0 kv_full | 1,2 qdo_full | 3,4 qdo_empty | 5,6 bb_full | 7,8 bb_empty | 9,10 s_full (query half
-  // a, b) | 11,12 p_ready (half a, b) | 13 dq_full | 14 fin | 15,16 dx_full (stage) | 17 dq_staged |
-  // 18 dq_stage_free | 19,20 p_free (half a, b: the dV MMA has read P^T_h) | 21 qdo_full, 22 qdo_empty
-  // of the third Q/dO stage
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
+  // a, b) | 11,12 p_ready (half a, b) | 13 dq_full | 14 fin (every MMA of the unit done) | 15,16
+  // dx_full (stage) | 17 dq_staged | 18 dq_stage_free | 19,20 p_free (half a, b: the dV MMA has read
+  // P^T_h) | 21 qdo_full, 22 qdo_empty of the third Q/dO stage | 23 dkdv_free (the unit's dK, dV
+  // are out of TMEM) | 24.. ring_full, ring_empty, ring_got (kRingB each)
+  constexpr int kNumBars = 24 + 3 * kRingB;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
   const uint32_t bar0 = smem_u32(bars);
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   auto qdo_full = [&](int sq) { return sq < 2 ? BAR(1 + sq) : BAR(21); };
   auto qdo_empty = [&](int sq) { return sq < 2 ? BAR(3 + sq) : BAR(22); };
+  auto ring_full = [&](int r) { return BAR(24 + r); };
+  auto ring_empty = [&](int r) { return BAR(24 + kRingB + r); };
+  auto ring_got = [&](int r) { return BAR(24 + 2 * kRingB + r); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -114,7 +137,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     mbar_init(BAR(0), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(BAR(1 + s), 1);
-      mbar_init(BAR(3 + s), 2);   // Q/dO stage free: both MMA issuers are done with it
+      mbar_init(BAR(3 + s), 2);   // Q/dO stage free: after S^T / dA^T and after the gradient MMAs
       mbar_init(BAR(5 + s), 1);
       mbar_init(BAR(7 + s), 2);   // bias/dX stage free: the MMAs read dX^T and the store warp sent it
       mbar_init(BAR(15 + s), kSiluThreadsB);   // both query halves of dX^T written
@@ -130,6 +153,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     mbar_init(BAR(22), 2);
     mbar_init(BAR(17), kSiluThreadsB / 2);     // the half-b warps staged a dQ tile
     mbar_init(BAR(18), 1);                     // the store warp's reduce-add has read the staging
+    mbar_init(BAR(23), kSiluThreadsB);
+    for (int r = 0; r < kRingB; ++r) {
+      mbar_init(ring_full(r), 1);
+      mbar_init(ring_empty(r), kRingReadersB);
+      mbar_init(ring_got(r), 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -159,61 +188,99 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const uint32_t sQ0 = smem_u32(smem + Lb::kQ0);
   const uint32_t sBT0 = smem_u32(smem + Lb::kBT0);
   const uint32_t sDQ = smem_u32(smem + Lb::kDQ);
-  const int krow = static_cast<int>(seq0) + kt * kQTile;
+
+  // Unit i of this CTA for one reading thread (false: the wait gave up); u >= total ends the
+  // sequence. The reader frees the ring slot once it holds the value.
+  auto take_unit = [&](int i, int& u) -> bool {
+    const int r = i % kRingB;
+    if (!mbar_wait(ring_full(r), (i / kRingB) & 1, abort_flag, ctl)) return false;
+    u = ring[r];
+    mbar_arrive(ring_empty(r));
+    return true;
+  };
+  auto take_unit_warp = [&](int i, int& u) -> bool {
+    int v = 0;
+    bool ok = true;
+    if (lane == 0) ok = take_unit(i, v);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    u = __shfl_sync(0xffffffffu, v, 0);
+    return ok;
+  };
 
   if (warp == kSiluWarpsB) {
-    // ---------------- TMA producer: K, V once; Q / dO of stage sq from lanes 2 sq, 2 sq + 1; the bias
-    // halves of stage st from lanes 8 + 2 st, 9 + 2 st (consecutive stages load from different threads)
-    if (lane == 0) mbar_arrive_expect_tx(BAR(0), 32768);
-    __syncwarp();
-    if (lane == 0) tma_load_2d(sK, &tmK, BAR(0), h * kD, krow);
-    if (lane == 1) tma_load_2d(sV, &tmV, BAR(0), h * kD, krow);
-    // Q and dO of tile s (3 stages) run one tile ahead of its bias (2 stages): waiting for a bias
-    // stage never delays the next Q / dO load
-    auto load_bias = [&](int s) -> bool {
-      const int st = s & 1, qt = kt + s;
-      if (s >= 2 && !mbar_wait_warp(BAR(7 + st), ((s >> 1) & 1) ^ 1, abort_flag, ctl)) return false;
-      const long long pair = pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt;
-      const int prow = static_cast<int>((pair * a.bias_heads + (a.bias_heads > 1 ? h : 0)) * kQTile);
-      if (lane == 0) mbar_arrive_expect_tx(BAR(5 + st), 32768);
-      __syncwarp();
-      const int hx = lane - 8 - 2 * st;
-      if (hx == 0 || hx == 1) tma_load_2d(sBT0 + st * 32768 + hx * 16384, &tmBT, BAR(5 + st), 64 * hx, prow);
-      return true;
-    };
+    // ---------------- TMA producer ----------------
+    // Per unit: Q and dO of step g (counted over the CTA's units) into stage g % 3 from lanes 2 sq,
+    // 2 sq + 1; K and V (lanes 0, 1) once every MMA of the previous unit has completed; the bias
+    // halves of step g into stage g % 2 from lanes 8 + 2 st, 9 + 2 st, one step behind its Q / dO
+    // (waiting for a bias stage never delays the next Q / dO load).
+    int G = 0;
     bool ok = true;
-    for (int s = 0; ok && s < nsteps; ++s) {
-      const int qt = kt + s, sq = s % 3;
-      if (s >= 3 && !mbar_wait_warp(qdo_empty(sq), ((s / 3) & 1) ^ 1, abort_flag, ctl)) break;
-      const int qrow = static_cast<int>(seq0) + qt * kQTile;
-      if (lane == 0) mbar_arrive_expect_tx(qdo_full(sq), 32768);
-      __syncwarp();
-      if (lane == 2 * sq) tma_load_2d(sQ0 + sq * 32768, &tmQ, qdo_full(sq), h * kD, qrow);
-      if (lane == 2 * sq + 1) tma_load_2d(sQ0 + sq * 32768 + 16384, &tmDO, qdo_full(sq), h * kD, qrow);
-      if (s >= 1) ok = load_bias(s - 1);
+    for (int i = 0; ok; ++i) {
+      int u;
+      if (!take_unit_warp(i, u) || u >= total) break;
+      const BwdUnit w = bwd_unit(A, u);
+      const int krow = static_cast<int>(w.seq0) + w.kt * kQTile;
+      auto load_bias = [&](int s) -> bool {
+        const int gs = G + s, st = gs & 1, qt = w.kt + s;
+        if (gs >= 2 && !mbar_wait_warp(BAR(7 + st), ((gs >> 1) & 1) ^ 1, abort_flag, ctl)) return false;
+        const long long pair = w.pbase + static_cast<long long>(qt) * (qt + 1) / 2 + w.kt;
+        const int prow = static_cast<int>((pair * a.bias_heads + (a.bias_heads > 1 ? w.h : 0)) * kQTile);
+        if (lane == 0) mbar_arrive_expect_tx(BAR(5 + st), 32768);
+        __syncwarp();
+        const int hx = lane - 8 - 2 * st;
+        if (hx == 0 || hx == 1) tma_load_2d(sBT0 + st * 32768 + hx * 16384, &tmBT, BAR(5 + st), 64 * hx, prow);
+        return true;
+      };
+      for (int s = 0; ok && s < w.nsteps; ++s) {
+        const int gs = G + s, qt = w.kt + s, sq = gs % 3;
+        if (gs >= 3 && !mbar_wait_warp(qdo_empty(sq), ((gs / 3) & 1) ^ 1, abort_flag, ctl)) {
+          ok = false;
+          break;
+        }
+        const int qrow = static_cast<int>(w.seq0) + qt * kQTile;
+        if (lane == 0) mbar_arrive_expect_tx(qdo_full(sq), 32768);
+        __syncwarp();
+        if (lane == 2 * sq) tma_load_2d(sQ0 + sq * 32768, &tmQ, qdo_full(sq), w.h * kD, qrow);
+        if (lane == 2 * sq + 1) tma_load_2d(sQ0 + sq * 32768 + 16384, &tmDO, qdo_full(sq), w.h * kD, qrow);
+        if (s == 0) {
+          if (i >= 1 && !mbar_wait_warp(BAR(14), (i - 1) & 1, abort_flag, ctl)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) mbar_arrive_expect_tx(BAR(0), 32768);
+          __syncwarp();
+          if (lane == 0) tma_load_2d(sK, &tmK, BAR(0), w.h * kD, krow);
+          if (lane == 1) tma_load_2d(sV, &tmV, BAR(0), w.h * kD, krow);
+        }
+        if (s >= 1) ok = load_bias(s - 1);
+      }
+      if (ok && w.nsteps > 0) ok = load_bias(w.nsteps - 1);
+      // every load of the unit is issued (its last steps are still to run): time to take the next
+      if (ok && lane == 0) mbar_arrive(ring_got(i % kRingB));
+      G += w.nsteps;
     }
-    if (ok && nsteps > 0) load_bias(nsteps - 1);
   } else if (warp == kSiluWarpsB + 1) {
-    // ---------------- tcgen05 issuer (warp 17; warp 19 idles) ----------------
-    // Per query tile s: S^T = K Q^T and dA^T = V dO^T over the whole tile (N = 128: a tcgen05.mma
+    // ---------------- tcgen05 issuer (warp 17) ----------------
+    // Per query tile: S^T = K Q^T and dA^T = V dO^T over the whole tile (N = 128: a tcgen05.mma
     // costs the same issue time at N = 64 and 128, so two 64-query halves would double it); once
     // both query halves' elementwise warps have written P^T (TMEM) and dX^T (shared memory), first
     // the next tile's S^T / dA^T (so that its elementwise work overlaps the gradient MMAs), then
     // dV += P^T_h dO_h and dK += dX^T_h Q_h for both halves and dQ_tile = dX K. The Q / dO stage
-    // is freed by two commits: after S^T / dA^T and after the gradient MMAs.
+    // is freed by two commits: after S^T / dA^T and after the gradient MMAs. A unit's first
+    // gradient MMAs (which overwrite dV and dK) wait until the previous unit's dV and dK are out of
+    // TMEM; its end is committed to `fin`.
     if (lane == 0) {
       constexpr uint32_t id_s = make_idesc_f16kind(128, 128, 0, 0, F16);
       constexpr uint32_t id_kmn = make_idesc_f16kind(128, 64, 0, 1, F16);
       constexpr uint32_t id_mnmn = make_idesc_f16kind(128, 64, 1, 1, F16);
-      bool ok = mbar_wait(BAR(0), 0, abort_flag, ctl);
       // base descriptors: K-major (lbo 16) and MN-major (lbo 16384, the 64-element block stride)
       const uint64_t k_km = make_sdesc_sw128(sK, 16, 1024), v_km = make_sdesc_sw128(sV, 16, 1024);
       const uint64_t k_mn = make_sdesc_sw128(sK, 16384, 1024);
       const uint64_t q_km = make_sdesc_sw128(sQ0, 16, 1024), q_mn = make_sdesc_sw128(sQ0, 16384, 1024);
       const uint64_t x_km = make_sdesc_sw128(sBT0, 16, 1024), x_mn = make_sdesc_sw128(sBT0, 16384, 1024);
-      auto issue_s = [&](int s) -> bool {
-        const int sq = s % 3;
-        if (!mbar_wait(qdo_full(sq), (s / 3) & 1, abort_flag, ctl)) return false;
+      auto issue_s = [&](int gs) -> bool {
+        const int sq = gs % 3;
+        if (!mbar_wait(qdo_full(sq), (gs / 3) & 1, abort_flag, ctl)) return false;
         tc_fence_after();
         const uint64_t qd = sdesc_add(q_km, sq * 32768), dod = sdesc_add(qd, 16384);
 #pragma unroll
@@ -227,11 +294,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         umma_commit(qdo_empty(sq));
         return true;
       };
-      auto issue_grad = [&](int s, int hh) {
-        const int st = s & 1, sq = s % 3;
+      auto issue_grad = [&](int gs, bool first, int hh) {
+        const int st = gs & 1, sq = gs % 3;
         const uint64_t qd = sdesc_add(q_mn, sq * 32768 + hh * 8192), dod = sdesc_add(qd, 16384);
         const uint64_t xd = sdesc_add(x_km, st * 32768 + hh * 16384);
-        const uint32_t acc0 = (s > 0 || hh > 0) ? 1u : 0u;
+        const uint32_t acc0 = (!first || hh > 0) ? 1u : 0u;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4)   // dV += P^T_h dO_h
           umma_f16_ts(tDV, tP + 32 * hh + 8 * k4, sdesc_add(dod, k4 * 2048), id_kmn, k4 > 0 ? 1u : acc0);
@@ -240,27 +307,42 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           umma_f16_ss(tDK, sdesc_add(xd, k4 * 32), sdesc_add(qd, k4 * 2048), id_kmn, k4 > 0 ? 1u : acc0);
         umma_commit(BAR(19 + hh));
       };
-      if (ok && nsteps > 0) ok = issue_s(0);
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int st = s & 1;
-        ok = mbar_wait(BAR(11), s & 1, abort_flag, ctl) && mbar_wait(BAR(12), s & 1, abort_flag, ctl);
-        if (!ok) break;
-        tc_fence_after();
-        if (s + 1 < nsteps && !issue_s(s + 1)) {
-          ok = false;
-          break;
-        }
-        issue_grad(s, 0);
-        issue_grad(s, 1);
-        const uint64_t xd = sdesc_add(x_mn, st * 32768);
+      int G = 0;
+      bool ok = true;
+      for (int i = 0; ok; ++i) {
+        int u;
+        if (!take_unit(i, u) || u >= total) break;
+        const BwdUnit w = bwd_unit(A, u);
+        if (!mbar_wait(BAR(0), i & 1, abort_flag, ctl) || !issue_s(G)) break;
+        for (int s = 0; ok && s < w.nsteps; ++s) {
+          const int gs = G + s, st = gs & 1;
+          ok = mbar_wait(BAR(11), gs & 1, abort_flag, ctl) && mbar_wait(BAR(12), gs & 1, abort_flag, ctl);
+          if (!ok) break;
+          tc_fence_after();
+          if (s + 1 < w.nsteps && !issue_s(gs + 1)) {
+            ok = false;
+            break;
+          }
+          if (s == 0 && i >= 1) {   // dV, dK of the previous unit read out of TMEM
+            if (!mbar_wait(BAR(23), (i - 1) & 1, abort_flag, ctl)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          issue_grad(gs, s == 0, 0);
+          issue_grad(gs, s == 0, 1);
+          const uint64_t xd = sdesc_add(x_mn, st * 32768);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)   // dQ_tile = dX K
-          umma_f16_ss(tDQ, sdesc_add(xd, kk * 2048), sdesc_add(k_mn, kk * 2048), id_mnmn, kk > 0 ? 1u : 0u);
-        umma_commit(BAR(13));
-        umma_commit(qdo_empty(s % 3));
-        umma_commit(BAR(7 + st));
+          for (int kk = 0; kk < 8; ++kk)   // dQ_tile = dX K
+            umma_f16_ss(tDQ, sdesc_add(xd, kk * 2048), sdesc_add(k_mn, kk * 2048), id_mnmn, kk > 0 ? 1u : 0u);
+          umma_commit(BAR(13));
+          umma_commit(qdo_empty(gs % 3));
+          umma_commit(BAR(7 + st));
+        }
+        if (ok) umma_commit(BAR(14));
+        G += w.nsteps;
       }
-      if (ok) umma_commit(BAR(14));
     }
   } else if (warp == kSiluWarpsB + 2) {
     // ---------------- TMA stores ----------------
@@ -270,36 +352,65 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // gradients are summed over the heads.
     // dQ reduce-adds from lanes 0 and 1, dX^T stores from lanes 2 and 3 (each lane waits for its own
     // bulk group; lane 0 then signals the barrier)
-    auto reduce_dq = [&](int j) -> bool {
-      if (!mbar_wait_warp(BAR(17), j & 1, abort_flag, ctl)) return false;
-      if (lane < 2) {
-        const int y = static_cast<int>(seq0) + (kt + j) * kQTile;
-        tma_reduce_add_2d(&tmDQ, sDQ + lane * 16384, h * kD + 32 * lane, y);
-        bulk_commit_group();
-        bulk_wait_group_read<0>();
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(18));
-      return true;
-    };
+    int G = 0;
     bool ok = true;
-    for (int s = 0; ok && s < nsteps; ++s) {
-      const int st = s & 1;
-      if (s >= 1 && !reduce_dq(s - 1)) { ok = false; break; }
-      if (!mbar_wait_warp(BAR(15 + st), (s >> 1) & 1, abort_flag, ctl)) { ok = false; break; }
-      if (lane == 2 || lane == 3) {
-        const int qt = kt + s;
-        const long long pair = pbase + static_cast<long long>(qt) * (qt + 1) / 2 + kt;
-        const int y = static_cast<int>((pair * a.H + h) * kQTile);
-        tma_store_2d(&tmDX, sBT0 + st * 32768 + (lane - 2) * 16384, 64 * (lane - 2), y);
-        bulk_commit_group();
-        bulk_wait_group_read<0>();
+    for (int i = 0; ok; ++i) {
+      int u;
+      if (!take_unit_warp(i, u) || u >= total) break;
+      const BwdUnit w = bwd_unit(A, u);
+      auto reduce_dq = [&](int gj, int qt) -> bool {
+        if (!mbar_wait_warp(BAR(17), gj & 1, abort_flag, ctl)) return false;
+        if (lane < 2) {
+          const int y = static_cast<int>(w.seq0) + qt * kQTile;
+          tma_reduce_add_2d(&tmDQ, sDQ + lane * 16384, w.h * kD + 32 * lane, y);
+          bulk_commit_group();
+          bulk_wait_group_read<0>();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(18));
+        return true;
+      };
+      for (int s = 0; ok && s < w.nsteps; ++s) {
+        const int gs = G + s, st = gs & 1;
+        if (s >= 1 && !reduce_dq(gs - 1, w.kt + s - 1)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait_warp(BAR(15 + st), (gs >> 1) & 1, abort_flag, ctl)) {
+          ok = false;
+          break;
+        }
+        if (lane == 2 || lane == 3) {
+          const int qt = w.kt + s;
+          const long long pair = w.pbase + static_cast<long long>(qt) * (qt + 1) / 2 + w.kt;
+          const int y = static_cast<int>((pair * a.H + w.h) * kQTile);
+          tma_store_2d(&tmDX, sBT0 + st * 32768 + (lane - 2) * 16384, 64 * (lane - 2), y);
+          bulk_commit_group();
+          bulk_wait_group_read<0>();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(7 + st));
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(7 + st));
+      if (ok && w.nsteps > 0) ok = reduce_dq(G + w.nsteps - 1, w.kt + w.nsteps - 1);
+      G += w.nsteps;
     }
-    if (ok && nsteps > 0) reduce_dq(nsteps - 1);
     bulk_wait_group_all();
+  } else if (warp == kSiluWarpsB + 3) {
+    // ---------------- unit scheduler ----------------
+    // unit 0 is blockIdx.x, later ones come from the counter, each taken once the producer has
+    // issued every load of the one before: a CTA claims its next unit a few steps before it can
+    // start it, so the units (longest first) go to the CTAs that come free first
+    if (lane == 0) {
+      for (int i = 0;; ++i) {
+        const int r = i % kRingB;
+        if (i >= 1 && !mbar_wait(ring_got((i - 1) % kRingB), ((i - 1) / kRingB) & 1, abort_flag, ctl)) break;
+        const int u = i == 0 ? static_cast<int>(blockIdx.x) : static_cast<int>(gridDim.x) + atomicAdd(A.sched, 1);
+        if (i >= kRingB && !mbar_wait(ring_empty(r), ((i / kRingB) - 1) & 1, abort_flag, ctl)) break;
+        ring[r] = u;
+        mbar_arrive(ring_full(r));
+        if (u >= total) break;
+      }
+    }
   } else if (warp < kSiluWarpsB) {
     // ---------------- elementwise warps ----------------
     // warp w: key rows [32 (w & 3), +32) (TMEM lane quadrant), query half hq = (w >> 2) & 1,
@@ -309,18 +420,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int sub = warp >> 3;
     const int rj = quad * 32 + lane;      // key row == TMEM lane of S^T, dA^T, dV, dK
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    // in a pack, queries past the end of the key row's own sequence are masked
-    int seg_end = n;
-    if (packed && rj < n) {
-      const long long g = seq0 + rj;
-      int s0 = b, s1 = b - kt_item;
-      while (s1 - s0 > 1) {
-        const int mid = (s0 + s1) >> 1;
-        if (a.offsets[mid] <= g) s0 = mid;
-        else s1 = mid;
-      }
-      seg_end = static_cast<int>(a.offsets[s0 + 1] - seq0);
-    }
     const float inv_N = a.inv_N;
     const float cN = 0.5f * inv_N;
     bool ok = true;
@@ -378,10 +477,29 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
     };
+    int G = 0;
+    for (int i = 0; ok; ++i) {
+      int u;
+      if (!take_unit_warp(i, u) || u >= total) break;
+      const BwdUnit w = bwd_unit(A, u);
+      const int kt = w.kt, n = w.n, nt = w.nt, nsteps = w.nsteps;
+      const long long seq0 = w.seq0;
+      // in a pack, queries past the end of the key row's own sequence are masked
+      int seg_end = n;
+      if (w.packed && rj < n) {
+        const long long g = seq0 + rj;
+        int s0 = w.b, s1 = w.b - w.kt_item;
+        while (s1 - s0 > 1) {
+          const int mid = (s0 + s1) >> 1;
+          if (a.offsets[mid] <= g) s0 = mid;
+          else s1 = mid;
+        }
+        seg_end = static_cast<int>(a.offsets[s0 + 1] - seq0);
+      }
     for (int s = 0; ok && s < nsteps; ++s) {
-      const int qt = kt + s, st = s & 1;
-      if (!mbar_wait(BAR(5 + st), (s >> 1) & 1, abort_flag, ctl) ||
-          !mbar_wait(BAR(9 + hq), s & 1, abort_flag, ctl)) {
+      const int gs = G + s, qt = kt + s, st = gs & 1;
+      if (!mbar_wait(BAR(5 + st), (gs >> 1) & 1, abort_flag, ctl) ||
+          !mbar_wait(BAR(9 + hq), gs & 1, abort_flag, ctl)) {
         ok = false;
         break;
       }
@@ -409,8 +527,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         uint32_t pp[8], dxp[8];
         if (need_mask) piece(sv, dav, hb, pp, dxp, true, c0, lo_col, hi_col);
         else piece(sv, dav, hb, pp, dxp, false, c0, lo_col, hi_col);
-        if (pc == 0 && s >= 1) {   // the previous tile's dV MMA has read P^T_h
-          if (!mbar_wait(BAR(19 + hq), (s - 1) & 1, abort_flag, ctl)) { ok = false; break; }
+        if (pc == 0 && gs >= 1) {   // the previous tile's dV MMA has read P^T_h
+          if (!mbar_wait(BAR(19 + hq), (gs - 1) & 1, abort_flag, ctl)) { ok = false; break; }
           tc_fence_after();
         }
         tmem_st_32x32b_x8(tP + lane_base + 32 * hq + 16 * sub + 8 * pc, pp);
@@ -422,22 +540,27 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       if (!ok) break;
       // (half b) the previous tile's dQ: its MMAs were issued after this tile's S^T_b
-      if (hq == 1 && s >= 1 && !stage_dq(s - 1)) { ok = false; break; }
+      if (hq == 1 && s >= 1 && !stage_dq(gs - 1)) { ok = false; break; }
       tmem_st_wait();
       tc_fence_before();
       fence_proxy_async_smem();
       mbar_arrive(BAR(11 + hq));    // P^T_h in TMEM, dX^T_h in shared memory
       mbar_arrive(BAR(15 + st));
     }
-    if (ok && hq == 1 && nsteps > 0 && !stage_dq(nsteps - 1)) ok = false;
-    if (ok && mbar_wait(BAR(14), 0, abort_flag, ctl)) {
+    if (ok && hq == 1 && nsteps > 0 && !stage_dq(G + nsteps - 1)) ok = false;
+    if (ok && !mbar_wait(BAR(14), i & 1, abort_flag, ctl)) ok = false;
+    if (ok) {
       tc_fence_after();
-      // dK, dV: key row = TMEM lane, columns [16 (2 hq + sub), +16)
+      // dK, dV: key row = TMEM lane, columns [16 (2 hq + sub), +16); then the accumulators are free
+      // for the next unit
       const int cc = 16 * (2 * hq + sub);
       uint32_t vk[16], vv[16];
       tmem_ld_32x32b_x16(tDK + lane_base + cc, vk);
       tmem_ld_32x32b_x16(tDV + lane_base + cc, vv);
       tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(BAR(23));
+      const int h = w.h;
       if (kt * kQTile + rj < n) {
         const long long row = seq0 + kt * kQTile + rj;
         float4* dk = reinterpret_cast<float4*>(A.dk + row * A.ld_g + h * kD + cc);
@@ -451,6 +574,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
     }
+    G += nsteps;
+    }
   }
 
   tc_fence_before();
@@ -460,6 +585,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tmem_dealloc(tmem, 512);
   }
 }
+
+// ----------------------------------------------------------------------------------------------
+// table gradients from the per-head dX^T tiles
+// ----------------------------------------------------------------------------------------------
+// Two blocks per causal tile pair, 64 key rows each. Thread (warp w, lane l) holds the fp32 head
+// sum of key rows j_k = 64 y + 8 w + 2 k + l / 16 (k < 4), queries [c0, c0 + 8), c0 = 8 (l % 16).
+//  d rab_pos: element (j, i) of the tile lies on diagonal i - j + 127 (relative position
+//   128 (qt - kt) + i - j). A thread's 32 elements fall on 14 diagonals (e - 2k = const), summed in
 
 // ----------------------------------------------------------------------------------------------
 // table gradients from the per-head dX^T tiles
@@ -662,7 +795,10 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   auto kern = f16 ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), BwdSmem::kTotal);
   if (e != cudaSuccess) return e;
-  const long long blocks = a.capacity * a.H;
+  // persistent: one CTA per SM (the units beyond the grid come from the work list's counter)
+  const long long units = a.capacity * a.H;
+  const long long blocks = units < sm_count() ? units : sm_count();
+  if (!A.sched) return cudaErrorInvalidValue;
   e = prof_record(kProfAttnBwd, false, st);
   if (e == cudaSuccess)
     e = launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(kThreadsB), BwdSmem::kTotal, st, tq, tk, tv, tdo,

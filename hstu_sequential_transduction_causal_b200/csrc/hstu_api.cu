@@ -204,10 +204,11 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
     A.bias_cached = 1;
   }
   A.kitems = reinterpret_cast<int32_t*>(w + lay.kitems); A.kcount = kcount;
+  A.sched = count + 5;   // [276, 280) of the workspace header region
   a.pack = reinterpret_cast<const int32_t*>(w + lay.f.pack);
   e = launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, a.status, st,
                       reinterpret_cast<long long*>(w + lay.f.pairs), reinterpret_cast<int32_t*>(w + lay.kitems),
-                      kcount, nullptr, reinterpret_cast<int32_t*>(w + lay.f.pack));
+                      kcount, A.sched, reinterpret_cast<int32_t*>(w + lay.f.pack));
   if (e == cudaSuccess) e = attn_bwd_tc(A, st);
   return cuda_status(e);
 }

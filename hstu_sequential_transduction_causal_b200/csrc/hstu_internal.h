@@ -196,6 +196,7 @@ struct AttnBwdArgs {
   void* dxt;                   // fp16 [max_pairs, H, 128 keys, 128 queries] dX^T of every (pair, head)
   const int32_t* kitems;       // backward work list (b, key tile)
   const int32_t* kcount;
+  int32_t* sched;              // the persistent backward's unit counter, zeroed by the work list
   int bias_cached;             // bias_t and bucket_t were written by the forward: no bias kernel
 };
 
