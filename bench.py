@@ -359,10 +359,12 @@ def main():
     dy = to_dev(wl.dy, torch.bfloat16, dev)
     y = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
     dx = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
-    sv = SavedActs.empty(T, D, torch.bfloat16, keep_z=backward, device=dev)
-    svs = sv.struct()
     adesc = H.make_attn_desc(Hh, D // Hh, D // Hh, 1.0 / wl.N, wl.pos_max_len, H.HSTU_F16, 4 * D, 4 * D, 4 * D, D)
     ldesc = H.make_layer_desc(D, Hh, 1.0 / wl.N, wl.pos_max_len, H.HSTU_BF16, H.HSTU_BF16, H.HSTU_BF16)
+    # with a backward, the forward also writes the attention backward's bias tiles (saved.attn_bias)
+    sv = SavedActs.empty(T, D, torch.bfloat16, keep_z=backward, device=dev,
+                         bias_cache_bytes=H.hstu_layer_bias_cache_size(ldesc, jag.struct) if backward else 0)
+    svs = sv.struct()
     ws = workspace(max(H.hstu_attn_workspace_size(adesc, jag.struct),
                        H.hstu_layer_bwd_workspace_size(ldesc, jag.struct) if backward else 0), dev)
     flat, views = grad_buffer(D, wl.pos_max_len, dev)
@@ -381,9 +383,10 @@ def main():
     # f1 GEMM | work list, bias tiles, attention | LN-gate | fp16 W2 copy, f2 GEMM
     n_fwd_kernels = 7
     # fp16 dy with the db2 partial sums | fp16 copies of x, W1, W2 (one launch) | dG with dW2 (one grouped
-    # GEMM launch) | LN-gate bwd | finish of db2, dgamma, dbeta | work list, transposed bias tiles, attention
-    # bwd, table gradients | dZ with the db1 partial sums | finish of db1 | dX with dW1 (one grouped launch)
-    n_bwd_kernels = 12
+    # GEMM launch) | LN-gate bwd | finish of db2, dgamma, dbeta | work list, attention bwd, table gradients
+    # (the transposed bias tiles come from the forward's cache) | dZ with the db1 partial sums | finish of
+    # db1 | dX with dW1 (one grouped launch)
+    n_bwd_kernels = 11
     names = ["uvqk", "attn", "norm_gate", "out_proj"] + (["backward"] if backward else [])
 
     def attention_forward():
