@@ -382,11 +382,11 @@ def main():
     # kernels of ours per step (cross-checked against the ncu launch list in profiles/)
     # f1 GEMM | work list, bias tiles, attention | LN-gate | fp16 W2 copy, f2 GEMM
     n_fwd_kernels = 7
-    # fp16 dy with the db2 partial sums | fp16 copies of x, W1, W2 (one launch) | dG with dW2 (one grouped
-    # GEMM launch) | LN-gate bwd | finish of db2, dgamma, dbeta | work list, attention bwd, table gradients
-    # (the transposed bias tiles come from the forward's cache) | dZ with the db1 partial sums | finish of
-    # db1 | dX with dW1 (one grouped launch)
-    n_bwd_kernels = 11
+    # fp16 dy with the db2 partial sums and the fp16 copies of x, W1, W2 (one launch) | dG with dW2 (one
+    # grouped GEMM launch) | LN-gate bwd | work list, attention bwd, table gradients (the transposed bias
+    # tiles come from the forward's cache) | dZ with the db1 partial sums | finish of db2, dgamma, dbeta
+    # and db1 (one launch) | dX with dW1 (one grouped launch)
+    n_bwd_kernels = 9
     names = ["uvqk", "attn", "norm_gate", "out_proj"] + (["backward"] if backward else [])
 
     def attention_forward():
@@ -401,8 +401,8 @@ def main():
     prof_ms = {k: [] for k in prof_kernels}
 
     # data parallelism: the gradient sum runs on a side stream, started by the events hstu_layer_bwd
-    # records when dW2, db2, dgamma, dbeta and the tables are final (reduced while dZ, db1, dW1 and dX
-    # are computed) and when dW1, db1 are final (reduced while the dX GEMM runs)
+    # records when dW2, db2, dgamma, dbeta, db1 and the tables are final (reduced while the launch that
+    # computes dX and dW1 runs) and when dW1 is final
     comm = torch.cuda.Stream(device=dev) if world > 1 else None
     n_late = 4 * D * D + 4 * D             # dW1, db1 lead the flat buffer
     if comm is not None and backward:

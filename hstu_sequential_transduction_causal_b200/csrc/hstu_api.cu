@@ -930,16 +930,14 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   float* part_ln = reinterpret_cast<float*>(wsb + lay.part_ln);
   float* part_dz = reinterpret_cast<float*>(wsb + lay.part_dz);
   int parts_dy = 0, parts_ln = 0;
-  // the fp16 copy of dY (unless the caller passed one) together with the partial sums of db2
-  e = rows_to_f16_colsum(T, D, y_dt, dy, dy_f16 ? nullptr : wsb + lay.dy_f16, part_dy, &parts_dy, st);
-  if (e != cudaSuccess) return cuda_status(e);
-  {   // the other fp16 GEMM operand copies, one launch
+  {   // one launch: the fp16 copy of dY (unless the caller passed one) with the partial sums of db2,
+      // and the other fp16 GEMM operand copies
     ConvertJob jobs[4];
     int nj = 0;
     if (!x_f16) jobs[nj++] = ConvertJob{x, wsb + lay.x_f16, T * D, x_dt};
     jobs[nj++] = ConvertJob{w->W1, w1_f16, 4ll * D * D, kDtBF16};
     jobs[nj++] = ConvertJob{w->W2, w2_f16, 1ll * D * D, kDtBF16};
-    e = convert_many_to_f16(jobs, nj, st);
+    e = rows_to_f16_colsum(T, D, y_dt, dy, dy_f16 ? nullptr : wsb + lay.dy_f16, part_dy, &parts_dy, jobs, nj, st);
   }
   if (e != cudaSuccess) return cuda_status(e);
   float* dG = reinterpret_cast<float*>(wsb + lay.dg);
@@ -963,34 +961,30 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
     g2.epi.kind = kEpiAtomic; g2.epi.out0 = gr->dW2; g2.epi.out0_dt = kDtF32; g2.epi.ld_out0 = D; g2.status = status;
     e = gemm_bf16_group(gg, 2, gemm_sched(ws), st);
   }
-  // 2. norm-gate backward: dO (fp16), dZ_U (fp16), partial dgamma | dbeta; then db2, dgamma and dbeta
-  // finished by one launch straight into the caller's buffers
+  // 2. norm-gate backward: dO (fp16), dZ_U (fp16), partial dgamma | dbeta (finished with db2 and db1
+  // after the dZ assembly)
   if (e == cudaSuccess)
     e = norm_gate_bwd(T, D, kDtF16, dG, static_cast<const float*>(saved->o), saved->uvqk, saved->z, 4ll * D, w->gamma,
                       w->beta, saved->mu, saved->rstd, dO, dz, 4ll * D, part_ln, &parts_ln, st, status);
-  if (e == cudaSuccess) {
-    const ColsumJob jobs[3] = {{part_dy, D, parts_dy, D, gr->db2},
-                               {part_ln, 2ll * D, parts_ln, D, gr->dgamma},
-                               {part_ln + D, 2ll * D, parts_ln, D, gr->dbeta}};
-    e = colsum_final_multi(jobs, 3, st);
-  }
   if (e != cudaSuccess) return cuda_status(e);
   // 3. attention backward
   const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
   s = run_attn_bwd(&ad, jag, uvqk + 2 * D * 2, uvqk + 3 * D * 2, uvqk + 1 * D * 2, dO, w->rab_pos, w->rab_time, dq, dk,
                    dv, D, gr->drab_pos, gr->drab_time, ws, st, nullptr, nullptr, saved->attn_bias);
   if (s != HSTU_OK) return s;
-  if (g_ready_events[0]) {   // dW2, db2, dgamma, dbeta and the table gradients are final
-    e = cudaEventRecord(g_ready_events[0], st);
-    if (e != cudaSuccess) return cuda_status(e);
-  }
-  // 4. SiLU backward into dZ[:, D:4D] with the partial sums of db1 = sum_t dZ, then their finish
+  // 4. SiLU backward into dZ[:, D:4D] with the partial sums of db1 = sum_t dZ; then db2, dgamma,
+  // dbeta and db1 finished by one launch straight into the caller's buffers
   int parts_dz = 0;
   e = dz_assemble(T, D, kDtF16, dv, dq, dk, saved->z, 4ll * D, dz, 4ll * D, part_dz, &parts_dz, st);
   if (e == cudaSuccess) {
-    const ColsumJob job{part_dz, 4ll * D, parts_dz, 4 * D, gr->db1};
-    e = colsum_final_multi(&job, 1, st);
+    const ColsumJob jobs[4] = {{part_dy, D, parts_dy, D, gr->db2},
+                               {part_ln, 2ll * D, parts_ln, D, gr->dgamma},
+                               {part_ln + D, 2ll * D, parts_ln, D, gr->dbeta},
+                               {part_dz, 4ll * D, parts_dz, 4 * D, gr->db1}};
+    e = colsum_final_multi(jobs, 4, st);
   }
+  // dW2, db2, dgamma, dbeta, db1 and the table gradients are final
+  if (e == cudaSuccess && g_ready_events[0]) e = cudaEventRecord(g_ready_events[0], st);
   // 5. f1 backward in one launch: dX = dY + dZ W1 and dW1 = dZ^T X (fp16 dZ, x and W1; dW1 split
   //    over K = T into units of about a third of a dX unit, reduced into the zeroed dW1)
   if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW1, 0, sizeof(float) * 4 * D * D, st);
@@ -1014,7 +1008,7 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
     g4.status = status;
     e = gemm_bf16_group(gg, 2, gemm_sched(ws), st);
   }
-  if (e == cudaSuccess && g_ready_events[1]) e = cudaEventRecord(g_ready_events[1], st);   // dW1, db1 final
+  if (e == cudaSuccess && g_ready_events[1]) e = cudaEventRecord(g_ready_events[1], st);   // dW1 final
   if (nin && e == cudaSuccess)
     e = ln_in_bwd(T, D, desc->x_dtype == HSTU_F32 ? kDtF32 : kDtBF16, desc->y_dtype == HSTU_F32 ? kDtF32 : kDtBF16,
                   reinterpret_cast<const float*>(wsb + nin_dxn), x, dy, nin->gamma, nin->mu, nin->rstd, dx, dx_f16,

@@ -254,10 +254,17 @@ cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const f
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
                         const void* z, int64_t ld_z, void* dz, int64_t ld_dz, float* partial, int* parts,
                         cudaStream_t st);
-// [T, D] rows (fp32, bf16 or fp16) to fp16 (out may be null) and their partial column sums into
-// partial [*parts, D] (at most kTailParts rows).
+// A tensor of n elements (fp32, bf16 or fp16) converted to fp16.
+struct ConvertJob {
+  const void* in;
+  void* out;
+  int64_t n;
+  int in_dt;
+};
+// One launch: [T, D] rows (fp32, bf16 or fp16) to fp16 (out may be null) with their partial column
+// sums into partial [*parts, D] (at most kTailParts rows), and up to four other tensors to fp16.
 cudaError_t rows_to_f16_colsum(int64_t T, int D, int in_dt, const void* in, void* out, float* partial, int* parts,
-                               cudaStream_t st);
+                               const ConvertJob* jobs, int njobs, cudaStream_t st);
 // Most partial rows rows_to_f16_colsum writes.
 constexpr int kTailParts = 296;
 // Several column-sum finishes in one launch.
@@ -276,14 +283,7 @@ struct ColsumJobs {
 cudaError_t colsum_final_multi(const ColsumJob* jobs, int njobs, cudaStream_t st);
 size_t colsum_partial_floats(int cols);
 cudaError_t convert_dtype(const void* in, int in_dt, void* out, int out_dt, int64_t n, cudaStream_t st);
-// Up to four conversions to fp16 (inputs fp32, bf16 or fp16) in one launch.
-struct ConvertJob {
-  const void* in;
-  void* out;
-  int64_t n;
-  int in_dt;
-};
-cudaError_t convert_many_to_f16(const ConvertJob* jobs, int njobs, cudaStream_t st);
+
 cudaError_t column_sum(const void* in, int dt, int64_t rows, int cols, int64_t ld, float* partial, float* out,
                        cudaStream_t st);
 

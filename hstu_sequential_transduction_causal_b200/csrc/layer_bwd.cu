@@ -307,18 +307,54 @@ dz_assemble_kernel(int64_t T, int D, const float* __restrict__ dv, const float* 
   }
 }
 
-// dY converted to fp16 (out, may be null when the caller holds an fp16 copy) and the partial column
-// sums of dY (the db2 of f2's bias): block b sums rows [b R, (b+1) R) into partial[b][0 .. D); its
-// threads own 8 columns each (D / 8 per row, 256 / (D / 8) rows side by side) and keep four rows'
-// loads in flight each.
+struct ConvertBatch {
+  ConvertJob job[4];
+  int first_block[5];   // block b converts job j with first_block[j] <= b < first_block[j + 1]
+  int njobs;
+};
+
+// Block blk of a batch of conversions to fp16: it finds its job, then 8 elements per thread.
+__device__ __forceinline__ void convert_block(const ConvertBatch& cb, int blk) {
+  int j = 0;
+  while (j + 1 < cb.njobs && blk >= cb.first_block[j + 1]) ++j;
+  const ConvertJob& jb = cb.job[j];
+  const int64_t i = (static_cast<int64_t>(blk - cb.first_block[j]) * blockDim.x + threadIdx.x) * 8;
+  if (i >= jb.n) return;
+  const int cnt = jb.n - i >= 8 ? 8 : static_cast<int>(jb.n - i);
+  float v[8];
+  if (cnt == 8) {
+    if (jb.in_dt == kDtF32) load_vec<8, kDtF32>(jb.in, i, v);
+    else if (jb.in_dt == kDtBF16) load_vec<8, kDtBF16>(jb.in, i, v);
+    else load_vec<8, kDtF16>(jb.in, i, v);
+    store_vec<8, kDtF16>(jb.out, i, v);
+  } else {
+    for (int k = 0; k < cnt; ++k) {
+      if (jb.in_dt == kDtF32) load_vec<1, kDtF32>(jb.in, i + k, &v[0]);
+      else if (jb.in_dt == kDtBF16) load_vec<1, kDtBF16>(jb.in, i + k, &v[0]);
+      else load_vec<1, kDtF16>(jb.in, i + k, &v[0]);
+      reinterpret_cast<__half*>(jb.out)[i + k] = __float2half_rn(v[0]);
+    }
+  }
+}
+
+// The backward's first launch, two independent jobs over one grid:
+// - blocks [0, col_blocks): dY converted to fp16 (out, may be null when the caller holds an fp16
+//   copy) and the partial column sums of dY (the db2 of f2's bias): block b sums rows [b R, (b+1) R)
+//   into partial[b][0 .. D); its threads own 8 columns each (D / 8 per row, 256 / (D / 8) rows side
+//   by side) and keep four rows' loads in flight each;
+// - the rest: the fp16 copies of the other GEMM operands (cb).
 template <int D, int IT>
 __global__ void __launch_bounds__(kTailThreads)
 rows_to_f16_colsum_kernel(int64_t T, const void* __restrict__ in, void* __restrict__ out, int64_t rows_per,
-                          float* __restrict__ partial) {
+                          float* __restrict__ partial, int col_blocks, ConvertBatch cb) {
   constexpr int TPR = D / 8, RP = kTailThreads / TPR, U = 4;
   static_assert(RP >= 1 && kTailThreads % TPR == 0, "whole rows per block");
   __shared__ float s_red[RP > 1 ? RP - 1 : 1][D];
   pdl_enter();
+  if (static_cast<int>(blockIdx.x) >= col_blocks) {   // (block-uniform)
+    convert_block(cb, static_cast<int>(blockIdx.x) - col_blocks);
+    return;
+  }
   const int g = threadIdx.x % TPR, rp = threadIdx.x / TPR;
   const int c = 8 * g;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * rows_per;
@@ -549,16 +585,30 @@ cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const flo
 }
 
 cudaError_t rows_to_f16_colsum(int64_t T, int D, int in_dt, const void* in, void* out, float* partial, int* parts,
-                               cudaStream_t st) {
+                               const ConvertJob* jobs, int njobs, cudaStream_t st) {
   *parts = 0;
-  if (T == 0) return cudaSuccess;
-  int64_t rows_per = 0;
-  const int g = tail_parts(T, &rows_per);
+  ConvertBatch cb{};
+  int nb = 0, k = 0;
+  for (int j = 0; j < njobs && j < 4; ++j) {
+    if (jobs[j].n <= 0) continue;
+    if (jobs[j].in_dt != kDtF32 && jobs[j].in_dt != kDtBF16 && jobs[j].in_dt != kDtF16) return cudaErrorInvalidValue;
+    cb.job[k] = jobs[j];
+    cb.first_block[k] = nb;
+    const int64_t blocks = ((jobs[j].n + 7) / 8 + 255) / 256;
+    if (nb + blocks > 0x3fffffffLL) return cudaErrorInvalidValue;
+    nb += static_cast<int>(blocks);
+    ++k;
+  }
+  cb.first_block[k] = nb;
+  cb.njobs = k;
+  int64_t rows_per = 1;
+  const int g = T > 0 ? tail_parts(T, &rows_per) : 0;
   *parts = g;
+  if (g + nb == 0) return cudaSuccess;
 #define HSTU_RC(DD, IT)                                                                                          \
   if (D == DD && in_dt == IT)                                                                                    \
-    return launch_pdl(rows_to_f16_colsum_kernel<DD, IT>, dim3(g), dim3(kTailThreads), 0, st, T, in, out, rows_per, \
-                      partial);
+    return launch_pdl(rows_to_f16_colsum_kernel<DD, IT>, dim3(g + nb), dim3(kTailThreads), 0, st, T, in, out,    \
+                      rows_per, partial, g, cb);
   HSTU_RC(256, kDtF32)
   HSTU_RC(512, kDtF32)
   HSTU_RC(256, kDtBF16)
@@ -583,58 +633,6 @@ cudaError_t colsum_final_multi(const ColsumJob* jobs, int njobs, cudaStream_t st
   cj.first_block[k] = nb;
   cj.njobs = k;
   return launch_pdl(colsum_final_multi_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, st, cj);
-}
-
-struct ConvertBatch {
-  ConvertJob job[4];
-  int first_block[5];   // block b converts job j with first_block[j] <= b < first_block[j + 1]
-  int njobs;
-};
-
-// Several tensors converted to fp16 by one launch: each block finds its job, then 8 elements per
-// thread as in convert_kernel.
-__global__ void __launch_bounds__(256)
-convert_many_kernel(ConvertBatch cb) {
-  pdl_enter();
-  int j = 0;
-  while (j + 1 < cb.njobs && static_cast<int>(blockIdx.x) >= cb.first_block[j + 1]) ++j;
-  const ConvertJob& jb = cb.job[j];
-  const int64_t i = (static_cast<int64_t>(blockIdx.x - cb.first_block[j]) * blockDim.x + threadIdx.x) * 8;
-  if (i >= jb.n) return;
-  const int cnt = jb.n - i >= 8 ? 8 : static_cast<int>(jb.n - i);
-  float v[8];
-  if (cnt == 8) {
-    if (jb.in_dt == kDtF32) load_vec<8, kDtF32>(jb.in, i, v);
-    else if (jb.in_dt == kDtBF16) load_vec<8, kDtBF16>(jb.in, i, v);
-    else load_vec<8, kDtF16>(jb.in, i, v);
-    store_vec<8, kDtF16>(jb.out, i, v);
-  } else {
-    for (int k = 0; k < cnt; ++k) {
-      if (jb.in_dt == kDtF32) load_vec<1, kDtF32>(jb.in, i + k, &v[0]);
-      else if (jb.in_dt == kDtBF16) load_vec<1, kDtBF16>(jb.in, i + k, &v[0]);
-      else load_vec<1, kDtF16>(jb.in, i + k, &v[0]);
-      reinterpret_cast<__half*>(jb.out)[i + k] = __float2half_rn(v[0]);
-    }
-  }
-}
-
-cudaError_t convert_many_to_f16(const ConvertJob* jobs, int njobs, cudaStream_t st) {
-  ConvertBatch cb{};
-  int nb = 0, k = 0;
-  for (int j = 0; j < njobs && j < 4; ++j) {
-    if (jobs[j].n <= 0) continue;
-    if (jobs[j].in_dt != kDtF32 && jobs[j].in_dt != kDtBF16 && jobs[j].in_dt != kDtF16) return cudaErrorInvalidValue;
-    cb.job[k] = jobs[j];
-    cb.first_block[k] = nb;
-    const int64_t blocks = ((jobs[j].n + 7) / 8 + 255) / 256;
-    if (nb + blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-    nb += static_cast<int>(blocks);
-    ++k;
-  }
-  if (k == 0) return cudaSuccess;
-  cb.first_block[k] = nb;
-  cb.njobs = k;
-  return launch_pdl(convert_many_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, st, cb);
 }
 
 cudaError_t convert_dtype(const void* in, int in_dt, void* out, int out_dt, int64_t n, cudaStream_t st) {

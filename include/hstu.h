@@ -494,9 +494,10 @@ hstu_status_t hstu_dp_partition(const int64_t* lengths, int32_t B, int32_t D, in
 
 /* Events for overlapping the gradient all-reduce of data parallelism with the rest of a backward:
  * until the next call, every hstu_layer_bwd of this host thread records `early` on its stream once
- * dW2, db2, dgamma, dbeta, drab_pos and drab_time are final (before the SiLU and f1 backward), and
- * `w1` once dW1 and db1 are final (before the dX GEMM). A communication stream that waits on them
- * can reduce those gradients while the remaining kernels run. Under stream capture they are
+ * dW2, db2, dgamma, dbeta, db1, drab_pos and drab_time are final (before the f1 backward GEMMs), and
+ * `w1` once dW1 is final too (after the launch that computes dX and dW1; with the input-LayerNorm
+ * variant, before its backward). A communication stream that waits on them can reduce those
+ * gradients while the remaining kernels run. Under stream capture they are
  * recorded as capture dependencies, so a stream that waits on them forks from the captured graph.
  * Both NULL disables; HSTU_ERR_INVALID_ARG when only one is NULL. */
 hstu_status_t hstu_layer_bwd_ready_events(void* early, void* w1);
