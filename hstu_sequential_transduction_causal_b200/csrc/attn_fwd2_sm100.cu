@@ -1024,9 +1024,15 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
   const int mt = (a.max_len + kQTile - 1) / kQTile;
   if (mt == 0) return cudaSuccess;
+  // with the layer's bias cache the kernel stages the backward's key-major tiles in dynamic shared memory
+  const int bias_dyn = a.bias_t_out ? kBiasStageBytes : 0;
+  if (bias_dyn) {
+    e = ensure_smem_attr(reinterpret_cast<const void*>(attn_bias_kernel), bias_dyn);
+    if (e != cudaSuccess) return e;
+  }
   e = launch_pdl(attn_bias_kernel,
                  dim3(static_cast<unsigned>(bias_tile_grid(a.max_pairs, a.bias_heads)), static_cast<unsigned>(a.bias_heads)),
-                 dim3(kBiasThreads), 0, st, a);
+                 dim3(kBiasThreads), bias_dyn, st, a);
   if (e != cudaSuccess) return e;
   const bool f16 = a.in_f16 != 0;
   // the persistent kernel's unit counter lives in the workspace header (reset by the work list), its

@@ -157,11 +157,18 @@ __device__ __forceinline__ SeqTables stage_seq_tables(const AttnArgs& a, long lo
 // tile; with a type term each element also adds rab_type[type_query][type_key]. BUCKETS: also the u8
 // bucket tile (head-independent, written by the hb = 0 blocks). False when `pair` is past the batch's
 // last pair. A block that calls it again must synchronise first (the staging arrays are reused).
+// Key-major staging of a query-major pass that also produces the backward's tiles: the fp16 tile
+// with rows of 130 halfs and the buckets with rows of 132 bytes (odd word strides: the transposed
+// stores of a half-warp fall in distinct banks).
+constexpr int kTStride = 130, kBStride = 132;
+constexpr int kBiasStageBytes = kQTile * kTStride * 2 + kQTile * kBStride;   // 50,176
+
 template <bool TRANSPOSED, bool BUCKETS>
 __device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, const BiasConst& cst, const SeqTables& sq,
                                                 long long pair, int hb, uint16_t* __restrict__ tile,
                                                 uint8_t* __restrict__ btile, uint16_t* __restrict__ tile_t,
-                                                uint8_t* __restrict__ btile_t) {
+                                                uint8_t* __restrict__ btile_t, uint16_t* __restrict__ s_tt,
+                                                uint8_t* __restrict__ s_tb) {
   __shared__ TileTimes s_t;
   __shared__ float s_win[256];
   __shared__ int s_ty[256];
@@ -187,7 +194,9 @@ __device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, const BiasCon
   const int cl = 2 * (tid & 15), rr = tid >> 4;
   // one pass over the tile: query-major (KEY_MAJOR false) or key-major; bout (nullable) receives the
   // buckets in the same layout
-  auto row_pass = [&](auto fast_tag, auto key_major_tag, uint16_t* __restrict__ out, uint8_t* __restrict__ bout) {
+  // stage (nullable): also write each element, key-major, into s_tt / s_tb
+  auto row_pass = [&](auto fast_tag, auto key_major_tag, uint16_t* __restrict__ out, uint8_t* __restrict__ bout,
+                      bool stage) {
     constexpr bool kFast = decltype(fast_tag)::value;
     constexpr bool kTr = decltype(key_major_tag)::value;
     // staging index of a row / column token: queries at [0, 128), keys at [128, 256)
@@ -220,19 +229,34 @@ __device__ __forceinline__ bool bias_tile_block(const AttnArgs& a, const BiasCon
           }
           v2[x] = v;
           bw |= static_cast<uint32_t>(bkt) << (8 * x);
+          if (stage) {
+            s_tt[c * kTStride + r] = __half_as_ushort(__float2half_rn(v));
+            s_tb[c * kBStride + r] = static_cast<uint8_t>(bkt);
+          }
         }
         *reinterpret_cast<uint32_t*>(out + r * kQTile + cl + 32 * e) = pack_f16x2(v2[0], v2[1]);
         if (bout) *reinterpret_cast<uint16_t*>(bout + r * kQTile + cl + 32 * e) = static_cast<uint16_t>(bw);
       }
     }
   };
-  auto pass = [&](auto key_major_tag, uint16_t* out, uint8_t* bout) {
-    if (fast) row_pass(BoolTag<true>{}, key_major_tag, out, bout);
-    else row_pass(BoolTag<false>{}, key_major_tag, out, bout);
-  };
-  pass(BoolTag<TRANSPOSED>{}, tile, BUCKETS && hb == 0 ? btile : nullptr);
-  // the backward's key-major tile and buckets as well (a forward that caches them for its backward)
-  if (!TRANSPOSED && tile_t) pass(BoolTag<true>{}, tile_t, hb == 0 ? btile_t : nullptr);
+  // the backward's key-major tile and buckets as well (a forward that caches them for its backward):
+  // staged transposed in shared memory by the same pass, then copied out row by row
+  const bool stage = !TRANSPOSED && tile_t && s_tt && s_tb;
+  if (fast) row_pass(BoolTag<true>{}, BoolTag<TRANSPOSED>{}, tile, BUCKETS && hb == 0 ? btile : nullptr, stage);
+  else row_pass(BoolTag<false>{}, BoolTag<TRANSPOSED>{}, tile, BUCKETS && hb == 0 ? btile : nullptr, stage);
+  if (stage) {
+    __syncthreads();
+    const uint32_t* st32 = reinterpret_cast<const uint32_t*>(s_tt);
+    uint32_t* gt = reinterpret_cast<uint32_t*>(tile_t);
+    for (int idx = tid; idx < kQTile * kQTile / 2; idx += kBiasThreads)
+      gt[idx] = st32[(idx >> 6) * (kTStride / 2) + (idx & 63)];
+    if (hb == 0 && btile_t) {
+      const uint32_t* sb32 = reinterpret_cast<const uint32_t*>(s_tb);
+      uint32_t* gb = reinterpret_cast<uint32_t*>(btile_t);
+      for (int idx = tid; idx < kQTile * kQTile / 4; idx += kBiasThreads)
+        gb[idx] = sb32[(idx >> 5) * (kBStride / 4) + (idx & 31)];
+    }
+  }
   return true;
 }
 
@@ -252,6 +276,15 @@ __device__ __forceinline__ void bias_tiles(const AttnArgs& a, uint16_t* __restri
   bias_const_load(s_c, a, hb);
   pdl_wait();
   const SeqTables sq = stage_seq_tables(a, s_pb, s_off, s_pack);
+  // the query-major kernel that also writes the backward's tiles is launched with kBiasStageBytes of
+  // dynamic shared memory for their staging
+  extern __shared__ __align__(16) uint8_t bias_stage_dyn[];
+  uint16_t* stt = nullptr;
+  uint8_t* stb = nullptr;
+  if (!TRANSPOSED && a.bias_t_out) {
+    stt = reinterpret_cast<uint16_t*>(bias_stage_dyn);
+    stb = bias_stage_dyn + kQTile * kTStride * 2;
+  }
   __syncthreads();
   for (long long p = blockIdx.x; p < a.max_pairs; p += gridDim.x) {
     uint16_t* tile = tiles + (p * a.bias_heads + hb) * (kQTile * kQTile);
@@ -259,7 +292,7 @@ __device__ __forceinline__ void bias_tiles(const AttnArgs& a, uint16_t* __restri
     uint16_t* tile_t = a.bias_t_out ? static_cast<uint16_t*>(a.bias_t_out) + (p * a.bias_heads + hb) * (kQTile * kQTile)
                                     : nullptr;
     uint8_t* btile_t = a.bucket_t_out ? static_cast<uint8_t*>(a.bucket_t_out) + p * (kQTile * kQTile) : nullptr;
-    if (!bias_tile_block<TRANSPOSED, BUCKETS>(a, s_c, sq, p, hb, tile, btile, tile_t, btile_t)) break;
+    if (!bias_tile_block<TRANSPOSED, BUCKETS>(a, s_c, sq, p, hb, tile, btile, tile_t, btile_t, stt, stb)) break;
     __syncthreads();
   }
 }
