@@ -1018,7 +1018,8 @@ cudaError_t launch_attn_persistent(const CUtensorMap& tq, const CUtensorMap& tk,
   return e;
 }
 
-cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
+cudaError_t attn_fwd_tc2(const AttnArgs& a_in, cudaStream_t st) {
+  AttnArgs a = a_in;
   cudaError_t e = upload_time_taus();
   if (e != cudaSuccess) return e;
   if (a.T == 0 || a.capacity == 0) return cudaSuccess;
@@ -1030,8 +1031,11 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a, cudaStream_t st) {
     e = ensure_smem_attr(reinterpret_cast<const void*>(attn_bias_kernel), bias_dyn);
     if (e != cudaSuccess) return e;
   }
+  a.bias_blocks = bias_tile_grid(a.max_pairs, a.bias_heads);
+  const int64_t cvt_blocks = a.cvt_n > 0 ? (a.cvt_n + 8 * kBiasThreads - 1) / (8 * kBiasThreads) : 0;
+  if (a.bias_blocks + cvt_blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   e = launch_pdl(attn_bias_kernel,
-                 dim3(static_cast<unsigned>(bias_tile_grid(a.max_pairs, a.bias_heads)), static_cast<unsigned>(a.bias_heads)),
+                 dim3(static_cast<unsigned>(a.bias_blocks + cvt_blocks), static_cast<unsigned>(a.bias_heads)),
                  dim3(kBiasThreads), bias_dyn, st, a);
   if (e != cudaSuccess) return e;
   const bool f16 = a.in_f16 != 0;

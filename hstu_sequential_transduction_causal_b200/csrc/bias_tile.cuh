@@ -19,6 +19,7 @@
 #include "sm100_ptx.cuh"
 #include "tile_pairs.cuh"
 #include "time_bucket_dev.cuh"
+#include "vec_io.cuh"
 
 namespace hstu {
 namespace {
@@ -272,6 +273,26 @@ __device__ __forceinline__ void bias_tiles(const AttnArgs& a, uint16_t* __restri
   __shared__ int64_t s_off[kSeqStage + 1];
   __shared__ int32_t s_pack[kSeqStage];
   const int hb = blockIdx.y;
+  const long long tile_blocks = a.bias_blocks > 0 ? a.bias_blocks : gridDim.x;
+  if (static_cast<long long>(blockIdx.x) >= tile_blocks) {   // an extra block: bf16 -> fp16 conversion
+    pdl_trigger();
+    pdl_wait();      // cvt_out may still be read by an earlier kernel (a previous layer's f2)
+    if (hb == 0) {
+      const int64_t i = ((static_cast<int64_t>(blockIdx.x) - tile_blocks) * kBiasThreads + threadIdx.x) * 8;
+      if (i + 8 <= a.cvt_n) {
+        float v[8];
+        load_vec<8, kDtBF16>(a.cvt_in, i, v);
+        store_vec<8, kDtF16>(a.cvt_out, i, v);
+      } else {
+        for (int64_t k = i; k < a.cvt_n; ++k) {
+          float f;
+          load_vec<1, kDtBF16>(a.cvt_in, k, &f);
+          reinterpret_cast<__half*>(a.cvt_out)[k] = __float2half_rn(f);
+        }
+      }
+    }
+    return;
+  }
   pdl_trigger();
   bias_const_load(s_c, a, hb);
   pdl_wait();
@@ -286,7 +307,7 @@ __device__ __forceinline__ void bias_tiles(const AttnArgs& a, uint16_t* __restri
     stb = bias_stage_dyn + kQTile * kTStride * 2;
   }
   __syncthreads();
-  for (long long p = blockIdx.x; p < a.max_pairs; p += gridDim.x) {
+  for (long long p = blockIdx.x; p < a.max_pairs; p += tile_blocks) {
     uint16_t* tile = tiles + (p * a.bias_heads + hb) * (kQTile * kQTile);
     uint8_t* btile = BUCKETS ? btiles + p * (kQTile * kQTile) : nullptr;
     uint16_t* tile_t = a.bias_t_out ? static_cast<uint16_t*>(a.bias_t_out) + (p * a.bias_heads + hb) * (kQTile * kQTile)

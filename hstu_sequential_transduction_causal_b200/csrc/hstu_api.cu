@@ -249,7 +249,8 @@ hstu_status_t check_attn(const hstu_attn_desc_t* d, const hstu_jagged_t* j) {
 hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, const void* q, const void* k,
                            const void* v, const float* rab_pos, const float* rab_time, void* out, void* ws,
                            cudaStream_t st, bool tile_pairs = true, const hstu_rab_ext_t* ext = nullptr,
-                           const int64_t* q_from = nullptr, void* bias_cache = nullptr) {
+                           const int64_t* q_from = nullptr, void* bias_cache = nullptr, const void* cvt_in = nullptr,
+                           void* cvt_out = nullptr, int64_t cvt_n = 0) {
   const int64_t cap = capacity_of(j);
   const int hb = ext && ext->per_head ? d->H : 1;
   const AttnWs lay = attn_ws_layout(j, hb);
@@ -283,6 +284,11 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
       a.bias_t_out = bias_cache;
       a.bucket_t_out = static_cast<uint8_t*>(bias_cache) + bias_cache_layout(j).bucket;
     }
+    if (cvt_n > 0) {   // a bf16 -> fp16 copy rides on the bias kernel's launch
+      a.cvt_in = cvt_in;
+      a.cvt_out = cvt_out;
+      a.cvt_n = cvt_n;
+    }
   }
   cudaError_t e = launch_worklist(j->offsets, j->B, j->T, j->max_len, items, count, a.status, st,
                                   pairs ? reinterpret_cast<long long*>(w + lay.pairs) : nullptr, nullptr, nullptr,
@@ -314,9 +320,10 @@ hstu_status_t run_uvqk(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t ac
 // g_dtype F16: W2 is read through an fp16 copy written to w2_f16 ([D, D]) first.
 hstu_status_t run_out_proj(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t g_dtype, const void* g_in,
                            const void* W2, const float* b2, const void* x, hstu_dtype_t x_dtype, void* y,
-                           hstu_dtype_t y_dtype, void* y_f16, int* status, cudaStream_t st, void* w2_f16) {
+                           hstu_dtype_t y_dtype, void* y_f16, int* status, cudaStream_t st, void* w2_f16,
+                           bool w2_ready = false) {
   const bool f16 = g_dtype == HSTU_F16;
-  if (f16) {
+  if (f16 && !w2_ready) {
     cudaError_t e = convert_dtype(W2, kDtBF16, w2_f16, kDtF16, static_cast<int64_t>(D) * D, st);
     if (e != cudaSuccess) return cuda_status(e);
   }
@@ -791,8 +798,12 @@ hstu_status_t run_layer_fwd(const hstu_layer_desc_t* desc, hstu_dtype_t resid_dt
   ad.dtype = act;
   const size_t es = act == HSTU_F32 ? 4 : 2;
   const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
+  // BF16 mode: the fp16 copy of W2 that f2 reads is written by extra blocks of the attention's bias
+  // kernel (one launch fewer)
+  const bool w2_early = desc->dtype == HSTU_BF16;
   s = run_attn_fwd(&ad, jag, uvqk + 2 * D * es, uvqk + 3 * D * es, uvqk + 1 * D * es, w->rab_pos, w->rab_time,
-                   saved->o, ws, st, true, nullptr, nullptr, saved->attn_bias);
+                   saved->o, ws, st, true, nullptr, nullptr, saved->attn_bias, w->W2, wsb + lay.w2_f16,
+                   w2_early ? static_cast<int64_t>(D) * D : 0);
   if (s != HSTU_OK) return s;
   // G in fp16 (BF16 mode): f2 then reads an fp16 copy of W2
   const hstu_dtype_t g_dt = desc->dtype == HSTU_BF16 ? HSTU_F16 : HSTU_F32;
@@ -800,7 +811,7 @@ hstu_status_t run_layer_fwd(const hstu_layer_desc_t* desc, hstu_dtype_t resid_dt
                                 desc->ln_eps, saved->g, saved->mu, saved->rstd, st, status);
   if (e != cudaSuccess) return cuda_status(e);
   return run_out_proj(T, D, desc->dtype, g_dt, saved->g, w->W2, w->b2, x, resid_dtype, y, desc->y_dtype, y_f16,
-                      status, st, wsb + lay.w2_f16);
+                      status, st, wsb + lay.w2_f16, w2_early);
 }
 
 }  // namespace

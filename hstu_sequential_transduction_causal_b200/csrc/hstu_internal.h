@@ -182,6 +182,12 @@ struct AttnArgs {
   // laid out as AttnBwdArgs::bias_t and ::bucket_t
   void* bias_t_out;
   void* bucket_t_out;
+  // (forward, cvt_n > 0) extra blocks of the bias kernel convert cvt_n bf16 values cvt_in to fp16 at
+  // cvt_out (the layer's fp16 W2 copy, read later by f2); bias_blocks: the grid's tile blocks
+  const void* cvt_in;
+  void* cvt_out;
+  int64_t cvt_n;
+  int64_t bias_blocks;
 };
 
 struct AttnBwdArgs {
