@@ -66,12 +66,12 @@ def test_linear_all_operand_layouts(a_mn, b_mn, accumulate, shape):
     assert_close(got, ref, 1e-4 * np.sqrt(K), 1e-4, what=f"linear a_mn={a_mn} b_mn={b_mn} acc={accumulate}")
 
 
-def _run_layer_fwd_bwd(wl, x_dtype=torch.bfloat16, bias_cache=None):
+def _run_layer_fwd_bwd(wl, x_dtype=torch.bfloat16, bias_cache=None, return_y=False):
     jag = JaggedBatch(wl.offsets, wl.timestamps)
     layer = DeviceLayer.upload(wl.layers[0], wl.D, wl.H, True)
     run = LayerRunner(layer, jag, 1.0 / wl.N, wl.pos_max_len, x_dtype, x_dtype, keep_z=True, bias_cache=bias_cache)
     x = to_dev(wl.x, x_dtype)
-    run.forward(x)
+    y = run.forward(x).float().cpu().numpy()
     D, T = wl.D, wl.T
     grads = [torch.full(s, float("nan"), dtype=torch.float32, device="cuda")
              for s in [(4 * D, D), (4 * D,), (D, D), (D,), (D,), (D,), (2 * wl.pos_max_len - 1,), (128,)]]
@@ -83,7 +83,8 @@ def _run_layer_fwd_bwd(wl, x_dtype=torch.bfloat16, bias_cache=None):
     torch.cuda.synchronize()
     assert H.hstu_sync_status(ws) == 0
     assert run.device_status() == 0
-    return dx.float().cpu().numpy(), [g.cpu().numpy() for g in grads]
+    out = dx.float().cpu().numpy(), [g.cpu().numpy() for g in grads]
+    return out + (y,) if return_y else out
 
 
 def _oracle_grads(wl):
@@ -146,6 +147,25 @@ def test_layer_bwd_bias_cache_matches_recompute():
     for name, a, b in zip(("dW1", "db1", "dW2", "db2", "dgamma", "dbeta", "drab_pos", "drab_time"), g_c, g_r):
         scale = max(float(np.abs(b).max()), 1e-30)
         assert np.abs(a - b).max() <= 1e-5 * scale, name
+
+
+def test_layer_fwd_bwd_more_sequences_than_staged_tables():
+    """600 sequences, most of them shorter than a tile (packed several to a diagonal tile), a few of
+    several tiles: more sequences than the bias kernels stage in shared memory, so their pair and
+    row lookups read the global tables. Y, dX and the gradients against the oracle, with the forward's
+    bias cache and with the backward recomputing its tiles."""
+    rng = np.random.default_rng(21)
+    lens = [int(v) for v in rng.integers(0, 40, 600)]
+    lens[7], lens[300], lens[599] = 300, 129, 700
+    wl = W.make_workload("c2", seed=8, lengths=lens, backward=True)
+    assert len(lens) > 512
+    dx, grads, y = _run_layer_fwd_bwd(wl, bias_cache=True, return_y=True)
+    args = (wl.offsets, wl.timestamps, wl.H, 1.0 / wl.N, wl.pos_max_len, THR)
+    ye, sv = O.layer_fwd(wl.x, wl.layers[0], *args)
+    assert_close(y, ye, *BF16_TOL, what="Y 600 sequences")
+    _compare(dx, grads, O.layer_bwd(wl.dy, wl.layers[0], sv, *args), _model_grads(wl), "600-sequences ")
+    dx_r, g_r = _run_layer_fwd_bwd(wl, bias_cache=False)
+    np.testing.assert_array_equal(dx, dx_r)
 
 
 def test_layer_bwd_d256_four_heads():
