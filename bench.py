@@ -382,11 +382,11 @@ def main():
     # kernels of ours per step (cross-checked against the ncu launch list in profiles/)
     # f1 GEMM | work list, bias tiles (with the fp16 W2 copy f2 reads), attention | LN-gate | f2 GEMM
     n_fwd_kernels = 6
-    # fp16 dy with the db2 partial sums and the fp16 copies of x, W1, W2 (one launch) | dG with dW2 (one
-    # grouped GEMM launch) | LN-gate bwd | work list, attention bwd, table gradients (the transposed bias
-    # tiles come from the forward's cache) | dZ with the db1 partial sums | finish of db2, dgamma, dbeta
-    # and db1 (one launch) | dX with dW1 (one grouped launch)
-    n_bwd_kernels = 9
+    # fp16 dy with the db2 partial sums, the fp16 copies of x, W1, W2 and the zeroed accumulators (one
+    # launch) | dG with dW2 (one grouped GEMM launch) | LN-gate bwd | attention bwd, table gradients (the
+    # transposed bias tiles and the work list come from the forward's cache) | dZ with the db1 partial
+    # sums | finish of db2, dgamma, dbeta and db1 (one launch) | dX with dW1 (one grouped launch)
+    n_bwd_kernels = 8
     names = ["uvqk", "attn", "norm_gate", "out_proj"] + (["backward"] if backward else [])
 
     def attention_forward():

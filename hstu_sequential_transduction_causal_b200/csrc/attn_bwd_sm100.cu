@@ -584,6 +584,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // Every unit this CTA will take is taken: the last CTA to get here puts the unit counter and the
+  // finished-CTA counter back to zero, so a later launch over the same work list (a second backward
+  // after one forward) starts from unit 0 without a work-list launch of its own.
+  if (warp == kSiluWarpsB + 3 && lane == 0) {
+    __threadfence();
+    if (atomicAdd(A.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      atomicExch(A.sched, 0);
+      atomicExch(A.sched + 1, 0);
+    }
+  }
 }
 
 // ----------------------------------------------------------------------------------------------

@@ -95,15 +95,23 @@ bool bwd_pairs_fit(const hstu_jagged_t* j, int H) {
 }
 
 // hstu_layer_saved_t.attn_bias: the backward's key-major fp16 half-bias tiles (32 KB per causal
-// pair), then the u8 bucket tiles (16 KB per pair), in the layout of the attention backward's own.
+// pair), then the u8 bucket tiles (16 KB per pair), in the layout of the attention backward's own;
+// then the batch's metadata the forward's work list writes for the backward: a 256-byte header
+// (int32 key-tile item count at 0, the persistent backward's unit and finished-CTA counters at 4
+// and 8), the key-tile work list, pair_base and the pack array.
 struct BiasCache {
-  size_t bucket, total;
+  size_t bucket, meta, kitems, pairs, pack, total;
 };
 BiasCache bias_cache_layout(const hstu_jagged_t* j) {
   const int64_t mp = attn_ws_layout(j).max_pairs;
+  const int64_t cap = capacity_of(j);
   BiasCache c{};
   c.bucket = align_up(static_cast<size_t>(mp) * kQTile * kQTile * 2, 256);
-  c.total = c.bucket + align_up(static_cast<size_t>(mp) * kQTile * kQTile, 256);
+  c.meta = c.bucket + align_up(static_cast<size_t>(mp) * kQTile * kQTile, 256);
+  c.kitems = c.meta + 256;
+  c.pairs = c.kitems + align_up(static_cast<size_t>(cap) * 8, 256);
+  c.pack = c.pairs + align_up(static_cast<size_t>(j->B + 1) * 8, 256);
+  c.total = c.pack + align_up(static_cast<size_t>(j->B) * 4, 256);
   return c;
 }
 
@@ -165,17 +173,20 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
                            const void* v, const void* d_out, const float* rab_pos, const float* rab_time, float* dq,
                            float* dk, float* dv, int64_t ld_g, float* d_rab_pos, float* d_rab_time, void* ws,
                            cudaStream_t st, const hstu_rab_ext_t* ext = nullptr, float* d_rab_type = nullptr,
-                           void* bias_cache = nullptr) {
+                           void* bias_cache = nullptr, bool zeroed = false) {
+  // zeroed: an earlier launch of the call already cleared d_rab_pos, d_rab_time and dq (T > 0)
   const int hb = ext && ext->per_head ? desc->H : 1;
   const int nt = ext ? ext->n_types : 0;
   const AttnBwdWs lay = attn_bwd_ws_layout(jag, desc->H, hb);
-  cudaError_t e =
-      cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * hb * (2 * static_cast<size_t>(desc->pos_max_len) - 1), st);
-  if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, sizeof(float) * hb * desc->n_time_buckets, st);
-  if (e == cudaSuccess && nt > 0) e = cudaMemsetAsync(d_rab_type, 0, sizeof(float) * hb * nt * nt, st);
-  if (e != cudaSuccess) return cuda_status(e);
+  cudaError_t e = cudaSuccess;
+  if (!zeroed || jag->T == 0) {
+    e = cudaMemsetAsync(d_rab_pos, 0, sizeof(float) * hb * (2 * static_cast<size_t>(desc->pos_max_len) - 1), st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_rab_time, 0, sizeof(float) * hb * desc->n_time_buckets, st);
+    if (e == cudaSuccess && nt > 0) e = cudaMemsetAsync(d_rab_type, 0, sizeof(float) * hb * nt * nt, st);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
   if (jag->T == 0) return HSTU_OK;
-  e = cudaMemsetAsync(dq, 0, sizeof(float) * static_cast<size_t>(jag->T) * ld_g, st);
+  if (!zeroed) e = cudaMemsetAsync(dq, 0, sizeof(float) * static_cast<size_t>(jag->T) * ld_g, st);
   if (e != cudaSuccess) return cuda_status(e);
   uint8_t* w = static_cast<uint8_t*>(ws);
   AttnBwdArgs A{};
@@ -198,17 +209,25 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
   a.bias_heads = hb; a.n_types = nt;
   if (nt > 0) { a.token_type = ext->token_type; a.rab_type = ext->rab_type; }
   A.bias_t = w + lay.bias_t; A.bucket_t = w + lay.bucket_t; A.dxt = w + lay.dxt;
-  if (bias_cache && hb == 1) {   // written by this batch's forward (shared tables only)
-    A.bias_t = bias_cache;
-    A.bucket_t = static_cast<uint8_t*>(bias_cache) + bias_cache_layout(jag).bucket;
-    A.bias_cached = 1;
-  }
   A.kitems = reinterpret_cast<int32_t*>(w + lay.kitems); A.kcount = kcount;
-  A.sched = count + 5;   // [276, 280) of the workspace header region
+  A.sched = count + 5;   // [276, 284) of the workspace header region
   a.pack = reinterpret_cast<const int32_t*>(w + lay.f.pack);
-  e = launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, a.status, st,
-                      reinterpret_cast<long long*>(w + lay.f.pairs), reinterpret_cast<int32_t*>(w + lay.kitems),
-                      kcount, A.sched, reinterpret_cast<int32_t*>(w + lay.f.pack));
+  if (bias_cache && hb == 1) {   // tiles and work list written by this batch's forward (shared tables only)
+    const BiasCache bc = bias_cache_layout(jag);
+    uint8_t* c = static_cast<uint8_t*>(bias_cache);
+    A.bias_t = bias_cache;
+    A.bucket_t = c + bc.bucket;
+    A.bias_cached = 1;
+    A.kitems = reinterpret_cast<const int32_t*>(c + bc.kitems);
+    A.kcount = reinterpret_cast<const int32_t*>(c + bc.meta);
+    A.sched = reinterpret_cast<int32_t*>(c + bc.meta) + 1;
+    a.pair_base = reinterpret_cast<const long long*>(c + bc.pairs);
+    a.pack = reinterpret_cast<const int32_t*>(c + bc.pack);
+  } else {
+    e = launch_worklist(jag->offsets, jag->B, jag->T, jag->max_len, items, count, a.status, st,
+                        reinterpret_cast<long long*>(w + lay.f.pairs), reinterpret_cast<int32_t*>(w + lay.kitems),
+                        kcount, nullptr, reinterpret_cast<int32_t*>(w + lay.f.pack), nullptr, A.sched);
+  }
   if (e == cudaSuccess) e = attn_bwd_tc(A, st);
   return cuda_status(e);
 }
@@ -272,6 +291,8 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
     a.n_types = ext->n_types; a.token_type = ext->token_type; a.rab_type = ext->rab_type;
   }
   const bool pairs = tile_pairs && is_tc_dtype(d->dtype);
+  int32_t* cache_kitems = nullptr;   // with the layer's bias cache: the backward's work list
+  int32_t* cache_meta = nullptr;
   if (pairs) {
     a.pair_base = reinterpret_cast<const long long*>(w + lay.pairs);
     a.bias = w + lay.bias;
@@ -280,9 +301,15 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
     a.urec = reinterpret_cast<const int32_t*>(w + lay.urec);
     // short sequences share tiles, except in a prefix append (whose rows start mid-sequence)
     if (!q_from) a.pack = reinterpret_cast<const int32_t*>(w + lay.pack);
-    if (bias_cache && hb == 1 && !q_from) {   // the backward's tiles too
+    if (bias_cache && hb == 1 && !q_from) {   // the backward's tiles and work list too
+      const BiasCache bc = bias_cache_layout(j);
+      uint8_t* c = static_cast<uint8_t*>(bias_cache);
       a.bias_t_out = bias_cache;
-      a.bucket_t_out = static_cast<uint8_t*>(bias_cache) + bias_cache_layout(j).bucket;
+      a.bucket_t_out = c + bc.bucket;
+      a.pair_base = reinterpret_cast<const long long*>(c + bc.pairs);
+      a.pack = reinterpret_cast<const int32_t*>(c + bc.pack);
+      cache_kitems = reinterpret_cast<int32_t*>(c + bc.kitems);
+      cache_meta = reinterpret_cast<int32_t*>(c + bc.meta);
     }
     if (cvt_n > 0) {   // a bf16 -> fp16 copy rides on the bias kernel's launch
       a.cvt_in = cvt_in;
@@ -291,9 +318,9 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
     }
   }
   cudaError_t e = launch_worklist(j->offsets, j->B, j->T, j->max_len, items, count, a.status, st,
-                                  pairs ? reinterpret_cast<long long*>(w + lay.pairs) : nullptr, nullptr, nullptr,
-                                  pairs ? a.unit_counter : nullptr, const_cast<int32_t*>(a.pack),
-                                  const_cast<int32_t*>(a.urec));
+                                  pairs ? const_cast<long long*>(a.pair_base) : nullptr, cache_kitems,
+                                  cache_meta, pairs ? a.unit_counter : nullptr, const_cast<int32_t*>(a.pack),
+                                  const_cast<int32_t*>(a.urec), cache_meta ? cache_meta + 1 : nullptr);
   if (e != cudaSuccess) return cuda_status(e);
   if (j->T == 0) return HSTU_OK;
   if (!is_tc_dtype(d->dtype)) e = attn_fwd_f32_simt(a, st);
@@ -941,26 +968,31 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   float* part_ln = reinterpret_cast<float*>(wsb + lay.part_ln);
   float* part_dz = reinterpret_cast<float*>(wsb + lay.part_dz);
   int parts_dy = 0, parts_ln = 0;
-  {   // one launch: the fp16 copy of dY (unless the caller passed one) with the partial sums of db2,
-      // and the other fp16 GEMM operand copies
-    ConvertJob jobs[4];
-    int nj = 0;
-    if (!x_f16) jobs[nj++] = ConvertJob{x, wsb + lay.x_f16, T * D, x_dt};
-    jobs[nj++] = ConvertJob{w->W1, w1_f16, 4ll * D * D, kDtBF16};
-    jobs[nj++] = ConvertJob{w->W2, w2_f16, 1ll * D * D, kDtBF16};
-    e = rows_to_f16_colsum(T, D, y_dt, dy, dy_f16 ? nullptr : wsb + lay.dy_f16, part_dy, &parts_dy, jobs, nj, st);
-  }
-  if (e != cudaSuccess) return cuda_status(e);
   float* dG = reinterpret_cast<float*>(wsb + lay.dg);
   void* dO = wsb + lay.dO;
   float* dq = reinterpret_cast<float*>(wsb + lay.dq);
   float* dk = reinterpret_cast<float*>(wsb + lay.dk);
   float* dv = reinterpret_cast<float*>(wsb + lay.dv);
   void* dz = wsb + lay.dz;
+  {   // one launch: the fp16 copy of dY (unless the caller passed one) with the partial sums of db2,
+      // the other fp16 GEMM operand copies, and zeros in every output a later launch accumulates
+      // into (dW2, dW1, dQ and the table gradients)
+    ConvertJob jobs[kMaxConvertJobs];
+    int nj = 0;
+    if (!x_f16) jobs[nj++] = ConvertJob{x, wsb + lay.x_f16, T * D, x_dt};
+    jobs[nj++] = ConvertJob{w->W1, w1_f16, 4ll * D * D, kDtBF16};
+    jobs[nj++] = ConvertJob{w->W2, w2_f16, 1ll * D * D, kDtBF16};
+    jobs[nj++] = ConvertJob{nullptr, gr->dW2, 1ll * D * D, kDtF32};
+    jobs[nj++] = ConvertJob{nullptr, gr->dW1, 4ll * D * D, kDtF32};
+    jobs[nj++] = ConvertJob{nullptr, dq, T * D, kDtF32};
+    jobs[nj++] = ConvertJob{nullptr, gr->drab_pos, 2ll * desc->pos_max_len - 1, kDtF32};
+    jobs[nj++] = ConvertJob{nullptr, gr->drab_time, desc->n_time_buckets, kDtF32};
+    e = rows_to_f16_colsum(T, D, y_dt, dy, dy_f16 ? nullptr : wsb + lay.dy_f16, part_dy, &parts_dy, jobs, nj, st);
+  }
+  if (e != cudaSuccess) return cuda_status(e);
   // 1. f2 backward: dG = dY W2 and dW2 = dY^T G in one launch (dW2 split over K = T into units of
   //    about half a dG unit, reduced into the zeroed dW2); db2 = sum_t dY
-  e = cudaMemsetAsync(gr->dW2, 0, sizeof(float) * D * D, st);
-  if (e == cudaSuccess) {
+  {
     GemmArgs gg[2] = {};
     GemmArgs& g = gg[0];
     g.A = dy_op; g.lda = D; g.a_mn = false; g.B = w2_f16; g.ldb = D; g.b_mn = true; g.f16 = true;
@@ -981,7 +1013,7 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   // 3. attention backward
   const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
   s = run_attn_bwd(&ad, jag, uvqk + 2 * D * 2, uvqk + 3 * D * 2, uvqk + 1 * D * 2, dO, w->rab_pos, w->rab_time, dq, dk,
-                   dv, D, gr->drab_pos, gr->drab_time, ws, st, nullptr, nullptr, saved->attn_bias);
+                   dv, D, gr->drab_pos, gr->drab_time, ws, st, nullptr, nullptr, saved->attn_bias, true);
   if (s != HSTU_OK) return s;
   // 4. SiLU backward into dZ[:, D:4D] with the partial sums of db1 = sum_t dZ; then db2, dgamma,
   // dbeta and db1 finished by one launch straight into the caller's buffers
@@ -998,7 +1030,6 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   if (e == cudaSuccess && g_ready_events[0]) e = cudaEventRecord(g_ready_events[0], st);
   // 5. f1 backward in one launch: dX = dY + dZ W1 and dW1 = dZ^T X (fp16 dZ, x and W1; dW1 split
   //    over K = T into units of about a third of a dX unit, reduced into the zeroed dW1)
-  if (e == cudaSuccess) e = cudaMemsetAsync(gr->dW1, 0, sizeof(float) * 4 * D * D, st);
   if (e == cudaSuccess) {
     GemmArgs gg[2] = {};
     GemmArgs& g3 = gg[1];

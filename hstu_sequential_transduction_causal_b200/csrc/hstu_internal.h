@@ -113,7 +113,8 @@ cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
 // each sequence's first causal (query tile, key tile) pair and, in pair_base[B], their total.
 // With kitems, also the attention backward's (sequence, key tile) list in the same cost order: the
 // key tile that visits t + 1 query tiles sits where the forward list has query tile t. With sched,
-// sched[0] (the persistent attention kernel's unit counter) is reset to 0. With pack (int32 [B]),
+// sched[0] (the persistent attention kernel's unit counter) is reset to 0; with sched2, sched2[0]
+// and sched2[1] (the persistent backward's unit and finished-CTA counters). With pack (int32 [B]),
 // runs of short sequences share a tile: pack[b] = k >= 2 marks the first of k packed sequences
 // (one item (b, -k) in both lists), 0 the other members, 1 a sequence on its own. With urec (needs
 // pair_base; int32 [capacity, 8], 16-byte aligned), the persistent attention forward's record of
@@ -121,7 +122,7 @@ cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
                             int32_t* count, int* status, cudaStream_t st, long long* pair_base = nullptr,
                             int32_t* kitems = nullptr, int32_t* kcount = nullptr, int32_t* sched = nullptr,
-                            int32_t* pack = nullptr, int32_t* urec = nullptr);
+                            int32_t* pack = nullptr, int32_t* urec = nullptr, int32_t* sched2 = nullptr);
 // The n_b x n_b time-bucket matrices of the test surface, tile by tile with the bias tiles' code.
 cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int max_len,
                                 int n_buckets, const int64_t* sq_offsets, uint8_t* out, cudaStream_t st);
@@ -202,7 +203,8 @@ struct AttnBwdArgs {
   void* dxt;                   // fp16 [max_pairs, H, 128 keys, 128 queries] dX^T of every (pair, head)
   const int32_t* kitems;       // backward work list (b, key tile)
   const int32_t* kcount;
-  int32_t* sched;              // the persistent backward's unit counter, zeroed by the work list
+  int32_t* sched;              // the persistent backward's unit counter and finished-CTA counter (two
+                               // ints): zero at launch (the work list zeroes them), zero again at exit
   int bias_cached;             // bias_t and bucket_t were written by the forward: no bias kernel
 };
 
@@ -260,15 +262,17 @@ cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const f
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
                         const void* z, int64_t ld_z, void* dz, int64_t ld_dz, float* partial, int* parts,
                         cudaStream_t st);
-// A tensor of n elements (fp32, bf16 or fp16) converted to fp16.
+// A tensor of n elements (fp32, bf16 or fp16) converted to fp16; with in == null, n fp32 zeros
+// written to out instead (an accumulated output cleared in the same launch).
 struct ConvertJob {
   const void* in;
   void* out;
   int64_t n;
   int in_dt;
 };
+constexpr int kMaxConvertJobs = 10;
 // One launch: [T, D] rows (fp32, bf16 or fp16) to fp16 (out may be null) with their partial column
-// sums into partial [*parts, D] (at most kTailParts rows), and up to four other tensors to fp16.
+// sums into partial [*parts, D] (at most kTailParts rows), and up to kMaxConvertJobs other jobs.
 cudaError_t rows_to_f16_colsum(int64_t T, int D, int in_dt, const void* in, void* out, float* partial, int* parts,
                                const ConvertJob* jobs, int njobs, cudaStream_t st);
 // Most partial rows rows_to_f16_colsum writes.

@@ -77,9 +77,12 @@ __device__ void write_unit_records(const int64_t* __restrict__ off, const int32_
 __global__ void __launch_bounds__(1024)
 worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items,
                 int32_t* count, int* status, long long* pair_base, int32_t* kitems, int32_t* kcount,
-                int32_t* sched, int32_t* pack, int32_t* urec) {
+                int32_t* sched, int32_t* pack, int32_t* urec, int32_t* sched2) {
   pdl_enter();
-  if (sched && threadIdx.x == 0) sched[0] = 0;   // the persistent attention's unit counter
+  if (threadIdx.x == 0) {   // the persistent attention kernels' unit (and finished-CTA) counters
+    if (sched) sched[0] = 0;
+    if (sched2) sched2[0] = sched2[1] = 0;
+  }
   __shared__ int s_warp[32];
   __shared__ int s_max_tiles;
   __shared__ int s_bad;
@@ -249,9 +252,12 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
 __global__ void __launch_bounds__(32)
 worklist_warp_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items, int32_t* count,
                      int* status, long long* pair_base, int32_t* kitems, int32_t* kcount, int32_t* sched,
-                     int32_t* pack, int32_t* urec) {
+                     int32_t* pack, int32_t* urec, int32_t* sched2) {
   pdl_enter();
-  if (sched && threadIdx.x == 0) sched[0] = 0;   // the persistent attention's unit counter
+  if (threadIdx.x == 0) {   // the persistent attention kernels' unit (and finished-CTA) counters
+    if (sched) sched[0] = 0;
+    if (sched2) sched2[0] = sched2[1] = 0;
+  }
   const int lane = threadIdx.x;
   const bool mine = lane < B;
   long long n = 0;
@@ -567,13 +573,13 @@ cudaError_t launch_ng(int64_t T, const void* o, int64_t ld_o, const void* u, int
 
 cudaError_t launch_worklist(const int64_t* offsets, int B, int64_t T, int max_len, int32_t* items,
                             int32_t* count, int* status, cudaStream_t st, long long* pair_base, int32_t* kitems,
-                            int32_t* kcount, int32_t* sched, int32_t* pack, int32_t* urec) {
+                            int32_t* kcount, int32_t* sched, int32_t* pack, int32_t* urec, int32_t* sched2) {
   if (urec && !pair_base) return cudaErrorInvalidValue;
   if (B >= 0 && B <= 32)
     return launch_pdl(worklist_warp_kernel, dim3(1), dim3(32), 0, st, offsets, B, T, max_len, items, count, status,
-                      pair_base, kitems, kcount, sched, pack, urec);
+                      pair_base, kitems, kcount, sched, pack, urec, sched2);
   return launch_pdl(worklist_kernel, dim3(1), dim3(1024), 0, st, offsets, B, T, max_len, items, count, status,
-                    pair_base, kitems, kcount, sched, pack, urec);
+                    pair_base, kitems, kcount, sched, pack, urec, sched2);
 }
 
 cudaError_t launch_time_buckets(const int64_t* offsets, const int64_t* ts, int B, int64_t T, int max_len,

@@ -308,12 +308,13 @@ dz_assemble_kernel(int64_t T, int D, const float* __restrict__ dv, const float* 
 }
 
 struct ConvertBatch {
-  ConvertJob job[4];
-  int first_block[5];   // block b converts job j with first_block[j] <= b < first_block[j + 1]
+  ConvertJob job[kMaxConvertJobs];
+  int first_block[kMaxConvertJobs + 1];   // block b runs job j with first_block[j] <= b < first_block[j + 1]
   int njobs;
 };
 
-// Block blk of a batch of conversions to fp16: it finds its job, then 8 elements per thread.
+// Block blk of a batch of conversions to fp16 (and zero fills): it finds its job, then 8 elements
+// per thread.
 __device__ __forceinline__ void convert_block(const ConvertBatch& cb, int blk) {
   int j = 0;
   while (j + 1 < cb.njobs && blk >= cb.first_block[j + 1]) ++j;
@@ -321,6 +322,16 @@ __device__ __forceinline__ void convert_block(const ConvertBatch& cb, int blk) {
   const int64_t i = (static_cast<int64_t>(blk - cb.first_block[j]) * blockDim.x + threadIdx.x) * 8;
   if (i >= jb.n) return;
   const int cnt = jb.n - i >= 8 ? 8 : static_cast<int>(jb.n - i);
+  if (!jb.in) {   // zero fill: 32-byte stores where out is 16-byte aligned, else word by word
+    float* o = static_cast<float*>(jb.out) + i;
+    if (cnt == 8 && (reinterpret_cast<uintptr_t>(jb.out) & 15) == 0) {
+      reinterpret_cast<float4*>(o)[0] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      reinterpret_cast<float4*>(o)[1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    } else {
+      for (int k = 0; k < cnt; ++k) o[k] = 0.0f;
+    }
+    return;
+  }
   float v[8];
   if (cnt == 8) {
     if (jb.in_dt == kDtF32) load_vec<8, kDtF32>(jb.in, i, v);
@@ -342,7 +353,8 @@ __device__ __forceinline__ void convert_block(const ConvertBatch& cb, int blk) {
 //   copy) and the partial column sums of dY (the db2 of f2's bias): block b sums rows [b R, (b+1) R)
 //   into partial[b][0 .. D); its threads own 8 columns each (D / 8 per row, 256 / (D / 8) rows side
 //   by side) and keep four rows' loads in flight each;
-// - the rest: the fp16 copies of the other GEMM operands (cb).
+// - the rest: the fp16 copies of the other GEMM operands and zero fills of the outputs later
+//   launches accumulate into (cb).
 template <int D, int IT>
 __global__ void __launch_bounds__(kTailThreads)
 rows_to_f16_colsum_kernel(int64_t T, const void* __restrict__ in, void* __restrict__ out, int64_t rows_per,
@@ -589,9 +601,12 @@ cudaError_t rows_to_f16_colsum(int64_t T, int D, int in_dt, const void* in, void
   *parts = 0;
   ConvertBatch cb{};
   int nb = 0, k = 0;
-  for (int j = 0; j < njobs && j < 4; ++j) {
+  if (njobs > kMaxConvertJobs) return cudaErrorInvalidValue;
+  for (int j = 0; j < njobs; ++j) {
     if (jobs[j].n <= 0) continue;
-    if (jobs[j].in_dt != kDtF32 && jobs[j].in_dt != kDtBF16 && jobs[j].in_dt != kDtF16) return cudaErrorInvalidValue;
+    if (!jobs[j].out) return cudaErrorInvalidValue;
+    if (jobs[j].in && jobs[j].in_dt != kDtF32 && jobs[j].in_dt != kDtBF16 && jobs[j].in_dt != kDtF16)
+      return cudaErrorInvalidValue;
     cb.job[k] = jobs[j];
     cb.first_block[k] = nb;
     const int64_t blocks = ((jobs[j].n + 7) / 8 + 255) / 256;

@@ -144,8 +144,10 @@ typedef struct hstu_layer_weights_t {
  * attn_bias (optional, BF16 mode; NULL = unused): hstu_layer_bias_cache_size(desc, jag) bytes,
  * 256-byte aligned. The forward then also writes there the attention backward's relative-bias
  * tiles (each causal 128 x 128 (query tile, key tile) pair's half-bias, key-major, and its time
- * buckets), and a backward given the same struct reads them instead of recomputing them. Valid
- * only for the batch and rab tables of the forward that wrote it. */
+ * buckets) and its key-tile work list, and a backward given the same struct reads them instead of
+ * recomputing them (one bias launch and one work-list launch fewer). The backward leaves the
+ * region as it found it, so several backwards may follow one forward. Valid only for the batch
+ * and rab tables of the forward that wrote it. */
 typedef struct hstu_layer_saved_t {
   void* uvqk;
   void* z;
@@ -418,7 +420,9 @@ hstu_status_t hstu_linear_bf16(int64_t M, int64_t N, int64_t K, const void* A, i
 size_t hstu_layer_bwd_workspace_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
 
 /* Bytes of hstu_layer_saved_t.attn_bias for this batch (0 for a batch hstu_attn_workspace_size
- * refuses): per causal tile pair a 32 KB fp16 half-bias tile and a 16 KB u8 bucket tile. */
+ * refuses): per causal tile pair a 32 KB fp16 half-bias tile and a 16 KB u8 bucket tile, then the
+ * batch's key-tile work list (8 bytes per tile), per-sequence pair numbering (8 bytes) and packing
+ * (4 bytes) after a 256-byte header. */
 size_t hstu_layer_bias_cache_size(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag);
 
 /* Whole layer backward (BF16 mode, D in {256, 512}), from the activations hstu_layer_fwd saved

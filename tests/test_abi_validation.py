@@ -399,7 +399,7 @@ def test_layer_bwd(L):
 
 def test_layer_bias_cache_size(L):
     """48 KB per causal tile pair (a 32 KB half-bias tile and a 16 KB bucket tile) of the batch's
-    pair bound; 0 for a refused descriptor or batch."""
+    pair bound, then the backward's work list; 0 for a refused descriptor or batch."""
     size = L.hstu_layer_bias_cache_size
     size.restype = ctypes.c_size_t
     # B = 2 sequences of at most 200 rows: 2 tiles each, so at most 3 causal pairs per sequence

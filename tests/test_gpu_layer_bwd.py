@@ -149,6 +149,38 @@ def test_layer_bwd_bias_cache_matches_recompute():
         assert np.abs(a - b).max() <= 1e-5 * scale, name
 
 
+def test_layer_bwd_twice_after_one_forward():
+    """With the bias cache the backward runs on the work list its forward wrote and leaves the
+    persistent kernel's unit counters at zero when it exits: a second backward after the same
+    forward computes the same dX (up to the order of dQ's fp32 reduce-adds) and gradients."""
+    wl = W.make_workload("c3", seed=7, lengths=[300, 1, 129, 700, 64, 0, 400], pos_max_len=1024, N=1024)
+    jag = JaggedBatch(wl.offsets, wl.timestamps)
+    layer = DeviceLayer.upload(wl.layers[0], wl.D, wl.H, True)
+    run = LayerRunner(layer, jag, 1.0 / wl.N, wl.pos_max_len, torch.bfloat16, torch.bfloat16, keep_z=True,
+                      bias_cache=True)
+    x = to_dev(wl.x, torch.bfloat16)
+    run.forward(x)
+    D, T = wl.D, wl.T
+    dy = to_dev(wl.dy, torch.bfloat16)
+    ws = workspace(H.hstu_layer_bwd_workspace_size(run.desc, jag.struct))
+    outs = []
+    for _ in range(2):
+        grads = [torch.full(s, float("nan"), dtype=torch.float32, device="cuda")
+                 for s in [(4 * D, D), (4 * D,), (D, D), (D,), (D,), (D,), (2 * wl.pos_max_len - 1,), (128,)]]
+        dx = torch.full((T, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        H.hstu_layer_bwd(run.desc, jag.struct, run.weights, x, None, run.saved_struct, dy, None, dx, None,
+                         H.layer_grads(*grads), ws)
+        torch.cuda.synchronize()
+        assert H.hstu_sync_status(ws) == 0
+        outs.append((dx.float().cpu().numpy(), [g.cpu().numpy() for g in grads]))
+    (dx1, g1), (dx2, g2) = outs
+    assert np.isfinite(dx2).all()
+    assert_close(dx2, dx1, 1e-3, 1e-2, what="dX of the second backward")
+    for name, a, b in zip(NAMES, g2, g1):
+        scale = max(float(np.abs(b).max()), 1e-30)
+        assert np.abs(a - b).max() <= 1e-5 * scale, name
+
+
 def test_layer_fwd_bwd_more_sequences_than_staged_tables():
     """600 sequences, most of them shorter than a tile (packed several to a diagonal tile), a few of
     several tiles: more sequences than the bias kernels stage in shared memory, so their pair and
