@@ -380,8 +380,9 @@ def main():
         flush.zero_()
         torch.sum(flush_rd, dim=0, out=flush_sink)
     # kernels of ours per step (cross-checked against the ncu launch list in profiles/)
-    # f1 GEMM | work list, bias tiles (with the fp16 W2 copy f2 reads), attention | LN-gate | f2 GEMM
-    n_fwd_kernels = 6
+    # f1 GEMM (its launch also computes the attention's work list) | bias tiles (with the fp16 W2 copy
+    # f2 reads), attention | LN-gate | f2 GEMM
+    n_fwd_kernels = 5
     # fp16 dy with the db2 partial sums, the fp16 copies of x, W1, W2 and the zeroed accumulators (one
     # launch) | dG with dW2 (one grouped GEMM launch) | LN-gate bwd | attention bwd, table gradients (the
     # transposed bias tiles and the work list come from the forward's cache) | dZ with the db1 partial

@@ -25,6 +25,7 @@
 
 #include "hstu_internal.h"
 #include "sm100_ptx.cuh"
+#include "worklist.cuh"
 
 namespace hstu {
 
@@ -82,6 +83,8 @@ struct GemmLaunch {
   GemmProb p[2];
   int nprob, total;
   int* sched;   // [0] next unit, [1] CTAs finished; zero between launches (the last CTA resets them)
+  int has_wl;   // static launches: the last CTA's scheduler warp (idle then) computes this work list
+  WorklistArgs wl;
 };
 
 struct Unit {
@@ -363,6 +366,8 @@ gemm_bf16_tc_kernel(const __grid_constant__ GemmMaps m0, const __grid_constant__
         mbar_arrive(ring_full(r));
         if (u >= L.total) break;
       }
+    } else if (L.has_wl && blockIdx.x == gridDim.x - 1) {
+      worklist_warp(L.wl);   // the CTA with the fewest units of the stride (whole warp)
     }
   } else {
     // epilogue warps 0-7: TMEM lanes 32 (warp % 4) .. +31 = output rows m0 + 32 (warp % 4) + lane,
@@ -574,8 +579,9 @@ GemmProb make_prob(const GemmArgs& g) {
 
 }  // namespace
 
-cudaError_t gemm_bf16_group(const GemmArgs* gs, int n, int* sched, cudaStream_t st) {
+cudaError_t gemm_bf16_group(const GemmArgs* gs, int n, int* sched, cudaStream_t st, const WorklistArgs* side) {
   if (!gs || n < 1 || n > 2) return cudaErrorInvalidValue;
+  if (side && (sched || side->B < 0 || side->B > 32)) return cudaErrorInvalidValue;
   GemmMaps maps[2];
   GemmLaunch L{};
   int k = 0;
@@ -589,13 +595,17 @@ cudaError_t gemm_bf16_group(const GemmArgs* gs, int n, int* sched, cudaStream_t 
     if (!status) status = g.status;
     ++k;
   }
-  if (k == 0) return cudaSuccess;
+  if (k == 0) return side ? cudaErrorInvalidValue : cudaSuccess;
   if (k == 1) maps[1] = maps[0];
   L.nprob = k;
   const int64_t total = static_cast<int64_t>(L.p[0].units) + (k > 1 ? L.p[1].units : 0);
   if (total >= (1ll << 30)) return cudaErrorInvalidValue;
   L.total = static_cast<int>(total);
   L.sched = sched;
+  if (side) {
+    L.has_wl = 1;
+    L.wl = *side;
+  }
   auto kern = gemm_bf16_tc_kernel;
   cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), GemmSmem::kTotal);
   if (e != cudaSuccess) return e;
@@ -603,10 +613,10 @@ cudaError_t gemm_bf16_group(const GemmArgs* gs, int n, int* sched, cudaStream_t 
   return launch_pdl(kern, dim3(grid), dim3(kThreads), GemmSmem::kTotal, st, maps[0], maps[1], L, wait_ctl(status));
 }
 
-cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st) {
-  if (g.M <= 0 || g.N <= 0) return cudaSuccess;
+cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st, const WorklistArgs* side) {
+  if (g.M <= 0 || g.N <= 0) return side ? cudaErrorInvalidValue : cudaSuccess;
   if (g.K <= 0) return cudaErrorInvalidValue;
-  return gemm_bf16_group(&g, 1, nullptr, st);
+  return gemm_bf16_group(&g, 1, nullptr, st, side);
 }
 
 cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st) {

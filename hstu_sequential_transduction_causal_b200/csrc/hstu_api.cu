@@ -263,13 +263,20 @@ hstu_status_t check_attn(const hstu_attn_desc_t* d, const hstu_jagged_t* j) {
   return HSTU_OK;
 }
 
+// An attention forward's kernel arguments and the work list they read (host values only).
+struct AttnFwdPlan {
+  AttnArgs a;
+  WorklistArgs wl;
+  bool pairs, tc;
+};
+
 // tile_pairs: the workspace has the full attn_ws_layout (bias tiles); otherwise only the work list
 // fits and the tensor-core path runs the kernel that evaluates the bias per element and head.
-hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, const void* q, const void* k,
-                           const void* v, const float* rab_pos, const float* rab_time, void* out, void* ws,
-                           cudaStream_t st, bool tile_pairs = true, const hstu_rab_ext_t* ext = nullptr,
-                           const int64_t* q_from = nullptr, void* bias_cache = nullptr, const void* cvt_in = nullptr,
-                           void* cvt_out = nullptr, int64_t cvt_n = 0) {
+AttnFwdPlan plan_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, const void* q, const void* k,
+                          const void* v, const float* rab_pos, const float* rab_time, void* out, void* ws,
+                          bool tile_pairs = true, const hstu_rab_ext_t* ext = nullptr, const int64_t* q_from = nullptr,
+                          void* bias_cache = nullptr, const void* cvt_in = nullptr, void* cvt_out = nullptr,
+                          int64_t cvt_n = 0) {
   const int64_t cap = capacity_of(j);
   const int hb = ext && ext->per_head ? d->H : 1;
   const AttnWs lay = attn_ws_layout(j, hb);
@@ -317,22 +324,43 @@ hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, co
       a.cvt_n = cvt_n;
     }
   }
-  cudaError_t e = launch_worklist(j->offsets, j->B, j->T, j->max_len, items, count, a.status, st,
-                                  pairs ? const_cast<long long*>(a.pair_base) : nullptr, cache_kitems,
-                                  cache_meta, pairs ? a.unit_counter : nullptr, const_cast<int32_t*>(a.pack),
-                                  const_cast<int32_t*>(a.urec), cache_meta ? cache_meta + 1 : nullptr);
+  AttnFwdPlan p{};
+  p.a = a;
+  p.pairs = pairs;
+  p.tc = is_tc_dtype(d->dtype);
+  p.wl = WorklistArgs{j->offsets, j->B, j->T, j->max_len, items, count, a.status,
+                      pairs ? const_cast<long long*>(a.pair_base) : nullptr, cache_kitems, cache_meta,
+                      pairs ? a.unit_counter : nullptr, const_cast<int32_t*>(a.pack), const_cast<int32_t*>(a.urec),
+                      cache_meta ? cache_meta + 1 : nullptr};
+  return p;
+}
+
+// wl_done: an earlier launch of the call already computed the plan's work list.
+hstu_status_t launch_attn_fwd(const AttnFwdPlan& p, cudaStream_t st, bool wl_done = false) {
+  const WorklistArgs& l = p.wl;
+  cudaError_t e = cudaSuccess;
+  if (!wl_done)
+    e = launch_worklist(l.off, l.B, l.T, l.max_len, l.items, l.count, l.status, st, l.pair_base, l.kitems, l.kcount,
+                        l.sched, l.pack, l.urec, l.sched2);
   if (e != cudaSuccess) return cuda_status(e);
-  if (j->T == 0) return HSTU_OK;
-  if (!is_tc_dtype(d->dtype)) e = attn_fwd_f32_simt(a, st);
-  else e = pairs ? attn_fwd_tc2(a, st) : attn_fwd_bf16_tc(a, st);
+  if (l.T == 0) return HSTU_OK;
+  if (!p.tc) e = attn_fwd_f32_simt(p.a, st);
+  else e = p.pairs ? attn_fwd_tc2(p.a, st) : attn_fwd_bf16_tc(p.a, st);
   return cuda_status(e);
+}
+
+hstu_status_t run_attn_fwd(const hstu_attn_desc_t* d, const hstu_jagged_t* j, const void* q, const void* k,
+                           const void* v, const float* rab_pos, const float* rab_time, void* out, void* ws,
+                           cudaStream_t st, bool tile_pairs = true, const hstu_rab_ext_t* ext = nullptr,
+                           const int64_t* q_from = nullptr) {
+  return launch_attn_fwd(plan_attn_fwd(d, j, q, k, v, rab_pos, rab_time, out, ws, tile_pairs, ext, q_from), st);
 }
 
 // f1: operands x, W1 of `dtype` (BF16 tensor cores or F32 CUDA cores); uvqk / z of act_dtype.
 // f16_ops: x and W1 are fp16 copies (the fp32-residual path) instead of bf16.
 hstu_status_t run_uvqk(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t act_dtype, const void* x, int64_t ld_x,
                        const void* W1, const float* b1, void* uvqk, void* z, int* status, cudaStream_t st,
-                       bool f16_ops = false) {
+                       bool f16_ops = false, const WorklistArgs* side = nullptr) {
   GemmArgs g{};
   g.A = x; g.lda = ld_x; g.a_mn = false;
   g.B = W1; g.ldb = D; g.b_mn = false; g.f16 = f16_ops;
@@ -341,7 +369,7 @@ hstu_status_t run_uvqk(int64_t T, int32_t D, hstu_dtype_t dtype, hstu_dtype_t ac
   g.epi.out0 = uvqk; g.epi.out0_dt = act_dtype; g.epi.ld_out0 = 4ll * D;
   g.epi.out1 = z; g.epi.out1_dt = act_dtype; g.epi.ld_out1 = 4ll * D;
   g.status = status;
-  return cuda_status(dtype == HSTU_BF16 ? gemm_bf16(g, st) : gemm_f32(g, st));
+  return cuda_status(dtype == HSTU_BF16 ? gemm_bf16(g, st, side) : gemm_f32(g, st));
 }
 
 // g_dtype F16: W2 is read through an fp16 copy written to w2_f16 ([D, D]) first.
@@ -820,17 +848,21 @@ hstu_status_t run_layer_fwd(const hstu_layer_desc_t* desc, hstu_dtype_t resid_dt
   // tensor-core mode keeps U|V|Q|K (and Z) in fp16: same MMA rate as bf16, 8x finer rounding of
   // the attention operands, whose errors LayerNorm(O) would otherwise amplify
   const hstu_dtype_t act = desc->dtype == HSTU_BF16 ? HSTU_F16 : HSTU_F32;
-  s = run_uvqk(T, D, desc->dtype, act, x_op, D, w1_op, w->b1, saved->uvqk, saved->z, status, st, x32);
-  if (s != HSTU_OK) return s;
   ad.dtype = act;
   const size_t es = act == HSTU_F32 ? 4 : 2;
   const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
   // BF16 mode: the fp16 copy of W2 that f2 reads is written by extra blocks of the attention's bias
   // kernel (one launch fewer)
   const bool w2_early = desc->dtype == HSTU_BF16;
-  s = run_attn_fwd(&ad, jag, uvqk + 2 * D * es, uvqk + 3 * D * es, uvqk + 1 * D * es, w->rab_pos, w->rab_time,
-                   saved->o, ws, st, true, nullptr, nullptr, saved->attn_bias, w->W2, wsb + lay.w2_f16,
-                   w2_early ? static_cast<int64_t>(D) * D : 0);
+  const AttnFwdPlan plan = plan_attn_fwd(&ad, jag, uvqk + 2 * D * es, uvqk + 3 * D * es, uvqk + 1 * D * es, w->rab_pos,
+                                         w->rab_time, saved->o, ws, true, nullptr, nullptr, saved->attn_bias, w->W2,
+                                         wsb + lay.w2_f16, w2_early ? static_cast<int64_t>(D) * D : 0);
+  // BF16 mode, up to 32 sequences: the attention's work list is computed inside the f1 launch
+  const bool wl_in_f1 = desc->dtype == HSTU_BF16 && jag->B <= 32;
+  s = run_uvqk(T, D, desc->dtype, act, x_op, D, w1_op, w->b1, saved->uvqk, saved->z, status, st, x32,
+               wl_in_f1 ? &plan.wl : nullptr);
+  if (s != HSTU_OK) return s;
+  s = launch_attn_fwd(plan, st, wl_in_f1);
   if (s != HSTU_OK) return s;
   // G in fp16 (BF16 mode): f2 then reads an fp16 copy of W2
   const hstu_dtype_t g_dt = desc->dtype == HSTU_BF16 ? HSTU_F16 : HSTU_F32;

@@ -98,12 +98,32 @@ cudaError_t ensure_smem_attr(const void* kernel, int bytes);
 // Multiprocessors of the current device (cached per device; 148 when the query fails).
 int sm_count();
 
-cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st);
+// A batch's work list for at most 32 sequences, as launch_worklist writes it (its arguments, below).
+struct WorklistArgs {
+  const int64_t* off;
+  int B;
+  int64_t T;
+  int max_len;
+  int32_t* items;
+  int32_t* count;
+  int* status;
+  long long* pair_base;
+  int32_t* kitems;
+  int32_t* kcount;
+  int32_t* sched;
+  int32_t* pack;
+  int32_t* urec;
+  int32_t* sched2;
+};
+
+// side (optional, B <= 32): the work list is computed in the same launch by a warp that the GEMM
+// leaves idle (one launch fewer before the kernels that read it).
+cudaError_t gemm_bf16(const GemmArgs& g, cudaStream_t st, const WorklistArgs* side = nullptr);
 // Two independent products in one launch (n = 1 or 2; empty products are skipped). With `sched`
 // (two ints, zero before the first launch; each launch leaves them zero) the CTAs take work units
 // from a global counter in order, so the caller lists the product with the larger units first;
-// without it every CTA runs a fixed stride of units.
-cudaError_t gemm_bf16_group(const GemmArgs* g, int n, int* sched, cudaStream_t st);
+// without it every CTA runs a fixed stride of units (and may carry a work list as `side`).
+cudaError_t gemm_bf16_group(const GemmArgs* g, int n, int* sched, cudaStream_t st, const WorklistArgs* side = nullptr);
 cudaError_t gemm_f32(const GemmArgs& g, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------------

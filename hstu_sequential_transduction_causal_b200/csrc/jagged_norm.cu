@@ -10,18 +10,14 @@
 #include "time_bucket_dev.cuh"
 #include "bias_tile.cuh"
 #include "vec_io.cuh"
+#include "worklist.cuh"
 
 namespace hstu {
 
 namespace {
 
-// Short sequences share a tile: a run of consecutive sequences of at most kPackMaxLen tokens each
-// (empty ones included) whose rows add up to at most 128 becomes one 128-row tile, so a batch of
-// short histories does not leave most of every tile empty. Greedy in batch order inside chunks of 32
-// sequences (chunks are packed independently, so a block packs them in parallel). pack[b]: k >= 2
-// for the first sequence of a pack of k, 0 for the other members, 1 for a sequence on its own.
-constexpr int kPackMaxLen = 64;
-
+// Short sequences share a tile (worklist.cuh: pack): greedy in batch order inside chunks of 32
+// sequences (chunks are packed independently, so a block packs them in parallel).
 __device__ void pack_chunk(const int64_t* __restrict__ off, int b0, int b1, int32_t* pack) {
   int i = b0;
   while (i < b1) {
@@ -41,28 +37,6 @@ __device__ void pack_chunk(const int64_t* __restrict__ off, int b0, int b1, int3
     pack[i] = k;
     for (int j = 1; j < k; ++j) pack[i + j] = 0;
     i += k;
-  }
-}
-
-// Unit records of the persistent attention forward, one per work item p: {b, tile, row0, n, pair0,
-// 0, 0, 0} (int32): the item, the first row and row count its tiles cover (a pack's rows for a pack),
-// and the index of its query tile's first causal pair. Run by threads [tid, tid + nthreads) after
-// items, count and pair_base are written and visible to them.
-__device__ void write_unit_records(const int64_t* __restrict__ off, const int32_t* items, int count,
-                                   const long long* pair_base, int32_t* urec, int tid, int nthreads) {
-  for (int p = tid; p < count; p += nthreads) {
-    const int b = items[2 * p], t = items[2 * p + 1];
-    const int k = t < 0 ? -t : 1;
-    const int qt = t < 0 ? 0 : t;
-    int4 r0, r1;
-    r0.x = b;
-    r0.y = t;
-    r0.z = static_cast<int>(off[b]);
-    r0.w = static_cast<int>(off[b + k] - off[b]);
-    r1.x = static_cast<int>(pair_base[b] + static_cast<long long>(qt) * (qt + 1) / 2);
-    r1.y = r1.z = r1.w = 0;
-    reinterpret_cast<int4*>(urec)[2 * p] = r0;
-    reinterpret_cast<int4*>(urec)[2 * p + 1] = r1;
   }
 }
 
@@ -247,76 +221,14 @@ worklist_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, 
   write_unit_records(off, items, s_base, pair_base, urec, tid, blockDim.x);
 }
 
-// The same lists for batches of at most 32 sequences, from a single warp (no block barriers):
-// lane b owns sequence b; the items are written tile index by tile index, longest first, as above.
+// The same lists for batches of at most 32 sequences, from a single warp (worklist.cuh).
 __global__ void __launch_bounds__(32)
 worklist_warp_kernel(const int64_t* __restrict__ off, int B, int64_t T, int max_len, int32_t* items, int32_t* count,
                      int* status, long long* pair_base, int32_t* kitems, int32_t* kcount, int32_t* sched,
                      int32_t* pack, int32_t* urec, int32_t* sched2) {
   pdl_enter();
-  if (threadIdx.x == 0) {   // the persistent attention kernels' unit (and finished-CTA) counters
-    if (sched) sched[0] = 0;
-    if (sched2) sched2[0] = sched2[1] = 0;
-  }
-  const int lane = threadIdx.x;
-  const bool mine = lane < B;
-  long long n = 0;
-  if (mine) n = off[lane + 1] - off[lane];
-  bool bad = (B < 0 || B > 32 || off[0] != 0 || off[B > 0 ? B : 0] != T || (mine && (n < 0 || n > max_len)));
-  bad = __any_sync(0xffffffffu, bad);
-  if (bad) {
-    if (lane == 0) {
-      *count = 0;
-      if (kcount) *kcount = 0;
-      report_error(status, kDevBadInput);
-      if (pair_base) pair_base[B > 0 && B <= 32 ? B : 0] = 0;
-    }
-    return;
-  }
-  const int nt_all = mine ? static_cast<int>((n + kQTile - 1) / kQTile) : 0;
-  int pk = 1;
-  if (pack) {
-    if (lane == 0) pack_chunk(off, 0, B, pack);
-    __syncwarp();
-    if (mine) pk = pack[lane];
-  }
-  const int nt = pk == 0 ? 0 : nt_all;   // a pack member's rows are in its pack's tile
-  int max_tiles = nt;
-#pragma unroll
-  for (int d = 16; d > 0; d >>= 1) max_tiles = max(max_tiles, __shfl_xor_sync(0xffffffffu, max_tiles, d));
-  int base = 0;
-  for (int t = max_tiles - 1; t >= 0; --t) {
-    const bool flag = nt > t;
-    const unsigned m = __ballot_sync(0xffffffffu, flag);
-    if (flag) {
-      const int pos = base + __popc(m & ((1u << lane) - 1u));
-      items[2 * pos] = lane;
-      items[2 * pos + 1] = pk >= 2 ? -pk : t;
-      if (kitems) {
-        kitems[2 * pos] = lane;
-        kitems[2 * pos + 1] = pk >= 2 ? -pk : nt - 1 - t;
-      }
-    }
-    base += __popc(m);
-  }
-  if (lane == 0) {
-    *count = base;
-    if (kcount) *kcount = base;
-  }
-  if (!pair_base) return;
-  const long long v = static_cast<long long>(nt_all) * (nt_all + 1) / 2;
-  long long inc = v;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const long long y = __shfl_up_sync(0xffffffffu, inc, d);
-    if (lane >= d) inc += y;
-  }
-  if (mine) pair_base[lane] = inc - v;
-  const long long total = __shfl_sync(0xffffffffu, inc, 31);
-  if (lane == 0) pair_base[B] = total;
-  if (!urec) return;
-  __syncwarp();
-  write_unit_records(off, items, base, pair_base, urec, lane, 32);
+  worklist_warp(WorklistArgs{off, B, T, max_len, items, count, status, pair_base, kitems, kcount, sched, pack, urec,
+                             sched2});
 }
 
 // Test surface of the attention's time-bucket index: block (x = qt * mt + kt, y = b) writes
