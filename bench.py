@@ -385,9 +385,9 @@ def main():
     n_fwd_kernels = 5
     # fp16 dy with the db2 partial sums, the fp16 copies of x, W1, W2 and the zeroed accumulators (one
     # launch) | dG with dW2 (one grouped GEMM launch) | LN-gate bwd | attention bwd, table gradients (the
-    # transposed bias tiles and the work list come from the forward's cache) | dZ with the db1 partial
-    # sums | finish of db2, dgamma, dbeta and db1 (one launch) | dX with dW1 (one grouped launch)
-    n_bwd_kernels = 8
+    # transposed bias tiles and the work list come from the forward's cache) | dZ with db1, and the
+    # finish of db2, dgamma and dbeta (one launch) | dX with dW1 (one grouped launch)
+    n_bwd_kernels = 7
     names = ["uvqk", "attn", "norm_gate", "out_proj"] + (["backward"] if backward else [])
 
     def attention_forward():

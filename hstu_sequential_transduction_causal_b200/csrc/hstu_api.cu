@@ -140,7 +140,7 @@ AttnBwdWs attn_bwd_ws_layout(const hstu_jagged_t* j, int H, int hb = 1) {
 // (fp32), dZ (fp16 [T, 4D]), reduction partials, dgamma | dbeta, and the fp16 GEMM operands: copies
 // of dy, x, W1 and W2 (both MMA operands share a type; G and dZ are fp16).
 struct LayerBwdWs {
-  size_t dg, dO, dq, dk, dv, dz, part_dy, part_ln, part_dz, dy_f16, x_f16, w1_f16, w2_f16, total;
+  size_t dg, dO, dq, dk, dv, dz, part_dy, part_ln, dy_f16, x_f16, w1_f16, w2_f16, total;
 };
 
 LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) {
@@ -154,11 +154,10 @@ LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) 
   w.dk = take(T * D * 4);
   w.dv = take(T * D * 4);
   w.dz = take(T * 4 * D * 2);
-  // partial column sums: db2 (from the fp16 copy of dY), dgamma | dbeta (LayerNorm backward), db1
-  // (dZ assembly, one row per 32 tokens)
+  // partial column sums: db2 (from the fp16 copy of dY), dgamma | dbeta (LayerNorm backward); db1 is
+  // added up by atomics
   w.part_dy = take(static_cast<size_t>(kTailParts) * D * 4);
   w.part_ln = take(static_cast<size_t>(norm_gate_bwd_blocks(j->T)) * 2 * D * 4);
-  w.part_dz = take(static_cast<size_t>((j->T + 31) / 32) * 4 * D * 4);
   w.dy_f16 = take(T * D * 2);
   w.x_f16 = take(T * D * 2);
   w.w1_f16 = take(4 * D * D * 2);
@@ -998,7 +997,6 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   void* w2_f16 = wsb + lay.w2_f16;
   float* part_dy = reinterpret_cast<float*>(wsb + lay.part_dy);
   float* part_ln = reinterpret_cast<float*>(wsb + lay.part_ln);
-  float* part_dz = reinterpret_cast<float*>(wsb + lay.part_dz);
   int parts_dy = 0, parts_ln = 0;
   float* dG = reinterpret_cast<float*>(wsb + lay.dg);
   void* dO = wsb + lay.dO;
@@ -1016,6 +1014,7 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
     jobs[nj++] = ConvertJob{w->W2, w2_f16, 1ll * D * D, kDtBF16};
     jobs[nj++] = ConvertJob{nullptr, gr->dW2, 1ll * D * D, kDtF32};
     jobs[nj++] = ConvertJob{nullptr, gr->dW1, 4ll * D * D, kDtF32};
+    jobs[nj++] = ConvertJob{nullptr, gr->db1, 4ll * D, kDtF32};
     jobs[nj++] = ConvertJob{nullptr, dq, T * D, kDtF32};
     jobs[nj++] = ConvertJob{nullptr, gr->drab_pos, 2ll * desc->pos_max_len - 1, kDtF32};
     jobs[nj++] = ConvertJob{nullptr, gr->drab_time, desc->n_time_buckets, kDtF32};
@@ -1047,16 +1046,16 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   s = run_attn_bwd(&ad, jag, uvqk + 2 * D * 2, uvqk + 3 * D * 2, uvqk + 1 * D * 2, dO, w->rab_pos, w->rab_time, dq, dk,
                    dv, D, gr->drab_pos, gr->drab_time, ws, st, nullptr, nullptr, saved->attn_bias, true);
   if (s != HSTU_OK) return s;
-  // 4. SiLU backward into dZ[:, D:4D] with the partial sums of db1 = sum_t dZ; then db2, dgamma,
-  // dbeta and db1 finished by one launch straight into the caller's buffers
+  // 4. SiLU backward into dZ[:, D:4D], with db1 = sum_t dZ added up by atomics (zeroed by the first
+  // launch); the first blocks of the same launch finish db2, dgamma and dbeta, all straight into the
+  // caller's buffers
   int parts_dz = 0;
-  e = dz_assemble(T, D, kDtF16, dv, dq, dk, saved->z, 4ll * D, dz, 4ll * D, part_dz, &parts_dz, st);
-  if (e == cudaSuccess) {
-    const ColsumJob jobs[4] = {{part_dy, D, parts_dy, D, gr->db2},
-                               {part_ln, 2ll * D, parts_ln, D, gr->dgamma},
-                               {part_ln + D, 2ll * D, parts_ln, D, gr->dbeta},
-                               {part_dz, 4ll * D, parts_dz, 4 * D, gr->db1}};
-    e = colsum_final_multi(jobs, 4, st);
+  {
+    const ColsumJob fin[3] = {{part_dy, D, parts_dy, D, gr->db2},
+                              {part_ln, 2ll * D, parts_ln, D, gr->dgamma},
+                              {part_ln + D, 2ll * D, parts_ln, D, gr->dbeta}};
+    e = dz_assemble(T, D, kDtF16, dv, dq, dk, saved->z, 4ll * D, dz, 4ll * D, nullptr, &parts_dz, st, gr->db1,
+                    fin, 3);
   }
   // dW2, db2, dgamma, dbeta, db1 and the table gradients are final
   if (e == cudaSuccess && g_ready_events[0]) e = cudaEventRecord(g_ready_events[0], st);

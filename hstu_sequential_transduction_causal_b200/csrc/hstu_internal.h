@@ -272,16 +272,32 @@ cudaError_t convert_f32_to_bf16(const float* in, void* out, int64_t n, cudaStrea
 int norm_gate_bwd_blocks(int64_t T);
 // dO = LayerNorm backward of dLn = dG (.) U; dZ_U = dG (.) Ln (.) SiLU'(Z_U) (fp16, stride ld_dz);
 // the partial sums of dgamma | dbeta into partial [*parts, 2D] (*parts <= norm_gate_bwd_blocks(T));
-// the caller finishes them (colsum_final_multi).
+// the caller finishes them (dz_assemble's finish jobs).
 cudaError_t norm_gate_bwd(int64_t T, int D, int act_dt, const float* dg, const float* o, const void* u,
                           const void* zu, int64_t ld_act, const float* gamma, const float* beta, const float* mu,
                           const float* rstd, void* d_o, void* dz, int64_t ld_dz, float* partial, int* parts,
                           cudaStream_t st, int* status = nullptr);
-// dZ[:, D:4D] = [dV | dQ | dK] (.) SiLU'(Z[:, D:4D]) in fp16 and the partial column sums of all of
-// dZ (dZ[:, 0:D] already written) into partial [*parts = ceil(T / 32), 4D]; D a multiple of 64.
+// A column-sum finish: the sum of a partial buffer's rows.
+struct ColsumJob {
+  const float* partial;   // parts rows of `ld` floats; the job reads columns [0, cols)
+  int64_t ld;
+  int parts;
+  int cols;
+  float* out;             // [cols]
+};
+struct ColsumJobs {
+  ColsumJob job[4];
+  int first_block[5];
+  int njobs;
+};
+// dZ[:, D:4D] = [dV | dQ | dK] (.) SiLU'(Z[:, D:4D]) in fp16 (dZ[:, 0:D] already written) and the
+// column sums of all of dZ in blocks of 32 rows: into partial [*parts = ceil(T / 32), 4D] (may be
+// null) and / or added by fp32 atomics into db1 = sum_t dZ (may be null; zero before the launch).
+// D a multiple of 64. With fin (up to four column sums whose partials earlier launches wrote), the
+// first blocks of the same launch finish those sums.
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
                         const void* z, int64_t ld_z, void* dz, int64_t ld_dz, float* partial, int* parts,
-                        cudaStream_t st);
+                        cudaStream_t st, float* db1 = nullptr, const ColsumJob* fin = nullptr, int nfin = 0);
 // A tensor of n elements (fp32, bf16 or fp16) converted to fp16; with in == null, n fp32 zeros
 // written to out instead (an accumulated output cleared in the same launch).
 struct ConvertJob {
@@ -297,20 +313,6 @@ cudaError_t rows_to_f16_colsum(int64_t T, int D, int in_dt, const void* in, void
                                const ConvertJob* jobs, int njobs, cudaStream_t st);
 // Most partial rows rows_to_f16_colsum writes.
 constexpr int kTailParts = 296;
-// Several column-sum finishes in one launch.
-struct ColsumJob {
-  const float* partial;   // parts rows of `ld` floats; the job reads columns [0, cols)
-  int64_t ld;
-  int parts;
-  int cols;
-  float* out;             // [cols]
-};
-struct ColsumJobs {
-  ColsumJob job[4];
-  int first_block[5];
-  int njobs;
-};
-cudaError_t colsum_final_multi(const ColsumJob* jobs, int njobs, cudaStream_t st);
 size_t colsum_partial_floats(int cols);
 cudaError_t convert_dtype(const void* in, int in_dt, void* out, int out_dt, int64_t n, cudaStream_t st);
 

@@ -260,17 +260,52 @@ norm_gate_bwd_staged_kernel(int64_t T, const float* __restrict__ dg, const float
 // only read back for their sums. The block's 32 rows are summed by shuffles (the 4 rows of a warp)
 // and shared memory (the 8 warps) into partial[row block][cols]; the sums are of the fp16 values
 // stored. Block b covers column block b % (4D / 64) of row block b / (4D / 64).
+// Block blk of a batch of column-sum finishes (job j sums parts rows, row stride ld, of its partial
+// buffer into out[0 .. cols)): 32 columns of one job, each summed over its partial rows by the 8
+// warps (rows p = warp mod 8) and then across warps through s_part.
+__device__ __forceinline__ void colsum_finish_block(const ColsumJobs& jobs, int blk, float (*s_part)[33]) {
+  int j = 0;
+  while (j + 1 < jobs.njobs && blk >= jobs.first_block[j + 1]) ++j;
+  const ColsumJob& jb = jobs.job[j];
+  const int cl = threadIdx.x & 31, slice = threadIdx.x >> 5;
+  const int c = (blk - jobs.first_block[j]) * 32 + cl;
+  float s0 = 0.0f, s1 = 0.0f;
+  if (c < jb.cols) {
+    int p = slice;
+    for (; p + 8 < jb.parts; p += 16) {
+      s0 += jb.partial[static_cast<int64_t>(p) * jb.ld + c];
+      s1 += jb.partial[static_cast<int64_t>(p + 8) * jb.ld + c];
+    }
+    if (p < jb.parts) s0 += jb.partial[static_cast<int64_t>(p) * jb.ld + c];
+  }
+  s_part[slice][cl] = s0 + s1;
+  __syncthreads();
+  if (slice == 0 && c < jb.cols) {
+    float t = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) t += s_part[k][cl];
+    jb.out[c] = t;
+  }
+}
+
 template <int AT>
 __global__ void __launch_bounds__(256)
 dz_assemble_kernel(int64_t T, int D, const float* __restrict__ dv, const float* __restrict__ dq,
                    const float* __restrict__ dk, const void* __restrict__ z, int64_t ld_z, void* __restrict__ dz,
-                   int64_t ld_dz, float* __restrict__ partial) {
+                   int64_t ld_dz, float* __restrict__ partial, float* __restrict__ db1, ColsumJobs fin,
+                   int fin_blocks) {
   __shared__ float s_red[8][64];
+  __shared__ float s_fin[8][33];
   pdl_enter();
+  if (static_cast<int>(blockIdx.x) < fin_blocks) {   // (block-uniform) a finish of an earlier launch's sums
+    colsum_finish_block(fin, static_cast<int>(blockIdx.x), s_fin);
+    return;
+  }
+  const int blk = static_cast<int>(blockIdx.x) - fin_blocks;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ncb = 4 * D / 64;
-  const int cb = static_cast<int>(blockIdx.x % ncb);
-  const int64_t rb = blockIdx.x / ncb;
+  const int cb = blk % ncb;
+  const int64_t rb = blk / ncb;
   const int c = 64 * cb + 8 * (lane & 7);   // column of dZ, in [0, 4D)
   const int64_t row = 32 * rb + 4 * warp + (lane >> 3);
   float v[8];
@@ -303,7 +338,8 @@ dz_assemble_kernel(int64_t T, int D, const float* __restrict__ dv, const float* 
     float t = 0.0f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) t += s_red[w][threadIdx.x];
-    partial[rb * 4 * D + 64 * cb + threadIdx.x] = t;
+    if (partial) partial[rb * 4 * D + 64 * cb + threadIdx.x] = t;
+    if (db1) atomicAdd(db1 + 64 * cb + threadIdx.x, t);
   }
 }
 
@@ -403,36 +439,6 @@ rows_to_f16_colsum_kernel(int64_t T, const void* __restrict__ in, void* __restri
   if (rp == 0)
 #pragma unroll
     for (int e = 0; e < 8; ++e) partial[static_cast<int64_t>(blockIdx.x) * D + c + e] = acc[e];
-}
-
-// Several column-sum finishes in one launch: job j sums parts rows (row stride ld) of its partial
-// buffer into out[0 .. cols); each block takes 32 columns of one job (as colsum_final_kernel).
-__global__ void __launch_bounds__(256)
-colsum_final_multi_kernel(ColsumJobs jobs) {
-  pdl_enter();
-  __shared__ float s_part[8][33];
-  int j = 0;
-  while (j + 1 < jobs.njobs && static_cast<int>(blockIdx.x) >= jobs.first_block[j + 1]) ++j;
-  const ColsumJob& jb = jobs.job[j];
-  const int cl = threadIdx.x & 31, slice = threadIdx.x >> 5;
-  const int c = (static_cast<int>(blockIdx.x) - jobs.first_block[j]) * 32 + cl;
-  float s0 = 0.0f, s1 = 0.0f;
-  if (c < jb.cols) {
-    int p = slice;
-    for (; p + 8 < jb.parts; p += 16) {
-      s0 += jb.partial[static_cast<int64_t>(p) * jb.ld + c];
-      s1 += jb.partial[static_cast<int64_t>(p + 8) * jb.ld + c];
-    }
-    if (p < jb.parts) s0 += jb.partial[static_cast<int64_t>(p) * jb.ld + c];
-  }
-  s_part[slice][cl] = s0 + s1;
-  __syncthreads();
-  if (slice == 0 && c < jb.cols) {
-    float t = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) t += s_part[k][cl];
-    jb.out[c] = t;
-  }
 }
 
 // partial[y][c] = sum over rows [y R, (y+1) R) of in[row][c]; one thread per column.
@@ -578,21 +584,41 @@ int tail_parts(int64_t T, int64_t* rows_per) {
 }
 }  // namespace
 
+namespace {
+// Packs up to four column-sum finishes (32 columns a block); returns the block count.
+int pack_colsum_jobs(const ColsumJob* jobs, int njobs, ColsumJobs* cj) {
+  *cj = ColsumJobs{};
+  int nb = 0, k = 0;
+  for (int j = 0; j < njobs && j < 4; ++j) {
+    if (jobs[j].cols <= 0) continue;
+    cj->job[k] = jobs[j];
+    cj->first_block[k] = nb;
+    nb += (jobs[j].cols + 31) / 32;
+    ++k;
+  }
+  cj->first_block[k] = nb;
+  cj->njobs = k;
+  return nb;
+}
+}  // namespace
+
 cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const float* dq, const float* dk,
                         const void* z, int64_t ld_z, void* dz, int64_t ld_dz, float* partial, int* parts,
-                        cudaStream_t st) {
+                        cudaStream_t st, float* db1, const ColsumJob* fin, int nfin) {
   *parts = static_cast<int>((T + 31) / 32);
   if (T == 0) return cudaSuccess;
-  if (D % 64) return cudaErrorInvalidValue;
+  if (D % 64 || nfin > 4) return cudaErrorInvalidValue;
   const int64_t blocks = static_cast<int64_t>(4 * D / 64) * *parts;
-  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>(blocks));
+  ColsumJobs cj;
+  const int fin_blocks = pack_colsum_jobs(fin, fin ? nfin : 0, &cj);
+  if (blocks + fin_blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(blocks + fin_blocks));
   if (act_dt == kDtF16)
     return launch_pdl(dz_assemble_kernel<kDtF16>, grid, dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz,
-                      partial);
+                      partial, db1, cj, fin_blocks);
   if (act_dt == kDtBF16)
     return launch_pdl(dz_assemble_kernel<kDtBF16>, grid, dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz,
-                      partial);
+                      partial, db1, cj, fin_blocks);
   return cudaErrorInvalidValue;
 }
 
@@ -634,21 +660,6 @@ cudaError_t rows_to_f16_colsum(int64_t T, int D, int in_dt, const void* in, void
   return cudaErrorInvalidValue;
 }
 
-cudaError_t colsum_final_multi(const ColsumJob* jobs, int njobs, cudaStream_t st) {
-  ColsumJobs cj{};
-  int nb = 0, k = 0;
-  for (int j = 0; j < njobs && j < 4; ++j) {
-    if (jobs[j].cols <= 0) continue;
-    cj.job[k] = jobs[j];
-    cj.first_block[k] = nb;
-    nb += (jobs[j].cols + 31) / 32;
-    ++k;
-  }
-  if (k == 0) return cudaSuccess;
-  cj.first_block[k] = nb;
-  cj.njobs = k;
-  return launch_pdl(colsum_final_multi_kernel, dim3(static_cast<unsigned>(nb)), dim3(256), 0, st, cj);
-}
 
 cudaError_t convert_dtype(const void* in, int in_dt, void* out, int out_dt, int64_t n, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
