@@ -396,8 +396,8 @@ def main():
 
     # CUDA events the library records right around its dominant kernels (hstu_profile_events); captured
     # into the step graph as event nodes, read after every timed replay
-    prof_kernels = [H.PROFILE_ATTN_FWD, H.PROFILE_NORM_FWD] + ([H.PROFILE_ATTN_BWD, H.PROFILE_NORM_BWD]
-                                                                if backward else [])
+    prof_kernels = [H.PROFILE_ATTN_FWD, H.PROFILE_NORM_FWD, H.PROFILE_BIAS] + (
+        [H.PROFILE_ATTN_BWD, H.PROFILE_NORM_BWD, H.PROFILE_TABLE_GRAD, H.PROFILE_DZ] if backward else [])
     prof_ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in prof_kernels}
     prof_ms = {k: [] for k in prof_kernels}
 
@@ -682,6 +682,21 @@ def main():
         rooflines["norm_gate_fwd"]["same_size_copy"] = {
             "achieved": cpy, "unit": "GB/s", "frac": rooflines["norm_gate_fwd"]["achieved"] / cpy,
             "what": "torch device copy of the same bytes from cold memory, CUDA events"}
+
+        def hbm_line(kernel, nbytes, what):
+            a_ = nbytes / (kern_ms[kernel] / 1e3) / 1e9
+            c_ = same_size_copy_gbs(nbytes)
+            return {"bound": "hbm", "achieved": a_, "peak": hbm_peak, "unit": "GB/s", "frac": a_ / hbm_peak,
+                    "algorithmic_bytes_per_launch": int(nbytes), "ms": kern_ms[kernel], "what": what,
+                    "same_size_copy": {"achieved": c_, "unit": "GB/s", "frac": a_ / c_,
+                                       "what": "torch device copy of the same bytes from cold memory, CUDA events"}}
+        # causal 128 x 128 tile pairs (this workload packs no sequence)
+        nt_b = (np.diff(wl.offsets) + 127) // 128
+        n_pairs = int(np.sum(nt_b * (nt_b + 1) // 2))
+        # bias tiles with the layer's cache: per pair the fp16 half-bias tile, its key-major copy and the
+        # u8 buckets written; the fp16 W2 copy (read bf16, write fp16); the timestamps read
+        rooflines["bias_tiles"] = hbm_line(H.PROFILE_BIAS, n_pairs * (32768 + 32768 + 16384) + 4 * D * D + 8 * T,
+                                           f"{n_pairs} causal tile pairs: 80 KB written per pair, + W2 copy")
         if backward:
             # attention backward: four contractions (P recompute not counted) = 2x the forward's flops
             bw = 2 * flops / (kern_ms[H.PROFILE_ATTN_BWD] / 1e3) / 1e12
@@ -698,6 +713,13 @@ def main():
             rooflines["norm_gate_bwd"]["same_size_copy"] = {
                 "achieved": cpy, "unit": "GB/s", "frac": a_ / cpy,
                 "what": "torch device copy of the same bytes from cold memory, CUDA events"}
+            # table gradients: every (pair, head) dX^T tile (fp16) and every pair's u8 bucket tile read
+            rooflines["table_gradients"] = hbm_line(
+                H.PROFILE_TABLE_GRAD, n_pairs * (wl.H * 32768 + 16384),
+                f"{n_pairs} pairs x {wl.H} heads of 32 KB dX^T + 16 KB buckets read")
+            # dZ assembly: dV, dQ, dK fp32 and Z[:, D:4D] fp16 read, dZ_U fp16 read back, dZ[:, D:4D] fp16
+            # written (the db2 / dgamma / dbeta finishes read a few partial rows more)
+            rooflines["dz_assembly"] = hbm_line(H.PROFILE_DZ, 26 * T * D, "26 bytes per token and feature")
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_oracle_sample(wl, backward)

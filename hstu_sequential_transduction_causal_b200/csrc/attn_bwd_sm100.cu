@@ -816,9 +816,13 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (e == cudaSuccess) e = prof_record(kProfAttnBwd, true, st);
   if (e != cudaSuccess) return e;
   auto tg = f16 ? attn_table_grad_kernel<true> : attn_table_grad_kernel<false>;
-  return launch_pdl(tg, dim3(static_cast<unsigned>(bias_grid_pairs(a.max_pairs, a.bias_heads) * 2), 2,
-                             static_cast<unsigned>(a.bias_heads)),
-                    dim3(kTgThreads), 0, st, A);
+  e = prof_record(kProfTableGrad, false, st);
+  if (e == cudaSuccess)
+    e = launch_pdl(tg, dim3(static_cast<unsigned>(bias_grid_pairs(a.max_pairs, a.bias_heads) * 2), 2,
+                            static_cast<unsigned>(a.bias_heads)),
+                   dim3(kTgThreads), 0, st, A);
+  if (e == cudaSuccess) e = prof_record(kProfTableGrad, true, st);
+  return e;
 }
 
 }  // namespace hstu

@@ -1034,9 +1034,12 @@ cudaError_t attn_fwd_tc2(const AttnArgs& a_in, cudaStream_t st) {
   a.bias_blocks = bias_tile_grid(a.max_pairs, a.bias_heads);
   const int64_t cvt_blocks = a.cvt_n > 0 ? (a.cvt_n + 8 * kBiasThreads - 1) / (8 * kBiasThreads) : 0;
   if (a.bias_blocks + cvt_blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  e = launch_pdl(attn_bias_kernel,
-                 dim3(static_cast<unsigned>(a.bias_blocks + cvt_blocks), static_cast<unsigned>(a.bias_heads)),
-                 dim3(kBiasThreads), bias_dyn, st, a);
+  e = prof_record(kProfBias, false, st);
+  if (e == cudaSuccess)
+    e = launch_pdl(attn_bias_kernel,
+                   dim3(static_cast<unsigned>(a.bias_blocks + cvt_blocks), static_cast<unsigned>(a.bias_heads)),
+                   dim3(kBiasThreads), bias_dyn, st, a);
+  if (e == cudaSuccess) e = prof_record(kProfBias, true, st);
   if (e != cudaSuccess) return e;
   const bool f16 = a.in_f16 != 0;
   // the persistent kernel's unit counter lives in the workspace header (reset by the work list), its

@@ -36,7 +36,10 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 // before and right after the dominant kernel of a call; under stream capture they become external
 // event-record nodes, so graph replays time the kernel too. Per host thread; no-op when unset.
 // ---------------------------------------------------------------------------------------------
-enum : int { kProfAttnFwd = 0, kProfAttnBwd = 1, kProfNormFwd = 2, kProfNormBwd = 3, kProfKernels = 4 };
+enum : int {
+  kProfAttnFwd = 0, kProfAttnBwd = 1, kProfNormFwd = 2, kProfNormBwd = 3, kProfBias = 4, kProfTableGrad = 5, kProfDz = 6,
+  kProfKernels = 7
+};
 cudaError_t prof_record(int kernel, bool stop, cudaStream_t st);
 
 // ---------------------------------------------------------------------------------------------

@@ -613,13 +613,15 @@ cudaError_t dz_assemble(int64_t T, int D, int act_dt, const float* dv, const flo
   const int fin_blocks = pack_colsum_jobs(fin, fin ? nfin : 0, &cj);
   if (blocks + fin_blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(blocks + fin_blocks));
-  if (act_dt == kDtF16)
-    return launch_pdl(dz_assemble_kernel<kDtF16>, grid, dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz,
-                      partial, db1, cj, fin_blocks);
-  if (act_dt == kDtBF16)
-    return launch_pdl(dz_assemble_kernel<kDtBF16>, grid, dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z, dz, ld_dz,
-                      partial, db1, cj, fin_blocks);
-  return cudaErrorInvalidValue;
+  if (act_dt != kDtF16 && act_dt != kDtBF16) return cudaErrorInvalidValue;
+  cudaError_t e = prof_record(kProfDz, false, st);
+  if (e == cudaSuccess)
+    e = act_dt == kDtF16 ? launch_pdl(dz_assemble_kernel<kDtF16>, grid, dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z,
+                                      dz, ld_dz, partial, db1, cj, fin_blocks)
+                         : launch_pdl(dz_assemble_kernel<kDtBF16>, grid, dim3(256), 0, st, T, D, dv, dq, dk, z, ld_z,
+                                      dz, ld_dz, partial, db1, cj, fin_blocks);
+  if (e == cudaSuccess) e = prof_record(kProfDz, true, st);
+  return e;
 }
 
 cudaError_t rows_to_f16_colsum(int64_t T, int D, int in_dt, const void* in, void* out, float* partial, int* parts,

@@ -244,6 +244,7 @@ def hstu_set_wait_limit(cycles: int) -> None:
 
 
 PROFILE_ATTN_FWD, PROFILE_ATTN_BWD, PROFILE_NORM_FWD, PROFILE_NORM_BWD = 0, 1, 2, 3
+PROFILE_BIAS, PROFILE_TABLE_GRAD, PROFILE_DZ = 4, 5, 6
 
 
 def hstu_profile_events(kernel: int, start=None, stop=None) -> None:

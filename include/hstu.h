@@ -199,7 +199,9 @@ void hstu_set_wait_limit(uint64_t cycles);
  * cudaEventElapsedTime(start, stop) is that kernel's device time (under stream capture the records
  * become external event nodes of the graph, re-recorded at each replay). kernel: 0 the attention
  * forward (hstu_attn_fwd, hstu_layer_fwd), 1 the attention backward (hstu_attn_bwd,
- * hstu_layer_bwd), 2 the LayerNorm (.) U forward, 3 its backward. start = stop = NULL disables.
+ * hstu_layer_bwd), 2 the LayerNorm (.) U forward, 3 its backward, 4 the forward's bias-tile kernel
+ * (with the layer's cache writes and fp16 W2 copy in hstu_layer_fwd), 5 the table gradients of the
+ * attention backward, 6 the layer backward's dZ assembly. start = stop = NULL disables.
  * HSTU_ERR_INVALID_ARG for another kernel number or only one NULL event. */
 hstu_status_t hstu_profile_events(int32_t kernel, void* start, void* stop);
 

@@ -513,11 +513,11 @@ def test_last_cuda_error_is_per_host_thread(L):
 
 
 def test_profile_events(L):
-    assert L.hstu_profile_events(4, fake(0), fake(1)) == INVALID        # no such kernel
+    assert L.hstu_profile_events(7, fake(0), fake(1)) == INVALID        # no such kernel
     assert L.hstu_profile_events(-1, None, None) == INVALID
     assert L.hstu_profile_events(0, fake(0), None) == INVALID           # one event only
     assert L.hstu_profile_events(0, None, fake(1)) == INVALID
-    for k in range(4):
+    for k in range(7):
         assert L.hstu_profile_events(k, None, None) == OK               # disabling is always fine
 
 
