@@ -77,19 +77,37 @@ struct BwdUnit {
   long long seq0, pbase;
 };
 
-__device__ __forceinline__ BwdUnit bwd_unit(const AttnBwdArgs& A, int u) {
+// What the scheduler warp publishes for a unit (its global lookups resolved while the CTA's current
+// unit still runs, so the other roles start the next unit without a chain of dependent loads).
+struct BwdRec {
+  int u, b, kt_item, n;
+  long long seq0, pbase;
+};
+
+__device__ __forceinline__ BwdRec bwd_rec(const AttnBwdArgs& A, int u) {
   const AttnArgs& a = A.f;
-  BwdUnit w;
+  BwdRec r{u, 0, 0, 0, 0, 0};
   const int item = u / a.H;
-  w.h = u - item * a.H;
-  w.b = A.kitems[2 * item];
-  w.kt_item = A.kitems[2 * item + 1];
+  r.b = A.kitems[2 * item];
+  r.kt_item = A.kitems[2 * item + 1];
+  pair_rows(a.offsets, a.pack, r.b, &r.seq0, &r.n);
+  r.pbase = a.pair_base[r.b];
+  return r;
+}
+
+__device__ __forceinline__ BwdUnit bwd_unit(const BwdRec& r, int H) {
+  BwdUnit w;
+  const int item = r.u / H;
+  w.h = r.u - item * H;
+  w.b = r.b;
+  w.kt_item = r.kt_item;
   w.packed = w.kt_item < 0;   // a pack of -kt_item short sequences: one diagonal tile
   w.kt = w.packed ? 0 : w.kt_item;
-  pair_rows(a.offsets, a.pack, w.b, &w.seq0, &w.n);
+  w.seq0 = r.seq0;
+  w.n = r.n;
   w.nt = (w.n + kQTile - 1) / kQTile;
   w.nsteps = w.nt - w.kt;     // query tiles kt .. nt-1
-  w.pbase = a.pair_base[w.b];
+  w.pbase = r.pbase;
   return w;
 }
 
@@ -120,7 +138,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   constexpr int kNumBars = 24 + 3 * kRingB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* ring = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile BwdRec* ring = reinterpret_cast<volatile BwdRec*>(tmem_slot + 2);   // kRingB records
+  static_assert(8 * kNumBars + 8 + kRingB * sizeof(BwdRec) <= 512 && (8 * kNumBars + 8) % 8 == 0, "barrier region");
   const uint32_t bar0 = smem_u32(bars);
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   auto qdo_full = [&](int sq) { return sq < 2 ? BAR(1 + sq) : BAR(21); };
@@ -190,20 +209,30 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const uint32_t sDQ = smem_u32(smem + Lb::kDQ);
 
   // Unit i of this CTA for one reading thread (false: the wait gave up); u >= total ends the
-  // sequence. The reader frees the ring slot once it holds the value.
-  auto take_unit = [&](int i, int& u) -> bool {
+  // sequence. The reader frees the ring slot once it holds the record.
+  auto take_unit = [&](int i, BwdRec& rec) -> bool {
     const int r = i % kRingB;
     if (!mbar_wait(ring_full(r), (i / kRingB) & 1, abort_flag, ctl)) return false;
-    u = ring[r];
+    rec.u = ring[r].u;
+    rec.b = ring[r].b;
+    rec.kt_item = ring[r].kt_item;
+    rec.n = ring[r].n;
+    rec.seq0 = ring[r].seq0;
+    rec.pbase = ring[r].pbase;
     mbar_arrive(ring_empty(r));
     return true;
   };
-  auto take_unit_warp = [&](int i, int& u) -> bool {
-    int v = 0;
+  auto take_unit_warp = [&](int i, BwdRec& rec) -> bool {
+    BwdRec v{0, 0, 0, 0, 0, 0};
     bool ok = true;
     if (lane == 0) ok = take_unit(i, v);
     ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-    u = __shfl_sync(0xffffffffu, v, 0);
+    rec.u = __shfl_sync(0xffffffffu, v.u, 0);
+    rec.b = __shfl_sync(0xffffffffu, v.b, 0);
+    rec.kt_item = __shfl_sync(0xffffffffu, v.kt_item, 0);
+    rec.n = __shfl_sync(0xffffffffu, v.n, 0);
+    rec.seq0 = __shfl_sync(0xffffffffu, v.seq0, 0);
+    rec.pbase = __shfl_sync(0xffffffffu, v.pbase, 0);
     return ok;
   };
 
@@ -216,10 +245,20 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     int G = 0;
     bool ok = true;
     for (int i = 0; ok; ++i) {
-      int u;
-      if (!take_unit_warp(i, u) || u >= total) break;
-      const BwdUnit w = bwd_unit(A, u);
+      BwdRec rec;
+      if (!take_unit_warp(i, rec) || rec.u >= total) break;
+      const BwdUnit w = bwd_unit(rec, a.H);
       const int krow = static_cast<int>(w.seq0) + w.kt * kQTile;
+      // K and V (read by this unit alone, so usually from DRAM) and the first bias tile into L2 now:
+      // their loads wait until the previous unit's last MMAs have completed
+      if (i >= 1 && lane == 0 && w.nsteps > 0) {
+        tma_prefetch_l2_2d(&tmK, w.h * kD, krow);
+        tma_prefetch_l2_2d(&tmV, w.h * kD, krow);
+        const long long pair0 = w.pbase + static_cast<long long>(w.kt) * (w.kt + 1) / 2 + w.kt;
+        const int prow0 = static_cast<int>((pair0 * a.bias_heads + (a.bias_heads > 1 ? w.h : 0)) * kQTile);
+        tma_prefetch_l2_2d(&tmBT, 0, prow0);
+        tma_prefetch_l2_2d(&tmBT, 64, prow0);
+      }
       auto load_bias = [&](int s) -> bool {
         const int gs = G + s, st = gs & 1, qt = w.kt + s;
         if (gs >= 2 && !mbar_wait_warp(BAR(7 + st), ((gs >> 1) & 1) ^ 1, abort_flag, ctl)) return false;
@@ -310,9 +349,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       int G = 0;
       bool ok = true;
       for (int i = 0; ok; ++i) {
-        int u;
-        if (!take_unit(i, u) || u >= total) break;
-        const BwdUnit w = bwd_unit(A, u);
+        BwdRec rec;
+        if (!take_unit(i, rec) || rec.u >= total) break;
+        const BwdUnit w = bwd_unit(rec, a.H);
         if (!mbar_wait(BAR(0), i & 1, abort_flag, ctl) || !issue_s(G)) break;
         for (int s = 0; ok && s < w.nsteps; ++s) {
           const int gs = G + s, st = gs & 1;
@@ -355,9 +394,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     int G = 0;
     bool ok = true;
     for (int i = 0; ok; ++i) {
-      int u;
-      if (!take_unit_warp(i, u) || u >= total) break;
-      const BwdUnit w = bwd_unit(A, u);
+      BwdRec rec;
+      if (!take_unit_warp(i, rec) || rec.u >= total) break;
+      const BwdUnit w = bwd_unit(rec, a.H);
       auto reduce_dq = [&](int gj, int qt) -> bool {
         if (!mbar_wait_warp(BAR(17), gj & 1, abort_flag, ctl)) return false;
         if (lane < 2) {
@@ -405,8 +444,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int r = i % kRingB;
         if (i >= 1 && !mbar_wait(ring_got((i - 1) % kRingB), ((i - 1) / kRingB) & 1, abort_flag, ctl)) break;
         const int u = i == 0 ? static_cast<int>(blockIdx.x) : static_cast<int>(gridDim.x) + atomicAdd(A.sched, 1);
+        const BwdRec rec = u < total ? bwd_rec(A, u) : BwdRec{u, 0, 0, 0, 0, 0};
         if (i >= kRingB && !mbar_wait(ring_empty(r), ((i / kRingB) - 1) & 1, abort_flag, ctl)) break;
-        ring[r] = u;
+        ring[r].u = rec.u;
+        ring[r].b = rec.b;
+        ring[r].kt_item = rec.kt_item;
+        ring[r].n = rec.n;
+        ring[r].seq0 = rec.seq0;
+        ring[r].pbase = rec.pbase;
         mbar_arrive(ring_full(r));
         if (u >= total) break;
       }
@@ -479,9 +524,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     };
     int G = 0;
     for (int i = 0; ok; ++i) {
-      int u;
-      if (!take_unit_warp(i, u) || u >= total) break;
-      const BwdUnit w = bwd_unit(A, u);
+      BwdRec rec;
+      if (!take_unit_warp(i, rec) || rec.u >= total) break;
+      const BwdUnit w = bwd_unit(rec, a.H);
       const int kt = w.kt, n = w.n, nt = w.nt, nsteps = w.nsteps;
       const long long seq0 = w.seq0;
       // in a pack, queries past the end of the key row's own sequence are masked
