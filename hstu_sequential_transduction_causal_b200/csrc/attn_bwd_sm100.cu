@@ -593,21 +593,50 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_arrive(BAR(15 + st));
     }
     if (ok && hq == 1 && nsteps > 0 && !stage_dq(G + nsteps - 1)) ok = false;
+    // dK, dV: key row = TMEM lane, columns [16 (2 hq + sub), +16) of the head
+    const int cc = 16 * (2 * hq + sub);
+    const bool row_in = kt * kQTile + rj < n;
+    const long long row = seq0 + kt * kQTile + rj;
+    // (layer backward) the Z_K, Z_V values of those columns, loaded while the unit's last MMAs drain
+    uint4 zk4[2] = {}, zv4[2] = {};
+    if (A.dz_k && ok && row_in) {
+      const long long zo = row * A.ld_z + w.h * kD + cc;
+      const uint4* zkp = reinterpret_cast<const uint4*>(static_cast<const __half*>(A.z_k) + zo);
+      const uint4* zvp = reinterpret_cast<const uint4*>(static_cast<const __half*>(A.z_v) + zo);
+      zk4[0] = zkp[0]; zk4[1] = zkp[1];
+      zv4[0] = zvp[0]; zv4[1] = zvp[1];
+    }
     if (ok && !mbar_wait(BAR(14), i & 1, abort_flag, ctl)) ok = false;
     if (ok) {
       tc_fence_after();
-      // dK, dV: key row = TMEM lane, columns [16 (2 hq + sub), +16); then the accumulators are free
-      // for the next unit
-      const int cc = 16 * (2 * hq + sub);
       uint32_t vk[16], vv[16];
       tmem_ld_32x32b_x16(tDK + lane_base + cc, vk);
       tmem_ld_32x32b_x16(tDV + lane_base + cc, vv);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(BAR(23));
+      mbar_arrive(BAR(23));   // the accumulators are free for the next unit
       const int h = w.h;
-      if (kt * kQTile + rj < n) {
-        const long long row = seq0 + kt * kQTile + rj;
+      if (row_in && A.dz_k) {
+        // dZ_K = dK (.) SiLU'(Z_K), dZ_V = (dV inv_N) (.) SiLU'(Z_V), rounded once to fp16
+        uint32_t ok2[8], ov2[8];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const uint32_t zkw = e2 < 4 ? (&zk4[0].x)[e2] : (&zk4[1].x)[e2 - 4];
+          const uint32_t zvw = e2 < 4 ? (&zv4[0].x)[e2] : (&zv4[1].x)[e2 - 4];
+          const float2 zk = unpack_f16x2(zkw), zv = unpack_f16x2(zvw);
+          ok2[e2] = pack_f16x2(__uint_as_float(vk[2 * e2]) * silu_grad(zk.x),
+                               __uint_as_float(vk[2 * e2 + 1]) * silu_grad(zk.y));
+          ov2[e2] = pack_f16x2((__uint_as_float(vv[2 * e2]) * inv_N) * silu_grad(zv.x),
+                               (__uint_as_float(vv[2 * e2 + 1]) * inv_N) * silu_grad(zv.y));
+        }
+        const long long zo = row * A.ld_z + h * kD + cc;
+        uint4* dzk = reinterpret_cast<uint4*>(static_cast<__half*>(A.dz_k) + zo);
+        uint4* dzv = reinterpret_cast<uint4*>(static_cast<__half*>(A.dz_v) + zo);
+        dzk[0] = make_uint4(ok2[0], ok2[1], ok2[2], ok2[3]);
+        dzk[1] = make_uint4(ok2[4], ok2[5], ok2[6], ok2[7]);
+        dzv[0] = make_uint4(ov2[0], ov2[1], ov2[2], ov2[3]);
+        dzv[1] = make_uint4(ov2[4], ov2[5], ov2[6], ov2[7]);
+      } else if (row_in) {
         float4* dk = reinterpret_cast<float4*>(A.dk + row * A.ld_g + h * kD + cc);
         float4* dvp = reinterpret_cast<float4*>(A.dv + row * A.ld_g + h * kD + cc);
 #pragma unroll

@@ -136,11 +136,12 @@ AttnBwdWs attn_bwd_ws_layout(const hstu_jagged_t* j, int H, int hb = 1) {
   return w;
 }
 
-// layer-backward workspace: the attention-backward layout, then dG (fp32), dO (fp16), dq | dk | dv
-// (fp32), dZ (fp16 [T, 4D]), reduction partials, dgamma | dbeta, and the fp16 GEMM operands: copies
-// of dy, x, W1 and W2 (both MMA operands share a type; G and dZ are fp16).
+// layer-backward workspace: the attention-backward layout, then dG (fp32), dO (fp16), dq (fp32; the
+// attention backward writes dZ_K and dZ_V itself), dZ (fp16 [T, 4D]), reduction partials,
+// dgamma | dbeta, and the fp16 GEMM operands: copies of dy, x, W1 and W2 (both MMA operands share
+// a type; G and dZ are fp16).
 struct LayerBwdWs {
-  size_t dg, dO, dq, dk, dv, dz, part_dy, part_ln, dy_f16, x_f16, w1_f16, w2_f16, total;
+  size_t dg, dO, dq, dz, part_dy, part_ln, dy_f16, x_f16, w1_f16, w2_f16, total;
 };
 
 LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) {
@@ -151,8 +152,6 @@ LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) 
   w.dg = take(T * D * 4);
   w.dO = take(T * D * 2);
   w.dq = take(T * D * 4);
-  w.dk = take(T * D * 4);
-  w.dv = take(T * D * 4);
   w.dz = take(T * 4 * D * 2);
   // partial column sums: db2 (from the fp16 copy of dY), dgamma | dbeta (LayerNorm backward); db1 is
   // added up by atomics
@@ -166,13 +165,23 @@ LayerBwdWs layer_bwd_layout(const hstu_layer_desc_t* d, const hstu_jagged_t* j) 
   return w;
 }
 
+// The layer backward's fused dK / dV epilogue: Z_K, Z_V read and dZ_K, dZ_V written (fp16, row
+// stride ld) instead of fp32 dk / dv.
+struct DzKV {
+  const void* z_k;
+  const void* z_v;
+  void* dz_k;
+  void* dz_v;
+  int64_t ld;
+};
+
 // Attention backward on the caller's stream; dq / dk / dv fp32 with row stride ld_g. Zeroes the
 // accumulated outputs (dq, the table gradients) first.
 hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* jag, const void* q, const void* k,
                            const void* v, const void* d_out, const float* rab_pos, const float* rab_time, float* dq,
                            float* dk, float* dv, int64_t ld_g, float* d_rab_pos, float* d_rab_time, void* ws,
                            cudaStream_t st, const hstu_rab_ext_t* ext = nullptr, float* d_rab_type = nullptr,
-                           void* bias_cache = nullptr, bool zeroed = false) {
+                           void* bias_cache = nullptr, bool zeroed = false, const DzKV* dzkv = nullptr) {
   // zeroed: an earlier launch of the call already cleared d_rab_pos, d_rab_time and dq (T > 0)
   const int hb = ext && ext->per_head ? desc->H : 1;
   const int nt = ext ? ext->n_types : 0;
@@ -210,6 +219,9 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
   A.bias_t = w + lay.bias_t; A.bucket_t = w + lay.bucket_t; A.dxt = w + lay.dxt;
   A.kitems = reinterpret_cast<int32_t*>(w + lay.kitems); A.kcount = kcount;
   A.sched = count + 5;   // [276, 284) of the workspace header region
+  if (dzkv) {
+    A.z_k = dzkv->z_k; A.z_v = dzkv->z_v; A.dz_k = dzkv->dz_k; A.dz_v = dzkv->dz_v; A.ld_z = dzkv->ld;
+  }
   a.pack = reinterpret_cast<const int32_t*>(w + lay.f.pack);
   if (bias_cache && hb == 1) {   // tiles and work list written by this batch's forward (shared tables only)
     const BiasCache bc = bias_cache_layout(jag);
@@ -1001,8 +1013,6 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   float* dG = reinterpret_cast<float*>(wsb + lay.dg);
   void* dO = wsb + lay.dO;
   float* dq = reinterpret_cast<float*>(wsb + lay.dq);
-  float* dk = reinterpret_cast<float*>(wsb + lay.dk);
-  float* dv = reinterpret_cast<float*>(wsb + lay.dv);
   void* dz = wsb + lay.dz;
   {   // one launch: the fp16 copy of dY (unless the caller passed one) with the partial sums of db2,
       // the other fp16 GEMM operand copies, and zeros in every output a later launch accumulates
@@ -1043,8 +1053,13 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   if (e != cudaSuccess) return cuda_status(e);
   // 3. attention backward
   const uint8_t* uvqk = static_cast<const uint8_t*>(saved->uvqk);
-  s = run_attn_bwd(&ad, jag, uvqk + 2 * D * 2, uvqk + 3 * D * 2, uvqk + 1 * D * 2, dO, w->rab_pos, w->rab_time, dq, dk,
-                   dv, D, gr->drab_pos, gr->drab_time, ws, st, nullptr, nullptr, saved->attn_bias, true);
+  // (the attention backward writes dZ_V and dZ_K itself, from Z, instead of fp32 dV and dK)
+  uint8_t* dzb = static_cast<uint8_t*>(dz);
+  const uint8_t* zb = static_cast<const uint8_t*>(saved->z);
+  const DzKV dzkv{zb + 3 * D * 2, zb + 1 * D * 2, dzb + 3 * D * 2, dzb + 1 * D * 2, 4ll * D};
+  s = run_attn_bwd(&ad, jag, uvqk + 2 * D * 2, uvqk + 3 * D * 2, uvqk + 1 * D * 2, dO, w->rab_pos, w->rab_time, dq,
+                   nullptr, nullptr, D, gr->drab_pos, gr->drab_time, ws, st, nullptr, nullptr, saved->attn_bias, true,
+                   &dzkv);
   if (s != HSTU_OK) return s;
   // 4. SiLU backward into dZ[:, D:4D], with db1 = sum_t dZ added up by atomics (zeroed by the first
   // launch); the first blocks of the same launch finish db2, dgamma and dbeta, all straight into the
@@ -1054,8 +1069,8 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
     const ColsumJob fin[3] = {{part_dy, D, parts_dy, D, gr->db2},
                               {part_ln, 2ll * D, parts_ln, D, gr->dgamma},
                               {part_ln + D, 2ll * D, parts_ln, D, gr->dbeta}};
-    e = dz_assemble(T, D, kDtF16, dv, dq, dk, saved->z, 4ll * D, dz, 4ll * D, nullptr, &parts_dz, st, gr->db1,
-                    fin, 3);
+    e = dz_assemble(T, D, kDtF16, nullptr, dq, nullptr, saved->z, 4ll * D, dz, 4ll * D, nullptr, &parts_dz, st,
+                    gr->db1, fin, 3);
   }
   // dW2, db2, dgamma, dbeta, db1 and the table gradients are final
   if (e == cudaSuccess && g_ready_events[0]) e = cudaEventRecord(g_ready_events[0], st);

@@ -229,6 +229,14 @@ struct AttnBwdArgs {
   int32_t* sched;              // the persistent backward's unit counter and finished-CTA counter (two
                                // ints): zero at launch (the work list zeroes them), zero again at exit
   int bias_cached;             // bias_t and bucket_t were written by the forward: no bias kernel
+  // Layer backward (optional): instead of dk / dv, the kernel writes dZ_K = dK (.) SiLU'(Z_K) and
+  // dZ_V = dV (.) SiLU'(Z_V) in fp16 (row stride ld_z, head h at column h d), Z read as fp16 with the
+  // same stride; dk and dv are then not written.
+  const void* z_k;
+  const void* z_v;
+  void* dz_k;
+  void* dz_v;
+  int64_t ld_z;
 };
 
 cudaError_t attn_bwd_tc(const AttnBwdArgs& a, cudaStream_t st);
@@ -293,8 +301,9 @@ struct ColsumJobs {
   int first_block[5];
   int njobs;
 };
-// dZ[:, D:4D] = [dV | dQ | dK] (.) SiLU'(Z[:, D:4D]) in fp16 (dZ[:, 0:D] already written) and the
-// column sums of all of dZ in blocks of 32 rows: into partial [*parts = ceil(T / 32), 4D] (may be
+// dZ[:, D:4D] = [dV | dQ | dK] (.) SiLU'(Z[:, D:4D]) in fp16 (dZ[:, 0:D] already written; with dv
+// and dk null, dZ_V and dZ_K too, which the attention backward then wrote) and the column sums of
+// all of dZ in blocks of 32 rows: into partial [*parts = ceil(T / 32), 4D] (may be
 // null) and / or added by fp32 atomics into db1 = sum_t dZ (may be null; zero before the launch).
 // D a multiple of 64. With fin (up to four column sums whose partials earlier launches wrote), the
 // first blocks of the same launch finish those sums.

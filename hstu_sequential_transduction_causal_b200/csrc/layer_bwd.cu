@@ -25,11 +25,6 @@ namespace hstu {
 
 namespace {
 
-__device__ __forceinline__ float silu_grad(float z) {
-  const float s = __fdividef(1.0f, 1.0f + __expf(fminf(-z, 80.0f)));
-  return s * (1.0f + z * (1.0f - s));
-}
-
 // One warp per token row (grid-stride over rows); lane l holds features 128 k + 4 l + i (k < VPT / 4,
 // i < 4): every load and store of the warp covers 128 consecutive features (coalesced). gamma and
 // beta are staged in shared memory (registers for two blocks per SM).
@@ -312,11 +307,12 @@ dz_assemble_kernel(int64_t T, int D, const float* __restrict__ dv, const float* 
 #pragma unroll
   for (int e = 0; e < 8; ++e) v[e] = 0.0f;
   if (row < T) {
-    if (c < D) {
+    const int blk = c < D ? -1 : (c - D) / D;
+    const float* g = blk == 0 ? dv : (blk == 1 ? dq : (blk == 2 ? dk : nullptr));
+    if (!g) {   // written by an earlier kernel (dZ_U; dZ_V and dZ_K when dv, dk are null): its sums only
       load_vec<8, kDtF16>(dz, row * ld_dz + c, v);
     } else {
-      const int blk = (c - D) / D, cc = (c - D) - blk * D;
-      const float* g = blk == 0 ? dv : (blk == 1 ? dq : dk);
+      const int cc = (c - D) - blk * D;
       float zv[8];
       load_vec<8, kDtF32>(g, row * D + cc, v);
       load_vec<8, AT>(z, row * ld_z + c, zv);

@@ -427,4 +427,11 @@ __device__ __forceinline__ float silu_tanh(float x) {
   return fmaf(h, tanh_f32_approx(h), h);
 }
 
+// SiLU'(z) = s (1 + z (1 - s)), s = sigmoid(z): the backward of f1's activation. Every kernel that
+// forms a piece of dZ = dS (.) SiLU'(Z) uses this one function, so each piece rounds alike.
+__device__ __forceinline__ float silu_grad(float z) {
+  const float s = __fdividef(1.0f, 1.0f + __expf(fminf(-z, 80.0f)));
+  return s * (1.0f + z * (1.0f - s));
+}
+
 }  // namespace hstu
