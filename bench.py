@@ -717,9 +717,9 @@ def main():
             rooflines["table_gradients"] = hbm_line(
                 H.PROFILE_TABLE_GRAD, n_pairs * (wl.H * 32768 + 16384),
                 f"{n_pairs} pairs x {wl.H} heads of 32 KB dX^T + 16 KB buckets read")
-            # dZ assembly: dV, dQ, dK fp32 and Z[:, D:4D] fp16 read, dZ_U fp16 read back, dZ[:, D:4D] fp16
-            # written (the db2 / dgamma / dbeta finishes read a few partial rows more)
-            rooflines["dz_assembly"] = hbm_line(H.PROFILE_DZ, 26 * T * D, "26 bytes per token and feature")
+            # dZ assembly: dQ fp32 and Z_Q fp16 read, dZ_Q fp16 written, dZ_U, dZ_V, dZ_K fp16 read back for
+            # db1 (the db2 / dgamma / dbeta finishes read a few partial rows more)
+            rooflines["dz_assembly"] = hbm_line(H.PROFILE_DZ, 14 * T * D, "14 bytes per token and feature")
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_oracle_sample(wl, backward)
