@@ -107,6 +107,14 @@ NAMES = ("dW1", "db1", "dW2", "db2", "dgamma", "dbeta", "drab_pos", "drab_time")
 STRICT_MISSES = {}
 
 
+def _assert_same_up_to_dq_order(a, b, what):
+    """dQ is summed over the key tiles by fp32 reduce-adds in no fixed order, so two runs of the same
+    backward may round an element of dZ_Q, and through it of dX, differently in its last bit: every
+    element within the bf16 bound of the other run, and at most 1 in 10^4 not bit-equal."""
+    assert_close(a, b, *BF16_TOL, what=what)
+    assert np.count_nonzero(a != b) <= max(1, a.size // 10000), what
+
+
 def _compare(dx, grads, ref, model, tag=""):
     """dx (an O(1) activation gradient) meets the bf16 bound |d| <= 1e-2 + 1e-2 |ref| element by
     element. The weight and table gradients are sums over all tokens; with 16-bit attention operands
@@ -138,12 +146,12 @@ def test_layer_bwd_ragged_d512():
 
 def test_layer_bwd_bias_cache_matches_recompute():
     """The backward reading the bias tiles its forward cached (hstu_layer_saved_t.attn_bias) computes
-    what it computes from tiles of its own: dx bit for bit (no reduction of unfixed order reaches
-    it), the gradients reduced by atomics up to the order of their fp32 additions."""
+    what it computes from tiles of its own: dx up to the order of dQ's fp32 reduce-adds, the
+    gradients reduced by atomics up to the order of their fp32 additions."""
     wl = W.make_workload("c3", seed=5, lengths=[300, 1, 129, 700, 64, 0, 400], pos_max_len=1024, N=1024)
     dx_c, g_c = _run_layer_fwd_bwd(wl, bias_cache=True)
     dx_r, g_r = _run_layer_fwd_bwd(wl, bias_cache=False)
-    np.testing.assert_array_equal(dx_c, dx_r)
+    _assert_same_up_to_dq_order(dx_c, dx_r, "dx cached vs recomputed bias")
     for name, a, b in zip(("dW1", "db1", "dW2", "db2", "dgamma", "dbeta", "drab_pos", "drab_time"), g_c, g_r):
         scale = max(float(np.abs(b).max()), 1e-30)
         assert np.abs(a - b).max() <= 1e-5 * scale, name
@@ -197,7 +205,7 @@ def test_layer_fwd_bwd_more_sequences_than_staged_tables():
     assert_close(y, ye, *BF16_TOL, what="Y 600 sequences")
     _compare(dx, grads, O.layer_bwd(wl.dy, wl.layers[0], sv, *args), _model_grads(wl), "600-sequences ")
     dx_r, g_r = _run_layer_fwd_bwd(wl, bias_cache=False)
-    np.testing.assert_array_equal(dx, dx_r)
+    _assert_same_up_to_dq_order(dx, dx_r, "dx cached vs recomputed bias, 600 sequences")
 
 
 def test_layer_bwd_d256_four_heads():
