@@ -850,7 +850,7 @@ attn_table_grad_kernel(AttnBwdArgs A) {
 
 }  // namespace
 
-cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
+cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st, const SideLaunch* side) {
   const AttnArgs& a = A.f;
   cudaError_t e = upload_time_taus();
   if (e != cudaSuccess) return e;
@@ -890,12 +890,19 @@ cudaError_t attn_bwd_tc(const AttnBwdArgs& A, cudaStream_t st) {
   if (e == cudaSuccess) e = prof_record(kProfAttnBwd, true, st);
   if (e != cudaSuccess) return e;
   auto tg = f16 ? attn_table_grad_kernel<true> : attn_table_grad_kernel<false>;
-  e = prof_record(kProfTableGrad, false, st);
+  cudaStream_t ts = st;
+  if (side) {   // fork: the table gradients overlap what the caller launches next on st
+    e = cudaEventRecord(side->fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+    if (e != cudaSuccess) return e;
+    ts = side->stream;
+  }
+  e = prof_record(kProfTableGrad, false, ts);
   if (e == cudaSuccess)
     e = launch_pdl(tg, dim3(static_cast<unsigned>(bias_grid_pairs(a.max_pairs, a.bias_heads) * 2), 2,
                             static_cast<unsigned>(a.bias_heads)),
-                   dim3(kTgThreads), 0, st, A);
-  if (e == cudaSuccess) e = prof_record(kProfTableGrad, true, st);
+                   dim3(kTgThreads), 0, ts, A);
+  if (e == cudaSuccess) e = prof_record(kProfTableGrad, true, ts);
   return e;
 }
 

@@ -21,6 +21,14 @@ namespace {
 thread_local int32_t g_last_cuda_error = 0;
 thread_local cudaEvent_t g_prof_events[kProfKernels][2] = {};
 thread_local cudaEvent_t g_ready_events[2] = {};   // hstu_layer_bwd_ready_events: early, w1
+// The layer backward's second stream, per host thread and device (created by the first call, which
+// runs outside any capture): the table gradients run there while the dZ assembly and the dX / dW1
+// GEMM run on the caller's stream, which joins it back before the call returns.
+struct SideRes {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr, dz = nullptr;
+};
+thread_local SideRes g_side[64];
 std::atomic<unsigned long long> g_wait_limit{1ull << 31};
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -181,7 +189,8 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
                            const void* v, const void* d_out, const float* rab_pos, const float* rab_time, float* dq,
                            float* dk, float* dv, int64_t ld_g, float* d_rab_pos, float* d_rab_time, void* ws,
                            cudaStream_t st, const hstu_rab_ext_t* ext = nullptr, float* d_rab_type = nullptr,
-                           void* bias_cache = nullptr, bool zeroed = false, const DzKV* dzkv = nullptr) {
+                           void* bias_cache = nullptr, bool zeroed = false, const DzKV* dzkv = nullptr,
+                           const SideLaunch* side = nullptr) {
   // zeroed: an earlier launch of the call already cleared d_rab_pos, d_rab_time and dq (T > 0)
   const int hb = ext && ext->per_head ? desc->H : 1;
   const int nt = ext ? ext->n_types : 0;
@@ -239,8 +248,25 @@ hstu_status_t run_attn_bwd(const hstu_attn_desc_t* desc, const hstu_jagged_t* ja
                         reinterpret_cast<long long*>(w + lay.f.pairs), reinterpret_cast<int32_t*>(w + lay.kitems),
                         kcount, nullptr, reinterpret_cast<int32_t*>(w + lay.f.pack), nullptr, A.sched);
   }
-  if (e == cudaSuccess) e = attn_bwd_tc(A, st);
+  if (e == cudaSuccess) e = attn_bwd_tc(A, st, side);
   return cuda_status(e);
+}
+
+cudaError_t side_res(SideRes** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  SideRes& r = g_side[dev];
+  if (!r.s) {
+    e = cudaStreamCreateWithFlags(&r.s, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.join, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r.dz, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+  }
+  *out = &r;
+  return cudaSuccess;
 }
 
 hstu_status_t check_jagged(const hstu_jagged_t* j) {
@@ -1057,9 +1083,13 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
   uint8_t* dzb = static_cast<uint8_t*>(dz);
   const uint8_t* zb = static_cast<const uint8_t*>(saved->z);
   const DzKV dzkv{zb + 3 * D * 2, zb + 1 * D * 2, dzb + 3 * D * 2, dzb + 1 * D * 2, 4ll * D};
+  SideRes* sr = nullptr;
+  e = side_res(&sr);
+  if (e != cudaSuccess) return cuda_status(e);
+  const SideLaunch sl{sr->s, sr->fork};
   s = run_attn_bwd(&ad, jag, uvqk + 2 * D * 2, uvqk + 3 * D * 2, uvqk + 1 * D * 2, dO, w->rab_pos, w->rab_time, dq,
                    nullptr, nullptr, D, gr->drab_pos, gr->drab_time, ws, st, nullptr, nullptr, saved->attn_bias, true,
-                   &dzkv);
+                   &dzkv, &sl);
   if (s != HSTU_OK) return s;
   // 4. SiLU backward into dZ[:, D:4D], with db1 = sum_t dZ added up by atomics (zeroed by the first
   // launch); the first blocks of the same launch finish db2, dgamma and dbeta, all straight into the
@@ -1072,8 +1102,13 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
     e = dz_assemble(T, D, kDtF16, nullptr, dq, nullptr, saved->z, 4ll * D, dz, 4ll * D, nullptr, &parts_dz, st,
                     gr->db1, fin, 3);
   }
-  // dW2, db2, dgamma, dbeta, db1 and the table gradients are final
-  if (e == cudaSuccess && g_ready_events[0]) e = cudaEventRecord(g_ready_events[0], st);
+  // dW2, db2, dgamma, dbeta, db1 (the caller's stream) and the table gradients (the second stream)
+  // are final: the early event is recorded on the second stream once it has also seen the former
+  if (e == cudaSuccess && g_ready_events[0]) {
+    e = cudaEventRecord(sr->dz, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sr->s, sr->dz, 0);
+    if (e == cudaSuccess) e = cudaEventRecord(g_ready_events[0], sr->s);
+  }
   // 5. f1 backward in one launch: dX = dY + dZ W1 and dW1 = dZ^T X (fp16 dZ, x and W1; dW1 split
   //    over K = T into units of about a third of a dX unit, reduced into the zeroed dW1)
   if (e == cudaSuccess) {
@@ -1101,7 +1136,10 @@ hstu_status_t run_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* 
     e = ln_in_bwd(T, D, desc->x_dtype == HSTU_F32 ? kDtF32 : kDtBF16, desc->y_dtype == HSTU_F32 ? kDtF32 : kDtBF16,
                   reinterpret_cast<const float*>(wsb + nin_dxn), x, dy, nin->gamma, nin->mu, nin->rstd, dx, dx_f16,
                   reinterpret_cast<float*>(wsb + nin_part), nin->dgamma, nin->dbeta, st);
-  return cuda_status(e);
+  // join: the caller's stream waits for the table gradients
+  cudaError_t ej = cudaEventRecord(sr->join, sr->s);
+  if (ej == cudaSuccess) ej = cudaStreamWaitEvent(st, sr->join, 0);
+  return cuda_status(e != cudaSuccess ? e : ej);
 }
 
 }  // namespace

@@ -239,7 +239,13 @@ struct AttnBwdArgs {
   int64_t ld_z;
 };
 
-cudaError_t attn_bwd_tc(const AttnBwdArgs& a, cudaStream_t st);
+// side (optional): the table gradients go to that stream instead, after it waits for the kernel
+// before them (fork: a reusable event recorded on st); the caller joins it back later.
+struct SideLaunch {
+  cudaStream_t stream;
+  cudaEvent_t fork;
+};
+cudaError_t attn_bwd_tc(const AttnBwdArgs& a, cudaStream_t st, const SideLaunch* side = nullptr);
 
 // Bound on the number of causal (query tile, key tile) pairs of a batch.
 int64_t attn_max_pairs(int64_t capacity, int max_len);
