@@ -435,7 +435,10 @@ size_t hstu_layer_bias_cache_size(const hstu_layer_desc_t* desc, const hstu_jagg
  * Steps: dG = dy W2,
  * dW2 = dy^T G, db2 = sum dy; LayerNorm (.) U backward (dO, dU, dgamma, dbeta); attention
  * backward (dQ, dK, dV, table gradients); dZ = [dU|dV|dQ|dK] (.) SiLU'(Z); dW1 = dZ^T X,
- * db1 = sum dZ, dX = dy + dZ W1. All gradients fp32 and overwritten. */
+ * db1 = sum dZ, dX = dy + dZ W1. All gradients fp32 and overwritten. The table gradients run on a
+ * second stream the library keeps per host thread and device (made by the first call, which must
+ * run outside any capture), forked from `stream` after the attention backward and joined back
+ * before the call's last operation on `stream`: work later enqueued on `stream` sees every output. */
 hstu_status_t hstu_layer_bwd(const hstu_layer_desc_t* desc, const hstu_jagged_t* jag,
                              const hstu_layer_weights_t* w, const void* x, const void* x_f16,
                              const hstu_layer_saved_t* saved, const void* dy, const void* dy_f16,
@@ -499,8 +502,9 @@ hstu_status_t hstu_dp_partition(const int64_t* lengths, int32_t B, int32_t D, in
                                 double* rank_cost);
 
 /* Events for overlapping the gradient all-reduce of data parallelism with the rest of a backward:
- * until the next call, every hstu_layer_bwd of this host thread records `early` on its stream once
- * dW2, db2, dgamma, dbeta, db1, drab_pos and drab_time are final (before the f1 backward GEMMs), and
+ * until the next call, every hstu_layer_bwd of this host thread records `early` once dW2, db2,
+ * dgamma, dbeta, db1, drab_pos and drab_time are final (before the f1 backward GEMMs; on the call's
+ * second stream, which has then seen all of them), and
  * `w1` once dW1 is final too (after the launch that computes dX and dW1; with the input-LayerNorm
  * variant, before its backward). A communication stream that waits on them can reduce those
  * gradients while the remaining kernels run. Under stream capture they are
