@@ -248,13 +248,6 @@ norm_gate_bwd_staged_kernel(int64_t T, const float* __restrict__ dg, const float
   }
 }
 
-// dZ[:, D:4D] = [dV | dQ | dK] (.) SiLU'(Z[:, D:4D]) in fp16 (g* are fp32 [T, D]), together with the
-// partial column sums of all of dZ (the db1 of f1's bias). A block covers 32 rows x 64 columns of
-// dZ: warp w takes rows 4w .. 4w+3, lane l row 4w + l / 8 and columns 8 (l % 8) .. +7, so each row's
-// 64 columns are one coalesced access. Columns [0, D) (dZ_U, written by the LayerNorm backward) are
-// only read back for their sums. The block's 32 rows are summed by shuffles (the 4 rows of a warp)
-// and shared memory (the 8 warps) into partial[row block][cols]; the sums are of the fp16 values
-// stored. Block b covers column block b % (4D / 64) of row block b / (4D / 64).
 // Block blk of a batch of column-sum finishes (job j sums parts rows, row stride ld, of its partial
 // buffer into out[0 .. cols)): 32 columns of one job, each summed over its partial rows by the 8
 // warps (rows p = warp mod 8) and then across warps through s_part.
@@ -283,6 +276,15 @@ __device__ __forceinline__ void colsum_finish_block(const ColsumJobs& jobs, int 
   }
 }
 
+// dZ[:, D:4D] = [dV | dQ | dK] (.) SiLU'(Z[:, D:4D]) in fp16 (g* are fp32 [T, D]), together with the
+// column sums of all of dZ (the db1 of f1's bias). After the first fin_blocks blocks (column-sum
+// finishes of earlier launches), a block covers 32 rows x 64 columns of dZ: warp w takes rows
+// 4w .. 4w+3, lane l row 4w + l / 8 and columns 8 (l % 8) .. +7, so each row's 64 columns are one
+// coalesced access. Columns [0, D) (dZ_U, written by the LayerNorm backward) are only read back for
+// their sums, and so are dZ_V and dZ_K when dv and dk are null (the attention backward wrote them).
+// The block's 32 rows are summed by shuffles (the 4 rows of a warp) and shared memory (the 8 warps)
+// into partial[row block][cols] and / or by fp32 atomics into db1; the sums are of the fp16 values
+// stored. Block b covers column block b % (4D / 64) of row block b / (4D / 64).
 template <int AT>
 __global__ void __launch_bounds__(256)
 dz_assemble_kernel(int64_t T, int D, const float* __restrict__ dv, const float* __restrict__ dq,
